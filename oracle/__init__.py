@@ -1,0 +1,15 @@
+"""fp64 CPU oracle (test infrastructure only; see ``gdn_oracle``).
+
+Parity status of each function: every function here is pinned by the
+``-m "not gpu"`` tests in ``tests/test_oracle_pins.py`` (closed forms,
+invariants, special cases that reduce to textbook routines, brute force on tiny
+inputs, and a hand-worked example under ``tests/golden/``).
+"""
+from .gdn_oracle import (  # noqa: F401
+    frame_output,
+    frame_statistics,
+    frame_update,
+    gdn_frame_forward,
+    gdn_frame_step,
+    la_block_causal,
+)

@@ -1,0 +1,131 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check that every one of
+them fails at least one pin. This shows the pins constrain each term, sign, index and
+operand order of the oracle, not only its happy path."""
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.gdn_oracle as go
+from tests import oracle_pins
+
+
+def _impl(stats=None, update=None, output=None, forward=None, la=None):
+    """An oracle copy with some pieces swapped; gdn_frame_step follows the swapped forward."""
+    stats = stats or go.frame_statistics
+    update = update or go.frame_update
+    output = output or go.frame_output
+
+    def fwd(q, k, v, gamma, beta, state_in, key_scale):
+        q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
+        B, T, N, H, D = q.shape
+        out = np.zeros(q.shape)
+        st = np.zeros((B, H, D, D))
+        for b in range(B):
+            for h in range(H):
+                S = np.zeros((D, D)) if state_in is None else np.array(state_in[b, h], float)
+                for t in range(T):
+                    A, Bm = stats(k[b, t, :, h], v[b, t, :, h], key_scale)
+                    S = update(S, A, Bm, float(gamma[b, t, h]), float(beta[b, t, h]))
+                    out[b, t, :, h] = output(q[b, t, :, h], S)
+                st[b, h] = S
+        return out, st
+
+    forward = forward or fwd
+
+    def step(q, k, v, gamma, beta, state_in, key_scale):
+        o, s = forward(np.asarray(q)[:, None], np.asarray(k)[:, None], np.asarray(v)[:, None],
+                       np.asarray(gamma)[:, None], np.asarray(beta)[:, None], state_in, key_scale)
+        return o[:, 0], s
+
+    return types.SimpleNamespace(gdn_frame_forward=forward, gdn_frame_step=step,
+                                 la_block_causal=la or oracle.la_block_causal,
+                                 frame_statistics=stats)
+
+
+def _old_state_forward(q, k, v, gamma, beta, state_in, key_scale):
+    """Mistake: frame t's output reads S_{t-1} instead of S_t."""
+    q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
+    B, T, N, H, D = q.shape
+    out = np.zeros(q.shape)
+    st = np.zeros((B, H, D, D))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((D, D)) if state_in is None else np.array(state_in[b, h], float)
+            for t in range(T):
+                out[b, t, :, h] = q[b, t, :, h] @ S.T
+                A, Bm = go.frame_statistics(k[b, t, :, h], v[b, t, :, h], key_scale)
+                S = go.frame_update(S, A, Bm, gamma[b, t, h], beta[b, t, h])
+            st[b, h] = S
+    return out, st
+
+
+def _la_variant(relu_q=True, relu_k=True, eps=1e-6, transpose_state=False, frame_causal=False):
+    def la(q, k, v, state_in, z_in, frames_per_block, eps_=1e-6):
+        q, k, v = np.asarray(q, float), np.asarray(k, float), np.asarray(v, float)
+        B, T, N, H, D = q.shape
+        F = 1 if frame_causal else int(frames_per_block)
+        out = np.zeros(q.shape)
+        so = np.zeros((B, H, D, D))
+        zo = np.zeros((B, H, D))
+        fq = (lambda x: np.maximum(x, 0)) if relu_q else (lambda x: x)
+        fk = (lambda x: np.maximum(x, 0)) if relu_k else (lambda x: x)
+        for b in range(B):
+            for h in range(H):
+                S = np.zeros((D, D)) if state_in is None else np.array(state_in[b, h], float)
+                z = np.zeros(D) if z_in is None else np.array(z_in[b, h], float)
+                for t0 in range(0, T, F):
+                    fr = range(t0, min(t0 + F, T))
+                    for t in fr:
+                        pk = fk(k[b, t, :, h])
+                        S = S + (v[b, t, :, h].T @ pk if transpose_state else pk.T @ v[b, t, :, h])
+                        z = z + pk.sum(0)
+                    for t in fr:
+                        pq = fq(q[b, t, :, h])
+                        with np.errstate(all="ignore"):
+                            out[b, t, :, h] = (pq @ S) / (pq @ z + eps)[:, None]
+                so[b, h], zo[b, h] = S, z
+        return out, so, zo
+    return la
+
+
+MUTANTS = {
+    "gamma_also_scales_beta_B": dict(update=lambda S, A, B, g, b: g * (S @ (np.eye(len(A)) - b * A) + b * B)),
+    "transposed_state_product": dict(update=lambda S, A, B, g, b: g * ((np.eye(len(A)) - b * A) @ S) + b * B),
+    "sign_of_delta_term": dict(update=lambda S, A, B, g, b: g * (S @ (np.eye(len(A)) + b * A)) + b * B),
+    "beta_dropped_on_A": dict(update=lambda S, A, B, g, b: g * (S @ (np.eye(len(A)) - A)) + b * B),
+    "beta_dropped_on_B": dict(update=lambda S, A, B, g, b: g * (S @ (np.eye(len(A)) - b * A)) + B),
+    "gamma_dropped": dict(update=lambda S, A, B, g, b: S @ (np.eye(len(A)) - b * A) + b * B),
+    "key_scale_once_on_A": dict(stats=lambda K, V, s: (s * (np.asarray(K, float).T @ np.asarray(K, float)),
+                                                       np.asarray(V, float).T @ (s * np.asarray(K, float)))),
+    "B_transposed": dict(stats=lambda K, V, s: ((s * np.asarray(K, float)).T @ (s * np.asarray(K, float)),
+                                                (s * np.asarray(K, float)).T @ np.asarray(V, float))),
+    "B_unscaled": dict(stats=lambda K, V, s: ((s * np.asarray(K, float)).T @ (s * np.asarray(K, float)),
+                                              np.asarray(V, float).T @ np.asarray(K, float))),
+    "output_not_transposed": dict(output=lambda Q, S: np.asarray(Q, float) @ S),
+    "output_reads_previous_state": dict(forward=_old_state_forward),
+    "la_no_relu_on_q": dict(la=_la_variant(relu_q=False)),
+    "la_no_relu_on_k": dict(la=_la_variant(relu_k=False)),
+    "la_eps_dropped": dict(la=_la_variant(eps=0.0)),
+    "la_state_transposed": dict(la=_la_variant(transpose_state=True)),
+    "la_frame_causal_not_block_causal": dict(la=_la_variant(frame_causal=True)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    impl = _impl(**MUTANTS[name])
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(impl)
+        except (AssertionError, FloatingPointError, ValueError):
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name} passes every pin"
+
+
+def test_unmutated_copy_passes():
+    impl = _impl()
+    for pin in oracle_pins.ALL_PINS:
+        pin(impl)
