@@ -1,0 +1,161 @@
+"""PyTorch binding of the C ABI (argument marshalling only; every step runs in libgdn.so).
+
+Tensors must be CUDA tensors of the dtypes and layouts ``include/gdn.h`` documents. Calls are
+asynchronous on ``stream`` (default: torch's current stream of the tensors' device).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from ._lib import LIB, GdnError, check
+
+__all__ = ["gdn_frame_forward", "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
+           "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
+           "gdn_la_workspace_bytes", "GdnError"]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _req(t: torch.Tensor, name: str, dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def gdn_frame_forward(q, k, v, gamma, beta, state_in=None, out=None, state_out=None,
+                      key_scale: Optional[float] = None, stream=None, want_state: bool = True):
+    """Frame-wise GDN over a clip. q, k, v: [B,T,N,H,D] bf16; gamma, beta: [B,T,H] f32;
+    state_in: [B,H,D,D] f32 or None. Returns (out, state_out)."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    _req(gamma, "gamma", torch.float32, (B, T, H))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _req(state_out, "state_out", torch.float32, (B, H, D, D))
+    if key_scale is None:
+        key_scale = 1.0 / math.sqrt(D * N)
+    with torch.cuda.device(q.device):
+        check("gdn_frame_forward", LIB.gdn_frame_forward(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
+            _ptr(state_out), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
+    return out, state_out
+
+
+def gdn_frame_step(q, k, v, gamma, beta, state_in=None, out=None, state_out=None,
+                   key_scale: Optional[float] = None, stream=None):
+    """One streaming step. q, k, v: [B,N,H,D] bf16; gamma, beta: [B,H] f32; state_in /
+    state_out: [B,H,D,D] f32 (pass the same tensor for an in-place update). Returns (out, state)."""
+    B, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, name, torch.bfloat16, (B, N, H, D))
+    _req(gamma, "gamma", torch.float32, (B, H))
+    _req(beta, "beta", torch.float32, (B, H))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, N, H, D))
+    if state_out is None:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    _req(state_out, "state_out", torch.float32, (B, H, D, D))
+    if key_scale is None:
+        key_scale = 1.0 / math.sqrt(D * N)
+    with torch.cuda.device(q.device):
+        check("gdn_frame_step", LIB.gdn_frame_step(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
+            _ptr(state_out), B, H, N, D, float(key_scale), _stream(stream, q.device)))
+    return out, state_out
+
+
+def gdn_frame_stats(k, v, key_scale: Optional[float] = None, A_out=None, B_out=None, stream=None):
+    """Per-frame statistics. Returns A [B,H,T,D,D] bf16 (s^2 K^T K) and B [B,H,T,D,D] f32
+    (s V^T K)."""
+    Bsz, T, N, H, D = k.shape
+    _req(k, "k", torch.bfloat16, (Bsz, T, N, H, D))
+    _req(v, "v", torch.bfloat16, (Bsz, T, N, H, D))
+    if A_out is None:
+        A_out = torch.empty((Bsz, H, T, D, D), dtype=torch.bfloat16, device=k.device)
+    if B_out is None:
+        B_out = torch.empty((Bsz, H, T, D, D), dtype=torch.float32, device=k.device)
+    _req(A_out, "A_out", torch.bfloat16, (Bsz, H, T, D, D))
+    _req(B_out, "B_out", torch.float32, (Bsz, H, T, D, D))
+    if key_scale is None:
+        key_scale = 1.0 / math.sqrt(D * N)
+    with torch.cuda.device(k.device):
+        check("gdn_frame_stats", LIB.gdn_frame_stats(
+            _ptr(k), _ptr(v), _ptr(A_out), _ptr(B_out), Bsz, H, T, N, D, float(key_scale),
+            _stream(stream, k.device)))
+    return A_out, B_out
+
+
+def gdn_block_causal_la(q, k, v, frames_per_block: int, state_in=None, z_in=None, out=None,
+                        state_out=None, z_out=None, stream=None):
+    """Block-causal linear attention with relu features and a normaliser. q, k, v:
+    [B,T,N,H,D] bf16; state [B,H,D,D] f32 (row = key index); z [B,H,D] f32.
+    Returns (out, state_out, z_out)."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if z_in is not None:
+        _req(z_in, "z_in", torch.float32, (B, H, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    if state_out is None:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    if z_out is None:
+        z_out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    _req(state_out, "state_out", torch.float32, (B, H, D, D))
+    _req(z_out, "z_out", torch.float32, (B, H, D))
+    with torch.cuda.device(q.device):
+        check("gdn_block_causal_la", LIB.gdn_block_causal_la(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(state_in), _ptr(z_in), _ptr(out), _ptr(state_out),
+            _ptr(z_out), B, H, T, N, D, int(frames_per_block), _stream(stream, q.device)))
+    return out, state_out, z_out
+
+
+def gdn_sync_status(stream=None, device=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word (0 = OK)."""
+    dev = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        return int(LIB.gdn_sync_status(_stream(stream, dev)))
+
+
+def gdn_release_workspace() -> None:
+    LIB.gdn_release_workspace()
+
+
+def gdn_workspace_bytes(B, H, T, N, D) -> int:
+    return int(LIB.gdn_workspace_bytes(B, H, T, N, D))
+
+
+def gdn_la_workspace_bytes(B, H, T, D) -> int:
+    return int(LIB.gdn_la_workspace_bytes(B, H, T, D))

@@ -1,0 +1,407 @@
+// Host side of the C ABI declared in include/gdn.h: argument validation, the cached per-GPU
+// workspace, TMA descriptor encoding and kernel launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gdn.h"
+#include "chain_kernel.cuh"
+#include "common.cuh"
+#include "la_scan_kernel.cuh"
+#include "output_kernel.cuh"
+#include "stats_kernel.cuh"
+
+namespace {
+
+using gdn::Problem;
+
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D tile (dims[0] contiguous) with 128B swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+               const cuuint64_t* dims, const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
+                  strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// q/k/v [B, T, N, H, D] bf16 -> 4-D map (D, H, N, B*T), box 64 x 1 x 128 x 1.
+bool tmap_tokens(CUtensorMap* m, const void* base, const Problem& p) {
+  const cuuint64_t dims[4] = {(cuuint64_t)p.D, (cuuint64_t)p.H, (cuuint64_t)p.N,
+                              (cuuint64_t)p.B * p.T};
+  const cuuint64_t strides[3] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.H * p.D * 2,
+                                 (cuuint64_t)p.N * p.H * p.D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box);
+}
+
+// [count, rows, D] matrices (bf16 or f32) -> 3-D map (D, rows, count), box (128 B) x DP x 1.
+bool tmap_mats(CUtensorMap* m, const void* base, bool f32, int D, int rows, long count, int DP) {
+  const int es = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)count};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)rows * D * es};
+  const cuuint32_t box[3] = {(cuuint32_t)(128 / es), (cuuint32_t)DP, 1};
+  return make_tmap(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   base, dims, strides, box);
+}
+
+// ------------------------------------------------------------------ device info / workspace
+struct DeviceState {
+  int sms = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  uint64_t attr_done = 0;  // bit per kernel instantiation whose smem attribute is set
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+gdn_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return GDN_ERR_CUDA;
+  DeviceState& d = g_dev[*dev];
+  if (d.sms == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    d.sms = sms;
+  }
+  return GDN_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+gdn_status get_workspace(int dev, size_t bytes, cudaStream_t stream, void** out) {
+  DeviceState& d = g_dev[dev];
+  if (d.ws_bytes >= bytes) {
+    *out = d.ws;
+    return GDN_OK;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return GDN_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return GDN_ERR_NO_MEMORY;
+  if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+  if (d.ws) cudaFree(d.ws);
+  d.ws = nullptr;
+  d.ws_bytes = 0;
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_NO_MEMORY;
+  }
+  d.ws = p;
+  d.ws_bytes = bytes;
+  *out = p;
+  return GDN_OK;
+}
+
+template <typename K>
+gdn_status ensure_smem_attr(int dev, int bit, K kernel, int bytes) {
+  DeviceState& d = g_dev[dev];
+  if (d.attr_done & (uint64_t(1) << bit)) return GDN_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return GDN_ERR_CUDA;
+  d.attr_done |= uint64_t(1) << bit;
+  return GDN_OK;
+}
+
+// ------------------------------------------------------------------ validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+gdn_status check_sizes(int B, int H, int T, int N, int D, int d_max) {
+  if (B < 1 || H < 1 || T < 1 || N < 1 || D < 1) return GDN_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > d_max) return GDN_ERR_UNSUPPORTED;
+  const double elems = double(B) * T * N * H * D;
+  if (elems > 4.0e18 || double(B) * T > 2147483647.0 || double(B) * H * T > 2147483647.0)
+    return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+gdn_status check_launch() {
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ kernel runners
+template <int DP>
+gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, void* A, float* Bm,
+                     cudaStream_t st) {
+  using L = gdn::StatsLayout<DP, false>;
+  CUtensorMap tk, tv;
+  if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_stats_kernel<DP, false>;
+  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 0 : 1, kern, L::kSmemBytes)) return s;
+  const long items = long(p.B) * p.T * p.H;
+  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, static_cast<__nv_bfloat16*>(A), Bm, p);
+  return check_launch();
+}
+
+template <int DP>
+gdn_status run_chain(int dev, const Problem& p, const void* A, const float* Bm,
+                     const float* gamma, const float* beta, const float* s_in, void* S_ws,
+                     float* s_out, cudaStream_t st) {
+  using L = gdn::ChainLayout<DP>;
+  const long count = long(p.B) * p.H * p.T;
+  CUtensorMap ta, tb;
+  if (!tmap_mats(&ta, A, false, p.D, p.D, count, DP) ||
+      !tmap_mats(&tb, Bm, true, p.D, p.D, count, DP))
+    return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_chain_kernel<DP>;
+  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 2 : 3, kern, L::kSmemBytes)) return s;
+  kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, tb, gamma, beta, s_in,
+                                                      static_cast<__nv_bfloat16*>(S_ws), s_out, p);
+  return check_launch();
+}
+
+template <int DP, bool kLA>
+gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws, int srows,
+                      void* out, int F, cudaStream_t st) {
+  using L = gdn::OutputLayout<DP, kLA>;
+  const long count = long(p.B) * p.H * p.T;
+  CUtensorMap tq, ts;
+  if (!tmap_tokens(&tq, q, p) || !tmap_mats(&ts, S_ws, false, p.D, srows, count, DP))
+    return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_output_kernel<DP, kLA>;
+  if (gdn_status s = ensure_smem_attr(dev, kLA ? 6 : (DP == 128 ? 4 : 5), kern, L::kSmemBytes))
+    return s;
+  const long items = long(p.B) * p.T * p.H;
+  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, ts, static_cast<__nv_bfloat16*>(out), p, F);
+  return check_launch();
+}
+
+struct ForwardWs {
+  void* A;
+  float* B;
+  void* S;
+};
+
+size_t forward_ws_bytes(long count, int D) {
+  const size_t m = size_t(D) * D;
+  return align256(count * m * 2) + align256(count * m * 4) + align256(count * m * 2);
+}
+
+ForwardWs carve_forward(void* base, long count, int D) {
+  const size_t m = size_t(D) * D;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  ForwardWs w;
+  w.A = p;
+  p += align256(count * m * 2);
+  w.B = reinterpret_cast<float*>(p);
+  p += align256(count * m * 4);
+  w.S = p;
+  return w;
+}
+
+gdn_status forward_impl(const void* q, const void* k, const void* v, const float* gamma,
+                        const float* beta, const float* s_in, void* out, float* s_out,
+                        const Problem& p, cudaStream_t st) {
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const long count = long(p.B) * p.H * p.T;
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, forward_ws_bytes(count, p.D), st, &base)) return s;
+  ForwardWs w = carve_forward(base, count, p.D);
+  if (p.D <= 64) {
+    if (gdn_status s = run_stats<64>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, st))
+      return s;
+    return run_output<64, false>(dev, p, q, w.S, p.D, out, 1, st);
+  }
+  if (gdn_status s = run_stats<128>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, st))
+    return s;
+  return run_output<128, false>(dev, p, q, w.S, p.D, out, 1, st);
+}
+
+gdn_status validate_common(const void* q, const void* k, const void* v, const void* out,
+                           const float* gamma, const float* beta, const float* s_in,
+                           const float* s_out, int B, int H, int T, int N, int D, float ks) {
+  if (!q || !k || !v || !out || !gamma || !beta) return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  if (!(std::isfinite(ks) && ks > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (s_in && !aligned16(s_in)) || (s_out && !aligned16(s_out)))
+    return GDN_ERR_MISALIGNED;
+  const size_t n = size_t(B) * T * N * H * D * 2;
+  if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
+    return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                             const float* gamma, const float* beta, const float* state_in,
+                             gdn_bf16* out, float* state_out, int B, int H, int T, int N, int D,
+                             float key_scale, gdn_stream_t stream) {
+  if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, T, N,
+                                     D, key_scale))
+    return s;
+  const Problem p{B, H, T, N, D, key_scale};
+  return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                          const float* gamma, const float* beta, const float* state_in,
+                          gdn_bf16* out, float* state_out, int B, int H, int N, int D,
+                          float key_scale, gdn_stream_t stream) {
+  if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, 1, N,
+                                     D, key_scale))
+    return s;
+  const Problem p{B, H, 1, N, D, key_scale};
+  return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_frame_stats(const gdn_bf16* k, const gdn_bf16* v, gdn_bf16* A_out, float* B_out,
+                           int B, int H, int T, int N, int D, float key_scale,
+                           gdn_stream_t stream) {
+  if (!k || !v || !A_out || !B_out) return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(A_out) || !aligned16(B_out))
+    return GDN_ERR_MISALIGNED;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const Problem p{B, H, T, N, D, key_scale};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (D <= 64) return run_stats<64>(dev, p, k, v, A_out, B_out, st);
+  return run_stats<128>(dev, p, k, v, A_out, B_out, st);
+}
+
+gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                               const float* state_in, const float* z_in, gdn_bf16* out,
+                               float* state_out, float* z_out, int B, int H, int T, int N, int D,
+                               int frames_per_block, gdn_stream_t stream) {
+  if (!q || !k || !v || !out) return GDN_ERR_INVALID_ARG;
+  if (frames_per_block < 1) return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 120)) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GDN_ERR_MISALIGNED;
+  const size_t n = size_t(B) * T * N * H * D * 2;
+  if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
+    return GDN_ERR_INVALID_ARG;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Problem p{B, H, T, N, D, 1.0f};
+  const long count = long(B) * H * T;
+  const size_t per = size_t(D + 1) * D;
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, align256(count * per * 4) + align256(count * per * 2),
+                                   st, &base))
+    return s;
+  float* Bws = static_cast<float*>(base);
+  void* Sws = static_cast<uint8_t*>(base) + align256(count * per * 4);
+  {
+    using L = gdn::StatsLayout<128, true>;
+    CUtensorMap tk, tv;
+    if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
+    auto kern = gdn::gdn_stats_kernel<128, true>;
+    if (gdn_status s = ensure_smem_attr(dev, 7, kern, L::kSmemBytes)) return s;
+    const int grid = static_cast<int>(count < g_dev[dev].sms ? count : g_dev[dev].sms);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, nullptr, Bws, p);
+    if (gdn_status s = check_launch()) return s;
+  }
+  {
+    dim3 grid(static_cast<unsigned>((per + 255) / 256), static_cast<unsigned>(B * H));
+    gdn::gdn_la_scan_kernel<<<grid, 256, 0, st>>>(Bws, static_cast<__nv_bfloat16*>(Sws), state_in,
+                                                  z_in, state_out, z_out, H, T, D,
+                                                  frames_per_block);
+    if (gdn_status s = check_launch()) return s;
+  }
+  return run_output<128, true>(dev, p, q, Sws, D + 1, out, frames_per_block, st);
+}
+
+size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {
+  (void)N;
+  if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
+  return forward_ws_bytes(long(B) * H * T, D);
+}
+
+size_t gdn_la_workspace_bytes(int B, int H, int T, int D) {
+  if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
+  const size_t count = size_t(B) * H * T, per = size_t(D + 1) * D;
+  return align256(count * per * 4) + align256(count * per * 2);
+}
+
+const char* gdn_status_string(gdn_status status) {
+  switch (status) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_INVALID_ARG: return "invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "unsupported head dimension";
+    case GDN_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case GDN_ERR_NO_MEMORY: return "workspace allocation failed";
+    case GDN_ERR_CUDA: return "CUDA error";
+    case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+gdn_status gdn_sync_status(gdn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  int code = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&code, gdn::g_status, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+  if (code != 0 && cudaMemcpyToSymbol(gdn::g_status, &zero, sizeof(int)) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return static_cast<gdn_status>(code);
+}
+
+void gdn_release_workspace(void) {
+  int dev;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (d.ws) {
+    cudaDeviceSynchronize();
+    cudaFree(d.ws);
+  }
+  d.ws = nullptr;
+  d.ws_bytes = 0;
+}
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,290 @@
+// Output: O_t = Q_t S_t^T for every frame of every head, in parallel (every token of frame t
+// reads the post-update state S_t, so attention is bidirectional inside a frame and causal
+// across frames).
+//
+// Per work item (b, t, h): S_t (bf16, D x D, row v / column k) is TMA-loaded once as a K-major
+// B operand; the frame's Q rows stream through a ring of 128-token TMA tiles (K-major A
+// operand); each tile is one 128 x DP x DP tcgen05 GEMM into a double-buffered TMEM
+// accumulator; the epilogue converts rows to bf16 and stores them to out[b, t, n, h, :].
+//
+// LA mode (block-causal linear attention): Q tiles are passed through relu in shared memory
+// by 4 transform warps before the MMA, the state row D holds the normaliser z, and the
+// epilogue divides the first D columns by (column D + 1e-6).
+//
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2..5 epilogue,
+// warps 6..9 (LA only) transform.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace gdn {
+
+template <int DP, bool kLA>
+struct OutputLayout {
+  static constexpr int kBoxes = DP / 64;
+  static constexpr int kQBytes = kBoxes * kBoxBytes;   // 128 tokens x DP bf16
+  static constexpr int kSBufBytes = DP * DP * 2;       // DP/64 blocks of DP rows x 128 B
+  static constexpr int kStages = (DP == 128) ? 4 : 8;
+  static constexpr int kThreads = kLA ? 320 : 192;
+  static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
+  static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 512 + 1024;
+};
+
+// state_rows: rows of one stored state (D for GDN, D+1 for LA).
+// frames_per_block: 1 for GDN (frame t reads S_t); F for LA (frame t reads the state at the end
+// of its block of F frames).
+template <int DP, bool kLA>
+__global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
+    gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_s, __nv_bfloat16* __restrict__ out,
+                      Problem p, int frames_per_block) {
+  using L = OutputLayout<DP, kLA>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1k(smem_raw);
+  uint8_t* s_buf = smem;                          // 2 state buffers
+  uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(q_ring + L::kStages * L::kQBytes);
+  uint64_t* ready = full + L::kStages;
+  uint64_t* empty = ready + L::kStages;
+  uint64_t* s_full = empty + L::kStages;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* acc_full = s_empty + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const long n_items = static_cast<long>(p.B) * p.T * p.H;
+  const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
+  const int F = frames_per_block;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&s_full[a], 1);
+      mbar_init(&s_empty[a], 1);
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_s);
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_state = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int li = 0;
+      for (long item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x, ++li) {
+        const int h = static_cast<int>(item % p.H);
+        const int bt = static_cast<int>(item / p.H);
+        const int b = bt / p.T;
+        const int t = bt - b * p.T;
+        const int t_state = (F <= 1) ? t : min((t / F + 1) * F, p.T) - 1;
+        const int srow = (b * p.H + h) * p.T + t_state;
+        const int sb = li & 1;
+        if (!mbar_wait(&s_empty[sb], ((li >> 1) & 1) ^ 1)) {
+          record_error(kErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&s_full[sb], L::kSBufBytes);
+#pragma unroll
+        for (int kb = 0; kb < L::kBoxes; ++kb)
+          tma_load_3d(s_buf + sb * L::kSBufBytes + kb * DP * 128, &tm_s, &s_full[sb], kb * 64, 0,
+                      srow, pol_state);
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) {
+            record_error(kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kQBytes);
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb)
+            tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, &tm_q, &full[stage],
+                        kb * 64, h, tile * kRowsPerTile, bt, pol_stream);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
+    int stage = 0;
+    uint32_t phase = 0;
+    int li = 0;
+    int tc = 0;  // tiles processed (accumulator ring position)
+    bool ok = true;
+    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
+      const int sb = li & 1;
+      if (!mbar_wait(&s_full[sb], (li >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint32_t s_base = smem_u32(s_buf + sb * L::kSBufBytes);
+      for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
+        const int acc = tc & 1;
+        if (!mbar_wait(&acc_empty[acc], ((tc >> 1) & 1) ^ 1) ||
+            !mbar_wait(kLA ? &ready[stage] : &full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t q_base = smem_u32(q_ring + stage * L::kQBytes);
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t da = smem_desc(q_base + kb * kBoxBytes + ks * 32, 16, 1024);
+              const uint64_t db = smem_desc(s_base + kb * DP * 128 + ks * 32, 16, 1024);
+              mma_bf16(tmem_base + acc * DP, da, db, idesc, (kb | ks) != 0);
+            }
+          }
+          mma_commit(&empty[stage]);
+          mma_commit(&acc_full[acc]);
+        }
+        __syncwarp();
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&s_empty[sb]);
+      __syncwarp();
+    }
+    if (!ok) {
+      record_error(kErrTimeout);
+      *abort_flag = 1;
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue
+    const uint32_t quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
+    const int D = p.D;
+    int tc = 0;
+    bool ok = true;
+    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int h = static_cast<int>(item % p.H);
+      const long bt = item / p.H;
+      for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
+        const int acc = tc & 1;
+        if (!mbar_wait(&acc_full[acc], (tc >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int n = tile * kRowsPerTile + row;
+        const uint32_t tacc = lane_base + acc * DP;
+        __nv_bfloat16* orow = out + ((bt * p.N + n) * p.H + h) * static_cast<long>(D);
+        float scale = 1.f;
+        if constexpr (kLA) {
+          float z[32];
+          tmem_ld32(tacc + (D / 32) * 32, z);
+          float den = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j == (D & 31)) den = z[j];
+          scale = 1.f / (den + 1e-6f);
+        }
+        float v[32];
+#pragma unroll 1
+        for (int c = 0; c < DP / 32; ++c) {
+          tmem_ld32(tacc + c * 32, v);
+          if (n < p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              const int col = c * 32 + j;
+              if (col < D) {
+                uint4 pk;
+                if constexpr (kLA) {
+                  pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
+                  pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
+                  pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
+                  pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
+                } else {
+                  pk.x = pack_bf16x2(v[j], v[j + 1]);
+                  pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+                  pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+                  pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
+                }
+                *reinterpret_cast<uint4*>(orow + col) = pk;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[acc]);
+      }
+    }
+    if (!ok) {
+      record_error(kErrTimeout);
+      *abort_flag = 1;
+    }
+  } else if constexpr (kLA) {
+    // ---------------------------------------------------------------- relu(Q) transform
+    const int tid = threadIdx.x - 192;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      for (int tile = 0; tile < n_tiles; ++tile) {
+        if (!mbar_wait(&full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes);
+        const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
+        for (int i = tid; i < L::kQBytes / 16; i += 128) {
+          uint4 x = qt[i];
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
+          qt[i] = x;
+        }
+        fence_async_smem();
+        mbar_arrive(&ready[stage]);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      record_error(kErrTimeout);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace gdn

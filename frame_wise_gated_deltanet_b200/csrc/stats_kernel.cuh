@@ -1,0 +1,316 @@
+// Frame statistics: for every frame t of every head, in parallel,
+//   GDN: A_t = s^2 K_t^T K_t  (stored bf16, D x D, row k', column k)
+//        B_t = s   V_t^T K_t  (stored f32,  D x D, row v,  column k)
+//   LA : B_t = [V_t | 1]^T relu(K_t)  (stored f32, (D+1) x D; row D is sum relu(k), the
+//        normaliser contribution)
+// as tcgen05 GEMMs contracting over the N tokens of the frame. K and V tiles (128 tokens x 64
+// dims per TMA box, 128B-swizzled) are both MMA operands in MN-major form, so the transposes
+// cost nothing. Accumulators live in TMEM (double-buffered across work items so the epilogue
+// of one frame overlaps the MMAs of the next).
+//
+// Warp roles (one CTA per SM, persistent over work items):
+//   warp 0      TMA producer (one elected thread)
+//   warp 1      TMEM allocator + MMA issuer (one elected thread)
+//   warps 2..5  epilogue: TMEM -> registers -> scale -> global
+//   warps 6..9  (LA only) in-place transform of each K/V stage: relu(K), ones column in V
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace gdn {
+
+template <int DP, bool kLA>
+struct StatsLayout {
+  static constexpr int kBoxes = DP / 64;                // 64-dim boxes per operand tile
+  static constexpr int kOpBytes = kBoxes * kBoxBytes;   // 128 tokens x DP dims, bf16
+  static constexpr int kStageBytes = 2 * kOpBytes;      // K tile + V tile
+  static constexpr int kStages = (DP == 128) ? 3 : 6;
+  static constexpr int kAccCols = kLA ? 128 : (DP == 128 ? 256 : 64);
+  static constexpr int kTmemCols = 2 * kAccCols;
+  static constexpr int kThreads = kLA ? 320 : 192;
+  static constexpr int kBarrierBytes = 512;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
+};
+
+// A_ws: [B*H*T, D, D] bf16 (GDN only). B_ws: [B*H*T, brows, D] f32, brows = D (GDN) or D+1 (LA).
+// Work item i = (b*T + t)*H + h; its workspace row is (b*H + h)*T + t.
+template <int DP, bool kLA>
+__global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
+    gdn_stats_kernel(const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
+                     float* __restrict__ B_ws, Problem p) {
+  using L = StatsLayout<DP, kLA>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1k(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
+  uint64_t* ready = full + L::kStages;   // LA: transformed stage
+  uint64_t* empty = ready + L::kStages;
+  uint64_t* acc_full = empty + L::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const long n_items = static_cast<long>(p.B) * p.T * p.H;
+  const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint64_t pol = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (long item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
+        const int h = static_cast<int>(item % p.H);
+        const int bt = static_cast<int>(item / p.H);
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) {
+            record_error(kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          uint8_t* st = smem + stage * L::kStageBytes;
+#pragma unroll
+          for (int j = 0; j < L::kBoxes; ++j) {
+            tma_load_4d(st + j * kBoxBytes, &tm_k, &full[stage], j * 64, h, tile * kRowsPerTile,
+                        bt, pol);
+            tma_load_4d(st + L::kOpBytes + j * kBoxBytes, &tm_v, &full[stage], j * 64, h,
+                        tile * kRowsPerTile, bt, pol);
+          }
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = kLA ? idesc_bf16(128, 128, true, true)
+                                   : (DP == 128 ? idesc_bf16(128, 128, true, true)
+                                                : idesc_bf16(128, 64, true, true));
+    int stage = 0;
+    uint32_t phase = 0;
+    int li = 0;
+    for (long item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
+      const int acc = li & 1;
+      const uint32_t aph = (li >> 1) & 1;
+      if (!mbar_wait(&acc_empty[acc], aph ^ 1)) {
+        record_error(kErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d = tmem_base + acc * L::kAccCols;
+      bool ok = true;
+      for (int tile = 0; tile < n_tiles; ++tile) {
+        if (!mbar_wait(kLA ? &ready[stage] : &full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t base = smem_u32(smem + stage * L::kStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < kRowsPerTile / 16; ++ks) {
+            const uint32_t accum = (tile | ks) != 0;
+            const uint32_t koff = ks * 16 * 128;  // 16 token rows of 128 B
+            if constexpr (kLA) {
+              const uint64_t dv = smem_desc(base + L::kOpBytes + koff, kBoxBytes, 1024);
+              const uint64_t dk = smem_desc(base + koff, kBoxBytes, 1024);
+              mma_bf16(d, dv, dk, idesc, accum);
+            } else if constexpr (DP == 128) {
+              const uint64_t dk = smem_desc(base + koff, kBoxBytes, 1024);
+              const uint64_t dv = smem_desc(base + L::kOpBytes + koff, kBoxBytes, 1024);
+              mma_bf16(d, dk, dk, idesc, accum);        // A_t = K^T K
+              mma_bf16(d + 128, dv, dk, idesc, accum);  // B_t = V^T K
+            } else {
+              // [K | V] stacked along M (K box then V box, kOpBytes apart) times K:
+              // TMEM rows 0..63 = K^T K, rows 64..127 = V^T K.
+              const uint64_t da = smem_desc(base + koff, L::kOpBytes, 1024);
+              const uint64_t db = smem_desc(base + koff, kBoxBytes, 1024);
+              mma_bf16(d, da, db, idesc, accum);
+            }
+          }
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) {
+        record_error(kErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      if (elect_one()) mma_commit(&acc_full[acc]);
+      __syncwarp();
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue
+    const uint32_t quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
+    const float s = p.key_scale;
+    const int D = p.D;
+    const int brows = kLA ? D + 1 : D;
+    int li = 0;
+    for (long item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
+      const int acc = li & 1;
+      const uint32_t aph = (li >> 1) & 1;
+      if (!mbar_wait(&acc_full[acc], aph)) {
+        record_error(kErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int h = static_cast<int>(item % p.H);
+      const long bt = item / p.H;
+      const long b = bt / p.T;
+      const long t = bt - b * p.T;
+      const long ws = (b * p.H + h) * p.T + t;
+      const uint32_t tacc = lane_base + acc * L::kAccCols;
+      float v[32];
+      if constexpr (kLA) {
+        // row = value index v (row D = normaliser); columns = key index
+        float* brow = B_ws + (ws * brows + row) * D;
+#pragma unroll 1
+        for (int c = 0; c < DP / 32; ++c) {
+          tmem_ld32(tacc + c * 32, v);
+          if (row < brows) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const int col = c * 32 + j;
+              if (col < D)
+                *reinterpret_cast<float4*>(brow + col) =
+                    make_float4(v[j] * s, v[j + 1] * s, v[j + 2] * s, v[j + 3] * s);
+            }
+          }
+        }
+      } else {
+        // DP == 128: A in columns [0,128), B in [128,256), TMEM row = matrix row.
+        // DP == 64 : one 64-column accumulator; rows 0..63 = A, rows 64..127 = B.
+        const bool is_a = (DP == 128) ? true : (row < 64);
+        const int mrow = (DP == 128) ? row : (row & 63);
+        const float s2 = s * s;
+#pragma unroll 1
+        for (int part = 0; part < (DP == 128 ? 2 : 1); ++part) {
+          const bool a_part = (DP == 128) ? (part == 0) : is_a;
+          const uint32_t col0 = (DP == 128) ? part * 128 : 0;
+#pragma unroll 1
+          for (int c = 0; c < DP / 32; ++c) {
+            tmem_ld32(tacc + col0 + c * 32, v);
+            if (mrow < D) {
+              if (a_part) {
+                __nv_bfloat16* arow = A_ws + (ws * D + mrow) * D;
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                  const int col = c * 32 + j;
+                  if (col < D) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(v[j] * s2, v[j + 1] * s2);
+                    pk.y = pack_bf16x2(v[j + 2] * s2, v[j + 3] * s2);
+                    pk.z = pack_bf16x2(v[j + 4] * s2, v[j + 5] * s2);
+                    pk.w = pack_bf16x2(v[j + 6] * s2, v[j + 7] * s2);
+                    *reinterpret_cast<uint4*>(arow + col) = pk;
+                  }
+                }
+              } else {
+                float* brow = B_ws + (ws * D + mrow) * D;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                  const int col = c * 32 + j;
+                  if (col < D)
+                    *reinterpret_cast<float4*>(brow + col) =
+                        make_float4(v[j] * s, v[j + 1] * s, v[j + 2] * s, v[j + 3] * s);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+    }
+  } else if constexpr (kLA) {
+    // ---------------------------------------------------------------- LA transform warps
+    const int tid = threadIdx.x - 192;  // 0..127
+    int stage = 0;
+    uint32_t phase = 0;
+    const int D = p.D;
+    for (long item = blockIdx.x; item < n_items; item += gridDim.x) {
+      bool ok = true;
+      for (int tile = 0; tile < n_tiles; ++tile) {
+        if (!mbar_wait(&full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + stage * L::kStageBytes;
+        // relu over the whole K tile (layout-agnostic elementwise)
+        uint4* kt = reinterpret_cast<uint4*>(st);
+        const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
+        for (int i = tid; i < L::kOpBytes / 16; i += 128) {
+          uint4 x = kt[i];
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
+          kt[i] = x;
+        }
+        // ones column at index D of every V row (token), for the normaliser
+        *reinterpret_cast<__nv_bfloat16*>(st + L::kOpBytes +
+                                          swz128_offset_bf16(tid, D, kBoxBytes)) =
+            __float2bfloat16(1.0f);
+        fence_async_smem();
+        mbar_arrive(&ready[stage]);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) {
+        record_error(kErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace gdn

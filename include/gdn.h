@@ -1,0 +1,142 @@
+/*
+ * gdn.h - C ABI of the frame-wise Gated DeltaNet (GDN) frame-scan library for NVIDIA B200
+ * (sm_100a). Every entry point is asynchronous on the caller's CUDA stream.
+ *
+ * The layer (one head; sources: "NVIDIA SANA-WM: минутное 720p видео с одной видеокарты",
+ * gen-hub.ru, section "Архитектура: четыре нетривиальных решения" -- decay gate gamma,
+ * delta-rule residual correction beta, constant D x D state, key scale 1/sqrt(D*S); "SANA-WM:
+ * Efficient Minute-Scale World Modeling with Hybrid Linear Diffusion Transformer", chatpaper.ai
+ * abstract, design (1) -- the GDN is frame-wise):
+ *
+ *     k' = key_scale * k
+ *     A_t = K'_t^T K'_t,   B_t = V_t^T K'_t                       (D x D each)
+ *     S_t = gamma_t * S_{t-1} (I - beta_t A_t) + beta_t B_t        (fp32 state, row v, col k)
+ *     O_t = Q_t S_t^T                                              (bf16 output)
+ *
+ * so attention is bidirectional within a frame (every token of frame t reads S_t) and causal
+ * across frames.
+ *
+ * Common conventions
+ *  - Pointers are DEVICE pointers owned by the caller; the library never frees them.
+ *  - q, k, v, out: [B, T, N, H, D] bfloat16 (gdn_bf16 = raw bf16 bits), contiguous, token-major
+ *    (frame t of head h is N rows of D values with a row stride of H*D elements).
+ *  - gamma, beta: [B, T, H] float32 (decay gate and delta-rule strength, used as given).
+ *  - state: [B, H, D, D] float32, row-major, row = value index, column = key index, so that
+ *    S k is a value. A NULL state_in means S_0 = 0; a NULL state_out skips the final store.
+ *  - D must be a multiple of 8 in [8, 128]; B, H, T, N >= 1; every tensor pointer must be
+ *    16-byte aligned (GDN_ERR_MISALIGNED otherwise).
+ *  - out must not overlap q, k or v (GDN_ERR_INVALID_ARG). state_out may equal state_in
+ *    (in-place streaming); any other partial overlap is undefined.
+ *  - Errors found on the host are returned before anything is launched. Launch failures return
+ *    GDN_ERR_CUDA. Kernels never trap: a device-side wait that exceeds its time limit records
+ *    GDN_ERR_TIMEOUT in a per-device status word that gdn_sync_status() reports.
+ *  - The library keeps one cached device workspace per GPU (see gdn_workspace_bytes); it grows
+ *    on demand (a device-wide synchronisation, refused with GDN_ERR_NO_MEMORY while the stream
+ *    is being captured) and is shared by all calls on that GPU: calls on different streams of
+ *    the same GPU must not run concurrently. gdn_release_workspace() frees it.
+ *  - No CPU fallback exists: without a CUDA device every call returns GDN_ERR_CUDA.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* A cudaStream_t. NULL means the legacy default stream. */
+typedef struct CUstream_st* gdn_stream_t;
+/* Raw bfloat16 bits. */
+typedef uint16_t gdn_bf16;
+
+typedef enum gdn_status {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1, /* null pointer, size out of range, overlapping out, bad scale */
+  GDN_ERR_UNSUPPORTED = 2, /* head dim not supported by this entry point */
+  GDN_ERR_MISALIGNED = 3,  /* a tensor pointer is not 16-byte aligned */
+  GDN_ERR_NO_MEMORY = 4,   /* workspace allocation failed (or growth during capture) */
+  GDN_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  GDN_ERR_TIMEOUT = 6      /* a device-side bounded wait ran out (from gdn_sync_status) */
+} gdn_status;
+
+/*
+ * gdn_frame_forward - frame-wise GDN over a whole clip of T frames.
+ * Computes out (all T frames) and, if state_out != NULL, S_T.
+ * key_scale: the scale applied to keys (1/sqrt(D*N) for the pages' setting); finite, > 0.
+ * Workspace: gdn_workspace_bytes(B, H, T, N, D) bytes (per-frame A_t, B_t and S_t).
+ */
+gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                             const float* gamma, const float* beta, const float* state_in,
+                             gdn_bf16* out, float* state_out, int B, int H, int T, int N, int D,
+                             float key_scale, gdn_stream_t stream);
+
+/*
+ * gdn_frame_step - one streaming step: one new frame per stream, carried state.
+ * q, k, v, out: [B, N, H, D] bf16; gamma, beta: [B, H] f32; state_in, state_out:
+ * [B, H, D, D] f32 (state_in may be NULL for S_0 = 0; state_out == state_in is allowed and is
+ * the usual streaming call). Equivalent to gdn_frame_forward with T = 1 (the chunk-causal and
+ * distilled autoregressive inference modes advance the state one latent frame at a time:
+ * gen-hub.ru SANA-WM article, section "Три режима на любой вкус").
+ */
+gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                          const float* gamma, const float* beta, const float* state_in,
+                          gdn_bf16* out, float* state_out, int B, int H, int N, int D,
+                          float key_scale, gdn_stream_t stream);
+
+/*
+ * gdn_frame_stats - the frame statistics alone, for every frame in parallel:
+ *   A_out[b,h,t] = A_t = s^2 K_t^T K_t   as bfloat16, [B, H, T, D, D] (row k', column k)
+ *   B_out[b,h,t] = B_t = s   V_t^T K_t   as float32,  [B, H, T, D, D] (row v,  column k)
+ * k, v: [B, T, N, H, D] bf16. Both outputs are caller-owned device buffers (no workspace).
+ */
+gdn_status gdn_frame_stats(const gdn_bf16* k, const gdn_bf16* v, gdn_bf16* A_out, float* B_out,
+                           int B, int H, int T, int N, int D, float key_scale,
+                           gdn_stream_t stream);
+
+/*
+ * gdn_block_causal_la - block-causal linear attention (the predecessor layer: "SANA-Video:
+ * Efficient Video Generation with Block Linear Diffusion Transformer", ICLR 2026 oral talk,
+ * block KV cache passage -- the D x D state of block i is the cached state of block i-1 plus
+ * block i's contribution). Blocks are frames_per_block consecutive frames (the last block may
+ * be shorter); every token of block j reads the state after block j:
+ *   S += relu(K_j)^T V_j,  z += sum_i relu(k_i),  o = relu(q) S / (relu(q) . z + 1e-6).
+ * q, k, v, out: [B, T, N, H, D] bf16. state_in/state_out: [B, H, D, D] f32 in the key-major
+ * layout of that formula (row = key index k, column = value index v); z_in/z_out: [B, H, D] f32.
+ * Any of state_in, z_in (S_0 = 0, z_0 = 0) and state_out, z_out may be NULL.
+ * D must be a multiple of 8 in [8, 120] (one spare column carries the normaliser).
+ * Workspace: gdn_la_workspace_bytes(B, H, T, D).
+ */
+gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                               const float* state_in, const float* z_in, gdn_bf16* out,
+                               float* state_out, float* z_out, int B, int H, int T, int N, int D,
+                               int frames_per_block, gdn_stream_t stream);
+
+/* Device workspace bytes gdn_frame_forward / gdn_frame_step need for these sizes. */
+size_t gdn_workspace_bytes(int B, int H, int T, int N, int D);
+/* Device workspace bytes gdn_block_causal_la needs. */
+size_t gdn_la_workspace_bytes(int B, int H, int T, int D);
+
+/* Static description of a status code (never NULL). */
+const char* gdn_status_string(gdn_status status);
+
+/*
+ * gdn_sync_status - synchronise `stream`, then return and clear the device status word of the
+ * current GPU: GDN_OK, GDN_ERR_TIMEOUT if a kernel gave up a bounded wait, or GDN_ERR_CUDA if
+ * the synchronisation itself failed.
+ */
+gdn_status gdn_sync_status(gdn_stream_t stream);
+
+/* Free the cached workspace of the current GPU (synchronises the device first). */
+void gdn_release_workspace(void);
+
+/* Library ABI version (major * 100 + minor). */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,101 @@
+"""The C-ABI library loads without a GPU, exports every symbol include/gdn.h declares, and its
+host-side argument checks answer before any CUDA call (CPU only; no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from frame_wise_gated_deltanet_b200 import build
+    build.build()
+    from frame_wise_gated_deltanet_b200 import _lib
+    return _lib.LIB
+
+
+def test_header_declares_the_entry_points():
+    syms = _declared_symbols()
+    for s in ("gdn_frame_forward", "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
+              "gdn_status_string", "gdn_sync_status", "gdn_release_workspace"):
+        assert s in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from frame_wise_gated_deltanet_b200 import _lib
+    syms = _declared_symbols()
+    for s in syms:
+        assert hasattr(lib, s), f"libgdn.so does not export {s}"
+        assert s in _lib.SIGNATURES, f"binding has no signature for {s}"
+    assert set(_lib.SIGNATURES) == set(syms)
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.gdn_status_string(code)
+    assert lib.gdn_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    # 720p clip: per frame-head A (bf16) + B (f32) + S (bf16) = 128 KiB
+    n = lib.gdn_workspace_bytes(1, 20, 961, 880, 128)
+    assert n >= 1 * 20 * 961 * 128 * 128 * (2 + 4 + 2)
+    assert n < 1 * 20 * 961 * 128 * 128 * (2 + 4 + 2) + 4096
+    assert lib.gdn_la_workspace_bytes(2, 20, 81, 112) >= 2 * 20 * 81 * 113 * 112 * 6
+    assert lib.gdn_workspace_bytes(0, 1, 1, 1, 8) == 0
+
+
+P = 4096  # a fake, 16-byte aligned "device address"; never dereferenced by these calls
+
+
+def _fwd(lib, q=P, k=P + 0x10000, v=P + 0x20000, g=P + 0x30000, b=P + 0x31000, si=None,
+         out=P + 0x40000, so=None, B=1, H=2, T=3, N=16, D=32, ks=0.1):
+    return lib.gdn_frame_forward(q, k, v, g, b, si, out, so, B, H, T, N, D, ks, None)
+
+
+def test_forward_rejects_bad_arguments_on_the_host(lib):
+    assert _fwd(lib, q=None) == 1
+    assert _fwd(lib, g=None) == 1
+    assert _fwd(lib, B=0) == 1
+    assert _fwd(lib, N=0) == 1
+    assert _fwd(lib, D=36) == 2     # not a multiple of 8
+    assert _fwd(lib, D=136) == 2    # above 128
+    assert _fwd(lib, ks=0.0) == 1
+    assert _fwd(lib, ks=float("nan")) == 1
+    assert _fwd(lib, q=P + 8) == 3  # misaligned
+    assert _fwd(lib, out=P + 0x10000) == 1  # out overlaps k
+
+
+def test_valid_call_without_gpu_fails_loudly(lib):
+    # Arguments pass the host checks, then the library needs a CUDA device: no CPU fallback.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _fwd(lib) == 5
+
+
+def test_la_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_block_causal_la
+    assert f(P, P + 0x10000, P + 0x20000, None, None, P + 0x40000, None, None, 1, 1, 4, 8, 128,
+             2, None) == 2  # D = 128 leaves no column for the normaliser
+    assert f(P, P + 0x10000, P + 0x20000, None, None, P + 0x40000, None, None, 1, 1, 4, 8, 32,
+             0, None) == 1  # frames_per_block < 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from frame_wise_gated_deltanet_b200 import api
+    q = torch.zeros((1, 2, 16, 2, 32), dtype=torch.bfloat16)
+    g = torch.zeros((1, 2, 2), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        api.gdn_frame_forward(q, q, q, g, g)
