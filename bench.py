@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark of the frame-wise Gated DeltaNet layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdn|reference]
+
+One step = one gdn_frame_forward over the 720p 60 s clip (B1 H20 D128 T961 N880, 22x40 latent
+grid, synthetic seeded bf16 inputs resident in HBM). Prints one JSON line (rank 0).
+
+* value: whole-job tokens*heads/s = (units all ranks processed) / (max over ranks of the
+  device time of K steps, CUDA events on the launching stream).
+* e2e: the same metric through the public API with pinned HOST buffers: every step copies
+  q, k, v, gamma, beta host->device and reads out and the final state back.
+* roofline: the dominant kernel (largest share of the timed region, timed live with CUDA
+  events the library records around each of its launches) against the measured HBM copy
+  bandwidth; traffic from the committed ncu summary when the kernel sources still match it.
+* cpu_baseline: the fp64 oracle on a bounded sample of the same workload (rank 0, N = 1).
+* --impl reference: the oracle itself as the reference arm (host cores, bounded samples).
+
+Multi-GPU (torchrun): every rank processes its own clip (independent problems, no collective
+on the data path), so scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN layer tokens·heads/sec and % of roofline (720p 60 s config, 1 B200)"
+UNIT = "tokens*heads/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def args_parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
+    ap.add_argument("--workload", default="720p")
+    ap.add_argument("--frames", type=int, default=0,
+                    help="truncate the clip to its first FRAMES frames (small profiling cases)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w):
+    """Bytes the layer must move per clip: Q, K, V read and O written (bf16), gamma and beta,
+    and the fp32 state written (S_0 = 0 is not read)."""
+    fh = w.B * w.H * w.T
+    return fh * (4 * w.N * w.D * 2) + w.B * w.T * w.H * 2 * 4 + w.B * w.H * w.D * w.D * 4
+
+
+def kernel_bytes(name, w):
+    """Algorithmic bytes per launch of each kernel of the forward (the bytes its stage must
+    move in the three-kernel design)."""
+    fh = w.B * w.H * w.T
+    nd2 = w.N * w.D * 2
+    dd = w.D * w.D
+    if name == "gdn_stats_kernel":       # read K, V; write A_t (bf16) and B_t (f32)
+        return fh * (2 * nd2 + dd * 2 + dd * 4)
+    if name == "gdn_chain_kernel":       # read A_t, B_t, gamma, beta; write S_t (bf16), S_T
+        return fh * (dd * 2 + dd * 4 + dd * 2 + 8) + w.B * w.H * dd * 4
+    if name == "gdn_output_kernel":      # read Q, S_t; write O
+        return fh * (2 * nd2 + dd * 2)
+    return None
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "frame_wise_gated_deltanet_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` from profiles/traffic.json, if it was taken on the
+    current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t["kernels"][kernel]
+        if t.get("source_digest") != source_digest() or e.get("workload") != workload:
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples of one GPU while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        self.t0 = time.time()
+
+    def stop(self):
+        self.t1 = time.time()
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # the sampler ran from just before to just after the timed region; keep loaded samples
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample_rate(w, heads, frames, seed=99):
+    """The fp64 oracle on a bounded sample of workload `w` (`heads` heads, `frames` frames, same
+    token count and head dim). Returns (tokens*heads/s, seconds, threads)."""
+    import numpy as np
+    import gdn_inputs
+    import oracle
+    x = gdn_inputs.clip_inputs(1, heads, frames, w.N, w.D, w.gamma_range, w.beta_range, seed=seed)
+    f = lambda t: t.float().numpy()
+    args = [f(x["q"]), f(x["k"]), f(x["v"]), f(x["gamma"]), f(x["beta"])]
+    t0 = time.perf_counter()
+    oracle.gdn_frame_forward(*args, None, w.key_scale)
+    dt = time.perf_counter() - t0
+    try:
+        import threadpoolctl
+        threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info())
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    return heads * frames * w.N / dt, dt, threads
+
+
+def run_reference(a, w):
+    """The oracle as the reference arm: each step is a bounded sample (1 head x 192 frames)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    heads, frames = 1, 192
+    for _ in range(a.warmup):
+        oracle_sample_rate(w, heads, frames)
+    rates, secs, threads = [], 0.0, 1
+    for _ in range(a.steps):
+        r, dt, threads = oracle_sample_rate(w, heads, frames)
+        rates.append(r)
+        secs += dt
+    units = a.steps * heads * frames * w.N
+    value = units / secs
+    sample = f"{heads} head x {frames} frames of the {w.name} clip (N={w.N}, D={w.D}) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def workload_config(w):
+    return {"workload": f"{w.name} GDN clip: B{w.B} H{w.H} D{w.D} T{w.T} N{w.N} ({w.grid} grid)",
+            "B": w.B, "H": w.H, "D": w.D, "T": w.T, "N": w.N, "key_scale": w.key_scale,
+            "gamma_range": list(w.gamma_range), "beta_range": list(w.beta_range),
+            "l2": "inputs (%.1f GB of q,k,v) larger than the 126 MB L2; no flush"
+                  % (3 * w.B * w.T * w.N * w.H * w.D * 2 / 1e9),
+            "parallelism": "independent clip per GPU"}
+
+
+def main():
+    a = args_parse()
+    import dataclasses
+    import gdn_inputs
+    w = gdn_inputs.WORKLOADS[a.workload]
+    if a.frames > 0:
+        w = dataclasses.replace(w, T=a.frames, name=f"{w.name}[:{a.frames}]")
+    if a.impl == "reference":
+        run_reference(a, w)
+        return
+
+    import torch
+    from frame_wise_gated_deltanet_b200 import _lib, api
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    g = gdn_inputs.workload_inputs(w, device=dev)
+    q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
+    out = torch.empty_like(q)
+    st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+    def step():
+        api.gdn_frame_forward(q, k, v, gam, bet, None, out, st, key_scale=w.key_scale,
+                              stream=stream)
+
+    for _ in range(max(a.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if api.gdn_sync_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    # per-launch events the library records around each kernel (created before arming)
+    n_ev = 2 * 8 * a.steps
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in evs:
+        e.record(stream)
+    import ctypes
+    handles = (ctypes.c_void_p * n_ev)(*[e.cuda_event for e in evs])
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid))
+
+    torch.cuda.synchronize()
+    barrier(world)
+    _lib.LIB.gdn_profile_arm(handles, n_ev)
+    sampler.start()
+    t_start.record(stream)
+    for _ in range(a.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    launches = _lib.LIB.gdn_profile_count()
+    names = [_lib.LIB.gdn_profile_kernel(i).decode() for i in range(launches)]
+    _lib.LIB.gdn_profile_arm(None, 0)
+    barrier(world)
+    status = api.gdn_sync_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    ms_local = t_start.elapsed_time(t_end)
+    ms = max_over_ranks(ms_local, world)
+    per_kernel = {}
+    for i, n in enumerate(names):
+        d = evs[2 * i].elapsed_time(evs[2 * i + 1])
+        tot, cnt = per_kernel.get(n, (0.0, 0))
+        per_kernel[n] = (tot + d, cnt + 1)
+    dom = max(per_kernel, key=lambda n: per_kernel[n][0])
+    dom_ms = per_kernel[dom][0] / per_kernel[dom][1]
+    hbm, peak_kind = peaks()
+    kb = kernel_bytes(dom, w)
+    achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
+    units = w.tokens_heads * world * a.steps
+    value = units / (ms * 1e-3)
+    path_bytes = algorithmic_bytes(w)
+    path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
+
+    # ---------------------------------------------------------------- end to end, host buffers
+    e2e = None
+    if not a.no_e2e:
+        e2e = measure_e2e(a, w, g, out, st, stream, world, dev)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w),
+        "roofline": {
+            "bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": (achieved / hbm) if achieved else None,
+            "peak_source": f"{peak_kind} HBM copy bandwidth",
+            "traffic": ncu_traffic(dom, w.name),
+            "algorithmic_bytes_per_launch": kb, "ms_per_launch": dom_ms,
+            "path": {"algorithmic_bytes_per_step": path_bytes, "achieved_gbs": path_gbs,
+                     "frac": path_gbs / hbm},
+        },
+        "kernels": {n: {"launches": c, "ms_total": t, "share": t / sum(x[0] for x in per_kernel.values())}
+                    for n, (t, c) in per_kernel.items()},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rate, secs, threads = oracle_sample_rate(w, 4, w.T)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"4 heads x {w.T} frames of the {w.name} clip shape "
+                                          f"(N={w.N}, D={w.D}), {secs:.1f} s of fp64 numpy"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def measure_e2e(a, w, g, out, st, stream, world, dev):
+    """Throughput through the public API with pinned host inputs and outputs."""
+    import torch
+    from frame_wise_gated_deltanet_b200 import api
+    try:
+        import psutil
+        need = sum(t.numel() * t.element_size() for t in (g["q"], g["k"], g["v"], out))
+        if psutil.virtual_memory().available < 1.5 * need * world:
+            return {"value": None, "unit": UNIT, "reason": "not enough host memory to pin"}
+    except ImportError:
+        pass
+    host = {n: torch.empty(g[n].shape, dtype=g[n].dtype, pin_memory=True)
+            for n in ("q", "k", "v", "gamma", "beta")}
+    for n in host:
+        host[n].copy_(g[n])
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    st_h = torch.empty(st.shape, dtype=st.dtype, pin_memory=True)
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+    dg, db = torch.empty_like(g["gamma"]), torch.empty_like(g["beta"])
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            dq.copy_(host["q"], non_blocking=True)
+            dk.copy_(host["k"], non_blocking=True)
+            dv.copy_(host["v"], non_blocking=True)
+            dg.copy_(host["gamma"], non_blocking=True)
+            db.copy_(host["beta"], non_blocking=True)
+            api.gdn_frame_forward(dq, dk, dv, dg, db, None, out, st, key_scale=w.key_scale,
+                                  stream=stream)
+            out_h.copy_(out, non_blocking=True)
+            st_h.copy_(st, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    steps = max(1, a.e2e_steps)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    s0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s0.elapsed_time(s1), world)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + st_h.numel() * st_h.element_size()
+    return {"value": w.tokens_heads * world * steps / (ms * 1e-3), "unit": UNIT,
+            "steps": steps, "ms_per_step": ms / steps, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    main()

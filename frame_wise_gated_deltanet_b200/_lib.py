@@ -36,6 +36,9 @@ SIGNATURES = {
     "gdn_sync_status": (_I, [_P]),
     "gdn_release_workspace": (None, []),
     "gdn_version": (_I, []),
+    "gdn_profile_arm": (_I, [_P, _I]),
+    "gdn_profile_count": (_I, []),
+    "gdn_profile_kernel": (ctypes.c_char_p, [_I]),
 }
 
 

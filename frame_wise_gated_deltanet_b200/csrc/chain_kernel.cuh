@@ -7,7 +7,8 @@
 // the epilogue into shared memory, A_t as a bf16 K-major operand loaded by TMA, f32
 // accumulate in TMEM). B_t (f32) arrives by TMA in 128B-swizzled 32-column blocks so that each
 // thread reads its own row without bank conflicts. Each S_t is written to the workspace as a
-// bf16 row-major D x D matrix, the operand of the output GEMM.
+// bf16 row-major D x D matrix (the operand of the output GEMM) by one TMA store of the bf16
+// operand tile, issued by the MMA thread before it reads the same tile for the next frame.
 //
 // Warp roles: warp 0 TMA producer (A_t, B_t, two stages, one frame ahead), warp 1 TMEM
 // allocator + MMA issuer, warps 2..9 epilogue (warp w owns rows 32*(w%4).. and column half
@@ -36,9 +37,10 @@ struct ChainLayout {
 template <int DP>
 __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
     gdn_chain_kernel(const __grid_constant__ CUtensorMap tm_a,
-                     const __grid_constant__ CUtensorMap tm_b, const float* __restrict__ gamma,
+                     const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_s, const float* __restrict__ gamma,
                      const float* __restrict__ beta, const float* __restrict__ state_in,
-                     __nv_bfloat16* __restrict__ S_ws, float* __restrict__ state_out, Problem p) {
+                     float* __restrict__ state_out, Problem p) {
   using L = ChainLayout<DP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
@@ -47,7 +49,8 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
   uint64_t* empty = full + L::kStages;
   uint64_t* mma_done = empty + L::kStages;
   uint64_t* s_ready = mma_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_ready + 1);
+  uint64_t* s_stored = s_ready + 1;  // the TMA store of the S tile has read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_stored + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id();
@@ -65,6 +68,7 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(s_ready, 256);
+    mbar_init(s_stored, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -82,9 +86,19 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
       const uint64_t pol = policy_evict_first();
+      // pull A_t and B_t of frames kPrefetch ahead into L2 so the per-frame loads below hit L2
+      constexpr int kPrefetch = 8;
+      auto prefetch = [&](int f) {
+#pragma unroll
+        for (int kb = 0; kb < DP / 64; ++kb) tma_prefetch_3d(&tm_a, kb * 64, 0, bh * T + f);
+#pragma unroll
+        for (int cb = 0; cb < DP / 32; ++cb) tma_prefetch_3d(&tm_b, cb * 32, 0, bh * T + f);
+      };
+      for (int f = 0; f < kPrefetch && f < T; ++f) prefetch(f);
       int stage = 0;
       uint32_t phase = 0;
       for (int t = 0; t < T; ++t) {
+        if (t + kPrefetch < T) prefetch(t + kPrefetch);
         if (!mbar_wait(&empty[stage], phase ^ 1)) {
           record_error(kErrTimeout);
           *abort_flag = 1;
@@ -109,16 +123,28 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
   } else if (warp == 1) {
     constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
     const uint32_t s_base = smem_u32(s_tile);
+    const uint64_t pol_s = policy_evict_last();
+    if (lane == 0) tma_prefetch_desc(&tm_s);
+    // The S tile holds S_{t-1} when step t starts; store it as frame t-1's state (t >= 1),
+    // then multiply it by A_t. The epilogue overwrites the tile only after both the MMAs
+    // (mma_done) and the store's read of the tile (s_stored) are complete.
+    auto store_tile = [&](int frame) {
+#pragma unroll
+      for (int kb = 0; kb < DP / 64; ++kb)
+        tma_store_3d(&tm_s, s_tile + kb * L::kSBlockBytes, kb * 64, 0, bh * T + frame, pol_s);
+      bulk_commit();
+    };
     int stage = 0;
     uint32_t phase = 0;
+    bool ok = true;
     for (int t = 0; t < T; ++t) {
       if (!mbar_wait(&full[stage], phase) || !mbar_wait(s_ready, t & 1)) {
-        record_error(kErrTimeout);
-        *abort_flag = 1;
+        ok = false;
         break;
       }
       tc_fence_after();
       if (elect_one()) {
+        if (t > 0) store_tile(t - 1);
         const uint32_t a_base = smem_u32(smem + stage * L::kStageBytes);
 #pragma unroll
         for (int kb = 0; kb < DP / 64; ++kb) {
@@ -130,12 +156,25 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
           }
         }
         mma_commit(mma_done);
+        bulk_wait_read<0>();
+        mbar_arrive(s_stored);
       }
       __syncwarp();
       if (++stage == L::kStages) {
         stage = 0;
         phase ^= 1;
       }
+    }
+    // the last state S_{T-1}
+    if (ok && !mbar_wait(s_ready, T & 1)) ok = false;
+    if (elect_one()) {
+      if (ok) store_tile(T - 1);
+      bulk_wait_all();
+    }
+    __syncwarp();
+    if (!ok) {
+      record_error(kErrTimeout);
+      *abort_flag = 1;
     }
   } else {
     // ---------------------------------------------------------------- epilogue (256 threads)
@@ -170,11 +209,26 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
 
     int stage = 0;
     uint32_t phase = 0;
+    // gamma_t, beta_t: each lane holds frame (32*blk + lane) of the current and next block of
+    // 32 frames; the value for frame t is shuffled from lane t % 32.
     const long gb_base = static_cast<long>(b) * T * p.H + h;
+    auto load_gb = [&](int blk, float& gv, float& bv) {
+      const int f = blk * 32 + static_cast<int>(lane);
+      gv = f < T ? __ldg(gamma + gb_base + static_cast<long>(f) * p.H) : 0.f;
+      bv = f < T ? __ldg(beta + gb_base + static_cast<long>(f) * p.H) : 0.f;
+    };
+    float g_cur, b_cur, g_next, b_next;
+    load_gb(0, g_next, b_next);
     for (int t = 0; t < T; ++t) {
-      const float g = __ldg(gamma + gb_base + static_cast<long>(t) * p.H);
-      const float be = __ldg(beta + gb_base + static_cast<long>(t) * p.H);
-      if (!mbar_wait(mma_done, t & 1) || !mbar_wait(&full[stage], phase)) {
+      if ((t & 31) == 0) {
+        g_cur = g_next;
+        b_cur = b_next;
+        load_gb((t >> 5) + 1, g_next, b_next);
+      }
+      const float g = __shfl_sync(0xffffffffu, g_cur, t & 31);
+      const float be = __shfl_sync(0xffffffffu, b_cur, t & 31);
+      if (!mbar_wait(mma_done, t & 1) || !mbar_wait(&full[stage], phase) ||
+          !mbar_wait(s_stored, t & 1)) {
         record_error(kErrTimeout);
         *abort_flag = 1;
         break;
@@ -200,20 +254,6 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
       tc_fence_before();
       mbar_arrive(s_ready);
       mbar_arrive(&empty[stage]);
-      if (row_ok) {
-        __nv_bfloat16* srow = S_ws + ((static_cast<long>(bh) * T + t) * D + v) * D;
-#pragma unroll
-        for (int j = 0; j < L::kCols; j += 8) {
-          if (c0 + j < D) {
-            uint4 pk;
-            pk.x = pack_bf16x2(S[j], S[j + 1]);
-            pk.y = pack_bf16x2(S[j + 2], S[j + 3]);
-            pk.z = pack_bf16x2(S[j + 4], S[j + 5]);
-            pk.w = pack_bf16x2(S[j + 6], S[j + 7]);
-            *reinterpret_cast<uint4*>(srow + c0 + j) = pk;
-          }
-        }
-      }
       if (++stage == L::kStages) {
         stage = 0;
         phase ^= 1;

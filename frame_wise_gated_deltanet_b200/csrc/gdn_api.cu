@@ -134,6 +134,31 @@ gdn_status ensure_smem_attr(int dev, int bit, K kernel, int bytes) {
   return GDN_OK;
 }
 
+// ------------------------------------------------------------------ launch profiling
+// When armed, every kernel launch records events[2i] before and events[2i+1] after launch i
+// on the launch's stream, until the caller's array is used up.
+constexpr int kMaxProfiled = 8192;
+cudaEvent_t* g_prof_events = nullptr;
+int g_prof_n = 0;
+int g_prof_count = 0;
+const char* g_prof_names[kMaxProfiled];
+
+struct ProfiledLaunch {
+  int slot = -1;
+  cudaStream_t st;
+  ProfiledLaunch(const char* name, cudaStream_t s) : st(s) {
+    if (g_prof_events != nullptr && 2 * g_prof_count + 1 < g_prof_n &&
+        g_prof_count < kMaxProfiled) {
+      slot = g_prof_count++;
+      g_prof_names[slot] = name;
+      cudaEventRecord(g_prof_events[2 * slot], st);
+    }
+  }
+  ~ProfiledLaunch() {
+    if (slot >= 0) cudaEventRecord(g_prof_events[2 * slot + 1], st);
+  }
+};
+
 // ------------------------------------------------------------------ validation
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -166,7 +191,10 @@ gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, vo
   if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 0 : 1, kern, L::kSmemBytes)) return s;
   const long items = long(p.B) * p.T * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
-  kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, static_cast<__nv_bfloat16*>(A), Bm, p);
+  {
+    ProfiledLaunch pl("gdn_stats_kernel", st);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, static_cast<__nv_bfloat16*>(A), Bm, p);
+  }
   return check_launch();
 }
 
@@ -176,14 +204,17 @@ gdn_status run_chain(int dev, const Problem& p, const void* A, const float* Bm,
                      float* s_out, cudaStream_t st) {
   using L = gdn::ChainLayout<DP>;
   const long count = long(p.B) * p.H * p.T;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ts;
   if (!tmap_mats(&ta, A, false, p.D, p.D, count, DP) ||
-      !tmap_mats(&tb, Bm, true, p.D, p.D, count, DP))
+      !tmap_mats(&tb, Bm, true, p.D, p.D, count, DP) ||
+      !tmap_mats(&ts, S_ws, false, p.D, p.D, count, DP))
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_chain_kernel<DP>;
   if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 2 : 3, kern, L::kSmemBytes)) return s;
-  kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, tb, gamma, beta, s_in,
-                                                      static_cast<__nv_bfloat16*>(S_ws), s_out, p);
+  {
+    ProfiledLaunch pl("gdn_chain_kernel", st);
+    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, tb, ts, gamma, beta, s_in, s_out, p);
+  }
   return check_launch();
 }
 
@@ -192,15 +223,19 @@ gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws
                       void* out, int F, cudaStream_t st) {
   using L = gdn::OutputLayout<DP, kLA>;
   const long count = long(p.B) * p.H * p.T;
-  CUtensorMap tq, ts;
-  if (!tmap_tokens(&tq, q, p) || !tmap_mats(&ts, S_ws, false, p.D, srows, count, DP))
+  CUtensorMap tq, ts, to;
+  if (!tmap_tokens(&tq, q, p) || !tmap_mats(&ts, S_ws, false, p.D, srows, count, DP) ||
+      !tmap_tokens(&to, out, p))
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_output_kernel<DP, kLA>;
   if (gdn_status s = ensure_smem_attr(dev, kLA ? 6 : (DP == 128 ? 4 : 5), kern, L::kSmemBytes))
     return s;
   const long items = long(p.B) * p.T * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
-  kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, ts, static_cast<__nv_bfloat16*>(out), p, F);
+  {
+    ProfiledLaunch pl("gdn_output_kernel", st);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, ts, to, p, F);
+  }
   return check_launch();
 }
 
@@ -340,11 +375,13 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
     auto kern = gdn::gdn_stats_kernel<128, true>;
     if (gdn_status s = ensure_smem_attr(dev, 7, kern, L::kSmemBytes)) return s;
     const int grid = static_cast<int>(count < g_dev[dev].sms ? count : g_dev[dev].sms);
+    ProfiledLaunch pl("gdn_stats_kernel_la", st);
     kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, nullptr, Bws, p);
     if (gdn_status s = check_launch()) return s;
   }
   {
     dim3 grid(static_cast<unsigned>((per + 255) / 256), static_cast<unsigned>(B * H));
+    ProfiledLaunch pl("gdn_la_scan_kernel", st);
     gdn::gdn_la_scan_kernel<<<grid, 256, 0, st>>>(Bws, static_cast<__nv_bfloat16*>(Sws), state_in,
                                                   z_in, state_out, z_out, H, T, D,
                                                   frames_per_block);
@@ -403,5 +440,25 @@ void gdn_release_workspace(void) {
 }
 
 int gdn_version(void) { return 100; }
+
+gdn_status gdn_profile_arm(void* const* events, int n) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (events == nullptr || n < 2) {
+    g_prof_events = nullptr;
+    g_prof_n = 0;
+  } else {
+    g_prof_events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+    g_prof_n = n;
+  }
+  g_prof_count = 0;
+  return GDN_OK;
+}
+
+int gdn_profile_count(void) { return g_prof_count; }
+
+const char* gdn_profile_kernel(int i) {
+  if (i < 0 || i >= g_prof_count) return "";
+  return g_prof_names[i];
+}
 
 }  // extern "C"

@@ -5,7 +5,9 @@
 // Per work item (b, t, h): S_t (bf16, D x D, row v / column k) is TMA-loaded once as a K-major
 // B operand; the frame's Q rows stream through a ring of 128-token TMA tiles (K-major A
 // operand); each tile is one 128 x DP x DP tcgen05 GEMM into a double-buffered TMEM
-// accumulator; the epilogue converts rows to bf16 and stores them to out[b, t, n, h, :].
+// accumulator; the epilogue converts rows to bf16 into a 128B-swizzled staging tile in shared
+// memory and one thread TMA-stores it to out[b, t, n, h, :] (rows past N and columns past D are
+// clipped by the tensor map), so global writes are whole coalesced lines.
 //
 // LA mode (block-causal linear attention): Q tiles are passed through relu in shared memory
 // by 4 transform warps before the MMA, the state row D holds the normaliser z, and the
@@ -25,10 +27,11 @@ struct OutputLayout {
   static constexpr int kBoxes = DP / 64;
   static constexpr int kQBytes = kBoxes * kBoxBytes;   // 128 tokens x DP bf16
   static constexpr int kSBufBytes = DP * DP * 2;       // DP/64 blocks of DP rows x 128 B
-  static constexpr int kStages = (DP == 128) ? 4 : 8;
+  static constexpr int kStages = (DP == 128) ? 3 : 8;
   static constexpr int kThreads = kLA ? 320 : 192;
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
-  static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 512 + 1024;
+  static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
+  static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + 512 + 1024;
 };
 
 // state_rows: rows of one stored state (D for GDN, D+1 for LA).
@@ -37,14 +40,15 @@ struct OutputLayout {
 template <int DP, bool kLA>
 __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
     gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_s, __nv_bfloat16* __restrict__ out,
-                      Problem p, int frames_per_block) {
+                      const __grid_constant__ CUtensorMap tm_s,
+                      const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
   using L = OutputLayout<DP, kLA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
   uint8_t* s_buf = smem;                          // 2 state buffers
   uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
-  uint64_t* full = reinterpret_cast<uint64_t*>(q_ring + L::kStages * L::kQBytes);
+  uint8_t* o_stage = q_ring + L::kStages * L::kQBytes;  // 2 output staging tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(o_stage + 2 * L::kOBytes);
   uint64_t* ready = full + L::kStages;
   uint64_t* empty = ready + L::kStages;
   uint64_t* s_full = empty + L::kStages;
@@ -185,6 +189,9 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
     const int D = p.D;
+    const bool leader = (threadIdx.x == 64);
+    const uint64_t pol_out = policy_evict_first();
+    if (leader) tma_prefetch_desc(&tm_o);
     int tc = 0;
     bool ok = true;
     for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -192,14 +199,15 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
       const long bt = item / p.H;
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
-        if (!mbar_wait(&acc_full[acc], (tc >> 1) & 1)) {
+        const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
+        // staging buffer tc&1 is free once the store issued two tiles ago has read it
+        if (leader) bulk_wait_read<1>();
+        if (named_bar_any(1, 128, !waited)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int n = tile * kRowsPerTile + row;
         const uint32_t tacc = lane_base + acc * DP;
-        __nv_bfloat16* orow = out + ((bt * p.N + n) * p.H + h) * static_cast<long>(D);
         float scale = 1.f;
         if constexpr (kLA) {
           float z[32];
@@ -210,36 +218,35 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
             if (j == (D & 31)) den = z[j];
           scale = 1.f / (den + 1e-6f);
         }
+        uint8_t* ob = o_stage + (tc & 1) * L::kOBytes;
         float v[32];
 #pragma unroll 1
         for (int c = 0; c < DP / 32; ++c) {
           tmem_ld32(tacc + c * 32, v);
-          if (n < p.N) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              const int col = c * 32 + j;
-              if (col < D) {
-                uint4 pk;
-                if constexpr (kLA) {
-                  pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
-                  pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
-                  pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
-                  pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
-                } else {
-                  pk.x = pack_bf16x2(v[j], v[j + 1]);
-                  pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
-                  pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
-                  pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
-                }
-                *reinterpret_cast<uint4*>(orow + col) = pk;
-              }
-            }
+          for (int j = 0; j < 32; j += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
+            pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
+            pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
+            pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
+            *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c * 32 + j, kBoxBytes)) = pk;
           }
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);
+        fence_async_smem();
+        named_bar(1, 128);
+        if (leader) {
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb)
+            tma_store_4d(&tm_o, ob + kb * kBoxBytes, kb * 64, h, tile * kRowsPerTile,
+                         static_cast<int>(bt), pol_out);
+          bulk_commit();
+        }
       }
     }
+    if (leader) bulk_wait_all();
     if (!ok) {
       record_error(kErrTimeout);
       *abort_flag = 1;

@@ -132,6 +132,19 @@ gdn_status gdn_sync_status(gdn_stream_t stream);
 /* Free the cached workspace of the current GPU (synchronises the device first). */
 void gdn_release_workspace(void);
 
+/*
+ * Launch profiling (CUDA events around every kernel the library launches).
+ * gdn_profile_arm(events, n): from now on, launch i (counted from this call) records
+ * events[2i] on its stream just before the kernel and events[2i+1] just after, while
+ * 2i+1 < n. events is an array of n cudaEvent_t created by the caller (the library neither
+ * creates nor destroys them and keeps the pointer until disarmed); events == NULL disarms.
+ * gdn_profile_count(): launches recorded since arming. gdn_profile_kernel(i): the kernel name
+ * of recorded launch i ("" if out of range). Not thread-safe against concurrent library calls.
+ */
+gdn_status gdn_profile_arm(void* const* events, int n);
+int gdn_profile_count(void);
+const char* gdn_profile_kernel(int i);
+
 /* Library ABI version (major * 100 + minor). */
 int gdn_version(void);
 
