@@ -19,6 +19,7 @@ STATUS = {
     4: "GDN_ERR_NO_MEMORY",
     5: "GDN_ERR_CUDA",
     6: "GDN_ERR_TIMEOUT",
+    7: "GDN_ERR_SCRATCH_LIMIT",
 }
 
 # Every symbol include/gdn.h declares, with (restype, argtypes).
@@ -27,6 +28,7 @@ _I = ctypes.c_int
 _F = ctypes.c_float
 SIGNATURES = {
     "gdn_frame_forward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "gdn_frame_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_stats": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_block_causal_la": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),

@@ -15,6 +15,12 @@
 #include "output_kernel.cuh"
 #include "stats_kernel.cuh"
 
+// Scratch of gdn_frame_forward_noalloc: a fixed 64 MiB array in device memory, reserved by the
+// CUDA module on every GPU that loads this library and held until the process exits. Host code
+// only sees a stand-in symbol; the device address comes from cudaGetSymbolAddress.
+static constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 using gdn::Problem;
@@ -284,6 +290,23 @@ gdn_status forward_impl(const void* q, const void* k, const void* v, const float
   return run_output<128, false>(dev, p, q, w.S, p.D, out, 1, st);
 }
 
+// Device address of g_noalloc_scratch on the current GPU, looked up once per GPU (with that GPU
+// current) and cached.
+void* g_noalloc_addr[kMaxDevices];
+
+gdn_status noalloc_scratch(int dev, void** out) {
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return GDN_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return GDN_OK;
+}
+
 gdn_status validate_common(const void* q, const void* k, const void* v, const void* out,
                            const float* gamma, const float* beta, const float* s_in,
                            const float* s_out, int B, int H, int T, int N, int D, float ks) {
@@ -313,6 +336,39 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
   const Problem p{B, H, T, N, D, key_scale};
   return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                     const float* gamma, const float* beta,
+                                     const float* state_in, gdn_bf16* out, float* state_out,
+                                     int B, int H, int T, int N, int D, float key_scale,
+                                     gdn_stream_t stream) {
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  const long count = long(B) * H * T;
+  if (forward_ws_bytes(count, D) > kNoAllocScratchBytes) return GDN_ERR_SCRATCH_LIMIT;
+  if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, T, N,
+                                     D, key_scale))
+    return s;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  void* base = nullptr;
+  if (gdn_status s = noalloc_scratch(dev, &base)) return s;
+  // Every scratch element (A_t, B_t, S_t) is written by this call before it is read, so nothing
+  // needs clearing between calls.
+  const ForwardWs w = carve_forward(base, count, D);
+  const Problem p{B, H, T, N, D, key_scale};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (D <= 64) {
+    if (gdn_status s = run_stats<64>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out, st))
+      return s;
+    return run_output<64, false>(dev, p, q, w.S, D, out, 1, st);
+  }
+  if (gdn_status s = run_stats<128>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out, st))
+    return s;
+  return run_output<128, false>(dev, p, q, w.S, D, out, 1, st);
 }
 
 gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
@@ -411,6 +467,8 @@ const char* gdn_status_string(gdn_status status) {
     case GDN_ERR_NO_MEMORY: return "workspace allocation failed";
     case GDN_ERR_CUDA: return "CUDA error";
     case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+    case GDN_ERR_SCRATCH_LIMIT:
+      return "problem needs more than the 64 MiB fixed scratch of gdn_frame_forward_noalloc";
   }
   return "unknown status";
 }

@@ -59,7 +59,8 @@ typedef enum gdn_status {
   GDN_ERR_MISALIGNED = 3,  /* a tensor pointer is not 16-byte aligned */
   GDN_ERR_NO_MEMORY = 4,   /* workspace allocation failed (or growth during capture) */
   GDN_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
-  GDN_ERR_TIMEOUT = 6      /* a device-side bounded wait ran out (from gdn_sync_status) */
+  GDN_ERR_TIMEOUT = 6,     /* a device-side bounded wait ran out (from gdn_sync_status) */
+  GDN_ERR_SCRATCH_LIMIT = 7 /* gdn_frame_forward_noalloc: problem too large for its scratch */
 } gdn_status;
 
 /*
@@ -72,6 +73,35 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
                              const float* gamma, const float* beta, const float* state_in,
                              gdn_bf16* out, float* state_out, int B, int H, int T, int N, int D,
                              float key_scale, gdn_stream_t stream);
+
+/*
+ * gdn_frame_forward_noalloc - gdn_frame_forward for callers that must not allocate device memory.
+ * (No counterpart in the paper: this is a deployment variant of the same computation.)
+ *
+ * Some callers cannot let a library call cudaMalloc: code inside an inference server or host
+ * framework that owns all device memory through its own pool (an allocation behind its back
+ * breaks its accounting and can fail or fragment), real-time loops where the device-wide
+ * synchronisation that growing gdn_frame_forward's workspace implies would stall other streams,
+ * and plugins whose memory budget is fixed when they are loaded. This entry point allocates
+ * nothing: its scratch is a fixed 64 MiB array in device memory that the library reserves on
+ * every GPU that loads it, held until the process exits.
+ *
+ * Arguments, layouts and results are exactly those of gdn_frame_forward; the caller still
+ * provides q, k, v, gamma, beta, state_in, out and state_out. Limits and behaviour:
+ *  - The problem must fit the scratch: gdn_workspace_bytes(B, H, T, N, D) <= 64 MiB (for D = 128
+ *    that is B*H*T <= 512 frame-heads). Larger problems return GDN_ERR_SCRATCH_LIMIT before
+ *    anything is launched.
+ *  - The first call on each GPU looks up the scratch's device address (with that GPU current) and
+ *    caches it; make that first call before any stream capture.
+ *  - All calls on a GPU share the one scratch array, which keeps the last call's contents (no call
+ *    needs it cleared: every element is written before it is read). Calls whose executions
+ *    overlap on the GPU (different streams, or different host threads) race on it.
+ */
+gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                     const float* gamma, const float* beta,
+                                     const float* state_in, gdn_bf16* out, float* state_out,
+                                     int B, int H, int T, int N, int D, float key_scale,
+                                     gdn_stream_t stream);
 
 /*
  * gdn_frame_step - one streaming step: one new frame per stream, carried state.
