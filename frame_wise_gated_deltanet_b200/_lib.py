@@ -39,6 +39,7 @@ SIGNATURES = {
     "gdn_release_workspace": (None, []),
     "gdn_version": (_I, []),
     "gdn_profile_arm": (_I, [_P, _I]),
+    "gdn_set_forward_mode": (_I, [_I]),
     "gdn_profile_count": (_I, []),
     "gdn_profile_kernel": (ctypes.c_char_p, [_I]),
 }

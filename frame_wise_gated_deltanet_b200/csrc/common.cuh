@@ -22,6 +22,33 @@ struct Problem {
   float key_scale;
 };
 
+// Hand-off state of the fused forward, in device memory and zeroed before each call. One
+// persistent grid runs three roles: stats CTAs write A_t, B_t into per-head rings of R slots,
+// chain CTAs consume them and write S_t into a ring of R slots, output CTAs consume S_t.
+struct Handoff {
+  int* stats_flag;  // [B*H*T] 1 once A_t, B_t of (bh, t) are in ring slot t % R
+  int* out_flag;    // [B*H*T] 1 once the output of (bh, t) has loaded S_t (its slot is free)
+  int* chain_prog;  // [B*H]   number of frames whose S_t the chain has stored
+  int* abort;       // set by the first CTA that gives up a wait; every wait then returns
+  int R;            // ring slots per head
+  int base;         // first blockIdx.x of this role
+  int count;        // CTAs in this role
+};
+
+__device__ __forceinline__ void give_up(const Handoff& hf, volatile int* local_abort) {
+  record_error(kErrTimeout);
+  if (hf.abort != nullptr) atomicExch(hf.abort, 1);
+  *local_abort = 1;
+}
+
+// B_t storage used between the statistics and the chain: element (v, k) of the D x D matrix at
+// float index ((k / 4) * D + v) * 4 + k % 4, i.e. 16-byte groups of four keys, consecutive value
+// rows adjacent. A warp handling 32 consecutive rows then reads or writes 512 contiguous bytes per
+// group, for both the writer (one thread per row) and the reader (one thread per row).
+__host__ __device__ __forceinline__ long b4_index(int v, int k, int D) {
+  return (static_cast<long>(k >> 2) * D + v) * 4 + (k & 3);
+}
+
 // TMA box: 64 bf16 (128 B, one swizzle row) x 128 rows.
 constexpr int kRowsPerTile = 128;
 constexpr int kBoxBytes = 128 * 128;  // 16 KB

@@ -1,0 +1,58 @@
+// Fused forward: one persistent, co-resident grid (cooperative launch, one CTA per SM) runs
+// the three stages concurrently so that the serial state chain overlaps the two HBM streams.
+//
+//   blocks [0, B*H)              chain role, one per (batch, head)
+//   blocks [B*H, B*H + n_stats)  stats role: A_t, B_t of frame-major items into ring slots
+//   blocks [.., gridDim.x)       output role: O_t from ring slots of S_t
+//
+// A_t (bf16), B_t (f32) and S_t (bf16) travel through per-head rings of R slots (a few tens of
+// MB, L2-resident: loaded and stored with evict_last while the q/k/v/out streams use
+// evict_first). Hand-off is by release/acquire flags in global memory with bounded waits;
+// every role processes its items in increasing frame order and every wait points at a
+// strictly earlier frame (or at the chain, which only waits on earlier frames), so with all
+// CTAs co-resident the grid cannot deadlock.
+#pragma once
+#include <cuda.h>
+
+#include "chain_kernel.cuh"
+#include "common.cuh"
+#include "output_kernel.cuh"
+#include "stats_kernel.cuh"
+
+namespace gdn {
+
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+template <int DP>
+struct FusedLayout {
+  static constexpr int kThreads = ChainLayout<DP>::kThreads;
+  static constexpr int kSmemBytes =
+      cmax(ChainLayout<DP>::kSmemBytes,
+           cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes));
+};
+
+template <int DP>
+__global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
+    gdn_fused_kernel(const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_o,
+                     const __grid_constant__ CUtensorMap tm_a_ring,
+                     const __grid_constant__ CUtensorMap tm_s_ring,
+                     __nv_bfloat16* __restrict__ A_ring, float* __restrict__ B_ring,
+                     const float* __restrict__ gamma, const float* __restrict__ beta,
+                     const float* __restrict__ state_in, float* __restrict__ state_out, Problem p,
+                     Handoff h_chain, Handoff h_stats, Handoff h_out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1k(smem_raw);
+  if (static_cast<int>(blockIdx.x) < h_stats.base) {
+    chain_body<DP, true>(&tm_a_ring, B_ring, &tm_s_ring, gamma, beta, state_in, state_out, p,
+                         h_chain, smem);
+  } else if (static_cast<int>(blockIdx.x) < h_out.base) {
+    stats_body<DP, false, true, true>(&tm_k, &tm_v, A_ring, B_ring, p, h_stats, smem);
+  } else {
+    output_body<DP, false, true>(&tm_q, &tm_s_ring, &tm_o, p, 1, h_out, smem);
+  }
+}
+
+}  // namespace gdn

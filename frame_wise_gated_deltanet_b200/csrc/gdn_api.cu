@@ -11,6 +11,7 @@
 #include "../../include/gdn.h"
 #include "chain_kernel.cuh"
 #include "common.cuh"
+#include "fused_kernel.cuh"
 #include "la_scan_kernel.cuh"
 #include "output_kernel.cuh"
 #include "stats_kernel.cuh"
@@ -187,14 +188,17 @@ gdn_status check_launch() {
 }
 
 // ------------------------------------------------------------------ kernel runners
-template <int DP>
+// kB4: B_t in the chain's interleaved layout (forward paths) or row-major (gdn_frame_stats).
+template <int DP, bool kB4>
 gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, void* A, float* Bm,
                      cudaStream_t st) {
   using L = gdn::StatsLayout<DP, false>;
   CUtensorMap tk, tv;
   if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_stats_kernel<DP, false>;
-  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 0 : 1, kern, L::kSmemBytes)) return s;
+  auto kern = gdn::gdn_stats_kernel<DP, false, kB4>;
+  if (gdn_status s = ensure_smem_attr(dev, (DP == 128 ? 0 : 1) + (kB4 ? 10 : 0), kern,
+                                      L::kSmemBytes))
+    return s;
   const long items = long(p.B) * p.T * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
   {
@@ -210,16 +214,15 @@ gdn_status run_chain(int dev, const Problem& p, const void* A, const float* Bm,
                      float* s_out, cudaStream_t st) {
   using L = gdn::ChainLayout<DP>;
   const long count = long(p.B) * p.H * p.T;
-  CUtensorMap ta, tb, ts;
+  CUtensorMap ta, ts;
   if (!tmap_mats(&ta, A, false, p.D, p.D, count, DP) ||
-      !tmap_mats(&tb, Bm, true, p.D, p.D, count, DP) ||
       !tmap_mats(&ts, S_ws, false, p.D, p.D, count, DP))
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_chain_kernel<DP>;
   if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 2 : 3, kern, L::kSmemBytes)) return s;
   {
     ProfiledLaunch pl("gdn_chain_kernel", st);
-    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, tb, ts, gamma, beta, s_in, s_out, p);
+    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, Bm, ts, gamma, beta, s_in, s_out, p);
   }
   return check_launch();
 }
@@ -268,23 +271,122 @@ ForwardWs carve_forward(void* base, long count, int D) {
   return w;
 }
 
+// ------------------------------------------------------------------ fused forward
+// 0 = choose automatically, 1 = always the three-kernel path, 2 = fused whenever it applies.
+int g_forward_mode = 0;
+constexpr int kRing = 16;  // ring slots per head of the fused forward
+
+struct FusedWs {
+  void* A;
+  float* B;
+  void* S;
+  int* flags;  // stats_flag [BH*T], out_flag [BH*T], chain_prog [BH], abort [1]
+  size_t flag_bytes;
+};
+
+size_t fused_ws_bytes(long bh, long T, int D) {
+  const size_t m = size_t(D) * D * bh * kRing;
+  const size_t flags = sizeof(int) * (2 * bh * T + bh + 1);
+  return align256(m * 2) + align256(m * 4) + align256(m * 2) + align256(flags);
+}
+
+FusedWs carve_fused(void* base, long bh, long T, int D) {
+  const size_t m = size_t(D) * D * bh * kRing;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  FusedWs w;
+  w.A = p;
+  p += align256(m * 2);
+  w.B = reinterpret_cast<float*>(p);
+  p += align256(m * 4);
+  w.S = p;
+  p += align256(m * 2);
+  w.flags = reinterpret_cast<int*>(p);
+  w.flag_bytes = sizeof(int) * (2 * bh * T + bh + 1);
+  return w;
+}
+
+// Whether the fused forward can run this problem on this GPU: every (batch, head) needs its own
+// chain CTA and enough SMs must remain for the two streaming roles.
+bool fused_applies(int dev, const Problem& p) {
+  if (g_forward_mode == 1) return false;
+  const int sms = g_dev[dev].sms;
+  const long bh = long(p.B) * p.H;
+  int coop = 0;
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+  if (!coop || sms - bh < 8) return false;
+  if (g_forward_mode == 2) return true;
+  return bh * 3 <= sms && p.T >= 4;
+}
+
+template <int DP>
+gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, const void* v,
+                     const float* gamma, const float* beta, const float* s_in, void* out,
+                     float* s_out, cudaStream_t st) {
+  using L = gdn::FusedLayout<DP>;
+  const int sms = g_dev[dev].sms;
+  const int bh = p.B * p.H;
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, fused_ws_bytes(bh, p.T, p.D), st, &base)) return s;
+  FusedWs w = carve_fused(base, bh, p.T, p.D);
+  if (cudaMemsetAsync(w.flags, 0, w.flag_bytes, st) != cudaSuccess) return GDN_ERR_CUDA;
+  CUtensorMap tk, tv, tq, to, ta, ts;
+  if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p) || !tmap_tokens(&tq, q, p) ||
+      !tmap_tokens(&to, out, p) || !tmap_mats(&ta, w.A, false, p.D, p.D, long(bh) * kRing, DP) ||
+      !tmap_mats(&ts, w.S, false, p.D, p.D, long(bh) * kRing, DP))
+    return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_fused_kernel<DP>;
+  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 8 : 9, kern, L::kSmemBytes)) return s;
+  // split the SMs left after the chains between the stats and output roles (~54 : 46, the
+  // ratio of their per-frame times)
+  const int workers = sms - bh;
+  int n_stats = (workers * 54 + 50) / 100;
+  if (n_stats < 1) n_stats = 1;
+  if (n_stats > workers - 1) n_stats = workers - 1;
+  int* f = w.flags;
+  const long ft = long(bh) * p.T;
+  gdn::Handoff hc{f, f + ft, f + 2 * ft, f + 2 * ft + bh, kRing, 0, bh};
+  gdn::Handoff hs = hc;
+  hs.base = bh;
+  hs.count = n_stats;
+  gdn::Handoff ho = hc;
+  ho.base = bh + n_stats;
+  ho.count = workers - n_stats;
+  __nv_bfloat16* a_ring = static_cast<__nv_bfloat16*>(w.A);
+  float* b_ring = w.B;
+  gdn::Problem pp = p;
+  void* args[] = {&tk, &tv, &tq, &to, &ta, &ts, &a_ring, &b_ring,
+                  const_cast<float**>(&gamma), const_cast<float**>(&beta),
+                  const_cast<float**>(&s_in), &s_out, &pp, &hc, &hs, &ho};
+  {
+    ProfiledLaunch pl("gdn_fused_kernel", st);
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(sms),
+                                    dim3(L::kThreads), args, L::kSmemBytes, st) != cudaSuccess)
+      return GDN_ERR_CUDA;
+  }
+  return check_launch();
+}
+
 gdn_status forward_impl(const void* q, const void* k, const void* v, const float* gamma,
                         const float* beta, const float* s_in, void* out, float* s_out,
                         const Problem& p, cudaStream_t st) {
   int dev;
   if (gdn_status s = current_device(&dev)) return s;
   std::lock_guard<std::mutex> lock(g_mu);
+  if (fused_applies(dev, p)) {
+    if (p.D <= 64) return run_fused<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+    return run_fused<128>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+  }
   const long count = long(p.B) * p.H * p.T;
   void* base = nullptr;
   if (gdn_status s = get_workspace(dev, forward_ws_bytes(count, p.D), st, &base)) return s;
   ForwardWs w = carve_forward(base, count, p.D);
   if (p.D <= 64) {
-    if (gdn_status s = run_stats<64>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
     if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, st))
       return s;
     return run_output<64, false>(dev, p, q, w.S, p.D, out, 1, st);
   }
-  if (gdn_status s = run_stats<128>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
   if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, st))
     return s;
   return run_output<128, false>(dev, p, q, w.S, p.D, out, 1, st);
@@ -360,12 +462,12 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
   const Problem p{B, H, T, N, D, key_scale};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (D <= 64) {
-    if (gdn_status s = run_stats<64>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
     if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out, st))
       return s;
     return run_output<64, false>(dev, p, q, w.S, D, out, 1, st);
   }
-  if (gdn_status s = run_stats<128>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
   if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out, st))
     return s;
   return run_output<128, false>(dev, p, q, w.S, D, out, 1, st);
@@ -396,8 +498,8 @@ gdn_status gdn_frame_stats(const gdn_bf16* k, const gdn_bf16* v, gdn_bf16* A_out
   std::lock_guard<std::mutex> lock(g_mu);
   const Problem p{B, H, T, N, D, key_scale};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (D <= 64) return run_stats<64>(dev, p, k, v, A_out, B_out, st);
-  return run_stats<128>(dev, p, k, v, A_out, B_out, st);
+  if (D <= 64) return run_stats<64, false>(dev, p, k, v, A_out, B_out, st);
+  return run_stats<128, false>(dev, p, k, v, A_out, B_out, st);
 }
 
 gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
@@ -428,7 +530,7 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
     using L = gdn::StatsLayout<128, true>;
     CUtensorMap tk, tv;
     if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
-    auto kern = gdn::gdn_stats_kernel<128, true>;
+    auto kern = gdn::gdn_stats_kernel<128, true, false>;
     if (gdn_status s = ensure_smem_attr(dev, 7, kern, L::kSmemBytes)) return s;
     const int grid = static_cast<int>(count < g_dev[dev].sms ? count : g_dev[dev].sms);
     ProfiledLaunch pl("gdn_stats_kernel_la", st);
@@ -449,7 +551,9 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {
   (void)N;
   if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
-  return forward_ws_bytes(long(B) * H * T, D);
+  const size_t split = forward_ws_bytes(long(B) * H * T, D);
+  const size_t fused = fused_ws_bytes(long(B) * H, T, D);
+  return split > fused ? split : fused;
 }
 
 size_t gdn_la_workspace_bytes(int B, int H, int T, int D) {
@@ -513,6 +617,13 @@ gdn_status gdn_profile_arm(void* const* events, int n) {
 }
 
 int gdn_profile_count(void) { return g_prof_count; }
+
+gdn_status gdn_set_forward_mode(int mode) {
+  if (mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_forward_mode = mode;
+  return GDN_OK;
+}
 
 const char* gdn_profile_kernel(int i) {
   if (i < 0 || i >= g_prof_count) return "";

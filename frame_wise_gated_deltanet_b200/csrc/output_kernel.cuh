@@ -15,6 +15,11 @@
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2..5 epilogue,
 // warps 6..9 (LA only) transform.
+//
+// Standalone (gdn_output_kernel): work item i = (b*T + t)*H + h, S_t at workspace row
+// (b*H+h)*T + t_state. Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h
+// (frame-major), S_t loaded from ring row (b*H+h)*R + t%R once chain_prog says it is there;
+// out_flag releases the slot as soon as S_t is in shared memory.
 #pragma once
 #include <cuda.h>
 
@@ -34,17 +39,38 @@ struct OutputLayout {
   static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + 512 + 1024;
 };
 
-// state_rows: rows of one stored state (D for GDN, D+1 for LA).
+struct OutputItem {
+  int h, bt, bh, t;
+};
+
+template <bool kFused>
+__device__ __forceinline__ OutputItem output_item(long item, const Problem& p) {
+  OutputItem it;
+  if constexpr (kFused) {
+    const int BH = p.B * p.H;
+    it.t = static_cast<int>(item / BH);
+    it.bh = static_cast<int>(item - static_cast<long>(it.t) * BH);
+    const int b = it.bh / p.H;
+    it.h = it.bh - b * p.H;
+    it.bt = b * p.T + it.t;
+  } else {
+    it.h = static_cast<int>(item % p.H);
+    it.bt = static_cast<int>(item / p.H);
+    const int b = it.bt / p.T;
+    it.t = it.bt - b * p.T;
+    it.bh = b * p.H + it.h;
+  }
+  return it;
+}
+
 // frames_per_block: 1 for GDN (frame t reads S_t); F for LA (frame t reads the state at the end
 // of its block of F frames).
-template <int DP, bool kLA>
-__global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
-    gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_s,
-                      const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
+template <int DP, bool kLA, bool kFused>
+__device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
+                                            const CUtensorMap* tm_o, const Problem& p,
+                                            int frames_per_block, const Handoff& hf,
+                                            uint8_t* smem) {
   using L = OutputLayout<DP, kLA>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1k(smem_raw);
   uint8_t* s_buf = smem;                          // 2 state buffers
   uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
   uint8_t* o_stage = q_ring + L::kStages * L::kQBytes;  // 2 output staging tiles
@@ -63,6 +89,8 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
   const long n_items = static_cast<long>(p.B) * p.T * p.H;
   const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
   const int F = frames_per_block;
+  const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
+  const long ncta = kFused ? hf.count : gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -90,42 +118,49 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
 
   if (warp == 0) {
     if (elect_one()) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_s);
+      tma_prefetch_desc(tm_q);
+      tma_prefetch_desc(tm_s);
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_state = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int li = 0;
-      for (long item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x, ++li) {
-        const int h = static_cast<int>(item % p.H);
-        const int bt = static_cast<int>(item / p.H);
-        const int b = bt / p.T;
-        const int t = bt - b * p.T;
-        const int t_state = (F <= 1) ? t : min((t / F + 1) * F, p.T) - 1;
-        const int srow = (b * p.H + h) * p.T + t_state;
+      for (long item = cta0; item < n_items && !*abort_flag; item += ncta, ++li) {
+        const OutputItem it = output_item<kFused>(item, p);
+        int srow;
+        if constexpr (kFused) {
+          srow = it.bh * hf.R + it.t % hf.R;
+        } else {
+          const int t_state = (F <= 1) ? it.t : min((it.t / F + 1) * F, p.T) - 1;
+          srow = it.bh * p.T + t_state;
+        }
         const int sb = li & 1;
         if (!mbar_wait(&s_empty[sb], ((li >> 1) & 1) ^ 1)) {
-          record_error(kErrTimeout);
-          *abort_flag = 1;
+          give_up(hf, abort_flag);
           break;
+        }
+        if constexpr (kFused) {
+          if (!wait_flag_ge(hf.chain_prog + it.bh, it.t + 1, hf.abort)) {
+            give_up(hf, abort_flag);
+            break;
+          }
+          fence_async_global();
         }
         mbar_arrive_expect_tx(&s_full[sb], L::kSBufBytes);
 #pragma unroll
         for (int kb = 0; kb < L::kBoxes; ++kb)
-          tma_load_3d(s_buf + sb * L::kSBufBytes + kb * DP * 128, &tm_s, &s_full[sb], kb * 64, 0,
+          tma_load_3d(s_buf + sb * L::kSBufBytes + kb * DP * 128, tm_s, &s_full[sb], kb * 64, 0,
                       srow, pol_state);
         for (int tile = 0; tile < n_tiles; ++tile) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            record_error(kErrTimeout);
-            *abort_flag = 1;
+            give_up(hf, abort_flag);
             break;
           }
           mbar_arrive_expect_tx(&full[stage], L::kQBytes);
 #pragma unroll
           for (int kb = 0; kb < L::kBoxes; ++kb)
-            tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, &tm_q, &full[stage],
-                        kb * 64, h, tile * kRowsPerTile, bt, pol_stream);
+            tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
+                        kb * 64, it.h, tile * kRowsPerTile, it.bt, pol_stream);
           if (++stage == L::kStages) {
             stage = 0;
             phase ^= 1;
@@ -140,11 +175,16 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
     int li = 0;
     int tc = 0;  // tiles processed (accumulator ring position)
     bool ok = true;
-    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
+    for (long item = cta0; item < n_items && ok; item += ncta, ++li) {
       const int sb = li & 1;
       if (!mbar_wait(&s_full[sb], (li >> 1) & 1)) {
         ok = false;
         break;
+      }
+      if constexpr (kFused) {
+        // S_t is in shared memory: its ring slot may be overwritten by the chain
+        const OutputItem it = output_item<kFused>(item, p);
+        if (lane == 0) st_release(hf.out_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
       }
       const uint32_t s_base = smem_u32(s_buf + sb * L::kSBufBytes);
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
@@ -179,10 +219,7 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
       if (elect_one()) mma_commit(&s_empty[sb]);
       __syncwarp();
     }
-    if (!ok) {
-      record_error(kErrTimeout);
-      *abort_flag = 1;
-    }
+    if (!ok) give_up(hf, abort_flag);
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue
     const uint32_t quarter = warp & 3;
@@ -191,12 +228,11 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
     const int D = p.D;
     const bool leader = (threadIdx.x == 64);
     const uint64_t pol_out = policy_evict_first();
-    if (leader) tma_prefetch_desc(&tm_o);
+    if (leader) tma_prefetch_desc(tm_o);
     int tc = 0;
     bool ok = true;
-    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int h = static_cast<int>(item % p.H);
-      const long bt = item / p.H;
+    for (long item = cta0; item < n_items && ok; item += ncta) {
+      const OutputItem it = output_item<kFused>(item, p);
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
         const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
@@ -240,24 +276,21 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
         if (leader) {
 #pragma unroll
           for (int kb = 0; kb < L::kBoxes; ++kb)
-            tma_store_4d(&tm_o, ob + kb * kBoxBytes, kb * 64, h, tile * kRowsPerTile,
-                         static_cast<int>(bt), pol_out);
+            tma_store_4d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h, tile * kRowsPerTile, it.bt,
+                         pol_out);
           bulk_commit();
         }
       }
     }
     if (leader) bulk_wait_all();
-    if (!ok) {
-      record_error(kErrTimeout);
-      *abort_flag = 1;
-    }
+    if (!ok) give_up(hf, abort_flag);
   } else if constexpr (kLA) {
     // ---------------------------------------------------------------- relu(Q) transform
     const int tid = threadIdx.x - 192;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    for (long item = cta0; item < n_items && ok; item += ncta) {
       for (int tile = 0; tile < n_tiles; ++tile) {
         if (!mbar_wait(&full[stage], phase)) {
           ok = false;
@@ -280,10 +313,7 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
         }
       }
     }
-    if (!ok) {
-      record_error(kErrTimeout);
-      *abort_flag = 1;
-    }
+    if (!ok) give_up(hf, abort_flag);
   }
 
   tc_fence_before();
@@ -292,6 +322,17 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
   }
+}
+
+template <int DP, bool kLA>
+__global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
+    gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_s,
+                      const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
+  extern __shared__ uint8_t smem_raw[];
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 0, 0};
+  output_body<DP, kLA, false>(&tm_q, &tm_s, &tm_o, p, frames_per_block, none,
+                              align1k(smem_raw));
 }
 
 }  // namespace gdn

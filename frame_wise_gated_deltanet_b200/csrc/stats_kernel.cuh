@@ -13,6 +13,11 @@
 //   warp 1      TMEM allocator + MMA issuer (one elected thread)
 //   warps 2..5  epilogue: TMEM -> registers -> scale -> global
 //   warps 6..9  (LA only) in-place transform of each K/V stage: relu(K), ones column in V
+//
+// Standalone (gdn_stats_kernel): work item i = (b*T + t)*H + h, results at workspace row
+// (b*H + h)*T + t. Fused (stats role of gdn_fused_kernel): work item i = t*B*H + (b*H + h)
+// (frame-major, so the chain finds early frames first), results at ring row (b*H+h)*R + t%R,
+// written only after the chain has released that slot, then published with stats_flag.
 #pragma once
 #include <cuda.h>
 
@@ -34,16 +39,41 @@ struct StatsLayout {
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
 };
 
-// A_ws: [B*H*T, D, D] bf16 (GDN only). B_ws: [B*H*T, brows, D] f32, brows = D (GDN) or D+1 (LA).
-// Work item i = (b*T + t)*H + h; its workspace row is (b*H + h)*T + t.
-template <int DP, bool kLA>
-__global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
-    gdn_stats_kernel(const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
-                     float* __restrict__ B_ws, Problem p) {
+struct StatsItem {
+  int h, bt, bh, t;
+  long row;  // workspace / ring row of the results
+};
+
+template <bool kFused>
+__device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, const Handoff& hf) {
+  StatsItem it;
+  if constexpr (kFused) {
+    const int BH = p.B * p.H;
+    it.t = static_cast<int>(item / BH);
+    it.bh = static_cast<int>(item - static_cast<long>(it.t) * BH);
+    const int b = it.bh / p.H;
+    it.h = it.bh - b * p.H;
+    it.bt = b * p.T + it.t;
+    it.row = static_cast<long>(it.bh) * hf.R + it.t % hf.R;
+  } else {
+    it.h = static_cast<int>(item % p.H);
+    it.bt = static_cast<int>(item / p.H);
+    const int b = it.bt / p.T;
+    it.t = it.bt - b * p.T;
+    it.bh = b * p.H + it.h;
+    it.row = static_cast<long>(it.bh) * p.T + it.t;
+  }
+  return it;
+}
+
+// kB4: B_t stored in the four-key interleaved layout of b4_index (the chain's input) instead of
+// row-major (the public gdn_frame_stats layout and the block-causal path).
+template <int DP, bool kLA, bool kFused, bool kB4>
+__device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                           __nv_bfloat16* __restrict__ A_ws,
+                                           float* __restrict__ B_ws, const Problem& p,
+                                           const Handoff& hf, uint8_t* smem) {
   using L = StatsLayout<DP, kLA>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1k(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
   uint64_t* ready = full + L::kStages;   // LA: transformed stage
   uint64_t* empty = ready + L::kStages;
@@ -56,6 +86,8 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
   const uint32_t lane = lane_id();
   const long n_items = static_cast<long>(p.B) * p.T * p.H;
   const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
+  const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
+  const long ncta = kFused ? hf.count : gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -82,28 +114,26 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (elect_one()) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(tm_k);
+      tma_prefetch_desc(tm_v);
       const uint64_t pol = policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
-      for (long item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
-        const int h = static_cast<int>(item % p.H);
-        const int bt = static_cast<int>(item / p.H);
+      for (long item = cta0; item < n_items && !*abort_flag; item += ncta) {
+        const StatsItem it = stats_item<kFused>(item, p, hf);
         for (int tile = 0; tile < n_tiles; ++tile) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            record_error(kErrTimeout);
-            *abort_flag = 1;
+            give_up(hf, abort_flag);
             break;
           }
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
           uint8_t* st = smem + stage * L::kStageBytes;
 #pragma unroll
           for (int j = 0; j < L::kBoxes; ++j) {
-            tma_load_4d(st + j * kBoxBytes, &tm_k, &full[stage], j * 64, h, tile * kRowsPerTile,
-                        bt, pol);
-            tma_load_4d(st + L::kOpBytes + j * kBoxBytes, &tm_v, &full[stage], j * 64, h,
-                        tile * kRowsPerTile, bt, pol);
+            tma_load_4d(st + j * kBoxBytes, tm_k, &full[stage], j * 64, it.h,
+                        tile * kRowsPerTile, it.bt, pol);
+            tma_load_4d(st + L::kOpBytes + j * kBoxBytes, tm_v, &full[stage], j * 64, it.h,
+                        tile * kRowsPerTile, it.bt, pol);
           }
           if (++stage == L::kStages) {
             stage = 0;
@@ -120,12 +150,11 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     int li = 0;
-    for (long item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
+    for (long item = cta0; item < n_items; item += ncta, ++li) {
       const int acc = li & 1;
       const uint32_t aph = (li >> 1) & 1;
       if (!mbar_wait(&acc_empty[acc], aph ^ 1)) {
-        record_error(kErrTimeout);
-        *abort_flag = 1;
+        give_up(hf, abort_flag);
         break;
       }
       tc_fence_after();
@@ -169,8 +198,7 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
         }
       }
       if (!ok) {
-        record_error(kErrTimeout);
-        *abort_flag = 1;
+        give_up(hf, abort_flag);
         break;
       }
       if (elect_one()) mma_commit(&acc_full[acc]);
@@ -181,24 +209,28 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
+    const bool leader = (threadIdx.x == 64);
     const float s = p.key_scale;
     const int D = p.D;
     const int brows = kLA ? D + 1 : D;
     int li = 0;
-    for (long item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
+    for (long item = cta0; item < n_items; item += ncta, ++li) {
       const int acc = li & 1;
       const uint32_t aph = (li >> 1) & 1;
-      if (!mbar_wait(&acc_full[acc], aph)) {
-        record_error(kErrTimeout);
-        *abort_flag = 1;
+      const StatsItem it = stats_item<kFused>(item, p, hf);
+      bool bad = !mbar_wait(&acc_full[acc], aph);
+      if constexpr (kFused) {
+        // ring slot t % R of this head is free once the chain has stored S_{t-R}
+        if (leader && !bad && it.t >= hf.R)
+          bad = !wait_flag_ge(hf.chain_prog + it.bh, it.t - hf.R + 1, hf.abort);
+        bad = named_bar_any(1, 128, bad);
+      }
+      if (bad) {
+        give_up(hf, abort_flag);
         break;
       }
       tc_fence_after();
-      const int h = static_cast<int>(item % p.H);
-      const long bt = item / p.H;
-      const long b = bt / p.T;
-      const long t = bt - b * p.T;
-      const long ws = (b * p.H + h) * p.T + t;
+      const long ws = it.row;
       const uint32_t tacc = lane_base + acc * L::kAccCols;
       float v[32];
       if constexpr (kLA) {
@@ -246,13 +278,15 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
                   }
                 }
               } else {
-                float* brow = B_ws + (ws * D + mrow) * D;
+                float* bmat = B_ws + ws * D * D;
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
                   const int col = c * 32 + j;
-                  if (col < D)
-                    *reinterpret_cast<float4*>(brow + col) =
+                  if (col < D) {
+                    const long off = kB4 ? b4_index(mrow, col, D) : static_cast<long>(mrow) * D + col;
+                    *reinterpret_cast<float4*>(bmat + off) =
                         make_float4(v[j] * s, v[j + 1] * s, v[j + 2] * s, v[j + 3] * s);
+                  }
                 }
               }
             }
@@ -261,6 +295,13 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
+      if constexpr (kFused) {
+        // publish: every epilogue thread's stores, then the flag (the chain reads by TMA)
+        fence_async_global();
+        __threadfence();
+        named_bar(1, 128);
+        if (leader) st_release(hf.stats_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
+      }
     }
   } else if constexpr (kLA) {
     // ---------------------------------------------------------------- LA transform warps
@@ -268,7 +309,7 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     const int D = p.D;
-    for (long item = blockIdx.x; item < n_items; item += gridDim.x) {
+    for (long item = cta0; item < n_items; item += ncta) {
       bool ok = true;
       for (int tile = 0; tile < n_tiles; ++tile) {
         if (!mbar_wait(&full[stage], phase)) {
@@ -298,8 +339,7 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
         }
       }
       if (!ok) {
-        record_error(kErrTimeout);
-        *abort_flag = 1;
+        give_up(hf, abort_flag);
         break;
       }
     }
@@ -311,6 +351,18 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
   }
+}
+
+// A_ws: [B*H*T, D, D] bf16 (GDN only). B_ws: [B*H*T, brows, D] f32, brows = D (GDN) or D+1 (LA),
+// row-major, or (kB4, GDN) each D x D matrix in the b4_index layout.
+template <int DP, bool kLA, bool kB4>
+__global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
+    gdn_stats_kernel(const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
+                     float* __restrict__ B_ws, Problem p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 0, 0};
+  stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw));
 }
 
 }  // namespace gdn

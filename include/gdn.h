@@ -67,7 +67,8 @@ typedef enum gdn_status {
  * gdn_frame_forward - frame-wise GDN over a whole clip of T frames.
  * Computes out (all T frames) and, if state_out != NULL, S_T.
  * key_scale: the scale applied to keys (1/sqrt(D*N) for the pages' setting); finite, > 0.
- * Workspace: gdn_workspace_bytes(B, H, T, N, D) bytes (per-frame A_t, B_t and S_t).
+ * Workspace: gdn_workspace_bytes(B, H, T, N, D) bytes (three-kernel path: per-frame A_t, B_t,
+ * S_t; fused path: per-head rings of A_t, B_t, S_t and hand-off flags).
  */
 gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
                              const float* gamma, const float* beta, const float* state_in,
@@ -174,6 +175,16 @@ void gdn_release_workspace(void);
 gdn_status gdn_profile_arm(void* const* events, int n);
 int gdn_profile_count(void);
 const char* gdn_profile_kernel(int i);
+
+/*
+ * gdn_set_forward_mode - how gdn_frame_forward / gdn_frame_step run (process-wide):
+ *   0 (default) automatic: the fused persistent kernel when B*H is at most a third of the SMs
+ *     and T >= 4, otherwise three kernels (statistics, state chain, output);
+ *   1 always the three kernels;
+ *   2 the fused kernel whenever it can run (B*H <= SMs - 8 and cooperative launch available).
+ * Both compute the same result. Returns GDN_ERR_INVALID_ARG for other values.
+ */
+gdn_status gdn_set_forward_mode(int mode);
 
 /* Library ABI version (major * 100 + minor). */
 int gdn_version(void);

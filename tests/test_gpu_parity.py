@@ -52,8 +52,18 @@ SHAPES = [
 ]
 
 
+@pytest.fixture
+def forward_mode(request):
+    """Run a test with gdn_set_forward_mode(mode) (1 = three kernels, 2 = fused persistent)."""
+    from frame_wise_gated_deltanet_b200 import _lib
+    assert _lib.LIB.gdn_set_forward_mode(request.param) == 0
+    yield request.param
+    _lib.LIB.gdn_set_forward_mode(0)
+
+
+@pytest.mark.parametrize("forward_mode", [1, 2], indirect=True, ids=["split", "fused"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B%dH%dT%dN%dD%d%s" % (s[:5] + ("s" if s[5] else "",)))
-def test_forward_matches_oracle(shape):
+def test_forward_matches_oracle(shape, forward_mode):
     B, H, T, N, D, with_state = shape
     x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=100 + D + N, state_std=0.3 if with_state else 0.0)
     ks = 1.0 / math.sqrt(D * N)
@@ -161,6 +171,39 @@ def test_stream_workload_sampled():
         eo = math.sqrt(o_err_num[p] / o_err_den[p])
         es = relf(f64(state[p[0], p[1]]), ref_state[p])
         assert eo <= O_TOL and es <= S_TOL, f"stream {p}: O err {eo:.2e}, S err {es:.2e}"
+
+
+@pytest.mark.parametrize("forward_mode", [1, 2], indirect=True, ids=["split", "fused"])
+def test_480p_workload_both_paths(forward_mode):
+    w = gdn_inputs.WORKLOADS["480p"]
+    x = gdn_inputs.workload_inputs(w)
+    g = to_cuda(x)
+    out, st = api().gdn_frame_forward(g["q"], g["k"], g["v"], g["gamma"], g["beta"], None,
+                                      key_scale=w.key_scale)
+    assert api().gdn_sync_status() == 0
+    o_ref, s_ref = oracle.gdn_frame_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["gamma"]),
+                                            f64(x["beta"]), None, w.key_scale)
+    assert relf(f64(out), o_ref) <= O_TOL
+    assert relf(f64(st), s_ref) <= S_TOL
+
+
+def test_fused_and_split_paths_agree_on_720p():
+    """Both forward paths on the full 720p clip: same kernels' arithmetic, so they agree to the
+    rounding of the bf16 copies of S (identical in practice)."""
+    from frame_wise_gated_deltanet_b200 import _lib
+    w = gdn_inputs.WORKLOADS["720p"]
+    g = gdn_inputs.workload_inputs(w, device="cuda")
+    res = {}
+    try:
+        for mode in (1, 2):
+            assert _lib.LIB.gdn_set_forward_mode(mode) == 0
+            res[mode] = api().gdn_frame_forward(g["q"], g["k"], g["v"], g["gamma"], g["beta"],
+                                                None, key_scale=w.key_scale)
+            assert api().gdn_sync_status() == 0
+    finally:
+        _lib.LIB.gdn_set_forward_mode(0)
+    assert torch.equal(res[1][1], res[2][1])
+    assert torch.equal(res[1][0], res[2][0])
 
 
 def test_split_resume_on_gpu():
