@@ -5,23 +5,28 @@
 //   * The identity part of the frame map is kept implicit and exact: S lives in fp32 registers
 //     of 16 epilogue warps (thread = one row v of S, a quarter of its columns); only the small
 //     correction S_{t-1} A_t goes through the tensor core (S as a bf16 K-major operand written
-//     by the epilogue into shared memory, A_t as a bf16 K-major operand loaded by TMA through a
-//     4-stage ring, f32 accumulate in TMEM).
-//   * B_t never touches shared memory: it is stored in the four-key interleaved layout of
-//     b4_index, so each epilogue warp loads its 32 rows x 4 keys as 512 contiguous bytes, and
-//     each thread loads its slice one frame ahead, into registers.
-//   * A storer warp TMA-stores each S_t (the bf16 operand tile, which is exactly the bf16 copy
-//     of the state the output GEMM needs) and does all hand-off bookkeeping, so the MMA warp
-//     only waits for the tile and A_t and issues the MMAs.
+//     by the epilogue into shared memory, A_t as a bf16 K-major operand loaded by TMA, f32
+//     accumulate in TMEM).
+//   * B_t is stored in the four-key interleaved layout of b4_index, so each epilogue warp copies
+//     its 32 rows x 4 keys as 512 contiguous bytes; every thread copies its own slice with
+//     cp.async into one of two shared-memory buffers two frames ahead, and reads it back
+//     conflict-free in the same layout.
+//   * The bf16 operand tile of S is kept in the no-swizzle core-matrix layout of s8_offset_bytes,
+//     which is also the global layout of S_t for the output GEMM: right after handing the tile
+//     to the MMA, each thread writes its 16-byte pieces of S_t to global memory (a warp writes
+//     512 contiguous bytes per key group), so nothing waits on a store of the tile.
+//   * The producer warp checks each frame's hand-off conditions right before loading its A_t and
+//     opens that frame's gate (a ring of 8 mbarriers) for the epilogue's B_t copy, so every wait
+//     of the chain is on a frame it actually needs next.
 //
-// Warps: 0..15 epilogue (warp w: rows 32*(w%4).., columns (w/4)*DP/4..), 16 TMA producer,
-// 17 TMEM allocator + MMA issuer, 18 storer.
+// Warps: 0..15 epilogue (warp w: rows 32*(w%4).., columns (w/4)*DP/4..), 16 TMA producer and
+// gate, 17 TMEM allocator + MMA issuer, 18 publisher (fused only).
 //
 // Standalone (gdn_chain_kernel): A_t, B_t, S_t at workspace row (b*H+h)*T + t; A_t, B_t of
 // later frames are prefetched into L2. Fused (chain role of gdn_fused_kernel, CTA
-// base + b*H + h): rows (b*H+h)*R + t%R of the rings; frame t is read once stats_flag says it
-// is there, S_t is stored into its slot once the output of frame t-R has released it, and
-// chain_prog is advanced after each store has completed.
+// base + b*H + h): rows (b*H+h)*R + t%R of the A/B rings and (b*H+h)*Rs + t%Rs of the S ring;
+// frame t is gated on stats_flag (A_t, B_t written) and on out_flag of frame t-Rs (its S slot
+// free), and chain_prog is advanced once every thread's part of S_t is visible.
 #pragma once
 #include <cuda.h>
 
@@ -32,36 +37,42 @@ namespace gdn {
 template <int DP>
 struct ChainLayout {
   static constexpr int kABytes = DP * DP * 2;   // A_t bf16: DP/64 blocks of DP rows x 128 B
-  static constexpr int kStages = 4;
-  static constexpr int kSBlockBytes = 128 * 128;          // S operand: 128 rows x 64 cols bf16
-  static constexpr int kSBytes = (DP / 64) * kSBlockBytes;
+  static constexpr int kStages = 2;             // A_t stages
+  static constexpr int kBBufBytes = DP * 512;   // B_t f32: [DP/4 key groups][128 rows][16 B]
+  static constexpr int kBBufs = 2;
+  static constexpr int kGate = 8;               // gate ring
+  static constexpr int kSBytes = DP * 256;      // S operand: [DP/8 key groups][128 rows][16 B]
   static constexpr int kEpiWarps = 16;
   static constexpr int kThreads = (kEpiWarps + 3) * 32;
   static constexpr int kWarpProducer = kEpiWarps;
   static constexpr int kWarpMma = kEpiWarps + 1;
-  static constexpr int kWarpStorer = kEpiWarps + 2;
+  static constexpr int kWarpPublisher = kEpiWarps + 2;
   static constexpr int kCols = DP / 4;  // columns of S per epilogue thread
   static constexpr int kTmemCols = 128;
-  static constexpr int kSmemBytes = kStages * kABytes + kSBytes + 512 + 1024;
+  static constexpr int kSmemBytes = kStages * kABytes + kBBufs * kBBufBytes + kSBytes + 512 + 1024;
 };
 
+// S_out: bf16 states, one DP*DP block per row (workspace or ring), layout of s8_offset_bytes.
 template <int DP, bool kFused>
 __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float* __restrict__ B_ws,
-                                           const CUtensorMap* tm_s,
+                                           __nv_bfloat16* __restrict__ S_out,
                                            const float* __restrict__ gamma,
                                            const float* __restrict__ beta,
                                            const float* __restrict__ state_in,
                                            float* __restrict__ state_out, const Problem& p,
                                            const Handoff& hf, uint8_t* smem) {
   using L = ChainLayout<DP>;
-  uint8_t* s_tile = smem + L::kStages * L::kABytes;
+  uint8_t* b_buf = smem + L::kStages * L::kABytes;
+  uint8_t* s_tile = b_buf + L::kBBufs * L::kBBufBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_tile + L::kSBytes);
   uint64_t* empty = full + L::kStages;
-  uint64_t* b_ready = empty + L::kStages;  // B_t of the stage's frame may be read
-  uint64_t* mma_done = b_ready + L::kStages;
-  uint64_t* s_ready = mma_done + 1;        // the S tile holds the new state
-  uint64_t* s_stored = s_ready + 1;        // the TMA store of the S tile has read it
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_stored + 1);
+  uint64_t* gate = empty + L::kStages;   // frame f (slot f % kGate) may be read and written
+  uint64_t* mma_done = gate + L::kGate;
+  uint64_t* s_ready = mma_done + 1;      // the S tile holds the new state
+  // fused: epilogue warps that have written their part of S_t to global memory, summed over
+  // frames (kEpiWarps per frame); a counter, not a barrier, so the publisher may lag freely
+  uint32_t* s_written = reinterpret_cast<uint32_t*>(s_ready + 1);
+  uint32_t* tmem_slot = s_written + 1;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id();
@@ -71,18 +82,19 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
   const int h = bh - b * p.H;
   const int T = p.T;
   const int D = p.D;
-  // row of frame f's A_t / B_t / S_t
+  // row of frame f's A_t / B_t, and of its S_t
   auto row_of = [&](int f) { return kFused ? bh * hf.R + f % hf.R : bh * T + f; };
+  auto srow_of = [&](int f) { return kFused ? bh * hf.Rs + f % hf.Rs : bh * T + f; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&b_ready[s], 1);
     }
+    for (int s = 0; s < L::kGate; ++s) mbar_init(&gate[s], 1);
     mbar_init(mma_done, 1);
     mbar_init(s_ready, L::kEpiWarps * 32);
-    mbar_init(s_stored, 1);
+    *s_written = 0;
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -96,7 +108,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == L::kWarpProducer) {
-    // ---------------------------------------------------------------- A_t via TMA, B_t gate
+    // ---------------------------------------------------------------- gate, A_t via TMA
     if (elect_one()) {
       tma_prefetch_desc(tm_a);
       const uint64_t pol = kFused ? policy_evict_last() : policy_evict_first();
@@ -109,24 +121,28 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       };
       if constexpr (!kFused)
         for (int f = 0; f < kPrefetch && f < T; ++f) prefetch(f);
+      // Gate frame t, then load A_t. Fused: frame t's A_t, B_t must be published and the output
+      // of frame t-Rs must have loaded S_{t-Rs} from the slot S_t will use. Gate slot
+      // t % kGate was last used by frame t - kGate, whose B copy the epilogue issued at step
+      // t - kGate - 2, before the MMA of step t - 2 that the empty-stage wait below follows.
       for (int t = 0; t < T; ++t) {
         const int stage = t % L::kStages;
         const uint32_t phase = (t / L::kStages) & 1;
         if constexpr (!kFused) {
           if (t + kPrefetch < T) prefetch(t + kPrefetch);
         }
-        if (!mbar_wait(&empty[stage], phase ^ 1)) {
+        bool ok = mbar_wait(&empty[stage], phase ^ 1);
+        if constexpr (kFused) {
+          ok = ok && wait_flag_ge(hf.stats_flag + static_cast<long>(bh) * T + t, 1, hf.abort);
+          ok = ok && (t < hf.Rs || wait_flag_ge(hf.out_flag + static_cast<long>(bh) * T + t - hf.Rs,
+                                                1, hf.abort));
+          fence_async_global();
+        }
+        if (!ok) {
           give_up(hf, abort_flag);
           break;
         }
-        if constexpr (kFused) {
-          if (!wait_flag_ge(hf.stats_flag + static_cast<long>(bh) * T + t, 1, hf.abort)) {
-            give_up(hf, abort_flag);
-            break;
-          }
-          fence_async_global();
-        }
-        mbar_arrive(&b_ready[stage]);
+        mbar_arrive(&gate[t % L::kGate]);
         mbar_arrive_expect_tx(&full[stage], L::kABytes);
         uint8_t* st = smem + stage * L::kABytes;
         const int row = row_of(t);
@@ -151,13 +167,12 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       if (elect_one()) {
         const uint32_t a_base = smem_u32(smem + stage * L::kABytes);
 #pragma unroll
-        for (int kb = 0; kb < DP / 64; ++kb) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t da = smem_desc(s_base + kb * L::kSBlockBytes + ks * 32, 16, 1024);
-            const uint64_t db = smem_desc(a_base + kb * DP * 128 + ks * 32, 16, 1024);
-            mma_bf16(tmem_base, da, db, idesc, (kb | ks) != 0);
-          }
+        for (int ks = 0; ks < DP / 16; ++ks) {
+          // S tile: key groups 2ks, 2ks+1 (2048 B apart), 8-row groups 128 B apart
+          const uint64_t da = smem_desc_noswz(s_base + ks * 2 * 2048, 2048, 128);
+          // A_t stage: 128B-swizzled, 64-key blocks of DP rows
+          const uint64_t db = smem_desc(a_base + (ks >> 2) * DP * 128 + (ks & 3) * 32, 16, 1024);
+          mma_bf16(tmem_base, da, db, idesc, ks != 0);
         }
         mma_commit(mma_done);
         mma_commit(&empty[stage]);
@@ -165,43 +180,30 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       __syncwarp();
     }
     if (!ok) give_up(hf, abort_flag);
-  } else if (warp == L::kWarpStorer) {
-    // ---------------------------------------------------------------- S_t -> global, hand-off
-    if (elect_one()) {
-      tma_prefetch_desc(tm_s);
-      const uint64_t pol_s = policy_evict_last();
-      // Phase 0 of s_ready is the initial state. Wait for it first: a parity wait only tells the
-      // current phase from the previous one, so every phase must be waited for in order.
-      bool ok = mbar_wait(s_ready, 0);
-      for (int f = 0; f < T && ok; ++f) {
-        // the tile holds S_f once the epilogue's (f+1)-th arrival completes s_ready
-        if (!mbar_wait(s_ready, (f + 1) & 1)) {
-          ok = false;
-          break;
-        }
-        if constexpr (kFused) {
-          // the slot of frame f last held S_{f-R}; its output must have loaded it
-          if (f >= hf.R &&
-              !wait_flag_ge(hf.out_flag + static_cast<long>(bh) * T + f - hf.R, 1, hf.abort)) {
-            ok = false;
-            mbar_arrive(s_stored);
+  } else if (warp == L::kWarpPublisher) {
+    // ---------------------------------------------------------------- fused: publish S_t
+    if constexpr (kFused) {
+      if (elect_one()) {
+        int published = 0;
+        unsigned long long t0 = globaltimer_ns();
+        while (published < T) {
+          const int done = static_cast<int>(ld_acquire_cta(s_written) / L::kEpiWarps);
+          if (done > published) {
+            // every epilogue warp's S stores happen-before its release-add, which this thread
+            // has acquired; the GPU-scope release makes them visible to the outputs (which
+            // fence the async proxy after their acquire)
+            st_release(hf.chain_prog + bh, done);
+            published = done;
+            t0 = globaltimer_ns();
+            continue;
+          }
+          if (*abort_flag || ld_acquire(hf.abort) != 0 || globaltimer_ns() - t0 > kWaitLimitNs) {
+            give_up(hf, abort_flag);
             break;
           }
-        }
-#pragma unroll
-        for (int kb = 0; kb < DP / 64; ++kb)
-          tma_store_3d(tm_s, s_tile + kb * L::kSBlockBytes, kb * 64, 0, row_of(f), pol_s);
-        bulk_commit();
-        bulk_wait_read<0>();
-        mbar_arrive(s_stored);
-        if constexpr (kFused) {
-          bulk_wait_all();
-          fence_async_global();
-          st_release(hf.chain_prog + bh, f + 1);
+          __nanosleep(32);
         }
       }
-      bulk_wait_all();
-      if (!ok) give_up(hf, abort_flag);
     }
   } else {
     // ---------------------------------------------------------------- epilogue (512 threads)
@@ -211,44 +213,54 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + c0;
     const bool row_ok = v < D;
     float S[L::kCols];
-    float Bv[L::kCols];
     const float* sin = state_in ? state_in + (static_cast<long>(bh) * D + v) * D : nullptr;
 #pragma unroll
     for (int j = 0; j < L::kCols; ++j) {
       const int col = c0 + j;
       S[j] = (sin != nullptr && row_ok && col < D) ? sin[col] : 0.f;
     }
+    auto pack8 = [&](int j) {
+      uint4 pk;
+      pk.x = pack_bf16x2(S[j], S[j + 1]);
+      pk.y = pack_bf16x2(S[j + 2], S[j + 3]);
+      pk.z = pack_bf16x2(S[j + 4], S[j + 5]);
+      pk.w = pack_bf16x2(S[j + 6], S[j + 7]);
+      return pk;
+    };
     auto write_s_tile = [&]() {
 #pragma unroll
-      for (int j = 0; j < L::kCols; j += 8) {
-        uint4 pk;
-        pk.x = pack_bf16x2(S[j], S[j + 1]);
-        pk.y = pack_bf16x2(S[j + 2], S[j + 3]);
-        pk.z = pack_bf16x2(S[j + 4], S[j + 5]);
-        pk.w = pack_bf16x2(S[j + 6], S[j + 7]);
-        *reinterpret_cast<uint4*>(s_tile + swz128_offset_bf16(v, c0 + j, L::kSBlockBytes)) = pk;
-      }
+      for (int j = 0; j < L::kCols; j += 8)
+        *reinterpret_cast<uint4*>(s_tile + ((c0 + j) >> 3) * 2048 + v * 16) = pack8(j);
     };
-    // B_f slice of this thread, from L2 (never L1: ring slots are rewritten)
-    auto load_b = [&](int f) {
+    // this thread's 16-byte group kg of row v in a B buffer
+    auto b_slot = [&](int buf, int kg) {
+      return b_buf + buf * L::kBBufBytes + (static_cast<uint32_t>(kg) * 128 + v) * 16;
+    };
+    // copy this thread's slice of B_f (from L2) into buffer f % 2, one commit group per frame
+    auto issue_b = [&](int f) -> bool {
+      if (!mbar_wait(&gate[f % L::kGate], (f / L::kGate) & 1)) return false;
       const float* bm = B_ws + static_cast<long>(row_of(f)) * D * D;
+      if (row_ok) {
 #pragma unroll
-      for (int j = 0; j < L::kCols; j += 4) {
-        const int col = c0 + j;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (row_ok && col < D) x = __ldcg(reinterpret_cast<const float4*>(bm + b4_index(v, col, D)));
-        Bv[j] = x.x;
-        Bv[j + 1] = x.y;
-        Bv[j + 2] = x.z;
-        Bv[j + 3] = x.w;
+        for (int j = 0; j < L::kCols; j += 4) {
+          const int col = c0 + j;
+          if (col < D) cp_async16(b_slot(f & 1, col >> 2), bm + b4_index(v, col, D));
+        }
       }
+      cp_async_commit();
+      return true;
     };
     write_s_tile();
     fence_async_smem();
     tc_fence_before();
-    bool ok = mbar_wait(&b_ready[0], 0);
+    bool ok = issue_b(0);
+    if (ok) {
+      if (T > 1)
+        ok = issue_b(1);
+      else
+        cp_async_commit();
+    }
     mbar_arrive(s_ready);
-    if (ok) load_b(0);
 
     // gamma_t, beta_t: each lane holds frame (32*blk + lane) of the current and next block of
     // 32 frames; the value for frame t is shuffled from lane t % 32.
@@ -268,10 +280,11 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       }
       const float g = __shfl_sync(0xffffffffu, g_cur, t & 31);
       const float be = __shfl_sync(0xffffffffu, b_cur, t & 31);
-      if (!mbar_wait(mma_done, t & 1) || (t > 0 && !mbar_wait(s_stored, (t - 1) & 1))) {
+      if (!mbar_wait(mma_done, t & 1)) {
         ok = false;
         break;
       }
+      cp_async_wait<1>();  // this thread's copy of B_t (B_{t+1} may still be in flight)
       tc_fence_after();
       const float gbe = g * be;
 #pragma unroll
@@ -279,22 +292,43 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
         float P[16];
         tmem_ld16(taddr + c, P);
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          S[c + j] = fmaf(g, S[c + j], fmaf(be, Bv[c + j], -gbe * P[j]));
+        for (int j = 0; j < 16; j += 4) {
+          const int col = c0 + c + j;
+          float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (row_ok && col < D) bv = *reinterpret_cast<const float4*>(b_slot(t & 1, col >> 2));
+          S[c + j] = fmaf(g, S[c + j], fmaf(be, bv.x, -gbe * P[j]));
+          S[c + j + 1] = fmaf(g, S[c + j + 1], fmaf(be, bv.y, -gbe * P[j + 1]));
+          S[c + j + 2] = fmaf(g, S[c + j + 2], fmaf(be, bv.z, -gbe * P[j + 2]));
+          S[c + j + 3] = fmaf(g, S[c + j + 3], fmaf(be, bv.w, -gbe * P[j + 3]));
+        }
       }
       write_s_tile();
       fence_async_smem();
       tc_fence_before();
-      // wait for frame t+1's gate before completing s_ready: the producer can only re-arm this
-      // stage's b_ready after the MMA of frame t+1, which needs this s_ready
-      if (t + 1 < T && !mbar_wait(&b_ready[(t + 1) % L::kStages], ((t + 1) / L::kStages) & 1)) {
-        ok = false;
-        mbar_arrive(s_ready);
-        break;
-      }
       mbar_arrive(s_ready);
-      if (t + 1 < T) load_b(t + 1);
+      // S_t to global (its slot was gated free): rows past D and M-padding rows hold zeros,
+      // rows >= DP (M-padding when DP == 64) are not part of the stored matrix
+      if (v < DP) {
+        uint8_t* srow = reinterpret_cast<uint8_t*>(S_out + static_cast<long>(srow_of(t)) * DP * DP);
+#pragma unroll
+        for (int j = 0; j < L::kCols; j += 8)
+          *reinterpret_cast<uint4*>(srow + s8_offset_bytes(v, c0 + j, DP)) = pack8(j);
+      }
+      if constexpr (kFused) {
+        __syncwarp();  // the warp's S stores before its lane 0's release-add
+        if (lane == 0) red_add_release_cta(s_written, 1);
+      }
+      // buffer t % 2 is free (this thread read its own slice above): copy B_{t+2} into it
+      if (t + 2 < T) {
+        if (!issue_b(t + 2)) {
+          ok = false;
+          break;
+        }
+      } else {
+        cp_async_commit();
+      }
     }
+    cp_async_wait<0>();
     if (!ok) give_up(hf, abort_flag);
     if (state_out != nullptr && row_ok) {
       float* so = state_out + (static_cast<long>(bh) * D + v) * D;
@@ -316,12 +350,12 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
 template <int DP>
 __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
     gdn_chain_kernel(const __grid_constant__ CUtensorMap tm_a, const float* __restrict__ B_ws,
-                     const __grid_constant__ CUtensorMap tm_s, const float* __restrict__ gamma,
+                     __nv_bfloat16* __restrict__ S_ws, const float* __restrict__ gamma,
                      const float* __restrict__ beta, const float* __restrict__ state_in,
                      float* __restrict__ state_out, Problem p) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 0, 0};
-  chain_body<DP, false>(&tm_a, B_ws, &tm_s, gamma, beta, state_in, state_out, p, none,
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  chain_body<DP, false>(&tm_a, B_ws, S_ws, gamma, beta, state_in, state_out, p, none,
                         align1k(smem_raw));
 }
 

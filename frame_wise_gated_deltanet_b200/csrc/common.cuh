@@ -24,13 +24,14 @@ struct Problem {
 
 // Hand-off state of the fused forward, in device memory and zeroed before each call. One
 // persistent grid runs three roles: stats CTAs write A_t, B_t into per-head rings of R slots,
-// chain CTAs consume them and write S_t into a ring of R slots, output CTAs consume S_t.
+// chain CTAs consume them and write S_t into per-head rings of Rs slots, output CTAs consume S_t.
 struct Handoff {
   int* stats_flag;  // [B*H*T] 1 once A_t, B_t of (bh, t) are in ring slot t % R
   int* out_flag;    // [B*H*T] 1 once the output of (bh, t) has loaded S_t (its slot is free)
   int* chain_prog;  // [B*H]   number of frames whose S_t the chain has stored
   int* abort;       // set by the first CTA that gives up a wait; every wait then returns
-  int R;            // ring slots per head
+  int R;            // A_t / B_t ring slots per head (how far the statistics may run ahead)
+  int Rs;           // S_t ring slots per head (how far the outputs may lag behind)
   int base;         // first blockIdx.x of this role
   int count;        // CTAs in this role
 };
@@ -47,6 +48,15 @@ __device__ __forceinline__ void give_up(const Handoff& hf, volatile int* local_a
 // group, for both the writer (one thread per row) and the reader (one thread per row).
 __host__ __device__ __forceinline__ long b4_index(int v, int k, int D) {
   return (static_cast<long>(k >> 2) * D + v) * 4 + (k & 3);
+}
+
+// S_t storage between the chain and the output GEMM: a DP x DP bf16 matrix (zero-padded past D)
+// as K-major 8 x 16-byte core matrices, element (v, k) at bf16 index ((k / 8) * DP + v) * 8 +
+// k % 8. It is directly a no-swizzle MMA operand (LBO = DP*16 bytes between key groups, SBO =
+// 128 bytes between 8-row groups), one contiguous DP*DP*2-byte block per frame, and a warp that
+// owns 32 consecutive rows writes it as 512 contiguous bytes per key group.
+__host__ __device__ __forceinline__ long s8_offset_bytes(int v, int k, int DP) {
+  return (static_cast<long>(k >> 3) * DP + v) * 16 + (k & 7) * 2;
 }
 
 // TMA box: 64 bf16 (128 B, one swizzle row) x 128 rows.

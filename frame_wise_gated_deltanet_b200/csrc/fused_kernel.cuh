@@ -6,8 +6,8 @@
 //   blocks [.., gridDim.x)       output role: O_t from ring slots of S_t
 //
 // A_t (bf16), B_t (f32) and S_t (bf16) travel through per-head rings of R slots (a few tens of
-// MB, L2-resident: loaded and stored with evict_last while the q/k/v/out streams use
-// evict_first). Hand-off is by release/acquire flags in global memory with bounded waits;
+// MB, meant to stay in L2: A_t and S_t are loaded with evict_last while the q/k/v/out streams
+// use evict_first). Hand-off is by release/acquire flags in global memory with bounded waits;
 // every role processes its items in increasing frame order and every wait points at a
 // strictly earlier frame (or at the chain, which only waits on earlier frames), so with all
 // CTAs co-resident the grid cannot deadlock.
@@ -38,20 +38,20 @@ __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_o,
                      const __grid_constant__ CUtensorMap tm_a_ring,
-                     const __grid_constant__ CUtensorMap tm_s_ring,
                      __nv_bfloat16* __restrict__ A_ring, float* __restrict__ B_ring,
+                     __nv_bfloat16* __restrict__ S_ring,
                      const float* __restrict__ gamma, const float* __restrict__ beta,
                      const float* __restrict__ state_in, float* __restrict__ state_out, Problem p,
                      Handoff h_chain, Handoff h_stats, Handoff h_out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
   if (static_cast<int>(blockIdx.x) < h_stats.base) {
-    chain_body<DP, true>(&tm_a_ring, B_ring, &tm_s_ring, gamma, beta, state_in, state_out, p,
+    chain_body<DP, true>(&tm_a_ring, B_ring, S_ring, gamma, beta, state_in, state_out, p,
                          h_chain, smem);
   } else if (static_cast<int>(blockIdx.x) < h_out.base) {
     stats_body<DP, false, true, true>(&tm_k, &tm_v, A_ring, B_ring, p, h_stats, smem);
   } else {
-    output_body<DP, false, true>(&tm_q, &tm_s_ring, &tm_o, p, 1, h_out, smem);
+    output_body<DP, false, true>(&tm_q, &tm_q, S_ring, &tm_o, p, 1, h_out, smem);
   }
 }
 

@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -214,15 +215,14 @@ gdn_status run_chain(int dev, const Problem& p, const void* A, const float* Bm,
                      float* s_out, cudaStream_t st) {
   using L = gdn::ChainLayout<DP>;
   const long count = long(p.B) * p.H * p.T;
-  CUtensorMap ta, ts;
-  if (!tmap_mats(&ta, A, false, p.D, p.D, count, DP) ||
-      !tmap_mats(&ts, S_ws, false, p.D, p.D, count, DP))
-    return GDN_ERR_CUDA;
+  CUtensorMap ta;
+  if (!tmap_mats(&ta, A, false, p.D, p.D, count, DP)) return GDN_ERR_CUDA;
   auto kern = gdn::gdn_chain_kernel<DP>;
   if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 2 : 3, kern, L::kSmemBytes)) return s;
   {
     ProfiledLaunch pl("gdn_chain_kernel", st);
-    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, Bm, ts, gamma, beta, s_in, s_out, p);
+    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, Bm, static_cast<__nv_bfloat16*>(S_ws),
+                                                        gamma, beta, s_in, s_out, p);
   }
   return check_launch();
 }
@@ -233,9 +233,12 @@ gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws
   using L = gdn::OutputLayout<DP, kLA>;
   const long count = long(p.B) * p.H * p.T;
   CUtensorMap tq, ts, to;
-  if (!tmap_tokens(&tq, q, p) || !tmap_mats(&ts, S_ws, false, p.D, srows, count, DP) ||
-      !tmap_tokens(&to, out, p))
-    return GDN_ERR_CUDA;
+  if (!tmap_tokens(&tq, q, p) || !tmap_tokens(&to, out, p)) return GDN_ERR_CUDA;
+  if (kLA) {
+    if (!tmap_mats(&ts, S_ws, false, p.D, srows, count, DP)) return GDN_ERR_CUDA;
+  } else {
+    ts = tq;  // unused: GDN states are bulk-copied from S_ws
+  }
   auto kern = gdn::gdn_output_kernel<DP, kLA>;
   if (gdn_status s = ensure_smem_attr(dev, kLA ? 6 : (DP == 128 ? 4 : 5), kern, L::kSmemBytes))
     return s;
@@ -243,7 +246,8 @@ gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
   {
     ProfiledLaunch pl("gdn_output_kernel", st);
-    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, ts, to, p, F);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(
+        tq, ts, static_cast<const __nv_bfloat16*>(S_ws), to, p, F);
   }
   return check_launch();
 }
@@ -254,9 +258,12 @@ struct ForwardWs {
   void* S;
 };
 
+int padded_dim(int D) { return D <= 64 ? 64 : 128; }
+
+// per frame-head: A_t bf16 D x D, B_t f32 D x D, S_t bf16 DP x DP (core-matrix layout)
 size_t forward_ws_bytes(long count, int D) {
-  const size_t m = size_t(D) * D;
-  return align256(count * m * 2) + align256(count * m * 4) + align256(count * m * 2);
+  const size_t m = size_t(D) * D, dp = padded_dim(D);
+  return align256(count * m * 2) + align256(count * m * 4) + align256(count * dp * dp * 2);
 }
 
 ForwardWs carve_forward(void* base, long count, int D) {
@@ -274,7 +281,29 @@ ForwardWs carve_forward(void* base, long count, int D) {
 // ------------------------------------------------------------------ fused forward
 // 0 = choose automatically, 1 = always the three-kernel path, 2 = fused whenever it applies.
 int g_forward_mode = 0;
-constexpr int kRing = 16;  // ring slots per head of the fused forward
+
+// Tuning of the fused forward, read once from the environment:
+//   GDN_FUSED_RING       A_t / B_t ring slots per head (default 16, 4..64)
+//   GDN_FUSED_SRING      S_t ring slots per head (default 32, 8..64)
+//   GDN_FUSED_STATS_PCT  share of the non-chain SMs given to the stats role (default 54, 20..80)
+int env_int(const char* name, int dflt, int lo, int hi) {
+  const char* s = getenv(name);
+  if (s == nullptr || *s == 0) return dflt;
+  const int v = atoi(s);
+  return v < lo ? lo : (v > hi ? hi : v);
+}
+int fused_ring() {
+  static const int r = env_int("GDN_FUSED_RING", 16, 4, 64);
+  return r;
+}
+int fused_sring() {
+  static const int r = env_int("GDN_FUSED_SRING", 32, 8, 64);
+  return r;
+}
+int fused_stats_pct() {
+  static const int p = env_int("GDN_FUSED_STATS_PCT", 54, 20, 80);
+  return p;
+}
 
 struct FusedWs {
   void* A;
@@ -285,13 +314,17 @@ struct FusedWs {
 };
 
 size_t fused_ws_bytes(long bh, long T, int D) {
+  const int kRing = fused_ring();
   const size_t m = size_t(D) * D * bh * kRing;
+  const size_t dp = padded_dim(D), ms = dp * dp * bh * fused_sring();
   const size_t flags = sizeof(int) * (2 * bh * T + bh + 1);
-  return align256(m * 2) + align256(m * 4) + align256(m * 2) + align256(flags);
+  return align256(m * 2) + align256(m * 4) + align256(ms * 2) + align256(flags);
 }
 
 FusedWs carve_fused(void* base, long bh, long T, int D) {
+  const int kRing = fused_ring();
   const size_t m = size_t(D) * D * bh * kRing;
+  const size_t dp = padded_dim(D), ms = dp * dp * bh * fused_sring();
   uint8_t* p = static_cast<uint8_t*>(base);
   FusedWs w;
   w.A = p;
@@ -299,7 +332,7 @@ FusedWs carve_fused(void* base, long bh, long T, int D) {
   w.B = reinterpret_cast<float*>(p);
   p += align256(m * 4);
   w.S = p;
-  p += align256(m * 2);
+  p += align256(ms * 2);
   w.flags = reinterpret_cast<int*>(p);
   w.flag_bytes = sizeof(int) * (2 * bh * T + bh + 1);
   return w;
@@ -325,26 +358,26 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   using L = gdn::FusedLayout<DP>;
   const int sms = g_dev[dev].sms;
   const int bh = p.B * p.H;
+  const int kRing = fused_ring();
   void* base = nullptr;
   if (gdn_status s = get_workspace(dev, fused_ws_bytes(bh, p.T, p.D), st, &base)) return s;
   FusedWs w = carve_fused(base, bh, p.T, p.D);
   if (cudaMemsetAsync(w.flags, 0, w.flag_bytes, st) != cudaSuccess) return GDN_ERR_CUDA;
-  CUtensorMap tk, tv, tq, to, ta, ts;
+  CUtensorMap tk, tv, tq, to, ta;
   if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p) || !tmap_tokens(&tq, q, p) ||
-      !tmap_tokens(&to, out, p) || !tmap_mats(&ta, w.A, false, p.D, p.D, long(bh) * kRing, DP) ||
-      !tmap_mats(&ts, w.S, false, p.D, p.D, long(bh) * kRing, DP))
+      !tmap_tokens(&to, out, p) || !tmap_mats(&ta, w.A, false, p.D, p.D, long(bh) * kRing, DP))
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_fused_kernel<DP>;
   if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 8 : 9, kern, L::kSmemBytes)) return s;
-  // split the SMs left after the chains between the stats and output roles (~54 : 46, the
-  // ratio of their per-frame times)
+  // split the SMs left after the chains between the stats and output roles (by default
+  // ~54 : 46, the ratio of their per-frame times)
   const int workers = sms - bh;
-  int n_stats = (workers * 54 + 50) / 100;
+  int n_stats = (workers * fused_stats_pct() + 50) / 100;
   if (n_stats < 1) n_stats = 1;
   if (n_stats > workers - 1) n_stats = workers - 1;
   int* f = w.flags;
   const long ft = long(bh) * p.T;
-  gdn::Handoff hc{f, f + ft, f + 2 * ft, f + 2 * ft + bh, kRing, 0, bh};
+  gdn::Handoff hc{f, f + ft, f + 2 * ft, f + 2 * ft + bh, kRing, fused_sring(), 0, bh};
   gdn::Handoff hs = hc;
   hs.base = bh;
   hs.count = n_stats;
@@ -353,8 +386,9 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   ho.count = workers - n_stats;
   __nv_bfloat16* a_ring = static_cast<__nv_bfloat16*>(w.A);
   float* b_ring = w.B;
+  __nv_bfloat16* s_ring = static_cast<__nv_bfloat16*>(w.S);
   gdn::Problem pp = p;
-  void* args[] = {&tk, &tv, &tq, &to, &ta, &ts, &a_ring, &b_ring,
+  void* args[] = {&tk, &tv, &tq, &to, &ta, &a_ring, &b_ring, &s_ring,
                   const_cast<float**>(&gamma), const_cast<float**>(&beta),
                   const_cast<float**>(&s_in), &s_out, &pp, &hc, &hs, &ho};
   {

@@ -2,8 +2,9 @@
 // reads the post-update state S_t, so attention is bidirectional inside a frame and causal
 // across frames).
 //
-// Per work item (b, t, h): S_t (bf16, D x D, row v / column k) is TMA-loaded once as a K-major
-// B operand; the frame's Q rows stream through a ring of 128-token TMA tiles (K-major A
+// Per work item (b, t, h): S_t is loaded once as a K-major B operand -- for GDN one contiguous
+// bulk copy of the DP x DP bf16 block in the core-matrix layout of s8_offset_bytes (the chain's
+// output), for LA a TMA load of the row-major (D+1) x D state; the frame's Q rows stream through a ring of 128-token TMA tiles (K-major A
 // operand); each tile is one 128 x DP x DP tcgen05 GEMM into a double-buffered TMEM
 // accumulator; the epilogue converts rows to bf16 into a 128B-swizzled staging tile in shared
 // memory and one thread TMA-stores it to out[b, t, n, h, :] (rows past N and columns past D are
@@ -18,7 +19,7 @@
 //
 // Standalone (gdn_output_kernel): work item i = (b*T + t)*H + h, S_t at workspace row
 // (b*H+h)*T + t_state. Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h
-// (frame-major), S_t loaded from ring row (b*H+h)*R + t%R once chain_prog says it is there;
+// (frame-major), S_t loaded from ring row (b*H+h)*Rs + t%Rs once chain_prog says it is there;
 // out_flag releases the slot as soon as S_t is in shared memory.
 #pragma once
 #include <cuda.h>
@@ -64,9 +65,11 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p) {
 }
 
 // frames_per_block: 1 for GDN (frame t reads S_t); F for LA (frame t reads the state at the end
-// of its block of F frames).
+// of its block of F frames). GDN states come from S_src (DP*DP bf16 per row, s8 layout); LA
+// states through tm_s.
 template <int DP, bool kLA, bool kFused>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
+                                            const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
                                             uint8_t* smem) {
@@ -119,7 +122,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   if (warp == 0) {
     if (elect_one()) {
       tma_prefetch_desc(tm_q);
-      tma_prefetch_desc(tm_s);
+      if constexpr (kLA) tma_prefetch_desc(tm_s);
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_state = policy_evict_last();
       int stage = 0;
@@ -129,7 +132,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         const OutputItem it = output_item<kFused>(item, p);
         int srow;
         if constexpr (kFused) {
-          srow = it.bh * hf.R + it.t % hf.R;
+          srow = it.bh * hf.Rs + it.t % hf.Rs;
         } else {
           const int t_state = (F <= 1) ? it.t : min((it.t / F + 1) * F, p.T) - 1;
           srow = it.bh * p.T + t_state;
@@ -147,10 +150,15 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           fence_async_global();
         }
         mbar_arrive_expect_tx(&s_full[sb], L::kSBufBytes);
+        if constexpr (kLA) {
 #pragma unroll
-        for (int kb = 0; kb < L::kBoxes; ++kb)
-          tma_load_3d(s_buf + sb * L::kSBufBytes + kb * DP * 128, tm_s, &s_full[sb], kb * 64, 0,
-                      srow, pol_state);
+          for (int kb = 0; kb < L::kBoxes; ++kb)
+            tma_load_3d(s_buf + sb * L::kSBufBytes + kb * DP * 128, tm_s, &s_full[sb], kb * 64,
+                        0, srow, pol_state);
+        } else {
+          bulk_load(s_buf + sb * L::kSBufBytes, S_src + static_cast<long>(srow) * DP * DP,
+                    L::kSBufBytes, &s_full[sb], pol_state);
+        }
         for (int tile = 0; tile < n_tiles; ++tile) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
             give_up(hf, abort_flag);
@@ -198,13 +206,15 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         if (elect_one()) {
           const uint32_t q_base = smem_u32(q_ring + stage * L::kQBytes);
 #pragma unroll
-          for (int kb = 0; kb < L::kBoxes; ++kb) {
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t da = smem_desc(q_base + kb * kBoxBytes + ks * 32, 16, 1024);
-              const uint64_t db = smem_desc(s_base + kb * DP * 128 + ks * 32, 16, 1024);
-              mma_bf16(tmem_base + acc * DP, da, db, idesc, (kb | ks) != 0);
-            }
+          for (int ks = 0; ks < DP / 16; ++ks) {
+            const uint64_t da =
+                smem_desc(q_base + (ks >> 2) * kBoxBytes + (ks & 3) * 32, 16, 1024);
+            // LA: row-major state through a 128B-swizzled TMA box; GDN: core matrices, key
+            // groups 2ks and 2ks+1 (DP*16 bytes apart), 8-row groups 128 bytes apart
+            const uint64_t db =
+                kLA ? smem_desc(s_base + (ks >> 2) * DP * 128 + (ks & 3) * 32, 16, 1024)
+                    : smem_desc_noswz(s_base + ks * 2 * DP * 16, DP * 16, 128);
+            mma_bf16(tmem_base + acc * DP, da, db, idesc, ks != 0);
           }
           mma_commit(&empty[stage]);
           mma_commit(&acc_full[acc]);
@@ -328,10 +338,11 @@ template <int DP, bool kLA>
 __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
     gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_s,
+                      const __nv_bfloat16* __restrict__ S_src,
                       const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 0, 0};
-  output_body<DP, kLA, false>(&tm_q, &tm_s, &tm_o, p, frames_per_block, none,
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  output_body<DP, kLA, false>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
                               align1k(smem_raw));
 }
 

@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
                      float* __restrict__ B_ws, Problem p) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
   stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw));
 }
 
