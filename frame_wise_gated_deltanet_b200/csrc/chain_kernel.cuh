@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
                      const float* __restrict__ beta, const float* __restrict__ state_in,
                      float* __restrict__ state_out, Problem p) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
   chain_body<DP, false>(&tm_a, B_ws, S_ws, gamma, beta, state_in, state_out, p, none,
                         align1k(smem_raw));
 }

@@ -30,10 +30,33 @@ struct Handoff {
   int* out_flag;    // [B*H*T] 1 once the output of (bh, t) has loaded S_t (its slot is free)
   int* chain_prog;  // [B*H]   number of frames whose S_t the chain has stored
   int* abort;       // set by the first CTA that gives up a wait; every wait then returns
+  int* next_item;   // this role's work counter (stats and output roles take items dynamically)
   int R;            // A_t / B_t ring slots per head (how far the statistics may run ahead)
   int Rs;           // S_t ring slots per head (how far the outputs may lag behind)
   int base;         // first blockIdx.x of this role
   int count;        // CTAs in this role
+};
+
+// Dynamic work distribution inside a CTA of the fused forward: the producer thread takes the
+// next item of its role from a global counter (so items start in global frame-major order,
+// whichever CTA is free) and passes the item id to the CTA's other warps through an 8-slot ring
+// of (id, mbarrier) pairs. The producer runs at most a few items ahead of the last consumer
+// (its tile stages and the two TMEM accumulators bound it), so 8 slots are never overrun.
+struct ItemRing {
+  int* ids;        // shared [8]
+  uint64_t* bars;  // shared [8], arrival count 1
+  __device__ __forceinline__ long produce(int li, int* counter, long n_items) {
+    long it = atomicAdd(counter, 1);
+    if (it >= n_items) it = -1;
+    ids[li & 7] = static_cast<int>(it);
+    mbar_arrive(&bars[li & 7]);
+    return it;
+  }
+  // -2 if the wait timed out, -1 once the role's items are exhausted
+  __device__ __forceinline__ long consume(int li) {
+    if (!mbar_wait(&bars[li & 7], (li >> 3) & 1)) return -2;
+    return ids[li & 7];
+  }
 };
 
 __device__ __forceinline__ void give_up(const Handoff& hf, volatile int* local_abort) {

@@ -283,7 +283,7 @@ ForwardWs carve_forward(void* base, long count, int D) {
 int g_forward_mode = 0;
 
 // Tuning of the fused forward, read once from the environment:
-//   GDN_FUSED_RING       A_t / B_t ring slots per head (default 16, 4..64)
+//   GDN_FUSED_RING       A_t / B_t ring slots per head (default 24, 4..64)
 //   GDN_FUSED_SRING      S_t ring slots per head (default 32, 8..64)
 //   GDN_FUSED_STATS_PCT  share of the non-chain SMs given to the stats role (default 54, 20..80)
 int env_int(const char* name, int dflt, int lo, int hi) {
@@ -293,7 +293,7 @@ int env_int(const char* name, int dflt, int lo, int hi) {
   return v < lo ? lo : (v > hi ? hi : v);
 }
 int fused_ring() {
-  static const int r = env_int("GDN_FUSED_RING", 16, 4, 64);
+  static const int r = env_int("GDN_FUSED_RING", 24, 4, 64);
   return r;
 }
 int fused_sring() {
@@ -309,7 +309,7 @@ struct FusedWs {
   void* A;
   float* B;
   void* S;
-  int* flags;  // stats_flag [BH*T], out_flag [BH*T], chain_prog [BH], abort [1]
+  int* flags;  // stats_flag [BH*T], out_flag [BH*T], chain_prog [BH], abort, 2 work counters
   size_t flag_bytes;
 };
 
@@ -317,7 +317,7 @@ size_t fused_ws_bytes(long bh, long T, int D) {
   const int kRing = fused_ring();
   const size_t m = size_t(D) * D * bh * kRing;
   const size_t dp = padded_dim(D), ms = dp * dp * bh * fused_sring();
-  const size_t flags = sizeof(int) * (2 * bh * T + bh + 1);
+  const size_t flags = sizeof(int) * (2 * bh * T + bh + 3);
   return align256(m * 2) + align256(m * 4) + align256(ms * 2) + align256(flags);
 }
 
@@ -334,7 +334,7 @@ FusedWs carve_fused(void* base, long bh, long T, int D) {
   w.S = p;
   p += align256(ms * 2);
   w.flags = reinterpret_cast<int*>(p);
-  w.flag_bytes = sizeof(int) * (2 * bh * T + bh + 1);
+  w.flag_bytes = sizeof(int) * (2 * bh * T + bh + 3);
   return w;
 }
 
@@ -377,13 +377,16 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   if (n_stats > workers - 1) n_stats = workers - 1;
   int* f = w.flags;
   const long ft = long(bh) * p.T;
-  gdn::Handoff hc{f, f + ft, f + 2 * ft, f + 2 * ft + bh, kRing, fused_sring(), 0, bh};
+  int* abort_word = f + 2 * ft + bh;
+  gdn::Handoff hc{f, f + ft, f + 2 * ft, abort_word, nullptr, kRing, fused_sring(), 0, bh};
   gdn::Handoff hs = hc;
   hs.base = bh;
   hs.count = n_stats;
+  hs.next_item = abort_word + 1;
   gdn::Handoff ho = hc;
   ho.base = bh + n_stats;
   ho.count = workers - n_stats;
+  ho.next_item = abort_word + 2;
   __nv_bfloat16* a_ring = static_cast<__nv_bfloat16*>(w.A);
   float* b_ring = w.B;
   __nv_bfloat16* s_ring = static_cast<__nv_bfloat16*>(w.S);

@@ -84,7 +84,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   uint64_t* s_empty = s_full + 2;
   uint64_t* acc_full = s_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 8), acc_empty + 2};  // fused only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id();
@@ -94,6 +95,18 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   const int F = frames_per_block;
   const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
   const long ncta = kFused ? hf.count : gridDim.x;
+  // item li of this CTA: standalone a static stride, fused the role's work counter. Returns -1
+  // when there are no more items, -2 on a timed-out wait.
+  auto producer_item = [&](int li) -> long {
+    if constexpr (kFused) return ring.produce(li, hf.next_item, n_items);
+    const long it = cta0 + static_cast<long>(li) * ncta;
+    return it < n_items ? it : -1;
+  };
+  auto consumer_item = [&](int li) -> long {
+    if constexpr (kFused) return ring.consume(li);
+    const long it = cta0 + static_cast<long>(li) * ncta;
+    return it < n_items ? it : -1;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -107,6 +120,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 128);
     }
+    for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -127,8 +141,9 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       const uint64_t pol_state = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      int li = 0;
-      for (long item = cta0; item < n_items && !*abort_flag; item += ncta, ++li) {
+      for (int li = 0; !*abort_flag; ++li) {
+        const long item = producer_item(li);
+        if (item < 0) break;
         const OutputItem it = output_item<kFused>(item, p);
         int srow;
         if constexpr (kFused) {
@@ -180,10 +195,12 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
     int stage = 0;
     uint32_t phase = 0;
-    int li = 0;
     int tc = 0;  // tiles processed (accumulator ring position)
     bool ok = true;
-    for (long item = cta0; item < n_items && ok; item += ncta, ++li) {
+    for (int li = 0; ok; ++li) {
+      const long item = consumer_item(li);
+      if (item == -2) ok = false;
+      if (item < 0) break;
       const int sb = li & 1;
       if (!mbar_wait(&s_full[sb], (li >> 1) & 1)) {
         ok = false;
@@ -241,7 +258,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     if (leader) tma_prefetch_desc(tm_o);
     int tc = 0;
     bool ok = true;
-    for (long item = cta0; item < n_items && ok; item += ncta) {
+    for (int li = 0; ok; ++li) {
+      const long item = consumer_item(li);
+      if (item == -2) ok = false;
+      if (item < 0) break;
       const OutputItem it = output_item<kFused>(item, p);
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
@@ -300,7 +320,9 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (long item = cta0; item < n_items && ok; item += ncta) {
+    for (int li = 0; ok; ++li) {
+      const long item = consumer_item(li);
+      if (item < 0) break;
       for (int tile = 0; tile < n_tiles; ++tile) {
         if (!mbar_wait(&full[stage], phase)) {
           ok = false;
@@ -341,7 +363,7 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
                       const __nv_bfloat16* __restrict__ S_src,
                       const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
   output_body<DP, kLA, false>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
                               align1k(smem_raw));
 }

@@ -79,7 +79,8 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
   uint64_t* empty = ready + L::kStages;
   uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 8), acc_empty + 2};  // fused only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id();
@@ -88,6 +89,18 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
   const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
   const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
   const long ncta = kFused ? hf.count : gridDim.x;
+  // item li of this CTA: standalone a static stride, fused the role's work counter. Returns -1
+  // when there are no more items, -2 on a timed-out wait.
+  auto producer_item = [&](int li) -> long {
+    if constexpr (kFused) return ring.produce(li, hf.next_item, n_items);
+    const long it = cta0 + static_cast<long>(li) * ncta;
+    return it < n_items ? it : -1;
+  };
+  auto consumer_item = [&](int li) -> long {
+    if constexpr (kFused) return ring.consume(li);
+    const long it = cta0 + static_cast<long>(li) * ncta;
+    return it < n_items ? it : -1;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -99,6 +112,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 128);
     }
+    for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -119,7 +133,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       const uint64_t pol = policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
-      for (long item = cta0; item < n_items && !*abort_flag; item += ncta) {
+      for (int li = 0; !*abort_flag; ++li) {
+        const long item = producer_item(li);
+        if (item < 0) break;
         const StatsItem it = stats_item<kFused>(item, p, hf);
         for (int tile = 0; tile < n_tiles; ++tile) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
@@ -149,8 +165,13 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
                                                 : idesc_bf16(128, 64, true, true));
     int stage = 0;
     uint32_t phase = 0;
-    int li = 0;
-    for (long item = cta0; item < n_items; item += ncta, ++li) {
+    for (int li = 0;; ++li) {
+      const long item = consumer_item(li);
+      if (item == -2) {
+        give_up(hf, abort_flag);
+        break;
+      }
+      if (item < 0) break;
       const int acc = li & 1;
       const uint32_t aph = (li >> 1) & 1;
       if (!mbar_wait(&acc_empty[acc], aph ^ 1)) {
@@ -213,8 +234,13 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     const float s = p.key_scale;
     const int D = p.D;
     const int brows = kLA ? D + 1 : D;
-    int li = 0;
-    for (long item = cta0; item < n_items; item += ncta, ++li) {
+    for (int li = 0;; ++li) {
+      const long item = consumer_item(li);
+      if (item == -2) {
+        give_up(hf, abort_flag);
+        break;
+      }
+      if (item < 0) break;
       const int acc = li & 1;
       const uint32_t aph = (li >> 1) & 1;
       const StatsItem it = stats_item<kFused>(item, p, hf);
@@ -309,7 +335,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     int stage = 0;
     uint32_t phase = 0;
     const int D = p.D;
-    for (long item = cta0; item < n_items; item += ncta) {
+    for (int li = 0;; ++li) {
+      const long item = consumer_item(li);
+      if (item < 0) break;
       bool ok = true;
       for (int tile = 0; tile < n_tiles; ++tile) {
         if (!mbar_wait(&full[stage], phase)) {
@@ -361,7 +389,7 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
                      float* __restrict__ B_ws, Problem p) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
   stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw));
 }
 
