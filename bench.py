@@ -85,6 +85,8 @@ def kernel_bytes(name, w):
         return fh * (dd * 2 + dd * 4 + dd * 2 + 8) + w.B * w.H * dd * 4
     if name == "gdn_output_kernel":      # read Q, S_t; write O
         return fh * (2 * nd2 + dd * 2)
+    if name == "gdn_fused_kernel":       # the whole path in one launch
+        return algorithmic_bytes(w)
     return None
 
 

@@ -71,7 +71,8 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
   uint64_t* s_ready = mma_done + 1;      // the S tile holds the new state
   // fused: epilogue warps that have written their part of S_t to global memory, summed over
   // frames (kEpiWarps per frame); a counter, not a barrier, so the publisher may lag freely
-  uint32_t* s_written = reinterpret_cast<uint32_t*>(s_ready + 1);
+  uint64_t* mma_drain = s_ready + 1;     // all of this CTA's MMAs are complete
+  uint32_t* s_written = reinterpret_cast<uint32_t*>(mma_drain + 1);
   uint32_t* tmem_slot = s_written + 1;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -94,6 +95,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     for (int s = 0; s < L::kGate; ++s) mbar_init(&gate[s], 1);
     mbar_init(mma_done, 1);
     mbar_init(s_ready, L::kEpiWarps * 32);
+    mbar_init(mma_drain, 1);
     *s_written = 0;
     *abort_flag = 0;
     fence_mbar_init();
@@ -125,6 +127,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       // of frame t-Rs must have loaded S_{t-Rs} from the slot S_t will use. Gate slot
       // t % kGate was last used by frame t - kGate, whose B copy the epilogue issued at step
       // t - kGate - 2, before the MMA of step t - 2 that the empty-stage wait below follows.
+      StageFills<L::kStages> fills;
       for (int t = 0; t < T; ++t) {
         const int stage = t % L::kStages;
         const uint32_t phase = (t / L::kStages) & 1;
@@ -149,7 +152,9 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
 #pragma unroll
         for (int kb = 0; kb < DP / 64; ++kb)
           tma_load_3d(st + kb * DP * 128, tm_a, &full[stage], kb * 64, 0, row, pol);
+        fills.filled(stage, phase);
       }
+      fills.drain(full);  // this thread's copies have landed, whatever the exit path
     }
   } else if (warp == L::kWarpMma) {
     // ---------------------------------------------------------------- MMA: P = S_{t-1} A_t
@@ -180,6 +185,10 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       __syncwarp();
     }
     if (!ok) give_up(hf, abort_flag);
+    // every MMA issued here has completed before TMEM is released
+    if (elect_one()) mma_commit(mma_drain);
+    __syncwarp();
+    mbar_wait(mma_drain, 0);
   } else if (warp == L::kWarpPublisher) {
     // ---------------------------------------------------------------- fused: publish S_t
     if constexpr (kFused) {
@@ -197,7 +206,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
             t0 = globaltimer_ns();
             continue;
           }
-          if (*abort_flag || ld_acquire(hf.abort) != 0 || globaltimer_ns() - t0 > kWaitLimitNs) {
+          if (*abort_flag || ld_acquire(hf.abort) != 0 || globaltimer_ns() - t0 > g_wait_limit_ns) {
             give_up(hf, abort_flag);
             break;
           }
@@ -354,7 +363,7 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
                      const float* __restrict__ beta, const float* __restrict__ state_in,
                      float* __restrict__ state_out, Problem p) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
   chain_body<DP, false>(&tm_a, B_ws, S_ws, gamma, beta, state_in, state_out, p, none,
                         align1k(smem_raw));
 }

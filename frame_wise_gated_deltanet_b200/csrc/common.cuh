@@ -33,6 +33,7 @@ struct Handoff {
   int* next_item;   // this role's work counter (stats and output roles take items dynamically)
   int R;            // A_t / B_t ring slots per head (how far the statistics may run ahead)
   int Rs;           // S_t ring slots per head (how far the outputs may lag behind)
+  int withhold;     // test hook: frame whose statistics of head 0 are never published (-1: none)
   int base;         // first blockIdx.x of this role
   int count;        // CTAs in this role
 };

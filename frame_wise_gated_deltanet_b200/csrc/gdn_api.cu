@@ -93,6 +93,8 @@ struct DeviceState {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
+int env_int(const char* name, int dflt, int lo, int hi);
+
 gdn_status current_device(int* dev) {
   if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return GDN_ERR_CUDA;
   DeviceState& d = g_dev[*dev];
@@ -100,6 +102,13 @@ gdn_status current_device(int* dev) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
       return GDN_ERR_CUDA;
+    // GDN_WAIT_LIMIT_MS: limit of the kernels' bounded waits (default 4000 ms)
+    const int ms = env_int("GDN_WAIT_LIMIT_MS", 4000, 1, 60000);
+    if (ms != 4000) {
+      const unsigned long long ns = static_cast<unsigned long long>(ms) * 1000000ull;
+      if (cudaMemcpyToSymbol(gdn::g_wait_limit_ns, &ns, sizeof(ns)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    }
     d.sms = sms;
   }
   return GDN_OK;
@@ -286,6 +295,9 @@ int g_forward_mode = 0;
 //   GDN_FUSED_RING       A_t / B_t ring slots per head (default 24, 4..64)
 //   GDN_FUSED_SRING      S_t ring slots per head (default 32, 8..64)
 //   GDN_FUSED_STATS_PCT  share of the non-chain SMs given to the stats role (default 54, 20..80)
+}  // namespace
+
+namespace {
 int env_int(const char* name, int dflt, int lo, int hi) {
   const char* s = getenv(name);
   if (s == nullptr || *s == 0) return dflt;
@@ -378,7 +390,12 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   int* f = w.flags;
   const long ft = long(bh) * p.T;
   int* abort_word = f + 2 * ft + bh;
-  gdn::Handoff hc{f, f + ft, f + 2 * ft, abort_word, nullptr, kRing, fused_sring(), 0, bh};
+  // GDN_TEST_WITHHOLD_FRAME (tests only): the statistics of this frame of head 0 are computed
+  // but never published, so the chain's wait for them runs out and the call reports
+  // GDN_ERR_TIMEOUT through gdn_sync_status
+  static const int withhold = env_int("GDN_TEST_WITHHOLD_FRAME", -1, -1, 1 << 30);
+  gdn::Handoff hc{f, f + ft, f + 2 * ft, abort_word, nullptr, kRing, fused_sring(), withhold,
+                  0, bh};
   gdn::Handoff hs = hc;
   hs.base = bh;
   hs.count = n_stats;

@@ -84,7 +84,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   uint64_t* s_empty = s_full + 2;
   uint64_t* acc_full = s_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
-  ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 8), acc_empty + 2};  // fused only
+  ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 9), acc_empty + 2};  // fused only
+  uint64_t* mma_drain = acc_empty + 2 + 8;  // all of this CTA's MMAs are complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -121,6 +122,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       mbar_init(&acc_empty[a], 128);
     }
     for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -139,6 +141,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       if constexpr (kLA) tma_prefetch_desc(tm_s);
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_state = policy_evict_last();
+      StageFills<L::kStages> fills;
+      StageFills<2> s_fills;
       int stage = 0;
       uint32_t phase = 0;
       for (int li = 0; !*abort_flag; ++li) {
@@ -174,6 +178,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           bulk_load(s_buf + sb * L::kSBufBytes, S_src + static_cast<long>(srow) * DP * DP,
                     L::kSBufBytes, &s_full[sb], pol_state);
         }
+        s_fills.filled(sb, (li >> 1) & 1);
         for (int tile = 0; tile < n_tiles; ++tile) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
             give_up(hf, abort_flag);
@@ -184,12 +189,16 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           for (int kb = 0; kb < L::kBoxes; ++kb)
             tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
                         kb * 64, it.h, tile * kRowsPerTile, it.bt, pol_stream);
+          fills.filled(stage, phase);
           if (++stage == L::kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      // this thread's copies have landed, whatever the exit path
+      fills.drain(full);
+      s_fills.drain(s_full);
     }
   } else if (warp == 1) {
     constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
@@ -247,6 +256,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       __syncwarp();
     }
     if (!ok) give_up(hf, abort_flag);
+    // every MMA issued here has completed before TMEM is released
+    if (elect_one()) mma_commit(mma_drain);
+    __syncwarp();
+    mbar_wait(mma_drain, 0);
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue
     const uint32_t quarter = warp & 3;
@@ -260,8 +273,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     bool ok = true;
     for (int li = 0; ok; ++li) {
       const long item = consumer_item(li);
-      if (item == -2) ok = false;
-      if (item < 0) break;
+      bool lost = item == -2;
+      if constexpr (kFused) lost = named_bar_any(1, 128, lost);  // uniform across the epilogue
+      if (lost) ok = false;
+      if (lost || item < 0) break;
       const OutputItem it = output_item<kFused>(item, p);
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
@@ -363,7 +378,7 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
                       const __nv_bfloat16* __restrict__ S_src,
                       const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
   output_body<DP, kLA, false>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
                               align1k(smem_raw));
 }

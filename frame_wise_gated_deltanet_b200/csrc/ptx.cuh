@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05 (TMEM
 // allocation, MMA, commit, loads) and the shared-memory matrix descriptors the MMA reads.
 //
-// Every wait here is bounded: a wait that does not complete within kWaitLimitNs of
+// Every wait here is bounded: a wait that does not complete within g_wait_limit_ns of
 // %globaltimer returns false, and the caller records GDN_ERR_TIMEOUT in the device status
 // word and unwinds instead of spinning forever.
 #pragma once
@@ -10,7 +10,8 @@
 
 namespace gdn {
 
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
+// Limit of every bounded wait, in ns of %globaltimer (4 s unless the host lowers it).
+__device__ unsigned long long g_wait_limit_ns = 4000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -74,7 +75,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > g_wait_limit_ns) return false;
   }
 }
 
@@ -106,7 +107,7 @@ __device__ __forceinline__ void fence_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Wait until *p >= target (acquire). Gives up, returning false, after kWaitLimitNs or as soon
+// Wait until *p >= target (acquire). Gives up, returning false, after g_wait_limit_ns or as soon
 // as *abort is non-zero (another CTA gave up first).
 __device__ __forceinline__ bool wait_flag_ge(const int* p, int target, const int* abort) {
   if (ld_acquire(p) >= target) return true;
@@ -114,10 +115,27 @@ __device__ __forceinline__ bool wait_flag_ge(const int* p, int target, const int
   while (true) {
     if (ld_acquire(p) >= target) return true;
     if (ld_acquire(abort) != 0) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > g_wait_limit_ns) return false;
     __nanosleep(64);
   }
 }
+
+// Last phase of each pipeline stage a producer thread filled, so that on any exit path it can
+// wait (bounded) for its own in-flight copies to land before the CTA releases its resources.
+template <int N>
+struct StageFills {
+  uint32_t last[N];
+  __device__ __forceinline__ StageFills() {
+#pragma unroll
+    for (int i = 0; i < N; ++i) last[i] = 0xFFFFFFFFu;
+  }
+  __device__ __forceinline__ void filled(int s, uint32_t phase) { last[s] = phase; }
+  __device__ __forceinline__ void drain(uint64_t* full) {
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (last[i] != 0xFFFFFFFFu) mbar_wait(&full[i], last[i]);
+  }
+};
 
 // ------------------------------------------------------------------ TMA (no multicast)
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

@@ -79,7 +79,8 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
   uint64_t* empty = ready + L::kStages;
   uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 2;
-  ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 8), acc_empty + 2};  // fused only
+  ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 9), acc_empty + 2};  // fused only
+  uint64_t* mma_drain = acc_empty + 2 + 8;  // all of this CTA's MMAs are complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -113,6 +114,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       mbar_init(&acc_empty[a], 128);
     }
     for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -131,6 +133,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       tma_prefetch_desc(tm_k);
       tma_prefetch_desc(tm_v);
       const uint64_t pol = policy_evict_first();
+      StageFills<L::kStages> fills;
       int stage = 0;
       uint32_t phase = 0;
       for (int li = 0; !*abort_flag; ++li) {
@@ -151,12 +154,14 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
             tma_load_4d(st + L::kOpBytes + j * kBoxBytes, tm_v, &full[stage], j * 64, it.h,
                         tile * kRowsPerTile, it.bt, pol);
           }
+          fills.filled(stage, phase);
           if (++stage == L::kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      fills.drain(full);  // this thread's copies have landed, whatever the exit path
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -225,6 +230,10 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       if (elect_one()) mma_commit(&acc_full[acc]);
       __syncwarp();
     }
+    // every MMA issued here has completed before TMEM is released
+    if (elect_one()) mma_commit(mma_drain);
+    __syncwarp();
+    mbar_wait(mma_drain, 0);
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue
     const uint32_t quarter = warp & 3;
@@ -236,7 +245,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     const int brows = kLA ? D + 1 : D;
     for (int li = 0;; ++li) {
       const long item = consumer_item(li);
-      if (item == -2) {
+      bool lost = item == -2;
+      if constexpr (kFused) lost = named_bar_any(1, 128, lost);  // uniform across the epilogue
+      if (lost) {
         give_up(hf, abort_flag);
         break;
       }
@@ -326,7 +337,8 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
         fence_async_global();
         __threadfence();
         named_bar(1, 128);
-        if (leader) st_release(hf.stats_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
+        if (leader && !(it.bh == 0 && it.t == hf.withhold))
+          st_release(hf.stats_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
       }
     }
   } else if constexpr (kLA) {
@@ -389,7 +401,7 @@ __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
                      float* __restrict__ B_ws, Problem p) {
   extern __shared__ uint8_t smem_raw[];
-  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, 0, 0};
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
   stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw));
 }
 

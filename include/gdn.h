@@ -35,6 +35,15 @@
  *    is being captured) and is shared by all calls on that GPU: calls on different streams of
  *    the same GPU must not run concurrently. gdn_release_workspace() frees it.
  *  - No CPU fallback exists: without a CUDA device every call returns GDN_ERR_CUDA.
+ *
+ * Environment (read once per process):
+ *  - GDN_WAIT_LIMIT_MS: limit of every device-side bounded wait (default 4000).
+ *  - GDN_FUSED_RING, GDN_FUSED_SRING, GDN_FUSED_STATS_PCT: ring depths of the fused forward's
+ *    A_t/B_t and S_t hand-off (default 24 and 32 frames per head) and the share of the non-chain
+ *    SMs given to the statistics role (default 54 %).
+ *  - GDN_TEST_WITHHOLD_FRAME: test hook only. The fused forward computes but never publishes the
+ *    statistics of this frame of head 0, so the call ends with GDN_ERR_TIMEOUT (after the wait
+ *    limit) instead of a result; used to test failure detection without faulting the GPU.
  */
 #ifndef GDN_H_
 #define GDN_H_
