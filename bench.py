@@ -67,10 +67,12 @@ def peaks():
 
 
 def algorithmic_bytes(w):
-    """Bytes the layer must move per clip: Q, K, V read and O written (bf16), gamma and beta,
-    and the fp32 state written (S_0 = 0 is not read)."""
+    """Bytes the layer must move per call: Q, K, V read and O written (bf16), gamma and beta,
+    the fp32 state written, and read when the call starts from a carried state."""
     fh = w.B * w.H * w.T
-    return fh * (4 * w.N * w.D * 2) + w.B * w.T * w.H * 2 * 4 + w.B * w.H * w.D * w.D * 4
+    state = w.B * w.H * w.D * w.D * 4
+    return (fh * (4 * w.N * w.D * 2) + w.B * w.T * w.H * 2 * 4 + state
+            + (state if w.kind == "stream" else 0))
 
 
 def kernel_bytes(name, w):
@@ -85,7 +87,7 @@ def kernel_bytes(name, w):
         return fh * (dd * 2 + dd * 4 + dd * 2 + 8) + w.B * w.H * dd * 4
     if name == "gdn_output_kernel":      # read Q, S_t; write O
         return fh * (2 * nd2 + dd * 2)
-    if name == "gdn_fused_kernel":       # the whole path in one launch
+    if name in ("gdn_fused_kernel", "gdn_step_kernel"):  # the whole path in one launch
         return algorithmic_bytes(w)
     return None
 
@@ -247,7 +249,8 @@ def run_reference(a, w):
 
 
 def workload_config(w):
-    return {"workload": f"{w.name} GDN clip: B{w.B} H{w.H} D{w.D} T{w.T} N{w.N} ({w.grid} grid)",
+    what = "streaming step" if w.kind == "stream" else "GDN clip"
+    return {"workload": f"{w.name} {what}: B{w.B} H{w.H} D{w.D} T{w.T} N{w.N} ({w.grid} grid)",
             "B": w.B, "H": w.H, "D": w.D, "T": w.T, "N": w.N, "key_scale": w.key_scale,
             "gamma_range": list(w.gamma_range), "beta_range": list(w.beta_range),
             "l2": "inputs (%.1f GB of q,k,v) larger than the 126 MB L2; no flush"
@@ -272,14 +275,27 @@ def main():
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    g = gdn_inputs.workload_inputs(w, device=dev)
-    q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
-    out = torch.empty_like(q)
-    st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    if w.kind == "stream":
+        # one streaming step per bench step: a new frame for every stream, state in place
+        g = gdn_inputs.workload_inputs(w, device=dev, step=0)
+        q, k, v = (g[n][:, 0].contiguous() for n in ("q", "k", "v"))
+        gam, bet = g["gamma"][:, 0].contiguous(), g["beta"][:, 0].contiguous()
+        st = gdn_inputs.workload_inputs(w, device=dev)["state"].contiguous()
+        out = torch.empty_like(q)
+        g = {"q": q, "k": k, "v": v, "gamma": gam, "beta": bet}
 
-    def step():
-        api.gdn_frame_forward(q, k, v, gam, bet, None, out, st, key_scale=w.key_scale,
-                              stream=stream)
+        def step():
+            api.gdn_frame_step(q, k, v, gam, bet, st, out, st, key_scale=w.key_scale,
+                               stream=stream)
+    else:
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
+        out = torch.empty_like(q)
+        st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+        def step():
+            api.gdn_frame_forward(q, k, v, gam, bet, None, out, st, key_scale=w.key_scale,
+                                  stream=stream)
 
     for _ in range(max(a.warmup, 3)):
         step()
@@ -337,7 +353,7 @@ def main():
     # ---------------------------------------------------------------- end to end, host buffers
     e2e = None
     if not a.no_e2e:
-        e2e = measure_e2e(a, w, g, out, st, stream, world, dev)
+        e2e = measure_e2e(a, w, g, out, st, stream, world, dev) if w.kind != "stream" else None
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,

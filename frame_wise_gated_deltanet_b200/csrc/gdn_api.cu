@@ -16,6 +16,7 @@
 #include "la_scan_kernel.cuh"
 #include "output_kernel.cuh"
 #include "stats_kernel.cuh"
+#include "step_kernel.cuh"
 
 // Scratch of gdn_frame_forward_noalloc: a fixed 64 MiB array in device memory, reserved by the
 // CUDA module on every GPU that loads this library and held until the process exits. Host code
@@ -463,6 +464,26 @@ gdn_status noalloc_scratch(int dev, void** out) {
   return GDN_OK;
 }
 
+// Fused single-frame step (64 < D <= 128): one persistent launch over (batch, head).
+gdn_status run_step(int dev, const Problem& p, const void* q, const void* k, const void* v,
+                    const float* gamma, const float* beta, const float* s_in, void* out,
+                    float* s_out, cudaStream_t st) {
+  using L = gdn::StepLayout;
+  CUtensorMap tq, tk, tv, to;
+  if (!tmap_tokens(&tq, q, p) || !tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p) ||
+      !tmap_tokens(&to, out, p))
+    return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_step_kernel;
+  if (gdn_status s = ensure_smem_attr(dev, 12, kern, L::kSmemBytes)) return s;
+  const long items = long(p.B) * p.H;
+  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  {
+    ProfiledLaunch pl("gdn_step_kernel", st);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, tk, tv, to, gamma, beta, s_in, s_out, p);
+  }
+  return check_launch();
+}
+
 gdn_status validate_common(const void* q, const void* k, const void* v, const void* out,
                            const float* gamma, const float* beta, const float* s_in,
                            const float* s_out, int B, int H, int T, int N, int D, float ks) {
@@ -535,6 +556,13 @@ gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* 
                                      D, key_scale))
     return s;
   const Problem p{B, H, 1, N, D, key_scale};
+  if (D > 64 && g_forward_mode != 1) {
+    int dev;
+    if (gdn_status s = current_device(&dev)) return s;
+    std::lock_guard<std::mutex> lock(g_mu);
+    return run_step(dev, p, q, k, v, gamma, beta, state_in, out, state_out,
+                    reinterpret_cast<cudaStream_t>(stream));
+  }
   return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
                       reinterpret_cast<cudaStream_t>(stream));
 }

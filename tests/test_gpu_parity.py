@@ -206,6 +206,55 @@ def test_fused_and_split_paths_agree_on_720p():
     assert torch.equal(res[1][0], res[2][0])
 
 
+STEP_SHAPES = [
+    # (B, H, N, D, with_state)
+    (2, 3, 100, 128, True),
+    (1, 2, 257, 112, True),     # padded head dim, ragged tokens
+    (3, 1, 880, 128, False),    # S_0 = 0
+    (2, 2, 16, 72, True),
+]
+
+
+@pytest.mark.parametrize("forward_mode", [1, 0], indirect=True, ids=["split", "fused"])
+@pytest.mark.parametrize("shape", STEP_SHAPES, ids=lambda s: "B%dH%dN%dD%d%s" % (s[:4] + ("s" if s[4] else "",)))
+def test_step_matches_oracle(shape, forward_mode):
+    """gdn_frame_step (fused one-pass kernel for D > 64, or the three kernels), state in place."""
+    B, H, N, D, with_state = shape
+    x = gdn_inputs.clip_inputs(B, H, 1, N, D, seed=500 + N + D, state_std=0.2 if with_state else 0.0)
+    ks = 1.0 / math.sqrt(D * N)
+    q, k, v = (x[n][:, 0].contiguous().cuda() for n in ("q", "k", "v"))
+    gam, bet = x["gamma"][:, 0].contiguous().cuda(), x["beta"][:, 0].contiguous().cuda()
+    state = x["state"].cuda() if with_state else torch.zeros((B, H, D, D), device="cuda")
+    out, st = api().gdn_frame_step(q, k, v, gam, bet, state if with_state else None,
+                                   state_out=state, key_scale=ks)
+    assert api().gdn_sync_status() == 0
+    o_ref, s_ref = oracle.gdn_frame_step(f64(x["q"][:, 0]), f64(x["k"][:, 0]), f64(x["v"][:, 0]),
+                                         f64(x["gamma"][:, 0]), f64(x["beta"][:, 0]),
+                                         f64(x["state"]) if with_state else None, ks)
+    assert relf(f64(out), o_ref) <= O_TOL
+    assert relf(f64(st), s_ref) <= S_TOL
+
+
+def test_step_paths_agree_on_stream_workload():
+    """The fused step and the three-kernel step on the full streaming workload (B16 H20 N880)."""
+    from frame_wise_gated_deltanet_b200 import _lib
+    w = gdn_inputs.WORKLOADS["stream"]
+    x = gdn_inputs.workload_inputs(w, device="cuda", step=0)
+    q, k, v = (x[n][:, 0].contiguous() for n in ("q", "k", "v"))
+    gam, bet = x["gamma"][:, 0].contiguous(), x["beta"][:, 0].contiguous()
+    s0 = gdn_inputs.workload_inputs(w, device="cuda")["state"]
+    res = {}
+    try:
+        for mode in (1, 0):
+            assert _lib.LIB.gdn_set_forward_mode(mode) == 0
+            res[mode] = api().gdn_frame_step(q, k, v, gam, bet, s0, key_scale=w.key_scale)
+            assert api().gdn_sync_status() == 0
+    finally:
+        _lib.LIB.gdn_set_forward_mode(0)
+    assert relf(f64(res[0][0]), f64(res[1][0])) <= 2e-3
+    assert relf(f64(res[0][1]), f64(res[1][1])) <= 1e-5
+
+
 def test_split_resume_on_gpu():
     """forward(T) equals forward(T1) then forward(T - T1) through the carried state."""
     B, H, T, N, D = 1, 2, 9, 150, 128
