@@ -71,6 +71,8 @@ def algorithmic_bytes(w):
     the fp32 state written, and read when the call starts from a carried state."""
     fh = w.B * w.H * w.T
     state = w.B * w.H * w.D * w.D * 4
+    if w.kind == "la":
+        return fh * (4 * w.N * w.D * 2) + state + w.B * w.H * w.D * 4
     return (fh * (4 * w.N * w.D * 2) + w.B * w.T * w.H * 2 * 4 + state
             + (state if w.kind == "stream" else 0))
 
@@ -188,14 +190,22 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Largest value of x over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, ms_local, world, device="cuda"):
+    """Whole-job throughput: every rank processed units_per_rank units; the job took the slowest
+    rank's device time. Returns (units per second, max ms)."""
+    ms = max_over_ranks(ms_local, world, device)
+    return units_per_rank * world / (ms * 1e-3), ms
 
 
 def oracle_sample_rate(w, heads, frames, seed=99):
@@ -249,7 +259,7 @@ def run_reference(a, w):
 
 
 def workload_config(w):
-    what = "streaming step" if w.kind == "stream" else "GDN clip"
+    what = {"stream": "streaming step", "la": "block-causal LA clip"}.get(w.kind, "GDN clip")
     return {"workload": f"{w.name} {what}: B{w.B} H{w.H} D{w.D} T{w.T} N{w.N} ({w.grid} grid)",
             "B": w.B, "H": w.H, "D": w.D, "T": w.T, "N": w.N, "key_scale": w.key_scale,
             "gamma_range": list(w.gamma_range), "beta_range": list(w.beta_range),
@@ -287,6 +297,17 @@ def main():
         def step():
             api.gdn_frame_step(q, k, v, gam, bet, st, out, st, key_scale=w.key_scale,
                                stream=stream)
+    elif w.kind == "la":
+        # block-causal linear attention over the clip
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        q, k, v = g["q"], g["k"], g["v"]
+        out = torch.empty_like(q)
+        st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+        zt = torch.empty((w.B, w.H, w.D), dtype=torch.float32, device=dev)
+
+        def step():
+            api.gdn_block_causal_la(q, k, v, w.frames_per_block, out=out, state_out=st,
+                                    z_out=zt, stream=stream)
     else:
         g = gdn_inputs.workload_inputs(w, device=dev)
         q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
@@ -334,7 +355,7 @@ def main():
         raise RuntimeError(f"device status {status} after the timed region")
 
     ms_local = t_start.elapsed_time(t_end)
-    ms = max_over_ranks(ms_local, world)
+    value, ms = job_throughput(w.tokens_heads * a.steps, ms_local, world)
     per_kernel = {}
     for i, n in enumerate(names):
         d = evs[2 * i].elapsed_time(evs[2 * i + 1])
@@ -345,15 +366,13 @@ def main():
     hbm, peak_kind = peaks()
     kb = kernel_bytes(dom, w)
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
-    units = w.tokens_heads * world * a.steps
-    value = units / (ms * 1e-3)
     path_bytes = algorithmic_bytes(w)
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
 
     # ---------------------------------------------------------------- end to end, host buffers
     e2e = None
     if not a.no_e2e:
-        e2e = measure_e2e(a, w, g, out, st, stream, world, dev) if w.kind != "stream" else None
+        e2e = measure_e2e(a, w, g, out, st, stream, world, dev) if w.kind == "gdn" else None
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -375,7 +394,7 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn":
         rate, secs, threads = oracle_sample_rate(w, 4, w.T)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"4 heads x {w.T} frames of the {w.name} clip shape "
