@@ -214,7 +214,8 @@ gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, vo
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
   {
     ProfiledLaunch pl("gdn_stats_kernel", st);
-    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, static_cast<__nv_bfloat16*>(A), Bm, p);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, static_cast<__nv_bfloat16*>(A), Bm, p,
+                                                   1);
   }
   return check_launch();
 }
@@ -241,7 +242,7 @@ template <int DP, bool kLA>
 gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws, int srows,
                       void* out, int F, cudaStream_t st) {
   using L = gdn::OutputLayout<DP, kLA>;
-  const long count = long(p.B) * p.H * p.T;
+  const long count = long(p.B) * p.H * ((p.T + F - 1) / F);  // stored states (per block for LA)
   CUtensorMap tq, ts, to;
   if (!tmap_tokens(&tq, q, p) || !tmap_tokens(&to, out, p)) return GDN_ERR_CUDA;
   if (kLA) {
@@ -600,7 +601,9 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
   std::lock_guard<std::mutex> lock(g_mu);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Problem p{B, H, T, N, D, 1.0f};
-  const long count = long(B) * H * T;
+  const int F = frames_per_block < T ? frames_per_block : T;
+  const int n_blocks = (T + F - 1) / F;
+  const long count = long(B) * H * n_blocks;
   const size_t per = size_t(D + 1) * D;
   void* base = nullptr;
   if (gdn_status s = get_workspace(dev, align256(count * per * 4) + align256(count * per * 2),
@@ -609,6 +612,7 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
   float* Bws = static_cast<float*>(base);
   void* Sws = static_cast<uint8_t*>(base) + align256(count * per * 4);
   {
+    // per-block statistics: one item per (batch, block, head)
     using L = gdn::StatsLayout<128, true>;
     CUtensorMap tk, tv;
     if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
@@ -616,18 +620,17 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
     if (gdn_status s = ensure_smem_attr(dev, 7, kern, L::kSmemBytes)) return s;
     const int grid = static_cast<int>(count < g_dev[dev].sms ? count : g_dev[dev].sms);
     ProfiledLaunch pl("gdn_stats_kernel_la", st);
-    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, nullptr, Bws, p);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, nullptr, Bws, p, F);
     if (gdn_status s = check_launch()) return s;
   }
   {
     dim3 grid(static_cast<unsigned>((per + 255) / 256), static_cast<unsigned>(B * H));
     ProfiledLaunch pl("gdn_la_scan_kernel", st);
     gdn::gdn_la_scan_kernel<<<grid, 256, 0, st>>>(Bws, static_cast<__nv_bfloat16*>(Sws), state_in,
-                                                  z_in, state_out, z_out, H, T, D,
-                                                  frames_per_block);
+                                                  z_in, state_out, z_out, n_blocks, D);
     if (gdn_status s = check_launch()) return s;
   }
-  return run_output<128, true>(dev, p, q, Sws, D + 1, out, frames_per_block, st);
+  return run_output<128, true>(dev, p, q, Sws, D + 1, out, F, st);
 }
 
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {
@@ -640,6 +643,7 @@ size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {
 
 size_t gdn_la_workspace_bytes(int B, int H, int T, int D) {
   if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
+  // upper bound: one block per frame
   const size_t count = size_t(B) * H * T, per = size_t(D + 1) * D;
   return align256(count * per * 4) + align256(count * per * 2);
 }

@@ -153,8 +153,9 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         if constexpr (kFused) {
           srow = it.bh * hf.Rs + it.t % hf.Rs;
         } else {
-          const int t_state = (F <= 1) ? it.t : min((it.t / F + 1) * F, p.T) - 1;
-          srow = it.bh * p.T + t_state;
+          // GDN: the frame's own state (F = 1); LA: the state after the frame's block
+          const int n_blocks = (p.T + F - 1) / F;
+          srow = it.bh * n_blocks + it.t / F;
         }
         const int sb = li & 1;
         if (!mbar_wait(&s_empty[sb], ((li >> 1) & 1) ^ 1)) {

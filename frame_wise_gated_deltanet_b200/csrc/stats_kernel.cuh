@@ -15,7 +15,8 @@
 //   warps 6..9  (LA only) in-place transform of each K/V stage: relu(K), ones column in V
 //
 // Standalone (gdn_stats_kernel): work item i = (b*T + t)*H + h, results at workspace row
-// (b*H + h)*T + t. Fused (stats role of gdn_fused_kernel): work item i = t*B*H + (b*H + h)
+// (b*H + h)*T + t; for LA an item is a block of frames_per_item frames (its statistics summed),
+// results at row (b*H + h)*n_blocks + block. Fused (stats role of gdn_fused_kernel): work item i = t*B*H + (b*H + h)
 // (frame-major, so the chain finds early frames first), results at ring row (b*H+h)*R + t%R,
 // written only after the chain has released that slot, then published with stats_flag.
 #pragma once
@@ -41,12 +42,17 @@ struct StatsLayout {
 
 struct StatsItem {
   int h, bt, bh, t;
+  int nf;    // frames accumulated into this item (block-causal LA: a block of frames)
   long row;  // workspace / ring row of the results
 };
 
+// fpb: frames per item (1 for GDN; the block length for block-causal LA, whose state only needs
+// each block's sum). Standalone items are (b, block, h) in that order.
 template <bool kFused>
-__device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, const Handoff& hf) {
+__device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, const Handoff& hf,
+                                                int fpb) {
   StatsItem it;
+  it.nf = 1;
   if constexpr (kFused) {
     const int BH = p.B * p.H;
     it.t = static_cast<int>(item / BH);
@@ -56,12 +62,16 @@ __device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, con
     it.bt = b * p.T + it.t;
     it.row = static_cast<long>(it.bh) * hf.R + it.t % hf.R;
   } else {
+    const int nblk = (p.T + fpb - 1) / fpb;
     it.h = static_cast<int>(item % p.H);
-    it.bt = static_cast<int>(item / p.H);
-    const int b = it.bt / p.T;
-    it.t = it.bt - b * p.T;
+    const int bj = static_cast<int>(item / p.H);
+    const int b = bj / nblk;
+    const int j = bj - b * nblk;
+    it.t = j * fpb;
+    it.nf = min(fpb, p.T - it.t);
+    it.bt = b * p.T + it.t;
     it.bh = b * p.H + it.h;
-    it.row = static_cast<long>(it.bh) * p.T + it.t;
+    it.row = static_cast<long>(it.bh) * nblk + j;
   }
   return it;
 }
@@ -72,7 +82,7 @@ template <int DP, bool kLA, bool kFused, bool kB4>
 __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                            __nv_bfloat16* __restrict__ A_ws,
                                            float* __restrict__ B_ws, const Problem& p,
-                                           const Handoff& hf, uint8_t* smem) {
+                                           const Handoff& hf, uint8_t* smem, int fpb = 1) {
   using L = StatsLayout<DP, kLA>;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
   uint64_t* ready = full + L::kStages;   // LA: transformed stage
@@ -86,7 +96,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const long n_items = static_cast<long>(p.B) * p.T * p.H;
+  const long n_items = static_cast<long>(p.B) * ((p.T + fpb - 1) / fpb) * p.H;
   const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
   const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
   const long ncta = kFused ? hf.count : gridDim.x;
@@ -139,8 +149,10 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       for (int li = 0; !*abort_flag; ++li) {
         const long item = producer_item(li);
         if (item < 0) break;
-        const StatsItem it = stats_item<kFused>(item, p, hf);
-        for (int tile = 0; tile < n_tiles; ++tile) {
+        const StatsItem it = stats_item<kFused>(item, p, hf, fpb);
+        for (int ft = 0; ft < it.nf * n_tiles; ++ft) {
+          const int tile = ft % n_tiles;
+          const int bt = it.bt + ft / n_tiles;
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
             give_up(hf, abort_flag);
             break;
@@ -150,9 +162,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
 #pragma unroll
           for (int j = 0; j < L::kBoxes; ++j) {
             tma_load_4d(st + j * kBoxBytes, tm_k, &full[stage], j * 64, it.h,
-                        tile * kRowsPerTile, it.bt, pol);
+                        tile * kRowsPerTile, bt, pol);
             tma_load_4d(st + L::kOpBytes + j * kBoxBytes, tm_v, &full[stage], j * 64, it.h,
-                        tile * kRowsPerTile, it.bt, pol);
+                        tile * kRowsPerTile, bt, pol);
           }
           fills.filled(stage, phase);
           if (++stage == L::kStages) {
@@ -185,8 +197,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       }
       tc_fence_after();
       const uint32_t d = tmem_base + acc * L::kAccCols;
+      const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
       bool ok = true;
-      for (int tile = 0; tile < n_tiles; ++tile) {
+      for (int tile = 0; tile < nf * n_tiles; ++tile) {
         if (!mbar_wait(kLA ? &ready[stage] : &full[stage], phase)) {
           ok = false;
           break;
@@ -254,7 +267,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       if (item < 0) break;
       const int acc = li & 1;
       const uint32_t aph = (li >> 1) & 1;
-      const StatsItem it = stats_item<kFused>(item, p, hf);
+      const StatsItem it = stats_item<kFused>(item, p, hf, fpb);
       bool bad = !mbar_wait(&acc_full[acc], aph);
       if constexpr (kFused) {
         // ring slot t % R of this head is free once the chain has stored S_{t-R}
@@ -350,8 +363,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     for (int li = 0;; ++li) {
       const long item = consumer_item(li);
       if (item < 0) break;
+      const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
       bool ok = true;
-      for (int tile = 0; tile < n_tiles; ++tile) {
+      for (int tile = 0; tile < nf * n_tiles; ++tile) {
         if (!mbar_wait(&full[stage], phase)) {
           ok = false;
           break;
@@ -399,10 +413,11 @@ template <int DP, bool kLA, bool kB4>
 __global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
     gdn_stats_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
-                     float* __restrict__ B_ws, Problem p) {
+                     float* __restrict__ B_ws, Problem p, int frames_per_item) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw));
+  stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw),
+                                  frames_per_item);
 }
 
 }  // namespace gdn
