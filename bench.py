@@ -53,6 +53,8 @@ def args_parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--forward-mode", type=int, default=0,
+                    help="gdn_set_forward_mode: 0 auto, 1 three kernels, 2 fused, 3 chunked")
     return ap.parse_args()
 
 
@@ -87,10 +89,20 @@ def kernel_bytes(name, w):
         return fh * (2 * nd2 + dd * 2 + dd * 4)
     if name == "gdn_chain_kernel":       # read A_t, B_t, gamma, beta; write S_t (bf16), S_T
         return fh * (dd * 2 + dd * 4 + dd * 2 + 8) + w.B * w.H * dd * 4
-    if name == "gdn_output_kernel":      # read Q, S_t; write O
+    if name == "gdn_output_kernel":      # read Q, S_t (per block for LA); write O
+        if w.kind == "la":
+            nblk = -(-w.T // w.frames_per_block)
+            return fh * 2 * nd2 + w.B * w.H * nblk * (w.D + 1) * w.D * 2
         return fh * (2 * nd2 + dd * 2)
     if name in ("gdn_fused_kernel", "gdn_step_kernel"):  # the whole path in one launch
         return algorithmic_bytes(w)
+    if w.kind == "la":
+        nblk = -(-w.T // w.frames_per_block)
+        sums = w.B * w.H * nblk * (w.D + 1) * w.D
+        if name == "gdn_stats_kernel_la":   # read K, V; write the per-block f32 sums
+            return fh * 2 * nd2 + sums * 4
+        if name == "gdn_la_scan_kernel":    # read the sums; write bf16 block states, (S, z)
+            return sums * (4 + 2) + w.B * w.H * (w.D + 1) * w.D * 4
     return None
 
 
@@ -284,6 +296,8 @@ def main():
 
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
+    if _lib.LIB.gdn_set_forward_mode(a.forward_mode) != 0:
+        raise ValueError(f"invalid --forward-mode {a.forward_mode}")
     stream = torch.cuda.current_stream(dev)
     if w.kind == "stream":
         # one streaming step per bench step: a new frame for every stream, state in place

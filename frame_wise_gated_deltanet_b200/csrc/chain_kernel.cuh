@@ -23,7 +23,10 @@
 // gate, 17 TMEM allocator + MMA issuer, 18 publisher (fused only).
 //
 // Standalone (gdn_chain_kernel): A_t, B_t, S_t at workspace row (b*H+h)*T + t; A_t, B_t of
-// later frames are prefetched into L2. Fused (chain role of gdn_fused_kernel, CTA
+// later frames are prefetched into L2. The standalone kernel also runs the two per-chunk jobs of
+// the chunked forward (ChainSeg): the replay of one chunk of frames from its chunk-start state,
+// and the composition of one chunk's affine frame maps (the same recurrence started from the
+// identity without B_t, or from zero with B_t). Fused (chain role of gdn_fused_kernel, CTA
 // base + b*H + h): rows (b*H+h)*R + t%R of the A/B rings and (b*H+h)*Rs + t%Rs of the S ring;
 // frame t is gated on stats_flag (A_t, B_t written) and on out_flag of frame t-Rs (its S slot
 // free), and chain_prog is advanced once every thread's part of S_t is visible.
@@ -33,6 +36,25 @@
 #include "common.cuh"
 
 namespace gdn {
+
+// What one CTA of the standalone chain kernel computes.
+//   kind 0 (replay): frames [c*L, min(T, (c+1)*L)) of head bh = blockIdx.x / nc, chunk
+//     c = blockIdx.x % nc, starting from state_in (c == 0) or from the chunk-start state at row
+//     bh*nc + c of `starts`; writes S_t of every frame and, for the clip's last chunk, state_out.
+//     With L = T and nc = 1 this is the plain per-head chain.
+//   kind 1 (composition): chunk c < nc - 1 of head bh, CTA pair (2*(bh*(nc-1) + c) + role).
+//     Frame t maps a state to S * M_t + C_t with M_t = gamma_t (I - beta_t A_t) and
+//     C_t = beta_t B_t; the same recurrence started from the identity without B_t yields
+//     P_c = M_{cL} ... M_{cL+L-1} (role 0), started from zero with B_t it yields the offset C_c
+//     (role 1), so the chunk's end state is S_start * P_c + C_c. Both go to the chunk's record
+//     in `maps` (layout at chunk_map_bytes).
+struct ChainSeg {
+  int L;
+  int nc;
+  int kind;
+  uint8_t* maps;
+  float* starts;
+};
 
 template <int DP>
 struct ChainLayout {
@@ -60,7 +82,8 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
                                            const float* __restrict__ beta,
                                            const float* __restrict__ state_in,
                                            float* __restrict__ state_out, const Problem& p,
-                                           const Handoff& hf, uint8_t* smem) {
+                                           const Handoff& hf, const ChainSeg& seg,
+                                           uint8_t* smem) {
   using L = ChainLayout<DP>;
   uint8_t* b_buf = smem + L::kStages * L::kABytes;
   uint8_t* s_tile = b_buf + L::kBBufs * L::kBBufBytes;
@@ -78,11 +101,43 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const int bh = kFused ? static_cast<int>(blockIdx.x) - hf.base : static_cast<int>(blockIdx.x);
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
   const int T = p.T;
   const int D = p.D;
+  const long DD = static_cast<long>(D) * D;
+  // this CTA's head, chunk and frames [t0, t1); the pointers it reads and writes are derived
+  // at their point of use (chunk_state) so that nothing extra stays live across the frame loop
+  int bh, chunk = 0, t0 = 0, t1 = T, map_role = -1;
+  if (kFused) {
+    bh = static_cast<int>(blockIdx.x) - hf.base;
+  } else if (seg.kind == 0) {
+    bh = static_cast<int>(blockIdx.x) / seg.nc;
+    chunk = static_cast<int>(blockIdx.x) - bh * seg.nc;
+    t0 = chunk * seg.L;
+    t1 = min(T, t0 + seg.L);
+  } else {
+    const int item = static_cast<int>(blockIdx.x) >> 1;
+    map_role = static_cast<int>(blockIdx.x) & 1;
+    bh = item / (seg.nc - 1);
+    chunk = item - bh * (seg.nc - 1);
+    t0 = chunk * seg.L;
+    t1 = t0 + seg.L;
+  }
+  const bool identity = map_role == 0;  // composition of P_c: start from I, no B_t
+  const bool use_b = map_role != 0;
+  // start state (nullptr: zero) and final state (nullptr: not stored) of this CTA
+  auto init_state = [&]() -> const float* {
+    if (map_role >= 0) return nullptr;  // composition: from I or from zero
+    if (kFused || chunk == 0) return state_in ? state_in + bh * DD : nullptr;
+    return seg.starts + (static_cast<long>(bh) * seg.nc + chunk) * DD;
+  };
+  auto final_state = [&]() -> float* {
+    if (kFused || (map_role < 0 && chunk == seg.nc - 1)) return state_out ? state_out + bh * DD : nullptr;
+    return nullptr;
+  };
+  const int n = t1 - t0;  // frames of this CTA; loop counters below are local (0..n-1)
+  const bool write_s = S_out != nullptr;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
   // row of frame f's A_t / B_t, and of its S_t
   auto row_of = [&](int f) { return kFused ? bh * hf.R + f % hf.R : bh * T + f; };
   auto srow_of = [&](int f) { return kFused ? bh * hf.Rs + f % hf.Rs : bh * T + f; };
@@ -115,24 +170,26 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       tma_prefetch_desc(tm_a);
       const uint64_t pol = kFused ? policy_evict_last() : policy_evict_first();
       constexpr int kPrefetch = 8;  // standalone: frames pulled into L2 ahead of use
-      auto prefetch = [&](int f) {
+      auto prefetch = [&](int f) {  // f: frame index
 #pragma unroll
         for (int kb = 0; kb < DP / 64; ++kb) tma_prefetch_3d(tm_a, kb * 64, 0, row_of(f));
-        bulk_prefetch_l2(B_ws + static_cast<long>(row_of(f)) * D * D,
-                         static_cast<uint32_t>(D * D * 4));
+        if (use_b)
+          bulk_prefetch_l2(B_ws + static_cast<long>(row_of(f)) * D * D,
+                           static_cast<uint32_t>(D * D * 4));
       };
       if constexpr (!kFused)
-        for (int f = 0; f < kPrefetch && f < T; ++f) prefetch(f);
+        for (int u = 0; u < kPrefetch && u < n; ++u) prefetch(t0 + u);
       // Gate frame t, then load A_t. Fused: frame t's A_t, B_t must be published and the output
       // of frame t-Rs must have loaded S_{t-Rs} from the slot S_t will use. Gate slot
       // t % kGate was last used by frame t - kGate, whose B copy the epilogue issued at step
       // t - kGate - 2, before the MMA of step t - 2 that the empty-stage wait below follows.
       StageFills<L::kStages> fills;
-      for (int t = 0; t < T; ++t) {
-        const int stage = t % L::kStages;
-        const uint32_t phase = (t / L::kStages) & 1;
+      for (int u = 0; u < n; ++u) {
+        const int t = t0 + u;
+        const int stage = u % L::kStages;
+        const uint32_t phase = (u / L::kStages) & 1;
         if constexpr (!kFused) {
-          if (t + kPrefetch < T) prefetch(t + kPrefetch);
+          if (u + kPrefetch < n) prefetch(t + kPrefetch);
         }
         bool ok = mbar_wait(&empty[stage], phase ^ 1);
         if constexpr (kFused) {
@@ -145,7 +202,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
           give_up(hf, abort_flag);
           break;
         }
-        mbar_arrive(&gate[t % L::kGate]);
+        mbar_arrive(&gate[u % L::kGate]);
         mbar_arrive_expect_tx(&full[stage], L::kABytes);
         uint8_t* st = smem + stage * L::kABytes;
         const int row = row_of(t);
@@ -161,10 +218,10 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
     const uint32_t s_base = smem_u32(s_tile);
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int stage = t % L::kStages;
-      const uint32_t phase = (t / L::kStages) & 1;
-      if (!mbar_wait(&full[stage], phase) || !mbar_wait(s_ready, t & 1)) {
+    for (int u = 0; u < n; ++u) {
+      const int stage = u % L::kStages;
+      const uint32_t phase = (u / L::kStages) & 1;
+      if (!mbar_wait(&full[stage], phase) || !mbar_wait(s_ready, u & 1)) {
         ok = false;
         break;
       }
@@ -222,11 +279,13 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + c0;
     const bool row_ok = v < D;
     float S[L::kCols];
-    const float* sin = state_in ? state_in + (static_cast<long>(bh) * D + v) * D : nullptr;
+    const float* s0 = init_state();
+    const float* sin = s0 ? s0 + static_cast<long>(v) * D : nullptr;
 #pragma unroll
     for (int j = 0; j < L::kCols; ++j) {
       const int col = c0 + j;
-      S[j] = (sin != nullptr && row_ok && col < D) ? sin[col] : 0.f;
+      const bool in = row_ok && col < D;
+      S[j] = identity ? (in && col == v ? 1.f : 0.f) : ((sin != nullptr && in) ? sin[col] : 0.f);
     }
     auto pack8 = [&](int j) {
       uint4 pk;
@@ -245,11 +304,12 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     auto b_slot = [&](int buf, int kg) {
       return b_buf + buf * L::kBBufBytes + (static_cast<uint32_t>(kg) * 128 + v) * 16;
     };
-    // copy this thread's slice of B_f (from L2) into buffer f % 2, one commit group per frame
+    // copy this thread's slice of B of local frame f (from L2) into buffer f % 2, one commit
+    // group per frame
     auto issue_b = [&](int f) -> bool {
       if (!mbar_wait(&gate[f % L::kGate], (f / L::kGate) & 1)) return false;
-      const float* bm = B_ws + static_cast<long>(row_of(f)) * D * D;
-      if (row_ok) {
+      const float* bm = B_ws + static_cast<long>(row_of(t0 + f)) * D * D;
+      if (row_ok && use_b) {
 #pragma unroll
         for (int j = 0; j < L::kCols; j += 4) {
           const int col = c0 + j;
@@ -264,7 +324,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     tc_fence_before();
     bool ok = issue_b(0);
     if (ok) {
-      if (T > 1)
+      if (n > 1)
         ok = issue_b(1);
       else
         cp_async_commit();
@@ -275,21 +335,22 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     // 32 frames; the value for frame t is shuffled from lane t % 32.
     const long gb_base = static_cast<long>(b) * T * p.H + h;
     auto load_gb = [&](int blk, float& gv, float& bv) {
-      const int f = blk * 32 + static_cast<int>(lane);
-      gv = f < T ? __ldg(gamma + gb_base + static_cast<long>(f) * p.H) : 0.f;
-      bv = f < T ? __ldg(beta + gb_base + static_cast<long>(f) * p.H) : 0.f;
+      const int f = t0 + blk * 32 + static_cast<int>(lane);
+      gv = f < t1 ? __ldg(gamma + gb_base + static_cast<long>(f) * p.H) : 0.f;
+      bv = f < t1 ? __ldg(beta + gb_base + static_cast<long>(f) * p.H) : 0.f;
     };
     float g_cur, b_cur, g_next, b_next;
     load_gb(0, g_next, b_next);
-    for (int t = 0; t < T && ok; ++t) {
-      if ((t & 31) == 0) {
+    for (int u = 0; u < n && ok; ++u) {
+      const int t = t0 + u;
+      if ((u & 31) == 0) {
         g_cur = g_next;
         b_cur = b_next;
-        load_gb((t >> 5) + 1, g_next, b_next);
+        load_gb((u >> 5) + 1, g_next, b_next);
       }
-      const float g = __shfl_sync(0xffffffffu, g_cur, t & 31);
-      const float be = __shfl_sync(0xffffffffu, b_cur, t & 31);
-      if (!mbar_wait(mma_done, t & 1)) {
+      const float g = __shfl_sync(0xffffffffu, g_cur, u & 31);
+      const float be = __shfl_sync(0xffffffffu, b_cur, u & 31);
+      if (!mbar_wait(mma_done, u & 1)) {
         ok = false;
         break;
       }
@@ -304,7 +365,8 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
         for (int j = 0; j < 16; j += 4) {
           const int col = c0 + c + j;
           float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (row_ok && col < D) bv = *reinterpret_cast<const float4*>(b_slot(t & 1, col >> 2));
+          if (use_b && row_ok && col < D)
+            bv = *reinterpret_cast<const float4*>(b_slot(u & 1, col >> 2));
           S[c + j] = fmaf(g, S[c + j], fmaf(be, bv.x, -gbe * P[j]));
           S[c + j + 1] = fmaf(g, S[c + j + 1], fmaf(be, bv.y, -gbe * P[j + 1]));
           S[c + j + 2] = fmaf(g, S[c + j + 2], fmaf(be, bv.z, -gbe * P[j + 2]));
@@ -317,7 +379,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       mbar_arrive(s_ready);
       // S_t to global (its slot was gated free): rows past D and M-padding rows hold zeros,
       // rows >= DP (M-padding when DP == 64) are not part of the stored matrix
-      if (v < DP) {
+      if (write_s && v < DP) {
         uint8_t* srow = reinterpret_cast<uint8_t*>(S_out + static_cast<long>(srow_of(t)) * DP * DP);
 #pragma unroll
         for (int j = 0; j < L::kCols; j += 8)
@@ -327,9 +389,9 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
         __syncwarp();  // the warp's S stores before its lane 0's release-add
         if (lane == 0) red_add_release_cta(s_written, 1);
       }
-      // buffer t % 2 is free (this thread read its own slice above): copy B_{t+2} into it
-      if (t + 2 < T) {
-        if (!issue_b(t + 2)) {
+      // buffer u % 2 is free (this thread read its own slice above): copy B of frame u + 2
+      if (u + 2 < n) {
+        if (!issue_b(u + 2)) {
           ok = false;
           break;
         }
@@ -339,12 +401,37 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     }
     cp_async_wait<0>();
     if (!ok) give_up(hf, abort_flag);
-    if (state_out != nullptr && row_ok) {
-      float* so = state_out + (static_cast<long>(bh) * D + v) * D;
+    float* const s_end = final_state();
+    if (ok && s_end != nullptr && row_ok) {
+      float* so = s_end + static_cast<long>(v) * D;
 #pragma unroll
       for (int j = 0; j < L::kCols; j += 4)
         if (c0 + j < D)
           *reinterpret_cast<float4*>(so + c0 + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+    uint8_t* const map_dst = map_role >= 0 ? seg.maps + (static_cast<long>(bh) * (seg.nc - 1) + chunk) *
+                                                         chunk_map_bytes(DP)
+                                           : nullptr;
+    if (ok && map_role == 0 && v < DP) {
+      // P_c transposed, split into bf16 hi + lo, as the scan's K-major B operand: element
+      // (n, k) = P_c[k][n] at s8_offset_bytes(n, k); this thread holds P_c row k = v
+#pragma unroll
+      for (int j = 0; j < L::kCols; ++j) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(S[j]);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(S[j] - __bfloat162float(hi));
+        const long off = s8_offset_bytes(c0 + j, v, DP);
+        *reinterpret_cast<__nv_bfloat16*>(map_dst + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(map_dst + DP * DP * 2 + off) = lo;
+      }
+    }
+    if (ok && map_role == 1 && row_ok) {
+      // C_c in the four-key interleaved layout of b4_index (read back like B_t)
+      float* cm = reinterpret_cast<float*>(map_dst + 2 * DP * DP * 2);
+#pragma unroll
+      for (int j = 0; j < L::kCols; j += 4)
+        if (c0 + j < D)
+          *reinterpret_cast<float4*>(cm + b4_index(v, c0 + j, D)) =
+              make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
   }
 
@@ -361,10 +448,10 @@ __global__ void __launch_bounds__(ChainLayout<DP>::kThreads, 1)
     gdn_chain_kernel(const __grid_constant__ CUtensorMap tm_a, const float* __restrict__ B_ws,
                      __nv_bfloat16* __restrict__ S_ws, const float* __restrict__ gamma,
                      const float* __restrict__ beta, const float* __restrict__ state_in,
-                     float* __restrict__ state_out, Problem p) {
+                     float* __restrict__ state_out, Problem p, ChainSeg seg) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  chain_body<DP, false>(&tm_a, B_ws, S_ws, gamma, beta, state_in, state_out, p, none,
+  chain_body<DP, false>(&tm_a, B_ws, S_ws, gamma, beta, state_in, state_out, p, none, seg,
                         align1k(smem_raw));
 }
 

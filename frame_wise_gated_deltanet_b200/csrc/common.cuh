@@ -83,6 +83,14 @@ __host__ __device__ __forceinline__ long s8_offset_bytes(int v, int k, int DP) {
   return (static_cast<long>(k >> 3) * DP + v) * 16 + (k & 7) * 2;
 }
 
+// Record of one chunk's composed frame maps in the chunked forward (S_end = S_start * P + C):
+// P transposed as two DP x DP bf16 matrices in the layout of s8_offset_bytes (the bf16 value
+// of P, then the bf16 value of the remainder P - hi), followed by C as D x D f32 in the layout of
+// b4_index. 128 KB at DP = 128.
+__host__ __device__ constexpr long chunk_map_bytes(int DP) {
+  return 2L * DP * DP * 2 + static_cast<long>(DP) * DP * 4;
+}
+
 // TMA box: 64 bf16 (128 B, one swizzle row) x 128 rows.
 constexpr int kRowsPerTile = 128;
 constexpr int kBoxBytes = 128 * 128;  // 16 KB

@@ -46,8 +46,9 @@ __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
   if (static_cast<int>(blockIdx.x) < h_stats.base) {
+    const ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
     chain_body<DP, true>(&tm_a_ring, B_ring, S_ring, gamma, beta, state_in, state_out, p,
-                         h_chain, smem);
+                         h_chain, whole, smem);
   } else if (static_cast<int>(blockIdx.x) < h_out.base) {
     stats_body<DP, false, true, true>(&tm_k, &tm_v, A_ring, B_ring, p, h_stats, smem);
   } else {

@@ -15,6 +15,7 @@
 #include "fused_kernel.cuh"
 #include "la_scan_kernel.cuh"
 #include "output_kernel.cuh"
+#include "scan_kernel.cuh"
 #include "stats_kernel.cuh"
 #include "step_kernel.cuh"
 
@@ -220,20 +221,40 @@ gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, vo
   return check_launch();
 }
 
+// seg.kind 0: one CTA per (head, chunk) replaying the chunk (the plain chain when seg.nc == 1);
+// seg.kind 1: a CTA pair per (head, chunk < nc - 1) composing the chunk's frame maps.
 template <int DP>
 gdn_status run_chain(int dev, const Problem& p, const void* A, const float* Bm,
                      const float* gamma, const float* beta, const float* s_in, void* S_ws,
-                     float* s_out, cudaStream_t st) {
+                     float* s_out, const gdn::ChainSeg& seg, cudaStream_t st) {
   using L = gdn::ChainLayout<DP>;
   const long count = long(p.B) * p.H * p.T;
   CUtensorMap ta;
   if (!tmap_mats(&ta, A, false, p.D, p.D, count, DP)) return GDN_ERR_CUDA;
   auto kern = gdn::gdn_chain_kernel<DP>;
   if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 2 : 3, kern, L::kSmemBytes)) return s;
+  const long bh = long(p.B) * p.H;
+  const long grid = seg.kind == 0 ? bh * seg.nc : 2 * bh * (seg.nc - 1);
+  if (grid < 1 || grid > 2147483647L) return GDN_ERR_INVALID_ARG;
   {
-    ProfiledLaunch pl("gdn_chain_kernel", st);
-    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, Bm, static_cast<__nv_bfloat16*>(S_ws),
-                                                        gamma, beta, s_in, s_out, p);
+    ProfiledLaunch pl(seg.kind == 0 ? (seg.nc == 1 ? "gdn_chain_kernel" : "gdn_chain_kernel_replay")
+                                    : "gdn_chain_kernel_compose",
+                      st);
+    kern<<<static_cast<unsigned>(grid), L::kThreads, L::kSmemBytes, st>>>(
+        ta, Bm, static_cast<__nv_bfloat16*>(S_ws), gamma, beta, s_in, s_out, p, seg);
+  }
+  return check_launch();
+}
+
+template <int DP>
+gdn_status run_scan(int dev, const Problem& p, const gdn::ChainSeg& seg, const float* s_in,
+                    cudaStream_t st) {
+  using L = gdn::ScanLayout<DP>;
+  auto kern = gdn::gdn_scan_kernel<DP>;
+  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 13 : 14, kern, L::kSmemBytes)) return s;
+  {
+    ProfiledLaunch pl("gdn_scan_kernel", st);
+    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(seg.maps, seg.starts, s_in, seg.nc, p.D);
   }
   return check_launch();
 }
@@ -290,7 +311,8 @@ ForwardWs carve_forward(void* base, long count, int D) {
 }
 
 // ------------------------------------------------------------------ fused forward
-// 0 = choose automatically, 1 = always the three-kernel path, 2 = fused whenever it applies.
+// 0 = choose automatically, 1 = always the three-kernel path, 2 = fused whenever it applies,
+// 3 = chunked.
 int g_forward_mode = 0;
 
 // Tuning of the fused forward, read once from the environment:
@@ -422,13 +444,123 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   return check_launch();
 }
 
+// ------------------------------------------------------------------ chunked forward
+// Frames are cut into chunks of L; the chain's serial path shrinks from T frame steps to
+// L (composition) + ceil(T/L) - 1 (scan) + L (replay), at about three times the chain's total
+// work. It pays when few (batch, head) chains run long clips, so that the chain and not HBM
+// bounds the other paths.
+
+// Per-step latencies on B200 used to choose the path and L (microseconds): one chain frame step
+// (D <= 64 / D <= 128), one inter-chunk scan step, and the fill and drain of a chain launch.
+constexpr double kChainStepUs[2] = {1.6, 2.0};
+constexpr double kScanStepUs = 1.5;
+constexpr double kLaunchFillUs = 3.0;
+constexpr double kHbmBytesPerUs = 6.0e6;
+
+struct ChunkPlan {
+  int L = 0;
+  int nc = 1;
+  double us = 0;  // estimated chain-side time (composition + scan + replay)
+};
+
+ChunkPlan plan_chunks(int dev, const Problem& p, int forced_L) {
+  const double tc = kChainStepUs[p.D <= 64 ? 0 : 1];
+  const long bh = long(p.B) * p.H;
+  const int sms = g_dev[dev].sms > 0 ? g_dev[dev].sms : 148;
+  auto waves = [&](long ctas) { return double((ctas + sms - 1) / sms); };
+  auto cost = [&](int L) {
+    const int nc = (p.T + L - 1) / L;
+    double us = waves(bh * nc) * (L * tc + kLaunchFillUs);
+    if (nc > 1)
+      us += waves(2 * bh * (nc - 1)) * (L * tc + kLaunchFillUs) + (nc - 1) * kScanStepUs +
+            kLaunchFillUs;
+    return us;
+  };
+  ChunkPlan best;
+  if (forced_L > 0) {
+    best.L = forced_L < p.T ? forced_L : p.T;
+  } else {
+    best.L = p.T;
+    double c = cost(p.T);
+    for (int L = 4; L < p.T && L <= 256; ++L) {  // gdn_workspace_bytes assumes L >= 4
+      const double x = cost(L);
+      if (x < c) {
+        c = x;
+        best.L = L;
+      }
+    }
+  }
+  best.nc = (p.T + best.L - 1) / best.L;
+  best.us = cost(best.L);
+  return best;
+}
+
+// GDN_CHUNK_LEN: frames per chunk of the chunked forward (0 or unset: chosen per problem)
+int chunk_len_override() { return env_int("GDN_CHUNK_LEN", 0, 0, 1 << 20); }
+
+size_t chunked_ws_bytes(long bh, long T, int D, int nc) {
+  const int dp = padded_dim(D);
+  return forward_ws_bytes(bh * T, D) + align256(size_t(bh) * (nc - 1) * gdn::chunk_map_bytes(dp)) +
+         align256(size_t(bh) * nc * D * D * 4);
+}
+
+// Whether the chunked forward is expected to beat the path chosen otherwise.
+bool chunked_pays(int dev, const Problem& p, bool fused) {
+  if (p.T < 16) return false;
+  const double tc = kChainStepUs[p.D <= 64 ? 0 : 1];
+  const double bh = double(p.B) * p.H;
+  const double io = bh * p.T * (4.0 * p.N * p.D * 2);
+  const double hbm = io / kHbmBytesPerUs;
+  const double plain = p.T * tc + kLaunchFillUs;
+  const double other = fused ? (hbm / 0.8 > plain ? hbm / 0.8 : plain) : hbm / 0.85 + plain;
+  const ChunkPlan c = plan_chunks(dev, p, 0);
+  if (c.nc < 2) return false;
+  // A_t, B_t written once and read twice, S_t written and read once
+  const double ws = bh * p.T * (20.0 * p.D * p.D + 4.0 * padded_dim(p.D) * padded_dim(p.D));
+  const double chunked = hbm / 0.85 + ws / kHbmBytesPerUs + c.us;
+  return chunked < 0.9 * other;
+}
+
+template <int DP>
+gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, const void* v,
+                       const float* gamma, const float* beta, const float* s_in, void* out,
+                       float* s_out, cudaStream_t st) {
+  const ChunkPlan plan = plan_chunks(dev, p, chunk_len_override());
+  const long bh = long(p.B) * p.H;
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, chunked_ws_bytes(bh, p.T, p.D, plan.nc), st, &base))
+    return s;
+  const long count = bh * p.T;
+  ForwardWs w = carve_forward(base, count, p.D);
+  uint8_t* maps = static_cast<uint8_t*>(base) + forward_ws_bytes(count, p.D);
+  float* starts = reinterpret_cast<float*>(
+      maps + align256(size_t(bh) * (plan.nc - 1) * gdn::chunk_map_bytes(DP)));
+  const gdn::ChainSeg compose{plan.L, plan.nc, 1, maps, starts};
+  const gdn::ChainSeg replay{plan.L, plan.nc, 0, maps, starts};
+  if (gdn_status s = run_stats<DP, true>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (plan.nc > 1) {
+    if (gdn_status s = run_chain<DP>(dev, p, w.A, w.B, gamma, beta, nullptr, nullptr, nullptr,
+                                     compose, st))
+      return s;
+    if (gdn_status s = run_scan<DP>(dev, p, compose, s_in, st)) return s;
+  }
+  if (gdn_status s = run_chain<DP>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, replay, st))
+    return s;
+  return run_output<DP, false>(dev, p, q, w.S, p.D, out, 1, st);
+}
+
 gdn_status forward_impl(const void* q, const void* k, const void* v, const float* gamma,
                         const float* beta, const float* s_in, void* out, float* s_out,
                         const Problem& p, cudaStream_t st) {
   int dev;
   if (gdn_status s = current_device(&dev)) return s;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (fused_applies(dev, p)) {
+  const bool fused = fused_applies(dev, p);
+  if (g_forward_mode == 3 || (g_forward_mode == 0 && chunked_pays(dev, p, fused))) {
+    if (p.D <= 64) return run_chunked<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+    return run_chunked<128>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+  }
+  if (fused) {
     if (p.D <= 64) return run_fused<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
     return run_fused<128>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
   }
@@ -436,14 +568,15 @@ gdn_status forward_impl(const void* q, const void* k, const void* v, const float
   void* base = nullptr;
   if (gdn_status s = get_workspace(dev, forward_ws_bytes(count, p.D), st, &base)) return s;
   ForwardWs w = carve_forward(base, count, p.D);
+  const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
   if (p.D <= 64) {
     if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
-    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, st))
+    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
       return s;
     return run_output<64, false>(dev, p, q, w.S, p.D, out, 1, st);
   }
   if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
-  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, st))
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
     return s;
   return run_output<128, false>(dev, p, q, w.S, p.D, out, 1, st);
 }
@@ -537,14 +670,17 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
   const ForwardWs w = carve_forward(base, count, D);
   const Problem p{B, H, T, N, D, key_scale};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const gdn::ChainSeg whole{T, 1, 0, nullptr, nullptr};
   if (D <= 64) {
     if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
-    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out, st))
+    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out,
+                                     whole, st))
       return s;
     return run_output<64, false>(dev, p, q, w.S, D, out, 1, st);
   }
   if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
-  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out, st))
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out,
+                                    whole, st))
     return s;
   return run_output<128, false>(dev, p, q, w.S, D, out, 1, st);
 }
@@ -638,7 +774,12 @@ size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {
   if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
   const size_t split = forward_ws_bytes(long(B) * H * T, D);
   const size_t fused = fused_ws_bytes(long(B) * H, T, D);
-  return split > fused ? split : fused;
+  // chunked: chunks of at least 4 frames unless GDN_CHUNK_LEN asks for shorter ones
+  const int forced = chunk_len_override();
+  const int min_len = forced > 0 && forced < 4 ? forced : 4;
+  const size_t chunked = chunked_ws_bytes(long(B) * H, T, D, (T + min_len - 1) / min_len);
+  size_t m = split > fused ? split : fused;
+  return m > chunked ? m : chunked;
 }
 
 size_t gdn_la_workspace_bytes(int B, int H, int T, int D) {
@@ -705,7 +846,7 @@ gdn_status gdn_profile_arm(void* const* events, int n) {
 int gdn_profile_count(void) { return g_prof_count; }
 
 gdn_status gdn_set_forward_mode(int mode) {
-  if (mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 3) return GDN_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_mu);
   g_forward_mode = mode;
   return GDN_OK;

@@ -78,6 +78,10 @@ WORKLOADS = {
                        seed=2, state_std=0.1, steps=64, grid="22x40"),
     "720p": Workload("720p", "gdn", 1, 20, 128, 961, 880, (0.95, 0.9999), (0.05, 0.95),
                      seed=3, grid="22x40"),
+    # two heads of the 720p clip: the per-GPU slice of the 720p layer split 10 ways by head,
+    # where the per-head state chain rather than HBM bounds the forward
+    "720p_2h": Workload("720p_2h", "gdn", 1, 2, 128, 961, 880, (0.95, 0.9999), (0.05, 0.95),
+                        seed=5, grid="22x40"),
     "la": Workload("la", "la", 2, 20, 112, 81, 390, seed=4, frames_per_block=3,
                    grid="15x26"),
 }

@@ -36,11 +36,13 @@
  *    the same GPU must not run concurrently. gdn_release_workspace() frees it.
  *  - No CPU fallback exists: without a CUDA device every call returns GDN_ERR_CUDA.
  *
- * Environment (read once per process):
+ * Environment (read once per process unless stated):
  *  - GDN_WAIT_LIMIT_MS: limit of every device-side bounded wait (default 4000).
  *  - GDN_FUSED_RING, GDN_FUSED_SRING, GDN_FUSED_STATS_PCT: ring depths of the fused forward's
  *    A_t/B_t and S_t hand-off (default 24 and 32 frames per head) and the share of the non-chain
  *    SMs given to the statistics role (default 54 %).
+ *  - GDN_CHUNK_LEN: frames per chunk of the chunked forward (read on every call; 0 or unset:
+ *    chosen per problem).
  *  - GDN_TEST_WITHHOLD_FRAME: test hook only. The fused forward computes but never publishes the
  *    statistics of this frame of head 0, so the call ends with GDN_ERR_TIMEOUT (after the wait
  *    limit) instead of a result; used to test failure detection without faulting the GPU.
@@ -76,8 +78,9 @@ typedef enum gdn_status {
  * gdn_frame_forward - frame-wise GDN over a whole clip of T frames.
  * Computes out (all T frames) and, if state_out != NULL, S_T.
  * key_scale: the scale applied to keys (1/sqrt(D*N) for the pages' setting); finite, > 0.
- * Workspace: gdn_workspace_bytes(B, H, T, N, D) bytes (three-kernel path: per-frame A_t, B_t,
- * S_t; fused path: per-head rings of A_t, B_t, S_t and hand-off flags).
+ * Workspace: gdn_workspace_bytes(B, H, T, N, D) bytes at most (three-kernel path: per-frame
+ * A_t, B_t, S_t; fused path: per-head rings of A_t, B_t, S_t and hand-off flags; chunked path:
+ * the three-kernel workspace plus per chunk one record of composed maps and one start state).
  */
 gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
                              const float* gamma, const float* beta, const float* state_in,
@@ -98,8 +101,9 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
  *
  * Arguments, layouts and results are exactly those of gdn_frame_forward; the caller still
  * provides q, k, v, gamma, beta, state_in, out and state_out. Limits and behaviour:
- *  - The problem must fit the scratch: gdn_workspace_bytes(B, H, T, N, D) <= 64 MiB (for D = 128
- *    that is B*H*T <= 512 frame-heads). Larger problems return GDN_ERR_SCRATCH_LIMIT before
+ *  - The problem must fit the scratch: the three-kernel workspace (A_t, B_t and S_t of every
+ *    frame-head, 128 KiB each at D = 128) must be at most 64 MiB (for D = 128 that is
+ *    B*H*T <= 512 frame-heads). Larger problems return GDN_ERR_SCRATCH_LIMIT before
  *    anything is launched.
  *  - The first call on each GPU looks up the scratch's device address (with that GPU current) and
  *    caches it; make that first call before any stream capture.
@@ -187,11 +191,18 @@ const char* gdn_profile_kernel(int i);
 
 /*
  * gdn_set_forward_mode - how gdn_frame_forward / gdn_frame_step run (process-wide):
- *   0 (default) automatic: the fused persistent kernel when B*H is at most a third of the SMs
- *     and T >= 4, otherwise three kernels (statistics, state chain, output);
+ *   0 (default) automatic: the chunked forward when an estimate of the per-head state chain's
+ *     latency says it pays (few (batch, head) chains over long clips, T >= 16), else the fused
+ *     persistent kernel when B*H is at most a third of the SMs and T >= 4, else three kernels
+ *     (statistics, state chain, output);
  *   1 always the three kernels;
- *   2 the fused kernel whenever it can run (B*H <= SMs - 8 and cooperative launch available).
- * Both compute the same result. Returns GDN_ERR_INVALID_ARG for other values.
+ *   2 the fused kernel whenever it can run (B*H <= SMs - 8 and cooperative launch available);
+ *   3 always the chunked forward: frames are cut into chunks of L (GDN_CHUNK_LEN, else chosen
+ *     per problem); each chunk's affine frame maps are composed in parallel (S_end = S_start P_c
+ *     + C_c, with P_c the ordered product of gamma_t (I - beta_t A_t) and C_c the accumulated
+ *     offset), one scan per head carries the state across chunks, and every chunk then replays
+ *     its frames from its start state to produce S_t for the outputs.
+ * All compute the same result up to rounding. Returns GDN_ERR_INVALID_ARG for other values.
  */
 gdn_status gdn_set_forward_mode(int mode);
 

@@ -6,6 +6,7 @@ Tolerances: relative Frobenius error of the output <= 1e-2 and of the final stat
 statistics A (stored bf16) <= 5e-3 and B (stored f32) <= 1e-5.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -54,14 +55,23 @@ SHAPES = [
 
 @pytest.fixture
 def forward_mode(request):
-    """Run a test with gdn_set_forward_mode(mode) (1 = three kernels, 2 = fused persistent)."""
+    """Run a test with gdn_set_forward_mode(mode) (1 = three kernels, 2 = fused persistent,
+    3 = chunked with chunks of 3 frames)."""
     from frame_wise_gated_deltanet_b200 import _lib
     assert _lib.LIB.gdn_set_forward_mode(request.param) == 0
-    yield request.param
-    _lib.LIB.gdn_set_forward_mode(0)
+    old = os.environ.get("GDN_CHUNK_LEN")
+    os.environ["GDN_CHUNK_LEN"] = "3"
+    try:
+        yield request.param
+    finally:
+        _lib.LIB.gdn_set_forward_mode(0)
+        if old is None:
+            os.environ.pop("GDN_CHUNK_LEN", None)
+        else:
+            os.environ["GDN_CHUNK_LEN"] = old
 
 
-@pytest.mark.parametrize("forward_mode", [1, 2], indirect=True, ids=["split", "fused"])
+@pytest.mark.parametrize("forward_mode", [1, 2, 3], indirect=True, ids=["split", "fused", "chunked"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B%dH%dT%dN%dD%d%s" % (s[:5] + ("s" if s[5] else "",)))
 def test_forward_matches_oracle(shape, forward_mode):
     B, H, T, N, D, with_state = shape
@@ -173,8 +183,8 @@ def test_stream_workload_sampled():
         assert eo <= O_TOL and es <= S_TOL, f"stream {p}: O err {eo:.2e}, S err {es:.2e}"
 
 
-@pytest.mark.parametrize("forward_mode", [1, 2], indirect=True, ids=["split", "fused"])
-def test_480p_workload_both_paths(forward_mode):
+@pytest.mark.parametrize("forward_mode", [1, 2, 3], indirect=True, ids=["split", "fused", "chunked"])
+def test_480p_workload_all_paths(forward_mode):
     w = gdn_inputs.WORKLOADS["480p"]
     x = gdn_inputs.workload_inputs(w)
     g = to_cuda(x)
@@ -204,6 +214,92 @@ def test_fused_and_split_paths_agree_on_720p():
         _lib.LIB.gdn_set_forward_mode(0)
     assert torch.equal(res[1][1], res[2][1])
     assert torch.equal(res[1][0], res[2][0])
+
+
+# --------------------------------------------------------------------------- chunked forward
+
+
+def _launched(fn):
+    """Names of the library's kernel launches made by fn()."""
+    from frame_wise_gated_deltanet_b200 import _lib
+    import ctypes
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(64)]
+    for e in evs:
+        e.record()  # creates the event
+    handles = (ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs])
+    _lib.LIB.gdn_profile_arm(handles, len(evs))
+    try:
+        fn()
+        torch.cuda.synchronize()
+        return [_lib.LIB.gdn_profile_kernel(i).decode()
+                for i in range(_lib.LIB.gdn_profile_count())]
+    finally:
+        _lib.LIB.gdn_profile_arm(None, 0)
+
+
+@pytest.mark.parametrize("case", [
+    # (B, H, T, N, D, L, with_state)
+    (1, 2, 37, 100, 128, 8, True),    # ragged last chunk (5 frames)
+    (1, 2, 37, 100, 128, 1, True),    # one frame per chunk: 36 scan steps
+    (1, 2, 37, 100, 128, 36, False),  # two chunks, the second of one frame
+    (1, 2, 37, 100, 128, 37, True),   # one chunk: the plain chain
+    (2, 3, 29, 64, 64, 4, True),
+    (1, 1, 50, 17, 8, 7, False),
+    (1, 2, 24, 130, 112, 5, True),
+    (1, 1, 33, 40, 48, 2, True),
+])
+def test_chunked_forward_matches_oracle(case):
+    """Chunked forward (per-chunk composition of the frame maps, inter-chunk scan, per-chunk
+    replay) for several chunk lengths, against the oracle."""
+    from frame_wise_gated_deltanet_b200 import _lib
+    B, H, T, N, D, L, with_state = case
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=700 + L + D, state_std=0.5 if with_state else 0.0)
+    ks = 1.0 / math.sqrt(D * N)
+    g = to_cuda(x)
+    old = os.environ.get("GDN_CHUNK_LEN")
+    os.environ["GDN_CHUNK_LEN"] = str(L)
+    try:
+        assert _lib.LIB.gdn_set_forward_mode(3) == 0
+        res = {}
+        names = _launched(lambda: res.update(r=api().gdn_frame_forward(
+            g["q"], g["k"], g["v"], g["gamma"], g["beta"], g["state"], key_scale=ks)))
+        out, st = res["r"]
+        assert api().gdn_sync_status() == 0
+    finally:
+        _lib.LIB.gdn_set_forward_mode(0)
+        if old is None:
+            os.environ.pop("GDN_CHUNK_LEN", None)
+        else:
+            os.environ["GDN_CHUNK_LEN"] = old
+    if L < T:
+        assert "gdn_scan_kernel" in names and "gdn_chain_kernel_compose" in names, names
+    o_ref, s_ref = oracle.gdn_frame_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["gamma"]),
+                                            f64(x["beta"]),
+                                            None if x["state"] is None else f64(x["state"]), ks)
+    eo, es = relf(f64(out), o_ref), relf(f64(st), s_ref)
+    assert eo <= O_TOL and es <= S_TOL, f"O err {eo:.2e}, S err {es:.2e}"
+
+
+def test_few_heads_long_clip_uses_chunked_path():
+    """Two heads over the 961 frames of the 720p clip (the per-GPU slice of the 720p layer under
+    10-way head sharding): the chain, not HBM, bounds the other paths, so the automatic choice
+    is the chunked forward; the oracle recomputes both heads over all frames."""
+    w = gdn_inputs.WORKLOADS["720p_2h"]
+    x = gdn_inputs.workload_inputs(w, device="cuda")
+    H = w.H
+    res = {}
+    names = _launched(lambda: res.update(r=api().gdn_frame_forward(
+        x["q"], x["k"], x["v"], x["gamma"], x["beta"], None, key_scale=w.key_scale)))
+    out, st = res["r"]
+    assert api().gdn_sync_status() == 0
+    assert "gdn_scan_kernel" in names, names
+    for h in range(H):
+        o_ref, s_ref = oracle.gdn_frame_forward(
+            _head_slice(x["q"], 0, h), _head_slice(x["k"], 0, h), _head_slice(x["v"], 0, h),
+            f64(x["gamma"][:, :, h:h + 1]), f64(x["beta"][:, :, h:h + 1]), None, w.key_scale)
+        eo = relf(_head_slice(out, 0, h), o_ref)
+        es = relf(f64(st[0, h]), s_ref[0, 0])
+        assert eo <= O_TOL and es <= S_TOL, f"head {h}: O err {eo:.2e}, S err {es:.2e}"
 
 
 STEP_SHAPES = [
