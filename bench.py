@@ -50,6 +50,8 @@ def args_parse():
     ap.add_argument("--workload", default="720p")
     ap.add_argument("--frames", type=int, default=0,
                     help="truncate the clip to its first FRAMES frames (small profiling cases)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (scaling studies)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -287,6 +289,8 @@ def main():
     w = gdn_inputs.WORKLOADS[a.workload]
     if a.frames > 0:
         w = dataclasses.replace(w, T=a.frames, name=f"{w.name}[:{a.frames}]")
+    if a.heads > 0:
+        w = dataclasses.replace(w, H=a.heads, name=f"{w.name}[H={a.heads}]")
     if a.impl == "reference":
         run_reference(a, w)
         return

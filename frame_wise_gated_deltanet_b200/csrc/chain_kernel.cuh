@@ -39,8 +39,9 @@ namespace gdn {
 
 // What one CTA of the standalone chain kernel computes.
 //   kind 0 (replay): frames [c*L, min(T, (c+1)*L)) of head bh = blockIdx.x / nc, chunk
-//     c = blockIdx.x % nc, starting from state_in (c == 0) or from the chunk-start state at row
-//     bh*nc + c of `starts`; writes S_t of every frame and, for the clip's last chunk, state_out.
+//     c = blockIdx.x % nc, starting from state_in (c == 0) or from the chunk-start state of
+//     record bh*nc + c in `starts` (layout at chunk_start_bytes, written by the inter-chunk
+//     scan); writes S_t of every frame and, for the clip's last chunk, state_out.
 //     With L = T and nc = 1 this is the plain per-head chain.
 //   kind 1 (composition): chunk c < nc - 1 of head bh, CTA pair (2*(bh*(nc-1) + c) + role).
 //     Frame t maps a state to S * M_t + C_t with M_t = gamma_t (I - beta_t A_t) and
@@ -53,7 +54,7 @@ struct ChainSeg {
   int nc;
   int kind;
   uint8_t* maps;
-  float* starts;
+  uint8_t* starts;
 };
 
 template <int DP>
@@ -125,10 +126,9 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
   const bool identity = map_role == 0;  // composition of P_c: start from I, no B_t
   const bool use_b = map_role != 0;
   // start state (nullptr: zero) and final state (nullptr: not stored) of this CTA
-  auto init_state = [&]() -> const float* {
-    if (map_role >= 0) return nullptr;  // composition: from I or from zero
-    if (kFused || chunk == 0) return state_in ? state_in + bh * DD : nullptr;
-    return seg.starts + (static_cast<long>(bh) * seg.nc + chunk) * DD;
+  auto init_state = [&]() -> const float* {  // row-major f32 start state, nullptr: zero
+    if (map_role >= 0 || (!kFused && chunk > 0)) return nullptr;
+    return state_in ? state_in + bh * DD : nullptr;
   };
   auto final_state = [&]() -> float* {
     if (kFused || (map_role < 0 && chunk == seg.nc - 1)) return state_out ? state_out + bh * DD : nullptr;
@@ -279,13 +279,28 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + c0;
     const bool row_ok = v < D;
     float S[L::kCols];
-    const float* s0 = init_state();
-    const float* sin = s0 ? s0 + static_cast<long>(v) * D : nullptr;
+    if (!kFused && map_role < 0 && chunk > 0) {
+      // chunk-start state from the scan, four-key interleaved (coalesced 16-byte reads)
+      const float* rec = reinterpret_cast<const float*>(
+          seg.starts + (static_cast<long>(bh) * seg.nc + chunk) * chunk_start_bytes(DP));
 #pragma unroll
-    for (int j = 0; j < L::kCols; ++j) {
-      const int col = c0 + j;
-      const bool in = row_ok && col < D;
-      S[j] = identity ? (in && col == v ? 1.f : 0.f) : ((sin != nullptr && in) ? sin[col] : 0.f);
+      for (int j = 0; j < L::kCols; j += 4) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row_ok && c0 + j < D) x = __ldcg(reinterpret_cast<const float4*>(rec + b4_index(v, c0 + j, D)));
+        S[j] = x.x;
+        S[j + 1] = x.y;
+        S[j + 2] = x.z;
+        S[j + 3] = x.w;
+      }
+    } else {
+      const float* s0 = init_state();
+      const float* sin = s0 ? s0 + static_cast<long>(v) * D : nullptr;
+#pragma unroll
+      for (int j = 0; j < L::kCols; ++j) {
+        const int col = c0 + j;
+        const bool in = row_ok && col < D;
+        S[j] = identity ? (in && col == v ? 1.f : 0.f) : ((sin != nullptr && in) ? sin[col] : 0.f);
+      }
     }
     auto pack8 = [&](int j) {
       uint4 pk;

@@ -91,6 +91,11 @@ __host__ __device__ constexpr long chunk_map_bytes(int DP) {
   return 2L * DP * DP * 2 + static_cast<long>(DP) * DP * 4;
 }
 
+// Start state of one chunk in the chunked forward: D x D f32 in the four-key interleaved layout
+// of b4_index (the scan's epilogue warps store and the replay's read 512 contiguous bytes per
+// warp and key group). Sized for DP so records stay 256-byte aligned.
+__host__ __device__ constexpr long chunk_start_bytes(int DP) { return static_cast<long>(DP) * DP * 4; }
+
 // TMA box: 64 bf16 (128 B, one swizzle row) x 128 rows.
 constexpr int kRowsPerTile = 128;
 constexpr int kBoxBytes = 128 * 128;  // 16 KB

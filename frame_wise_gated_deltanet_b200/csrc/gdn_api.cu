@@ -450,12 +450,18 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
 // work. It pays when few (batch, head) chains run long clips, so that the chain and not HBM
 // bounds the other paths.
 
-// Per-step latencies on B200 used to choose the path and L (microseconds): one chain frame step
-// (D <= 64 / D <= 128), one inter-chunk scan step, and the fill and drain of a chain launch.
+// Costs on B200 used to choose the path and L, fitted to measurements on the 720p clip shape
+// with 1..8 heads: one frame step of the standalone and of the fused chain (D <= 64 / D <= 128,
+// microseconds), one inter-chunk scan step, the fill and drain of a launch, the HBM bandwidth
+// the fused kernel and the streaming kernels reach, and the bandwidth the composition and replay
+// launches reach while all their CTAs pull A_t / B_t at once (bytes per microsecond).
 constexpr double kChainStepUs[2] = {1.6, 2.0};
-constexpr double kScanStepUs = 1.5;
-constexpr double kLaunchFillUs = 3.0;
-constexpr double kHbmBytesPerUs = 6.0e6;
+constexpr double kFusedChainStepUs[2] = {1.7, 2.1};
+constexpr double kScanStepUs = 2.8;
+constexpr double kLaunchFillUs = 5.0;
+constexpr double kFusedBytesPerUs = 5.5e6;
+constexpr double kStreamBytesPerUs = 5.77e6;
+constexpr double kChainSideBytesPerUs = 4.5e6;
 
 struct ChunkPlan {
   int L = 0;
@@ -467,13 +473,20 @@ ChunkPlan plan_chunks(int dev, const Problem& p, int forced_L) {
   const double tc = kChainStepUs[p.D <= 64 ? 0 : 1];
   const long bh = long(p.B) * p.H;
   const int sms = g_dev[dev].sms > 0 ? g_dev[dev].sms : 148;
+  const double dd = double(p.D) * p.D, dp2 = double(padded_dim(p.D)) * padded_dim(p.D);
+  // composition reads A_t (P) and A_t, B_t (C); the replay reads A_t, B_t and writes S_t
+  const double compose_floor = bh * p.T * dd * 8.0 / kChainSideBytesPerUs;
+  const double replay_floor = bh * p.T * (dd * 6.0 + dp2 * 2.0) / kChainSideBytesPerUs;
   auto waves = [&](long ctas) { return double((ctas + sms - 1) / sms); };
   auto cost = [&](int L) {
     const int nc = (p.T + L - 1) / L;
-    double us = waves(bh * nc) * (L * tc + kLaunchFillUs);
-    if (nc > 1)
-      us += waves(2 * bh * (nc - 1)) * (L * tc + kLaunchFillUs) + (nc - 1) * kScanStepUs +
-            kLaunchFillUs;
+    const double replay = waves(bh * nc) * L * tc;
+    double us = (replay > replay_floor ? replay : replay_floor) + kLaunchFillUs;
+    if (nc > 1) {
+      const double compose = waves(2 * bh * (nc - 1)) * L * tc;
+      us += (compose > compose_floor ? compose : compose_floor) + kLaunchFillUs +
+            (nc - 1) * kScanStepUs + kLaunchFillUs;
+    }
     return us;
   };
   ChunkPlan best;
@@ -501,23 +514,27 @@ int chunk_len_override() { return env_int("GDN_CHUNK_LEN", 0, 0, 1 << 20); }
 size_t chunked_ws_bytes(long bh, long T, int D, int nc) {
   const int dp = padded_dim(D);
   return forward_ws_bytes(bh * T, D) + align256(size_t(bh) * (nc - 1) * gdn::chunk_map_bytes(dp)) +
-         align256(size_t(bh) * nc * D * D * 4);
+         align256(size_t(bh) * nc * gdn::chunk_start_bytes(dp));
 }
 
 // Whether the chunked forward is expected to beat the path chosen otherwise.
 bool chunked_pays(int dev, const Problem& p, bool fused) {
   if (p.T < 16) return false;
-  const double tc = kChainStepUs[p.D <= 64 ? 0 : 1];
+  const int dx = p.D <= 64 ? 0 : 1;
   const double bh = double(p.B) * p.H;
-  const double io = bh * p.T * (4.0 * p.N * p.D * 2);
-  const double hbm = io / kHbmBytesPerUs;
-  const double plain = p.T * tc + kLaunchFillUs;
-  const double other = fused ? (hbm / 0.8 > plain ? hbm / 0.8 : plain) : hbm / 0.85 + plain;
+  const double dp2 = double(padded_dim(p.D)) * padded_dim(p.D);
+  const double io = bh * p.T * (4.0 * p.N * p.D * 2);          // Q, K, V read, O written
+  const double ws = bh * p.T * (6.0 * p.D * p.D + 2.0 * dp2);  // A_t, B_t written, S_t read
+  double other;
+  if (fused) {
+    const double hbm = io / kFusedBytesPerUs, chain = p.T * kFusedChainStepUs[dx] + kLaunchFillUs;
+    other = hbm > chain ? hbm : chain;
+  } else {
+    other = (io + ws) / kStreamBytesPerUs + p.T * kChainStepUs[dx] + 3 * kLaunchFillUs;
+  }
   const ChunkPlan c = plan_chunks(dev, p, 0);
   if (c.nc < 2) return false;
-  // A_t, B_t written once and read twice, S_t written and read once
-  const double ws = bh * p.T * (20.0 * p.D * p.D + 4.0 * padded_dim(p.D) * padded_dim(p.D));
-  const double chunked = hbm / 0.85 + ws / kHbmBytesPerUs + c.us;
+  const double chunked = (io + ws) / kStreamBytesPerUs + c.us;
   return chunked < 0.9 * other;
 }
 
@@ -533,8 +550,7 @@ gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, 
   const long count = bh * p.T;
   ForwardWs w = carve_forward(base, count, p.D);
   uint8_t* maps = static_cast<uint8_t*>(base) + forward_ws_bytes(count, p.D);
-  float* starts = reinterpret_cast<float*>(
-      maps + align256(size_t(bh) * (plan.nc - 1) * gdn::chunk_map_bytes(DP)));
+  uint8_t* starts = maps + align256(size_t(bh) * (plan.nc - 1) * gdn::chunk_map_bytes(DP));
   const gdn::ChainSeg compose{plan.L, plan.nc, 1, maps, starts};
   const gdn::ChainSeg replay{plan.L, plan.nc, 0, maps, starts};
   if (gdn_status s = run_stats<DP, true>(dev, p, k, v, w.A, w.B, st)) return s;

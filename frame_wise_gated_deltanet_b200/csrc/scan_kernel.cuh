@@ -9,6 +9,11 @@
 // splits of both factors, S_hi P_hi + S_hi P_lo + S_lo P_hi, accumulated in f32 in TMEM. The
 // dropped S_lo P_lo term is about 2^-16 of the product. S itself stays f32 in registers.
 //
+// The epilogue stores every chunk-start state in the four-key interleaved layout (512 contiguous
+// bytes per warp and store). Row-major stores (128 bytes per lane, lanes a row apart) doubled
+// the step time, and a bulk copy of the shared-memory operand tiles by the MMA thread was slower
+// than these coalesced stores.
+//
 // Warps: 0..15 epilogue (thread = row v of S, DP/4 columns), 16 bulk-copy producer of the P_c
 // records (two stages), 17 TMEM allocator + MMA issuer.
 #pragma once
@@ -30,11 +35,11 @@ struct ScanLayout {
   static constexpr int kSmemBytes = kStages * kPBytes + 2 * kSBytes + 256 + 1024;
 };
 
-// maps: nc - 1 records per head (chunk_map_bytes(DP) each); starts: nc D x D f32 matrices per
-// head, row-major (row v, column k); row bh*nc + c receives the start state of chunk c >= 1.
+// maps: nc - 1 records per head (chunk_map_bytes(DP) each); starts: nc records per head
+// (chunk_start_bytes(DP) each); record bh*nc + c receives the start state of chunk c >= 1.
 template <int DP>
 __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
-    gdn_scan_kernel(const uint8_t* __restrict__ maps, float* __restrict__ starts,
+    gdn_scan_kernel(const uint8_t* __restrict__ maps, uint8_t* __restrict__ starts,
                     const float* __restrict__ state_in, int nc, int D) {
   using L = ScanLayout<DP>;
   extern __shared__ uint8_t smem_raw[];
@@ -208,6 +213,7 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) S[cc + j] = P[j] + C[cc + j];
       }
+
       if (c + 1 < steps) {
         write_tiles();
         fence_async_smem();
@@ -216,11 +222,13 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
       }
       // start state of chunk c + 1
       if (row_ok) {
-        float* so = starts + (static_cast<long>(bh) * nc + c + 1) * DD + static_cast<long>(v) * D;
+        float* so = reinterpret_cast<float*>(
+            starts + (static_cast<long>(bh) * nc + c + 1) * chunk_start_bytes(DP));
 #pragma unroll
         for (int j = 0; j < L::kCols; j += 4)
           if (c0 + j < D)
-            *reinterpret_cast<float4*>(so + c0 + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            __stcg(reinterpret_cast<float4*>(so + b4_index(v, c0 + j, D)),
+                   make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
       }
     }
     if (!ok) give_up(none, abort_flag);
