@@ -29,6 +29,7 @@ _F = ctypes.c_float
 SIGNATURES = {
     "gdn_frame_forward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "gdn_frame_forward_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_stats": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_block_causal_la": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),

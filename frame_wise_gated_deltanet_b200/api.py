@@ -12,7 +12,7 @@ import torch
 
 from ._lib import LIB, GdnError, check
 
-__all__ = ["gdn_frame_forward", "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
+__all__ = ["gdn_frame_forward", "gdn_frame_forward_host", "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
            "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
            "gdn_la_workspace_bytes", "GdnError"]
 
@@ -64,6 +64,50 @@ def gdn_frame_forward(q, k, v, gamma, beta, state_in=None, out=None, state_out=N
         check("gdn_frame_forward", LIB.gdn_frame_forward(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
             _ptr(state_out), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
+    return out, state_out
+
+
+def _req_host(t: torch.Tensor, name: str, dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gdn_frame_forward_host(q, k, v, gamma, beta, state_in=None, out=None, state_out=None,
+                           key_scale: Optional[float] = None, stream=None, device=None,
+                           want_state: bool = True):
+    """gdn_frame_forward on HOST tensors (pinned for overlap), streamed through the GPU in
+    segments of frames. Asynchronous on ``stream`` of ``device`` (default: the current CUDA
+    device): synchronise it before reading out / state_out. Returns (out, state_out); missing
+    outputs are allocated as pinned host tensors."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req_host(t, name, torch.bfloat16, (B, T, N, H, D))
+    _req_host(gamma, "gamma", torch.float32, (B, T, H))
+    _req_host(beta, "beta", torch.float32, (B, T, H))
+    if state_in is not None:
+        _req_host(state_in, "state_in", torch.float32, (B, H, D, D))
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    _req_host(out, "out", torch.bfloat16, (B, T, N, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, pin_memory=True)
+    if state_out is not None:
+        _req_host(state_out, "state_out", torch.float32, (B, H, D, D))
+    if key_scale is None:
+        key_scale = 1.0 / math.sqrt(D * N)
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        check("gdn_frame_forward_host", LIB.gdn_frame_forward_host(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
+            _ptr(state_out), B, H, T, N, D, float(key_scale), _stream(stream, device)))
     return out, state_out
 
 

@@ -39,9 +39,10 @@ namespace gdn {
 
 // What one CTA of the standalone chain kernel computes.
 //   kind 0 (replay): frames [c*L, min(T, (c+1)*L)) of head bh = blockIdx.x / nc, chunk
-//     c = blockIdx.x % nc, starting from state_in (c == 0) or from the chunk-start state of
+//     c = blockIdx.x % nc, starting from state_in (nc == 1) or from the chunk-start state of
 //     record bh*nc + c in `starts` (layout at chunk_start_bytes, written by the inter-chunk
-//     scan); writes S_t of every frame and, for the clip's last chunk, state_out.
+//     scan; record 0 is the scan's copy of state_in); writes S_t of every frame and, for the
+//     clip's last chunk, state_out.
 //     With L = T and nc = 1 this is the plain per-head chain.
 //   kind 1 (composition): chunk c < nc - 1 of head bh, CTA pair (2*(bh*(nc-1) + c) + role).
 //     Frame t maps a state to S * M_t + C_t with M_t = gamma_t (I - beta_t A_t) and
@@ -126,8 +127,10 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
   const bool identity = map_role == 0;  // composition of P_c: start from I, no B_t
   const bool use_b = map_role != 0;
   // start state (nullptr: zero) and final state (nullptr: not stored) of this CTA
+  // start state from the scan's records (chunked replay) instead of state_in
+  const bool start_from_record = !kFused && map_role < 0 && seg.nc > 1;
   auto init_state = [&]() -> const float* {  // row-major f32 start state, nullptr: zero
-    if (map_role >= 0 || (!kFused && chunk > 0)) return nullptr;
+    if (map_role >= 0 || start_from_record) return nullptr;
     return state_in ? state_in + bh * DD : nullptr;
   };
   auto final_state = [&]() -> float* {
@@ -279,7 +282,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + c0;
     const bool row_ok = v < D;
     float S[L::kCols];
-    if (!kFused && map_role < 0 && chunk > 0) {
+    if (start_from_record) {
       // chunk-start state from the scan, four-key interleaved (coalesced 16-byte reads)
       const float* rec = reinterpret_cast<const float*>(
           seg.starts + (static_cast<long>(bh) * seg.nc + chunk) * chunk_start_bytes(DP));

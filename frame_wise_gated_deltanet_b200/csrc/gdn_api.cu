@@ -649,6 +649,154 @@ gdn_status validate_common(const void* q, const void* k, const void* v, const vo
   return GDN_OK;
 }
 
+
+// ------------------------------------------------------------------ host-resident clips
+// gdn_frame_forward_host streams a clip held in host memory through the GPU in segments of
+// frames: segment i's inputs are copied in on a copy-in stream while segment i-1 is computed on
+// the caller's stream and segment i-2's output is copied out on a copy-out stream (two staging
+// buffers, ordered by events). The state is carried on the device from segment to segment, so
+// the frame recurrence is split exactly as a resumed clip.
+struct HostPipe {
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t entry, in_done[2], comp_done[2], out_done[2], fin;
+  void* buf = nullptr;
+  size_t bytes = 0;
+  bool ready = false;
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;
+
+gdn_status pipe_init(int dev, HostPipe& hp) {
+  if (hp.ready) return GDN_OK;
+  if (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  cudaEvent_t* evs[] = {&hp.entry, &hp.in_done[0], &hp.in_done[1], &hp.comp_done[0],
+                        &hp.comp_done[1], &hp.out_done[0], &hp.out_done[1], &hp.fin};
+  for (cudaEvent_t* e : evs)
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
+  (void)dev;
+  hp.ready = true;
+  return GDN_OK;
+}
+
+// Frames per segment: GDN_HOST_SEGMENT_FRAMES, else about 256 MB of q/k/v per segment.
+int host_segment_frames(const Problem& p) {
+  const int forced = env_int("GDN_HOST_SEGMENT_FRAMES", 0, 0, 1 << 30);
+  if (forced > 0) return forced < p.T ? forced : p.T;
+  const double per_frame = 3.0 * p.B * p.N * p.H * p.D * 2;
+  int f = static_cast<int>((256.0 * (1 << 20)) / per_frame);
+  if (f < 1) f = 1;
+  return f < p.T ? f : p.T;
+}
+
+struct SegBufs {
+  uint8_t *q, *k, *v, *out;
+  float *g, *b;
+};
+
+gdn_status forward_host_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const float* gamma, const float* beta, const float* s_in,
+                             uint16_t* out, float* s_out, const Problem& p, cudaStream_t st) {
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (gdn_status s = pipe_init(dev, hp)) return s;
+  const int F = host_segment_frames(p);
+  const size_t tok = size_t(p.N) * p.H * p.D;            // elements of one frame of one batch
+  const size_t seg_tok = align256(size_t(p.B) * F * tok * 2);
+  const size_t seg_gb = align256(size_t(p.B) * F * p.H * 4);
+  const size_t per_buf = 4 * seg_tok + 2 * seg_gb;
+  const size_t state_bytes = align256(size_t(p.B) * p.H * p.D * p.D * 4);
+  const size_t need = 2 * per_buf + state_bytes;
+  if (hp.bytes < need) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return GDN_ERR_NO_MEMORY;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    if (hp.buf) cudaFree(hp.buf);
+    hp.buf = nullptr;
+    hp.bytes = 0;
+    if (cudaMalloc(&hp.buf, need) != cudaSuccess) {
+      cudaGetLastError();
+      return GDN_ERR_NO_MEMORY;
+    }
+    hp.bytes = need;
+  }
+  uint8_t* base = static_cast<uint8_t*>(hp.buf);
+  SegBufs sb[2];
+  for (int i = 0; i < 2; ++i) {
+    uint8_t* b0 = base + i * per_buf;
+    sb[i].q = b0;
+    sb[i].k = b0 + seg_tok;
+    sb[i].v = b0 + 2 * seg_tok;
+    sb[i].out = b0 + 3 * seg_tok;
+    sb[i].g = reinterpret_cast<float*>(b0 + 4 * seg_tok);
+    sb[i].b = reinterpret_cast<float*>(b0 + 4 * seg_tok + seg_gb);
+  }
+  float* dstate = reinterpret_cast<float*>(base + 2 * per_buf);
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // everything earlier on the caller's stream (including a previous call's pipeline) first
+  if (!ok(cudaEventRecord(hp.entry, st)) || !ok(cudaStreamWaitEvent(hp.s_in, hp.entry, 0)) ||
+      !ok(cudaStreamWaitEvent(hp.s_out, hp.entry, 0)))
+    return GDN_ERR_CUDA;
+  if (s_in != nullptr &&
+      !ok(cudaMemcpyAsync(dstate, s_in, size_t(p.B) * p.H * p.D * p.D * 4,
+                          cudaMemcpyHostToDevice, st)))
+    return GDN_ERR_CUDA;
+  const int n_seg = (p.T + F - 1) / F;
+  for (int i = 0; i < n_seg; ++i) {
+    const int j = i & 1;
+    const int t0 = i * F;
+    const int f = p.T - t0 < F ? p.T - t0 : F;
+    // copy in (after segment i-2's compute has released buffer j)
+    if (i >= 2 && !ok(cudaStreamWaitEvent(hp.s_in, hp.comp_done[j], 0))) return GDN_ERR_CUDA;
+    for (int b = 0; b < p.B; ++b) {
+      const size_t src = (size_t(b) * p.T + t0) * tok, dst = size_t(b) * f * tok;
+      const size_t n = size_t(f) * tok * 2;
+      if (!ok(cudaMemcpyAsync(sb[j].q + dst * 2, q + src, n, cudaMemcpyHostToDevice, hp.s_in)) ||
+          !ok(cudaMemcpyAsync(sb[j].k + dst * 2, k + src, n, cudaMemcpyHostToDevice, hp.s_in)) ||
+          !ok(cudaMemcpyAsync(sb[j].v + dst * 2, v + src, n, cudaMemcpyHostToDevice, hp.s_in)))
+        return GDN_ERR_CUDA;
+      const size_t gsrc = (size_t(b) * p.T + t0) * p.H, gdst = size_t(b) * f * p.H;
+      const size_t gn = size_t(f) * p.H * 4;
+      if (!ok(cudaMemcpyAsync(sb[j].g + gdst, gamma + gsrc, gn, cudaMemcpyHostToDevice,
+                              hp.s_in)) ||
+          !ok(cudaMemcpyAsync(sb[j].b + gdst, beta + gsrc, gn, cudaMemcpyHostToDevice, hp.s_in)))
+        return GDN_ERR_CUDA;
+    }
+    if (!ok(cudaEventRecord(hp.in_done[j], hp.s_in))) return GDN_ERR_CUDA;
+    // compute (after the copy-in, and after segment i-2's output has left buffer j)
+    if (!ok(cudaStreamWaitEvent(st, hp.in_done[j], 0))) return GDN_ERR_CUDA;
+    if (i >= 2 && !ok(cudaStreamWaitEvent(st, hp.out_done[j], 0))) return GDN_ERR_CUDA;
+    const Problem ps{p.B, p.H, f, p.N, p.D, p.key_scale};
+    const float* sin = (i == 0 && s_in == nullptr) ? nullptr : dstate;
+    if (gdn_status s = forward_impl(sb[j].q, sb[j].k, sb[j].v, sb[j].g, sb[j].b, sin, sb[j].out,
+                                    dstate, ps, st))
+      return s;
+    if (!ok(cudaEventRecord(hp.comp_done[j], st))) return GDN_ERR_CUDA;
+    // copy out
+    if (!ok(cudaStreamWaitEvent(hp.s_out, hp.comp_done[j], 0))) return GDN_ERR_CUDA;
+    for (int b = 0; b < p.B; ++b) {
+      const size_t dst = (size_t(b) * p.T + t0) * tok, src = size_t(b) * f * tok;
+      if (!ok(cudaMemcpyAsync(out + dst, sb[j].out + src * 2, size_t(f) * tok * 2,
+                              cudaMemcpyDeviceToHost, hp.s_out)))
+        return GDN_ERR_CUDA;
+    }
+    if (!ok(cudaEventRecord(hp.out_done[j], hp.s_out))) return GDN_ERR_CUDA;
+  }
+  if (s_out != nullptr &&
+      !ok(cudaMemcpyAsync(s_out, dstate, size_t(p.B) * p.H * p.D * p.D * 4,
+                          cudaMemcpyDeviceToHost, hp.s_out)))
+    return GDN_ERR_CUDA;
+  // the caller's stream completes only after every copy of this call
+  if (!ok(cudaEventRecord(hp.fin, hp.s_out)) || !ok(cudaStreamWaitEvent(st, hp.fin, 0)) ||
+      !ok(cudaStreamWaitEvent(hp.s_in, hp.fin, 0)))
+    return GDN_ERR_CUDA;
+  return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -699,6 +847,21 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
                                     whole, st))
     return s;
   return run_output<128, false>(dev, p, q, w.S, D, out, 1, st);
+}
+
+gdn_status gdn_frame_forward_host(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                  const float* gamma, const float* beta, const float* state_in,
+                                  gdn_bf16* out, float* state_out, int B, int H, int T, int N,
+                                  int D, float key_scale, gdn_stream_t stream) {
+  if (!q || !k || !v || !out || !gamma || !beta) return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  const size_t n = size_t(B) * T * N * H * D * 2;
+  if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
+    return GDN_ERR_INVALID_ARG;
+  const Problem p{B, H, T, N, D, key_scale};
+  return forward_host_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,

@@ -36,7 +36,9 @@ struct ScanLayout {
 };
 
 // maps: nc - 1 records per head (chunk_map_bytes(DP) each); starts: nc records per head
-// (chunk_start_bytes(DP) each); record bh*nc + c receives the start state of chunk c >= 1.
+// (chunk_start_bytes(DP) each); record bh*nc + c receives the start state of chunk c (record 0:
+// a copy of state_in, so that the replays never read state_in while the last one writes
+// state_out, which may be the same memory).
 template <int DP>
 __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
     gdn_scan_kernel(const uint8_t* __restrict__ maps, uint8_t* __restrict__ starts,
@@ -154,6 +156,18 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
 #pragma unroll
     for (int j = 0; j < L::kCols; ++j)
       S[j] = (sin != nullptr && row_ok && c0 + j < D) ? sin[c0 + j] : 0.f;
+    // start state of chunk 0
+    auto store_start = [&](int c) {
+      if (!row_ok) return;
+      float* so = reinterpret_cast<float*>(
+          starts + (static_cast<long>(bh) * nc + c) * chunk_start_bytes(DP));
+#pragma unroll
+      for (int j = 0; j < L::kCols; j += 4)
+        if (c0 + j < D)
+          __stcg(reinterpret_cast<float4*>(so + b4_index(v, c0 + j, D)),
+                 make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+    };
+    store_start(0);
     // S as bf16 hi and lo operand tiles (core-matrix layout, rows past D are zero)
     auto write_tiles = [&]() {
 #pragma unroll
@@ -220,16 +234,7 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(s_ready);
       }
-      // start state of chunk c + 1
-      if (row_ok) {
-        float* so = reinterpret_cast<float*>(
-            starts + (static_cast<long>(bh) * nc + c + 1) * chunk_start_bytes(DP));
-#pragma unroll
-        for (int j = 0; j < L::kCols; j += 4)
-          if (c0 + j < D)
-            __stcg(reinterpret_cast<float4*>(so + b4_index(v, c0 + j, D)),
-                   make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
-      }
+      store_start(c + 1);
     }
     if (!ok) give_up(none, abort_flag);
   }

@@ -43,6 +43,7 @@
  *    SMs given to the statistics role (default 54 %).
  *  - GDN_CHUNK_LEN: frames per chunk of the chunked forward (read on every call; 0 or unset:
  *    chosen per problem).
+ *  - GDN_HOST_SEGMENT_FRAMES: frames per segment of gdn_frame_forward_host (read on every call).
  *  - GDN_TEST_WITHHOLD_FRAME: test hook only. The fused forward computes but never publishes the
  *    statistics of this frame of head 0, so the call ends with GDN_ERR_TIMEOUT (after the wait
  *    limit) instead of a result; used to test failure detection without faulting the GPU.
@@ -86,6 +87,32 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
                              const float* gamma, const float* beta, const float* state_in,
                              gdn_bf16* out, float* state_out, int B, int H, int T, int N, int D,
                              float key_scale, gdn_stream_t stream);
+
+/*
+ * gdn_frame_forward_host - gdn_frame_forward on a clip held in HOST memory.
+ * (No counterpart in the paper: a deployment variant for clips that do not stay on the GPU,
+ * e.g. minute-long videos whose activations are kept in host memory between layers.)
+ *
+ * q, k, v, gamma, beta, out and the nullable state_in / state_out are HOST pointers with the
+ * layouts of gdn_frame_forward; they need no alignment. Page-locked (pinned) host memory lets
+ * the copies run asynchronously and overlap; pageable memory works but serialises them.
+ * The clip is streamed through the GPU in segments of frames (GDN_HOST_SEGMENT_FRAMES frames,
+ * read on every call; default about 256 MB of q/k/v per segment): while segment i is computed
+ * on `stream`, segment i+1's inputs are copied in and segment i-1's output is copied out on two
+ * internal copy streams, ordered by events, through two device staging buffers. The state is
+ * carried on the device between segments, so the result is that of gdn_frame_forward over the
+ * whole clip, computed as a clip resumed at the segment boundaries (same values up to the
+ * rounding of the bf16 copies of S).
+ * Asynchronous: when `stream` completes, out and state_out hold the result and the inputs may
+ * be reused; read them only after synchronising `stream`. Device memory: two staging buffers of
+ * one segment each (cached per GPU and grown on demand like the workspace) plus the workspace of
+ * one segment's forward. Host-side errors are returned before anything is enqueued; an error
+ * while enqueuing leaves the earlier segments enqueued.
+ */
+gdn_status gdn_frame_forward_host(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                  const float* gamma, const float* beta, const float* state_in,
+                                  gdn_bf16* out, float* state_out, int B, int H, int T, int N,
+                                  int D, float key_scale, gdn_stream_t stream);
 
 /*
  * gdn_frame_forward_noalloc - gdn_frame_forward for callers that must not allocate device memory.

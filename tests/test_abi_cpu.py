@@ -26,8 +26,9 @@ def lib():
 
 def test_header_declares_the_entry_points():
     syms = _declared_symbols()
-    for s in ("gdn_frame_forward", "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
-              "gdn_status_string", "gdn_sync_status", "gdn_release_workspace"):
+    for s in ("gdn_frame_forward", "gdn_frame_forward_host", "gdn_frame_step", "gdn_frame_stats",
+              "gdn_block_causal_la", "gdn_status_string", "gdn_sync_status",
+              "gdn_release_workspace"):
         assert s in syms
 
 
@@ -77,6 +78,24 @@ def test_forward_rejects_bad_arguments_on_the_host(lib):
     assert _fwd(lib, ks=float("nan")) == 1
     assert _fwd(lib, q=P + 8) == 3  # misaligned
     assert _fwd(lib, out=P + 0x10000) == 1  # out overlaps k
+
+
+def _fwd_host(lib, q=P, k=P + 0x10000, v=P + 0x20000, g=P + 0x30000, b=P + 0x31000, si=None,
+              out=P + 0x40000, so=None, B=1, H=2, T=3, N=16, D=32, ks=0.1):
+    return lib.gdn_frame_forward_host(q, k, v, g, b, si, out, so, B, H, T, N, D, ks, None)
+
+
+def test_forward_host_rejects_bad_arguments_on_the_host(lib):
+    assert _fwd_host(lib, v=None) == 1
+    assert _fwd_host(lib, out=None) == 1
+    assert _fwd_host(lib, T=0) == 1
+    assert _fwd_host(lib, D=20) == 2
+    assert _fwd_host(lib, ks=-1.0) == 1
+    assert _fwd_host(lib, out=P + 0x20000) == 1   # out overlaps v
+    # host buffers need no 16-byte alignment; without a GPU the call then fails loudly
+    import torch
+    if not torch.cuda.is_available():
+        assert _fwd_host(lib, q=P + 2) == 5
 
 
 def test_valid_call_without_gpu_fails_loudly(lib):

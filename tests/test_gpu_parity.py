@@ -302,6 +302,64 @@ def test_few_heads_long_clip_uses_chunked_path():
         assert eo <= O_TOL and es <= S_TOL, f"head {h}: O err {eo:.2e}, S err {es:.2e}"
 
 
+@pytest.mark.parametrize("forward_mode", [1, 2, 3], indirect=True, ids=["split", "fused", "chunked"])
+def test_forward_state_in_place(forward_mode):
+    """state_out may be state_in: every path reads the start state before any CTA writes the
+    final one (the chunked replay reads the scan's copy)."""
+    B, H, T, N, D = 1, 2, 17, 64, 128
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=41, state_std=0.4)
+    ks = 1.0 / math.sqrt(D * N)
+    g = to_cuda(x)
+    st = g["state"].clone()
+    out, st2 = api().gdn_frame_forward(g["q"], g["k"], g["v"], g["gamma"], g["beta"], st,
+                                       state_out=st, key_scale=ks)
+    assert api().gdn_sync_status() == 0 and st2 is st
+    o_ref, s_ref = oracle.gdn_frame_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["gamma"]),
+                                            f64(x["beta"]), f64(x["state"]), ks)
+    eo, es = relf(f64(out), o_ref), relf(f64(st), s_ref)
+    assert eo <= O_TOL and es <= S_TOL, f"O err {eo:.2e}, S err {es:.2e}"
+
+
+@pytest.mark.parametrize("case", [
+    # (B, H, T, N, D, segment frames, with_state)
+    (2, 3, 13, 50, 64, 4, True),     # ragged last segment, two batches
+    (1, 2, 30, 100, 128, 7, True),
+    (1, 2, 9, 33, 128, 0, False),    # automatic segment size: one segment
+    (3, 1, 5, 20, 32, 1, True),      # one frame per segment
+])
+def test_forward_host_matches_oracle(case):
+    """gdn_frame_forward_host: pinned host tensors streamed through the GPU in segments."""
+    B, H, T, N, D, seg, with_state = case
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=900 + T, state_std=0.3 if with_state else 0.0)
+    ks = 1.0 / math.sqrt(D * N)
+    pin = {k: (None if t is None else t.pin_memory()) for k, t in x.items()}
+    old = os.environ.get("GDN_HOST_SEGMENT_FRAMES")
+    os.environ["GDN_HOST_SEGMENT_FRAMES"] = str(seg)
+    try:
+        out, st = api().gdn_frame_forward_host(pin["q"], pin["k"], pin["v"], pin["gamma"],
+                                               pin["beta"], pin["state"], key_scale=ks)
+        assert api().gdn_sync_status() == 0
+    finally:
+        if old is None:
+            os.environ.pop("GDN_HOST_SEGMENT_FRAMES", None)
+        else:
+            os.environ["GDN_HOST_SEGMENT_FRAMES"] = old
+    assert not out.is_cuda and not st.is_cuda
+    o_ref, s_ref = oracle.gdn_frame_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["gamma"]),
+                                            f64(x["beta"]),
+                                            None if x["state"] is None else f64(x["state"]), ks)
+    eo, es = relf(f64(out), o_ref), relf(f64(st), s_ref)
+    assert eo <= O_TOL and es <= S_TOL, f"O err {eo:.2e}, S err {es:.2e}"
+    # the device entry point on the same inputs: the same recurrence split at segment bounds,
+    # possibly through another path (the whole clip and a segment may pick different kernels),
+    # so they agree to rounding, not bit for bit
+    g = to_cuda(x)
+    od, sd = api().gdn_frame_forward(g["q"], g["k"], g["v"], g["gamma"], g["beta"], g["state"],
+                                     key_scale=ks)
+    torch.cuda.synchronize()
+    assert relf(f64(out), f64(od)) <= 3e-3 and relf(f64(st), f64(sd)) <= 3e-4
+
+
 STEP_SHAPES = [
     # (B, H, N, D, with_state)
     (2, 3, 100, 128, True),
