@@ -108,10 +108,25 @@ def kernel_bytes(name, w):
     return None
 
 
-def source_digest():
+# Sources each kernel is built from: an ncu traffic figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "gdn_fused_kernel": ["fused_kernel.cuh", "chain_kernel.cuh", "stats_kernel.cuh",
+                         "output_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_step_kernel": ["step_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_stats_kernel": ["stats_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_stats_kernel_la": ["stats_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_output_kernel": ["output_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_chain_kernel": ["chain_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_scan_kernel": ["scan_kernel.cuh", "common.cuh", "ptx.cuh"],
+}
+
+
+def source_digest(kernel=None):
+    """sha256 prefix of the kernel's source files (all of csrc/ when the kernel is unknown)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "frame_wise_gated_deltanet_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc))
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -119,13 +134,13 @@ def source_digest():
 
 def ncu_traffic(kernel, workload):
     """DRAM bytes per launch of `kernel` from profiles/traffic.json, if it was taken on the
-    current kernel sources; else None."""
+    kernel's current sources and on this workload; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
         e = t["kernels"][kernel]
-        if t.get("source_digest") != source_digest() or e.get("workload") != workload:
+        if e.get("source_digest") != source_digest(kernel) or e.get("workload") != workload:
             return None
         return float(e["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
