@@ -90,6 +90,9 @@ struct DeviceState {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   uint64_t attr_done = 0;  // bit per kernel instantiation whose smem attribute is set
+  int* step_flags = nullptr;  // hand-off words of the step kernel (persist across launches)
+  long step_items = 0;
+  int step_epoch = 0;
 };
 
 std::mutex g_mu;
@@ -614,22 +617,55 @@ gdn_status noalloc_scratch(int dev, void** out) {
   return GDN_OK;
 }
 
-// Fused single-frame step (64 < D <= 128): one persistent launch over (batch, head).
+// Single-frame step (64 < D <= 128): one cooperative launch; statistics units and output units
+// are taken dynamically (the workspace holds the per-item S' tiles and the hand-off flags).
 gdn_status run_step(int dev, const Problem& p, const void* q, const void* k, const void* v,
                     const float* gamma, const float* beta, const float* s_in, void* out,
                     float* s_out, cudaStream_t st) {
   using L = gdn::StepLayout;
+  const long items = long(p.B) * p.H;
+  DeviceState& d = g_dev[dev];
+  // persistent flag words: ready [items] (epochs), next_unit, done, abort; zeroed when allocated
+  if (d.step_items < items || d.step_epoch >= 0x7fffff00) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return GDN_ERR_NO_MEMORY;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    if (d.step_flags) cudaFree(d.step_flags);
+    d.step_flags = nullptr;
+    d.step_items = 0;
+    const size_t bytes = sizeof(int) * (items + 3);
+    if (cudaMalloc(&d.step_flags, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return GDN_ERR_NO_MEMORY;
+    }
+    if (cudaMemset(d.step_flags, 0, bytes) != cudaSuccess) return GDN_ERR_CUDA;
+    d.step_items = items;
+    d.step_epoch = 0;
+  }
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, align256(size_t(items) * L::kTileBytes), st, &base))
+    return s;
+  int* f = d.step_flags;
+  gdn::StepShared sh{f, f + d.step_items, f + d.step_items + 1, f + d.step_items + 2,
+                     static_cast<uint8_t*>(base), ++d.step_epoch};
   CUtensorMap tq, tk, tv, to;
   if (!tmap_tokens(&tq, q, p) || !tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p) ||
       !tmap_tokens(&to, out, p))
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_step_kernel;
   if (gdn_status s = ensure_smem_attr(dev, 12, kern, L::kSmemBytes)) return s;
-  const long items = long(p.B) * p.H;
-  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  const int n_tiles = (p.N + gdn::kRowsPerTile - 1) / gdn::kRowsPerTile;
+  const long units = items * (1 + (n_tiles + L::kOutTiles - 1) / L::kOutTiles);
+  const int grid = static_cast<int>(units < d.sms ? units : d.sms);
+  gdn::Problem pp = p;
+  void* args[] = {&tq, &tk, &tv, &to, const_cast<float**>(&gamma), const_cast<float**>(&beta),
+                  const_cast<float**>(&s_in), &s_out, &pp, &sh};
   {
     ProfiledLaunch pl("gdn_step_kernel", st);
-    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, tk, tv, to, gamma, beta, s_in, s_out, p);
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
+                                    dim3(L::kThreads), args, L::kSmemBytes, st) != cudaSuccess)
+      return GDN_ERR_CUDA;
   }
   return check_launch();
 }
@@ -1005,6 +1041,10 @@ void gdn_release_workspace(void) {
   }
   d.ws = nullptr;
   d.ws_bytes = 0;
+  if (d.step_flags) cudaFree(d.step_flags);
+  d.step_flags = nullptr;
+  d.step_items = 0;
+  d.step_epoch = 0;
 }
 
 int gdn_version(void) { return 100; }

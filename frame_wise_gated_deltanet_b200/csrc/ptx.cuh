@@ -193,6 +193,14 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, 
       : "memory");
 }
 
+// Bulk (non-tensor) copy of `bytes` contiguous bytes shared -> global, bulk-group completion.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(gdst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
