@@ -14,8 +14,10 @@
 // by 4 transform warps before the MMA, the state row D holds the normaliser z, and the
 // epilogue divides the first D columns by (column D + 1e-6).
 //
-// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2..5 epilogue,
-// warps 6..9 (LA only) transform.
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2 .. 2+4G-1
+// epilogue (G column groups of 4 warps; warp w reads TMEM lanes 32*(w%4) and DP/G columns), then
+// (LA only) 4 transform warps. The epilogue sets the pace of a tile (TMEM read-out, bf16
+// conversion, staging): with G = 1 a tile took about 1.7 us per SM, under the HBM share.
 //
 // Standalone (gdn_output_kernel): work item i = (b*T + t)*H + h, S_t at workspace row
 // (b*H+h)*T + t_state. Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h
@@ -28,13 +30,16 @@
 
 namespace gdn {
 
-template <int DP, bool kLA>
+template <int DP, bool kLA, int kG = 4>
 struct OutputLayout {
+  static constexpr int kEpiWarps = 4 * kG;
+  static constexpr int kCols = DP / kG;                // columns per epilogue thread
+  static constexpr int kChunk = kCols < 32 ? kCols : 32;
   static constexpr int kBoxes = DP / 64;
   static constexpr int kQBytes = kBoxes * kBoxBytes;   // 128 tokens x DP bf16
   static constexpr int kSBufBytes = DP * DP * 2;       // DP/64 blocks of DP rows x 128 B
   static constexpr int kStages = (DP == 128) ? 3 : 8;
-  static constexpr int kThreads = kLA ? 320 : 192;
+  static constexpr int kThreads = (2 + kEpiWarps + (kLA ? 4 : 0)) * 32;
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
   static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
   static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + 512 + 1024;
@@ -67,13 +72,14 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p) {
 // frames_per_block: 1 for GDN (frame t reads S_t); F for LA (frame t reads the state at the end
 // of its block of F frames). GDN states come from S_src (DP*DP bf16 per row, s8 layout); LA
 // states through tm_s.
-template <int DP, bool kLA, bool kFused>
+template <int DP, bool kLA, bool kFused, int kG>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
                                             const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
                                             uint8_t* smem) {
-  using L = OutputLayout<DP, kLA>;
+  using L = OutputLayout<DP, kLA, kG>;
+  constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                          // 2 state buffers
   uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
   uint8_t* o_stage = q_ring + L::kStages * L::kQBytes;  // 2 output staging tiles
@@ -119,7 +125,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       mbar_init(&s_full[a], 1);
       mbar_init(&s_empty[a], 1);
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+      mbar_init(&acc_empty[a], kEpiThreads);
     }
     for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
     mbar_init(mma_drain, 1);
@@ -261,9 +267,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     if (elect_one()) mma_commit(mma_drain);
     __syncwarp();
     mbar_wait(mma_drain, 0);
-  } else if (warp < 6) {
+  } else if (warp < 2 + L::kEpiWarps) {
     // ---------------------------------------------------------------- epilogue
     const uint32_t quarter = warp & 3;
+    const int c0 = ((warp - 2) >> 2) * L::kCols;  // first column of this warp's group
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
     const int D = p.D;
@@ -275,7 +282,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     for (int li = 0; ok; ++li) {
       const long item = consumer_item(li);
       bool lost = item == -2;
-      if constexpr (kFused) lost = named_bar_any(1, 128, lost);  // uniform across the epilogue
+      if constexpr (kFused) lost = named_bar_any(1, kEpiThreads, lost);  // uniform across the epilogue
       if (lost) ok = false;
       if (lost || item < 0) break;
       const OutputItem it = output_item<kFused>(item, p);
@@ -284,41 +291,40 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
         // staging buffer tc&1 is free once the store issued two tiles ago has read it
         if (leader) bulk_wait_read<1>();
-        if (named_bar_any(1, 128, !waited)) {
+        if (named_bar_any(1, kEpiThreads, !waited)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t tacc = lane_base + acc * DP;
-        float scale = 1.f;
-        if constexpr (kLA) {
-          float z[32];
-          tmem_ld32(tacc + (D / 32) * 32, z);
-          float den = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j == (D & 31)) den = z[j];
-          scale = 1.f / (den + 1e-6f);
-        }
+        // warps whose 32 rows are all past the frame's last token skip the read-out: the TMA
+        // store clips at N, so their staging rows are never written to memory
         uint8_t* ob = o_stage + (tc & 1) * L::kOBytes;
-        float v[32];
+        if (static_cast<int>(quarter) * 32 < p.N - tile * kRowsPerTile) {
+          const uint32_t tacc = lane_base + acc * DP;
+          float scale = 1.f;
+          if constexpr (kLA) scale = 1.f / (tmem_ld1(tacc + D) + 1e-6f);  // normaliser, column D
+          float v[L::kChunk];
 #pragma unroll 1
-        for (int c = 0; c < DP / 32; ++c) {
-          tmem_ld32(tacc + c * 32, v);
+          for (int c = c0; c < c0 + L::kCols; c += L::kChunk) {
+            if constexpr (L::kChunk == 32)
+              tmem_ld32(tacc + c, v);
+            else
+              tmem_ld16(tacc + c, v);
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
-            pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
-            pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
-            pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
-            *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c * 32 + j, kBoxBytes)) = pk;
+            for (int j = 0; j < L::kChunk; j += 8) {
+              uint4 pk;
+              pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
+              pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
+              pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
+              pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
+              *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c + j, kBoxBytes)) = pk;
+            }
           }
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);
         fence_async_smem();
-        named_bar(1, 128);
+        named_bar(1, kEpiThreads);
         if (leader) {
 #pragma unroll
           for (int kb = 0; kb < L::kBoxes; ++kb)
@@ -332,7 +338,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     if (!ok) give_up(hf, abort_flag);
   } else if constexpr (kLA) {
     // ---------------------------------------------------------------- relu(Q) transform
-    const int tid = threadIdx.x - 192;
+    const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -344,14 +350,19 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           ok = false;
           break;
         }
-        uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes);
         const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
-        for (int i = tid; i < L::kQBytes / 16; i += 128) {
-          uint4 x = qt[i];
-          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+        // rows past the frame's last token were zero-filled by the TMA load: relu keeps them
+        const int valid = min(kRowsPerTile, p.N - tile * kRowsPerTile);
+#pragma unroll 1
+        for (int kb = 0; kb < L::kBoxes; ++kb) {
+          uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes + kb * kBoxBytes);
+          for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
+            uint4 x = qt[i];
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-          qt[i] = x;
+            for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
+            qt[i] = x;
+          }
         }
         fence_async_smem();
         mbar_arrive(&ready[stage]);
@@ -380,7 +391,7 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  output_body<DP, kLA, false>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
+  output_body<DP, kLA, false, 4>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
                               align1k(smem_raw));
 }
 

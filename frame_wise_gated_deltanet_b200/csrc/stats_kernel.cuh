@@ -371,15 +371,20 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
           break;
         }
         uint8_t* st = smem + stage * L::kStageBytes;
-        // relu over the whole K tile (layout-agnostic elementwise)
-        uint4* kt = reinterpret_cast<uint4*>(st);
+        // relu over the K tile's token rows (elementwise, so the swizzle does not matter);
+        // rows past the frame's last token were zero-filled by the TMA load and stay zero
         const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
-        for (int i = tid; i < L::kOpBytes / 16; i += 128) {
-          uint4 x = kt[i];
-          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+        const int valid = min(kRowsPerTile, p.N - (tile % n_tiles) * kRowsPerTile);
+#pragma unroll 1
+        for (int kb = 0; kb < L::kOpBytes / kBoxBytes; ++kb) {
+          uint4* kt = reinterpret_cast<uint4*>(st + kb * kBoxBytes);
+          for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
+            uint4 x = kt[i];
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-          kt[i] = x;
+            for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
+            kt[i] = x;
+          }
         }
         // ones column at index D of every V row (token), for the normaliser
         *reinterpret_cast<__nv_bfloat16*>(st + L::kOpBytes +
