@@ -6,10 +6,12 @@ invariants, special cases that reduce to textbook routines, brute force on tiny
 inputs, and a hand-worked example under ``tests/golden/``).
 """
 from .gdn_oracle import (  # noqa: F401
+    e4m3_decode,
     frame_output,
     frame_statistics,
     frame_update,
     gdn_frame_forward,
+    gdn_frame_forward_fp8,
     gdn_frame_step,
     la_block_causal,
 )

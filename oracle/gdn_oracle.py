@@ -48,10 +48,12 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
+    "e4m3_decode",
     "frame_statistics",
     "frame_update",
     "frame_output",
     "gdn_frame_forward",
+    "gdn_frame_forward_fp8",
     "gdn_frame_step",
     "la_block_causal",
 ]
@@ -165,3 +167,35 @@ def la_block_causal(q, k, v, state_in, z_in, frames_per_block: int, eps: float =
             s_out[b, h] = S
             z_out[b, h] = z
     return out, s_out, z_out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of every 8-bit E4M3 floating-point code, by the format's definition (the OCP 8-bit
+    floating-point E4M3 encoding without infinities): bit 7 sign, bits 6..3 exponent e with bias
+    7, bits 2..0 mantissa m; e = 0 encodes the subnormals (m / 8) * 2**-6, the code S.1111.111
+    is NaN, every other code is (1 + m / 8) * 2**(e - 7). Largest finite magnitude 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c & 0x80) != 0, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64))
+    value = np.where(e == 0, (m / 8.0) * 2.0 ** -6, normal)
+    value = np.where((e == 15) & (m == 7), np.nan, value)
+    return sign * value
+
+
+def gdn_frame_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, gamma, beta, state_in,
+                          key_scale: float):
+    """The layer on 8-bit E4M3 inputs with one scale per (batch, frame, head).
+
+    The SANA-Streaming entry of the jefxiong.cn AIGC digest (2026-06-01), item 1, contribution
+    (3), pairs the fused GDN kernel with mixed-precision quantisation to keep the tensor cores
+    busy, and gives no quantiser. Reading adopted: q = decode(q8) * q_scale[b, t, h] for every
+    token and dim of frame t of head h (likewise k and v), then exactly the layer of
+    ``gdn_frame_forward`` on those values. q8, k8, v8: [B, T, N, H, D] uint8 codes; scales
+    [B, T, H]."""
+    def dequant(x8, scale):
+        return e4m3_decode(x8) * _f64(scale)[:, :, None, :, None]
+
+    return gdn_frame_forward(dequant(q8, q_scale), dequant(k8, k_scale), dequant(v8, v_scale),
+                             gamma, beta, state_in, key_scale)

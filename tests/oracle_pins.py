@@ -1,8 +1,9 @@
 """Pins for the fp64 oracle: checks against facts that do not come from the oracle.
 
 Each ``pin_*`` function takes an implementation namespace ``impl`` (an object
-with ``gdn_frame_forward``, ``gdn_frame_step``, ``la_block_causal`` and
-``frame_statistics`` attributes, the same signatures as ``oracle.gdn_oracle``)
+with ``gdn_frame_forward``, ``gdn_frame_step``, ``la_block_causal``,
+``frame_statistics``, ``e4m3_decode`` and ``gdn_frame_forward_fp8`` attributes,
+the same signatures as ``oracle.gdn_oracle``)
 and raises ``AssertionError`` if the implementation disagrees with:
 
 * the hand-worked examples under ``tests/golden/``;
@@ -10,6 +11,8 @@ and raises ``AssertionError`` if the implementation disagrees with:
 * special cases that reduce to a textbook routine (N = 1 is the token-wise
   gated delta rule in residual form; block-causal LA equals brute-force
   quadratic block-causal attention);
+* the E4M3 format's definition (landmark codes, ordering, spacing) and the
+  scale algebra of the fp8 forward;
 * exact invariants (delta-rule exactness for orthonormal keys; the consistent
   linear map is a fixed point; split/resume through the state; linearity in
   (V, S_0); causality across frames and bidirectionality inside a frame; the
@@ -355,6 +358,71 @@ def pin_la_resume(impl):
     _close(z2, z, 1e-12, "LA resume z")
 
 
+def pin_e4m3_landmarks(impl):
+    """E4M3 codes whose values the format's definition fixes (sign, 4-bit exponent with bias 7,
+    3-bit mantissa, exponent 0 for subnormals, S.1111.111 for NaN, no infinities)."""
+    table = {
+        0x00: 0.0, 0x80: -0.0,
+        0x01: 2.0 ** -9,             # smallest subnormal: 1/8 * 2^-6
+        0x07: 7.0 * 2.0 ** -9,       # largest subnormal
+        0x08: 2.0 ** -6,             # smallest normal
+        0x30: 0.5, 0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0xB8: -1.0,
+        0x77: 240.0,                 # 1.875 * 2^7
+        0x7E: 448.0, 0xFE: -448.0,   # largest finite magnitude
+    }
+    codes = np.array(sorted(table), dtype=np.uint8)
+    got = impl.e4m3_decode(codes)
+    want = np.array([table[int(c)] for c in codes])
+    assert np.array_equal(got, want), (got, want)
+    assert np.all(np.isnan(impl.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))))
+
+
+def pin_e4m3_ordering(impl):
+    """Positive codes 0x00..0x7E decode to strictly increasing values, each negative code is the
+    negated positive one, and inside one exponent the spacing is 2^(e-10) (2^-9 subnormal)."""
+    pos = impl.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)
+    neg = impl.e4m3_decode(np.arange(0x80, 0xFF, dtype=np.uint8))
+    assert np.array_equal(neg, -pos)
+    for e in range(1, 16):
+        lo = e << 3
+        hi = min(lo + 7, 0x7E)
+        d = np.diff(impl.e4m3_decode(np.arange(lo, hi + 1, dtype=np.uint8)))
+        assert np.all(d == 2.0 ** (e - 10)), (e, d)
+    assert np.all(np.diff(pos[:8]) == 2.0 ** -9)
+
+
+def pin_fp8_scales(impl):
+    """Per-frame scales of the fp8 forward: q's scale scales O; k's scale trades against the key
+    scale; v's scale together with S_0 scales (O, S_T) (linearity in (V, S_0)); with unit scales
+    it is the forward on the decoded values."""
+    rng = _rng(21)
+    B, T, N, H, D = 1, 3, 5, 2, 4
+    codes = [rng.integers(0, 0x7F, size=(B, T, N, H, D)).astype(np.uint8)
+             | (rng.integers(0, 2, size=(B, T, N, H, D)).astype(np.uint8) << 7) for _ in range(3)]
+    sq, sk, sv = (rng.uniform(0.001, 0.01, size=(B, T, H)) for _ in range(3))
+    g = rng.uniform(0.9, 0.999, size=(B, T, H))
+    be = rng.uniform(0.1, 0.9, size=(B, T, H))
+    S0 = rng.standard_normal((B, H, D, D))
+    ks = 0.3
+    o, s = impl.gdn_frame_forward_fp8(*codes, sq, sk, sv, g, be, S0, ks)
+    o2, s2 = impl.gdn_frame_forward_fp8(*codes, 3.0 * sq, sk, sv, g, be, S0, ks)
+    _close(o2, 3.0 * o, 1e-11, "q scale")
+    _close(s2, s, 1e-12, "q scale leaves the state")
+    o3, s3 = impl.gdn_frame_forward_fp8(*codes, sq, 4.0 * sk, sv, g, be, S0, ks / 4.0)
+    _close(o3, o, 1e-11, "k scale vs key scale")
+    _close(s3, s, 1e-11, "k scale vs key scale (state)")
+    o4, s4 = impl.gdn_frame_forward_fp8(*codes, sq, sk, 2.0 * sv, g, be, 2.0 * S0, ks)
+    _close(o4, 2.0 * o, 1e-11, "v scale with S_0")
+    _close(s4, 2.0 * s, 1e-11, "v scale with S_0 (state)")
+    one = np.ones((B, T, H))
+    dec = [impl.e4m3_decode(c) for c in codes]
+    o5, s5 = impl.gdn_frame_forward_fp8(*codes, one, one, one, g, be, S0, ks)
+    o6, s6 = impl.gdn_frame_forward(*dec, g, be, S0, ks)
+    _close(o5, o6, 1e-12, "unit scales")
+    _close(s5, s6, 1e-12, "unit scales (state)")
+
+
 GDN_PINS = [
     pin_hand_example,
     pin_single_frame_closed_form,
@@ -370,4 +438,5 @@ GDN_PINS = [
     pin_step_is_single_frame,
 ]
 LA_PINS = [pin_la_hand_example, pin_la_brute_force, pin_la_resume]
-ALL_PINS = GDN_PINS + LA_PINS
+FP8_PINS = [pin_e4m3_landmarks, pin_e4m3_ordering, pin_fp8_scales]
+ALL_PINS = GDN_PINS + LA_PINS + FP8_PINS

@@ -11,8 +11,25 @@ import oracle.gdn_oracle as go
 from tests import oracle_pins
 
 
-def _impl(stats=None, update=None, output=None, forward=None, la=None):
-    """An oracle copy with some pieces swapped; gdn_frame_step follows the swapped forward."""
+def _decode_variant(bias=7, subnormals=True):
+    """e4m3 decoding with a planted mistake."""
+    def decode(codes):
+        c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+        sign = np.where((c & 0x80) != 0, -1.0, 1.0)
+        e = (c >> 3) & 0xF
+        m = (c & 0x7).astype(np.float64)
+        normal = (1.0 + m / 8.0) * np.exp2((e - bias).astype(np.float64))
+        val = np.where(e == 0, (m / 8.0) * 2.0 ** (1 - bias), normal) if subnormals else normal
+        val = np.where((e == 15) & (m == 7), np.nan, val)
+        return sign * val
+    return decode
+
+
+def _impl(stats=None, update=None, output=None, forward=None, la=None, decode=None,
+          swap_kv_scales=False):
+    """An oracle copy with some pieces swapped; gdn_frame_step and the fp8 forward follow the
+    swapped forward and decoder."""
+    decode = decode or go.e4m3_decode
     stats = stats or go.frame_statistics
     update = update or go.frame_update
     output = output or go.frame_output
@@ -39,9 +56,17 @@ def _impl(stats=None, update=None, output=None, forward=None, la=None):
                        np.asarray(gamma)[:, None], np.asarray(beta)[:, None], state_in, key_scale)
         return o[:, 0], s
 
+    def fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, gamma, beta, state_in, key_scale):
+        if swap_kv_scales:
+            k_scale, v_scale = v_scale, k_scale
+        deq = lambda x8, sc: decode(x8) * np.asarray(sc, float)[:, :, None, :, None]
+        return forward(deq(q8, q_scale), deq(k8, k_scale), deq(v8, v_scale), gamma, beta,
+                       state_in, key_scale)
+
     return types.SimpleNamespace(gdn_frame_forward=forward, gdn_frame_step=step,
                                  la_block_causal=la or oracle.la_block_causal,
-                                 frame_statistics=stats)
+                                 frame_statistics=stats, e4m3_decode=decode,
+                                 gdn_frame_forward_fp8=fwd_fp8)
 
 
 def _old_state_forward(q, k, v, gamma, beta, state_in, key_scale):
@@ -110,6 +135,9 @@ MUTANTS = {
     "la_eps_dropped": dict(la=_la_variant(eps=0.0)),
     "la_state_transposed": dict(la=_la_variant(transpose_state=True)),
     "la_frame_causal_not_block_causal": dict(la=_la_variant(frame_causal=True)),
+    "e4m3_exponent_bias_8": dict(decode=_decode_variant(bias=8)),
+    "e4m3_subnormals_read_as_normals": dict(decode=_decode_variant(subnormals=False)),
+    "fp8_k_and_v_scales_swapped": dict(swap_kv_scales=True),
 }
 
 

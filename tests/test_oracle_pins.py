@@ -11,6 +11,8 @@ IMPL = types.SimpleNamespace(
     gdn_frame_step=oracle.gdn_frame_step,
     la_block_causal=oracle.la_block_causal,
     frame_statistics=oracle.frame_statistics,
+    e4m3_decode=oracle.e4m3_decode,
+    gdn_frame_forward_fp8=oracle.gdn_frame_forward_fp8,
 )
 
 
