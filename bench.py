@@ -55,6 +55,8 @@ def args_parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="E4M3 q, k, v with per-(frame, head) scales (gdn_frame_forward_fp8)")
     ap.add_argument("--forward-mode", type=int, default=0,
                     help="gdn_set_forward_mode: 0 auto, 1 three kernels, 2 fused, 3 chunked")
     return ap.parse_args()
@@ -70,22 +72,31 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes(w):
-    """Bytes the layer must move per call: Q, K, V read and O written (bf16), gamma and beta,
-    the fp32 state written, and read when the call starts from a carried state."""
+def algorithmic_bytes(w, fp8=False):
+    """Bytes the layer must move per call: Q, K, V read (bf16, or E4M3 plus three f32 scales per
+    frame-head) and O written (bf16), gamma and beta, the fp32 state written, and read when the
+    call starts from a carried state."""
     fh = w.B * w.H * w.T
     state = w.B * w.H * w.D * w.D * 4
     if w.kind == "la":
         return fh * (4 * w.N * w.D * 2) + state + w.B * w.H * w.D * 4
-    return (fh * (4 * w.N * w.D * 2) + w.B * w.T * w.H * 2 * 4 + state
+    qkv = fh * (3 * w.N * w.D + 3 * 4) if fp8 else fh * 3 * w.N * w.D * 2
+    return (qkv + fh * w.N * w.D * 2 + w.B * w.T * w.H * 2 * 4 + state
             + (state if w.kind == "stream" else 0))
 
 
-def kernel_bytes(name, w):
+def kernel_bytes(name, w, fp8=False):
     """Algorithmic bytes per launch of each kernel of the forward (the bytes its stage must
     move in the three-kernel design)."""
     fh = w.B * w.H * w.T
     nd2 = w.N * w.D * 2
+    if fp8:
+        if name == "gdn_stats_kernel":     # read K, V (E4M3); write A_t (bf16) and B_t (f32)
+            return fh * (2 * w.N * w.D + w.D * w.D * 6 + 8)
+        if name == "gdn_output_kernel":    # read Q (E4M3), S_t; write O (bf16)
+            return fh * (w.N * w.D + nd2 + w.D * w.D * 2 + 4)
+        if name == "gdn_fused_kernel":
+            return algorithmic_bytes(w, True)
     dd = w.D * w.D
     if name == "gdn_stats_kernel":       # read K, V; write A_t (bf16) and B_t (f32)
         return fh * (2 * nd2 + dd * 2 + dd * 4)
@@ -341,6 +352,21 @@ def main():
         def step():
             api.gdn_block_causal_la(q, k, v, w.frames_per_block, out=out, state_out=st,
                                     z_out=zt, stream=stream)
+    elif a.fp8:
+        # E4M3 q, k, v with one absmax scale per (batch, frame, head)
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        f8 = {}
+        for n in ("q", "k", "v"):
+            f8[n], f8["s" + n] = gdn_inputs.quantize_e4m3(g[n])
+        out = torch.empty_like(g["q"])
+        del g["q"], g["k"], g["v"]
+        gam, bet = g["gamma"], g["beta"]
+        st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+        def step():
+            api.gdn_frame_forward_fp8(f8["q"], f8["k"], f8["v"], f8["sq"], f8["sk"], f8["sv"],
+                                      gam, bet, None, out, st, key_scale=w.key_scale,
+                                      stream=stream)
     else:
         g = gdn_inputs.workload_inputs(w, device=dev)
         q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
@@ -397,26 +423,28 @@ def main():
     dom = max(per_kernel, key=lambda n: per_kernel[n][0])
     dom_ms = per_kernel[dom][0] / per_kernel[dom][1]
     hbm, peak_kind = peaks()
-    kb = kernel_bytes(dom, w)
+    kb = kernel_bytes(dom, w, a.fp8)
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
-    path_bytes = algorithmic_bytes(w)
+    path_bytes = algorithmic_bytes(w, a.fp8)
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
 
     # ---------------------------------------------------------------- end to end, host buffers
     e2e = None
     if not a.no_e2e:
-        e2e = measure_e2e(a, w, g, out, st, stream, world, dev) if w.kind == "gdn" else None
+        e2e = (measure_e2e(a, w, g, out, st, stream, world, dev)
+               if w.kind == "gdn" and not a.fp8 else None)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 q/k/v, bf16 out" if a.fp8 else "bf16", "data": "synthetic",
         "config": workload_config(w),
         "roofline": {
             "bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": (achieved / hbm) if achieved else None,
             "peak_source": f"{peak_kind} HBM copy bandwidth",
-            "traffic": ncu_traffic(dom, w.name),
+            "traffic": ncu_traffic(dom, w.name + ("+fp8" if a.fp8 else "")),
             "algorithmic_bytes_per_launch": kb, "ms_per_launch": dom_ms,
             "path": {"algorithmic_bytes_per_step": path_bytes, "achieved_gbs": path_gbs,
                      "frac": path_gbs / hbm},
@@ -427,7 +455,7 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn":
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn" and not a.fp8:
         rate, secs, threads = oracle_sample_rate(w, 4, w.T)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"4 heads x {w.T} frames of the {w.name} clip shape "

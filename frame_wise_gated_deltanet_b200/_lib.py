@@ -30,6 +30,7 @@ SIGNATURES = {
     "gdn_frame_forward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_forward_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "gdn_frame_forward_fp8": (_I, [_P] * 11 + [_I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_stats": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_block_causal_la": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),

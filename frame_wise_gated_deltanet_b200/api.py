@@ -12,7 +12,8 @@ import torch
 
 from ._lib import LIB, GdnError, check
 
-__all__ = ["gdn_frame_forward", "gdn_frame_forward_host", "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
+__all__ = ["gdn_frame_forward", "gdn_frame_forward_fp8", "gdn_frame_forward_host",
+           "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
            "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
            "gdn_la_workspace_bytes", "GdnError"]
 
@@ -64,6 +65,43 @@ def gdn_frame_forward(q, k, v, gamma, beta, state_in=None, out=None, state_out=N
         check("gdn_frame_forward", LIB.gdn_frame_forward(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
             _ptr(state_out), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
+    return out, state_out
+
+
+def _codes(t: torch.Tensor, name: str, shape) -> torch.Tensor:
+    """E4M3 codes as uint8: accepts torch.uint8 or torch.float8_e4m3fn CUDA tensors."""
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    _req(t, name, torch.uint8, shape)
+    return t
+
+
+def gdn_frame_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, gamma, beta, state_in=None,
+                          out=None, state_out=None, key_scale: Optional[float] = None,
+                          stream=None, want_state: bool = True):
+    """Frame-wise GDN on E4M3 q, k, v ([B,T,N,H,D], uint8 codes or float8_e4m3fn) with scales
+    [B,T,H] f32 (x = decode(x8) * x_scale[b,t,h]). Returns (out bf16, state_out)."""
+    B, T, N, H, D = q8.shape
+    q8, k8, v8 = (_codes(t, n, (B, T, N, H, D)) for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")))
+    for name, t in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale),
+                    ("gamma", gamma), ("beta", beta)):
+        _req(t, name, torch.float32, (B, T, H))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if out is None:
+        out = torch.empty((B, T, N, H, D), dtype=torch.bfloat16, device=q8.device)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q8.device)
+    if state_out is not None:
+        _req(state_out, "state_out", torch.float32, (B, H, D, D))
+    if key_scale is None:
+        key_scale = 1.0 / math.sqrt(D * N)
+    with torch.cuda.device(q8.device):
+        check("gdn_frame_forward_fp8", LIB.gdn_frame_forward_fp8(
+            _ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+            _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out), _ptr(state_out),
+            B, H, T, N, D, float(key_scale), _stream(stream, q8.device)))
     return out, state_out
 
 

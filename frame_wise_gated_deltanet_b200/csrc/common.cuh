@@ -20,6 +20,10 @@ constexpr int kErrTimeout = 6;  // == GDN_ERR_TIMEOUT
 struct Problem {
   int B, H, T, N, D;
   float key_scale;
+  // fp8 (e4m3) inputs: per (b, t, h) scales [B, T, H] f32, q = q8 * q_scale etc.; unused for bf16
+  const float* q_scale = nullptr;
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
 };
 
 // Hand-off state of the fused forward, in device memory and zeroed before each call. One

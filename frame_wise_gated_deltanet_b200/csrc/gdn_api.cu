@@ -51,7 +51,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D tile (dims[0] contiguous) with 128B swizzle, zero fill out of bounds.
+// Tiled map (dims[0] contiguous) with 128B swizzle, zero fill out of bounds.
 bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
                const cuuint64_t* dims, const cuuint64_t* strides_bytes, const cuuint32_t* box) {
   EncodeTiledFn fn = encode_fn();
@@ -72,6 +72,23 @@ bool tmap_tokens(CUtensorMap* m, const void* base, const Problem& p) {
                                  (cuuint64_t)p.N * p.H * p.D * 2};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box);
+}
+
+// e4m3 q/k/v [B, T, N, H, D] bytes -> 4-D map (D, H, N, B*T), box 128 x 1 x 128 x 1 (one
+// 128-byte swizzled row of 128 dims per token; dims past D read as zero). D % 16 == 0.
+bool tmap_tokens_f8(CUtensorMap* m, const void* base, const Problem& p) {
+  const cuuint64_t dims[4] = {(cuuint64_t)p.D, (cuuint64_t)p.H, (cuuint64_t)p.N,
+                              (cuuint64_t)p.B * p.T};
+  const cuuint64_t strides[3] = {(cuuint64_t)p.D, (cuuint64_t)p.H * p.D,
+                                 (cuuint64_t)p.N * p.H * p.D};
+  const cuuint32_t box[4] = {128, 1, 128, 1};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box);
+}
+
+// Token map of q, k or v in the element type of the path.
+template <bool kF8>
+bool tmap_in(CUtensorMap* m, const void* base, const Problem& p) {
+  return kF8 ? tmap_tokens_f8(m, base, p) : tmap_tokens(m, base, p);
 }
 
 // [count, rows, D] matrices (bf16 or f32) -> 3-D map (D, rows, count), box (128 B) x DP x 1.
@@ -204,15 +221,15 @@ gdn_status check_launch() {
 
 // ------------------------------------------------------------------ kernel runners
 // kB4: B_t in the chain's interleaved layout (forward paths) or row-major (gdn_frame_stats).
-template <int DP, bool kB4>
+template <int DP, bool kB4, bool kF8 = false>
 gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, void* A, float* Bm,
                      cudaStream_t st) {
-  using L = gdn::StatsLayout<DP, false>;
+  using L = gdn::StatsLayout<DP, false, kF8>;
   CUtensorMap tk, tv;
-  if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_stats_kernel<DP, false, kB4>;
-  if (gdn_status s = ensure_smem_attr(dev, (DP == 128 ? 0 : 1) + (kB4 ? 10 : 0), kern,
-                                      L::kSmemBytes))
+  if (!tmap_in<kF8>(&tk, k, p) || !tmap_in<kF8>(&tv, v, p)) return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_stats_kernel<DP, false, kB4, kF8>;
+  if (gdn_status s = ensure_smem_attr(
+          dev, kF8 ? 15 : (DP == 128 ? 0 : 1) + (kB4 ? 10 : 0), kern, L::kSmemBytes))
     return s;
   const long items = long(p.B) * p.T * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
@@ -262,20 +279,21 @@ gdn_status run_scan(int dev, const Problem& p, const gdn::ChainSeg& seg, const f
   return check_launch();
 }
 
-template <int DP, bool kLA>
+template <int DP, bool kLA, bool kF8 = false>
 gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws, int srows,
                       void* out, int F, cudaStream_t st) {
-  using L = gdn::OutputLayout<DP, kLA>;
+  using L = gdn::OutputLayout<DP, kLA, 4, kF8>;
   const long count = long(p.B) * p.H * ((p.T + F - 1) / F);  // stored states (per block for LA)
   CUtensorMap tq, ts, to;
-  if (!tmap_tokens(&tq, q, p) || !tmap_tokens(&to, out, p)) return GDN_ERR_CUDA;
+  if (!tmap_in<kF8>(&tq, q, p) || !tmap_tokens(&to, out, p)) return GDN_ERR_CUDA;
   if (kLA) {
     if (!tmap_mats(&ts, S_ws, false, p.D, srows, count, DP)) return GDN_ERR_CUDA;
   } else {
     ts = tq;  // unused: GDN states are bulk-copied from S_ws
   }
-  auto kern = gdn::gdn_output_kernel<DP, kLA>;
-  if (gdn_status s = ensure_smem_attr(dev, kLA ? 6 : (DP == 128 ? 4 : 5), kern, L::kSmemBytes))
+  auto kern = gdn::gdn_output_kernel<DP, kLA, kF8>;
+  if (gdn_status s = ensure_smem_attr(dev, kF8 ? 16 : (kLA ? 6 : (DP == 128 ? 4 : 5)), kern,
+                                      L::kSmemBytes))
     return s;
   const long items = long(p.B) * p.T * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
@@ -390,7 +408,7 @@ bool fused_applies(int dev, const Problem& p) {
   return bh * 3 <= sms && p.T >= 4;
 }
 
-template <int DP>
+template <int DP, bool kF8 = false>
 gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, const void* v,
                      const float* gamma, const float* beta, const float* s_in, void* out,
                      float* s_out, cudaStream_t st) {
@@ -403,11 +421,12 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   FusedWs w = carve_fused(base, bh, p.T, p.D);
   if (cudaMemsetAsync(w.flags, 0, w.flag_bytes, st) != cudaSuccess) return GDN_ERR_CUDA;
   CUtensorMap tk, tv, tq, to, ta;
-  if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p) || !tmap_tokens(&tq, q, p) ||
+  if (!tmap_in<kF8>(&tk, k, p) || !tmap_in<kF8>(&tv, v, p) || !tmap_in<kF8>(&tq, q, p) ||
       !tmap_tokens(&to, out, p) || !tmap_mats(&ta, w.A, false, p.D, p.D, long(bh) * kRing, DP))
     return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_fused_kernel<DP>;
-  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 8 : 9, kern, L::kSmemBytes)) return s;
+  auto kern = gdn::gdn_fused_kernel<DP, kF8>;
+  if (gdn_status s = ensure_smem_attr(dev, kF8 ? 17 : (DP == 128 ? 8 : 9), kern, L::kSmemBytes))
+    return s;
   // split the SMs left after the chains between the stats and output roles (by default
   // ~54 : 46, the ratio of their per-frame times)
   const int workers = sms - bh;
@@ -541,7 +560,7 @@ bool chunked_pays(int dev, const Problem& p, bool fused) {
   return chunked < 0.9 * other;
 }
 
-template <int DP>
+template <int DP, bool kF8 = false>
 gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, const void* v,
                        const float* gamma, const float* beta, const float* s_in, void* out,
                        float* s_out, cudaStream_t st) {
@@ -556,7 +575,7 @@ gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, 
   uint8_t* starts = maps + align256(size_t(bh) * (plan.nc - 1) * gdn::chunk_map_bytes(DP));
   const gdn::ChainSeg compose{plan.L, plan.nc, 1, maps, starts};
   const gdn::ChainSeg replay{plan.L, plan.nc, 0, maps, starts};
-  if (gdn_status s = run_stats<DP, true>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_stats<DP, true, kF8>(dev, p, k, v, w.A, w.B, st)) return s;
   if (plan.nc > 1) {
     if (gdn_status s = run_chain<DP>(dev, p, w.A, w.B, gamma, beta, nullptr, nullptr, nullptr,
                                      compose, st))
@@ -565,7 +584,41 @@ gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, 
   }
   if (gdn_status s = run_chain<DP>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, replay, st))
     return s;
-  return run_output<DP, false>(dev, p, q, w.S, p.D, out, 1, st);
+  return run_output<DP, false, kF8>(dev, p, q, w.S, p.D, out, 1, st);
+}
+
+// kF8: e4m3 q, k, v (scales in p; 64 < D <= 128, checked by the caller).
+template <bool kF8>
+gdn_status forward_path(int dev, const void* q, const void* k, const void* v, const float* gamma,
+                        const float* beta, const float* s_in, void* out, float* s_out,
+                        const Problem& p, cudaStream_t st) {
+  constexpr int kDP = 128;
+  const bool fused = fused_applies(dev, p);
+  if (g_forward_mode == 3 || (g_forward_mode == 0 && chunked_pays(dev, p, fused))) {
+    if (!kF8 && p.D <= 64)
+      return run_chunked<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+    return run_chunked<kDP, kF8>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+  }
+  if (fused) {
+    if (!kF8 && p.D <= 64)
+      return run_fused<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+    return run_fused<kDP, kF8>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+  }
+  const long count = long(p.B) * p.H * p.T;
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, forward_ws_bytes(count, p.D), st, &base)) return s;
+  ForwardWs w = carve_forward(base, count, p.D);
+  const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
+  if (!kF8 && p.D <= 64) {
+    if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
+      return s;
+    return run_output<64, false>(dev, p, q, w.S, p.D, out, 1, st);
+  }
+  if (gdn_status s = run_stats<kDP, true, kF8>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_chain<kDP>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
+    return s;
+  return run_output<kDP, false, kF8>(dev, p, q, w.S, p.D, out, 1, st);
 }
 
 gdn_status forward_impl(const void* q, const void* k, const void* v, const float* gamma,
@@ -574,30 +627,9 @@ gdn_status forward_impl(const void* q, const void* k, const void* v, const float
   int dev;
   if (gdn_status s = current_device(&dev)) return s;
   std::lock_guard<std::mutex> lock(g_mu);
-  const bool fused = fused_applies(dev, p);
-  if (g_forward_mode == 3 || (g_forward_mode == 0 && chunked_pays(dev, p, fused))) {
-    if (p.D <= 64) return run_chunked<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
-    return run_chunked<128>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
-  }
-  if (fused) {
-    if (p.D <= 64) return run_fused<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
-    return run_fused<128>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
-  }
-  const long count = long(p.B) * p.H * p.T;
-  void* base = nullptr;
-  if (gdn_status s = get_workspace(dev, forward_ws_bytes(count, p.D), st, &base)) return s;
-  ForwardWs w = carve_forward(base, count, p.D);
-  const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
-  if (p.D <= 64) {
-    if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
-    if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
-      return s;
-    return run_output<64, false>(dev, p, q, w.S, p.D, out, 1, st);
-  }
-  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
-  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
-    return s;
-  return run_output<128, false>(dev, p, q, w.S, p.D, out, 1, st);
+  if (p.k_scale != nullptr)
+    return forward_path<true>(dev, q, k, v, gamma, beta, s_in, out, s_out, p, st);
+  return forward_path<false>(dev, q, k, v, gamma, beta, s_in, out, s_out, p, st);
 }
 
 // Device address of g_noalloc_scratch on the current GPU, looked up once per GPU (with that GPU
@@ -883,6 +915,31 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
                                     whole, st))
     return s;
   return run_output<128, false>(dev, p, q, w.S, D, out, 1, st);
+}
+
+gdn_status gdn_frame_forward_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v,
+                                 const float* q_scale, const float* k_scale,
+                                 const float* v_scale, const float* gamma, const float* beta,
+                                 const float* state_in, gdn_bf16* out, float* state_out, int B,
+                                 int H, int T, int N, int D, float key_scale,
+                                 gdn_stream_t stream) {
+  if (!q || !k || !v || !out || !gamma || !beta || !q_scale || !k_scale || !v_scale)
+    return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  if (D <= 64 || D % 16 != 0) return GDN_ERR_UNSUPPORTED;
+  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+    return GDN_ERR_MISALIGNED;
+  const size_t n8 = size_t(B) * T * N * H * D, n16 = n8 * 2;
+  if (overlaps(out, n16, q, n8) || overlaps(out, n16, k, n8) || overlaps(out, n16, v, n8))
+    return GDN_ERR_INVALID_ARG;
+  Problem p{B, H, T, N, D, key_scale};
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 gdn_status gdn_frame_forward_host(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,

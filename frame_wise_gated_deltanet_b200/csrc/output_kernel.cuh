@@ -13,6 +13,9 @@
 // LA mode (block-causal linear attention): Q tiles are passed through relu in shared memory
 // by 4 transform warps before the MMA, the state row D holds the normaliser z, and the
 // epilogue divides the first D columns by (column D + 1e-6).
+// fp8 mode (e4m3 Q, DP = 128): the Q tile is TMA-loaded into the second box of its bf16 stage,
+// the 4 transform warps convert it in place (exactly), and the epilogue multiplies by the
+// frame's Q scale.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2 .. 2+4G-1
 // epilogue (G column groups of 4 warps; warp w reads TMEM lanes 32*(w%4) and DP/G columns), then
@@ -30,8 +33,10 @@
 
 namespace gdn {
 
-template <int DP, bool kLA, int kG = 4>
+template <int DP, bool kLA, int kG = 4, bool kF8 = false>
 struct OutputLayout {
+  static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
+  static constexpr bool kTransform = kLA || kF8;
   static constexpr int kEpiWarps = 4 * kG;
   static constexpr int kCols = DP / kG;                // columns per epilogue thread
   static constexpr int kChunk = kCols < 32 ? kCols : 32;
@@ -39,7 +44,8 @@ struct OutputLayout {
   static constexpr int kQBytes = kBoxes * kBoxBytes;   // 128 tokens x DP bf16
   static constexpr int kSBufBytes = DP * DP * 2;       // DP/64 blocks of DP rows x 128 B
   static constexpr int kStages = (DP == 128) ? 3 : 8;
-  static constexpr int kThreads = (2 + kEpiWarps + (kLA ? 4 : 0)) * 32;
+  static constexpr int kThreads = (2 + kEpiWarps + (kTransform ? 4 : 0)) * 32;
+  static constexpr int kQLoadBytes = kF8 ? kQBytes / 2 : kQBytes;  // TMA bytes per Q tile
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
   static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
   static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + 512 + 1024;
@@ -72,13 +78,13 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p) {
 // frames_per_block: 1 for GDN (frame t reads S_t); F for LA (frame t reads the state at the end
 // of its block of F frames). GDN states come from S_src (DP*DP bf16 per row, s8 layout); LA
 // states through tm_s.
-template <int DP, bool kLA, bool kFused, int kG>
+template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
                                             const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
                                             uint8_t* smem) {
-  using L = OutputLayout<DP, kLA, kG>;
+  using L = OutputLayout<DP, kLA, kG, kF8>;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                          // 2 state buffers
   uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
@@ -191,11 +197,17 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
             give_up(hf, abort_flag);
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], L::kQBytes);
+          mbar_arrive_expect_tx(&full[stage], L::kQLoadBytes);
+          if constexpr (kF8) {
+            // one 128-byte-wide e4m3 box, into the stage's second bf16 box
+            tma_load_4d(q_ring + stage * L::kQBytes + kBoxBytes, tm_q, &full[stage], 0, it.h,
+                        tile * kRowsPerTile, it.bt, pol_stream);
+          } else {
 #pragma unroll
-          for (int kb = 0; kb < L::kBoxes; ++kb)
-            tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
-                        kb * 64, it.h, tile * kRowsPerTile, it.bt, pol_stream);
+            for (int kb = 0; kb < L::kBoxes; ++kb)
+              tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
+                          kb * 64, it.h, tile * kRowsPerTile, it.bt, pol_stream);
+          }
           fills.filled(stage, phase);
           if (++stage == L::kStages) {
             stage = 0;
@@ -231,7 +243,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
         if (!mbar_wait(&acc_empty[acc], ((tc >> 1) & 1) ^ 1) ||
-            !mbar_wait(kLA ? &ready[stage] : &full[stage], phase)) {
+            !mbar_wait(L::kTransform ? &ready[stage] : &full[stage], phase)) {
           ok = false;
           break;
         }
@@ -303,6 +315,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           const uint32_t tacc = lane_base + acc * DP;
           float scale = 1.f;
           if constexpr (kLA) scale = 1.f / (tmem_ld1(tacc + D) + 1e-6f);  // normaliser, column D
+          if constexpr (kF8) scale = __ldg(p.q_scale + static_cast<long>(it.bt) * p.H + it.h);
           float v[L::kChunk];
 #pragma unroll 1
           for (int c = c0; c < c0 + L::kCols; c += L::kChunk) {
@@ -336,45 +349,72 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     }
     if (leader) bulk_wait_all();
     if (!ok) give_up(hf, abort_flag);
-  } else if constexpr (kLA) {
-    // ---------------------------------------------------------------- relu(Q) transform
-    const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int li = 0; ok; ++li) {
-      const long item = consumer_item(li);
-      if (item < 0) break;
-      for (int tile = 0; tile < n_tiles; ++tile) {
-        if (!mbar_wait(&full[stage], phase)) {
-          ok = false;
-          break;
-        }
-        const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
-        // rows past the frame's last token were zero-filled by the TMA load: relu keeps them
-        const int valid = min(kRowsPerTile, p.N - tile * kRowsPerTile);
-#pragma unroll 1
-        for (int kb = 0; kb < L::kBoxes; ++kb) {
-          uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes + kb * kBoxBytes);
-          for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
-            uint4 x = qt[i];
-            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-            qt[i] = x;
+  } else if (L::kTransform && warp < 2 + L::kEpiWarps + 4) {
+    // (the fused kernel's output CTAs have more warps: the rest stay idle)
+    if constexpr (kF8) {
+      // ---------------------------------------------------------------- e4m3 Q conversion
+      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // the token row it converts
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int li = 0; ok; ++li) {
+        const long item = consumer_item(li);
+        if (item < 0) break;
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          e4m3_row_to_bf16_tile(q_ring + stage * L::kQBytes, tid);
+          fence_async_smem();
+          mbar_arrive(&ready[stage]);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
           }
         }
-        fence_async_smem();
-        mbar_arrive(&ready[stage]);
-        if (++stage == L::kStages) {
-          stage = 0;
-          phase ^= 1;
+      }
+      if (!ok) give_up(hf, abort_flag);
+    } else if constexpr (kLA) {
+      // ---------------------------------------------------------------- relu(Q) transform
+      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int li = 0; ok; ++li) {
+        const long item = consumer_item(li);
+        if (item < 0) break;
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
+          // rows past the frame's last token were zero-filled by the TMA load: relu keeps them
+          const int valid = min(kRowsPerTile, p.N - tile * kRowsPerTile);
+  #pragma unroll 1
+          for (int kb = 0; kb < L::kBoxes; ++kb) {
+            uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes + kb * kBoxBytes);
+            for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
+              uint4 x = qt[i];
+              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+  #pragma unroll
+              for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
+              qt[i] = x;
+            }
+          }
+          fence_async_smem();
+          mbar_arrive(&ready[stage]);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
+      if (!ok) give_up(hf, abort_flag);
     }
-    if (!ok) give_up(hf, abort_flag);
-  }
 
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -383,16 +423,16 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   }
 }
 
-template <int DP, bool kLA>
-__global__ void __launch_bounds__(OutputLayout<DP, kLA>::kThreads, 1)
+template <int DP, bool kLA, bool kF8 = false>
+__global__ void __launch_bounds__(OutputLayout<DP, kLA, 4, kF8>::kThreads, 1)
     gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_s,
                       const __nv_bfloat16* __restrict__ S_src,
                       const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  output_body<DP, kLA, false, 4>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
-                              align1k(smem_raw));
+  output_body<DP, kLA, false, 4, kF8>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
+                                      align1k(smem_raw));
 }
 
 }  // namespace gdn

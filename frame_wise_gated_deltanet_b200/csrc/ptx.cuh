@@ -7,6 +7,8 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 namespace gdn {
 
@@ -365,6 +367,48 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 e4m3 values (byte i = element i) -> 16 bf16 (lo: elements 0..7, hi: 8..15). Every e4m3
+// value is exactly representable in fp16 and in bf16, so the conversion is exact.
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4& in, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t pair =
+        static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
+    const __half2 h2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3));
+    const __nv_bfloat162 b2 = __float22bfloat162_rn(__half22float2(h2));
+    o[i] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// An fp8 operand tile converted in place into the bf16 operand layout. The tile holds 128 token
+// rows; the bf16 form is two 128B-swizzled TMA boxes of 64 dims (box0 at `tile`, box1 at
+// tile + 16 KB, row r at r * 128 in each); the fp8 form was TMA-loaded 128B-swizzled into the
+// box1 region (row r: 128 e4m3 values at tile + 16 KB + r * 128). Thread `row` converts its own
+// row: it reads all of fp8 row r before writing box1 row r, which occupies the same bytes.
+__device__ __forceinline__ void e4m3_row_to_bf16_tile(uint8_t* tile, int row) {
+  uint8_t* b0 = tile + row * 128;
+  uint8_t* b1 = tile + 16384 + row * 128;
+  const uint32_t sw = row & 7;
+  uint4 in[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) in[c] = *reinterpret_cast<const uint4*>(b1 + ((c ^ sw) << 4));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    // fp8 chunk c = dims 16c..16c+15 -> bf16 chunks 2c, 2c+1 of the 16 chunks of 8 dims
+    uint4 lo, hi;
+    e4m3x16_to_bf16(in[c], lo, hi);
+    const int k0 = 2 * c, k1 = 2 * c + 1;          // 8-dim chunk index over 128 dims
+    uint8_t* d0 = (k0 < 8 ? b0 : b1) + (((k0 & 7) ^ sw) << 4);
+    uint8_t* d1 = (k1 < 8 ? b0 : b1) + (((k1 & 7) ^ sw) << 4);
+    *reinterpret_cast<uint4*>(d0) = lo;
+    *reinterpret_cast<uint4*>(d1) = hi;
+  }
 }
 
 // 32 lanes x one 32-bit column (wait included).

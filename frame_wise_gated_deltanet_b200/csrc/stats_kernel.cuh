@@ -12,7 +12,10 @@
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one elected thread)
 //   warps 2..5  epilogue: TMEM -> registers -> scale -> global
-//   warps 6..9  (LA only) in-place transform of each K/V stage: relu(K), ones column in V
+//   warps 6..   (LA and fp8 only) in-place transform of each K/V stage: relu(K) and a ones
+//               column in V (LA, warps 6..9), or e4m3 -> bf16 conversion of K and V (fp8
+//               inputs, DP = 128, warps 6..13, one token row of K or V per thread: the fp8
+//               tiles are TMA-loaded into the second box of each bf16 operand tile)
 //
 // Standalone (gdn_stats_kernel): work item i = (b*T + t)*H + h, results at workspace row
 // (b*H + h)*T + t; for LA an item is a block of frames_per_item frames (its statistics summed),
@@ -26,15 +29,19 @@
 
 namespace gdn {
 
-template <int DP, bool kLA>
+template <int DP, bool kLA, bool kF8 = false>
 struct StatsLayout {
+  static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
+  static constexpr bool kTransform = kLA || kF8;
   static constexpr int kBoxes = DP / 64;                // 64-dim boxes per operand tile
   static constexpr int kOpBytes = kBoxes * kBoxBytes;   // 128 tokens x DP dims, bf16
   static constexpr int kStageBytes = 2 * kOpBytes;      // K tile + V tile
   static constexpr int kStages = (DP == 128) ? 3 : 6;
   static constexpr int kAccCols = kLA ? 128 : (DP == 128 ? 256 : 64);
   static constexpr int kTmemCols = 2 * kAccCols;
-  static constexpr int kThreads = kLA ? 320 : 192;
+  static constexpr int kTransformThreads = kF8 ? 256 : 128;
+  static constexpr int kThreads = 192 + (kTransform ? kTransformThreads : 0);
+  static constexpr int kLoadBytes = kF8 ? kStageBytes / 2 : kStageBytes;  // TMA bytes per stage
   static constexpr int kBarrierBytes = 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
@@ -78,14 +85,14 @@ __device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, con
 
 // kB4: B_t stored in the four-key interleaved layout of b4_index (the chain's input) instead of
 // row-major (the public gdn_frame_stats layout and the block-causal path).
-template <int DP, bool kLA, bool kFused, bool kB4>
+template <int DP, bool kLA, bool kFused, bool kB4, bool kF8 = false>
 __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                            __nv_bfloat16* __restrict__ A_ws,
                                            float* __restrict__ B_ws, const Problem& p,
                                            const Handoff& hf, uint8_t* smem, int fpb = 1) {
-  using L = StatsLayout<DP, kLA>;
+  using L = StatsLayout<DP, kLA, kF8>;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
-  uint64_t* ready = full + L::kStages;   // LA: transformed stage
+  uint64_t* ready = full + L::kStages;   // LA / fp8: transformed stage
   uint64_t* empty = ready + L::kStages;
   uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 2;
@@ -116,7 +123,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 128);
+      mbar_init(&ready[s], L::kTransformThreads);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -157,14 +164,22 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
             give_up(hf, abort_flag);
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          mbar_arrive_expect_tx(&full[stage], L::kLoadBytes);
           uint8_t* st = smem + stage * L::kStageBytes;
+          if constexpr (kF8) {
+            // one 128-byte-wide e4m3 box per operand, into its second bf16 box
+            tma_load_4d(st + kBoxBytes, tm_k, &full[stage], 0, it.h, tile * kRowsPerTile, bt,
+                        pol);
+            tma_load_4d(st + L::kOpBytes + kBoxBytes, tm_v, &full[stage], 0, it.h,
+                        tile * kRowsPerTile, bt, pol);
+          } else {
 #pragma unroll
-          for (int j = 0; j < L::kBoxes; ++j) {
-            tma_load_4d(st + j * kBoxBytes, tm_k, &full[stage], j * 64, it.h,
-                        tile * kRowsPerTile, bt, pol);
-            tma_load_4d(st + L::kOpBytes + j * kBoxBytes, tm_v, &full[stage], j * 64, it.h,
-                        tile * kRowsPerTile, bt, pol);
+            for (int j = 0; j < L::kBoxes; ++j) {
+              tma_load_4d(st + j * kBoxBytes, tm_k, &full[stage], j * 64, it.h,
+                          tile * kRowsPerTile, bt, pol);
+              tma_load_4d(st + L::kOpBytes + j * kBoxBytes, tm_v, &full[stage], j * 64, it.h,
+                          tile * kRowsPerTile, bt, pol);
+            }
           }
           fills.filled(stage, phase);
           if (++stage == L::kStages) {
@@ -200,7 +215,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
       bool ok = true;
       for (int tile = 0; tile < nf * n_tiles; ++tile) {
-        if (!mbar_wait(kLA ? &ready[stage] : &full[stage], phase)) {
+        if (!mbar_wait(L::kTransform ? &ready[stage] : &full[stage], phase)) {
           ok = false;
           break;
         }
@@ -283,6 +298,14 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       const long ws = it.row;
       const uint32_t tacc = lane_base + acc * L::kAccCols;
       float v[32];
+      // fp8: the dequantisation scales of this frame's K and V enter A and B here
+      float fa = s * s, fb = s;
+      if constexpr (kF8) {
+        const long gi = static_cast<long>(it.bt) * p.H + it.h;
+        const float sk = __ldg(p.k_scale + gi), sv = __ldg(p.v_scale + gi);
+        fa *= sk * sk;
+        fb *= sk * sv;
+      }
       if constexpr (kLA) {
         // row = value index v (row D = normaliser); columns = key index
         float* brow = B_ws + (ws * brows + row) * D;
@@ -304,7 +327,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
         // DP == 64 : one 64-column accumulator; rows 0..63 = A, rows 64..127 = B.
         const bool is_a = (DP == 128) ? true : (row < 64);
         const int mrow = (DP == 128) ? row : (row & 63);
-        const float s2 = s * s;
+        const float s2 = fa;
 #pragma unroll 1
         for (int part = 0; part < (DP == 128 ? 2 : 1); ++part) {
           const bool a_part = (DP == 128) ? (part == 0) : is_a;
@@ -335,7 +358,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
                   if (col < D) {
                     const long off = kB4 ? b4_index(mrow, col, D) : static_cast<long>(mrow) * D + col;
                     *reinterpret_cast<float4*>(bmat + off) =
-                        make_float4(v[j] * s, v[j + 1] * s, v[j + 2] * s, v[j + 3] * s);
+                        make_float4(v[j] * fb, v[j + 1] * fb, v[j + 2] * fb, v[j + 3] * fb);
                   }
                 }
               }
@@ -354,56 +377,87 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
           st_release(hf.stats_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
       }
     }
-  } else if constexpr (kLA) {
-    // ---------------------------------------------------------------- LA transform warps
-    const int tid = threadIdx.x - 192;  // 0..127
-    int stage = 0;
-    uint32_t phase = 0;
-    const int D = p.D;
-    for (int li = 0;; ++li) {
-      const long item = consumer_item(li);
-      if (item < 0) break;
-      const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
-      bool ok = true;
-      for (int tile = 0; tile < nf * n_tiles; ++tile) {
-        if (!mbar_wait(&full[stage], phase)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + stage * L::kStageBytes;
-        // relu over the K tile's token rows (elementwise, so the swizzle does not matter);
-        // rows past the frame's last token were zero-filled by the TMA load and stay zero
-        const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
-        const int valid = min(kRowsPerTile, p.N - (tile % n_tiles) * kRowsPerTile);
-#pragma unroll 1
-        for (int kb = 0; kb < L::kOpBytes / kBoxBytes; ++kb) {
-          uint4* kt = reinterpret_cast<uint4*>(st + kb * kBoxBytes);
-          for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
-            uint4 x = kt[i];
-            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-            kt[i] = x;
+  } else if (L::kTransform && warp < 6 + L::kTransformThreads / 32) {
+    // (the fused kernel's stats CTAs have more warps: the rest stay idle)
+    if constexpr (kF8) {
+      // ---------------------------------------------------------------- fp8 conversion warps
+      const int tid = threadIdx.x - 192;  // 0..255: K row tid, or V row tid - 128
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int li = 0;; ++li) {
+        const long item = consumer_item(li);
+        if (item < 0) break;
+        bool ok = true;
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * L::kStageBytes;
+          e4m3_row_to_bf16_tile(st + (tid >> 7) * L::kOpBytes, tid & 127);
+          fence_async_smem();
+          mbar_arrive(&ready[stage]);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
           }
         }
-        // ones column at index D of every V row (token), for the normaliser
-        *reinterpret_cast<__nv_bfloat16*>(st + L::kOpBytes +
-                                          swz128_offset_bf16(tid, D, kBoxBytes)) =
-            __float2bfloat16(1.0f);
-        fence_async_smem();
-        mbar_arrive(&ready[stage]);
-        if (++stage == L::kStages) {
-          stage = 0;
-          phase ^= 1;
+        if (!ok) {
+          give_up(hf, abort_flag);
+          break;
         }
       }
-      if (!ok) {
-        give_up(hf, abort_flag);
-        break;
+    } else if constexpr (kLA) {
+      // ---------------------------------------------------------------- LA transform warps
+      const int tid = threadIdx.x - 192;  // 0..127
+      int stage = 0;
+      uint32_t phase = 0;
+      const int D = p.D;
+      for (int li = 0;; ++li) {
+        const long item = consumer_item(li);
+        if (item < 0) break;
+        const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
+        bool ok = true;
+        for (int tile = 0; tile < nf * n_tiles; ++tile) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * L::kStageBytes;
+          // relu over the K tile's token rows (elementwise, so the swizzle does not matter);
+          // rows past the frame's last token were zero-filled by the TMA load and stay zero
+          const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
+          const int valid = min(kRowsPerTile, p.N - (tile % n_tiles) * kRowsPerTile);
+  #pragma unroll 1
+          for (int kb = 0; kb < L::kOpBytes / kBoxBytes; ++kb) {
+            uint4* kt = reinterpret_cast<uint4*>(st + kb * kBoxBytes);
+            for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
+              uint4 x = kt[i];
+              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+  #pragma unroll
+              for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
+              kt[i] = x;
+            }
+          }
+          // ones column at index D of every V row (token), for the normaliser
+          *reinterpret_cast<__nv_bfloat16*>(st + L::kOpBytes +
+                                            swz128_offset_bf16(tid, D, kBoxBytes)) =
+              __float2bfloat16(1.0f);
+          fence_async_smem();
+          mbar_arrive(&ready[stage]);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) {
+          give_up(hf, abort_flag);
+          break;
+        }
       }
     }
-  }
 
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -414,15 +468,15 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
 
 // A_ws: [B*H*T, D, D] bf16 (GDN only). B_ws: [B*H*T, brows, D] f32, brows = D (GDN) or D+1 (LA),
 // row-major, or (kB4, GDN) each D x D matrix in the b4_index layout.
-template <int DP, bool kLA, bool kB4>
-__global__ void __launch_bounds__(StatsLayout<DP, kLA>::kThreads, 1)
+template <int DP, bool kLA, bool kB4, bool kF8 = false>
+__global__ void __launch_bounds__(StatsLayout<DP, kLA, kF8>::kThreads, 1)
     gdn_stats_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
                      float* __restrict__ B_ws, Problem p, int frames_per_item) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  stats_body<DP, kLA, false, kB4>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw),
-                                  frames_per_item);
+  stats_body<DP, kLA, false, kB4, kF8>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw),
+                                       frames_per_item);
 }
 
 }  // namespace gdn

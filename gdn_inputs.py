@@ -147,3 +147,17 @@ def workload_inputs(w: Workload, device="cpu", step: Optional[int] = None) -> di
                 "v": normal_bf16(shape, g, device), "state": None, "z": None}
     return clip_inputs(w.B, w.H, w.T, w.N, w.D, w.gamma_range, w.beta_range, seed=w.seed,
                        state_std=w.state_std, device=device)
+
+
+def quantize_e4m3(x):
+    """8-bit E4M3 codes of x [B, T, N, H, D] with one absmax scale per (batch, frame, head):
+    scale = max |x| / 448 over the frame's tokens and dims (1 for an all-zero slice), codes =
+    x / scale rounded to nearest even by torch's float8_e4m3fn conversion. Returns (uint8 codes
+    [B, T, N, H, D], f32 scales [B, T, H]) on x's device. This stands in for the projection
+    that would emit fp8 activations; it is input generation, not part of the layer."""
+    import torch
+    xf = x.float()
+    amax = xf.abs().amax(dim=(2, 4))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (xf / scale[:, :, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()

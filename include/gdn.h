@@ -89,6 +89,29 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
                              float key_scale, gdn_stream_t stream);
 
 /*
+ * gdn_frame_forward_fp8 - gdn_frame_forward on 8-bit E4M3 q, k, v with one scale per
+ * (batch, frame, head) (the SANA-Streaming entry of the jefxiong.cn AIGC digest, 2026-06-01,
+ * item 1, contribution (3): mixed-precision quantisation to keep the tensor cores busy; the
+ * pages give no quantiser, so the layer is defined on the dequantised values).
+ *
+ * q, k, v: [B, T, N, H, D] E4M3 codes (OCP 8-bit floating point, no infinities), device
+ * pointers; q_scale, k_scale, v_scale: [B, T, H] f32, so that q[b,t,n,h,:] = decode(q8) *
+ * q_scale[b,t,h] (likewise k, v). gamma, beta, state_in, out (bf16), state_out, key_scale: as
+ * gdn_frame_forward. The kernels convert the codes to bf16 in shared memory (exact) and apply
+ * the scales in their f32 epilogues (A gets key_scale^2 k_scale^2, B key_scale k_scale v_scale,
+ * O q_scale), so the result is the bf16 layer's on the dequantised inputs up to f32 rounding
+ * while q, k, v cost one byte per element to read.
+ * Supported head dims: 64 < D <= 128, D % 16 == 0 (GDN_ERR_UNSUPPORTED otherwise). The same
+ * path choice as gdn_frame_forward (fused, three kernels, chunked) and the same workspace.
+ */
+gdn_status gdn_frame_forward_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v,
+                                 const float* q_scale, const float* k_scale,
+                                 const float* v_scale, const float* gamma, const float* beta,
+                                 const float* state_in, gdn_bf16* out, float* state_out, int B,
+                                 int H, int T, int N, int D, float key_scale,
+                                 gdn_stream_t stream);
+
+/*
  * gdn_frame_forward_host - gdn_frame_forward on a clip held in HOST memory.
  * (No counterpart in the paper: a deployment variant for clips that do not stay on the GPU,
  * e.g. minute-long videos whose activations are kept in host memory between layers.)

@@ -13,7 +13,7 @@ HEADER = os.path.join(ROOT, "include", "gdn.h")
 def _declared_symbols():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -96,6 +96,20 @@ def test_forward_host_rejects_bad_arguments_on_the_host(lib):
     import torch
     if not torch.cuda.is_available():
         assert _fwd_host(lib, q=P + 2) == 5
+
+
+def test_forward_fp8_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_frame_forward_fp8
+    args = lambda D=128, qs=P + 0x50000, ks=0.1: (P, P + 0x10000, P + 0x20000, qs, P + 0x51000,
+                                                  P + 0x52000, P + 0x30000, P + 0x31000, None,
+                                                  P + 0x40000, None, 1, 2, 3, 16, D, ks, None)
+    assert f(*args(qs=None)) == 1
+    assert f(*args(D=64)) == 2      # fp8 path: 64 < D <= 128
+    assert f(*args(D=120)) == 2     # D % 16 != 0
+    assert f(*args(ks=0.0)) == 1
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*args()) == 5
 
 
 def test_valid_call_without_gpu_fails_loudly(lib):

@@ -360,6 +360,74 @@ def test_forward_host_matches_oracle(case):
     assert relf(f64(out), f64(od)) <= 3e-3 and relf(f64(st), f64(sd)) <= 3e-4
 
 
+# --------------------------------------------------------------------------- fp8 inputs
+
+
+def _fp8_clip(B, H, T, N, D, seed, with_state):
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=seed, state_std=0.3 if with_state else 0.0)
+    q8, sq = gdn_inputs.quantize_e4m3(x["q"])
+    k8, sk = gdn_inputs.quantize_e4m3(x["k"])
+    v8, sv = gdn_inputs.quantize_e4m3(x["v"])
+    return dict(q8=q8, k8=k8, v8=v8, sq=sq, sk=sk, sv=sv, gamma=x["gamma"], beta=x["beta"],
+                state=x["state"])
+
+
+def _fp8_oracle(c, ks):
+    return oracle.gdn_frame_forward_fp8(c["q8"].cpu().numpy(), c["k8"].cpu().numpy(),
+                                        c["v8"].cpu().numpy(), f64(c["sq"]), f64(c["sk"]),
+                                        f64(c["sv"]), f64(c["gamma"]), f64(c["beta"]),
+                                        None if c["state"] is None else f64(c["state"]), ks)
+
+
+FP8_SHAPES = [
+    # (B, H, T, N, D, with_state)
+    (1, 2, 5, 200, 128, True),
+    (2, 3, 4, 129, 112, False),   # ragged tail, padded head dim
+    (1, 1, 3, 64, 80, True),
+    (1, 2, 20, 33, 96, True),
+    (1, 1, 1, 880, 128, False),   # one frame
+]
+
+
+@pytest.mark.parametrize("forward_mode", [1, 2, 3], indirect=True, ids=["split", "fused", "chunked"])
+@pytest.mark.parametrize("shape", FP8_SHAPES, ids=lambda s: "B%dH%dT%dN%dD%d%s" % (s[:5] + ("s" if s[5] else "",)))
+def test_fp8_forward_matches_oracle(shape, forward_mode):
+    """E4M3 q, k, v with per-(frame, head) scales against the oracle on the decoded values."""
+    B, H, T, N, D, with_state = shape
+    c = _fp8_clip(B, H, T, N, D, seed=600 + N + D, with_state=with_state)
+    ks = 1.0 / math.sqrt(D * N)
+    g = to_cuda(c)
+    out, st = api().gdn_frame_forward_fp8(g["q8"], g["k8"], g["v8"], g["sq"], g["sk"], g["sv"],
+                                          g["gamma"], g["beta"], g["state"], key_scale=ks)
+    assert api().gdn_sync_status() == 0
+    o_ref, s_ref = _fp8_oracle(c, ks)
+    eo, es = relf(f64(out), o_ref), relf(f64(st), s_ref)
+    assert eo <= O_TOL and es <= S_TOL, f"O err {eo:.2e}, S err {es:.2e}"
+
+
+def test_fp8_720p_sampled_heads():
+    """The 720p clip quantised to E4M3 (per frame and head), in the launch configuration of the
+    benchmark's fp8 line; the oracle recomputes two heads over all 961 frames."""
+    w = gdn_inputs.WORKLOADS["720p"]
+    x = gdn_inputs.workload_inputs(w, device="cuda")
+    c = {}
+    for n in ("q", "k", "v"):
+        c[n + "8"], c["s" + n] = gdn_inputs.quantize_e4m3(x[n])
+    del x["q"], x["k"], x["v"]
+    out, st = api().gdn_frame_forward_fp8(c["q8"], c["k8"], c["v8"], c["sq"], c["sk"], c["sv"],
+                                          x["gamma"], x["beta"], None, key_scale=w.key_scale)
+    assert api().gdn_sync_status() == 0
+    for h in (0, w.H - 1):
+        sl = lambda t: t[:, :, :, h:h + 1].contiguous().cpu().numpy()
+        sc = lambda t: f64(t[:, :, h:h + 1])
+        o_ref, s_ref = oracle.gdn_frame_forward_fp8(
+            sl(c["q8"]), sl(c["k8"]), sl(c["v8"]), sc(c["sq"]), sc(c["sk"]), sc(c["sv"]),
+            f64(x["gamma"][:, :, h:h + 1]), f64(x["beta"][:, :, h:h + 1]), None, w.key_scale)
+        eo = relf(_head_slice(out, 0, h), o_ref)
+        es = relf(f64(st[0, h]), s_ref[0, 0])
+        assert eo <= O_TOL and es <= S_TOL, f"head {h}: O err {eo:.2e}, S err {es:.2e}"
+
+
 STEP_SHAPES = [
     # (B, H, N, D, with_state)
     (2, 3, 100, 128, True),
