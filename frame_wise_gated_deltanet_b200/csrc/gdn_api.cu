@@ -85,6 +85,15 @@ bool tmap_tokens_f8(CUtensorMap* m, const void* base, const Problem& p) {
   return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box);
 }
 
+// q/k/v/out [B, T, N, H, D] bf16 as flattened token rows -> 3-D map (D, H, B*T*N), box
+// 64 x 1 x 128 (block-causal LA: a block's frames are consecutive rows).
+bool tmap_rows(CUtensorMap* m, const void* base, const Problem& p) {
+  const cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.H, (cuuint64_t)p.B * p.T * p.N};
+  const cuuint64_t strides[2] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.H * p.D * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box);
+}
+
 // Token map of q, k or v in the element type of the path.
 template <bool kF8>
 bool tmap_in(CUtensorMap* m, const void* base, const Problem& p) {
@@ -285,7 +294,11 @@ gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws
   using L = gdn::OutputLayout<DP, kLA, 4, kF8>;
   const long count = long(p.B) * p.H * ((p.T + F - 1) / F);  // stored states (per block for LA)
   CUtensorMap tq, ts, to;
-  if (!tmap_in<kF8>(&tq, q, p) || !tmap_tokens(&to, out, p)) return GDN_ERR_CUDA;
+  if (kLA) {
+    if (!tmap_rows(&tq, q, p) || !tmap_rows(&to, out, p)) return GDN_ERR_CUDA;
+  } else if (!tmap_in<kF8>(&tq, q, p) || !tmap_tokens(&to, out, p)) {
+    return GDN_ERR_CUDA;
+  }
   if (kLA) {
     if (!tmap_mats(&ts, S_ws, false, p.D, srows, count, DP)) return GDN_ERR_CUDA;
   } else {
@@ -295,12 +308,13 @@ gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws
   if (gdn_status s = ensure_smem_attr(dev, kF8 ? 16 : (kLA ? 6 : (DP == 128 ? 4 : 5)), kern,
                                       L::kSmemBytes))
     return s;
-  const long items = long(p.B) * p.T * p.H;
+  const long items = long(p.B) * (kLA ? (p.T + F - 1) / F : p.T) * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
   {
     ProfiledLaunch pl("gdn_output_kernel", st);
     kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(
-        tq, ts, static_cast<const __nv_bfloat16*>(S_ws), to, p, F);
+        tq, ts, static_cast<const __nv_bfloat16*>(S_ws), to, p, F,
+        static_cast<__nv_bfloat16*>(out));
   }
   return check_launch();
 }
@@ -1000,6 +1014,8 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
   if (!q || !k || !v || !out) return GDN_ERR_INVALID_ARG;
   if (frames_per_block < 1) return GDN_ERR_INVALID_ARG;
   if (gdn_status s = check_sizes(B, H, T, N, D, 120)) return s;
+  // token rows are addressed as one flattened TMA coordinate
+  if (double(B) * T * N >= 2147483647.0) return GDN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GDN_ERR_MISALIGNED;
   const size_t n = size_t(B) * T * N * H * D * 2;
   if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
@@ -1023,7 +1039,7 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
     // per-block statistics: one item per (batch, block, head)
     using L = gdn::StatsLayout<128, true>;
     CUtensorMap tk, tv;
-    if (!tmap_tokens(&tk, k, p) || !tmap_tokens(&tv, v, p)) return GDN_ERR_CUDA;
+    if (!tmap_rows(&tk, k, p) || !tmap_rows(&tv, v, p)) return GDN_ERR_CUDA;
     auto kern = gdn::gdn_stats_kernel<128, true, false>;
     if (gdn_status s = ensure_smem_attr(dev, 7, kern, L::kSmemBytes)) return s;
     const int grid = static_cast<int>(count < g_dev[dev].sms ? count : g_dev[dev].sms);

@@ -22,8 +22,9 @@
 // (LA only) 4 transform warps. The epilogue sets the pace of a tile (TMEM read-out, bf16
 // conversion, staging): with G = 1 a tile took about 1.7 us per SM, under the HBM share.
 //
-// Standalone (gdn_output_kernel): work item i = (b*T + t)*H + h, S_t at workspace row
-// (b*H+h)*T + t_state. Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h
+// Standalone (gdn_output_kernel): GDN work item i = (b*T + t)*H + h, S_t at workspace row
+// (b*H+h)*T + t; LA work item i = (b*n_blocks + j)*H + h, a block of frames over the flattened
+// token rows, its state at row (b*H+h)*n_blocks + j. Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h
 // (frame-major), S_t loaded from ring row (b*H+h)*Rs + t%Rs once chain_prog says it is there;
 // out_flag releases the slot as soon as S_t is in shared memory.
 #pragma once
@@ -53,12 +54,34 @@ struct OutputLayout {
 
 struct OutputItem {
   int h, bt, bh, t;
+  int n_tiles;  // 128-row tiles of the item
+  int rows;     // token rows of the item (LA: all frames of its block)
+  int row0;     // LA: first row in the flattened (b, t, n) token space of the 3-D maps
+  long srow;    // LA: row of the block's state
 };
 
-template <bool kFused>
-__device__ __forceinline__ OutputItem output_item(long item, const Problem& p) {
+// GDN items are frames (b, t, h); LA items are blocks (b, j, h) of F frames, whose N*F rows are
+// contiguous in the flattened token space, so their tiles span frames (10 tiles of 128 rows for
+// 3 frames of 390 tokens instead of 3 x 4).
+template <bool kFused, bool kLA = false>
+__device__ __forceinline__ OutputItem output_item(long item, const Problem& p, int F = 1) {
   OutputItem it;
-  if constexpr (kFused) {
+  it.rows = p.N;
+  it.row0 = 0;
+  it.srow = 0;
+  if constexpr (kLA) {
+    const int nblk = (p.T + F - 1) / F;
+    it.h = static_cast<int>(item % p.H);
+    const int bj = static_cast<int>(item / p.H);
+    const int b = bj / nblk;
+    const int j = bj - b * nblk;
+    it.t = j * F;
+    it.bt = b * p.T + it.t;
+    it.bh = b * p.H + it.h;
+    it.rows = min(F, p.T - it.t) * p.N;
+    it.row0 = it.bt * p.N;
+    it.srow = static_cast<long>(it.bh) * nblk + j;
+  } else if constexpr (kFused) {
     const int BH = p.B * p.H;
     it.t = static_cast<int>(item / BH);
     it.bh = static_cast<int>(item - static_cast<long>(it.t) * BH);
@@ -72,18 +95,22 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p) {
     it.t = it.bt - b * p.T;
     it.bh = b * p.H + it.h;
   }
+  it.n_tiles = (it.rows + kRowsPerTile - 1) / kRowsPerTile;
   return it;
 }
 
 // frames_per_block: 1 for GDN (frame t reads S_t); F for LA (frame t reads the state at the end
 // of its block of F frames). GDN states come from S_src (DP*DP bf16 per row, s8 layout); LA
 // states through tm_s.
+// LA: tm_q and tm_o are 3-D maps over the flattened token rows, and out (the raw output) takes
+// the row stores of a block's last, partial tile (a 128-row TMA store would also overwrite the
+// first rows of the next block, which another CTA writes).
 template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
                                             const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
-                                            uint8_t* smem) {
+                                            uint8_t* smem, __nv_bfloat16* out = nullptr) {
   using L = OutputLayout<DP, kLA, kG, kF8>;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                          // 2 state buffers
@@ -103,9 +130,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const long n_items = static_cast<long>(p.B) * p.T * p.H;
-  const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
   const int F = frames_per_block;
+  const long n_items = static_cast<long>(p.B) * (kLA ? (p.T + F - 1) / F : p.T) * p.H;
   const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
   const long ncta = kFused ? hf.count : gridDim.x;
   // item li of this CTA: standalone a static stride, fused the role's work counter. Returns -1
@@ -160,7 +186,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       for (int li = 0; !*abort_flag; ++li) {
         const long item = producer_item(li);
         if (item < 0) break;
-        const OutputItem it = output_item<kFused>(item, p);
+        const OutputItem it = output_item<kFused, kLA>(item, p, F);
         int srow;
         if constexpr (kFused) {
           srow = it.bh * hf.Rs + it.t % hf.Rs;
@@ -192,13 +218,19 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
                     L::kSBufBytes, &s_full[sb], pol_state);
         }
         s_fills.filled(sb, (li >> 1) & 1);
-        for (int tile = 0; tile < n_tiles; ++tile) {
+        for (int tile = 0; tile < it.n_tiles; ++tile) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
             give_up(hf, abort_flag);
             break;
           }
           mbar_arrive_expect_tx(&full[stage], L::kQLoadBytes);
-          if constexpr (kF8) {
+          if constexpr (kLA) {
+            // 128 flattened token rows (they may run into the next frame of the block)
+#pragma unroll
+            for (int kb = 0; kb < L::kBoxes; ++kb)
+              tma_load_3d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
+                          kb * 64, it.h, it.row0 + tile * kRowsPerTile, pol_stream);
+          } else if constexpr (kF8) {
             // one 128-byte-wide e4m3 box, into the stage's second bf16 box
             tma_load_4d(q_ring + stage * L::kQBytes + kBoxBytes, tm_q, &full[stage], 0, it.h,
                         tile * kRowsPerTile, it.bt, pol_stream);
@@ -234,13 +266,13 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         ok = false;
         break;
       }
+      const OutputItem it = output_item<kFused, kLA>(item, p, F);
       if constexpr (kFused) {
         // S_t is in shared memory: its ring slot may be overwritten by the chain
-        const OutputItem it = output_item<kFused>(item, p);
         if (lane == 0) st_release(hf.out_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
       }
       const uint32_t s_base = smem_u32(s_buf + sb * L::kSBufBytes);
-      for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
+      for (int tile = 0; tile < it.n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
         if (!mbar_wait(&acc_empty[acc], ((tc >> 1) & 1) ^ 1) ||
             !mbar_wait(L::kTransform ? &ready[stage] : &full[stage], phase)) {
@@ -297,9 +329,13 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       if constexpr (kFused) lost = named_bar_any(1, kEpiThreads, lost);  // uniform across the epilogue
       if (lost) ok = false;
       if (lost || item < 0) break;
-      const OutputItem it = output_item<kFused>(item, p);
-      for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
+      const OutputItem it = output_item<kFused, kLA>(item, p, F);
+      for (int tile = 0; tile < it.n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
+        const int valid = min(kRowsPerTile, it.rows - tile * kRowsPerTile);
+        // LA: a block's last tile runs into the next block's rows, so its valid rows are stored
+        // row by row instead of through the TMA box
+        const bool row_stores = kLA && valid < kRowsPerTile;
         const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
         // staging buffer tc&1 is free once the store issued two tiles ago has read it
         if (leader) bulk_wait_read<1>();
@@ -308,10 +344,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           break;
         }
         tc_fence_after();
-        // warps whose 32 rows are all past the frame's last token skip the read-out: the TMA
-        // store clips at N, so their staging rows are never written to memory
+        // warps whose 32 rows are all past the item's last token skip the read-out: the TMA
+        // store clips at N (GDN), and LA stores such tiles row by row
         uint8_t* ob = o_stage + (tc & 1) * L::kOBytes;
-        if (static_cast<int>(quarter) * 32 < p.N - tile * kRowsPerTile) {
+        if (static_cast<int>(quarter) * 32 < valid) {
           const uint32_t tacc = lane_base + acc * DP;
           float scale = 1.f;
           if constexpr (kLA) scale = 1.f / (tmem_ld1(tacc + D) + 1e-6f);  // normaliser, column D
@@ -330,7 +366,14 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
               pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
               pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
               pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
-              *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c + j, kBoxBytes)) = pk;
+              if (row_stores) {
+                if (row < valid && c + j < D)
+                  *reinterpret_cast<uint4*>(
+                      out + (static_cast<long>(it.row0 + tile * kRowsPerTile + row) * p.H + it.h) *
+                                D + c + j) = pk;
+              } else {
+                *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c + j, kBoxBytes)) = pk;
+              }
             }
           }
         }
@@ -338,11 +381,16 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         mbar_arrive(&acc_empty[acc]);
         fence_async_smem();
         named_bar(1, kEpiThreads);
-        if (leader) {
+        if (leader && !row_stores) {
 #pragma unroll
-          for (int kb = 0; kb < L::kBoxes; ++kb)
-            tma_store_4d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h, tile * kRowsPerTile, it.bt,
-                         pol_out);
+          for (int kb = 0; kb < L::kBoxes; ++kb) {
+            if constexpr (kLA)
+              tma_store_3d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h,
+                           it.row0 + tile * kRowsPerTile, pol_out);
+            else
+              tma_store_4d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h, tile * kRowsPerTile, it.bt,
+                           pol_out);
+          }
           bulk_commit();
         }
       }
@@ -360,6 +408,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       for (int li = 0; ok; ++li) {
         const long item = consumer_item(li);
         if (item < 0) break;
+        const int n_tiles = output_item<kFused, kLA>(item, p, F).n_tiles;
         for (int tile = 0; tile < n_tiles; ++tile) {
           if (!mbar_wait(&full[stage], phase)) {
             ok = false;
@@ -384,14 +433,16 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       for (int li = 0; ok; ++li) {
         const long item = consumer_item(li);
         if (item < 0) break;
-        for (int tile = 0; tile < n_tiles; ++tile) {
+        const OutputItem it = output_item<kFused, kLA>(item, p, F);
+        for (int tile = 0; tile < it.n_tiles; ++tile) {
           if (!mbar_wait(&full[stage], phase)) {
             ok = false;
             break;
           }
           const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
-          // rows past the frame's last token were zero-filled by the TMA load: relu keeps them
-          const int valid = min(kRowsPerTile, p.N - tile * kRowsPerTile);
+          // rows past the block's last token belong to other blocks: their outputs are not
+          // stored, so they need no relu
+          const int valid = min(kRowsPerTile, it.rows - tile * kRowsPerTile);
   #pragma unroll 1
           for (int kb = 0; kb < L::kBoxes; ++kb) {
             uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes + kb * kBoxBytes);
@@ -428,11 +479,12 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA, 4, kF8>::kThreads, 1)
     gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_s,
                       const __nv_bfloat16* __restrict__ S_src,
-                      const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block) {
+                      const __grid_constant__ CUtensorMap tm_o, Problem p, int frames_per_block,
+                      __nv_bfloat16* out) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
   output_body<DP, kLA, false, 4, kF8>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
-                                      align1k(smem_raw));
+                                      align1k(smem_raw), out);
 }
 
 }  // namespace gdn

@@ -18,8 +18,9 @@
 //               tiles are TMA-loaded into the second box of each bf16 operand tile)
 //
 // Standalone (gdn_stats_kernel): work item i = (b*T + t)*H + h, results at workspace row
-// (b*H + h)*T + t; for LA an item is a block of frames_per_item frames (its statistics summed),
-// results at row (b*H + h)*n_blocks + block. Fused (stats role of gdn_fused_kernel): work item i = t*B*H + (b*H + h)
+// (b*H + h)*T + t; for LA an item is a block of frames_per_item frames (its statistics summed
+// over its token rows, read through 3-D maps of the flattened (b, t, n) rows so that tiles span
+// frames), results at row (b*H + h)*n_blocks + block. Fused (stats role of gdn_fused_kernel): work item i = t*B*H + (b*H + h)
 // (frame-major, so the chain finds early frames first), results at ring row (b*H+h)*R + t%R,
 // written only after the chain has released that slot, then published with stats_flag.
 #pragma once
@@ -105,6 +106,11 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
   const uint32_t lane = lane_id();
   const long n_items = static_cast<long>(p.B) * ((p.T + fpb - 1) / fpb) * p.H;
   const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
+  // tiles of an item of nf frames: LA items are blocks whose nf*N token rows are contiguous in
+  // the flattened (b, t, n) rows of its 3-D maps, so its tiles span frames
+  auto item_tiles = [&](int nf) {
+    return kLA ? (nf * p.N + kRowsPerTile - 1) / kRowsPerTile : nf * n_tiles;
+  };
   const long cta0 = kFused ? blockIdx.x - hf.base : blockIdx.x;
   const long ncta = kFused ? hf.count : gridDim.x;
   // item li of this CTA: standalone a static stride, fused the role's work counter. Returns -1
@@ -157,7 +163,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
         const long item = producer_item(li);
         if (item < 0) break;
         const StatsItem it = stats_item<kFused>(item, p, hf, fpb);
-        for (int ft = 0; ft < it.nf * n_tiles; ++ft) {
+        for (int ft = 0; ft < item_tiles(it.nf); ++ft) {
           const int tile = ft % n_tiles;
           const int bt = it.bt + ft / n_tiles;
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
@@ -166,7 +172,17 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
           }
           mbar_arrive_expect_tx(&full[stage], L::kLoadBytes);
           uint8_t* st = smem + stage * L::kStageBytes;
-          if constexpr (kF8) {
+          if constexpr (kLA) {
+            // 128 flattened token rows from the block's first row (they may cross frames; rows
+            // past the block are zeroed in K by the transform warps)
+            const int row = it.bt * p.N + ft * kRowsPerTile;
+#pragma unroll
+            for (int j = 0; j < L::kBoxes; ++j) {
+              tma_load_3d(st + j * kBoxBytes, tm_k, &full[stage], j * 64, it.h, row, pol);
+              tma_load_3d(st + L::kOpBytes + j * kBoxBytes, tm_v, &full[stage], j * 64, it.h,
+                          row, pol);
+            }
+          } else if constexpr (kF8) {
             // one 128-byte-wide e4m3 box per operand, into its second bf16 box
             tma_load_4d(st + kBoxBytes, tm_k, &full[stage], 0, it.h, tile * kRowsPerTile, bt,
                         pol);
@@ -214,7 +230,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       const uint32_t d = tmem_base + acc * L::kAccCols;
       const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
       bool ok = true;
-      for (int tile = 0; tile < nf * n_tiles; ++tile) {
+      for (int tile = 0; tile < item_tiles(nf); ++tile) {
         if (!mbar_wait(L::kTransform ? &ready[stage] : &full[stage], phase)) {
           ok = false;
           break;
@@ -418,25 +434,26 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
         if (item < 0) break;
         const int nf = stats_item<kFused>(item, p, hf, fpb).nf;
         bool ok = true;
-        for (int tile = 0; tile < nf * n_tiles; ++tile) {
+        for (int tile = 0; tile < item_tiles(nf); ++tile) {
           if (!mbar_wait(&full[stage], phase)) {
             ok = false;
             break;
           }
           uint8_t* st = smem + stage * L::kStageBytes;
           // relu over the K tile's token rows (elementwise, so the swizzle does not matter);
-          // rows past the frame's last token were zero-filled by the TMA load and stay zero
+          // rows past the block's last token hold other blocks' keys (or zero fill past the
+          // tensor) and are zeroed, so they add nothing to the block's sums
           const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
-          const int valid = min(kRowsPerTile, p.N - (tile % n_tiles) * kRowsPerTile);
-  #pragma unroll 1
+          const int valid = min(kRowsPerTile, nf * p.N - tile * kRowsPerTile);
+#pragma unroll 1
           for (int kb = 0; kb < L::kOpBytes / kBoxBytes; ++kb) {
             uint4* kt = reinterpret_cast<uint4*>(st + kb * kBoxBytes);
-            for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
+            for (int i = tid; i < kRowsPerTile * 8; i += 128) {  // 8 x 16 B per 128-byte row
               uint4 x = kt[i];
               __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
-  #pragma unroll
+#pragma unroll
               for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-              kt[i] = x;
+              kt[i] = (i >> 3) < valid ? x : make_uint4(0u, 0u, 0u, 0u);
             }
           }
           // ones column at index D of every V row (token), for the normaliser
