@@ -150,11 +150,12 @@ def ncu_traffic(kernel, workload):
     try:
         with open(path) as f:
             t = json.load(f)
-        e = t["kernels"][kernel]
-        if e.get("source_digest") != source_digest(kernel) or e.get("workload") != workload:
-            return None
-        return float(e["dram_bytes_per_launch"])
-    except (OSError, KeyError, ValueError):
+        entries = t["kernels"][kernel]
+        for e in entries if isinstance(entries, list) else [entries]:
+            if e.get("source_digest") == source_digest(kernel) and e.get("workload") == workload:
+                return float(e["dram_bytes_per_launch"])
+        return None
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
