@@ -262,6 +262,8 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
             // has acquired; the GPU-scope release makes them visible to the outputs (which
             // fence the async proxy after their acquire)
             st_release(hf.chain_prog + bh, done);
+            for (int f = published; f < done; ++f)  // queue the frames for the outputs
+              st_release(hf.ready_items + atomicAdd(hf.ready_tail, 1), f * p.B * p.H + bh + 1);
             published = done;
             t0 = globaltimer_ns();
             continue;

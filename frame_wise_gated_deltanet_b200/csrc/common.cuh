@@ -40,6 +40,11 @@ struct Handoff {
   int withhold;     // test hook: frame whose statistics of head 0 are never published (-1: none)
   int base;         // first blockIdx.x of this role
   int count;        // CTAs in this role
+  // outputs in publish order: the chain appends item t*B*H + bh (+1) at ready_items[ready_tail++]
+  // as soon as S_t is visible, and output CTAs take queue positions from next_item, so an output
+  // CTA only waits when no published state is left anywhere (not on one lagging head)
+  int* ready_items = nullptr;  // [B*H*T], 0 = not yet written
+  int* ready_tail = nullptr;
 };
 
 // Dynamic work distribution inside a CTA of the fused forward: the producer thread takes the
@@ -53,6 +58,17 @@ struct ItemRing {
   __device__ __forceinline__ long produce(int li, int* counter, long n_items) {
     long it = atomicAdd(counter, 1);
     if (it >= n_items) it = -1;
+    ids[li & 7] = static_cast<int>(it);
+    mbar_arrive(&bars[li & 7]);
+    return it;
+  }
+  // Same, with the item taken from a queue of published items: queue position from the counter,
+  // then (bounded) wait until that position is written. -2 if the wait ran out.
+  __device__ __forceinline__ long produce_queued(int li, int* counter, const int* queue,
+                                                 long n_items, const int* abort) {
+    const long pos = atomicAdd(counter, 1);
+    long it = -1;
+    if (pos < n_items) it = wait_flag_ge(queue + pos, 1, abort) ? ld_acquire(queue + pos) - 1 : -2;
     ids[li & 7] = static_cast<int>(it);
     mbar_arrive(&bars[li & 7]);
     return it;

@@ -351,8 +351,10 @@ ForwardWs carve_forward(void* base, long count, int D) {
 int g_forward_mode = 0;
 
 // Tuning of the fused forward, read once from the environment:
-//   GDN_FUSED_RING       A_t / B_t ring slots per head (default 24, 4..64)
-//   GDN_FUSED_SRING      S_t ring slots per head (default 32, 8..64)
+//   GDN_FUSED_RING       A_t / B_t ring slots per head (default 8, 4..64)
+//   GDN_FUSED_SRING      S_t ring slots per head (default 16, 8..64)
+// (with the outputs' publish-order queue, rings of 8 / 16 frames measured fastest on every box
+// tried; deeper rings only grow the L2 working set)
 //   GDN_FUSED_STATS_PCT  share of the non-chain SMs given to the stats role (default 54, 20..80)
 }  // namespace
 
@@ -364,11 +366,11 @@ int env_int(const char* name, int dflt, int lo, int hi) {
   return v < lo ? lo : (v > hi ? hi : v);
 }
 int fused_ring() {
-  static const int r = env_int("GDN_FUSED_RING", 24, 4, 64);
+  static const int r = env_int("GDN_FUSED_RING", 8, 4, 64);
   return r;
 }
 int fused_sring() {
-  static const int r = env_int("GDN_FUSED_SRING", 32, 8, 64);
+  static const int r = env_int("GDN_FUSED_SRING", 16, 8, 64);
   return r;
 }
 int fused_stats_pct() {
@@ -380,7 +382,8 @@ struct FusedWs {
   void* A;
   float* B;
   void* S;
-  int* flags;  // stats_flag [BH*T], out_flag [BH*T], chain_prog [BH], abort, 2 work counters
+  int* flags;  // stats_flag [BH*T], out_flag [BH*T], chain_prog [BH], abort, 2 work counters,
+               // ready_tail, ready_items [BH*T] (the outputs' queue)
   size_t flag_bytes;
 };
 
@@ -388,7 +391,7 @@ size_t fused_ws_bytes(long bh, long T, int D) {
   const int kRing = fused_ring();
   const size_t m = size_t(D) * D * bh * kRing;
   const size_t dp = padded_dim(D), ms = dp * dp * bh * fused_sring();
-  const size_t flags = sizeof(int) * (2 * bh * T + bh + 3);
+  const size_t flags = sizeof(int) * (3 * bh * T + bh + 4);
   return align256(m * 2) + align256(m * 4) + align256(ms * 2) + align256(flags);
 }
 
@@ -405,7 +408,7 @@ FusedWs carve_fused(void* base, long bh, long T, int D) {
   w.S = p;
   p += align256(ms * 2);
   w.flags = reinterpret_cast<int*>(p);
-  w.flag_bytes = sizeof(int) * (2 * bh * T + bh + 3);
+  w.flag_bytes = sizeof(int) * (3 * bh * T + bh + 4);
   return w;
 }
 
@@ -456,6 +459,8 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   static const int withhold = env_int("GDN_TEST_WITHHOLD_FRAME", -1, -1, 1 << 30);
   gdn::Handoff hc{f, f + ft, f + 2 * ft, abort_word, nullptr, kRing, fused_sring(), withhold,
                   0, bh};
+  hc.ready_tail = abort_word + 3;
+  hc.ready_items = abort_word + 4;
   gdn::Handoff hs = hc;
   hs.base = bh;
   hs.count = n_stats;

@@ -24,9 +24,11 @@
 //
 // Standalone (gdn_output_kernel): GDN work item i = (b*T + t)*H + h, S_t at workspace row
 // (b*H+h)*T + t; LA work item i = (b*n_blocks + j)*H + h, a block of frames over the flattened
-// token rows, its state at row (b*H+h)*n_blocks + j. Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h
-// (frame-major), S_t loaded from ring row (b*H+h)*Rs + t%Rs once chain_prog says it is there;
-// out_flag releases the slot as soon as S_t is in shared memory.
+// token rows, its state at row (b*H+h)*n_blocks + j.
+// Fused (output role of gdn_fused_kernel): work item i = t*B*H + b*H + h, taken in the order the
+// chains published them (a queue the chain CTAs append to), S_t loaded from ring row
+// (b*H+h)*Rs + t%Rs (chain_prog is checked again); out_flag releases the slot as soon as S_t
+// is in shared memory.
 #pragma once
 #include <cuda.h>
 
@@ -137,7 +139,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   // item li of this CTA: standalone a static stride, fused the role's work counter. Returns -1
   // when there are no more items, -2 on a timed-out wait.
   auto producer_item = [&](int li) -> long {
-    if constexpr (kFused) return ring.produce(li, hf.next_item, n_items);
+    if constexpr (kFused)
+      return ring.produce_queued(li, hf.next_item, hf.ready_items, n_items, hf.abort);
     const long it = cta0 + static_cast<long>(li) * ncta;
     return it < n_items ? it : -1;
   };

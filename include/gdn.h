@@ -39,7 +39,7 @@
  * Environment (read once per process unless stated):
  *  - GDN_WAIT_LIMIT_MS: limit of every device-side bounded wait (default 4000).
  *  - GDN_FUSED_RING, GDN_FUSED_SRING, GDN_FUSED_STATS_PCT: ring depths of the fused forward's
- *    A_t/B_t and S_t hand-off (default 24 and 32 frames per head) and the share of the non-chain
+ *    A_t/B_t and S_t hand-off (default 8 and 16 frames per head) and the share of the non-chain
  *    SMs given to the statistics role (default 54 %).
  *  - GDN_CHUNK_LEN: frames per chunk of the chunked forward (read on every call; 0 or unset:
  *    chosen per problem).
