@@ -280,9 +280,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-__device__ __forceinline__ void fence_acq_rel_gpu() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
 
 // Generic-proxy writes to shared memory -> visible to the async proxy (TMA, tcgen05.mma).
 __device__ __forceinline__ void fence_async_smem() {
@@ -423,9 +420,6 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // ------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 format (version 1).
@@ -476,14 +470,6 @@ __device__ __forceinline__ uint32_t swz128_offset_bf16(uint32_t r, uint32_t c,
   return blk * block_bytes + r * 128u + chunk * 16u + (cc & 7) * 2u;
 }
 
-// Same for fp32 data with 128 B rows (32 floats) and 32-column blocks `block_bytes` apart.
-__device__ __forceinline__ uint32_t swz128_offset_f32(uint32_t r, uint32_t c,
-                                                      uint32_t block_bytes) {
-  const uint32_t blk = c >> 5;
-  const uint32_t cc = c & 31;
-  const uint32_t chunk = (cc >> 2) ^ (r & 7);
-  return blk * block_bytes + r * 128u + chunk * 16u + (cc & 3) * 4u;
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

@@ -11,7 +11,7 @@
 // Warp roles (one CTA per SM, persistent over work items):
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one elected thread)
-//   warps 2..5  epilogue: TMEM -> registers -> scale -> global
+//   warps 2..5  epilogue: TMEM -> registers -> scale -> global (LA: per-block sums)
 //   warps 6..   (LA and fp8 only) in-place transform of each K/V stage: relu(K) and a ones
 //               column in V (LA, warps 6..9), or e4m3 -> bf16 conversion of K and V (fp8
 //               inputs, DP = 128, warps 6..13, one token row of K or V per thread: the fp8
