@@ -174,6 +174,10 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
  * the usual streaming call). Equivalent to gdn_frame_forward with T = 1 (the chunk-causal and
  * distilled autoregressive inference modes advance the state one latent frame at a time:
  * gen-hub.ru SANA-WM article, section "Три режима на любой вкус").
+ * For 64 < D <= 128 (and forward mode != 1) one cooperative launch of the step kernel does the
+ * whole step in one pass over q, k, v and the state (statistics units and output units taken
+ * dynamically); other head dims use the three-kernel path with T = 1. The step kernel keeps a
+ * few per-GPU hand-off words (allocated once, zero-initialised) in addition to the workspace.
  */
 gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
                           const float* gamma, const float* beta, const float* state_in,
