@@ -473,13 +473,17 @@ def measure_e2e(a, w, g, out, st, stream, world, dev):
     host inputs and outputs: every step copies q, k, v, gamma, beta in and out, state out."""
     import torch
     from frame_wise_gated_deltanet_b200 import api
+    # every rank takes the same decision (a rank that skipped would leave the others waiting
+    # in the collectives below)
+    short = 0.0
     try:
         import psutil
         need = sum(t.numel() * t.element_size() for t in (g["q"], g["k"], g["v"], out))
-        if psutil.virtual_memory().available < 1.5 * need * world:
-            return {"value": None, "unit": UNIT, "reason": "not enough host memory to pin"}
+        short = 1.0 if psutil.virtual_memory().available < 1.5 * need * world else 0.0
     except ImportError:
         pass
+    if max_over_ranks(short, world) > 0:
+        return {"value": None, "unit": UNIT, "reason": "not enough host memory to pin"}
     host = {n: torch.empty(g[n].shape, dtype=g[n].dtype, pin_memory=True)
             for n in ("q", "k", "v", "gamma", "beta")}
     for n in host:
