@@ -381,7 +381,8 @@ def main():
     for _ in range(max(a.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    if api.gdn_sync_status() != 0:
+    # status checks are collective, so that every rank stops together
+    if max_over_ranks(float(api.gdn_sync_status() != 0), world) > 0:
         raise RuntimeError("device status error during warm-up")
 
     # per-launch events the library records around each kernel (created before arming)
@@ -411,8 +412,8 @@ def main():
     _lib.LIB.gdn_profile_arm(None, 0)
     barrier(world)
     status = api.gdn_sync_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
+    if max_over_ranks(float(status != 0), world) > 0:
+        raise RuntimeError(f"device status {status} after the timed region (this rank)")
 
     ms_local = t_start.elapsed_time(t_end)
     value, ms = job_throughput(w.tokens_heads * a.steps, ms_local, world)
@@ -498,7 +499,7 @@ def measure_e2e(a, w, g, out, st, stream, world, dev):
 
     e2e_step()
     torch.cuda.synchronize()
-    if api.gdn_sync_status(stream) != 0:
+    if max_over_ranks(float(api.gdn_sync_status(stream) != 0), world) > 0:
         raise RuntimeError("device status error in the end-to-end leg")
     steps = max(1, a.e2e_steps)
     s0 = torch.cuda.Event(enable_timing=True)
