@@ -25,7 +25,9 @@ def _rank(rank, world, port, q):
                             world_size=world, timeout=datetime.timedelta(seconds=60))
     ms_local = 10.0 * (rank + 1)  # rank 1 is the slow one
     value, ms = bench.job_throughput(1000, ms_local, world, device="cpu")
-    q.put((rank, value, ms))
+    # a decision one rank takes (e.g. "skip the end-to-end leg", "device error") reaches all
+    flag = bench.max_over_ranks(1.0 if rank == 1 else 0.0, world, device="cpu")
+    q.put((rank, value, ms, flag))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -42,9 +44,10 @@ def test_job_throughput_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, value, ms in res:
+    for rank, value, ms, flag in res:
         assert ms == pytest.approx(20.0)                    # the slowest rank's time
         assert value == pytest.approx(2 * 1000 / 20e-3)     # units of all ranks / that time
+        assert flag == 1.0                                  # every rank sees rank 1's decision
 
 
 def test_single_rank_needs_no_collective():
