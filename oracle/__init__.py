@@ -10,6 +10,8 @@ from .gdn_oracle import (  # noqa: F401
     frame_output,
     frame_statistics,
     frame_update,
+    frame_update_backward,
+    gdn_frame_backward,
     gdn_frame_forward,
     gdn_frame_forward_fp8,
     gdn_frame_step,

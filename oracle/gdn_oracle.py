@@ -52,6 +52,8 @@ __all__ = [
     "frame_statistics",
     "frame_update",
     "frame_output",
+    "frame_update_backward",
+    "gdn_frame_backward",
     "gdn_frame_forward",
     "gdn_frame_forward_fp8",
     "gdn_frame_step",
@@ -199,3 +201,93 @@ def gdn_frame_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, gamma, beta, st
 
     return gdn_frame_forward(dequant(q8, q_scale), dequant(k8, k_scale), dequant(v8, v_scale),
                              gamma, beta, state_in, key_scale)
+
+
+def frame_update_backward(S_prev, A, B, gamma: float, beta: float, G):
+    """Adjoint of ``frame_update``: given G = dL/dS_t, return the gradients that flow to the
+    update's inputs, (dS_prev, dA, dB, dgamma, dbeta).
+
+    The chatpaper.ai abstract of SANA-WM says the model is trained natively on one-minute
+    clips, so the layer needs its backward pass. This function is the chain rule applied to
+    S_t = gamma * S_prev @ M + beta * B, where M = I - beta * A:
+      dS_prev = gamma * G @ M^T
+      dA      = -gamma * beta * S_prev^T @ G
+      dB      = beta * G
+      dgamma  = <G, S_prev @ M>
+      dbeta   = <G, B - gamma * S_prev @ A>
+    <X, Y> is the sum of X * Y over all elements."""
+    D = A.shape[0]
+    M = np.eye(D) - beta * A
+    dS_prev = gamma * (G @ M.T)
+    dA = -gamma * beta * (S_prev.T @ G)
+    dB = beta * G
+    dgamma = float(np.sum(G * (S_prev @ M)))
+    dbeta = float(np.sum(G * (B - gamma * (S_prev @ A))))
+    return dS_prev, dA, dB, dgamma, dbeta
+
+
+def gdn_frame_backward(q, k, v, gamma, beta, state_in, d_out, d_state_out, key_scale: float):
+    """Gradients of the frame-wise GDN layer (``gdn_frame_forward``) for given output and
+    final-state cotangents.
+
+    The chatpaper.ai abstract of SANA-WM says the model is trained natively on one-minute
+    clips. gen-hub.ru, "Архитектура", says the 1/sqrt(D*S) key scale replaced L2 key
+    normalisation and removed NaN divergence in training. So the backward is taken through
+    the key scale: k' = s * k, and dk = s * dk'.
+
+    Arguments: q, k, v, d_out: [B, T, N, H, D]; gamma, beta: [B, T, H]; state_in,
+    d_state_out: [B, H, D, D] or None (zero).
+    Returns (dq, dk, dv [B,T,N,H,D], dgamma, dbeta [B,T,H], dstate_in [B,H,D,D]), all
+    float64.
+
+    Per (batch, head): first the forward, keeping every S_t. Then the frames in reverse with
+    G = dL/dS_t:
+      G_t    = dO_t^T Q_t + (what frame t+1 passed back; d_state_out for the last frame)
+      dQ_t   = dO_t S_t                    (from O_t = Q_t S_t^T)
+      then ``frame_update_backward`` gives dA_t, dB_t, dgamma_t, dbeta_t and what flows to
+      S_{t-1}
+      dK'_t  = K'_t (dA_t + dA_t^T) + V_t dB_t    (A_t = K'^T K', B_t = V^T K')
+      dV_t   = K'_t dB_t^T
+    The gradient that reaches S_0 is dstate_in."""
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    d_out = np.asarray(d_out)
+    gamma = _f64(gamma)
+    beta = _f64(beta)
+    s = float(key_scale)
+    Bsz, T, N, H, D = q.shape
+    dq = np.zeros((Bsz, T, N, H, D))
+    dk = np.zeros((Bsz, T, N, H, D))
+    dv = np.zeros((Bsz, T, N, H, D))
+    dgamma = np.zeros((Bsz, T, H))
+    dbeta = np.zeros((Bsz, T, H))
+    dstate_in = np.zeros((Bsz, H, D, D))
+    for b in range(Bsz):
+        for h in range(H):
+            # forward, keeping S_{t-1} and the statistics of every frame
+            S = np.zeros((D, D)) if state_in is None else _f64(state_in[b, h]).copy()
+            states = [S]
+            stats = []
+            for t in range(T):
+                A, Bm = frame_statistics(k[b, t, :, h, :], v[b, t, :, h, :], s)
+                stats.append((A, Bm))
+                S = frame_update(S, A, Bm, gamma[b, t, h], beta[b, t, h])
+                states.append(S)
+            # reverse
+            G = np.zeros((D, D)) if d_state_out is None else _f64(d_state_out[b, h]).copy()
+            for t in range(T - 1, -1, -1):
+                Q = _f64(q[b, t, :, h, :])
+                Ks = s * _f64(k[b, t, :, h, :])
+                V = _f64(v[b, t, :, h, :])
+                dO = _f64(d_out[b, t, :, h, :])
+                G = G + dO.T @ Q
+                dq[b, t, :, h, :] = dO @ states[t + 1]
+                A, Bm = stats[t]
+                G, dA, dB, dgamma[b, t, h], dbeta[b, t, h] = frame_update_backward(
+                    states[t], A, Bm, gamma[b, t, h], beta[b, t, h], G)
+                dKs = Ks @ (dA + dA.T) + V @ dB
+                dk[b, t, :, h, :] = s * dKs
+                dv[b, t, :, h, :] = Ks @ dB.T
+            dstate_in[b, h] = G
+    return dq, dk, dv, dgamma, dbeta, dstate_in

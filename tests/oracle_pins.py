@@ -2,7 +2,8 @@
 
 Each ``pin_*`` function takes an implementation namespace ``impl`` (an object
 with ``gdn_frame_forward``, ``gdn_frame_step``, ``la_block_causal``,
-``frame_statistics``, ``e4m3_decode`` and ``gdn_frame_forward_fp8`` attributes,
+``frame_statistics``, ``e4m3_decode``, ``gdn_frame_forward_fp8`` and ``gdn_frame_backward``
+attributes,
 the same signatures as ``oracle.gdn_oracle``)
 and raises ``AssertionError`` if the implementation disagrees with:
 
@@ -16,7 +17,11 @@ and raises ``AssertionError`` if the implementation disagrees with:
 * exact invariants (delta-rule exactness for orthonormal keys; the consistent
   linear map is a fixed point; split/resume through the state; linearity in
   (V, S_0); causality across frames and bidirectionality inside a frame; the
-  unrolled affine-map product form of the recurrence).
+  unrolled affine-map product form of the recurrence);
+* for the backward: central differences of the forward, the exact dot-product (adjoint)
+  identity of the map (V, S_0) -> (O, S_T), which is linear, the textbook gradients of
+  unnormalised linear attention (one frame from a zero state), and linearity in the
+  cotangents.
 
 ``tests/test_oracle_mutations.py`` plants plausible mistakes in copies of the
 oracle and checks that each one fails at least one pin.
@@ -423,6 +428,103 @@ def pin_fp8_scales(impl):
     _close(s5, s6, 1e-12, "unit scales (state)")
 
 
+# --------------------------------------------------------------------------- backward pins
+
+def _bwd_case(rng, B=2, T=3, N=3, H=2, D=3):
+    q, k, v, gamma, beta = _rand_clip(B, T, N, H, D, rng, g=(0.5, 1.0), b=(0.1, 0.9))
+    S0 = rng.standard_normal((B, H, D, D))
+    dO = rng.standard_normal((B, T, N, H, D))
+    dS = rng.standard_normal((B, H, D, D))
+    return q, k, v, gamma, beta, S0, dO, dS
+
+
+def pin_bwd_finite_differences(impl):
+    """Every gradient against central differences of the (pinned) forward, for the scalar
+    L = <dO, O> + <dS_T, S_T>. The forward is a polynomial in every input, so central
+    differences with step 1e-5 are exact to about 1e-9 here."""
+    rng = _rng(101)
+    q, k, v, gamma, beta, S0, dO, dS = _bwd_case(rng)
+    D, N = q.shape[-1], q.shape[2]
+    ks = 1.0 / np.sqrt(D * N)
+    params = {"q": q, "k": k, "v": v, "gamma": gamma, "beta": beta, "S0": S0}
+
+    def loss(p):
+        o, st = impl.gdn_frame_forward(p["q"], p["k"], p["v"], p["gamma"], p["beta"], p["S0"], ks)
+        return float(np.sum(dO * o) + np.sum(dS * st))
+
+    grads = impl.gdn_frame_backward(q, k, v, gamma, beta, S0, dO, dS, ks)
+    names = ["q", "k", "v", "gamma", "beta", "S0"]
+    h = 1e-5
+    for name, g in zip(names, grads):
+        fd = np.zeros(params[name].shape)
+        for idx in np.ndindex(*params[name].shape):
+            p_plus = {n: a.copy() for n, a in params.items()}
+            p_minus = {n: a.copy() for n, a in params.items()}
+            p_plus[name][idx] += h
+            p_minus[name][idx] -= h
+            fd[idx] = (loss(p_plus) - loss(p_minus)) / (2 * h)
+        _close(g, fd, 1e-7, f"d{name} vs central differences")
+
+
+def pin_bwd_adjoint_identity(impl):
+    """The forward is linear in (V, S_0) jointly with q, k, gamma, beta fixed (no constant
+    term). So for any direction (dV, dS0) the dot-product test must hold:
+    <grad_V, dV> + <grad_S0, dS0> = <dO, O(dV, dS0)> + <dS_T, S_T(dV, dS0)>.
+    This is exact up to rounding, at a size (T = 6, D = 5) where differences would be slow."""
+    rng = _rng(102)
+    q, k, v, gamma, beta, S0, dO, dS = _bwd_case(rng, B=1, T=6, N=4, H=2, D=5)
+    ks = 1.0 / np.sqrt(5 * 4)
+    grads = impl.gdn_frame_backward(q, k, v, gamma, beta, S0, dO, dS, ks)
+    dV = rng.standard_normal(v.shape)
+    dS0 = rng.standard_normal(S0.shape)
+    o, st = impl.gdn_frame_forward(q, k, dV, gamma, beta, dS0, ks)
+    lhs = float(np.sum(grads[2] * dV) + np.sum(grads[5] * dS0))
+    rhs = float(np.sum(dO * o) + np.sum(dS * st))
+    assert abs(lhs - rhs) <= 1e-10 * max(1.0, abs(rhs)), f"adjoint identity: {lhs} vs {rhs}"
+
+
+def pin_bwd_single_frame_closed_form(impl):
+    """One frame from S_0 = 0: S_1 = beta V^T K', so O = beta Q K'^T V (plain unnormalised
+    linear attention over the frame, K' = s K). With L = <dO, O> (no state cotangent) the
+    textbook gradients are dQ = beta dO V^T K', dV = beta K' Q^T dO, dK = s beta V dO^T Q,
+    dbeta = <dO, Q K'^T V>, dgamma = 0 (the gate multiplies the zero state), and
+    dS_0 = gamma (dO^T Q)(I - beta A)."""
+    rng = _rng(103)
+    N, D = 5, 4
+    q, k, v, gamma, beta = _rand_clip(1, 1, N, 1, D, rng)
+    dO = rng.standard_normal(q.shape)
+    s = 0.37
+    Q, K, V, g = q[0, 0, :, 0], k[0, 0, :, 0], v[0, 0, :, 0], dO[0, 0, :, 0]
+    be, ga = beta[0, 0, 0], gamma[0, 0, 0]
+    Ks = s * K
+    dq, dk, dv, dgamma, dbeta, dS0 = impl.gdn_frame_backward(q, k, v, gamma, beta, None, dO,
+                                                            None, s)
+    _close(dq[0, 0, :, 0], be * g @ V.T @ Ks, 1e-12, "dQ")
+    _close(dv[0, 0, :, 0], be * Ks @ Q.T @ g, 1e-12, "dV")
+    _close(dk[0, 0, :, 0], s * be * V @ g.T @ Q, 1e-12, "dK")
+    _close(dbeta[0, 0, 0], np.sum(g * (Q @ Ks.T @ V)), 1e-12, "dbeta")
+    _close(dgamma[0, 0, 0], 0.0, 1e-12, "dgamma")
+    _close(dS0[0, 0], ga * (g.T @ Q) @ (np.eye(D) - be * Ks.T @ Ks), 1e-12, "dS0")
+
+
+def pin_bwd_cotangent_linearity(impl):
+    """The backward is linear in the cotangents (dO, dS_T): zero cotangents give zero
+    gradients, and a combination of cotangents gives the same combination of gradients."""
+    rng = _rng(104)
+    q, k, v, gamma, beta, S0, dO, dS = _bwd_case(rng, B=1, T=4, N=3, H=1, D=4)
+    dO2 = rng.standard_normal(dO.shape)
+    dS2 = rng.standard_normal(dS.shape)
+    ks = 0.25
+    zero = impl.gdn_frame_backward(q, k, v, gamma, beta, S0, np.zeros_like(dO), None, ks)
+    for z in zero:
+        _close(z, np.zeros_like(z), 0.0, "zero cotangents")
+    g1 = impl.gdn_frame_backward(q, k, v, gamma, beta, S0, dO, dS, ks)
+    g2 = impl.gdn_frame_backward(q, k, v, gamma, beta, S0, dO2, dS2, ks)
+    g3 = impl.gdn_frame_backward(q, k, v, gamma, beta, S0, 2 * dO - 3 * dO2, 2 * dS - 3 * dS2, ks)
+    for a, b, c in zip(g1, g2, g3):
+        _close(c, 2 * a - 3 * b, 1e-12, "cotangent linearity")
+
+
 GDN_PINS = [
     pin_hand_example,
     pin_single_frame_closed_form,
@@ -439,4 +541,10 @@ GDN_PINS = [
 ]
 LA_PINS = [pin_la_hand_example, pin_la_brute_force, pin_la_resume]
 FP8_PINS = [pin_e4m3_landmarks, pin_e4m3_ordering, pin_fp8_scales]
-ALL_PINS = GDN_PINS + LA_PINS + FP8_PINS
+BWD_PINS = [
+    pin_bwd_finite_differences,
+    pin_bwd_adjoint_identity,
+    pin_bwd_single_frame_closed_form,
+    pin_bwd_cotangent_linearity,
+]
+ALL_PINS = GDN_PINS + LA_PINS + FP8_PINS + BWD_PINS

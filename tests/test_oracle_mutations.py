@@ -26,7 +26,7 @@ def _decode_variant(bias=7, subnormals=True):
 
 
 def _impl(stats=None, update=None, output=None, forward=None, la=None, decode=None,
-          swap_kv_scales=False):
+          swap_kv_scales=False, backward=None):
     """An oracle copy with some pieces swapped; gdn_frame_step and the fp8 forward follow the
     swapped forward and decoder."""
     decode = decode or go.e4m3_decode
@@ -66,7 +66,8 @@ def _impl(stats=None, update=None, output=None, forward=None, la=None, decode=No
     return types.SimpleNamespace(gdn_frame_forward=forward, gdn_frame_step=step,
                                  la_block_causal=la or oracle.la_block_causal,
                                  frame_statistics=stats, e4m3_decode=decode,
-                                 gdn_frame_forward_fp8=fwd_fp8)
+                                 gdn_frame_forward_fp8=fwd_fp8,
+                                 gdn_frame_backward=backward or oracle.gdn_frame_backward)
 
 
 def _old_state_forward(q, k, v, gamma, beta, state_in, key_scale):
@@ -115,6 +116,59 @@ def _la_variant(relu_q=True, relu_k=True, eps=1e-6, transpose_state=False, frame
     return la
 
 
+def _bwd_variant(mistake):
+    """The backward with one planted mistake (named by ``mistake``)."""
+    def bwd(q, k, v, gamma, beta, state_in, d_out, d_state_out, s):
+        q, k, v, d_out = (np.asarray(x, float) for x in (q, k, v, d_out))
+        B, T, N, H, D = q.shape
+        dq, dk, dv = np.zeros(q.shape), np.zeros(q.shape), np.zeros(q.shape)
+        dg, db = np.zeros((B, T, H)), np.zeros((B, T, H))
+        ds0 = np.zeros((B, H, D, D))
+        I = np.eye(D)
+        for b in range(B):
+            for h in range(H):
+                S = np.zeros((D, D)) if state_in is None else np.array(state_in[b, h], float)
+                states, stats = [S], []
+                for t in range(T):
+                    A, Bm = go.frame_statistics(k[b, t, :, h], v[b, t, :, h], s)
+                    stats.append((A, Bm))
+                    S = go.frame_update(S, A, Bm, gamma[b, t, h], beta[b, t, h])
+                    states.append(S)
+                G = np.zeros((D, D)) if d_state_out is None else np.array(d_state_out[b, h], float)
+                for t in range(T - 1, -1, -1):
+                    Q, Ks, V, dO = q[b, t, :, h], s * k[b, t, :, h], v[b, t, :, h], d_out[b, t, :, h]
+                    g, be = gamma[b, t, h], beta[b, t, h]
+                    A, Bm = stats[t]
+                    Sp = states[t]
+                    if mistake == "state_grad_not_carried":
+                        G = dO.T @ Q
+                    else:
+                        G = G + (Q.T @ dO if mistake == "E_transposed" else dO.T @ Q)
+                    dq[b, t, :, h] = dO @ (Sp if mistake == "dq_reads_previous_state" else states[t + 1])
+                    M = I - be * A
+                    Sg = states[t + 1] if mistake == "dgamma_reads_new_state" else Sp
+                    dg[b, t, h] = np.sum(G * (Sg @ M))
+                    sign = 1.0 if mistake == "dbeta_gamma_term_sign" else -1.0
+                    db[b, t, h] = np.sum(G * (Bm + sign * g * (Sp @ A)))
+                    dA = -g * be * (Sp.T @ G)
+                    dB = be * G
+                    sym = 2 * dA if mistake == "dA_not_symmetrised" else dA + dA.T
+                    dKs = Ks @ sym + V @ dB
+                    dk[b, t, :, h] = dKs if mistake == "key_scale_dropped_on_dk" else s * dKs
+                    dv[b, t, :, h] = Ks @ (dB if mistake == "dv_dB_not_transposed" else dB.T)
+                    G = g * ((M @ G) if mistake == "gate_on_wrong_side" else (G @ M.T))
+                ds0[b, h] = G
+        return dq, dk, dv, dg, db, ds0
+    return bwd
+
+
+BWD_MISTAKES = [
+    "E_transposed", "state_grad_not_carried", "dq_reads_previous_state", "dgamma_reads_new_state",
+    "dbeta_gamma_term_sign", "dA_not_symmetrised", "key_scale_dropped_on_dk",
+    "dv_dB_not_transposed", "gate_on_wrong_side",
+]
+
+
 MUTANTS = {
     "gamma_also_scales_beta_B": dict(update=lambda S, A, B, g, b: g * (S @ (np.eye(len(A)) - b * A) + b * B)),
     "transposed_state_product": dict(update=lambda S, A, B, g, b: g * ((np.eye(len(A)) - b * A) @ S) + b * B),
@@ -138,6 +192,7 @@ MUTANTS = {
     "e4m3_exponent_bias_8": dict(decode=_decode_variant(bias=8)),
     "e4m3_subnormals_read_as_normals": dict(decode=_decode_variant(subnormals=False)),
     "fp8_k_and_v_scales_swapped": dict(swap_kv_scales=True),
+    **{"bwd_" + m: dict(backward=_bwd_variant(m)) for m in BWD_MISTAKES},
 }
 
 
@@ -154,6 +209,6 @@ def test_mutant_is_caught(name):
 
 
 def test_unmutated_copy_passes():
-    impl = _impl()
+    impl = _impl(backward=_bwd_variant("none"))
     for pin in oracle_pins.ALL_PINS:
         pin(impl)

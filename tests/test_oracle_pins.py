@@ -13,6 +13,7 @@ IMPL = types.SimpleNamespace(
     frame_statistics=oracle.frame_statistics,
     e4m3_decode=oracle.e4m3_decode,
     gdn_frame_forward_fp8=oracle.gdn_frame_forward_fp8,
+    gdn_frame_backward=oracle.gdn_frame_backward,
 )
 
 
