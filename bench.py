@@ -15,6 +15,8 @@ grid, synthetic seeded bf16 inputs resident in HBM). Prints one JSON line (rank 
   bandwidth; traffic from the committed ncu summary when the kernel sources still match it.
 * cpu_baseline: the fp64 oracle on a bounded sample of the same workload (rank 0, N = 1).
 * --impl reference: the oracle itself as the reference arm (host cores, bounded samples).
+* --backward: one step = one gdn_frame_backward (the gradients for a seeded d_out) instead of
+  the forward; no e2e leg.
 
 Multi-GPU (torchrun): every rank processes its own clip (independent problems, no collective
 on the data path), so scaling is weak.
@@ -37,6 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GDN layer tokens·heads/sec and % of roofline (720p 60 s config, 1 B200)"
+METRIC_BWD = "GDN layer backward tokens·heads/sec (720p 60 s config, 1 B200)"
 UNIT = "tokens*heads/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -57,6 +60,8 @@ def args_parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8", action="store_true",
                     help="E4M3 q, k, v with per-(frame, head) scales (gdn_frame_forward_fp8)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time gdn_frame_backward (the training pass) instead of the forward")
     ap.add_argument("--forward-mode", type=int, default=0,
                     help="gdn_set_forward_mode: 0 auto, 1 three kernels, 2 fused, 3 chunked")
     return ap.parse_args()
@@ -85,6 +90,14 @@ def algorithmic_bytes(w, fp8=False):
             + (state if w.kind == "stream" else 0))
 
 
+def backward_bytes(w):
+    """Bytes the backward must move per call: Q, K, V, dO read and dQ, dK, dV written (bf16),
+    gamma and beta read, d_gamma and d_beta written, the fp32 S_0 read and dS_0 written."""
+    fh = w.B * w.H * w.T
+    state = w.B * w.H * w.D * w.D * 4
+    return fh * 7 * w.N * w.D * 2 + w.B * w.T * w.H * 4 * 4 + 2 * state
+
+
 def kernel_bytes(name, w, fp8=False):
     """Algorithmic bytes per launch of each kernel of the forward (the bytes its stage must
     move in the three-kernel design)."""
@@ -98,6 +111,13 @@ def kernel_bytes(name, w, fp8=False):
         if name == "gdn_fused_kernel":
             return algorithmic_bytes(w, True)
     dd = w.D * w.D
+    if name.startswith("gdn_bwd_token_kernel_d"):  # read X tiles and frame matrices; write out
+        terms = 2 if name.endswith("_dk") else 1
+        return fh * ((terms + 1) * nd2 + terms * dd * 2)
+    if name == "gdn_bwd_chain_kernel":   # read A_t, E_t, gamma, beta; write G_t (bf16), dS_0
+        return fh * (dd * 2 + dd * 4 + dd * 2 + 8) + w.B * w.H * dd * 4
+    if name == "gdn_bwd_frame_kernel":   # read S_{t-1}, G_t, A_t, B_t; write W'_t, dgamma, dbeta
+        return fh * (dd * 2 * 3 + dd * 4 + dd * 2 + 16)
     if name == "gdn_stats_kernel":       # read K, V; write A_t (bf16) and B_t (f32)
         return fh * (2 * nd2 + dd * 2 + dd * 4)
     if name == "gdn_chain_kernel":       # read A_t, B_t, gamma, beta; write S_t (bf16), S_T
@@ -129,6 +149,11 @@ KERNEL_SOURCES = {
     "gdn_output_kernel": ["output_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_chain_kernel": ["chain_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_scan_kernel": ["scan_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_chain_kernel": ["bwd_chain_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_frame_kernel": ["bwd_frame_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_token_kernel_dq": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_token_kernel_dv": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_token_kernel_dk": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
 }
 
 
@@ -249,17 +274,22 @@ def job_throughput(units_per_rank, ms_local, world, device="cuda"):
     return units_per_rank * world / (ms * 1e-3), ms
 
 
-def oracle_sample_rate(w, heads, frames, seed=99):
+def oracle_sample_rate(w, heads, frames, seed=99, backward=False):
     """The fp64 oracle on a bounded sample of workload `w` (`heads` heads, `frames` frames, same
-    token count and head dim). Returns (tokens*heads/s, seconds, threads)."""
+    token count and head dim), forward or backward. Returns (tokens*heads/s, seconds, threads)."""
     import numpy as np
     import gdn_inputs
     import oracle
     x = gdn_inputs.clip_inputs(1, heads, frames, w.N, w.D, w.gamma_range, w.beta_range, seed=seed)
     f = lambda t: t.float().numpy()
     args = [f(x["q"]), f(x["k"]), f(x["v"]), f(x["gamma"]), f(x["beta"])]
+    if backward:
+        c = gdn_inputs.cotangents(1, heads, frames, w.N, w.D, seed=seed + 1)
     t0 = time.perf_counter()
-    oracle.gdn_frame_forward(*args, None, w.key_scale)
+    if backward:
+        oracle.gdn_frame_backward(*args, None, f(c["d_out"]), None, w.key_scale)
+    else:
+        oracle.gdn_frame_forward(*args, None, w.key_scale)
     dt = time.perf_counter() - t0
     try:
         import threadpoolctl
@@ -368,6 +398,17 @@ def main():
             api.gdn_frame_forward_fp8(f8["q"], f8["k"], f8["v"], f8["sq"], f8["sk"], f8["sv"],
                                       gam, bet, None, out, st, key_scale=w.key_scale,
                                       stream=stream)
+    elif a.backward:
+        # the training pass: gradients of the clip for seeded cotangents of the output
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
+        d_out = gdn_inputs.cotangents(w.B, w.H, w.T, w.N, w.D, seed=w.seed + 50,
+                                      device=dev)["d_out"]
+        out = st = None
+
+        def step():
+            api.gdn_frame_backward(q, k, v, gam, bet, d_out, key_scale=w.key_scale,
+                                   stream=stream)
     else:
         g = gdn_inputs.workload_inputs(w, device=dev)
         q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
@@ -427,17 +468,18 @@ def main():
     hbm, peak_kind = peaks()
     kb = kernel_bytes(dom, w, a.fp8)
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
-    path_bytes = algorithmic_bytes(w, a.fp8)
+    path_bytes = backward_bytes(w) if a.backward else algorithmic_bytes(w, a.fp8)
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
 
     # ---------------------------------------------------------------- end to end, host buffers
     e2e = None
     if not a.no_e2e:
         e2e = (measure_e2e(a, w, g, out, st, stream, world, dev)
-               if w.kind == "gdn" and not a.fp8 else None)
+               if w.kind == "gdn" and not a.fp8 and not a.backward else None)
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "metric": METRIC_BWD if a.backward else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 q/k/v, bf16 out" if a.fp8 else "bf16", "data": "synthetic",
@@ -458,10 +500,13 @@ def main():
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn" and not a.fp8:
-        rate, secs, threads = oracle_sample_rate(w, 4, w.T)
+        heads = 1 if a.backward else 4
+        rate, secs, threads = oracle_sample_rate(w, heads, w.T, backward=a.backward)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"4 heads x {w.T} frames of the {w.name} clip shape "
-                                          f"(N={w.N}, D={w.D}), {secs:.1f} s of fp64 numpy"}
+                                "sample": f"{heads} head(s) x {w.T} frames of the {w.name} clip "
+                                          f"shape (N={w.N}, D={w.D}), "
+                                          f"{'backward' if a.backward else 'forward'}, "
+                                          f"{secs:.1f} s of fp64 numpy"}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

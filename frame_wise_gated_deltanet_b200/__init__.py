@@ -8,12 +8,14 @@ there is no CPU fallback.
 _API = (
     "gdn_frame_forward",
     "gdn_frame_step",
+    "gdn_frame_backward",
     "gdn_frame_stats",
     "gdn_block_causal_la",
     "gdn_sync_status",
     "gdn_release_workspace",
     "gdn_workspace_bytes",
     "gdn_la_workspace_bytes",
+    "gdn_backward_workspace_bytes",
     "GdnError",
 )
 __all__ = list(_API)

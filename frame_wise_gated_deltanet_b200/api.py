@@ -13,7 +13,7 @@ import torch
 from ._lib import LIB, GdnError, check
 
 __all__ = ["gdn_frame_forward", "gdn_frame_forward_fp8", "gdn_frame_forward_host",
-           "gdn_frame_step", "gdn_frame_stats", "gdn_block_causal_la",
+           "gdn_frame_step", "gdn_frame_backward", "gdn_backward_workspace_bytes", "gdn_frame_stats", "gdn_block_causal_la",
            "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
            "gdn_la_workspace_bytes", "GdnError"]
 
@@ -175,6 +175,35 @@ def gdn_frame_step(q, k, v, gamma, beta, state_in=None, out=None, state_out=None
     return out, state_out
 
 
+def gdn_frame_backward(q, k, v, gamma, beta, d_out, state_in=None, d_state_out=None,
+                       key_scale: Optional[float] = None, stream=None,
+                       want_state_grad: bool = True):
+    """Gradients of gdn_frame_forward for the cotangents d_out ([B,T,N,H,D] bf16) and
+    d_state_out ([B,H,D,D] f32 or None). Returns (dq, dk, dv, d_gamma, d_beta, d_state_in);
+    d_state_in is None when want_state_grad is False. 64 < D <= 128."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("d_out", d_out)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    _req(gamma, "gamma", torch.float32, (B, T, H))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if d_state_out is not None:
+        _req(d_state_out, "d_state_out", torch.float32, (B, H, D, D))
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    d_gamma, d_beta = torch.empty_like(gamma), torch.empty_like(beta)
+    d_state_in = (torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+                  if want_state_grad else None)
+    if key_scale is None:
+        key_scale = 1.0 / math.sqrt(D * N)
+    with torch.cuda.device(q.device):
+        check("gdn_frame_backward", LIB.gdn_frame_backward(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(d_out),
+            _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_gamma), _ptr(d_beta),
+            _ptr(d_state_in), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
+    return dq, dk, dv, d_gamma, d_beta, d_state_in
+
+
 def gdn_frame_stats(k, v, key_scale: Optional[float] = None, A_out=None, B_out=None, stream=None):
     """Per-frame statistics. Returns A [B,H,T,D,D] bf16 (s^2 K^T K) and B [B,H,T,D,D] f32
     (s V^T K)."""
@@ -237,6 +266,10 @@ def gdn_release_workspace() -> None:
 
 def gdn_workspace_bytes(B, H, T, N, D) -> int:
     return int(LIB.gdn_workspace_bytes(B, H, T, N, D))
+
+
+def gdn_backward_workspace_bytes(B, H, T, N, D) -> int:
+    return int(LIB.gdn_backward_workspace_bytes(B, H, T, N, D))
 
 
 def gdn_la_workspace_bytes(B, H, T, D) -> int:

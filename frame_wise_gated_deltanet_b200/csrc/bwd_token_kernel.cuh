@@ -1,0 +1,290 @@
+// Token-side gradient GEMMs of the backward, every frame of every head in parallel. Per frame
+// (b, t, h) and 128-token tile, one accumulator sums kTerms products X_i Y_i^(T) of a token
+// tile X_i (TMA, 128B swizzle, K-major) and a frame matrix Y_i (bf16 DP x DP in the s8 layout,
+// one bulk copy per frame); the epilogue scales the tile and TMA-stores it as bf16:
+//
+//   dQ_t = dO_t S_t                      (1 term, Y = S_t read MN-major: contraction over v)
+//   dV_t = s beta_t * K_t G_t^T          (1 term, Y = G_t read K-major: contraction over k)
+//   dK_t = s beta_t * (V_t G_t + K_t W'_t)   (2 terms: G_t MN-major, W'_t K-major)
+//
+// with s the key scale, G_t = dL/dS_t from the backward chain and W'_t = -s gamma_t (S_{t-1}^T
+// G_t + G_t^T S_{t-1}) from the per-frame kernel (K_t here is the unscaled key tile, so both
+// factors of s are in these scalars).
+//
+// The same pipeline as the forward's output GEMM: warp 0 TMA producer, warp 1 TMEM allocator +
+// MMA issuer, warps 2..17 epilogue (4 column groups of 4 warps). One term: two frame-matrix
+// buffers, three token stages, two staging tiles. Two terms: one buffer per frame matrix, two
+// stages of two token tiles, one staging tile (227 KB of shared memory either way).
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace gdn {
+
+template <int DP, int kTerms>
+struct BwdTokenLayout {
+  static_assert(DP == 128 && (kTerms == 1 || kTerms == 2), "DP = 128, one or two terms");
+  static constexpr int kEpiWarps = 16;
+  static constexpr int kCols = DP / 4;  // columns per epilogue thread
+  static constexpr int kBoxes = DP / 64;
+  static constexpr int kXBytes = kBoxes * kBoxBytes;  // one 128-token tile
+  static constexpr int kYBytes = DP * DP * 2;
+  static constexpr int kYBufs = kTerms == 1 ? 2 : 1;
+  static constexpr int kStages = kTerms == 1 ? 3 : 2;
+  static constexpr int kOBufs = kTerms == 1 ? 2 : 1;
+  static constexpr int kStageBytes = kTerms * kXBytes;
+  static constexpr int kThreads = (2 + kEpiWarps) * 32;
+  static constexpr int kTmemCols = 2 * DP;
+  static constexpr int kOBytes = kXBytes;
+  static constexpr int kSmemBytes =
+      kYBufs * kTerms * kYBytes + kStages * kStageBytes + kOBufs * kOBytes + 512 + 1024;
+};
+
+struct BwdTokenArgs {
+  const __nv_bfloat16* Y0;  // frame matrices of term 0 / 1, DP*DP bf16 per row (b*H+h)*T + t
+  const __nv_bfloat16* Y1;
+  const float* beta;        // non-null: scale by key_scale * beta[b, t, h], else 1
+};
+
+// kMN0 / kMN1: the term's frame matrix is read MN-major (contraction over its rows).
+template <int DP, int kTerms, bool kMN0, bool kMN1>
+__global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms>::kThreads, 1)
+    gdn_bwd_token_kernel(const __grid_constant__ CUtensorMap tm_x0,
+                         const __grid_constant__ CUtensorMap tm_x1,
+                         const __grid_constant__ CUtensorMap tm_o, BwdTokenArgs a, Problem p) {
+  using L = BwdTokenLayout<DP, kTerms>;
+  constexpr int kEpiThreads = 32 * L::kEpiWarps;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1k(smem_raw);
+  uint8_t* y_buf = smem;                                     // [kYBufs][kTerms] frame matrices
+  uint8_t* x_ring = y_buf + L::kYBufs * kTerms * L::kYBytes;   // [kStages][kTerms] token tiles
+  uint8_t* o_stage = x_ring + L::kStages * L::kStageBytes;    // [kOBufs] staging tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(o_stage + L::kOBufs * L::kOBytes);
+  uint64_t* empty = full + L::kStages;
+  uint64_t* y_full = empty + L::kStages;
+  uint64_t* y_empty = y_full + 2;
+  uint64_t* acc_full = y_empty + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* mma_drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const long n_items = static_cast<long>(p.B) * p.T * p.H;
+  const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
+  const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
+  // item i = (b*T + t)*H + h
+  auto decode = [&](long item, int& bt, int& h, long& yrow) {
+    h = static_cast<int>(item % p.H);
+    bt = static_cast<int>(item / p.H);
+    const int b = bt / p.T;
+    const int t = bt - b * p.T;
+    yrow = (static_cast<long>(b) * p.H + h) * p.T + t;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&y_full[i], 1);
+      mbar_init(&y_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiThreads);
+    }
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_x0);
+      if (kTerms == 2) tma_prefetch_desc(&tm_x1);
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_frame = policy_evict_last();
+      StageFills<L::kStages> fills;
+      StageFills<2> y_fills;
+      int stage = 0;
+      uint32_t phase = 0;
+      int li = 0;
+      for (long item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x, ++li) {
+        int bt, h;
+        long yrow;
+        decode(item, bt, h, yrow);
+        const int yb = li % L::kYBufs;
+        const uint32_t yph = (li / L::kYBufs) & 1;
+        if (!mbar_wait(&y_empty[yb], yph ^ 1)) {
+          give_up(none, abort_flag);
+          break;
+        }
+        mbar_arrive_expect_tx(&y_full[yb], kTerms * L::kYBytes);
+        uint8_t* yd = y_buf + yb * kTerms * L::kYBytes;
+        bulk_load(yd, a.Y0 + yrow * DP * DP, L::kYBytes, &y_full[yb], pol_frame);
+        if (kTerms == 2)
+          bulk_load(yd + L::kYBytes, a.Y1 + yrow * DP * DP, L::kYBytes, &y_full[yb], pol_frame);
+        y_fills.filled(yb, yph);
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) {
+            give_up(none, abort_flag);
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          uint8_t* xd = x_ring + stage * L::kStageBytes;
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb) {
+            tma_load_4d(xd + kb * kBoxBytes, &tm_x0, &full[stage], kb * 64, h,
+                        tile * kRowsPerTile, bt, pol_stream);
+            if (kTerms == 2)
+              tma_load_4d(xd + L::kXBytes + kb * kBoxBytes, &tm_x1, &full[stage], kb * 64, h,
+                          tile * kRowsPerTile, bt, pol_stream);
+          }
+          fills.filled(stage, phase);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      fills.drain(full);
+      y_fills.drain(y_full);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc0 = idesc_bf16(128, DP, false, kMN0);
+    constexpr uint32_t idesc1 = idesc_bf16(128, DP, false, kMN1);
+    int stage = 0;
+    uint32_t phase = 0;
+    int tc = 0;
+    bool ok = true;
+    int li = 0;
+    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
+      const int yb = li % L::kYBufs;
+      if (!mbar_wait(&y_full[yb], (li / L::kYBufs) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint32_t y_base = smem_u32(y_buf + yb * kTerms * L::kYBytes);
+      for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
+        const int acc = tc & 1;
+        if (!mbar_wait(&acc_empty[acc], ((tc >> 1) & 1) ^ 1) || !mbar_wait(&full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t x_base = smem_u32(x_ring + stage * L::kStageBytes);
+#pragma unroll
+          for (int term = 0; term < kTerms; ++term) {
+            const bool mn = term == 0 ? kMN0 : kMN1;
+            const uint32_t xb = x_base + term * L::kXBytes;
+            const uint32_t yt = y_base + term * L::kYBytes;
+#pragma unroll
+            for (int ks = 0; ks < DP / 16; ++ks) {
+              const uint64_t da = smem_desc(xb + (ks >> 2) * kBoxBytes + (ks & 3) * 32, 16, 1024);
+              // s8 frame matrix: K-major (contraction over its keys: key groups 2ks, 2ks+1,
+              // DP*16 bytes apart) or MN-major (contraction over its rows: 8-row groups 2ks,
+              // 2ks+1, 128 bytes apart; key groups DP*16 bytes apart)
+              const uint64_t db = mn ? smem_desc_noswz(yt + ks * 256, 128, DP * 16)
+                                     : smem_desc_noswz(yt + ks * 2 * DP * 16, DP * 16, 128);
+              mma_bf16(tmem_base + acc * DP, da, db, term == 0 ? idesc0 : idesc1,
+                       (term | ks) != 0);
+            }
+          }
+          mma_commit(&empty[stage]);
+          mma_commit(&acc_full[acc]);
+        }
+        __syncwarp();
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&y_empty[yb]);
+      __syncwarp();
+    }
+    if (!ok) give_up(none, abort_flag);
+    if (elect_one()) mma_commit(mma_drain);
+    __syncwarp();
+    mbar_wait(mma_drain, 0);
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const uint32_t quarter = warp & 3;
+    const int c0 = ((warp - 2) >> 2) * L::kCols;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
+    const bool leader = (threadIdx.x == 64);
+    const uint64_t pol_out = policy_evict_first();
+    if (leader) tma_prefetch_desc(&tm_o);
+    int tc = 0;
+    bool ok = true;
+    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      int bt, h;
+      long yrow;
+      decode(item, bt, h, yrow);
+      const float scale =
+          a.beta ? p.key_scale * __ldg(a.beta + static_cast<long>(bt) * p.H + h) : 1.f;
+      for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
+        const int acc = tc & 1;
+        const int valid = min(kRowsPerTile, p.N - tile * kRowsPerTile);
+        const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
+        // the staging tile is free once the store issued kOBufs tiles ago has read it
+        if (leader) bulk_wait_read<L::kOBufs - 1>();
+        if (named_bar_any(1, kEpiThreads, !waited)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* ob = o_stage + (tc % L::kOBufs) * L::kOBytes;
+        if (static_cast<int>(quarter) * 32 < valid) {
+          const uint32_t tacc = lane_base + acc * DP;
+          float v[32];
+          tmem_ld32(tacc + c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
+            pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
+            pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
+            pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
+            *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c0 + j, kBoxBytes)) = pk;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[acc]);
+        fence_async_smem();
+        named_bar(1, kEpiThreads);
+        if (leader) {
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb)
+            tma_store_4d(&tm_o, ob + kb * kBoxBytes, kb * 64, h, tile * kRowsPerTile, bt,
+                         pol_out);
+          bulk_commit();
+        }
+      }
+    }
+    if (leader) bulk_wait_all();
+    if (!ok) give_up(none, abort_flag);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace gdn

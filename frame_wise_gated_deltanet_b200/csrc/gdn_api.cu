@@ -10,6 +10,9 @@
 #include <mutex>
 
 #include "../../include/gdn.h"
+#include "bwd_chain_kernel.cuh"
+#include "bwd_frame_kernel.cuh"
+#include "bwd_token_kernel.cuh"
 #include "chain_kernel.cuh"
 #include "common.cuh"
 #include "fused_kernel.cuh"
@@ -737,6 +740,134 @@ gdn_status validate_common(const void* q, const void* k, const void* v, const vo
 }
 
 
+// ------------------------------------------------------------------ backward
+// Workspace of gdn_frame_backward, per frame-head: the forward's A_t (bf16 D x D), B_t (f32),
+// S_t (bf16 DP x DP), E_t = dO^T Q (f32), G_t (bf16 DP x DP) and W'_t (bf16 DP x DP; before the
+// per-frame kernel writes it, the same space takes the unused Q^T Q of the E statistics).
+struct BackwardWs {
+  void* A;
+  float* B;
+  void* S;
+  float* E;
+  void* G;
+  void* W;
+};
+
+size_t backward_ws_bytes(long count, int D) {
+  const size_t m = size_t(D) * D, dp2 = size_t(128) * 128;
+  return align256(count * m * 2) + align256(count * m * 4) + 3 * align256(count * dp2 * 2) +
+         align256(count * m * 4);
+}
+
+BackwardWs carve_backward(void* base, long count, int D) {
+  const size_t m = size_t(D) * D, dp2 = size_t(128) * 128;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  BackwardWs w;
+  w.A = p;
+  p += align256(count * m * 2);
+  w.B = reinterpret_cast<float*>(p);
+  p += align256(count * m * 4);
+  w.S = p;
+  p += align256(count * dp2 * 2);
+  w.E = reinterpret_cast<float*>(p);
+  p += align256(count * m * 4);
+  w.G = p;
+  p += align256(count * dp2 * 2);
+  w.W = p;
+  return w;
+}
+
+gdn_status run_bwd_chain(int dev, const Problem& p, const void* A, const float* E,
+                         const float* gamma, const float* beta, const float* d_state_out,
+                         void* G, float* d_state_in, cudaStream_t st) {
+  using L = gdn::BwdChainLayout<128>;
+  const long count = long(p.B) * p.H * p.T;
+  CUtensorMap ta;
+  if (!tmap_mats(&ta, A, false, p.D, p.D, count, 128)) return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_bwd_chain_kernel<128>;
+  if (gdn_status s = ensure_smem_attr(dev, 20, kern, L::kSmemBytes)) return s;
+  {
+    ProfiledLaunch pl("gdn_bwd_chain_kernel", st);
+    kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, E, static_cast<__nv_bfloat16*>(G),
+                                                        gamma, beta, d_state_out, d_state_in, p);
+  }
+  return check_launch();
+}
+
+gdn_status run_bwd_frame(int dev, const Problem& p, const BackwardWs& w, const float* state_in,
+                         const float* gamma, const float* beta, float* d_gamma, float* d_beta,
+                         cudaStream_t st) {
+  using L = gdn::BwdFrameLayout<128>;
+  auto kern = gdn::gdn_bwd_frame_kernel<128>;
+  if (gdn_status s = ensure_smem_attr(dev, 21, kern, L::kSmemBytes)) return s;
+  const long items = long(p.B) * p.H * p.T;
+  const long cap = 3L * g_dev[dev].sms;  // three CTAs of 67 KB shared memory per SM
+  const int grid = static_cast<int>(items < cap ? items : cap);
+  {
+    ProfiledLaunch pl("gdn_bwd_frame_kernel", st);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(
+        static_cast<const __nv_bfloat16*>(w.S), static_cast<const __nv_bfloat16*>(w.G),
+        static_cast<const __nv_bfloat16*>(w.A), w.B, state_in, gamma, beta,
+        static_cast<__nv_bfloat16*>(w.W), d_gamma, d_beta, p);
+  }
+  return check_launch();
+}
+
+// One of the token GEMMs of the backward: out = scale * sum over terms of X_i Y_i^(T).
+template <int kTerms, bool kMN0, bool kMN1>
+gdn_status run_bwd_token(int dev, const Problem& p, const void* x0, const void* x1,
+                         const void* Y0, const void* Y1, const float* beta, void* out,
+                         const char* name, int attr_bit, cudaStream_t st) {
+  using L = gdn::BwdTokenLayout<128, kTerms>;
+  CUtensorMap t0, t1, to;
+  if (!tmap_tokens(&t0, x0, p) || !tmap_tokens(&t1, kTerms == 2 ? x1 : x0, p) ||
+      !tmap_tokens(&to, out, p))
+    return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_bwd_token_kernel<128, kTerms, kMN0, kMN1>;
+  if (gdn_status s = ensure_smem_attr(dev, attr_bit, kern, L::kSmemBytes)) return s;
+  const long items = long(p.B) * p.T * p.H;
+  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  const gdn::BwdTokenArgs a{static_cast<const __nv_bfloat16*>(Y0),
+                            static_cast<const __nv_bfloat16*>(Y1), beta};
+  {
+    ProfiledLaunch pl(name, st);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(t0, t1, to, a, p);
+  }
+  return check_launch();
+}
+
+// The whole backward (64 < D <= 128): recompute the forward's statistics and states, then the
+// output statistics E_t, the backward chain, the per-frame kernel and the three token GEMMs.
+gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
+                         const float* gamma, const float* beta, const float* s_in,
+                         const void* d_out, const float* ds_out, void* dq, void* dk, void* dv,
+                         float* d_gamma, float* d_beta, float* ds_in, const Problem& p,
+                         cudaStream_t st) {
+  const long count = long(p.B) * p.H * p.T;
+  void* base = nullptr;
+  if (gdn_status s = get_workspace(dev, backward_ws_bytes(count, p.D), st, &base)) return s;
+  const BackwardWs w = carve_backward(base, count, p.D);
+  const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
+  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole, st))
+    return s;
+  Problem pe = p;  // E_t = dO^T Q: the "B" statistic of (key = q, value = dO), key scale 1
+  pe.key_scale = 1.0f;
+  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, st)) return s;
+  if (gdn_status s = run_bwd_chain(dev, p, w.A, w.E, gamma, beta, ds_out, w.G, ds_in, st))
+    return s;
+  if (gdn_status s = run_bwd_frame(dev, p, w, s_in, gamma, beta, d_gamma, d_beta, st)) return s;
+  if (gdn_status s = run_bwd_token<1, true, false>(dev, p, d_out, nullptr, w.S, nullptr, nullptr,
+                                                   dq, "gdn_bwd_token_kernel_dq", 22, st))
+    return s;
+  if (gdn_status s = run_bwd_token<1, false, false>(dev, p, k, nullptr, w.G, nullptr, beta, dv,
+                                                    "gdn_bwd_token_kernel_dv", 23, st))
+    return s;
+  return run_bwd_token<2, true, false>(dev, p, v, k, w.G, w.W, beta, dk,
+                                       "gdn_bwd_token_kernel_dk", 24, st);
+}
+
+
 // ------------------------------------------------------------------ host-resident clips
 // gdn_frame_forward_host streams a clip held in host memory through the GPU in segments of
 // frames: segment i's inputs are copied in on a copy-in stream while segment i-1 is computed on
@@ -1060,6 +1191,54 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
     if (gdn_status s = check_launch()) return s;
   }
   return run_output<128, true>(dev, p, q, Sws, D + 1, out, F, st);
+}
+
+gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                              const float* gamma, const float* beta, const float* state_in,
+                              const gdn_bf16* d_out, const float* d_state_out, gdn_bf16* dq,
+                              gdn_bf16* dk, gdn_bf16* dv, float* d_gamma, float* d_beta,
+                              float* d_state_in, int B, int H, int T, int N, int D,
+                              float key_scale, gdn_stream_t stream) {
+  if (!q || !k || !v || !gamma || !beta || !d_out || !dq || !dk || !dv || !d_gamma || !d_beta)
+    return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  if (D <= 64) return GDN_ERR_UNSUPPORTED;
+  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  const void* dev_ptrs[] = {q, k, v, gamma, beta, d_out, dq, dk, dv, d_gamma, d_beta};
+  for (const void* ptr : dev_ptrs)
+    if (!aligned16(ptr)) return GDN_ERR_MISALIGNED;
+  if ((state_in && !aligned16(state_in)) || (d_state_out && !aligned16(d_state_out)) ||
+      (d_state_in && !aligned16(d_state_in)))
+    return GDN_ERR_MISALIGNED;
+  // outputs must not overlap the inputs or each other (d_state_in may alias d_state_out: each
+  // element is read once before it is written, by the same thread)
+  const size_t n = size_t(B) * T * N * H * D * 2, ng = size_t(B) * T * H * 4,
+               ns = size_t(B) * H * D * D * 4;
+  const void* ins[] = {q, k, v, d_out};
+  const void* outs[] = {dq, dk, dv};
+  for (const void* o : outs) {
+    for (const void* i : ins)
+      if (overlaps(o, n, i, n)) return GDN_ERR_INVALID_ARG;
+    for (const void* o2 : outs)
+      if (o != o2 && overlaps(o, n, o2, n)) return GDN_ERR_INVALID_ARG;
+  }
+  if (overlaps(d_gamma, ng, d_beta, ng) || overlaps(d_gamma, ng, gamma, ng) ||
+      overlaps(d_gamma, ng, beta, ng) || overlaps(d_beta, ng, gamma, ng) ||
+      overlaps(d_beta, ng, beta, ng))
+    return GDN_ERR_INVALID_ARG;
+  if (d_state_in && state_in && overlaps(d_state_in, ns, state_in, ns)) return GDN_ERR_INVALID_ARG;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const Problem p{B, H, T, N, D, key_scale};
+  return backward_path(dev, q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv,
+                       d_gamma, d_beta, d_state_in, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D) {
+  (void)N;
+  if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
+  return backward_ws_bytes(long(B) * H * T, D);
 }
 
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {

@@ -125,6 +125,20 @@ def clip_inputs(B: int, H: int, T: int, N: int, D: int, gamma_range=(0.9, 0.999)
     return {"q": q, "k": k, "v": v, "gamma": gamma, "beta": beta, "state": state}
 
 
+def cotangents(B: int, H: int, T: int, N: int, D: int, seed: int = 0, state_std: float = 0.0,
+               device="cpu") -> dict:
+    """Cotangents for the backward: d_out ([B,T,N,H,D] bf16, N(0,1)) and d_state_out
+    ([B,H,D,D] f32, N(0, state_std^2), or None when state_std is 0). Draw order: d_out,
+    d_state_out."""
+    g = _generator(seed, device)
+    d_out = normal_bf16((B, T, N, H, D), g, device)
+    d_state = None
+    if state_std > 0.0:
+        d_state = state_std * torch.randn((B, H, D, D), generator=g, device=device,
+                                          dtype=torch.float32)
+    return {"d_out": d_out, "d_state": d_state}
+
+
 def workload_inputs(w: Workload, device="cpu", step: Optional[int] = None) -> dict:
     """Inputs of a named workload.
 

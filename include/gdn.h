@@ -212,6 +212,44 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
                                float* state_out, float* z_out, int B, int H, int T, int N, int D,
                                int frames_per_block, gdn_stream_t stream);
 
+/*
+ * gdn_frame_backward - gradients of gdn_frame_forward, for training.
+ * (The chatpaper.ai abstract of SANA-WM says the model is trained natively on one-minute
+ * clips. The gen-hub.ru article, section "Архитектура", introduces the 1/sqrt(D*S) key scale as
+ * a training-stability fix. The pages give no backward; this is the chain rule of the forward.)
+ *
+ * Given the forward's inputs (q, k, v, gamma, beta, state_in) and the cotangents d_out
+ * (dL/dout, [B, T, N, H, D] bf16) and d_state_out (dL/dS_T, [B, H, D, D] f32, NULL = zero),
+ * computes dq, dk, dv ([B, T, N, H, D] bf16; dk is the gradient of the UNSCALED keys),
+ * d_gamma, d_beta ([B, T, H] f32) and, if d_state_in != NULL, dL/dS_0 ([B, H, D, D] f32).
+ * With G_t = dL/dS_t:
+ *   G_{T-1} = d_state_out + dO_{T-1}^T Q_{T-1},
+ *   G_{t-1} = gamma_t G_t (I - beta_t A_t) + dO_{t-1}^T Q_{t-1},  d_state_in = gamma_0 G_0 (I - beta_0 A_0),
+ *   dq_t = dO_t S_t,  dv_t = s beta_t K_t G_t^T,  dk_t = s beta_t (V_t G_t + K_t W'_t),
+ *   W'_t = -s gamma_t (S_{t-1}^T G_t + G_t^T S_{t-1}),
+ *   d_gamma_t = <G_t, S_{t-1}> - beta_t <G_t, S_{t-1} A_t>,  d_beta_t = <G_t, B_t> - gamma_t <G_t, S_{t-1} A_t>,
+ * with s = key_scale, A_t, B_t the forward's frame statistics and S_t the forward's states,
+ * which this call recomputes (nothing is kept from a forward call).
+ * Steps (8 launches on `stream`): the forward's statistics and state chain (S_t as bf16), the
+ * statistics E_t = dO_t^T Q_t, a reverse state chain for G_t (bf16 copies kept), a per-frame
+ * kernel for W'_t, d_gamma, d_beta, and three token GEMMs for dq, dv, dk.
+ * D must be a multiple of 8 in (64, 128] (GDN_ERR_UNSUPPORTED otherwise). All pointers are
+ * device pointers, 16-byte aligned. state_in, d_state_out and d_state_in may be NULL.
+ * dq, dk, dv must not overlap each other or q, k, v, d_out; d_gamma, d_beta must not overlap
+ * each other or gamma, beta; d_state_in must not overlap state_in (it may alias d_state_out).
+ * Workspace: gdn_backward_workspace_bytes(B, H, T, N, D) bytes, about 256 KB per frame-head
+ * at D = 128 (the shared per-GPU workspace grows to it).
+ */
+gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                              const float* gamma, const float* beta, const float* state_in,
+                              const gdn_bf16* d_out, const float* d_state_out, gdn_bf16* dq,
+                              gdn_bf16* dk, gdn_bf16* dv, float* d_gamma, float* d_beta,
+                              float* d_state_in, int B, int H, int T, int N, int D,
+                              float key_scale, gdn_stream_t stream);
+
+/* Device workspace bytes gdn_frame_backward needs for these sizes. */
+size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D);
+
 /* Device workspace bytes gdn_frame_forward / gdn_frame_step need for these sizes. */
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D);
 /* Device workspace bytes gdn_block_causal_la needs. */

@@ -135,3 +135,32 @@ def test_binding_refuses_cpu_tensors():
     g = torch.zeros((1, 2, 2), dtype=torch.float32)
     with pytest.raises(ValueError):
         api.gdn_frame_forward(q, q, q, g, g)
+
+
+def test_backward_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_frame_backward
+    # q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv, d_gamma, d_beta, d_state_in
+    def args(D=128, dq=P + 0x60000, dgam=P + 0x90000, ks=0.1, q=P, dsi=None, si=None):
+        return (q, P + 0x10000, P + 0x20000, P + 0x30000, P + 0x31000, si, P + 0x40000, None,
+                dq, P + 0x70000, P + 0x80000, dgam, P + 0x91000, dsi, 1, 2, 3, 16, D, ks, None)
+    assert f(*args(q=None)) == 1
+    assert f(*args(D=64)) == 2            # backward: 64 < D <= 128
+    assert f(*args(D=100)) == 2           # D % 8 != 0
+    assert f(*args(ks=float("nan"))) == 1
+    assert f(*args(dq=P + 0x60008)) == 3  # misaligned
+    assert f(*args(dq=P + 0x10000)) == 1  # dq overlaps k
+    assert f(*args(dgam=P + 0x31000)) == 1  # d_gamma overlaps beta
+    assert f(*args(si=P + 0xA0000, dsi=P + 0xA0000)) == 1  # d_state_in overlaps state_in
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*args()) == 5
+    assert lib.gdn_backward_workspace_bytes(1, 20, 961, 880, 128) > 19220 * 250_000
+
+
+def test_backward_binding_refuses_cpu_tensors():
+    import torch
+    from frame_wise_gated_deltanet_b200 import api
+    q = torch.zeros((1, 2, 16, 2, 128), dtype=torch.bfloat16)
+    g = torch.zeros((1, 2, 2), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        api.gdn_frame_backward(q, q, q, g, g, q)
