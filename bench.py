@@ -111,6 +111,8 @@ def kernel_bytes(name, w, fp8=False):
         if name == "gdn_fused_kernel":
             return algorithmic_bytes(w, True)
     dd = w.D * w.D
+    if name == "gdn_bwd_token_kernel_dkdv":  # read V, K, G_t, W'_t; write dK, dV
+        return fh * (4 * nd2 + 2 * dd * 2)
     if name.startswith("gdn_bwd_token_kernel_d"):  # read X tiles and frame matrices; write out
         terms = 2 if name.endswith("_dk") else 1
         return fh * ((terms + 1) * nd2 + terms * dd * 2)
@@ -154,6 +156,7 @@ KERNEL_SOURCES = {
     "gdn_bwd_token_kernel_dq": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_bwd_token_kernel_dv": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_bwd_token_kernel_dk": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_token_kernel_dkdv": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
 }
 
 
@@ -427,7 +430,7 @@ def main():
         raise RuntimeError("device status error during warm-up")
 
     # per-launch events the library records around each kernel (created before arming)
-    n_ev = 2 * 8 * a.steps
+    n_ev = 2 * 8 * a.steps  # at most 8 launches per step
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     for e in evs:
         e.record(stream)

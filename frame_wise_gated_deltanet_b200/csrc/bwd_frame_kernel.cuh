@@ -14,7 +14,12 @@
 // no-swizzle core-matrix layout along either index, so S^T G reads the same tiles the forward's
 // K-major GEMMs read, with LBO = 128 bytes between 8-row groups (the contraction index) and
 // SBO = DP*16 bytes between 8-key groups. One item per loop iteration and CTA (4 warps,
-// thread = TMEM lane = row); several CTAs per SM hide the latency of the loads.
+// thread = TMEM lane = row); two CTAs per SM hide each other's load latency.
+//
+// Every operand arrives with one round of memory latency: S_{t-1}, G_t and A_t by bulk copies
+// on one mbarrier, and each thread's row of B_t (32 float4 in the four-key interleaved layout)
+// as plain loads issued before that wait. <W, A> reads A_t by columns (A_t is symmetric), so
+// the 32 lanes of a warp read 64 contiguous bytes of shared memory.
 #pragma once
 #include <cuda.h>
 
@@ -27,7 +32,7 @@ struct BwdFrameLayout {
   static constexpr int kTileBytes = DP * DP * 2;
   static constexpr int kThreads = 128;
   static constexpr int kTmemCols = DP < 32 ? 32 : DP;
-  static constexpr int kSmemBytes = 2 * kTileBytes + 256 + 1024;
+  static constexpr int kSmemBytes = 3 * kTileBytes + 256 + 1024;  // S, G, A tiles
 };
 
 // S_ws, G_ws, W_out: bf16 DP x DP per row (s8 layout), row (b*H+h)*T + t; A_ws: bf16 D x D
@@ -46,7 +51,8 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
   uint8_t* smem = align1k(smem_raw);
   uint8_t* s_tile = smem;
   uint8_t* g_tile = smem + L::kTileBytes;
-  uint64_t* loaded = reinterpret_cast<uint64_t*>(g_tile + L::kTileBytes);
+  uint8_t* a_tile = g_tile + L::kTileBytes;  // A_t, D x D bf16 row-major
+  uint64_t* loaded = reinterpret_cast<uint64_t*>(a_tile + L::kTileBytes);
   uint64_t* mma_done = loaded + 1;
   uint64_t* mma_drain = mma_done + 1;  // all of this CTA's MMAs are complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
@@ -88,9 +94,21 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
     // ------------------------------------------------ S_{t-1} and G_t into shared memory
     if (tid == 0) {
       const uint64_t pol = policy_evict_first();
-      mbar_arrive_expect_tx(loaded, t >= 1 ? 2 * L::kTileBytes : L::kTileBytes);
+      const uint32_t a_bytes = static_cast<uint32_t>(DD * 2);
+      mbar_arrive_expect_tx(loaded, (t >= 1 ? 2 * L::kTileBytes : L::kTileBytes) + a_bytes);
       if (t >= 1) bulk_load(s_tile, S_ws + (row - 1) * DP * DP, L::kTileBytes, loaded, pol);
       bulk_load(g_tile, G_ws + row * DP * DP, L::kTileBytes, loaded, pol);
+      bulk_load(a_tile, A_ws + row * DD, a_bytes, loaded, pol);
+    }
+    // this thread's row r of B_t, 4 keys per float4 (in flight while the copies land)
+    float4 bq[DP / 4];
+    {
+      const float* bm = B_ws + row * DD;
+#pragma unroll
+      for (int i = 0; i < DP / 4; ++i)
+        bq[i] = (r < D && i < D / 4)
+                    ? __ldcs(reinterpret_cast<const float4*>(bm + b4_index(r, i * 4, D)))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (t == 0) {
       // S_{-1} = state_in, converted to the bf16 s8 layout (row r, 8 keys per 16 bytes)
@@ -142,24 +160,22 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
       __syncwarp();
     }
     // ------------------------------------------------ <G, S> and <G, B> (row r of each)
+    // (tiles are zero past D, and so is bq)
     float gs = 0.f, gb = 0.f, gsa = 0.f;
-    if (r < D) {
-      const float* bm = B_ws + row * DD;
-      for (int kg = 0; kg < D / 8; ++kg) {
-        const uint4 gv = *reinterpret_cast<const uint4*>(g_tile + kg * (DP * 16) + r * 16);
-        const uint4 sv = *reinterpret_cast<const uint4*>(s_tile + kg * (DP * 16) + r * 16);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
-        const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv);
-        const float4 b0 = __ldcs(reinterpret_cast<const float4*>(bm + b4_index(r, kg * 8, D)));
-        const float4 b1 = __ldcs(reinterpret_cast<const float4*>(bm + b4_index(r, kg * 8 + 4, D)));
-        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 gf = __bfloat1622float2(g2[j]);
-          const float2 sf = __bfloat1622float2(s2[j]);
-          gs = fmaf(gf.x, sf.x, fmaf(gf.y, sf.y, gs));
-          gb = fmaf(gf.x, bb[2 * j], fmaf(gf.y, bb[2 * j + 1], gb));
-        }
+    for (int kg = 0; kg < DP / 8; ++kg) {
+      const uint4 gv = *reinterpret_cast<const uint4*>(g_tile + kg * (DP * 16) + r * 16);
+      const uint4 sv = *reinterpret_cast<const uint4*>(s_tile + kg * (DP * 16) + r * 16);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+      const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv);
+      const float bb[8] = {bq[2 * kg].x,     bq[2 * kg].y,     bq[2 * kg].z,     bq[2 * kg].w,
+                           bq[2 * kg + 1].x, bq[2 * kg + 1].y, bq[2 * kg + 1].z, bq[2 * kg + 1].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 gf = __bfloat1622float2(g2[j]);
+        const float2 sf = __bfloat1622float2(s2[j]);
+        gs = fmaf(gf.x, sf.x, fmaf(gf.y, sf.y, gs));
+        gb = fmaf(gf.x, bb[2 * j], fmaf(gf.y, bb[2 * j + 1], gb));
       }
     }
     // ------------------------------------------------ read W row r: <W, A>, W' to global
@@ -168,23 +184,18 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
     const float gam = __ldg(gamma + (static_cast<long>(b) * T + t) * p.H + h);
     const float bet = __ldg(beta + (static_cast<long>(b) * T + t) * p.H + h);
     const float wscale = -p.key_scale * gam;
-    const __nv_bfloat16* arow = A_ws + row * DD + static_cast<long>(r) * D;
+    // column r of A_t (= row r: A_t is symmetric); lanes read consecutive elements
+    const __nv_bfloat16* acol = reinterpret_cast<const __nv_bfloat16*>(a_tile) + r;
     uint8_t* wdst = reinterpret_cast<uint8_t*>(W_out + row * DP * DP);
 #pragma unroll 1
     for (int c = 0; c < DP; c += 32) {
       float w[32];
       tmem_ld32(taddr + c, w);
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        if (r < D && c + j < D) {
-          const uint4 av = __ldcs(reinterpret_cast<const uint4*>(arow + c + j));
-          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&av);
+      for (int j = 0; j < 32; ++j)
+        if (r < D && c + j < D) gsa = fmaf(w[j], __bfloat162float(acol[(c + j) * D]), gsa);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 af = __bfloat1622float2(a2[e]);
-            gsa = fmaf(w[j + 2 * e], af.x, fmaf(w[j + 2 * e + 1], af.y, gsa));
-          }
-        }
+      for (int j = 0; j < 32; j += 8) {
         uint4 pk;
         pk.x = pack_bf16x2(wscale * w[j], wscale * w[j + 1]);
         pk.y = pack_bf16x2(wscale * w[j + 2], wscale * w[j + 3]);

@@ -7,6 +7,9 @@
 //   dV_t = s beta_t * K_t G_t^T          (1 term, Y = G_t read K-major: contraction over k)
 //   dK_t = s beta_t * (V_t G_t + K_t W'_t)   (2 terms: G_t MN-major, W'_t K-major)
 //
+// kDualV: dK_t and dV_t from one pass (the K tile and G_t are shared): a second accumulator
+// takes K_t G_t^T, and the epilogue stores both tiles through one staging buffer.
+//
 // with s the key scale, G_t = dL/dS_t from the backward chain and W'_t = -s gamma_t (S_{t-1}^T
 // G_t + G_t^T S_{t-1}) from the per-frame kernel (K_t here is the unscaled key tile, so both
 // factors of s are in these scalars).
@@ -22,9 +25,11 @@
 
 namespace gdn {
 
-template <int DP, int kTerms>
+template <int DP, int kTerms, bool kDualV = false>
 struct BwdTokenLayout {
   static_assert(DP == 128 && (kTerms == 1 || kTerms == 2), "DP = 128, one or two terms");
+  static_assert(!kDualV || kTerms == 2, "the dK/dV pass has two terms");
+  static constexpr int kAccs = kDualV ? 2 : 1;  // accumulators per tile
   static constexpr int kEpiWarps = 16;
   static constexpr int kCols = DP / 4;  // columns per epilogue thread
   static constexpr int kBoxes = DP / 64;
@@ -35,7 +40,7 @@ struct BwdTokenLayout {
   static constexpr int kOBufs = kTerms == 1 ? 2 : 1;
   static constexpr int kStageBytes = kTerms * kXBytes;
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
-  static constexpr int kTmemCols = 2 * DP;
+  static constexpr int kTmemCols = 2 * kAccs * DP;
   static constexpr int kOBytes = kXBytes;
   static constexpr int kSmemBytes =
       kYBufs * kTerms * kYBytes + kStages * kStageBytes + kOBufs * kOBytes + 512 + 1024;
@@ -48,12 +53,15 @@ struct BwdTokenArgs {
 };
 
 // kMN0 / kMN1: the term's frame matrix is read MN-major (contraction over its rows).
-template <int DP, int kTerms, bool kMN0, bool kMN1>
-__global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms>::kThreads, 1)
+// kDualV: tm_o2 takes s beta_t * X1 Y0^T (Y0 read K-major) from a second accumulator.
+template <int DP, int kTerms, bool kMN0, bool kMN1, bool kDualV = false>
+__global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 1)
     gdn_bwd_token_kernel(const __grid_constant__ CUtensorMap tm_x0,
                          const __grid_constant__ CUtensorMap tm_x1,
-                         const __grid_constant__ CUtensorMap tm_o, BwdTokenArgs a, Problem p) {
-  using L = BwdTokenLayout<DP, kTerms>;
+                         const __grid_constant__ CUtensorMap tm_o,
+                         const __grid_constant__ CUtensorMap tm_o2, BwdTokenArgs a, Problem p) {
+  using L = BwdTokenLayout<DP, kTerms, kDualV>;
+  constexpr int kAccs = L::kAccs;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
@@ -199,8 +207,19 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms>::kThreads, 1)
               // 2ks+1, 128 bytes apart; key groups DP*16 bytes apart)
               const uint64_t db = mn ? smem_desc_noswz(yt + ks * 256, 128, DP * 16)
                                      : smem_desc_noswz(yt + ks * 2 * DP * 16, DP * 16, 128);
-              mma_bf16(tmem_base + acc * DP, da, db, term == 0 ? idesc0 : idesc1,
+              mma_bf16(tmem_base + acc * kAccs * DP, da, db, term == 0 ? idesc0 : idesc1,
                        (term | ks) != 0);
+            }
+          }
+          if constexpr (kDualV) {
+            // second accumulator: X1 Y0^T, Y0 read K-major
+            constexpr uint32_t idesc_k = idesc_bf16(128, DP, false, false);
+            const uint32_t xb = x_base + L::kXBytes;
+#pragma unroll
+            for (int ks = 0; ks < DP / 16; ++ks) {
+              const uint64_t da = smem_desc(xb + (ks >> 2) * kBoxBytes + (ks & 3) * 32, 16, 1024);
+              const uint64_t db = smem_desc_noswz(y_base + ks * 2 * DP * 16, DP * 16, 128);
+              mma_bf16(tmem_base + (acc * kAccs + 1) * DP, da, db, idesc_k, ks != 0);
             }
           }
           mma_commit(&empty[stage]);
@@ -228,8 +247,12 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms>::kThreads, 1)
     const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
     const bool leader = (threadIdx.x == 64);
     const uint64_t pol_out = policy_evict_first();
-    if (leader) tma_prefetch_desc(&tm_o);
+    if (leader) {
+      tma_prefetch_desc(&tm_o);
+      if (kDualV) tma_prefetch_desc(&tm_o2);
+    }
     int tc = 0;
+    int nst = 0;  // staging tiles used (ring position)
     bool ok = true;
     for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       int bt, h;
@@ -241,38 +264,49 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms>::kThreads, 1)
         const int acc = tc & 1;
         const int valid = min(kRowsPerTile, p.N - tile * kRowsPerTile);
         const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
-        // the staging tile is free once the store issued kOBufs tiles ago has read it
-        if (leader) bulk_wait_read<L::kOBufs - 1>();
-        if (named_bar_any(1, kEpiThreads, !waited)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint8_t* ob = o_stage + (tc % L::kOBufs) * L::kOBytes;
-        if (static_cast<int>(quarter) * 32 < valid) {
-          const uint32_t tacc = lane_base + acc * DP;
-          float v[32];
-          tmem_ld32(tacc + c0, v);
+        bool lost = false;
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
-            pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
-            pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
-            pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
-            *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c0 + j, kBoxBytes)) = pk;
+        for (int o = 0; o < kAccs; ++o, ++nst) {
+          // the staging tile is free once the store issued kOBufs tiles ago has read it
+          if (leader) bulk_wait_read<L::kOBufs - 1>();
+          if (named_bar_any(1, kEpiThreads, !waited)) {
+            lost = true;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* ob = o_stage + (nst % L::kOBufs) * L::kOBytes;
+          if (static_cast<int>(quarter) * 32 < valid) {
+            const uint32_t tacc = lane_base + (acc * kAccs + o) * DP;
+            float v[32];
+            tmem_ld32(tacc + c0, v);
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 pk;
+              pk.x = pack_bf16x2(v[j] * scale, v[j + 1] * scale);
+              pk.y = pack_bf16x2(v[j + 2] * scale, v[j + 3] * scale);
+              pk.z = pack_bf16x2(v[j + 4] * scale, v[j + 5] * scale);
+              pk.w = pack_bf16x2(v[j + 6] * scale, v[j + 7] * scale);
+              *reinterpret_cast<uint4*>(ob + swz128_offset_bf16(row, c0 + j, kBoxBytes)) = pk;
+            }
+          }
+          if (o == kAccs - 1) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+          }
+          fence_async_smem();
+          named_bar(1, kEpiThreads);
+          if (leader) {
+            const CUtensorMap* tmo = o == 0 ? &tm_o : &tm_o2;
+#pragma unroll
+            for (int kb = 0; kb < L::kBoxes; ++kb)
+              tma_store_4d(tmo, ob + kb * kBoxBytes, kb * 64, h, tile * kRowsPerTile, bt,
+                           pol_out);
+            bulk_commit();
           }
         }
-        tc_fence_before();
-        mbar_arrive(&acc_empty[acc]);
-        fence_async_smem();
-        named_bar(1, kEpiThreads);
-        if (leader) {
-#pragma unroll
-          for (int kb = 0; kb < L::kBoxes; ++kb)
-            tma_store_4d(&tm_o, ob + kb * kBoxBytes, kb * 64, h, tile * kRowsPerTile, bt,
-                         pol_out);
-          bulk_commit();
+        if (lost) {
+          ok = false;
+          break;
         }
       }
     }

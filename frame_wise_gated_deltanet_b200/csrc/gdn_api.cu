@@ -122,6 +122,9 @@ struct DeviceState {
   int* step_flags = nullptr;  // hand-off words of the step kernel (persist across launches)
   long step_items = 0;
   int step_epoch = 0;
+  // second stream of the backward (work that overlaps the state chains) and its fork/join events
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
 };
 
 std::mutex g_mu;
@@ -233,9 +236,10 @@ gdn_status check_launch() {
 
 // ------------------------------------------------------------------ kernel runners
 // kB4: B_t in the chain's interleaved layout (forward paths) or row-major (gdn_frame_stats).
+// max_ctas > 0 caps the grid (the backward runs it beside the state chain's CTAs).
 template <int DP, bool kB4, bool kF8 = false>
 gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, void* A, float* Bm,
-                     cudaStream_t st) {
+                     cudaStream_t st, int max_ctas = 0) {
   using L = gdn::StatsLayout<DP, false, kF8>;
   CUtensorMap tk, tv;
   if (!tmap_in<kF8>(&tk, k, p) || !tmap_in<kF8>(&tv, v, p)) return GDN_ERR_CUDA;
@@ -244,7 +248,8 @@ gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, vo
           dev, kF8 ? 15 : (DP == 128 ? 0 : 1) + (kB4 ? 10 : 0), kern, L::kSmemBytes))
     return s;
   const long items = long(p.B) * p.T * p.H;
-  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  const long cap = max_ctas > 0 ? max_ctas : g_dev[dev].sms;
+  const int grid = static_cast<int>(items < cap ? items : cap);
   {
     ProfiledLaunch pl("gdn_stats_kernel", st);
     kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tk, tv, static_cast<__nv_bfloat16*>(A), Bm, p,
@@ -801,7 +806,7 @@ gdn_status run_bwd_frame(int dev, const Problem& p, const BackwardWs& w, const f
   auto kern = gdn::gdn_bwd_frame_kernel<128>;
   if (gdn_status s = ensure_smem_attr(dev, 21, kern, L::kSmemBytes)) return s;
   const long items = long(p.B) * p.H * p.T;
-  const long cap = 3L * g_dev[dev].sms;  // three CTAs of 67 KB shared memory per SM
+  const long cap = 2L * g_dev[dev].sms;  // two CTAs of 98 KB shared memory per SM
   const int grid = static_cast<int>(items < cap ? items : cap);
   {
     ProfiledLaunch pl("gdn_bwd_frame_kernel", st);
@@ -813,31 +818,54 @@ gdn_status run_bwd_frame(int dev, const Problem& p, const BackwardWs& w, const f
   return check_launch();
 }
 
-// One of the token GEMMs of the backward: out = scale * sum over terms of X_i Y_i^(T).
-template <int kTerms, bool kMN0, bool kMN1>
+// One of the token GEMMs of the backward: out = scale * sum over terms of X_i Y_i^(T)
+// (kDualV: also out2 = scale * X1 Y0^T).
+template <int kTerms, bool kMN0, bool kMN1, bool kDualV = false>
 gdn_status run_bwd_token(int dev, const Problem& p, const void* x0, const void* x1,
                          const void* Y0, const void* Y1, const float* beta, void* out,
-                         const char* name, int attr_bit, cudaStream_t st) {
-  using L = gdn::BwdTokenLayout<128, kTerms>;
-  CUtensorMap t0, t1, to;
+                         const char* name, int attr_bit, cudaStream_t st, int max_ctas = 0,
+                         void* out2 = nullptr) {
+  using L = gdn::BwdTokenLayout<128, kTerms, kDualV>;
+  CUtensorMap t0, t1, to, to2;
   if (!tmap_tokens(&t0, x0, p) || !tmap_tokens(&t1, kTerms == 2 ? x1 : x0, p) ||
-      !tmap_tokens(&to, out, p))
+      !tmap_tokens(&to, out, p) || !tmap_tokens(&to2, kDualV ? out2 : out, p))
     return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_bwd_token_kernel<128, kTerms, kMN0, kMN1>;
+  auto kern = gdn::gdn_bwd_token_kernel<128, kTerms, kMN0, kMN1, kDualV>;
   if (gdn_status s = ensure_smem_attr(dev, attr_bit, kern, L::kSmemBytes)) return s;
   const long items = long(p.B) * p.T * p.H;
-  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  const long cap = max_ctas > 0 ? max_ctas : g_dev[dev].sms;
+  const int grid = static_cast<int>(items < cap ? items : cap);
   const gdn::BwdTokenArgs a{static_cast<const __nv_bfloat16*>(Y0),
                             static_cast<const __nv_bfloat16*>(Y1), beta};
   {
     ProfiledLaunch pl(name, st);
-    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(t0, t1, to, a, p);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(t0, t1, to, to2, a, p);
   }
   return check_launch();
 }
 
 // The whole backward (64 < D <= 128): recompute the forward's statistics and states, then the
-// output statistics E_t, the backward chain, the per-frame kernel and the three token GEMMs.
+// output statistics E_t, the backward chain, the per-frame kernel and the token passes (dq;
+// dk and dv together).
+//
+// The two state chains run one CTA per head and leave most SMs idle, so when the heads fill at
+// most a quarter of the SMs, independent work runs beside them on a second stream (fork and join
+// through events, so the call stays ordered on `st` and can be captured in a graph):
+//   st:  stats(k, v) -> forward chain (S_t) -----> [E] backward chain (G_t) -> frame -> dk,dv -> [dq]
+//   aux:            [A] stats(q, dO) (E_t) --> [S] dq
+// The aux kernels' grids leave the chains' SMs free (a persistent grid that waited for them
+// would finish its last items after the chain).
+gdn_status aux_stream(int dev, DeviceState** out) {
+  DeviceState& d = g_dev[dev];
+  if (d.aux == nullptr) {
+    if (cudaStreamCreateWithFlags(&d.aux, cudaStreamNonBlocking) != cudaSuccess) return GDN_ERR_CUDA;
+    for (cudaEvent_t& e : d.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
+  }
+  *out = &d;
+  return GDN_OK;
+}
+
 gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
                          const float* gamma, const float* beta, const float* s_in,
                          const void* d_out, const float* ds_out, void* dq, void* dk, void* dv,
@@ -848,25 +876,41 @@ gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
   if (gdn_status s = get_workspace(dev, backward_ws_bytes(count, p.D), st, &base)) return s;
   const BackwardWs w = carve_backward(base, count, p.D);
   const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
-  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
-  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole, st))
-    return s;
   Problem pe = p;  // E_t = dO^T Q: the "B" statistic of (key = q, value = dO), key scale 1
   pe.key_scale = 1.0f;
-  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, st)) return s;
+  const long bh = long(p.B) * p.H;
+  const int sms = g_dev[dev].sms;
+  const bool overlap = bh * 4 <= sms;
+  DeviceState* d = nullptr;
+  if (overlap)
+    if (gdn_status s = aux_stream(dev, &d)) return s;
+  const int side = overlap ? static_cast<int>(sms - bh) : 0;  // aux grids beside the chains
+  cudaStream_t sx = overlap ? d->aux : st;
+  auto link = [&](cudaStream_t from, cudaStream_t to, int e) -> gdn_status {
+    if (!overlap) return GDN_OK;
+    if (cudaEventRecord(d->ev[e], from) != cudaSuccess) return GDN_ERR_CUDA;
+    return cudaStreamWaitEvent(to, d->ev[e], 0) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  };
+  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the forward statistics
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole, st))
+    return s;
+  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, sx, side)) return s;
+  if (gdn_status s = link(st, sx, 1)) return s;  // [S]: dq after the forward chain
+  if (gdn_status s = link(sx, st, 2)) return s;  // [E]: backward chain after E_t
+  if (gdn_status s = run_bwd_token<1, true, false>(dev, p, d_out, nullptr, w.S, nullptr, nullptr,
+                                                   dq, "gdn_bwd_token_kernel_dq", 22, sx, side))
+    return s;
   if (gdn_status s = run_bwd_chain(dev, p, w.A, w.E, gamma, beta, ds_out, w.G, ds_in, st))
     return s;
   if (gdn_status s = run_bwd_frame(dev, p, w, s_in, gamma, beta, d_gamma, d_beta, st)) return s;
-  if (gdn_status s = run_bwd_token<1, true, false>(dev, p, d_out, nullptr, w.S, nullptr, nullptr,
-                                                   dq, "gdn_bwd_token_kernel_dq", 22, st))
+  // dK and dV in one pass over the K tiles
+  if (gdn_status s = run_bwd_token<2, true, false, true>(dev, p, v, k, w.G, w.W, beta, dk,
+                                                         "gdn_bwd_token_kernel_dkdv", 25, st, 0,
+                                                         dv))
     return s;
-  if (gdn_status s = run_bwd_token<1, false, false>(dev, p, k, nullptr, w.G, nullptr, beta, dv,
-                                                    "gdn_bwd_token_kernel_dv", 23, st))
-    return s;
-  return run_bwd_token<2, true, false>(dev, p, v, k, w.G, w.W, beta, dk,
-                                       "gdn_bwd_token_kernel_dk", 24, st);
+  return link(sx, st, 3);  // [dq]: the call ends on `st` after everything
 }
-
 
 // ------------------------------------------------------------------ host-resident clips
 // gdn_frame_forward_host streams a clip held in host memory through the GPU in segments of
@@ -1302,6 +1346,12 @@ void gdn_release_workspace(void) {
   d.step_flags = nullptr;
   d.step_items = 0;
   d.step_epoch = 0;
+  for (cudaEvent_t& e : d.ev) {
+    if (e) cudaEventDestroy(e);
+    e = nullptr;
+  }
+  if (d.aux) cudaStreamDestroy(d.aux);
+  d.aux = nullptr;
 }
 
 int gdn_version(void) { return 100; }

@@ -230,9 +230,12 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
  *   d_gamma_t = <G_t, S_{t-1}> - beta_t <G_t, S_{t-1} A_t>,  d_beta_t = <G_t, B_t> - gamma_t <G_t, S_{t-1} A_t>,
  * with s = key_scale, A_t, B_t the forward's frame statistics and S_t the forward's states,
  * which this call recomputes (nothing is kept from a forward call).
- * Steps (8 launches on `stream`): the forward's statistics and state chain (S_t as bf16), the
- * statistics E_t = dO_t^T Q_t, a reverse state chain for G_t (bf16 copies kept), a per-frame
- * kernel for W'_t, d_gamma, d_beta, and three token GEMMs for dq, dv, dk.
+ * Steps (7 launches): the forward's statistics and state chain (S_t as bf16), the statistics
+ * E_t = dO_t^T Q_t, a reverse state chain for G_t (bf16 copies kept), a per-frame kernel for
+ * W'_t, d_gamma, d_beta, and two token passes (dq; dk with dv). When B*H is at most a quarter
+ * of the SM count, the E_t statistics and the dq pass run on an internal second stream beside
+ * the two state chains (forked from and joined back to `stream` through events, so the call
+ * is ordered on `stream` like any other and may be captured in a CUDA graph).
  * D must be a multiple of 8 in (64, 128] (GDN_ERR_UNSUPPORTED otherwise). All pointers are
  * device pointers, 16-byte aligned. state_in, d_state_out and d_state_in may be NULL.
  * dq, dk, dv must not overlap each other or q, k, v, d_out; d_gamma, d_beta must not overlap
