@@ -430,7 +430,7 @@ def main():
         raise RuntimeError("device status error during warm-up")
 
     # per-launch events the library records around each kernel (created before arming)
-    n_ev = 2 * 8 * a.steps  # at most 8 launches per step
+    n_ev = 2 * 16 * a.steps  # at most 16 launches per step
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     for e in evs:
         e.record(stream)
@@ -469,7 +469,13 @@ def main():
     dom = max(per_kernel, key=lambda n: per_kernel[n][0])
     dom_ms = per_kernel[dom][0] / per_kernel[dom][1]
     hbm, peak_kind = peaks()
+    # algorithmic bytes per launch: the kernel's bytes per step over its launches per step (the
+    # backward's statistics kernel makes two full passes per step; its segmented kernels split
+    # one pass over several launches)
     kb = kernel_bytes(dom, w, a.fp8)
+    if kb:
+        passes = 2 if (a.backward and dom == "gdn_stats_kernel") else 1
+        kb = kb * passes * a.steps / per_kernel[dom][1]
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
     path_bytes = backward_bytes(w) if a.backward else algorithmic_bytes(w, a.fp8)
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9

@@ -20,6 +20,11 @@
 // thread for its own slice with cp.async (four-key interleaved layout) two frames ahead. Every
 // G_t is also written to global memory as bf16 in the s8 layout, for the gradient GEMMs.
 //
+// A launch may cover a segment of frames [t_lo, t_hi) (walked from t_hi - 1 down to t_lo): it
+// starts from dS_T + E_{T-1} when t_hi = T, else from G_{t_hi-1} carried in f32 by the previous
+// segment's launch, and it ends with dS_0 when t_lo = 0, else with G_{t_lo-1} carried to the
+// next launch. The gradient passes of a finished segment then run while the chain continues.
+//
 // Warps: 0..15 epilogue, 16 TMA producer of A_t, 17 TMEM allocator + MMA issuer.
 #pragma once
 #include <cuda.h>
@@ -46,13 +51,16 @@ struct BwdChainLayout {
 
 // A_t: through tm_a, rows (b*H+h)*T + t of the forward statistics; E_ws: f32 D x D per row
 // (b4_index layout); G_out: bf16 DP x DP per row (s8 layout); d_state_out / d_state_in: f32
-// [B*H][D][D] row-major, nullptr = zero / not stored.
+// [B*H][D][D] row-major, nullptr = zero / not stored; carry: f32 [B*H][D][D] row-major, read
+// when t_hi < T and written when t_lo > 0 (the same memory is read and then written by the
+// same thread, so one buffer serves every segment).
 template <int DP>
 __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
     gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_a, const float* __restrict__ E_ws,
                          __nv_bfloat16* __restrict__ G_out, const float* __restrict__ gamma,
                          const float* __restrict__ beta, const float* __restrict__ d_state_out,
-                         float* __restrict__ d_state_in, Problem p) {
+                         float* __restrict__ d_state_in, float* carry, int t_lo, int t_hi,
+                         Problem p) {
   using L = BwdChainLayout<DP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
@@ -75,7 +83,8 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
   const int b = bh / p.H;
   const int h = bh - b * p.H;
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  // step u handles frame t = T-1-u: its MMA is G_t A_t
+  const int n = t_hi - t_lo;  // steps of this launch
+  // step u handles frame t = t_hi-1-u: its MMA is G_t A_t
   auto row_of = [&](int t) { return static_cast<long>(bh) * T + t; };
 
   if (threadIdx.x == 0) {
@@ -111,13 +120,13 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
         if (t >= 1)
           bulk_prefetch_l2(E_ws + row_of(t - 1) * DD, static_cast<uint32_t>(DD * 4));
       };
-      for (int u = 0; u < kPrefetch && u < T; ++u) prefetch(T - 1 - u);
+      for (int u = 0; u < kPrefetch && u < n; ++u) prefetch(t_hi - 1 - u);
       StageFills<L::kStages> fills;
-      for (int u = 0; u < T; ++u) {
-        const int t = T - 1 - u;
+      for (int u = 0; u < n; ++u) {
+        const int t = t_hi - 1 - u;
         const int stage = u % L::kStages;
         const uint32_t phase = (u / L::kStages) & 1;
-        if (u + kPrefetch < T) prefetch(t - kPrefetch);
+        if (u + kPrefetch < n) prefetch(t - kPrefetch);
         if (!mbar_wait(&empty[stage], phase ^ 1)) {
           give_up(none, abort_flag);
           break;
@@ -137,7 +146,7 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
     constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
     const uint32_t g_base = smem_u32(g_tile);
     bool ok = true;
-    for (int u = 0; u < T; ++u) {
+    for (int u = 0; u < n; ++u) {
       const int stage = u % L::kStages;
       const uint32_t phase = (u / L::kStages) & 1;
       if (!mbar_wait(&full[stage], phase) || !mbar_wait(g_ready, u & 1)) {
@@ -170,9 +179,11 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
     const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + c0;
     const bool row_ok = v < D;
     float X[L::kCols];
+    const bool first = t_hi == T;  // this launch starts at the clip's last frame
     {
-      // G_{T-1} = dS_T + E_{T-1}
-      const float* ds = d_state_out ? d_state_out + bh * DD + static_cast<long>(v) * D : nullptr;
+      // G_{T-1} = dS_T + E_{T-1}, or G_{t_hi-1} from the previous segment
+      const float* src = first ? d_state_out : carry;
+      const float* ds = src ? src + bh * DD + static_cast<long>(v) * D : nullptr;
       const float* el = E_ws + row_of(T - 1) * DD;
 #pragma unroll
       for (int j = 0; j < L::kCols; j += 4) {
@@ -180,8 +191,8 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
         float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         if (row_ok && col < D) {
-          e = __ldcg(reinterpret_cast<const float4*>(el + b4_index(v, col, D)));
-          if (ds) s = *reinterpret_cast<const float4*>(ds + col);
+          if (first) e = __ldcg(reinterpret_cast<const float4*>(el + b4_index(v, col, D)));
+          if (ds) s = __ldcg(reinterpret_cast<const float4*>(ds + col));
         }
         X[j] = s.x + e.x;
         X[j + 1] = s.y + e.y;
@@ -211,11 +222,12 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
     auto e_slot = [&](int buf, int kg) {
       return e_buf + buf * L::kEBufBytes + (static_cast<uint32_t>(kg) * 128 + v) * 16;
     };
-    // copy f (f = 0 .. T-2) brings E of frame T-2-f into buffer f % 2; one commit group per f,
-    // empty past the last copy so that the group count stays uniform
+    // copy f (f = 0 .. n-1, while frame t_hi-2-f exists) brings E of frame t_hi-2-f into
+    // buffer f % 2; one commit group per f, empty past the last copy so that the group count
+    // stays uniform
     auto issue_e = [&](int f) {
-      if (f <= T - 2 && row_ok) {
-        const float* em = E_ws + row_of(T - 2 - f) * DD;
+      if (f < n && t_hi - 2 - f >= 0 && row_ok) {
+        const float* em = E_ws + row_of(t_hi - 2 - f) * DD;
 #pragma unroll
         for (int j = 0; j < L::kCols; j += 4) {
           const int col = c0 + j;
@@ -230,20 +242,20 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
     fence_async_smem();
     tc_fence_before();
     mbar_arrive(g_ready);
-    store_g(T - 1);
+    if (first) store_g(T - 1);  // (a later segment's G_{t_hi-1} was stored by the previous one)
 
-    // gamma_t, beta_t of frames T-1-(32*blk + lane), shuffled from lane u % 32 at step u
+    // gamma_t, beta_t of frames t_hi-1-(32*blk + lane), shuffled from lane u % 32 at step u
     const long gb_base = static_cast<long>(b) * T * p.H + h;
     auto load_gb = [&](int blk, float& gv, float& bv) {
-      const int f = T - 1 - (blk * 32 + static_cast<int>(lane));
-      gv = f >= 0 ? __ldg(gamma + gb_base + static_cast<long>(f) * p.H) : 0.f;
-      bv = f >= 0 ? __ldg(beta + gb_base + static_cast<long>(f) * p.H) : 0.f;
+      const int f = t_hi - 1 - (blk * 32 + static_cast<int>(lane));
+      gv = f >= t_lo ? __ldg(gamma + gb_base + static_cast<long>(f) * p.H) : 0.f;
+      bv = f >= t_lo ? __ldg(beta + gb_base + static_cast<long>(f) * p.H) : 0.f;
     };
     float g_cur, b_cur, g_next, b_next;
     load_gb(0, g_next, b_next);
     bool ok = true;
-    for (int u = 0; u < T; ++u) {
-      const int t = T - 1 - u;
+    for (int u = 0; u < n; ++u) {
+      const int t = t_hi - 1 - u;
       if ((u & 31) == 0) {
         g_cur = g_next;
         b_cur = b_next;
@@ -276,20 +288,23 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
         }
       }
       if (has_e) {
-        // X = G_{t-1}: the operand of the next step's MMA (with A_{t-1})
-        write_tile();
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(g_ready);
+        // X = G_{t-1}: the operand of the next step's MMA (with A_{t-1}), unless t = t_lo
+        if (u + 1 < n) {
+          write_tile();
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(g_ready);
+        }
         store_g(t - 1);
       }
       issue_e(u + 2);  // buffer u % 2 is free (this thread read its own slice above)
     }
     cp_async_wait<0>();
     if (!ok) give_up(none, abort_flag);
-    if (ok && d_state_in != nullptr && row_ok) {
-      // X = dS_0 after the first frame's step
-      float* so = d_state_in + bh * DD + static_cast<long>(v) * D;
+    // X = dS_0 after the first frame's step, or G_{t_lo-1} for the next segment
+    float* const x_dst = t_lo == 0 ? d_state_in : carry;
+    if (ok && x_dst != nullptr && row_ok) {
+      float* so = x_dst + bh * DD + static_cast<long>(v) * D;
 #pragma unroll
       for (int j = 0; j < L::kCols; j += 4)
         if (c0 + j < D)

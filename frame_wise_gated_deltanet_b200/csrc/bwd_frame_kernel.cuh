@@ -37,7 +37,8 @@ struct BwdFrameLayout {
 
 // S_ws, G_ws, W_out: bf16 DP x DP per row (s8 layout), row (b*H+h)*T + t; A_ws: bf16 D x D
 // row-major per row; B_ws: f32 D x D per row (b4_index layout); state_in: f32 [B*H][D][D]
-// row-major (S_{-1}; nullptr = zero); d_gamma, d_beta: [B, T, H].
+// row-major (S_{-1}; nullptr = zero); d_gamma, d_beta: [B, T, H]. Items: frames [t_lo, t_hi)
+// of every head.
 template <int DP>
 __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
     gdn_bwd_frame_kernel(const __nv_bfloat16* __restrict__ S_ws,
@@ -45,7 +46,8 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
                          const __nv_bfloat16* __restrict__ A_ws, const float* __restrict__ B_ws,
                          const float* __restrict__ state_in, const float* __restrict__ gamma,
                          const float* __restrict__ beta, __nv_bfloat16* __restrict__ W_out,
-                         float* __restrict__ d_gamma, float* __restrict__ d_beta, Problem p) {
+                         float* __restrict__ d_gamma, float* __restrict__ d_beta, int t_lo,
+                         int t_hi, Problem p) {
   using L = BwdFrameLayout<DP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
@@ -64,7 +66,8 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
   const int T = p.T;
   const int D = p.D;
   const long DD = static_cast<long>(D) * D;
-  const long n_items = static_cast<long>(p.B) * p.H * T;
+  const int nt = t_hi - t_lo;
+  const long n_items = static_cast<long>(p.B) * p.H * nt;
 
   if (tid == 0) {
     mbar_init(loaded, 1);
@@ -86,11 +89,11 @@ __global__ void __launch_bounds__(BwdFrameLayout<DP>::kThreads)
 
   int li = 0;
   for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
-    const int bh = static_cast<int>(item / T);
-    const int t = static_cast<int>(item - static_cast<long>(bh) * T);
+    const int bh = static_cast<int>(item / nt);
+    const int t = t_lo + static_cast<int>(item - static_cast<long>(bh) * nt);
     const int b = bh / p.H;
     const int h = bh - b * p.H;
-    const long row = item;  // (b*H + h)*T + t
+    const long row = static_cast<long>(bh) * T + t;
     // ------------------------------------------------ S_{t-1} and G_t into shared memory
     if (tid == 0) {
       const uint64_t pol = policy_evict_first();

@@ -50,6 +50,7 @@ struct BwdTokenArgs {
   const __nv_bfloat16* Y0;  // frame matrices of term 0 / 1, DP*DP bf16 per row (b*H+h)*T + t
   const __nv_bfloat16* Y1;
   const float* beta;        // non-null: scale by key_scale * beta[b, t, h], else 1
+  int t_lo, t_hi;           // the frames [t_lo, t_hi) of every head
 };
 
 // kMN0 / kMN1: the term's frame matrix is read MN-major (contraction over its rows).
@@ -80,15 +81,17 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const long n_items = static_cast<long>(p.B) * p.T * p.H;
+  const int nt = a.t_hi - a.t_lo;
+  const long n_items = static_cast<long>(p.B) * nt * p.H;
   const int n_tiles = (p.N + kRowsPerTile - 1) / kRowsPerTile;
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  // item i = (b*T + t)*H + h
+  // item i = (b*nt + t - t_lo)*H + h; bt = b*T + t
   auto decode = [&](long item, int& bt, int& h, long& yrow) {
     h = static_cast<int>(item % p.H);
-    bt = static_cast<int>(item / p.H);
-    const int b = bt / p.T;
-    const int t = bt - b * p.T;
+    const int r = static_cast<int>(item / p.H);
+    const int b = r / nt;
+    const int t = a.t_lo + (r - b * nt);
+    bt = b * p.T + t;
     yrow = (static_cast<long>(b) * p.H + h) * p.T + t;
   };
 

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -124,7 +125,7 @@ struct DeviceState {
   int step_epoch = 0;
   // second stream of the backward (work that overlaps the state chains) and its fork/join events
   cudaStream_t aux = nullptr;
-  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 };
 
 std::mutex g_mu;
@@ -748,7 +749,8 @@ gdn_status validate_common(const void* q, const void* k, const void* v, const vo
 // ------------------------------------------------------------------ backward
 // Workspace of gdn_frame_backward, per frame-head: the forward's A_t (bf16 D x D), B_t (f32),
 // S_t (bf16 DP x DP), E_t = dO^T Q (f32), G_t (bf16 DP x DP) and W'_t (bf16 DP x DP; before the
-// per-frame kernel writes it, the same space takes the unused Q^T Q of the E statistics).
+// per-frame kernel writes it, the same space takes the unused Q^T Q of the E statistics); per
+// head the f32 G carried between segments of the backward chain.
 struct BackwardWs {
   void* A;
   float* B;
@@ -756,12 +758,13 @@ struct BackwardWs {
   float* E;
   void* G;
   void* W;
+  float* C;
 };
 
-size_t backward_ws_bytes(long count, int D) {
+size_t backward_ws_bytes(long count, int D, long bh) {
   const size_t m = size_t(D) * D, dp2 = size_t(128) * 128;
   return align256(count * m * 2) + align256(count * m * 4) + 3 * align256(count * dp2 * 2) +
-         align256(count * m * 4);
+         align256(count * m * 4) + align256(bh * m * 4);
 }
 
 BackwardWs carve_backward(void* base, long count, int D) {
@@ -779,12 +782,15 @@ BackwardWs carve_backward(void* base, long count, int D) {
   w.G = p;
   p += align256(count * dp2 * 2);
   w.W = p;
+  p += align256(count * dp2 * 2);
+  w.C = reinterpret_cast<float*>(p);
   return w;
 }
 
 gdn_status run_bwd_chain(int dev, const Problem& p, const void* A, const float* E,
                          const float* gamma, const float* beta, const float* d_state_out,
-                         void* G, float* d_state_in, cudaStream_t st) {
+                         void* G, float* d_state_in, float* carry, int t_lo, int t_hi,
+                         cudaStream_t st) {
   using L = gdn::BwdChainLayout<128>;
   const long count = long(p.B) * p.H * p.T;
   CUtensorMap ta;
@@ -794,26 +800,28 @@ gdn_status run_bwd_chain(int dev, const Problem& p, const void* A, const float* 
   {
     ProfiledLaunch pl("gdn_bwd_chain_kernel", st);
     kern<<<p.B * p.H, L::kThreads, L::kSmemBytes, st>>>(ta, E, static_cast<__nv_bfloat16*>(G),
-                                                        gamma, beta, d_state_out, d_state_in, p);
+                                                        gamma, beta, d_state_out, d_state_in,
+                                                        carry, t_lo, t_hi, p);
   }
   return check_launch();
 }
 
 gdn_status run_bwd_frame(int dev, const Problem& p, const BackwardWs& w, const float* state_in,
                          const float* gamma, const float* beta, float* d_gamma, float* d_beta,
-                         cudaStream_t st) {
+                         int t_lo, int t_hi, cudaStream_t st, int max_sms = 0) {
   using L = gdn::BwdFrameLayout<128>;
   auto kern = gdn::gdn_bwd_frame_kernel<128>;
   if (gdn_status s = ensure_smem_attr(dev, 21, kern, L::kSmemBytes)) return s;
-  const long items = long(p.B) * p.H * p.T;
-  const long cap = 2L * g_dev[dev].sms;  // two CTAs of 98 KB shared memory per SM
+  const long items = long(p.B) * p.H * (t_hi - t_lo);
+  // two CTAs of 98 KB shared memory per SM
+  const long cap = 2L * (max_sms > 0 ? max_sms : g_dev[dev].sms);
   const int grid = static_cast<int>(items < cap ? items : cap);
   {
     ProfiledLaunch pl("gdn_bwd_frame_kernel", st);
     kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(
         static_cast<const __nv_bfloat16*>(w.S), static_cast<const __nv_bfloat16*>(w.G),
         static_cast<const __nv_bfloat16*>(w.A), w.B, state_in, gamma, beta,
-        static_cast<__nv_bfloat16*>(w.W), d_gamma, d_beta, p);
+        static_cast<__nv_bfloat16*>(w.W), d_gamma, d_beta, t_lo, t_hi, p);
   }
   return check_launch();
 }
@@ -824,7 +832,8 @@ template <int kTerms, bool kMN0, bool kMN1, bool kDualV = false>
 gdn_status run_bwd_token(int dev, const Problem& p, const void* x0, const void* x1,
                          const void* Y0, const void* Y1, const float* beta, void* out,
                          const char* name, int attr_bit, cudaStream_t st, int max_ctas = 0,
-                         void* out2 = nullptr) {
+                         void* out2 = nullptr, int t_lo = 0, int t_hi = -1) {
+  if (t_hi < 0) t_hi = p.T;
   using L = gdn::BwdTokenLayout<128, kTerms, kDualV>;
   CUtensorMap t0, t1, to, to2;
   if (!tmap_tokens(&t0, x0, p) || !tmap_tokens(&t1, kTerms == 2 ? x1 : x0, p) ||
@@ -832,11 +841,11 @@ gdn_status run_bwd_token(int dev, const Problem& p, const void* x0, const void* 
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_bwd_token_kernel<128, kTerms, kMN0, kMN1, kDualV>;
   if (gdn_status s = ensure_smem_attr(dev, attr_bit, kern, L::kSmemBytes)) return s;
-  const long items = long(p.B) * p.T * p.H;
+  const long items = long(p.B) * (t_hi - t_lo) * p.H;
   const long cap = max_ctas > 0 ? max_ctas : g_dev[dev].sms;
   const int grid = static_cast<int>(items < cap ? items : cap);
   const gdn::BwdTokenArgs a{static_cast<const __nv_bfloat16*>(Y0),
-                            static_cast<const __nv_bfloat16*>(Y1), beta};
+                            static_cast<const __nv_bfloat16*>(Y1), beta, t_lo, t_hi};
   {
     ProfiledLaunch pl(name, st);
     kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(t0, t1, to, to2, a, p);
@@ -849,12 +858,14 @@ gdn_status run_bwd_token(int dev, const Problem& p, const void* x0, const void* 
 // dk and dv together).
 //
 // The two state chains run one CTA per head and leave most SMs idle, so when the heads fill at
-// most a quarter of the SMs, independent work runs beside them on a second stream (fork and join
-// through events, so the call stays ordered on `st` and can be captured in a graph):
-//   st:  stats(k, v) -> forward chain (S_t) -----> [E] backward chain (G_t) -> frame -> dk,dv -> [dq]
-//   aux:            [A] stats(q, dO) (E_t) --> [S] dq
-// The aux kernels' grids leave the chains' SMs free (a persistent grid that waited for them
-// would finish its last items after the chain).
+// most a quarter of the SMs, the rest runs beside them on a second stream (fork and join through
+// events, so the call stays ordered on `st` and can be captured in a graph), and the backward
+// chain is launched in segments of frames, last segment first, so that the per-frame and dk/dv
+// passes of a finished segment run while the chain walks the next one:
+//   st:  stats(k,v) -> forward chain -> [E] chain seg 1 -> chain seg 2 -> ... -> [end]
+//   aux:      [A] stats(q,dO) -> [S] dq -> [seg 1] frame, dk/dv -> [seg 2] frame, dk/dv -> ...
+// Kernels on the second stream that run beside a chain get grids that leave the chains' SMs free
+// (a persistent grid that waited for them would finish its last items after the chain).
 gdn_status aux_stream(int dev, DeviceState** out) {
   DeviceState& d = g_dev[dev];
   if (d.aux == nullptr) {
@@ -872,25 +883,30 @@ gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
                          float* d_gamma, float* d_beta, float* ds_in, const Problem& p,
                          cudaStream_t st) {
   const long count = long(p.B) * p.H * p.T;
+  const long bh = long(p.B) * p.H;
   void* base = nullptr;
-  if (gdn_status s = get_workspace(dev, backward_ws_bytes(count, p.D), st, &base)) return s;
+  if (gdn_status s = get_workspace(dev, backward_ws_bytes(count, p.D, bh), st, &base)) return s;
   const BackwardWs w = carve_backward(base, count, p.D);
   const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
   Problem pe = p;  // E_t = dO^T Q: the "B" statistic of (key = q, value = dO), key scale 1
   pe.key_scale = 1.0f;
-  const long bh = long(p.B) * p.H;
   const int sms = g_dev[dev].sms;
   const bool overlap = bh * 4 <= sms;
   DeviceState* d = nullptr;
   if (overlap)
     if (gdn_status s = aux_stream(dev, &d)) return s;
-  const int side = overlap ? static_cast<int>(sms - bh) : 0;  // aux grids beside the chains
+  const int side = overlap ? static_cast<int>(sms - bh) : 0;  // SMs beside the chains
   cudaStream_t sx = overlap ? d->aux : st;
   auto link = [&](cudaStream_t from, cudaStream_t to, int e) -> gdn_status {
     if (!overlap) return GDN_OK;
     if (cudaEventRecord(d->ev[e], from) != cudaSuccess) return GDN_ERR_CUDA;
     return cudaStreamWaitEvent(to, d->ev[e], 0) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
   };
+  // segments of the backward chain: about GDN_BWD_SEGMENT_FRAMES frames each (default 240)
+  const int seg_target = env_int("GDN_BWD_SEGMENT_FRAMES", 240, 1, 1 << 20);
+  const int n_seg = overlap ? std::max(1, (p.T + seg_target / 2) / seg_target) : 1;
+  const int seg_len = (p.T + n_seg - 1) / n_seg;
+
   if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
   if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the forward statistics
   if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole, st))
@@ -901,15 +917,22 @@ gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
   if (gdn_status s = run_bwd_token<1, true, false>(dev, p, d_out, nullptr, w.S, nullptr, nullptr,
                                                    dq, "gdn_bwd_token_kernel_dq", 22, sx, side))
     return s;
-  if (gdn_status s = run_bwd_chain(dev, p, w.A, w.E, gamma, beta, ds_out, w.G, ds_in, st))
-    return s;
-  if (gdn_status s = run_bwd_frame(dev, p, w, s_in, gamma, beta, d_gamma, d_beta, st)) return s;
-  // dK and dV in one pass over the K tiles
-  if (gdn_status s = run_bwd_token<2, true, false, true>(dev, p, v, k, w.G, w.W, beta, dk,
-                                                         "gdn_bwd_token_kernel_dkdv", 25, st, 0,
-                                                         dv))
-    return s;
-  return link(sx, st, 3);  // [dq]: the call ends on `st` after everything
+  for (int hi = p.T, lo; hi > 0; hi = lo) {
+    lo = std::max(0, hi - seg_len);
+    if (gdn_status s = run_bwd_chain(dev, p, w.A, w.E, gamma, beta, ds_out, w.G, ds_in, w.C, lo,
+                                     hi, st))
+      return s;
+    if (gdn_status s = link(st, sx, 4)) return s;  // [segment]: its G_t are stored
+    // the last segment's passes run after the chain: full grids
+    const int g = lo == 0 ? 0 : side;
+    if (gdn_status s = run_bwd_frame(dev, p, w, s_in, gamma, beta, d_gamma, d_beta, lo, hi, sx, g))
+      return s;
+    // dK and dV in one pass over the K tiles
+    if (gdn_status s = run_bwd_token<2, true, false, true>(
+            dev, p, v, k, w.G, w.W, beta, dk, "gdn_bwd_token_kernel_dkdv", 25, sx, g, dv, lo, hi))
+      return s;
+  }
+  return link(sx, st, 3);  // [end]: the call ends on `st` after everything
 }
 
 // ------------------------------------------------------------------ host-resident clips
@@ -1282,7 +1305,7 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
 size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D) {
   (void)N;
   if (B < 1 || H < 1 || T < 1 || D < 1) return 0;
-  return backward_ws_bytes(long(B) * H * T, D);
+  return backward_ws_bytes(long(B) * H * T, D, long(B) * H);
 }
 
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D) {

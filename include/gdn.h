@@ -44,6 +44,8 @@
  *  - GDN_CHUNK_LEN: frames per chunk of the chunked forward (read on every call; 0 or unset:
  *    chosen per problem).
  *  - GDN_HOST_SEGMENT_FRAMES: frames per segment of gdn_frame_forward_host (read on every call).
+ *  - GDN_BWD_SEGMENT_FRAMES: frames per segment of gdn_frame_backward's reverse state chain when
+ *    its gradient passes overlap the chain (default 240; read on every call).
  *  - GDN_TEST_WITHHOLD_FRAME: test hook only. The fused forward computes but never publishes the
  *    statistics of this frame of head 0, so the call ends with GDN_ERR_TIMEOUT (after the wait
  *    limit) instead of a result; used to test failure detection without faulting the GPU.
@@ -233,9 +235,10 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
  * Steps (7 launches): the forward's statistics and state chain (S_t as bf16), the statistics
  * E_t = dO_t^T Q_t, a reverse state chain for G_t (bf16 copies kept), a per-frame kernel for
  * W'_t, d_gamma, d_beta, and two token passes (dq; dk with dv). When B*H is at most a quarter
- * of the SM count, the E_t statistics and the dq pass run on an internal second stream beside
- * the two state chains (forked from and joined back to `stream` through events, so the call
- * is ordered on `stream` like any other and may be captured in a CUDA graph).
+ * of the SM count, the E_t statistics, the dq pass and the per-frame and dk/dv passes run on an
+ * internal second stream beside the two state chains, the reverse chain in segments of about
+ * GDN_BWD_SEGMENT_FRAMES frames (forked from and joined back to `stream` through events, so the
+ * call is ordered on `stream` like any other and may be captured in a CUDA graph).
  * D must be a multiple of 8 in (64, 128] (GDN_ERR_UNSUPPORTED otherwise). All pointers are
  * device pointers, 16-byte aligned. state_in, d_state_out and d_state_in may be NULL.
  * dq, dk, dv must not overlap each other or q, k, v, d_out; d_gamma, d_beta must not overlap

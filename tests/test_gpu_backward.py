@@ -9,6 +9,7 @@ gradients are sums of products of two rounded factors; d_state_in only carries t
 the chain's bf16 operand, like the forward's final state.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -79,6 +80,41 @@ def test_backward_matches_oracle(shape):
     got = api().gdn_frame_backward(g["q"], g["k"], g["v"], g["gamma"], g["beta"], gc["d_out"],
                                    state_in=g["state"], d_state_out=gc["d_state"], key_scale=ks)
     assert api().gdn_sync_status() == 0
+    check_against_oracle(x, c, got, ks)
+
+
+SEGMENTED = [
+    # (B, H, T, N, D, with_state, frames per segment of the reverse chain)
+    (1, 2, 10, 150, 128, True, 3),   # segments of 4, 4 and 2 frames
+    (2, 1, 7, 64, 96, False, 2),     # a segment ending at frame 0 after carried ones
+    (1, 3, 5, 200, 128, True, 1),    # one frame per segment
+]
+
+
+@pytest.mark.parametrize("shape", SEGMENTED, ids=lambda s: "B%dH%dT%dN%dD%d%s_seg%d" % (s[:5] + ("s" if s[5] else "", s[6])))
+def test_backward_segmented_chain_matches_oracle(shape):
+    """The reverse state chain in several launches (G carried in f32 between them), with each
+    segment's per-frame and dk/dv passes on the second stream beside the next segment."""
+    B, H, T, N, D, with_state, seg = shape
+    old = os.environ.get("GDN_BWD_SEGMENT_FRAMES")
+    os.environ["GDN_BWD_SEGMENT_FRAMES"] = str(seg)
+    try:
+        x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=750 + T + seg,
+                                   state_std=0.3 if with_state else 0.0)
+        c = gdn_inputs.cotangents(B, H, T, N, D, seed=850 + T + seg,
+                                  state_std=1.0 if with_state else 0.0)
+        ks = 1.0 / math.sqrt(D * N)
+        g = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+        gc = {k: (None if v is None else v.cuda()) for k, v in c.items()}
+        got = api().gdn_frame_backward(g["q"], g["k"], g["v"], g["gamma"], g["beta"],
+                                       gc["d_out"], state_in=g["state"],
+                                       d_state_out=gc["d_state"], key_scale=ks)
+        assert api().gdn_sync_status() == 0
+    finally:
+        if old is None:
+            os.environ.pop("GDN_BWD_SEGMENT_FRAMES", None)
+        else:
+            os.environ["GDN_BWD_SEGMENT_FRAMES"] = old
     check_against_oracle(x, c, got, ks)
 
 
