@@ -497,7 +497,8 @@ def main():
             "bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": (achieved / hbm) if achieved else None,
             "peak_source": f"{peak_kind} HBM copy bandwidth",
-            "traffic": ncu_traffic(dom, w.name + ("+fp8" if a.fp8 else "")),
+            "traffic": ncu_traffic(dom, w.name + ("+fp8" if a.fp8 else "")
+                                   + ("+bwd" if a.backward else "")),
             "algorithmic_bytes_per_launch": kb, "ms_per_launch": dom_ms,
             "path": {"algorithmic_bytes_per_step": path_bytes, "achieved_gbs": path_gbs,
                      "frac": path_gbs / hbm},
