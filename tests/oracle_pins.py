@@ -18,7 +18,8 @@ and raises ``AssertionError`` if the implementation disagrees with:
   linear map is a fixed point; split/resume through the state; linearity in
   (V, S_0); causality across frames and bidirectionality inside a frame; the
   unrolled affine-map product form of the recurrence);
-* for the backward: central differences of the forward, the exact dot-product (adjoint)
+* for the backward: a hand-worked scalar example (``tests/golden/``), central differences of
+  the forward, the exact dot-product (adjoint)
   identity of the map (V, S_0) -> (O, S_T), which is linear, the textbook gradients of
   unnormalised linear attention (one frame from a zero state), and linearity in the
   cotangents.
@@ -438,6 +439,26 @@ def _bwd_case(rng, B=2, T=3, N=3, H=2, D=3):
     return q, k, v, gamma, beta, S0, dO, dS
 
 
+def pin_bwd_hand_example(impl):
+    """Exact rationals worked by hand (tests/golden/gdn_backward_hand_example.json): a scalar
+    head (D = N = 1) over two frames, every gradient from the derivative of the definition."""
+    from fractions import Fraction
+    with open(os.path.join(GOLDEN, "gdn_backward_hand_example.json")) as f:
+        g = json.load(f)
+    tok = lambda x: np.array(x, dtype=np.float64).reshape(1, 2, 1, 1, 1)  # [1,T,N,H,D]
+    fr = lambda xs: np.array([float(Fraction(x)) for x in xs])
+    dq, dk, dv, dgam, dbet, ds0 = impl.gdn_frame_backward(
+        tok(g["q"]), tok(g["k"]), tok(g["v"]), np.array(g["gamma"]).reshape(1, 2, 1),
+        np.array(g["beta"]).reshape(1, 2, 1), np.full((1, 1, 1, 1), g["state_in"]),
+        tok(g["d_out"]), np.full((1, 1, 1, 1), g["d_state_out"]), g["key_scale"])
+    _close(dq.ravel(), fr(g["expected_dq"]), 1e-14, "hand example dq")
+    _close(dk.ravel(), fr(g["expected_dk"]), 1e-14, "hand example dk")
+    _close(dv.ravel(), fr(g["expected_dv"]), 1e-14, "hand example dv")
+    _close(dgam.ravel(), fr(g["expected_dgamma"]), 1e-14, "hand example dgamma")
+    _close(dbet.ravel(), fr(g["expected_dbeta"]), 1e-14, "hand example dbeta")
+    _close(ds0.ravel(), fr([g["expected_dstate_in"]]), 1e-14, "hand example dS_0")
+
+
 def pin_bwd_finite_differences(impl):
     """Every gradient against central differences of the (pinned) forward, for the scalar
     L = <dO, O> + <dS_T, S_T>. The forward is a polynomial in every input, so central
@@ -542,6 +563,7 @@ GDN_PINS = [
 LA_PINS = [pin_la_hand_example, pin_la_brute_force, pin_la_resume]
 FP8_PINS = [pin_e4m3_landmarks, pin_e4m3_ordering, pin_fp8_scales]
 BWD_PINS = [
+    pin_bwd_hand_example,
     pin_bwd_finite_differences,
     pin_bwd_adjoint_identity,
     pin_bwd_single_frame_closed_form,
