@@ -238,7 +238,9 @@ gdn_status gdn_block_causal_la(const gdn_bf16* q, const gdn_bf16* k, const gdn_b
  * of the SM count, the E_t statistics, the dq pass and the per-frame and dk/dv passes run on an
  * internal second stream beside the two state chains, the reverse chain in segments of about
  * GDN_BWD_SEGMENT_FRAMES frames (forked from and joined back to `stream` through events, so the
- * call is ordered on `stream` like any other and may be captured in a CUDA graph).
+ * call is ordered on `stream` like any other). The first such call on a GPU creates that stream
+ * and its events, and sizes the workspace; to capture the call in a CUDA graph, make one
+ * uncaptured call with the same sizes first.
  * D must be a multiple of 8 in (64, 128] (GDN_ERR_UNSUPPORTED otherwise). All pointers are
  * device pointers, 16-byte aligned. state_in, d_state_out and d_state_in may be NULL.
  * dq, dk, dv must not overlap each other or q, k, v, d_out; d_gamma, d_beta must not overlap
