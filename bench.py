@@ -141,6 +141,17 @@ def kernel_bytes(name, w, fp8=False):
     return None
 
 
+def per_launch_bytes(name, w, fp8, backward, steps, launches):
+    """Algorithmic bytes per launch: the kernel's bytes per step over its launches per step. The
+    backward's statistics kernel makes two full passes per step, (k, v) and (q, dO); its
+    segmented kernels split one pass over several launches."""
+    kb = kernel_bytes(name, w, fp8)
+    if not kb or launches < 1:
+        return None
+    passes = 2 if (backward and name == "gdn_stats_kernel") else 1
+    return kb * passes * steps / launches
+
+
 # Sources each kernel is built from: an ncu traffic figure stays valid while these are unchanged.
 KERNEL_SOURCES = {
     "gdn_fused_kernel": ["fused_kernel.cuh", "chain_kernel.cuh", "stats_kernel.cuh",
@@ -469,13 +480,7 @@ def main():
     dom = max(per_kernel, key=lambda n: per_kernel[n][0])
     dom_ms = per_kernel[dom][0] / per_kernel[dom][1]
     hbm, peak_kind = peaks()
-    # algorithmic bytes per launch: the kernel's bytes per step over its launches per step (the
-    # backward's statistics kernel makes two full passes per step; its segmented kernels split
-    # one pass over several launches)
-    kb = kernel_bytes(dom, w, a.fp8)
-    if kb:
-        passes = 2 if (a.backward and dom == "gdn_stats_kernel") else 1
-        kb = kb * passes * a.steps / per_kernel[dom][1]
+    kb = per_launch_bytes(dom, w, a.fp8, a.backward, a.steps, per_kernel[dom][1])
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
     path_bytes = backward_bytes(w) if a.backward else algorithmic_bytes(w, a.fp8)
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
