@@ -169,3 +169,38 @@ def test_backward_720p_sampled_heads():
     assert api().gdn_sync_status() == 0
     for h in (0, w.H - 1):
         check_against_oracle(x, c, got, w.key_scale, h_sl=slice(h, h + 1))
+
+
+def test_backward_in_a_cuda_graph():
+    """After one uncaptured call (which sizes the workspace and creates the internal stream), the
+    backward can be captured in a CUDA graph: the fork to the internal stream and the join back
+    are event nodes of the graph. Replays give the uncaptured call's result bit for bit."""
+    B, H, T, N, D = 1, 2, 9, 100, 128
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=905, state_std=0.3, device="cuda")
+    c = gdn_inputs.cotangents(B, H, T, N, D, seed=906, state_std=1.0, device="cuda")
+    a = api()
+    old = os.environ.get("GDN_BWD_SEGMENT_FRAMES")
+    os.environ["GDN_BWD_SEGMENT_FRAMES"] = "3"  # three segments: the second stream is used
+    try:
+        ref = a.gdn_frame_backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], c["d_out"],
+                                   state_in=x["state"], d_state_out=c["d_state"])
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                got = a.gdn_frame_backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"],
+                                           c["d_out"], state_in=x["state"],
+                                           d_state_out=c["d_state"], stream=s)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        assert a.gdn_sync_status() == 0
+    finally:
+        if old is None:
+            os.environ.pop("GDN_BWD_SEGMENT_FRAMES", None)
+        else:
+            os.environ["GDN_BWD_SEGMENT_FRAMES"] = old
+    for r, o in zip(ref, got):
+        assert torch.equal(r, o)
