@@ -17,6 +17,7 @@ grid, synthetic seeded bf16 inputs resident in HBM). Prints one JSON line (rank 
 * --impl reference: the oracle itself as the reference arm (host cores, bounded samples).
 * --backward: one step = one gdn_frame_backward (the gradients for a seeded d_out) instead of
   the forward; no e2e leg.
+* --rope: one step = gdn_rope_3d of the clip's q and k in place; no e2e or CPU-baseline leg.
 
 Multi-GPU (torchrun): every rank processes its own clip (independent problems, no collective
 on the data path), so scaling is weak.
@@ -40,6 +41,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GDN layer tokens·heads/sec and % of roofline (720p 60 s config, 1 B200)"
 METRIC_BWD = "GDN layer backward tokens·heads/sec (720p 60 s config, 1 B200)"
+METRIC_ROPE = "3D RoPE of q and k, tokens·heads/sec (720p 60 s config, 1 B200)"
 UNIT = "tokens*heads/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -62,6 +64,8 @@ def args_parse():
                     help="E4M3 q, k, v with per-(frame, head) scales (gdn_frame_forward_fp8)")
     ap.add_argument("--backward", action="store_true",
                     help="time gdn_frame_backward (the training pass) instead of the forward")
+    ap.add_argument("--rope", action="store_true",
+                    help="time gdn_rope_3d on the clip's q and k (in place) instead of the forward")
     ap.add_argument("--forward-mode", type=int, default=0,
                     help="gdn_set_forward_mode: 0 auto, 1 three kernels, 2 fused, 3 chunked")
     return ap.parse_args()
@@ -98,6 +102,11 @@ def backward_bytes(w):
     return fh * 7 * w.N * w.D * 2 + w.B * w.T * w.H * 4 * 4 + 2 * state
 
 
+def rope_bytes(w):
+    """Bytes of the 3D RoPE prologue per call: q and k read and written (bf16)."""
+    return w.B * w.H * w.T * 4 * w.N * w.D * 2
+
+
 def kernel_bytes(name, w, fp8=False):
     """Algorithmic bytes per launch of each kernel of the forward (the bytes its stage must
     move in the three-kernel design)."""
@@ -111,6 +120,8 @@ def kernel_bytes(name, w, fp8=False):
         if name == "gdn_fused_kernel":
             return algorithmic_bytes(w, True)
     dd = w.D * w.D
+    if name == "gdn_rope_kernel":        # one tensor read and written
+        return fh * 2 * nd2
     if name == "gdn_bwd_token_kernel_dkdv":  # read V, K, G_t, W'_t; write dK, dV
         return fh * (4 * nd2 + 2 * dd * 2)
     if name.startswith("gdn_bwd_token_kernel_d"):  # read X tiles and frame matrices; write out
@@ -148,7 +159,8 @@ def per_launch_bytes(name, w, fp8, backward, steps, launches):
     kb = kernel_bytes(name, w, fp8)
     if not kb or launches < 1:
         return None
-    passes = 2 if (backward and name == "gdn_stats_kernel") else 1
+    # (the RoPE step rotates q and k: two launches of one full pass each)
+    passes = 2 if ((backward and name == "gdn_stats_kernel") or name == "gdn_rope_kernel") else 1
     return kb * passes * steps / launches
 
 
@@ -412,6 +424,16 @@ def main():
             api.gdn_frame_forward_fp8(f8["q"], f8["k"], f8["v"], f8["sq"], f8["sk"], f8["sv"],
                                       gam, bet, None, out, st, key_scale=w.key_scale,
                                       stream=stream)
+    elif a.rope:
+        # the 3D RoPE prologue of the clip's q and k, in place (22 x 40 latent grid at 720p)
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        q, k = g["q"], g["k"]
+        gh, gw = (int(x) for x in w.grid.split("x"))
+        out = st = None
+
+        def step():
+            api.gdn_rope_3d(q, gh, gw, out=q, stream=stream)
+            api.gdn_rope_3d(k, gh, gw, out=k, stream=stream)
     elif a.backward:
         # the training pass: gradients of the clip for seeded cotangents of the output
         g = gdn_inputs.workload_inputs(w, device=dev)
@@ -482,17 +504,19 @@ def main():
     hbm, peak_kind = peaks()
     kb = per_launch_bytes(dom, w, a.fp8, a.backward, a.steps, per_kernel[dom][1])
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
-    path_bytes = backward_bytes(w) if a.backward else algorithmic_bytes(w, a.fp8)
+    path_bytes = (rope_bytes(w) if a.rope else
+                  backward_bytes(w) if a.backward else algorithmic_bytes(w, a.fp8))
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
 
     # ---------------------------------------------------------------- end to end, host buffers
     e2e = None
     if not a.no_e2e:
         e2e = (measure_e2e(a, w, g, out, st, stream, world, dev)
-               if w.kind == "gdn" and not a.fp8 and not a.backward else None)
+               if w.kind == "gdn" and not a.fp8 and not a.backward and not a.rope else None)
 
     line = {
-        "metric": METRIC_BWD if a.backward else METRIC, "value": value, "unit": UNIT,
+        "metric": METRIC_ROPE if a.rope else METRIC_BWD if a.backward else METRIC,
+        "value": value, "unit": UNIT,
         "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
@@ -514,7 +538,8 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn" and not a.fp8:
+    if (rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn" and not a.fp8
+            and not a.rope):
         heads = 1 if a.backward else 4
         rate, secs, threads = oracle_sample_rate(w, heads, w.T, backward=a.backward)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",

@@ -13,7 +13,7 @@ import torch
 from ._lib import LIB, GdnError, check
 
 __all__ = ["gdn_frame_forward", "gdn_frame_forward_fp8", "gdn_frame_forward_host",
-           "gdn_frame_step", "gdn_frame_backward", "gdn_backward_workspace_bytes", "gdn_frame_stats", "gdn_block_causal_la",
+           "gdn_frame_step", "gdn_frame_backward", "gdn_backward_workspace_bytes", "gdn_rope_3d", "gdn_frame_stats", "gdn_block_causal_la",
            "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
            "gdn_la_workspace_bytes", "GdnError"]
 
@@ -202,6 +202,22 @@ def gdn_frame_backward(q, k, v, gamma, beta, d_out, state_in=None, d_state_out=N
             _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_gamma), _ptr(d_beta),
             _ptr(d_state_in), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
     return dq, dk, dv, d_gamma, d_beta, d_state_in
+
+
+def gdn_rope_3d(x, grid_h: int, grid_w: int, base: float = 10000.0, t_offset: int = 0,
+                out=None, stream=None):
+    """3D RoPE of q or k ([B,T,N,H,D] bf16, N = grid_h * grid_w). out=x rotates in place.
+    Returns out."""
+    B, T, N, H, D = x.shape
+    _req(x, "x", torch.bfloat16, (B, T, N, H, D))
+    if out is None:
+        out = torch.empty_like(x)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    with torch.cuda.device(x.device):
+        check("gdn_rope_3d", LIB.gdn_rope_3d(
+            _ptr(x), _ptr(out), B, T, N, H, D, int(grid_h), int(grid_w), float(base),
+            int(t_offset), _stream(stream, x.device)))
+    return out
 
 
 def gdn_frame_stats(k, v, key_scale: Optional[float] = None, A_out=None, B_out=None, stream=None):

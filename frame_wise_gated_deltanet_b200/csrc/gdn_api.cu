@@ -19,6 +19,7 @@
 #include "fused_kernel.cuh"
 #include "la_scan_kernel.cuh"
 #include "output_kernel.cuh"
+#include "rope_kernel.cuh"
 #include "scan_kernel.cuh"
 #include "stats_kernel.cuh"
 #include "step_kernel.cuh"
@@ -1300,6 +1301,60 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
   const Problem p{B, H, T, N, D, key_scale};
   return backward_path(dev, q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv,
                        d_gamma, d_beta, d_state_in, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int H, int D,
+                       int grid_h, int grid_w, float base, int t_offset, gdn_stream_t stream) {
+  if (!x || !y) return GDN_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || N < 1 || H < 1 || D < 1 || grid_h < 1 || grid_w < 1 || t_offset < 0)
+    return GDN_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 1024) return GDN_ERR_UNSUPPORTED;
+  if (double(grid_h) * grid_w != double(N)) return GDN_ERR_INVALID_ARG;
+  if (!(std::isfinite(base) && base > 1.f)) return GDN_ERR_INVALID_ARG;
+  if (double(T) + t_offset > 2147483647.0) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return GDN_ERR_MISALIGNED;
+  const size_t n = size_t(B) * T * N * H * D * 2;
+  if (x != y && overlaps(x, n, y, n)) return GDN_ERR_INVALID_ARG;
+  gdn::RopeDims r;
+  r.B = B;
+  r.T = T;
+  r.N = N;
+  r.H = H;
+  r.D = D;
+  r.grid_w = grid_w;
+  r.d_h = 2 * (D / 6);
+  r.d_w = r.d_h;
+  r.d_t = D - 2 * r.d_h;
+  r.off_h = T * (r.d_t / 2);
+  r.off_w = r.off_h + grid_h * (r.d_h / 2);
+  const long n_tab = long(r.off_w) + long(grid_w) * (r.d_w / 2);
+  if (double(T) * (r.d_t / 2) + double(grid_h) * (r.d_h / 2) + double(grid_w) * (r.d_w / 2) >
+      2147483647.0)
+    return GDN_ERR_INVALID_ARG;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* base_ws = nullptr;
+  if (gdn_status s = get_workspace(dev, align256(size_t(n_tab) * sizeof(float2)), st, &base_ws))
+    return s;
+  float2* tab = static_cast<float2*>(base_ws);
+  {
+    ProfiledLaunch pl("gdn_rope_table_kernel", st);
+    gdn::gdn_rope_table_kernel<<<static_cast<unsigned>((n_tab + 255) / 256), 256, 0, st>>>(
+        tab, r, t_offset, std::log2(double(base)));
+    if (gdn_status s = check_launch()) return s;
+  }
+  const long n_vec = long(B) * T * N * H * (D / 8);
+  const long want = (n_vec + 255) / 256;
+  const long cap = 16L * g_dev[dev].sms;  // grid-stride: 16 blocks of 256 threads per SM
+  {
+    ProfiledLaunch pl("gdn_rope_kernel", st);
+    gdn::gdn_rope_kernel<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<__nv_bfloat16*>(y), tab, r,
+        n_vec);
+  }
+  return check_launch();
 }
 
 size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D) {

@@ -258,6 +258,31 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
 /* Device workspace bytes gdn_frame_backward needs for these sizes. */
 size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D);
 
+/*
+ * gdn_rope_3d - 3D rotary position embedding of q or k before the attention layers.
+ * (The transcript of the ICLR 2026 oral talk "SANA-Video: Efficient Video Generation with Block
+ * Linear Diffusion Transformer" introduces a 3D RoPE for the linear attention. The pages give no
+ * formula and do not say whether SANA-WM's GDN blocks apply it; the caller decides. The reading
+ * below is the plainest one.)
+ *
+ * x, y: [B, T, N, H, D] bf16 device pointers, 16-byte aligned. y may equal x (in place); any
+ * other overlap is rejected. The N tokens of a frame are a grid_h x grid_w latent grid, row-major
+ * (token n at row n / grid_w, column n % grid_w). The head dimension splits into three even
+ * slices: time d_t, rows d_h and columns d_w, with d_h = d_w = 2 * floor(D / 6) and
+ * d_t = D - 2 * d_h (44 / 42 / 42 at D = 128). In each slice of width d, the pairs
+ * (x_{2i}, x_{2i+1}) rotate by pos * base^(-2i / d):
+ *   (x, y) -> (x cos a - y sin a, x sin a + y cos a).
+ * pos is t + t_offset for the time slice (t_offset: absolute index of the clip's first frame, so
+ * a streaming step continues a clip), the row for the row slice, the column for the column slice.
+ * The angles are computed in double precision, the rotation in f32, and the result is rounded
+ * to bf16.
+ * D must be a multiple of 8 (GDN_ERR_UNSUPPORTED otherwise). grid_h * grid_w == N, base > 1 and
+ * t_offset >= 0 are required (GDN_ERR_INVALID_ARG). Two launches. Workspace: the cos/sin table,
+ * 8 * (T * d_t / 2 + grid_h * d_h / 2 + grid_w * d_w / 2) bytes, from the shared workspace.
+ */
+gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int H, int D,
+                       int grid_h, int grid_w, float base, int t_offset, gdn_stream_t stream);
+
 /* Device workspace bytes gdn_frame_forward / gdn_frame_step need for these sizes. */
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D);
 /* Device workspace bytes gdn_block_causal_la needs. */

@@ -164,3 +164,19 @@ def test_backward_binding_refuses_cpu_tensors():
     g = torch.zeros((1, 2, 2), dtype=torch.float32)
     with pytest.raises(ValueError):
         api.gdn_frame_backward(q, q, q, g, g, q)
+
+
+def test_rope_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_rope_3d
+    args = lambda D=128, gh=2, gw=8, base=10000.0, toff=0, y=P + 0x40000: (
+        P, y, 1, 3, 16, 2, D, gh, gw, base, toff, None)
+    assert f(*args(D=100)) == 2          # D % 8 != 0
+    assert f(*args(gh=3)) == 1           # grid_h * grid_w != N
+    assert f(*args(base=1.0)) == 1
+    assert f(*args(toff=-1)) == 1
+    assert f(*args(y=P + 0x10)) == 1     # partial overlap with x
+    assert f(*args(y=P + 0x40008)) == 3  # misaligned
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*args()) == 5
+        assert f(*args(y=P)) == 5        # in place passes the host checks
