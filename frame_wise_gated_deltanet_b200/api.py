@@ -2,10 +2,10 @@
 
 Tensors must be CUDA tensors of the dtypes and layouts ``include/gdn.h`` documents. Calls are
 asynchronous on ``stream`` (default: torch's current stream of the tensors' device).
+``key_scale=None`` passes 0 to the library, which then applies the layer's default key scale.
 """
 from __future__ import annotations
 
-import math
 from typing import Optional
 
 import torch
@@ -35,6 +35,12 @@ def _req(t: torch.Tensor, name: str, dtype, shape) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def _scale(key_scale) -> float:
+    """key_scale as the C ABI takes it: None becomes 0.0, which tells the library to apply the
+    layer's default scale (no arithmetic here)."""
+    return 0.0 if key_scale is None else float(key_scale)
+
+
 def _stream(stream, device) -> int:
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -59,12 +65,10 @@ def gdn_frame_forward(q, k, v, gamma, beta, state_in=None, out=None, state_out=N
         state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
     if state_out is not None:
         _req(state_out, "state_out", torch.float32, (B, H, D, D))
-    if key_scale is None:
-        key_scale = 1.0 / math.sqrt(D * N)
     with torch.cuda.device(q.device):
         check("gdn_frame_forward", LIB.gdn_frame_forward(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
-            _ptr(state_out), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
+            _ptr(state_out), B, H, T, N, D, _scale(key_scale), _stream(stream, q.device)))
     return out, state_out
 
 
@@ -95,13 +99,11 @@ def gdn_frame_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, gamma, beta, st
         state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q8.device)
     if state_out is not None:
         _req(state_out, "state_out", torch.float32, (B, H, D, D))
-    if key_scale is None:
-        key_scale = 1.0 / math.sqrt(D * N)
     with torch.cuda.device(q8.device):
         check("gdn_frame_forward_fp8", LIB.gdn_frame_forward_fp8(
             _ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
             _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out), _ptr(state_out),
-            B, H, T, N, D, float(key_scale), _stream(stream, q8.device)))
+            B, H, T, N, D, _scale(key_scale), _stream(stream, q8.device)))
     return out, state_out
 
 
@@ -139,13 +141,11 @@ def gdn_frame_forward_host(q, k, v, gamma, beta, state_in=None, out=None, state_
         state_out = torch.empty((B, H, D, D), dtype=torch.float32, pin_memory=True)
     if state_out is not None:
         _req_host(state_out, "state_out", torch.float32, (B, H, D, D))
-    if key_scale is None:
-        key_scale = 1.0 / math.sqrt(D * N)
     device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(device):
         check("gdn_frame_forward_host", LIB.gdn_frame_forward_host(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
-            _ptr(state_out), B, H, T, N, D, float(key_scale), _stream(stream, device)))
+            _ptr(state_out), B, H, T, N, D, _scale(key_scale), _stream(stream, device)))
     return out, state_out
 
 
@@ -166,12 +166,10 @@ def gdn_frame_step(q, k, v, gamma, beta, state_in=None, out=None, state_out=None
     if state_out is None:
         state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
     _req(state_out, "state_out", torch.float32, (B, H, D, D))
-    if key_scale is None:
-        key_scale = 1.0 / math.sqrt(D * N)
     with torch.cuda.device(q.device):
         check("gdn_frame_step", LIB.gdn_frame_step(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
-            _ptr(state_out), B, H, N, D, float(key_scale), _stream(stream, q.device)))
+            _ptr(state_out), B, H, N, D, _scale(key_scale), _stream(stream, q.device)))
     return out, state_out
 
 
@@ -194,13 +192,11 @@ def gdn_frame_backward(q, k, v, gamma, beta, d_out, state_in=None, d_state_out=N
     d_gamma, d_beta = torch.empty_like(gamma), torch.empty_like(beta)
     d_state_in = (torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
                   if want_state_grad else None)
-    if key_scale is None:
-        key_scale = 1.0 / math.sqrt(D * N)
     with torch.cuda.device(q.device):
         check("gdn_frame_backward", LIB.gdn_frame_backward(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(d_out),
             _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_gamma), _ptr(d_beta),
-            _ptr(d_state_in), B, H, T, N, D, float(key_scale), _stream(stream, q.device)))
+            _ptr(d_state_in), B, H, T, N, D, _scale(key_scale), _stream(stream, q.device)))
     return dq, dk, dv, d_gamma, d_beta, d_state_in
 
 
@@ -232,11 +228,9 @@ def gdn_frame_stats(k, v, key_scale: Optional[float] = None, A_out=None, B_out=N
         B_out = torch.empty((Bsz, H, T, D, D), dtype=torch.float32, device=k.device)
     _req(A_out, "A_out", torch.bfloat16, (Bsz, H, T, D, D))
     _req(B_out, "B_out", torch.float32, (Bsz, H, T, D, D))
-    if key_scale is None:
-        key_scale = 1.0 / math.sqrt(D * N)
     with torch.cuda.device(k.device):
         check("gdn_frame_stats", LIB.gdn_frame_stats(
-            _ptr(k), _ptr(v), _ptr(A_out), _ptr(B_out), Bsz, H, T, N, D, float(key_scale),
+            _ptr(k), _ptr(v), _ptr(A_out), _ptr(B_out), Bsz, H, T, N, D, _scale(key_scale),
             _stream(stream, k.device)))
     return A_out, B_out
 

@@ -232,6 +232,19 @@ gdn_status check_sizes(int B, int H, int T, int N, int D, int d_max) {
   return GDN_OK;
 }
 
+// The key scale of a call: 0 selects the pages' 1/sqrt(D*N) (D head dim, N tokens per frame;
+// gen-hub.ru SANA-WM article, "Архитектура"), any other value must be finite and > 0 and is used
+// as given. Returns false for an invalid value. D and N are already validated (>= 1).
+bool resolve_key_scale(float ks, int D, int N, float* out) {
+  if (ks == 0.f) {
+    *out = static_cast<float>(1.0 / std::sqrt(double(D) * double(N)));
+    return true;
+  }
+  if (!(std::isfinite(ks) && ks > 0.f)) return false;
+  *out = ks;
+  return true;
+}
+
 gdn_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -736,7 +749,8 @@ gdn_status validate_common(const void* q, const void* k, const void* v, const vo
                            const float* s_out, int B, int H, int T, int N, int D, float ks) {
   if (!q || !k || !v || !out || !gamma || !beta) return GDN_ERR_INVALID_ARG;
   if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
-  if (!(std::isfinite(ks) && ks > 0.f)) return GDN_ERR_INVALID_ARG;
+  float ks_eff;
+  if (!resolve_key_scale(ks, D, N, &ks_eff)) return GDN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
       (s_in && !aligned16(s_in)) || (s_out && !aligned16(s_out)))
     return GDN_ERR_MISALIGNED;
@@ -1094,6 +1108,7 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
   if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, T, N,
                                      D, key_scale))
     return s;
+  resolve_key_scale(key_scale, D, N, &key_scale);  // validated above
   const Problem p{B, H, T, N, D, key_scale};
   return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p,
                       reinterpret_cast<cudaStream_t>(stream));
@@ -1110,6 +1125,7 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
   if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, T, N,
                                      D, key_scale))
     return s;
+  resolve_key_scale(key_scale, D, N, &key_scale);  // validated above
   int dev;
   if (gdn_status s = current_device(&dev)) return s;
   std::lock_guard<std::mutex> lock(g_mu);
@@ -1145,7 +1161,7 @@ gdn_status gdn_frame_forward_fp8(const uint8_t* q, const uint8_t* k, const uint8
     return GDN_ERR_INVALID_ARG;
   if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
   if (D <= 64 || D % 16 != 0) return GDN_ERR_UNSUPPORTED;
-  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!resolve_key_scale(key_scale, D, N, &key_scale)) return GDN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
       (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
     return GDN_ERR_MISALIGNED;
@@ -1166,7 +1182,7 @@ gdn_status gdn_frame_forward_host(const gdn_bf16* q, const gdn_bf16* k, const gd
                                   int D, float key_scale, gdn_stream_t stream) {
   if (!q || !k || !v || !out || !gamma || !beta) return GDN_ERR_INVALID_ARG;
   if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
-  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!resolve_key_scale(key_scale, D, N, &key_scale)) return GDN_ERR_INVALID_ARG;
   const size_t n = size_t(B) * T * N * H * D * 2;
   if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
     return GDN_ERR_INVALID_ARG;
@@ -1182,6 +1198,7 @@ gdn_status gdn_frame_step(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* 
   if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, 1, N,
                                      D, key_scale))
     return s;
+  resolve_key_scale(key_scale, D, N, &key_scale);  // validated above
   const Problem p{B, H, 1, N, D, key_scale};
   if (D > 64 && g_forward_mode != 1) {
     int dev;
@@ -1199,7 +1216,7 @@ gdn_status gdn_frame_stats(const gdn_bf16* k, const gdn_bf16* v, gdn_bf16* A_out
                            gdn_stream_t stream) {
   if (!k || !v || !A_out || !B_out) return GDN_ERR_INVALID_ARG;
   if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
-  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!resolve_key_scale(key_scale, D, N, &key_scale)) return GDN_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(A_out) || !aligned16(B_out))
     return GDN_ERR_MISALIGNED;
   int dev;
@@ -1271,7 +1288,7 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
     return GDN_ERR_INVALID_ARG;
   if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
   if (D <= 64) return GDN_ERR_UNSUPPORTED;
-  if (!(std::isfinite(key_scale) && key_scale > 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!resolve_key_scale(key_scale, D, N, &key_scale)) return GDN_ERR_INVALID_ARG;
   const void* dev_ptrs[] = {q, k, v, gamma, beta, d_out, dq, dk, dv, d_gamma, d_beta};
   for (const void* ptr : dev_ptrs)
     if (!aligned16(ptr)) return GDN_ERR_MISALIGNED;
@@ -1414,12 +1431,27 @@ void gdn_release_workspace(void) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& d = g_dev[dev];
-  if (d.ws) {
-    cudaDeviceSynchronize();
-    cudaFree(d.ws);
-  }
+  cudaDeviceSynchronize();
+  if (d.ws) cudaFree(d.ws);
   d.ws = nullptr;
   d.ws_bytes = 0;
+  // per-context facts cached on the host: looked up again by the next call (after a context
+  // reset the old kernel attributes and the scratch address no longer hold)
+  d.attr_done = 0;
+  g_noalloc_addr[dev] = nullptr;
+  {
+    std::lock_guard<std::mutex> pl(g_pipe_mu);
+    HostPipe& hp = g_pipe[dev];
+    if (hp.ready) {
+      if (hp.buf) cudaFree(hp.buf);
+      cudaStreamDestroy(hp.s_in);
+      cudaStreamDestroy(hp.s_out);
+      cudaEvent_t evs[] = {hp.entry, hp.in_done[0], hp.in_done[1], hp.comp_done[0],
+                           hp.comp_done[1], hp.out_done[0], hp.out_done[1], hp.fin};
+      for (cudaEvent_t e : evs) cudaEventDestroy(e);
+    }
+    hp = HostPipe();
+  }
   if (d.step_flags) cudaFree(d.step_flags);
   d.step_flags = nullptr;
   d.step_items = 0;
@@ -1430,6 +1462,7 @@ void gdn_release_workspace(void) {
   }
   if (d.aux) cudaStreamDestroy(d.aux);
   d.aux = nullptr;
+  cudaGetLastError();  // handles of a context that was reset report errors: nothing to act on
 }
 
 int gdn_version(void) { return 100; }

@@ -25,6 +25,11 @@
  *    S k is a value. A NULL state_in means S_0 = 0; a NULL state_out skips the final store.
  *  - D must be a multiple of 8 in [8, 128]; B, H, T, N >= 1; every tensor pointer must be
  *    16-byte aligned (GDN_ERR_MISALIGNED otherwise).
+ *  - key_scale (every GDN entry point that takes one): 0 selects the pages' key scale
+ *    1/sqrt(D*N), computed by the library in double precision and rounded to f32 (D the head dim,
+ *    N the tokens per frame of the call; gen-hub.ru article, "Архитектура"); any other value
+ *    must be finite and > 0 and is used as given (1 for unscaled keys). Negative, NaN or
+ *    infinite values return GDN_ERR_INVALID_ARG.
  *  - out must not overlap q, k or v (GDN_ERR_INVALID_ARG). state_out may equal state_in
  *    (in-place streaming); any other partial overlap is undefined.
  *  - Errors found on the host are returned before anything is launched. Launch failures return
@@ -80,7 +85,7 @@ typedef enum gdn_status {
 /*
  * gdn_frame_forward - frame-wise GDN over a whole clip of T frames.
  * Computes out (all T frames) and, if state_out != NULL, S_T.
- * key_scale: the scale applied to keys (1/sqrt(D*N) for the pages' setting); finite, > 0.
+ * key_scale: the scale applied to keys; 0 selects the pages' 1/sqrt(D*N) (see above).
  * Workspace: gdn_workspace_bytes(B, H, T, N, D) bytes at most (three-kernel path: per-frame
  * A_t, B_t, S_t; fused path: per-head rings of A_t, B_t, S_t and hand-off flags; chunked path:
  * the three-kernel workspace plus per chunk one record of composed maps and one start state).
@@ -298,7 +303,14 @@ const char* gdn_status_string(gdn_status status);
  */
 gdn_status gdn_sync_status(gdn_stream_t stream);
 
-/* Free the cached workspace of the current GPU (synchronises the device first). */
+/*
+ * Free the cached workspace of the current GPU (synchronises the device first), with the
+ * step kernel's hand-off words, the backward's second stream and the host-buffer pipeline's
+ * staging buffers and streams. It also forgets what the library cached about the current
+ * CUDA context (kernel shared-memory attributes, the device address of
+ * gdn_frame_forward_noalloc's scratch), so after a context reset (cudaDeviceReset) call it
+ * once, with that GPU current, before the next library call on that GPU.
+ */
 void gdn_release_workspace(void);
 
 /*

@@ -74,8 +74,9 @@ def test_forward_rejects_bad_arguments_on_the_host(lib):
     assert _fwd(lib, N=0) == 1
     assert _fwd(lib, D=36) == 2     # not a multiple of 8
     assert _fwd(lib, D=136) == 2    # above 128
-    assert _fwd(lib, ks=0.0) == 1
+    assert _fwd(lib, ks=-0.5) == 1
     assert _fwd(lib, ks=float("nan")) == 1
+    assert _fwd(lib, ks=float("inf")) == 1
     assert _fwd(lib, q=P + 8) == 3  # misaligned
     assert _fwd(lib, out=P + 0x10000) == 1  # out overlaps k
 
@@ -106,7 +107,7 @@ def test_forward_fp8_rejects_bad_arguments_on_the_host(lib):
     assert f(*args(qs=None)) == 1
     assert f(*args(D=64)) == 2      # fp8 path: 64 < D <= 128
     assert f(*args(D=120)) == 2     # D % 16 != 0
-    assert f(*args(ks=0.0)) == 1
+    assert f(*args(ks=-1.0)) == 1
     import torch
     if not torch.cuda.is_available():
         assert f(*args()) == 5
@@ -180,3 +181,21 @@ def test_rope_rejects_bad_arguments_on_the_host(lib):
     if not torch.cuda.is_available():
         assert f(*args()) == 5
         assert f(*args(y=P)) == 5        # in place passes the host checks
+
+
+def test_zero_key_scale_selects_the_default_in_the_library(lib):
+    """key_scale == 0 is the documented request for the layer's 1/sqrt(D*N): the host checks
+    accept it (and the call then needs a GPU), and the header states the convention."""
+    import torch
+    text = open(HEADER).read()
+    assert "0 selects the pages' key scale" in text and "1/sqrt(D*N)" in text
+    if not torch.cuda.is_available():
+        assert _fwd(lib, ks=0.0) == 5
+        assert _fwd_host(lib, ks=0.0) == 5
+
+
+def test_binding_holds_no_key_scale_arithmetic():
+    """The Python binding passes key_scale through (None as 0); the default scale is computed
+    in the library."""
+    src = open(os.path.join(ROOT, "frame_wise_gated_deltanet_b200", "api.py")).read()
+    assert "sqrt" not in src and "import math" not in src
