@@ -44,6 +44,7 @@ METRIC_BWD = "GDN layer backward tokens·heads/sec (720p 60 s config, 1 B200)"
 METRIC_ROPE = "3D RoPE of q and k, tokens·heads/sec (720p 60 s config, 1 B200)"
 UNIT = "tokens*heads/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def args_parse():
@@ -66,6 +67,12 @@ def args_parse():
                     help="time gdn_frame_backward (the training pass) instead of the forward")
     ap.add_argument("--rope", action="store_true",
                     help="time gdn_rope_3d on the clip's q and k (in place) instead of the forward")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other configurations' records (480p, stream, LA, fp8, "
+                         "backward, RoPE) that the default 720p run adds to its line")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="under torchrun: 'heads' splits one clip's heads over the ranks "
+                         "(strong scaling) instead of one clip per rank (weak scaling)")
     ap.add_argument("--forward-mode", type=int, default=0,
                     help="gdn_set_forward_mode: 0 auto, 1 three kernels, 2 fused, 3 chunked")
     return ap.parse_args()
@@ -79,6 +86,25 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 tensor peak in TFLOP/s: the measured burst figure (a kernel timed alone), else
+    the recipe's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured dense bf16 (cuBLAS, burst)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback dense bf16"
+
+
+def softmax_flops(B, H, T, N, D, F):
+    """Algorithmic flops of chunk-causal softmax attention: 2*D for a query-key score and 2*D
+    for its share of P V, over every visible (query, key) pair."""
+    pairs = sum(N * min(T, (t // F + 1) * F) * N for t in range(T))
+    return B * H * 4 * D * pairs
 
 
 def algorithmic_bytes(w, fp8=False):
@@ -325,6 +351,21 @@ def oracle_sample_rate(w, heads, frames, seed=99, backward=False):
     return heads * frames * w.N / dt, dt, threads
 
 
+def host_info():
+    """The host's usable cores (affinity mask) and CPU model, for the CPU baseline's record."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": cores, "cpu_model": model}
+
+
 def run_reference(a, w):
     """The oracle as the reference arm: each step is a bounded sample (1 head x 192 frames)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -348,21 +389,23 @@ def run_reference(a, w):
         "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": dict({"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                              "sample": sample}, **host_info()),
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
 
 
-def workload_config(w):
+def workload_config(w, shard=False, world=1):
     what = {"stream": "streaming step", "la": "block-causal LA clip"}.get(w.kind, "GDN clip")
+    par = ("one clip's heads split over %d GPUs (contiguous head ranges, no collective)" % world
+           if shard else "independent clip per GPU")
     return {"workload": f"{w.name} {what}: B{w.B} H{w.H} D{w.D} T{w.T} N{w.N} ({w.grid} grid)",
             "B": w.B, "H": w.H, "D": w.D, "T": w.T, "N": w.N, "key_scale": w.key_scale,
             "gamma_range": list(w.gamma_range), "beta_range": list(w.beta_range),
             "l2": "inputs (%.1f GB of q,k,v) larger than the 126 MB L2; no flush"
                   % (3 * w.B * w.T * w.N * w.H * w.D * 2 / 1e9),
-            "parallelism": "independent clip per GPU"}
+            "parallelism": par}
 
 
 def main():
@@ -383,6 +426,18 @@ def main():
 
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
+    # --shard heads: the ranks split one clip's heads (strong scaling; per-rank byte counts use
+    # the rank's own heads); otherwise every rank runs its own clip (weak scaling)
+    shard = a.shard == "heads" and world > 1
+    if a.shard == "heads" and (w.kind != "gdn" or a.fp8 or a.backward or a.rope):
+        raise ValueError("--shard heads applies to the bf16 forward of a GDN clip")
+    w_rank = w
+    if shard:
+        from frame_wise_gated_deltanet_b200.parallel import head_range
+        h0, h1 = head_range(w.H, world, rank)
+        if h1 == h0:
+            raise ValueError(f"--shard heads: rank {rank} of {world} would own no head of {w.H}")
+        w_rank = dataclasses.replace(w, H=h1 - h0, name=f"{w.name}[heads {h0}:{h1}]")
     if _lib.LIB.gdn_set_forward_mode(a.forward_mode) != 0:
         raise ValueError(f"invalid --forward-mode {a.forward_mode}")
     stream = torch.cuda.current_stream(dev)
@@ -447,9 +502,16 @@ def main():
                                    stream=stream)
     else:
         g = gdn_inputs.workload_inputs(w, device=dev)
+        if shard:
+            # this rank's heads of the one clip, as a column-parallel projection hands them over
+            from frame_wise_gated_deltanet_b200.parallel import shard_heads
+            g = {n: (None if t is None else
+                     shard_heads(t, world, rank, {5: 3, 3: 2, 4: 1}[t.dim()]))
+                 for n, t in g.items()}
+            torch.cuda.empty_cache()
         q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
         out = torch.empty_like(q)
-        st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+        st = torch.empty((w_rank.B, w_rank.H, w.D, w.D), dtype=torch.float32, device=dev)
 
         def step():
             api.gdn_frame_forward(q, k, v, gam, bet, None, out, st, key_scale=w.key_scale,
@@ -493,7 +555,12 @@ def main():
         raise RuntimeError(f"device status {status} after the timed region (this rank)")
 
     ms_local = t_start.elapsed_time(t_end)
-    value, ms = job_throughput(w.tokens_heads * a.steps, ms_local, world)
+    if shard:  # one clip over all ranks: its units once, in the slowest rank's time
+        ms = max_over_ranks(ms_local, world)
+        value = w.tokens_heads * a.steps / (ms * 1e-3)
+    else:
+        value, ms = job_throughput(w.tokens_heads * a.steps, ms_local, world)
+    w_all, w = w, w_rank  # per-rank byte accounting below
     per_kernel = {}
     for i, n in enumerate(names):
         d = evs[2 * i].elapsed_time(evs[2 * i + 1])
@@ -513,15 +580,26 @@ def main():
     if not a.no_e2e:
         e2e = (measure_e2e(a, w, g, out, st, stream, world, dev)
                if w.kind == "gdn" and not a.fp8 and not a.backward and not a.rope else None)
+        if shard and e2e and e2e.get("ms_per_step"):
+            # the ranks' copies and computes cover one clip: its units in the slowest rank's time
+            e2e["value"] = w_all.tokens_heads / (e2e["ms_per_step"] * 1e-3)
+
+    workloads = None
+    if (not a.no_workloads and world == 1 and w.kind == "gdn" and w.name == "720p" and not a.fp8
+            and not a.backward and not a.rope):
+        sampler2 = ClockSampler("GPU-" + str(props.uuid))
+        sampler2.start()
+        workloads = measure_workloads(dev, stream, g)
+        workloads["clocks"] = sampler2.stop()
 
     line = {
         "metric": METRIC_ROPE if a.rope else METRIC_BWD if a.backward else METRIC,
         "value": value, "unit": UNIT,
         "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if shard else "weak", "vs_baseline": None,
         "dtype": "e4m3 q/k/v, bf16 out" if a.fp8 else "bf16", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w_all, shard, world),
         "roofline": {
             "bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": (achieved / hbm) if achieved else None,
@@ -538,20 +616,291 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
     }
+    if workloads is not None:
+        line["workloads"] = workloads
     if (rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn" and not a.fp8
             and not a.rope):
         heads = 1 if a.backward else 4
         rate, secs, threads = oracle_sample_rate(w, heads, w.T, backward=a.backward)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"{heads} head(s) x {w.T} frames of the {w.name} clip "
-                                          f"shape (N={w.N}, D={w.D}), "
-                                          f"{'backward' if a.backward else 'forward'}, "
-                                          f"{secs:.1f} s of fp64 numpy"}
+        line["cpu_baseline"] = dict({"value": rate, "unit": UNIT, "cores": threads,
+                                     "kind": "oracle",
+                                     "sample": f"{heads} head(s) x {w.T} frames of the {w.name} "
+                                               f"clip shape (N={w.N}, D={w.D}), "
+                                               f"{'backward' if a.backward else 'forward'}, "
+                                               f"{secs:.1f} s of fp64 numpy"}, **host_info())
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def timed(step, steps, stream, max_launches_per_step=16):
+    """Run step() `steps` times between two CUDA events on `stream`, with the library's per-launch
+    events armed. Returns (ms for all steps, {kernel: (ms total, launches)}, launches)."""
+    import ctypes
+    import torch
+    from frame_wise_gated_deltanet_b200 import _lib
+    n_ev = 2 * max_launches_per_step * steps
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in evs:
+        e.record(stream)  # creates the event
+    handles = (ctypes.c_void_p * n_ev)(*[e.cuda_event for e in evs])
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    _lib.LIB.gdn_profile_arm(handles, n_ev)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = _lib.LIB.gdn_profile_count()
+    names = [_lib.LIB.gdn_profile_kernel(i).decode() for i in range(launches)]
+    _lib.LIB.gdn_profile_arm(None, 0)
+    per_kernel = {}
+    for i, n in enumerate(names):
+        d = evs[2 * i].elapsed_time(evs[2 * i + 1])
+        tot, cnt = per_kernel.get(n, (0.0, 0))
+        per_kernel[n] = (tot + d, cnt + 1)
+    return t0.elapsed_time(t1), per_kernel, launches
+
+
+def rotating(copies):
+    """A callable returning the next of `copies` on each call (inputs of a workload smaller than
+    L2 rotate over enough copies that each step reads data no earlier step left in L2)."""
+    state = {"i": -1}
+
+    def nxt():
+        state["i"] = (state["i"] + 1) % len(copies)
+        return copies[state["i"]]
+    return nxt
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def n_copies(bytes_per_step):
+    """Copies of a workload's inputs so that the ones a step reads were last read two L2 sizes
+    of traffic ago (1 when one copy is already larger than twice the L2)."""
+    return max(1, -(-2 * L2_BYTES // max(bytes_per_step, 1)) + 1) if bytes_per_step < 2 * L2_BYTES else 1
+
+
+def workload_record(label, w, step, stream, path_bytes, kernel_bytes_fn, units_per_step,
+                    warmup=3, target_ms=400.0, max_steps=400, flops_per_step=None,
+                    tensor_peak=None, l2_note="", launches_per_step=16):
+    """Time one extra workload of the run: warm-up, then about target_ms of steps. Returns its
+    record: ms per step, tokens*heads/s, the dominant kernel with its roofline fraction against
+    the measured peak, and the whole path's fraction."""
+    import torch
+    from frame_wise_gated_deltanet_b200 import api
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.gdn_sync_status() != 0:
+        raise RuntimeError(f"device status error in the {label} warm-up")
+    ms1, _, _ = timed(step, 1, stream, launches_per_step)
+    steps = int(max(3, min(max_steps, target_ms / max(ms1, 1e-3))))
+    ms, per_kernel, launches = timed(step, steps, stream, launches_per_step)
+    if api.gdn_sync_status() != 0:
+        raise RuntimeError(f"device status error in the {label} timed region")
+    hbm, peak_kind = peaks()
+    dom = max(per_kernel, key=lambda n: per_kernel[n][0])
+    dom_ms = per_kernel[dom][0] / per_kernel[dom][1]
+    kb = kernel_bytes_fn(dom, per_kernel[dom][1], steps)
+    step_ms = ms / steps
+    rec = {
+        "workload": w if isinstance(w, str) else workload_config(w)["workload"],
+        "ms_per_step": step_ms,
+        "tokens_heads_per_s": units_per_step / (step_ms * 1e-3),
+        "steps": steps, "warmup": warmup,
+        "gpu_launches": launches,
+        "dominant_kernel": {"name": dom, "ms_per_launch": dom_ms,
+                            "share": per_kernel[dom][0] / sum(t for t, _ in per_kernel.values())},
+        "path": {"bound": "hbm", "algorithmic_bytes_per_step": path_bytes,
+                 "achieved_gbs": path_bytes / (step_ms * 1e-3) / 1e9,
+                 "peak_gbs": hbm, "frac": path_bytes / (step_ms * 1e-3) / 1e9 / hbm,
+                 "peak_source": f"{peak_kind} HBM copy bandwidth"},
+        "kernels": {n: {"launches": c, "ms_total": t} for n, (t, c) in per_kernel.items()},
+        "l2": l2_note or "inputs larger than the 126 MB L2; no flush",
+    }
+    if kb:
+        rec["dominant_kernel"].update(
+            {"algorithmic_bytes_per_launch": kb, "achieved_gbs": kb / (dom_ms * 1e-3) / 1e9,
+             "frac": kb / (dom_ms * 1e-3) / 1e9 / hbm})
+    if flops_per_step and tensor_peak:
+        tf = flops_per_step / (step_ms * 1e-3) / 1e12
+        rec["path"] = {"bound": "tensor", "algorithmic_flops_per_step": flops_per_step,
+                       "achieved_tflops": tf, "peak_tflops": tensor_peak[0],
+                       "frac": tf / tensor_peak[0], "peak_source": tensor_peak[1]}
+        fpl = flops_per_step * steps / per_kernel[dom][1]  # flops per launch of the kernel
+        ktf = fpl / (dom_ms * 1e-3) / 1e12
+        rec["dominant_kernel"].update({"algorithmic_flops_per_launch": fpl,
+                                       "achieved_tflops": ktf, "frac": ktf / tensor_peak[0],
+                                       "bound": "tensor"})
+    return rec
+
+
+def measure_workloads(dev, stream, g720=None):
+    """The other configurations of the layer, timed in the same run as the contract line: the
+    480p clip, the streaming workload (64 chained single-frame steps per step), the block-causal
+    LA clip, and on the 720p clip the E4M3-input forward, the backward and the standalone 3D RoPE
+    of q and k. Each record: ms per step, tokens*heads/s, the dominant kernel's and the path's
+    fraction of the measured roofline."""
+    import torch
+    import gdn_inputs
+    from frame_wise_gated_deltanet_b200 import api
+    W = gdn_inputs.WORKLOADS
+    recs = {}
+    tok_bytes = lambda w: w.B * w.T * w.N * w.H * w.D * 2
+
+    # ---- 480p clip (inputs smaller than L2: rotate over copies)
+    w = W["480p"]
+    base = gdn_inputs.workload_inputs(w, device=dev)
+    inb = 3 * tok_bytes(w)
+    nc = n_copies(inb)
+    sets = []
+    for _ in range(nc):
+        c = {k: (None if v is None else v.clone()) for k, v in base.items()}
+        sets.append((c, torch.empty_like(c["q"])))
+    st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    nxt = rotating(sets)
+
+    def step_480():
+        c, o = nxt()
+        api.gdn_frame_forward(c["q"], c["k"], c["v"], c["gamma"], c["beta"], None, o, st,
+                              key_scale=w.key_scale, stream=stream)
+    recs["480p"] = workload_record(
+        "480p", w, step_480, stream, algorithmic_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, False, s, l), w.tokens_heads,
+        l2_note=f"{nc} copies of the inputs ({inb / 1e6:.0f} MB of q,k,v each) rotated, so a "
+                f"step's inputs were evicted from the 126 MB L2 by the steps before it")
+    del base, sets
+
+    # ---- streaming workload: one step = 64 chained gdn_frame_step calls, state in place
+    w = W["stream"]
+    frames = []
+    for j in range(4):  # four distinct frames (216 MB of q,k,v each) cycled over the 64 calls
+        x = gdn_inputs.workload_inputs(w, device=dev, step=j)
+        frames.append({n: x[n][:, 0].contiguous() for n in ("q", "k", "v", "gamma", "beta")})
+    state = gdn_inputs.workload_inputs(w, device=dev)["state"].contiguous()
+    out_s = torch.empty_like(frames[0]["q"])
+
+    def step_stream():
+        for j in range(w.steps):
+            f = frames[j % len(frames)]
+            api.gdn_frame_step(f["q"], f["k"], f["v"], f["gamma"], f["beta"], state, out_s,
+                               state, key_scale=w.key_scale, stream=stream)
+    recs["stream"] = workload_record(
+        "stream", f"streaming decode: {w.steps} chained gdn_frame_step calls of B{w.B} H{w.H} "
+                  f"D{w.D} N{w.N} ({w.grid} grid), state in place",
+        step_stream, stream, w.steps * algorithmic_bytes(w),
+        lambda n, l, s, w=w: kernel_bytes(n, w), w.steps * w.tokens_heads,
+        launches_per_step=w.steps + 4, target_ms=300.0)
+    recs["stream"]["per_call_ms"] = recs["stream"]["ms_per_step"] / w.steps
+    del frames, state, out_s
+
+    # ---- block-causal LA clip
+    w = W["la"]
+    g = gdn_inputs.workload_inputs(w, device=dev)
+    out_la = torch.empty_like(g["q"])
+    st_la = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    z_la = torch.empty((w.B, w.H, w.D), dtype=torch.float32, device=dev)
+
+    def step_la():
+        api.gdn_block_causal_la(g["q"], g["k"], g["v"], w.frames_per_block, out=out_la,
+                                state_out=st_la, z_out=z_la, stream=stream)
+    recs["la"] = workload_record(
+        "la", w, step_la, stream, algorithmic_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, False, s, l), w.tokens_heads)
+    del g, out_la
+
+    # ---- 720p clip: fp8 inputs, backward, standalone 3D RoPE
+    w = W["720p"]
+    g = g720 if g720 is not None else gdn_inputs.workload_inputs(w, device=dev)
+    f8 = {}
+    for n in ("q", "k", "v"):
+        f8[n], f8["s" + n] = gdn_inputs.quantize_e4m3(g[n])
+    out8 = torch.empty_like(g["q"])
+    st8 = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+    def step_fp8():
+        api.gdn_frame_forward_fp8(f8["q"], f8["k"], f8["v"], f8["sq"], f8["sk"], f8["sv"],
+                                  g["gamma"], g["beta"], None, out8, st8, key_scale=w.key_scale,
+                                  stream=stream)
+    recs["720p_fp8"] = workload_record(
+        "720p_fp8", w.name + " clip, E4M3 q/k/v with per-(frame, head) scales", step_fp8,
+        stream, algorithmic_bytes(w, True),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, True, False, s, l), w.tokens_heads,
+        target_ms=150.0)
+    del f8, out8
+
+    d_out = gdn_inputs.cotangents(w.B, w.H, w.T, w.N, w.D, seed=w.seed + 50,
+                                  device=dev)["d_out"]
+
+    def step_bwd():
+        api.gdn_frame_backward(g["q"], g["k"], g["v"], g["gamma"], g["beta"], d_out,
+                               key_scale=w.key_scale, stream=stream)
+    recs["720p_backward"] = workload_record(
+        "720p_backward", w.name + " clip, gdn_frame_backward (dq, dk, dv, dgamma, dbeta, dS_0)",
+        step_bwd, stream, backward_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, True, s, l), w.tokens_heads,
+        target_ms=150.0)
+    del d_out
+    torch.cuda.empty_cache()
+
+    gh, gw = (int(x) for x in w.grid.split("x"))
+    qr, kr = torch.empty_like(g["q"]), torch.empty_like(g["k"])
+
+    def step_rope():
+        api.gdn_rope_3d(g["q"], gh, gw, out=qr, stream=stream)
+        api.gdn_rope_3d(g["k"], gh, gw, out=kr, stream=stream)
+    recs["720p_rope_standalone"] = workload_record(
+        "720p_rope_standalone", w.name + " clip, gdn_rope_3d of q and k (out of place)",
+        step_rope, stream, rope_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, False, s, l), w.tokens_heads,
+        target_ms=150.0)
+    del qr, kr
+    torch.cuda.empty_cache()
+
+    # ---- fused 3D RoPE prologue: the 720p forward with q and k rotated inside the kernels
+    out_r = torch.empty_like(g["q"])
+    st_r = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+    def step_rope_fused():
+        api.gdn_frame_forward_rope(g["q"], g["k"], g["v"], g["gamma"], g["beta"], gh, gw,
+                                   out=out_r, state_out=st_r, key_scale=w.key_scale,
+                                   stream=stream)
+    recs["720p_rope_fused"] = workload_record(
+        "720p_rope_fused", w.name + " clip, gdn_frame_forward_rope (3D RoPE of q and k fused "
+                                    "into the statistics and output kernels)",
+        step_rope_fused, stream, algorithmic_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, False, s, l), w.tokens_heads,
+        target_ms=150.0)
+    del out_r
+    if g720 is None:
+        del g
+    torch.cuda.empty_cache()
+
+    # ---- chunk-causal softmax attention of the hybrid blocks (tensor-bound)
+    for label, (B, H, T, N, D, F) in (("softmax_480p", (1, 32, 21, 390, 64, 3)),
+                                      ("softmax_720p21", (1, 20, 21, 880, 128, 3))):
+        x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=1500 + D, device=dev)
+        o = torch.empty_like(x["q"])
+
+        def step_sm(x=x, o=o, F=F):
+            api.gdn_softmax_attention(x["q"], x["k"], x["v"], F, out=o, stream=stream)
+        fl = softmax_flops(B, H, T, N, D, F)
+        inb = 4 * B * T * N * H * D * 2
+        recs[label] = workload_record(
+            label, f"chunk-causal softmax attention B{B} H{H} D{D} T{T} N{N}, chunks of {F} "
+                   f"frames (q, k, v, out {inb / 1e6:.0f} MB)",
+            step_sm, stream, inb, lambda n, l, s: None, B * H * T * N, target_ms=200.0,
+            flops_per_step=fl, tensor_peak=tensor_peak(),
+            l2_note="compute-bound: K and V are meant to be re-read from L2 by a head's query "
+                    "tiles; no flush")
+        del x, o
+    return recs
 
 
 def measure_e2e(a, w, g, out, st, stream, world, dev):

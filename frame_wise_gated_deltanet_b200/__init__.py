@@ -7,9 +7,11 @@ there is no CPU fallback.
 """
 _API = (
     "gdn_frame_forward",
+    "gdn_frame_forward_rope",
     "gdn_frame_step",
     "gdn_frame_backward",
     "gdn_rope_3d",
+    "gdn_softmax_attention",
     "gdn_frame_stats",
     "gdn_block_causal_la",
     "gdn_sync_status",

@@ -31,10 +31,12 @@ SIGNATURES = {
     "gdn_frame_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_forward_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_forward_fp8": (_I, [_P] * 11 + [_I, _I, _I, _I, _I, _F, _P]),
+    "gdn_frame_forward_rope": (_I, [_P] * 8 + [_I, _I, _I, _I, _I, _F, _I, _I, _F, _I, _P]),
     "gdn_frame_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_backward": (_I, [_P] * 14 + [_I, _I, _I, _I, _I, _F, _P]),
     "gdn_backward_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "gdn_rope_3d": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "gdn_softmax_attention": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_stats": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_block_causal_la": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "gdn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),

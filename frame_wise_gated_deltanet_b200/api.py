@@ -13,6 +13,7 @@ import torch
 from ._lib import LIB, GdnError, check
 
 __all__ = ["gdn_frame_forward", "gdn_frame_forward_fp8", "gdn_frame_forward_host",
+           "gdn_frame_forward_rope", "gdn_softmax_attention",
            "gdn_frame_step", "gdn_frame_backward", "gdn_backward_workspace_bytes", "gdn_rope_3d", "gdn_frame_stats", "gdn_block_causal_la",
            "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
            "gdn_la_workspace_bytes", "GdnError"]
@@ -69,6 +70,34 @@ def gdn_frame_forward(q, k, v, gamma, beta, state_in=None, out=None, state_out=N
         check("gdn_frame_forward", LIB.gdn_frame_forward(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
             _ptr(state_out), B, H, T, N, D, _scale(key_scale), _stream(stream, q.device)))
+    return out, state_out
+
+
+def gdn_frame_forward_rope(q, k, v, gamma, beta, grid_h: int, grid_w: int,
+                           rope_base: float = 10000.0, t_offset: int = 0, state_in=None,
+                           out=None, state_out=None, key_scale: Optional[float] = None,
+                           stream=None, want_state: bool = True):
+    """gdn_frame_forward on q and k rotated by the 3D RoPE (N = grid_h * grid_w tokens per
+    frame), the rotation fused into the layer's kernels. Returns (out, state_out)."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    _req(gamma, "gamma", torch.float32, (B, T, H))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _req(state_out, "state_out", torch.float32, (B, H, D, D))
+    with torch.cuda.device(q.device):
+        check("gdn_frame_forward_rope", LIB.gdn_frame_forward_rope(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
+            _ptr(state_out), B, H, T, N, D, _scale(key_scale), int(grid_h), int(grid_w),
+            float(rope_base), int(t_offset), _stream(stream, q.device)))
     return out, state_out
 
 
@@ -213,6 +242,24 @@ def gdn_rope_3d(x, grid_h: int, grid_w: int, base: float = 10000.0, t_offset: in
         check("gdn_rope_3d", LIB.gdn_rope_3d(
             _ptr(x), _ptr(out), B, T, N, H, D, int(grid_h), int(grid_w), float(base),
             int(t_offset), _stream(stream, x.device)))
+    return out
+
+
+def gdn_softmax_attention(q, k, v, frames_per_chunk: int, scale: Optional[float] = None,
+                          out=None, stream=None):
+    """Chunk-causal softmax attention over the clip's tokens (q, k, v, out: [B,T,N,H,D] bf16;
+    frames_per_chunk >= T is bidirectional). scale=None lets the library use 1/sqrt(D).
+    Returns out."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    with torch.cuda.device(q.device):
+        check("gdn_softmax_attention", LIB.gdn_softmax_attention(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, N, D, int(frames_per_chunk),
+            0.0 if scale is None else float(scale), _stream(stream, q.device)))
     return out
 
 

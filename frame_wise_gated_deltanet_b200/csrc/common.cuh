@@ -16,6 +16,17 @@ __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_status, 0,
 
 constexpr int kErrTimeout = 6;  // == GDN_ERR_TIMEOUT
 
+// 3D rotary position embedding applied to q and k inside the forward's statistics and output
+// kernels (see rope_kernel.cuh for the reading). tab holds (cos, sin) per (axis, position,
+// pair): frame t's time pairs at t * pt, grid row r's pairs at off_h + r * ph, grid column c's
+// at off_w + c * ph (the row and column slices have the same width).
+struct RopeArgs {
+  const float2* tab = nullptr;
+  int grid_w = 1;
+  int pt = 0, ph = 0;        // pairs of the time slice and of the row (= column) slice
+  int off_h = 0, off_w = 0;  // first table entries of the row and column axes
+};
+
 // One problem: q/k/v/out are [B, T, N, H, D] bf16, gamma/beta [B, T, H] f32.
 struct Problem {
   int B, H, T, N, D;
@@ -24,6 +35,8 @@ struct Problem {
   const float* q_scale = nullptr;
   const float* k_scale = nullptr;
   const float* v_scale = nullptr;
+  // 3D RoPE of q and k (forward with the rotary prologue only)
+  RopeArgs rope;
 };
 
 // Hand-off state of the fused forward, in device memory and zeroed before each call. One

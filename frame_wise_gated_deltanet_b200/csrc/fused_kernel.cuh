@@ -34,15 +34,18 @@ template <int DP>
 struct FusedLayout {
   static constexpr int kThreads = ChainLayout<DP>::kThreads;
   static_assert(kThreads >= StatsLayout<DP, false, DP == 128>::kThreads &&
-                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, DP == 128>::kThreads,
+                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, DP == 128>::kThreads &&
+                    kThreads >= StatsLayout<DP, false, false, true>::kThreads &&
+                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, false, true>::kThreads,
                 "the chain role's CTA size must cover the other roles' warps");
   static constexpr int kSmemBytes =
       cmax(ChainLayout<DP>::kSmemBytes,
            cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes));
 };
 
-// kF8: e4m3 q, k, v with per (b, t, h) scales in p (DP = 128 only).
-template <int DP, bool kF8 = false>
+// kF8: e4m3 q, k, v with per (b, t, h) scales in p (DP = 128 only). kRope: q and k rotated by
+// the 3D RoPE of p.rope in shared memory by the statistics and output roles.
+template <int DP, bool kF8 = false, bool kRope = false>
 __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
     gdn_fused_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -61,10 +64,11 @@ __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
     chain_body<DP, true>(&tm_a_ring, B_ring, S_ring, gamma, beta, state_in, state_out, p,
                          h_chain, whole, smem);
   } else if (static_cast<int>(blockIdx.x) < h_out.base) {
-    stats_body<DP, false, true, true, kF8>(&tm_k, &tm_v, A_ring, B_ring, p, h_stats, smem);
+    stats_body<DP, false, true, true, kF8, kRope>(&tm_k, &tm_v, A_ring, B_ring, p, h_stats,
+                                                  smem);
   } else {
-    output_body<DP, false, true, kFusedOutGroups, kF8>(&tm_q, &tm_q, S_ring, &tm_o, p, 1, h_out,
-                                                       smem);
+    output_body<DP, false, true, kFusedOutGroups, kF8, kRope>(&tm_q, &tm_q, S_ring, &tm_o, p, 1,
+                                                              h_out, smem);
   }
 }
 

@@ -21,6 +21,7 @@
 #include "output_kernel.cuh"
 #include "rope_kernel.cuh"
 #include "scan_kernel.cuh"
+#include "softmax_kernel.cuh"
 #include "stats_kernel.cuh"
 #include "step_kernel.cuh"
 
@@ -99,6 +100,16 @@ bool tmap_rows(CUtensorMap* m, const void* base, const Problem& p) {
   return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box);
 }
 
+// q/k/v/out [B, T, N, H, D] bf16 as (D, H, T*N, B): a clip's tokens as one row axis, so tiles
+// span frames and rows past the clip read as zero and are not stored (softmax attention).
+bool tmap_clip(CUtensorMap* m, const void* base, int B, int H, int L, int D) {
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2,
+                                 (cuuint64_t)L * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box);
+}
+
 // Token map of q, k or v in the element type of the path.
 template <bool kF8>
 bool tmap_in(CUtensorMap* m, const void* base, const Problem& p) {
@@ -127,6 +138,9 @@ struct DeviceState {
   // second stream of the backward (work that overlaps the state chains) and its fork/join events
   cudaStream_t aux = nullptr;
   cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  // (cos, sin) table of gdn_frame_forward_rope (kept apart from the forward's workspace)
+  float2* rope_tab = nullptr;
+  size_t rope_tab_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -155,28 +169,51 @@ gdn_status current_device(int* dev) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-gdn_status get_workspace(int dev, size_t bytes, cudaStream_t stream, void** out) {
-  DeviceState& d = g_dev[dev];
-  if (d.ws_bytes >= bytes) {
-    *out = d.ws;
-    return GDN_OK;
-  }
+// GDN_POISON_WORKSPACE=1 (testing aid, read once): every call fills the workspace bytes it will
+// use with 0xFF (NaN as f32 and bf16) on its stream before its kernels run, so a kernel that reads
+// workspace it did not write first produces NaN instead of a silently plausible value.
+bool poison_workspace() {
+  static const bool on = [] {
+    const char* s = getenv("GDN_POISON_WORKSPACE");
+    return s != nullptr && s[0] == '1';
+  }();
+  return on;
+}
+
+gdn_status poison(void* p, size_t bytes, cudaStream_t stream) {
+  if (!poison_workspace() || bytes == 0) return GDN_OK;
+  return cudaMemsetAsync(p, 0xFF, bytes, stream) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Grows a library-owned device buffer in stream order: the old buffer is released by
+// cudaFreeAsync on `stream` (after the work already enqueued there, which includes every earlier
+// call's use of it: calls on one GPU are ordered on the caller's stream) and the new one is
+// taken by cudaMallocAsync from the device's default memory pool, so growing does not
+// synchronise the device or other streams. Refused with GDN_ERR_NO_MEMORY while `stream` is being
+// captured (the buffer outlives any graph).
+gdn_status grow_buffer(void** buf, size_t* have, size_t bytes, cudaStream_t stream) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return GDN_ERR_CUDA;
   if (cs != cudaStreamCaptureStatusNone) return GDN_ERR_NO_MEMORY;
-  if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
-  if (d.ws) cudaFree(d.ws);
-  d.ws = nullptr;
-  d.ws_bytes = 0;
+  if (*buf != nullptr && cudaFreeAsync(*buf, stream) != cudaSuccess) return GDN_ERR_CUDA;
+  *buf = nullptr;
+  *have = 0;
   void* p = nullptr;
-  if (cudaMalloc(&p, bytes) != cudaSuccess) {
+  if (cudaMallocAsync(&p, bytes, stream) != cudaSuccess) {
     cudaGetLastError();
     return GDN_ERR_NO_MEMORY;
   }
-  d.ws = p;
-  d.ws_bytes = bytes;
-  *out = p;
+  *buf = p;
+  *have = bytes;
   return GDN_OK;
+}
+
+gdn_status get_workspace(int dev, size_t bytes, cudaStream_t stream, void** out) {
+  DeviceState& d = g_dev[dev];
+  if (d.ws_bytes < bytes)
+    if (gdn_status s = grow_buffer(&d.ws, &d.ws_bytes, bytes, stream)) return s;
+  *out = d.ws;
+  return poison(d.ws, bytes, stream);
 }
 
 template <typename K>
@@ -252,16 +289,16 @@ gdn_status check_launch() {
 // ------------------------------------------------------------------ kernel runners
 // kB4: B_t in the chain's interleaved layout (forward paths) or row-major (gdn_frame_stats).
 // max_ctas > 0 caps the grid (the backward runs it beside the state chain's CTAs).
-template <int DP, bool kB4, bool kF8 = false>
+template <int DP, bool kB4, bool kF8 = false, bool kRope = false>
 gdn_status run_stats(int dev, const Problem& p, const void* k, const void* v, void* A, float* Bm,
                      cudaStream_t st, int max_ctas = 0) {
-  using L = gdn::StatsLayout<DP, false, kF8>;
+  using L = gdn::StatsLayout<DP, false, kF8, kRope>;
   CUtensorMap tk, tv;
   if (!tmap_in<kF8>(&tk, k, p) || !tmap_in<kF8>(&tv, v, p)) return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_stats_kernel<DP, false, kB4, kF8>;
-  if (gdn_status s = ensure_smem_attr(
-          dev, kF8 ? 15 : (DP == 128 ? 0 : 1) + (kB4 ? 10 : 0), kern, L::kSmemBytes))
-    return s;
+  auto kern = gdn::gdn_stats_kernel<DP, false, kB4, kF8, kRope>;
+  const int bit = kRope ? 40 + (DP == 128 ? 0 : 1)
+                        : (kF8 ? 15 : (DP == 128 ? 0 : 1) + (kB4 ? 10 : 0));
+  if (gdn_status s = ensure_smem_attr(dev, bit, kern, L::kSmemBytes)) return s;
   const long items = long(p.B) * p.T * p.H;
   const long cap = max_ctas > 0 ? max_ctas : g_dev[dev].sms;
   const int grid = static_cast<int>(items < cap ? items : cap);
@@ -311,10 +348,10 @@ gdn_status run_scan(int dev, const Problem& p, const gdn::ChainSeg& seg, const f
   return check_launch();
 }
 
-template <int DP, bool kLA, bool kF8 = false>
+template <int DP, bool kLA, bool kF8 = false, bool kRope = false>
 gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws, int srows,
                       void* out, int F, cudaStream_t st) {
-  using L = gdn::OutputLayout<DP, kLA, 4, kF8>;
+  using L = gdn::OutputLayout<DP, kLA, 4, kF8, kRope>;
   const long count = long(p.B) * p.H * ((p.T + F - 1) / F);  // stored states (per block for LA)
   CUtensorMap tq, ts, to;
   if (kLA) {
@@ -327,10 +364,9 @@ gdn_status run_output(int dev, const Problem& p, const void* q, const void* S_ws
   } else {
     ts = tq;  // unused: GDN states are bulk-copied from S_ws
   }
-  auto kern = gdn::gdn_output_kernel<DP, kLA, kF8>;
-  if (gdn_status s = ensure_smem_attr(dev, kF8 ? 16 : (kLA ? 6 : (DP == 128 ? 4 : 5)), kern,
-                                      L::kSmemBytes))
-    return s;
+  auto kern = gdn::gdn_output_kernel<DP, kLA, kF8, kRope>;
+  const int bit = kRope ? 42 + (DP == 128 ? 0 : 1) : (kF8 ? 16 : (kLA ? 6 : (DP == 128 ? 4 : 5)));
+  if (gdn_status s = ensure_smem_attr(dev, bit, kern, L::kSmemBytes)) return s;
   const long items = long(p.B) * (kLA ? (p.T + F - 1) / F : p.T) * p.H;
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
   {
@@ -448,7 +484,7 @@ bool fused_applies(int dev, const Problem& p) {
   return bh * 3 <= sms && p.T >= 4;
 }
 
-template <int DP, bool kF8 = false>
+template <int DP, bool kF8 = false, bool kRope = false>
 gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, const void* v,
                      const float* gamma, const float* beta, const float* s_in, void* out,
                      float* s_out, cudaStream_t st) {
@@ -464,9 +500,9 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   if (!tmap_in<kF8>(&tk, k, p) || !tmap_in<kF8>(&tv, v, p) || !tmap_in<kF8>(&tq, q, p) ||
       !tmap_tokens(&to, out, p) || !tmap_mats(&ta, w.A, false, p.D, p.D, long(bh) * kRing, DP))
     return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_fused_kernel<DP, kF8>;
-  if (gdn_status s = ensure_smem_attr(dev, kF8 ? 17 : (DP == 128 ? 8 : 9), kern, L::kSmemBytes))
-    return s;
+  auto kern = gdn::gdn_fused_kernel<DP, kF8, kRope>;
+  const int bit = kRope ? 44 + (DP == 128 ? 0 : 1) : (kF8 ? 17 : (DP == 128 ? 8 : 9));
+  if (gdn_status s = ensure_smem_attr(dev, bit, kern, L::kSmemBytes)) return s;
   // split the SMs left after the chains between the stats and output roles (by default
   // ~54 : 46, the ratio of their per-frame times)
   const int workers = sms - bh;
@@ -602,7 +638,7 @@ bool chunked_pays(int dev, const Problem& p, bool fused) {
   return chunked < 0.9 * other;
 }
 
-template <int DP, bool kF8 = false>
+template <int DP, bool kF8 = false, bool kRope = false>
 gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, const void* v,
                        const float* gamma, const float* beta, const float* s_in, void* out,
                        float* s_out, cudaStream_t st) {
@@ -617,7 +653,7 @@ gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, 
   uint8_t* starts = maps + align256(size_t(bh) * (plan.nc - 1) * gdn::chunk_map_bytes(DP));
   const gdn::ChainSeg compose{plan.L, plan.nc, 1, maps, starts};
   const gdn::ChainSeg replay{plan.L, plan.nc, 0, maps, starts};
-  if (gdn_status s = run_stats<DP, true, kF8>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_stats<DP, true, kF8, kRope>(dev, p, k, v, w.A, w.B, st)) return s;
   if (plan.nc > 1) {
     if (gdn_status s = run_chain<DP>(dev, p, w.A, w.B, gamma, beta, nullptr, nullptr, nullptr,
                                      compose, st))
@@ -626,11 +662,12 @@ gdn_status run_chunked(int dev, const Problem& p, const void* q, const void* k, 
   }
   if (gdn_status s = run_chain<DP>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, replay, st))
     return s;
-  return run_output<DP, false, kF8>(dev, p, q, w.S, p.D, out, 1, st);
+  return run_output<DP, false, kF8, kRope>(dev, p, q, w.S, p.D, out, 1, st);
 }
 
-// kF8: e4m3 q, k, v (scales in p; 64 < D <= 128, checked by the caller).
-template <bool kF8>
+// kF8: e4m3 q, k, v (scales in p; 64 < D <= 128, checked by the caller). kRope: q and k rotated
+// by the 3D RoPE of p.rope inside the statistics and output kernels.
+template <bool kF8, bool kRope = false>
 gdn_status forward_path(int dev, const void* q, const void* k, const void* v, const float* gamma,
                         const float* beta, const float* s_in, void* out, float* s_out,
                         const Problem& p, cudaStream_t st) {
@@ -638,13 +675,13 @@ gdn_status forward_path(int dev, const void* q, const void* k, const void* v, co
   const bool fused = fused_applies(dev, p);
   if (g_forward_mode == 3 || (g_forward_mode == 0 && chunked_pays(dev, p, fused))) {
     if (!kF8 && p.D <= 64)
-      return run_chunked<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
-    return run_chunked<kDP, kF8>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+      return run_chunked<64, false, kRope>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+    return run_chunked<kDP, kF8, kRope>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
   }
   if (fused) {
     if (!kF8 && p.D <= 64)
-      return run_fused<64>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
-    return run_fused<kDP, kF8>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+      return run_fused<64, false, kRope>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
+    return run_fused<kDP, kF8, kRope>(dev, p, q, k, v, gamma, beta, s_in, out, s_out, st);
   }
   const long count = long(p.B) * p.H * p.T;
   void* base = nullptr;
@@ -652,15 +689,15 @@ gdn_status forward_path(int dev, const void* q, const void* k, const void* v, co
   ForwardWs w = carve_forward(base, count, p.D);
   const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
   if (!kF8 && p.D <= 64) {
-    if (gdn_status s = run_stats<64, true>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = run_stats<64, true, false, kRope>(dev, p, k, v, w.A, w.B, st)) return s;
     if (gdn_status s = run_chain<64>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
       return s;
-    return run_output<64, false>(dev, p, q, w.S, p.D, out, 1, st);
+    return run_output<64, false, false, kRope>(dev, p, q, w.S, p.D, out, 1, st);
   }
-  if (gdn_status s = run_stats<kDP, true, kF8>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_stats<kDP, true, kF8, kRope>(dev, p, k, v, w.A, w.B, st)) return s;
   if (gdn_status s = run_chain<kDP>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, s_out, whole, st))
     return s;
-  return run_output<kDP, false, kF8>(dev, p, q, w.S, p.D, out, 1, st);
+  return run_output<kDP, false, kF8, kRope>(dev, p, q, w.S, p.D, out, 1, st);
 }
 
 gdn_status forward_impl(const void* q, const void* k, const void* v, const float* gamma,
@@ -671,6 +708,8 @@ gdn_status forward_impl(const void* q, const void* k, const void* v, const float
   std::lock_guard<std::mutex> lock(g_mu);
   if (p.k_scale != nullptr)
     return forward_path<true>(dev, q, k, v, gamma, beta, s_in, out, s_out, p, st);
+  if (p.rope.tab != nullptr)
+    return forward_path<false, true>(dev, q, k, v, gamma, beta, s_in, out, s_out, p, st);
   return forward_path<false>(dev, q, k, v, gamma, beta, s_in, out, s_out, p, st);
 }
 
@@ -701,19 +740,16 @@ gdn_status run_step(int dev, const Problem& p, const void* q, const void* k, con
   DeviceState& d = g_dev[dev];
   // persistent flag words: ready [items] (epochs), next_unit, done, abort; zeroed when allocated
   if (d.step_items < items || d.step_epoch >= 0x7fffff00) {
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GDN_ERR_CUDA;
-    if (cs != cudaStreamCaptureStatusNone) return GDN_ERR_NO_MEMORY;
-    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
-    if (d.step_flags) cudaFree(d.step_flags);
-    d.step_flags = nullptr;
-    d.step_items = 0;
     const size_t bytes = sizeof(int) * (items + 3);
-    if (cudaMalloc(&d.step_flags, bytes) != cudaSuccess) {
-      cudaGetLastError();
-      return GDN_ERR_NO_MEMORY;
+    void* buf = d.step_flags;
+    size_t have = 0;
+    d.step_items = 0;
+    if (gdn_status s = grow_buffer(&buf, &have, bytes, st)) {
+      d.step_flags = static_cast<int*>(buf);
+      return s;
     }
-    if (cudaMemset(d.step_flags, 0, bytes) != cudaSuccess) return GDN_ERR_CUDA;
+    d.step_flags = static_cast<int*>(buf);
+    if (cudaMemsetAsync(d.step_flags, 0, bytes, st) != cudaSuccess) return GDN_ERR_CUDA;
     d.step_items = items;
     d.step_epoch = 0;
   }
@@ -1010,20 +1046,9 @@ gdn_status forward_host_impl(const uint16_t* q, const uint16_t* k, const uint16_
   const size_t per_buf = 4 * seg_tok + 2 * seg_gb;
   const size_t state_bytes = align256(size_t(p.B) * p.H * p.D * p.D * 4);
   const size_t need = 2 * per_buf + state_bytes;
-  if (hp.bytes < need) {
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GDN_ERR_CUDA;
-    if (cs != cudaStreamCaptureStatusNone) return GDN_ERR_NO_MEMORY;
-    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
-    if (hp.buf) cudaFree(hp.buf);
-    hp.buf = nullptr;
-    hp.bytes = 0;
-    if (cudaMalloc(&hp.buf, need) != cudaSuccess) {
-      cudaGetLastError();
-      return GDN_ERR_NO_MEMORY;
-    }
-    hp.bytes = need;
-  }
+  // (a previous call's copies on the internal streams are ordered before `st`'s later work)
+  if (hp.bytes < need)
+    if (gdn_status s = grow_buffer(&hp.buf, &hp.bytes, need, st)) return s;
   uint8_t* base = static_cast<uint8_t*>(hp.buf);
   SegBufs sb[2];
   for (int i = 0; i < 2; ++i) {
@@ -1097,9 +1122,146 @@ gdn_status forward_host_impl(const uint16_t* q, const uint16_t* k, const uint16_
   return GDN_OK;
 }
 
+// Host checks of the 3D RoPE arguments shared by gdn_rope_3d and gdn_frame_forward_rope, and
+// the table's dimensions (time, row and column slices of the head dimension).
+gdn_status rope_dims(int B, int T, int N, int H, int D, int grid_h, int grid_w, float base,
+                     int t_offset, gdn::RopeDims* r, long* n_tab) {
+  if (B < 1 || T < 1 || N < 1 || H < 1 || D < 1 || grid_h < 1 || grid_w < 1 || t_offset < 0)
+    return GDN_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 1024) return GDN_ERR_UNSUPPORTED;
+  if (double(grid_h) * grid_w != double(N)) return GDN_ERR_INVALID_ARG;
+  if (!(std::isfinite(base) && base > 1.f)) return GDN_ERR_INVALID_ARG;
+  if (double(T) + t_offset > 2147483647.0) return GDN_ERR_INVALID_ARG;
+  if (double(N) * H * (D / 8) > 2147483647.0 || double(B) * T > 2147483647.0)
+    return GDN_ERR_INVALID_ARG;
+  r->B = B;
+  r->T = T;
+  r->N = N;
+  r->H = H;
+  r->D = D;
+  r->grid_w = grid_w;
+  r->d_h = 2 * (D / 6);
+  r->d_w = r->d_h;
+  r->d_t = D - 2 * r->d_h;
+  if (double(T) * (r->d_t / 2) + double(grid_h) * (r->d_h / 2) + double(grid_w) * (r->d_w / 2) >
+      2147483647.0)
+    return GDN_ERR_INVALID_ARG;
+  r->off_h = T * (r->d_t / 2);
+  r->off_w = r->off_h + grid_h * (r->d_h / 2);
+  *n_tab = long(r->off_w) + long(grid_w) * (r->d_w / 2);
+  return GDN_OK;
+}
+
+gdn_status launch_rope_table(float2* tab, const gdn::RopeDims& r, long n_tab, int t_offset,
+                             float base, cudaStream_t st) {
+  ProfiledLaunch pl("gdn_rope_table_kernel", st);
+  gdn::gdn_rope_table_kernel<<<static_cast<unsigned>((n_tab + 255) / 256), 256, 0, st>>>(
+      tab, r, t_offset, std::log2(double(base)));
+  return check_launch();
+}
+
+// The per-GPU buffer of gdn_frame_forward_rope's table, grown like the workspace.
+gdn_status get_rope_table(int dev, size_t bytes, cudaStream_t stream, float2** out) {
+  DeviceState& d = g_dev[dev];
+  if (d.rope_tab_bytes < bytes) {
+    void* buf = d.rope_tab;
+    gdn_status s = grow_buffer(&buf, &d.rope_tab_bytes, bytes, stream);
+    d.rope_tab = static_cast<float2*>(buf);
+    if (s) return s;
+  }
+  *out = d.rope_tab;
+  return GDN_OK;
+}
+
+// Chunk-causal softmax attention: one persistent CTA per SM over (b, h, query tile) items.
+template <int DP>
+gdn_status run_softmax(int dev, const void* q, const void* k, const void* v, void* out, int B,
+                       int H, int T, int N, int D, int F, float scale, cudaStream_t st) {
+  using L = gdn::SoftmaxLayout<DP>;
+  const int Ltok = T * N;
+  CUtensorMap tq, tk, tv, to;
+  if (!tmap_clip(&tq, q, B, H, Ltok, D) || !tmap_clip(&tk, k, B, H, Ltok, D) ||
+      !tmap_clip(&tv, v, B, H, Ltok, D) || !tmap_clip(&to, out, B, H, Ltok, D))
+    return GDN_ERR_CUDA;
+  auto kern = gdn::gdn_softmax_kernel<DP>;
+  if (gdn_status s = ensure_smem_attr(dev, DP == 128 ? 46 : 47, kern, L::kSmemBytes)) return s;
+  const long items = long(B) * H * ((Ltok + gdn::kRowsPerTile - 1) / gdn::kRowsPerTile);
+  const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
+  // scores enter the base-2 exponential as S * scale * log2(e)
+  const float c = static_cast<float>(double(scale) * 1.4426950408889634);
+  {
+    ProfiledLaunch pl("gdn_softmax_kernel", st);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, tk, tv, to, B, H, T, N, F, c);
+  }
+  return check_launch();
+}
+
 }  // namespace
 
 extern "C" {
+
+gdn_status gdn_softmax_attention(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                 gdn_bf16* out, int B, int H, int T, int N, int D,
+                                 int frames_per_chunk, float scale, gdn_stream_t stream) {
+  if (!q || !k || !v || !out) return GDN_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || T < 1 || N < 1 || D < 1 || frames_per_chunk < 1)
+    return GDN_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 128) return GDN_ERR_UNSUPPORTED;
+  if (double(T) * N >= 2147483647.0 || double(B) * H * T * N * D > 4.0e18)
+    return GDN_ERR_INVALID_ARG;
+  if (scale == 0.f) {
+    scale = static_cast<float>(1.0 / std::sqrt(double(D)));
+  } else if (!(std::isfinite(scale) && scale > 0.f)) {
+    return GDN_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return GDN_ERR_MISALIGNED;
+  const size_t n = size_t(B) * T * N * H * D * 2;
+  if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
+    return GDN_ERR_INVALID_ARG;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int F = frames_per_chunk < T ? frames_per_chunk : T;
+  if (D <= 64) return run_softmax<64>(dev, q, k, v, out, B, H, T, N, D, F, scale, st);
+  return run_softmax<128>(dev, q, k, v, out, B, H, T, N, D, F, scale, st);
+}
+
+
+gdn_status gdn_frame_forward_rope(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                  const float* gamma, const float* beta, const float* state_in,
+                                  gdn_bf16* out, float* state_out, int B, int H, int T, int N,
+                                  int D, float key_scale, int grid_h, int grid_w,
+                                  float rope_base, int t_offset, gdn_stream_t stream) {
+  if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, T, N,
+                                     D, key_scale))
+    return s;
+  resolve_key_scale(key_scale, D, N, &key_scale);  // validated above
+  gdn::RopeDims r;
+  long n_tab = 0;
+  if (gdn_status s = rope_dims(B, T, N, H, D, grid_h, grid_w, rope_base, t_offset, &r, &n_tab))
+    return s;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float2* tab = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (gdn_status s = get_rope_table(dev, align256(size_t(n_tab) * sizeof(float2)), st, &tab))
+      return s;
+    if (gdn_status s = launch_rope_table(tab, r, n_tab, t_offset, rope_base, st)) return s;
+  }
+  Problem p{B, H, T, N, D, key_scale};
+  p.rope.tab = tab;
+  p.rope.grid_w = grid_w;
+  p.rope.pt = r.d_t / 2;
+  p.rope.ph = r.d_h / 2;
+  p.rope.off_h = r.off_h;
+  p.rope.off_w = r.off_w;
+  return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p, st);
+}
+
 
 gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
                              const float* gamma, const float* beta, const float* state_in,
@@ -1133,6 +1295,8 @@ gdn_status gdn_frame_forward_noalloc(const gdn_bf16* q, const gdn_bf16* k, const
   if (gdn_status s = noalloc_scratch(dev, &base)) return s;
   // Every scratch element (A_t, B_t, S_t) is written by this call before it is read, so nothing
   // needs clearing between calls.
+  if (gdn_status s = poison(base, forward_ws_bytes(count, D), reinterpret_cast<cudaStream_t>(stream)))
+    return s;
   const ForwardWs w = carve_forward(base, count, D);
   const Problem p{B, H, T, N, D, key_scale};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1323,31 +1487,13 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
 gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int H, int D,
                        int grid_h, int grid_w, float base, int t_offset, gdn_stream_t stream) {
   if (!x || !y) return GDN_ERR_INVALID_ARG;
-  if (B < 1 || T < 1 || N < 1 || H < 1 || D < 1 || grid_h < 1 || grid_w < 1 || t_offset < 0)
-    return GDN_ERR_INVALID_ARG;
-  if (D % 8 != 0 || D > 1024) return GDN_ERR_UNSUPPORTED;
-  if (double(grid_h) * grid_w != double(N)) return GDN_ERR_INVALID_ARG;
-  if (!(std::isfinite(base) && base > 1.f)) return GDN_ERR_INVALID_ARG;
-  if (double(T) + t_offset > 2147483647.0) return GDN_ERR_INVALID_ARG;
+  gdn::RopeDims r;
+  long n_tab = 0;
+  if (gdn_status s = rope_dims(B, T, N, H, D, grid_h, grid_w, base, t_offset, &r, &n_tab))
+    return s;
   if (!aligned16(x) || !aligned16(y)) return GDN_ERR_MISALIGNED;
   const size_t n = size_t(B) * T * N * H * D * 2;
   if (x != y && overlaps(x, n, y, n)) return GDN_ERR_INVALID_ARG;
-  gdn::RopeDims r;
-  r.B = B;
-  r.T = T;
-  r.N = N;
-  r.H = H;
-  r.D = D;
-  r.grid_w = grid_w;
-  r.d_h = 2 * (D / 6);
-  r.d_w = r.d_h;
-  r.d_t = D - 2 * r.d_h;
-  r.off_h = T * (r.d_t / 2);
-  r.off_w = r.off_h + grid_h * (r.d_h / 2);
-  const long n_tab = long(r.off_w) + long(grid_w) * (r.d_w / 2);
-  if (double(T) * (r.d_t / 2) + double(grid_h) * (r.d_h / 2) + double(grid_w) * (r.d_w / 2) >
-      2147483647.0)
-    return GDN_ERR_INVALID_ARG;
   int dev;
   if (gdn_status s = current_device(&dev)) return s;
   std::lock_guard<std::mutex> lock(g_mu);
@@ -1356,20 +1502,16 @@ gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int 
   if (gdn_status s = get_workspace(dev, align256(size_t(n_tab) * sizeof(float2)), st, &base_ws))
     return s;
   float2* tab = static_cast<float2*>(base_ws);
-  {
-    ProfiledLaunch pl("gdn_rope_table_kernel", st);
-    gdn::gdn_rope_table_kernel<<<static_cast<unsigned>((n_tab + 255) / 256), 256, 0, st>>>(
-        tab, r, t_offset, std::log2(double(base)));
-    if (gdn_status s = check_launch()) return s;
-  }
-  const long n_vec = long(B) * T * N * H * (D / 8);
-  const long want = (n_vec + 255) / 256;
-  const long cap = 16L * g_dev[dev].sms;  // grid-stride: 16 blocks of 256 threads per SM
+  if (gdn_status s = launch_rope_table(tab, r, n_tab, t_offset, base, st)) return s;
+  // one block row per frame of one batch element, kRopeVecs vectors per thread
+  const int frame_vecs = N * H * (D / 8);
+  const long per_block = 256L * gdn::kRopeVecs;
+  const long chunks = std::min(65535L, (long(frame_vecs) + per_block - 1) / per_block);
   {
     ProfiledLaunch pl("gdn_rope_kernel", st);
-    gdn::gdn_rope_kernel<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<__nv_bfloat16*>(y), tab, r,
-        n_vec);
+    gdn::gdn_rope_kernel<<<dim3(static_cast<unsigned>(B * T), static_cast<unsigned>(chunks)), 256,
+                           0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x),
+                                    reinterpret_cast<__nv_bfloat16*>(y), tab, r, frame_vecs);
   }
   return check_launch();
 }
@@ -1439,6 +1581,9 @@ void gdn_release_workspace(void) {
   // reset the old kernel attributes and the scratch address no longer hold)
   d.attr_done = 0;
   g_noalloc_addr[dev] = nullptr;
+  if (d.rope_tab) cudaFree(d.rope_tab);
+  d.rope_tab = nullptr;
+  d.rope_tab_bytes = 0;
   {
     std::lock_guard<std::mutex> pl(g_pipe_mu);
     HostPipe& hp = g_pipe[dev];

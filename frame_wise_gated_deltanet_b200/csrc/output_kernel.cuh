@@ -16,6 +16,8 @@
 // fp8 mode (e4m3 Q, DP = 128): the Q tile is TMA-loaded into the second box of its bf16 stage,
 // the 4 transform warps convert it in place (exactly), and the epilogue multiplies by the
 // frame's Q scale.
+// RoPE mode (the fused 3D rotary prologue): 4 * DP/64 transform warps rotate each Q tile in
+// place (one 64-dim box of one token row per thread) before the MMA.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2 .. 2+4G-1
 // epilogue (G column groups of 4 warps; warp w reads TMEM lanes 32*(w%4) and DP/G columns), then
@@ -33,13 +35,17 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "rope_kernel.cuh"
 
 namespace gdn {
 
-template <int DP, bool kLA, int kG = 4, bool kF8 = false>
+template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false>
 struct OutputLayout {
   static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
-  static constexpr bool kTransform = kLA || kF8;
+  static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
+  static constexpr bool kTransform = kLA || kF8 || kRope;
+  // transform warps: 4 (one token row each), or for RoPE one 64-dim box of a row per thread
+  static constexpr int kXfWarps = kRope ? 4 * (DP / 64) : 4;
   static constexpr int kEpiWarps = 4 * kG;
   static constexpr int kCols = DP / kG;                // columns per epilogue thread
   static constexpr int kChunk = kCols < 32 ? kCols : 32;
@@ -47,7 +53,7 @@ struct OutputLayout {
   static constexpr int kQBytes = kBoxes * kBoxBytes;   // 128 tokens x DP bf16
   static constexpr int kSBufBytes = DP * DP * 2;       // DP/64 blocks of DP rows x 128 B
   static constexpr int kStages = (DP == 128) ? 3 : 8;
-  static constexpr int kThreads = (2 + kEpiWarps + (kTransform ? 4 : 0)) * 32;
+  static constexpr int kThreads = (2 + kEpiWarps + (kTransform ? kXfWarps : 0)) * 32;
   static constexpr int kQLoadBytes = kF8 ? kQBytes / 2 : kQBytes;  // TMA bytes per Q tile
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
   static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
@@ -107,13 +113,13 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p, i
 // LA: tm_q and tm_o are 3-D maps over the flattened token rows, and out (the raw output) takes
 // the row stores of a block's last, partial tile (a 128-row TMA store would also overwrite the
 // first rows of the next block, which another CTA writes).
-template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false>
+template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false, bool kRope = false>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
                                             const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
                                             uint8_t* smem, __nv_bfloat16* out = nullptr) {
-  using L = OutputLayout<DP, kLA, kG, kF8>;
+  using L = OutputLayout<DP, kLA, kG, kF8, kRope>;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                          // 2 state buffers
   uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
@@ -153,7 +159,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 128);
+      mbar_init(&ready[s], 32 * L::kXfWarps);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -400,9 +406,37 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     }
     if (leader) bulk_wait_all();
     if (!ok) give_up(hf, abort_flag);
-  } else if (L::kTransform && warp < 2 + L::kEpiWarps + 4) {
+  } else if (L::kTransform && warp < 2 + L::kEpiWarps + L::kXfWarps) {
     // (the fused kernel's output CTAs have more warps: the rest stay idle)
-    if constexpr (kF8) {
+    if constexpr (kRope) {
+      // ---------------------------------------------------------------- RoPE of the Q tiles
+      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // Q row tid % 128, box tid / 128
+      const int row = tid & 127, box = tid >> 7;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int li = 0; ok; ++li) {
+        const long item = consumer_item(li);
+        if (item < 0) break;
+        const OutputItem it = output_item<kFused, kLA>(item, p, F);
+        for (int tile = 0; tile < it.n_tiles; ++tile) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          const int n = tile * kRowsPerTile + row;
+          if (n < p.N)
+            rope_rotate_row(q_ring + stage * L::kQBytes, row, box, n, it.t, p.D, p.rope);
+          fence_async_smem();
+          mbar_arrive(&ready[stage]);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) give_up(hf, abort_flag);
+    } else if constexpr (kF8) {
       // ---------------------------------------------------------------- e4m3 Q conversion
       const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // the token row it converts
       int stage = 0;
@@ -477,8 +511,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   }
 }
 
-template <int DP, bool kLA, bool kF8 = false>
-__global__ void __launch_bounds__(OutputLayout<DP, kLA, 4, kF8>::kThreads, 1)
+template <int DP, bool kLA, bool kF8 = false, bool kRope = false>
+__global__ void __launch_bounds__(OutputLayout<DP, kLA, 4, kF8, kRope>::kThreads, 1)
     gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_s,
                       const __nv_bfloat16* __restrict__ S_src,
@@ -486,8 +520,8 @@ __global__ void __launch_bounds__(OutputLayout<DP, kLA, 4, kF8>::kThreads, 1)
                       __nv_bfloat16* out) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  output_body<DP, kLA, false, 4, kF8>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block, none,
-                                      align1k(smem_raw), out);
+  output_body<DP, kLA, false, 4, kF8, kRope>(&tm_q, &tm_s, S_src, &tm_o, p, frames_per_block,
+                                             none, align1k(smem_raw), out);
 }
 
 }  // namespace gdn

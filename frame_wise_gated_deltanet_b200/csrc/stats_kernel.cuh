@@ -12,10 +12,12 @@
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one elected thread)
 //   warps 2..5  epilogue: TMEM -> registers -> scale -> global (LA: per-block sums)
-//   warps 6..   (LA and fp8 only) in-place transform of each K/V stage: relu(K) and a ones
-//               column in V (LA, warps 6..9), or e4m3 -> bf16 conversion of K and V (fp8
+//   warps 6..   (LA, fp8 and RoPE only) in-place transform of each K/V stage: relu(K) and a
+//               ones column in V (LA, warps 6..9), or e4m3 -> bf16 conversion of K and V (fp8
 //               inputs, DP = 128, warps 6..13, one token row of K or V per thread: the fp8
-//               tiles are TMA-loaded into the second box of each bf16 operand tile)
+//               tiles are TMA-loaded into the second box of each bf16 operand tile), or the 3D
+//               rotary embedding of the K tile (RoPE, warps 6..6+4*DP/64-1, one 64-dim box of
+//               one token row per thread; V is not rotated)
 //
 // Standalone (gdn_stats_kernel): work item i = (b*T + t)*H + h, results at workspace row
 // (b*H + h)*T + t; for LA an item is a block of frames_per_item frames (its statistics summed
@@ -27,20 +29,23 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "rope_kernel.cuh"
 
 namespace gdn {
 
-template <int DP, bool kLA, bool kF8 = false>
+template <int DP, bool kLA, bool kF8 = false, bool kRope = false>
 struct StatsLayout {
   static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
-  static constexpr bool kTransform = kLA || kF8;
+  static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
+  static constexpr bool kTransform = kLA || kF8 || kRope;
   static constexpr int kBoxes = DP / 64;                // 64-dim boxes per operand tile
   static constexpr int kOpBytes = kBoxes * kBoxBytes;   // 128 tokens x DP dims, bf16
   static constexpr int kStageBytes = 2 * kOpBytes;      // K tile + V tile
   static constexpr int kStages = (DP == 128) ? 3 : 6;
   static constexpr int kAccCols = kLA ? 128 : (DP == 128 ? 256 : 64);
   static constexpr int kTmemCols = 2 * kAccCols;
-  static constexpr int kTransformThreads = kF8 ? 256 : 128;
+  // fp8: one K or V row per thread; RoPE: one 64-dim box of one K row per thread
+  static constexpr int kTransformThreads = kF8 ? 256 : (kRope ? 128 * kBoxes : 128);
   static constexpr int kThreads = 192 + (kTransform ? kTransformThreads : 0);
   static constexpr int kLoadBytes = kF8 ? kStageBytes / 2 : kStageBytes;  // TMA bytes per stage
   static constexpr int kBarrierBytes = 512;
@@ -86,12 +91,12 @@ __device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, con
 
 // kB4: B_t stored in the four-key interleaved layout of b4_index (the chain's input) instead of
 // row-major (the public gdn_frame_stats layout and the block-causal path).
-template <int DP, bool kLA, bool kFused, bool kB4, bool kF8 = false>
+template <int DP, bool kLA, bool kFused, bool kB4, bool kF8 = false, bool kRope = false>
 __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                            __nv_bfloat16* __restrict__ A_ws,
                                            float* __restrict__ B_ws, const Problem& p,
                                            const Handoff& hf, uint8_t* smem, int fpb = 1) {
-  using L = StatsLayout<DP, kLA, kF8>;
+  using L = StatsLayout<DP, kLA, kF8, kRope>;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
   uint64_t* ready = full + L::kStages;   // LA / fp8: transformed stage
   uint64_t* empty = ready + L::kStages;
@@ -395,7 +400,37 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     }
   } else if (L::kTransform && warp < 6 + L::kTransformThreads / 32) {
     // (the fused kernel's stats CTAs have more warps: the rest stay idle)
-    if constexpr (kF8) {
+    if constexpr (kRope) {
+      // ---------------------------------------------------------------- RoPE of the K tiles
+      const int tid = threadIdx.x - 192;  // K row tid % 128, 64-dim box tid / 128
+      const int row = tid & 127, box = tid >> 7;
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int li = 0;; ++li) {
+        const long item = consumer_item(li);
+        if (item < 0) break;
+        const int t = stats_item<kFused>(item, p, hf, fpb).t;
+        bool ok = true;
+        for (int tile = 0; tile < n_tiles; ++tile) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          const int n = tile * kRowsPerTile + row;
+          if (n < p.N) rope_rotate_row(smem + stage * L::kStageBytes, row, box, n, t, p.D, p.rope);
+          fence_async_smem();
+          mbar_arrive(&ready[stage]);
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) {
+          give_up(hf, abort_flag);
+          break;
+        }
+      }
+    } else if constexpr (kF8) {
       // ---------------------------------------------------------------- fp8 conversion warps
       const int tid = threadIdx.x - 192;  // 0..255: K row tid, or V row tid - 128
       int stage = 0;
@@ -485,15 +520,15 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
 
 // A_ws: [B*H*T, D, D] bf16 (GDN only). B_ws: [B*H*T, brows, D] f32, brows = D (GDN) or D+1 (LA),
 // row-major, or (kB4, GDN) each D x D matrix in the b4_index layout.
-template <int DP, bool kLA, bool kB4, bool kF8 = false>
-__global__ void __launch_bounds__(StatsLayout<DP, kLA, kF8>::kThreads, 1)
+template <int DP, bool kLA, bool kB4, bool kF8 = false, bool kRope = false>
+__global__ void __launch_bounds__(StatsLayout<DP, kLA, kF8, kRope>::kThreads, 1)
     gdn_stats_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ A_ws,
                      float* __restrict__ B_ws, Problem p, int frames_per_item) {
   extern __shared__ uint8_t smem_raw[];
   const Handoff none{nullptr, nullptr, nullptr, nullptr, nullptr, 1, 1, -1, 0, 0};
-  stats_body<DP, kLA, false, kB4, kF8>(&tm_k, &tm_v, A_ws, B_ws, p, none, align1k(smem_raw),
-                                       frames_per_item);
+  stats_body<DP, kLA, false, kB4, kF8, kRope>(&tm_k, &tm_v, A_ws, B_ws, p, none,
+                                              align1k(smem_raw), frames_per_item);
 }
 
 }  // namespace gdn

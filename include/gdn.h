@@ -36,9 +36,14 @@
  *    GDN_ERR_CUDA. Kernels never trap: a device-side wait that exceeds its time limit records
  *    GDN_ERR_TIMEOUT in a per-device status word that gdn_sync_status() reports.
  *  - The library keeps one cached device workspace per GPU (see gdn_workspace_bytes); it grows
- *    on demand (a device-wide synchronisation, refused with GDN_ERR_NO_MEMORY while the stream
- *    is being captured) and is shared by all calls on that GPU: calls on different streams of
- *    the same GPU must not run concurrently. gdn_release_workspace() frees it.
+ *    on demand in stream order (cudaFreeAsync of the old buffer and cudaMallocAsync of the new
+ *    one on the caller's stream, from the device's default memory pool: no device-wide
+ *    synchronisation; refused with GDN_ERR_NO_MEMORY while the stream is being captured) and is
+ *    shared by all calls on that GPU: calls on different streams of the same GPU must not run
+ *    concurrently (order them, e.g. by events). gdn_release_workspace() frees it.
+ *  - GDN_POISON_WORKSPACE=1 (testing aid, read once per process): every call first fills the
+ *    workspace bytes it uses with 0xFF (NaN as f32 and bf16) on its stream, so that a kernel
+ *    reading workspace it has not written shows up as NaN in the results.
  *  - No CPU fallback exists: without a CUDA device every call returns GDN_ERR_CUDA.
  *
  * Environment (read once per process unless stated):
@@ -94,6 +99,27 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
                              const float* gamma, const float* beta, const float* state_in,
                              gdn_bf16* out, float* state_out, int B, int H, int T, int N, int D,
                              float key_scale, gdn_stream_t stream);
+
+/*
+ * gdn_frame_forward_rope - gdn_frame_forward on q and k rotated by the 3D rotary position
+ * embedding of gdn_rope_3d (see there for the reading of the SANA-Video talk transcript's 3D
+ * RoPE), with the rotation fused into the layer's kernels: the statistics kernel rotates each K
+ * tile and the output kernel each Q tile in shared memory, between the TMA load and the tensor
+ * cores, so q and k are read once and never rewritten. The result equals gdn_rope_3d of q and of
+ * k (same f32 arithmetic and bf16 rounding of the rotated values) followed by gdn_frame_forward.
+ * Arguments: those of gdn_frame_forward, then the latent grid of a frame (grid_h * grid_w == N,
+ * token n at row n / grid_w, column n % grid_w), the rotary base (> 1, finite; 10000 is usual)
+ * and t_offset (>= 0, the absolute index of the clip's first frame, so a resumed clip continues
+ * its time positions). Host-side errors as gdn_frame_forward and gdn_rope_3d. Same path choice
+ * (fused, three kernels, chunked) and workspace as gdn_frame_forward, plus a per-GPU cos/sin
+ * table of 8 * (T * d_t / 2 + grid_h * d_h / 2 + grid_w * d_w / 2) bytes (grown like the
+ * workspace, freed by gdn_release_workspace), computed by one extra launch on `stream`.
+ */
+gdn_status gdn_frame_forward_rope(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                  const float* gamma, const float* beta, const float* state_in,
+                                  gdn_bf16* out, float* state_out, int B, int H, int T, int N,
+                                  int D, float key_scale, int grid_h, int grid_w,
+                                  float rope_base, int t_offset, gdn_stream_t stream);
 
 /*
  * gdn_frame_forward_fp8 - gdn_frame_forward on 8-bit E4M3 q, k, v with one scale per
@@ -287,6 +313,27 @@ size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D);
  */
 gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int H, int D,
                        int grid_h, int grid_w, float base, int t_offset, gdn_stream_t stream);
+
+/*
+ * gdn_softmax_attention - the softmax attention of the hybrid DiT's softmax blocks (the
+ * ai-papers.net SANA-WM article, section "ハイブリッドアテンション機構", and the gen-hub.ru article,
+ * section "Архитектура: четыре нетривиальных решения": softmax attention in blocks 3, 7, 11, 15
+ * and 19 of 20; the same gen-hub.ru article, section "Три режима на любой вкус": bidirectional and
+ * chunk-causal autoregressive generation). Per (batch, head), over the clip's T*N tokens:
+ *   out = softmax(Q K^T * scale + M) V,
+ * where a token of frame t sees every token of the frames t' < (t / F + 1) * F (F =
+ * frames_per_chunk): bidirectional inside a chunk of F frames, causal across chunks; F >= T is
+ * full bidirectional attention. q and k arrive with any positional encoding already applied.
+ * q, k, v, out: [B, T, N, H, D] bf16 device pointers (the layout of the GDN entry points),
+ * 16-byte aligned; out must not overlap q, k or v. scale: 0 selects 1/sqrt(D); otherwise finite
+ * and > 0. D a multiple of 8 in [8, 128] (GDN_ERR_UNSUPPORTED otherwise); T*N < 2^31.
+ * One launch, no workspace: a persistent tcgen05 kernel (S = Q K^T and O += P V on the tensor
+ * cores with accumulators in TMEM, an online softmax with f32 row statistics, P rounded to bf16
+ * for the second product, O / l rounded to bf16).
+ */
+gdn_status gdn_softmax_attention(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                 gdn_bf16* out, int B, int H, int T, int N, int D,
+                                 int frames_per_chunk, float scale, gdn_stream_t stream);
 
 /* Device workspace bytes gdn_frame_forward / gdn_frame_step need for these sizes. */
 size_t gdn_workspace_bytes(int B, int H, int T, int N, int D);

@@ -198,4 +198,42 @@ def test_binding_holds_no_key_scale_arithmetic():
     """The Python binding passes key_scale through (None as 0); the default scale is computed
     in the library."""
     src = open(os.path.join(ROOT, "frame_wise_gated_deltanet_b200", "api.py")).read()
-    assert "sqrt" not in src and "import math" not in src
+    for pattern in ("math.", "np.sqrt", "torch.sqrt", "rsqrt", "** 0.5", "** -0.5", "import math"):
+        assert pattern not in src, pattern
+
+
+def test_forward_rope_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_frame_forward_rope
+
+    def args(D=32, gh=4, gw=4, base=10000.0, toff=0, ks=0.1, q=P):
+        return (q, P + 0x10000, P + 0x20000, P + 0x30000, P + 0x31000, None, P + 0x40000, None,
+                1, 2, 3, 16, D, ks, gh, gw, base, toff, None)
+    assert f(*args(q=None)) == 1
+    assert f(*args(D=36)) == 2           # not a multiple of 8
+    assert f(*args(gh=3)) == 1           # grid_h * grid_w != N
+    assert f(*args(base=1.0)) == 1
+    assert f(*args(base=float("nan"))) == 1
+    assert f(*args(toff=-1)) == 1
+    assert f(*args(ks=-1.0)) == 1
+    assert f(*args(q=P + 8)) == 3        # misaligned
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*args()) == 5
+
+
+def test_softmax_attention_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_softmax_attention
+
+    def args(D=64, F=2, scale=0.0, out=P + 0x40000, q=P):
+        return (q, P + 0x10000, P + 0x20000, out, 1, 2, 3, 16, D, F, scale, None)
+    assert f(*args(q=None)) == 1
+    assert f(*args(F=0)) == 1            # frames_per_chunk < 1
+    assert f(*args(D=36)) == 2           # not a multiple of 8
+    assert f(*args(D=136)) == 2          # above 128
+    assert f(*args(scale=-1.0)) == 1
+    assert f(*args(scale=float("inf"))) == 1
+    assert f(*args(out=P + 0x10000)) == 1  # out overlaps k
+    assert f(*args(out=P + 0x40008)) == 3  # misaligned
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*args()) == 5
