@@ -42,6 +42,8 @@ sys.path.insert(0, ROOT)
 METRIC = "GDN layer tokens·heads/sec and % of roofline (720p 60 s config, 1 B200)"
 METRIC_BWD = "GDN layer backward tokens·heads/sec (720p 60 s config, 1 B200)"
 METRIC_ROPE = "3D RoPE of q and k, tokens·heads/sec (720p 60 s config, 1 B200)"
+METRIC_ROPE_FUSED = "GDN layer with fused 3D RoPE of q and k, tokens·heads/sec (720p 60 s config, 1 B200)"
+METRIC_SOFTMAX = "chunk-causal softmax attention tokens·heads/sec and % of bf16 tensor peak (1 B200)"
 UNIT = "tokens*heads/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -67,6 +69,9 @@ def args_parse():
                     help="time gdn_frame_backward (the training pass) instead of the forward")
     ap.add_argument("--rope", action="store_true",
                     help="time gdn_rope_3d on the clip's q and k (in place) instead of the forward")
+    ap.add_argument("--rope-fused", action="store_true",
+                    help="time gdn_frame_forward_rope (the forward with the 3D RoPE of q and k "
+                         "fused into its kernels) instead of the forward")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other configurations' records (480p, stream, LA, fp8, "
                          "backward, RoPE) that the default 720p run adds to its line")
@@ -429,7 +434,7 @@ def main():
     # --shard heads: the ranks split one clip's heads (strong scaling; per-rank byte counts use
     # the rank's own heads); otherwise every rank runs its own clip (weak scaling)
     shard = a.shard == "heads" and world > 1
-    if a.shard == "heads" and (w.kind != "gdn" or a.fp8 or a.backward or a.rope):
+    if a.shard == "heads" and (w.kind != "gdn" or a.fp8 or a.backward or a.rope or a.rope_fused):
         raise ValueError("--shard heads applies to the bf16 forward of a GDN clip")
     w_rank = w
     if shard:
@@ -479,6 +484,26 @@ def main():
             api.gdn_frame_forward_fp8(f8["q"], f8["k"], f8["v"], f8["sq"], f8["sk"], f8["sv"],
                                       gam, bet, None, out, st, key_scale=w.key_scale,
                                       stream=stream)
+    elif w.kind == "softmax":
+        # chunk-causal softmax attention of the hybrid blocks over the clip's tokens
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        q, k, v = g["q"], g["k"], g["v"]
+        out = torch.empty_like(q)
+        st = None
+
+        def step():
+            api.gdn_softmax_attention(q, k, v, w.frames_per_block, out=out, stream=stream)
+    elif a.rope_fused:
+        # the forward with the 3D RoPE of q and k fused into its statistics and output kernels
+        g = gdn_inputs.workload_inputs(w, device=dev)
+        q, k, v, gam, bet = g["q"], g["k"], g["v"], g["gamma"], g["beta"]
+        gh, gw = (int(x) for x in w.grid.split("x"))
+        out = torch.empty_like(q)
+        st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+        def step():
+            api.gdn_frame_forward_rope(q, k, v, gam, bet, gh, gw, out=out, state_out=st,
+                                       key_scale=w.key_scale, stream=stream)
     elif a.rope:
         # the 3D RoPE prologue of the clip's q and k, in place (22 x 40 latent grid at 720p)
         g = gdn_inputs.workload_inputs(w, device=dev)
@@ -571,7 +596,10 @@ def main():
     hbm, peak_kind = peaks()
     kb = per_launch_bytes(dom, w, a.fp8, a.backward, a.steps, per_kernel[dom][1])
     achieved = kb / (dom_ms * 1e-3) / 1e9 if kb else None
-    path_bytes = (rope_bytes(w) if a.rope else
+    sm_flops = (softmax_flops(w.B, w.H, w.T, w.N, w.D, w.frames_per_block)
+                if w.kind == "softmax" else None)
+    path_bytes = (4 * w.B * w.T * w.N * w.H * w.D * 2 if w.kind == "softmax" else
+                  rope_bytes(w) if a.rope else
                   backward_bytes(w) if a.backward else algorithmic_bytes(w, a.fp8))
     path_gbs = path_bytes / (ms / a.steps * 1e-3) / 1e9
 
@@ -579,21 +607,23 @@ def main():
     e2e = None
     if not a.no_e2e:
         e2e = (measure_e2e(a, w, g, out, st, stream, world, dev)
-               if w.kind == "gdn" and not a.fp8 and not a.backward and not a.rope else None)
+               if w.kind == "gdn" and not a.fp8 and not a.backward and not a.rope
+               and not a.rope_fused else None)
         if shard and e2e and e2e.get("ms_per_step"):
             # the ranks' copies and computes cover one clip: its units in the slowest rank's time
             e2e["value"] = w_all.tokens_heads / (e2e["ms_per_step"] * 1e-3)
 
     workloads = None
     if (not a.no_workloads and world == 1 and w.kind == "gdn" and w.name == "720p" and not a.fp8
-            and not a.backward and not a.rope):
+            and not a.backward and not a.rope and not a.rope_fused):
         sampler2 = ClockSampler("GPU-" + str(props.uuid))
         sampler2.start()
         workloads = measure_workloads(dev, stream, g)
         workloads["clocks"] = sampler2.stop()
 
     line = {
-        "metric": METRIC_ROPE if a.rope else METRIC_BWD if a.backward else METRIC,
+        "metric": (METRIC_ROPE if a.rope else METRIC_BWD if a.backward else
+                   METRIC_ROPE_FUSED if a.rope_fused else METRIC),
         "value": value, "unit": UNIT,
         "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
@@ -618,8 +648,21 @@ def main():
     }
     if workloads is not None:
         line["workloads"] = workloads
+    if sm_flops:
+        # a contraction: measured against the dense bf16 tensor peak
+        tp, tp_kind = tensor_peak()
+        fpl = sm_flops * a.steps / per_kernel[dom][1]
+        ktf = fpl / (dom_ms * 1e-3) / 1e12
+        ptf = sm_flops / (ms / a.steps * 1e-3) / 1e12
+        line["metric"] = METRIC_SOFTMAX
+        line["roofline"] = {"bound": "tensor", "kernel": dom, "achieved": ktf, "peak": tp,
+                            "unit": "TFLOP/s", "frac": ktf / tp, "peak_source": tp_kind,
+                            "traffic": ncu_traffic(dom, w.name),
+                            "algorithmic_flops_per_launch": fpl, "ms_per_launch": dom_ms,
+                            "path": {"algorithmic_flops_per_step": sm_flops,
+                                     "achieved_tflops": ptf, "frac": ptf / tp}}
     if (rank == 0 and world == 1 and not a.no_cpu_baseline and w.kind == "gdn" and not a.fp8
-            and not a.rope):
+            and not a.rope and not a.rope_fused):
         heads = 1 if a.backward else 4
         rate, secs, threads = oracle_sample_rate(w, heads, w.T, backward=a.backward)
         line["cpu_baseline"] = dict({"value": rate, "unit": UNIT, "cores": threads,
@@ -883,9 +926,10 @@ def measure_workloads(dev, stream, g720=None):
     torch.cuda.empty_cache()
 
     # ---- chunk-causal softmax attention of the hybrid blocks (tensor-bound)
-    for label, (B, H, T, N, D, F) in (("softmax_480p", (1, 32, 21, 390, 64, 3)),
-                                      ("softmax_720p21", (1, 20, 21, 880, 128, 3))):
-        x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=1500 + D, device=dev)
+    for label in ("softmax_480p", "softmax_720p21"):
+        ws = W[label]
+        B, H, T, N, D, F = ws.B, ws.H, ws.T, ws.N, ws.D, ws.frames_per_block
+        x = gdn_inputs.workload_inputs(ws, device=dev)
         o = torch.empty_like(x["q"])
 
         def step_sm(x=x, o=o, F=F):

@@ -10,6 +10,8 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgdn.so")
+# the same sources with the device-side address, size and coordinate checks (include/gdn.h)
+DEBUG_LIB_PATH = os.path.join(HERE, "libgdn_debug.so")
 
 STATUS = {
     0: "GDN_OK",
@@ -45,6 +47,8 @@ SIGNATURES = {
     "gdn_sync_status": (_I, [_P]),
     "gdn_release_workspace": (None, []),
     "gdn_version": (_I, []),
+    "gdn_debug_checks": (_I, []),
+    "gdn_debug_report": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_longlong)]),
     "gdn_profile_arm": (_I, [_P, _I]),
     "gdn_set_forward_mode": (_I, [_I]),
     "gdn_profile_count": (_I, []),

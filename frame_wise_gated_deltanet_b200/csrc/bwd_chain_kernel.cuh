@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(mma_done, 1);
-    mbar_init(g_ready, L::kEpiWarps * 32);
+    mbar_init(g_ready, L::kEpiWarps);  // one arrival per epilogue warp
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -241,7 +241,8 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
     write_tile();
     fence_async_smem();
     tc_fence_before();
-    mbar_arrive(g_ready);
+    __syncwarp();  // the warp's tile writes and fences first
+    if (lane == 0) mbar_arrive(g_ready);
     if (first) store_g(T - 1);  // (a later segment's G_{t_hi-1} was stored by the previous one)
 
     // gamma_t, beta_t of frames t_hi-1-(32*blk + lane), shuffled from lane u % 32 at step u
@@ -293,7 +294,8 @@ __global__ void __launch_bounds__(BwdChainLayout<DP>::kThreads, 1)
           write_tile();
           fence_async_smem();
           tc_fence_before();
-          mbar_arrive(g_ready);
+          __syncwarp();  // the warp's tile writes and fences first
+          if (lane == 0) mbar_arrive(g_ready);
         }
         store_g(t - 1);
       }

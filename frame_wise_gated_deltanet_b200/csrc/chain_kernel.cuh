@@ -152,7 +152,7 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
     }
     for (int s = 0; s < L::kGate; ++s) mbar_init(&gate[s], 1);
     mbar_init(mma_done, 1);
-    mbar_init(s_ready, L::kEpiWarps * 32);
+    mbar_init(s_ready, L::kEpiWarps);  // one arrival per epilogue warp
     mbar_init(mma_drain, 1);
     *s_written = 0;
     *abort_flag = 0;
@@ -349,7 +349,8 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       else
         cp_async_commit();
     }
-    mbar_arrive(s_ready);
+    __syncwarp();  // the warp's tile writes and fences first
+    if (lane == 0) mbar_arrive(s_ready);
 
     // gamma_t, beta_t: each lane holds frame (32*blk + lane) of the current and next block of
     // 32 frames; the value for frame t is shuffled from lane t % 32.
@@ -396,7 +397,8 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       write_s_tile();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(s_ready);
+      __syncwarp();  // the warp's tile writes and fences first
+      if (lane == 0) mbar_arrive(s_ready);
       // S_t to global (its slot was gated free): rows past D and M-padding rows hold zeros,
       // rows >= DP (M-padding when DP == 64) are not part of the stored matrix
       if (write_s && v < DP) {

@@ -1612,6 +1612,32 @@ void gdn_release_workspace(void) {
 
 int gdn_version(void) { return 100; }
 
+int gdn_debug_checks(void) {
+#ifdef GDN_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int gdn_debug_report(int* site, long long* value) {
+  int s = 0;
+  long long v = 0;
+  if (cudaMemcpyFromSymbol(&s, gdn::g_debug_site, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&v, gdn::g_debug_value, sizeof(long long)) != cudaSuccess)
+    return -1;
+  if (site) *site = s;
+  if (value) *value = v;
+  if (s != 0) {
+    const int zero = 0;
+    const long long zl = 0;
+    if (cudaMemcpyToSymbol(gdn::g_debug_site, &zero, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(gdn::g_debug_value, &zl, sizeof(long long)) != cudaSuccess)
+      return -1;
+  }
+  return s != 0 ? 1 : 0;
+}
+
 gdn_status gdn_profile_arm(void* const* events, int n) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (events == nullptr || n < 2) {

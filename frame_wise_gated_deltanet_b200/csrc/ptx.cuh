@@ -139,6 +139,57 @@ struct StageFills {
   }
 };
 
+// ------------------------------------------------------------------ debug checks
+// The debug library (libgdn_debug.so, compiled with -DGDN_DEBUG) checks every TMA, bulk and
+// cp.async copy and every MMA operand address before it is issued: shared-memory ranges inside
+// the CTA's allocation, the 16-byte alignments and sizes the copies require, TMA coordinates
+// (innermost coordinate a multiple of 16 bytes' worth of elements, no negative store
+// coordinate). A violation records its site and the offending value in g_debug_site /
+// g_debug_value (first one wins; read and cleared by gdn_debug_report) and the copy is skipped,
+// so the call ends on a bounded wait and an error status rather than on a memory fault. Release
+// builds compile the checks out.
+__device__ int g_debug_site;
+__device__ long long g_debug_value;
+
+enum DebugSite : int {
+  kSiteTmaLoadSmem = 1,   // TMA load destination outside shared memory or not 128-B aligned
+  kSiteTmaLoadCoord = 2,  // TMA load innermost coordinate not a multiple of 16
+  kSiteTmaStoreSmem = 3,  // TMA store source outside shared memory or not 128-B aligned
+  kSiteTmaStoreCoord = 4, // TMA store coordinate negative or innermost not a multiple of 16
+  kSiteBulkSmem = 5,      // bulk copy shared range outside the allocation or misaligned
+  kSiteBulkGlobal = 6,    // bulk copy global address or size not a multiple of 16
+  kSiteCpAsync = 7,       // cp.async addresses misaligned or shared address out of range
+  kSiteDescriptor = 8,    // MMA operand start address outside shared memory
+};
+
+#ifdef GDN_DEBUG
+// The dynamic shared memory of the running kernel (every kernel here keeps all of its shared
+// data there: its extern array starts at the same address as this one).
+extern __shared__ uint8_t gdn_dyn_smem[];
+
+__device__ __forceinline__ bool smem_range_ok(uint32_t saddr, uint32_t bytes) {
+  uint32_t dyn;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(gdn_dyn_smem));
+  return saddr >= base && saddr + bytes <= base + dyn;
+}
+
+// false (and the violation recorded) unless `ok`
+__device__ __forceinline__ bool debug_check(bool ok, int site, long long value) {
+  if (ok) return true;
+  if (atomicCAS(&g_debug_site, 0, site) == 0) atomicExch(reinterpret_cast<unsigned long long*>(
+                                                             &g_debug_value),
+                                                         static_cast<unsigned long long>(value));
+  return false;
+}
+#define GDN_DEBUG_CHECK(cond, site, value) \
+  if (!::gdn::debug_check((cond), (site), static_cast<long long>(value))) return
+#else
+#define GDN_DEBUG_CHECK(cond, site, value) \
+  do {                                     \
+  } while (0)
+#endif
+
 // ------------------------------------------------------------------ TMA (no multicast)
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -158,6 +209,9 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int c0,
                                             int c1, int c2, uint64_t policy) {
+  GDN_DEBUG_CHECK((smem_u32(dst) & 127) == 0 && smem_range_ok(smem_u32(dst), 1), kSiteTmaLoadSmem,
+                  smem_u32(dst));
+  GDN_DEBUG_CHECK((c0 & 15) == 0, kSiteTmaLoadCoord, c0);
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::"
       "cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
@@ -168,6 +222,9 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, uint64_t* bar, int c0,
                                             int c1, int c2, int c3, uint64_t policy) {
+  GDN_DEBUG_CHECK((smem_u32(dst) & 127) == 0 && smem_range_ok(smem_u32(dst), 1), kSiteTmaLoadSmem,
+                  smem_u32(dst));
+  GDN_DEBUG_CHECK((c0 & 15) == 0, kSiteTmaLoadCoord, c0);
   asm volatile(
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::"
       "cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
@@ -179,6 +236,10 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, uint64_
 // TMA tile store smem -> global (bulk-group completion), with an L2 cache policy.
 __device__ __forceinline__ void tma_store_4d(const void* tmap, const void* src, int c0, int c1,
                                              int c2, int c3, uint64_t policy) {
+  GDN_DEBUG_CHECK((smem_u32(src) & 127) == 0 && smem_range_ok(smem_u32(src), 1),
+                  kSiteTmaStoreSmem, smem_u32(src));
+  GDN_DEBUG_CHECK((c0 & 15) == 0 && (c0 | c1 | c2 | c3) >= 0, kSiteTmaStoreCoord,
+                  (static_cast<long long>(c2) << 32) | static_cast<uint32_t>(c0));
   asm volatile(
       "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group.L2::cache_hint"
       " [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(reinterpret_cast<uint64_t>(tmap)),
@@ -188,6 +249,10 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, const void* src, 
 
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int c0, int c1,
                                              int c2, uint64_t policy) {
+  GDN_DEBUG_CHECK((smem_u32(src) & 127) == 0 && smem_range_ok(smem_u32(src), 1),
+                  kSiteTmaStoreSmem, smem_u32(src));
+  GDN_DEBUG_CHECK((c0 & 15) == 0 && (c0 | c1 | c2) >= 0, kSiteTmaStoreCoord,
+                  (static_cast<long long>(c2) << 32) | static_cast<uint32_t>(c0));
   asm volatile(
       "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint"
       " [%0, {%2, %3, %4}], [%1], %5;" ::"l"(reinterpret_cast<uint64_t>(tmap)),
@@ -197,6 +262,10 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, 
 
 // Bulk (non-tensor) copy of `bytes` contiguous bytes shared -> global, bulk-group completion.
 __device__ __forceinline__ void bulk_store(void* gdst, const void* src, uint32_t bytes) {
+  GDN_DEBUG_CHECK((smem_u32(src) & 15) == 0 && smem_range_ok(smem_u32(src), bytes), kSiteBulkSmem,
+                  smem_u32(src));
+  GDN_DEBUG_CHECK((reinterpret_cast<uintptr_t>(gdst) & 15) == 0 && (bytes & 15) == 0,
+                  kSiteBulkGlobal, reinterpret_cast<uintptr_t>(gdst));
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
                    reinterpret_cast<uint64_t>(gdst)),
                "r"(smem_u32(src)), "r"(bytes)
@@ -244,6 +313,9 @@ __device__ __forceinline__ bool named_bar_any(int id, int count, bool pred) {
 // 16-byte asynchronous copy global -> shared through L2 only (no L1 allocation), tracked per
 // thread by commit/wait groups.
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  GDN_DEBUG_CHECK((smem_u32(smem_dst) & 15) == 0 && smem_range_ok(smem_u32(smem_dst), 16) &&
+                      (reinterpret_cast<uintptr_t>(gsrc) & 15) == 0,
+                  kSiteCpAsync, reinterpret_cast<uintptr_t>(gsrc));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
                : "memory");
 }
@@ -273,6 +345,10 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 // Bulk (non-tensor) copy of `bytes` contiguous bytes global -> shared, completing on an mbarrier.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar, uint64_t policy) {
+  GDN_DEBUG_CHECK((smem_u32(dst) & 15) == 0 && smem_range_ok(smem_u32(dst), bytes), kSiteBulkSmem,
+                  smem_u32(dst));
+  GDN_DEBUG_CHECK((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (bytes & 15) == 0,
+                  kSiteBulkGlobal, reinterpret_cast<uintptr_t>(src));
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
@@ -459,6 +535,9 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
 //                    8-row K groups SBO bytes apart.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
                                               uint32_t sbo_bytes) {
+#ifdef GDN_DEBUG
+  if (!debug_check(smem_range_ok(saddr, 16), kSiteDescriptor, saddr)) saddr = 0;
+#endif
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
@@ -473,6 +552,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 // SBO = bytes between core matrices adjacent along M/N.
 __device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t lbo_bytes,
                                                     uint32_t sbo_bytes) {
+#ifdef GDN_DEBUG
+  if (!debug_check(smem_range_ok(saddr, 16), kSiteDescriptor, saddr)) saddr = 0;
+#endif
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(mma_done, 1);
-    mbar_init(s_ready, L::kEpiWarps * 32);
+    mbar_init(s_ready, L::kEpiWarps);  // one arrival per epilogue warp
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
       write_tiles();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(s_ready);
+      __syncwarp();  // the warp's tile writes and fences first
+      if (lane == 0) mbar_arrive(s_ready);
     }
     for (int c = 0; c < steps; ++c) {
       // this thread's slice of C_c, loaded while the MMA runs
@@ -232,7 +233,8 @@ __global__ void __launch_bounds__(ScanLayout<DP>::kThreads, 1)
         write_tiles();
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(s_ready);
+        __syncwarp();  // the warp's tile writes and fences first
+        if (lane == 0) mbar_arrive(s_ready);
       }
       store_start(c + 1);
     }

@@ -23,6 +23,8 @@ are used):
 * ``stream`` B16 H20 D128 N880 (22x40 grid), 64 chained single-frame steps
 * ``720p``   B1 H20 D128 T961 N880 (22x40 grid), a 60 s clip
 * ``la``     B2 H20 D112 T81  N390, block-causal linear attention, 3 frames/block
+* ``softmax_480p`` / ``softmax_720p21``: chunk-causal softmax attention (chunks of 3 frames)
+  of B1 H32 D64 T21 N390 and B1 H20 D128 T21 N880
 
 q, k, v are N(0, 1) drawn in float32 and rounded to bfloat16 (round to nearest
 even). gamma and beta are uniform in the stated ranges, drawn and kept in
@@ -42,7 +44,7 @@ class Workload:
     """One synthetic workload: shapes, gate ranges, seed and kind."""
 
     name: str
-    kind: str  # "gdn" (whole clip), "stream" (chained single-frame steps) or "la"
+    kind: str  # "gdn" (whole clip), "stream" (chained steps), "la" or "softmax"
     B: int
     H: int
     D: int
@@ -53,7 +55,7 @@ class Workload:
     seed: int = 0
     state_std: float = 0.0  # 0 -> the clip starts from S_0 = 0
     steps: int = 0  # "stream": number of chained single-frame calls
-    frames_per_block: int = 0  # "la": frames per causal block
+    frames_per_block: int = 0  # "la": frames per causal block; "softmax": per chunk
     grid: str = ""  # latent token grid of one frame, for the record
 
     @property
@@ -84,6 +86,12 @@ WORKLOADS = {
                         seed=5, grid="22x40"),
     "la": Workload("la", "la", 2, 20, 112, 81, 390, seed=4, frames_per_block=3,
                    grid="15x26"),
+    # chunk-causal softmax attention of the hybrid blocks (chunks of 3 frames): the 480p clip's
+    # shape, and 21 frames of the 720p grid (its full 961 frames are quadratic in the tokens)
+    "softmax_480p": Workload("softmax_480p", "softmax", 1, 32, 64, 21, 390, seed=1564,
+                             frames_per_block=3, grid="15x26"),
+    "softmax_720p21": Workload("softmax_720p21", "softmax", 1, 20, 128, 21, 880, seed=1628,
+                               frames_per_block=3, grid="22x40"),
 }
 
 
@@ -154,7 +162,7 @@ def workload_inputs(w: Workload, device="cpu", step: Optional[int] = None) -> di
             return {"state": st}
         return clip_inputs(w.B, w.H, 1, w.N, w.D, w.gamma_range, w.beta_range,
                            seed=1000 * w.seed + step, device=device)
-    if w.kind == "la":
+    if w.kind in ("la", "softmax"):
         g = _generator(w.seed, device)
         shape = (w.B, w.T, w.N, w.H, w.D)
         return {"q": normal_bf16(shape, g, device), "k": normal_bf16(shape, g, device),

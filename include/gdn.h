@@ -393,6 +393,24 @@ gdn_status gdn_set_forward_mode(int mode);
 /* Library ABI version (major * 100 + minor). */
 int gdn_version(void);
 
+/*
+ * Debug library (libgdn_debug.so, the same sources built with -DGDN_DEBUG; the stand-in for a
+ * memory checker on machines where none can run). Every TMA, bulk and cp.async copy and every
+ * tensor-core operand address is checked on the device before it is issued: shared-memory
+ * ranges inside the kernel's allocation, the copies' 16-byte alignments and sizes, TMA
+ * coordinates (innermost coordinate a multiple of 16 elements, no negative store coordinate).
+ * A violation skips the copy (the call then ends on a bounded wait with GDN_ERR_TIMEOUT, never on
+ * a fault) and records its site (1 TMA load shared address, 2 TMA load coordinate, 3 TMA store
+ * shared address, 4 TMA store coordinate, 5 bulk copy shared range, 6 bulk copy global address
+ * or size, 7 cp.async address, 8 MMA operand address) and the offending value.
+ * gdn_debug_checks(): 1 in the debug library, 0 in the release library (which compiles the checks
+ * out). gdn_debug_report(site, value): synchronous; 1 if a violation was recorded since the last
+ * report (site and value filled, the record cleared), 0 if none, -1 on a CUDA error. Either
+ * pointer may be NULL.
+ */
+int gdn_debug_checks(void);
+int gdn_debug_report(int* site, long long* value);
+
 #ifdef __cplusplus
 }
 #endif

@@ -237,3 +237,15 @@ def test_softmax_attention_rejects_bad_arguments_on_the_host(lib):
     import torch
     if not torch.cuda.is_available():
         assert f(*args()) == 5
+
+
+def test_debug_library_builds_and_exports_the_same_symbols(lib):
+    """libgdn_debug.so (the device-side checks) exports every declared symbol and says it has
+    the checks; the release library compiles them out."""
+    from frame_wise_gated_deltanet_b200 import _lib, build
+    build.build(debug=True)
+    dbg = _lib.load(_lib.DEBUG_LIB_PATH)
+    for s in _declared_symbols():
+        assert hasattr(dbg, s), f"libgdn_debug.so does not export {s}"
+    assert dbg.gdn_debug_checks() == 1
+    assert lib.gdn_debug_checks() == 0

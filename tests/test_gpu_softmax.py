@@ -84,20 +84,14 @@ def test_softmax_attention_deterministic():
     assert torch.equal(a, b)
 
 
-# the benchmark's two softmax workloads: the 480p clip's shape and 21 frames of the 720p grid,
-# chunk-causal with chunks of 3 frames
-BENCH = [
-    ("softmax_480p", 1, 32, 21, 390, 64, 3),
-    ("softmax_720p21", 1, 20, 21, 880, 128, 3),
-]
-
-
-@pytest.mark.parametrize("case", BENCH, ids=lambda c: c[0])
-def test_softmax_attention_bench_workloads_all_heads(case):
-    """The benchmark's softmax workloads in their launch configuration; the oracle recomputes
-    every head, and the errors are those of the whole output tensor."""
-    name, B, H, T, N, D, F = case
-    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=1500 + D, device="cuda")
+@pytest.mark.parametrize("name", ["softmax_480p", "softmax_720p21"])
+def test_softmax_attention_bench_workloads_all_heads(name):
+    """The benchmark's softmax workloads (the 480p clip's shape and 21 frames of the 720p grid,
+    chunks of 3 frames) in their launch configuration; the oracle recomputes every head, and the
+    errors are those of the whole output tensor."""
+    w = gdn_inputs.WORKLOADS[name]
+    H, F = w.H, w.frames_per_block
+    x = gdn_inputs.workload_inputs(w, device="cuda")
     out = api().gdn_softmax_attention(x["q"], x["k"], x["v"], F)
     assert api().gdn_sync_status() == 0
 
@@ -113,8 +107,8 @@ def test_softmax_attention_bench_workloads_all_heads(case):
 
     tot = pu.RelF()
     worst = 0.0
-    for e, w in pu.pool_map(one, range(H), bytes_per_task=4e9):
+    for e, wst in pu.pool_map(one, range(H), bytes_per_task=4e9):
         tot.merge(e)
-        worst = max(worst, w)
+        worst = max(worst, wst)
     pu.log(name + "_all_heads", out=tot, worst_element_of_bound=worst)
     assert tot.value <= O_TOL and worst <= 1.0, f"relF {tot.value:.2e}, worst {worst:.2f}"
