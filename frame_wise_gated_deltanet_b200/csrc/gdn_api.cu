@@ -1189,9 +1189,17 @@ gdn_status run_softmax(int dev, const void* q, const void* k, const void* v, voi
   const int grid = static_cast<int>(items < g_dev[dev].sms ? items : g_dev[dev].sms);
   // scores enter the base-2 exponential as S * scale * log2(e)
   const float c = static_cast<float>(double(scale) * 1.4426950408889634);
+  // (batch, head) pairs per group: their K and V (re-read by every query tile) within ~48 MB of L2
+  const double kv_bytes = 2.0 * Ltok * D * 2;
+  const long bh = long(B) * H;
+  const int G = static_cast<int>(std::max(1L, std::min(bh, static_cast<long>(48.0e6 / kv_bytes))));
+  void* ws = nullptr;  // the work counter
+  if (gdn_status s = get_workspace(dev, 256, st, &ws)) return s;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return GDN_ERR_CUDA;
   {
     ProfiledLaunch pl("gdn_softmax_kernel", st);
-    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, tk, tv, to, B, H, T, N, F, c);
+    kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(tq, tk, tv, to, B, H, T, N, F, c,
+                                                   static_cast<int*>(ws), G);
   }
   return check_launch();
 }
@@ -1503,15 +1511,17 @@ gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int 
     return s;
   float2* tab = static_cast<float2*>(base_ws);
   if (gdn_status s = launch_rope_table(tab, r, n_tab, t_offset, base, st)) return s;
-  // one block row per frame of one batch element, kRopeVecs vectors per thread
-  const int frame_vecs = N * H * (D / 8);
-  const long per_block = 256L * gdn::kRopeVecs;
-  const long chunks = std::min(65535L, (long(frame_vecs) + per_block - 1) / per_block);
+  // one block row per frame of one batch element, one block per kRopeTokens of its tokens
+  const long chunks = (long(N) + gdn::kRopeTokens - 1) / gdn::kRopeTokens;
+  if (chunks > 65535) return GDN_ERR_INVALID_ARG;
   {
     ProfiledLaunch pl("gdn_rope_kernel", st);
-    gdn::gdn_rope_kernel<<<dim3(static_cast<unsigned>(B * T), static_cast<unsigned>(chunks)), 256,
-                           0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x),
-                                    reinterpret_cast<__nv_bfloat16*>(y), tab, r, frame_vecs);
+    // a thread per 16-byte vector of a token (H*D/8 of them, rounded up to whole warps)
+    const int per_tok = H * (D / 8);
+    const int threads = std::min(gdn::kRopeMaxThreads, (per_tok + 31) / 32 * 32);
+    gdn::gdn_rope_kernel<<<dim3(static_cast<unsigned>(B * T), static_cast<unsigned>(chunks)),
+                           threads, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x),
+                                    reinterpret_cast<__nv_bfloat16*>(y), tab, r);
   }
   return check_launch();
 }

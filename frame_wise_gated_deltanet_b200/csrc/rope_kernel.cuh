@@ -55,63 +55,60 @@ __global__ void __launch_bounds__(256)
   tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
 }
 
-// x, y: [B, T, N, H, D] bf16 (may be the same memory). Grid (B*T, chunks): blockIdx.x is one
-// frame of one batch element, whose N*H*D/8 16-byte vectors (frame_vecs) the blockIdx.y chunks
-// cover; all index arithmetic is 32-bit and the frame index is per block. Each thread loads
-// kRopeVecs vectors (a block's stride apart, so a warp's accesses stay coalesced) before it
-// rotates and stores any of them: several loads in flight per thread. It reads and writes only
-// its own vectors, so in place is safe.
-constexpr int kRopeVecs = 4;
+// x, y: [B, T, N, H, D] bf16 (may be the same memory). Grid (B*T, token chunks): blockIdx.x is
+// one frame of one batch element, blockIdx.y a chunk of kRopeTokens of its tokens. A token's
+// H*D/8 16-byte vectors are consecutive, so thread i of a block owns vector i (and i + blockDim,
+// ...) of every token of the chunk: the head-dim group of its vector, hence which axis each of
+// its 4 pairs belongs to and the time pairs' (cos, sin), is fixed for the whole chunk; only the
+// grid row and column advance from token to token (incrementally, no division per vector).
+// Each thread reads and writes only its own vectors, so in place is safe.
+constexpr int kRopeTokens = 16;
+constexpr int kRopeMaxThreads = 512;
 
-__device__ __forceinline__ void rope_rotate_vec(uint4& raw, int vi, int per_tok, int per_row,
-                                                const float2* __restrict__ tab,
-                                                const float2* __restrict__ tab_t,
-                                                const RopeDims& r) {
-  const int n = vi / per_tok;
-  const int dg = (vi - n * per_tok) % per_row;
-  const int row = n / r.grid_w;
-  const int col = n - row * r.grid_w;
-  __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int d = dg * 8 + 2 * p;  // first dim of the pair (slices have even widths)
-    float2 cs;
-    if (d < r.d_t)
-      cs = tab_t[d / 2];
-    else if (d < r.d_t + r.d_h)
-      cs = tab[r.off_h + row * (r.d_h / 2) + (d - r.d_t) / 2];
-    else
-      cs = tab[r.off_w + col * (r.d_w / 2) + (d - r.d_t - r.d_h) / 2];
-    const float2 v = __bfloat1622float2(p2[p]);
-    p2[p] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
-  }
-}
-
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kRopeMaxThreads)
     gdn_rope_kernel(const __nv_bfloat16* x, __nv_bfloat16* y, const float2* __restrict__ tab,
-                    RopeDims r, int frame_vecs) {
+                    RopeDims r) {
   const int bt = blockIdx.x;
   const int t = bt % r.T;
   const int per_row = r.D / 8;  // 16-byte vectors per (token, head)
   const int per_tok = per_row * r.H;
-  const long frame0 = static_cast<long>(bt) * frame_vecs;
+  const int n0 = blockIdx.y * kRopeTokens;
+  const int n1 = min(r.N, n0 + kRopeTokens);
+  const long frame0 = static_cast<long>(bt) * r.N * per_tok;
   const uint4* src = reinterpret_cast<const uint4*>(x) + frame0;
   uint4* dst = reinterpret_cast<uint4*>(y) + frame0;
-  const float2* tab_t = tab + t * (r.d_t / 2);
-  const int span = kRopeVecs * blockDim.x;  // vectors one block handles per round
-  for (int v0 = blockIdx.y * span + threadIdx.x; v0 < frame_vecs; v0 += gridDim.y * span) {
-    uint4 raw[kRopeVecs];
+  const int pt = r.d_t / 2, ph = r.d_h / 2;
+  for (int li = threadIdx.x; li < per_tok; li += blockDim.x) {
+    const int dg = li % per_row;
+    // the 4 pairs of this vector: axis (0 time, 1 row, 2 column) and index within the axis
+    int axis[4], idx[4];
+    float2 cs_t[4];
 #pragma unroll
-    for (int u = 0; u < kRopeVecs; ++u) {
-      const int vi = v0 + u * blockDim.x;
-      if (vi < frame_vecs) raw[u] = __ldcs(src + vi);
+    for (int p = 0; p < 4; ++p) {
+      const int j = dg * 4 + p;  // pair index over the head dimension
+      axis[p] = j < pt ? 0 : (j < pt + ph ? 1 : 2);
+      idx[p] = axis[p] == 0 ? j : (axis[p] == 1 ? j - pt : j - pt - ph);
+      cs_t[p] = axis[p] == 0 ? __ldg(tab + t * pt + idx[p]) : make_float2(1.f, 0.f);
     }
+    int row = n0 / r.grid_w;
+    int col = n0 - row * r.grid_w;
+#pragma unroll 4
+    for (int n = n0; n < n1; ++n) {
+      const long vi = static_cast<long>(n) * per_tok + li;
+      uint4 raw = __ldcs(src + vi);
+      __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
 #pragma unroll
-    for (int u = 0; u < kRopeVecs; ++u) {
-      const int vi = v0 + u * blockDim.x;
-      if (vi < frame_vecs) {
-        rope_rotate_vec(raw[u], vi, per_tok, per_row, tab, tab_t, r);
-        __stcs(dst + vi, raw[u]);
+      for (int p = 0; p < 4; ++p) {
+        const float2 cs = axis[p] == 0 ? cs_t[p]
+                          : axis[p] == 1 ? __ldg(tab + r.off_h + row * ph + idx[p])
+                                         : __ldg(tab + r.off_w + col * ph + idx[p]);
+        const float2 v = __bfloat1622float2(p2[p]);
+        p2[p] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
+      }
+      __stcs(dst + vi, raw);
+      if (++col == r.grid_w) {
+        col = 0;
+        ++row;
       }
     }
   }
@@ -126,27 +123,39 @@ __device__ __forceinline__ void rope_rotate_row(uint8_t* tile, int row, int box,
                                                 int D, const RopeArgs& ra) {
   const int rg = n / ra.grid_w;
   const int cg = n - rg * ra.grid_w;
-  const int tb = t * ra.pt;                            // index of time pair 0
-  const int rb = ra.off_h + rg * ra.ph - ra.pt;        // + j: row pair j - pt
+  const int tb = t * ra.pt;                              // index of time pair 0
+  const int rb = ra.off_h + rg * ra.ph - ra.pt;          // + j: row pair j - pt
   const int cb = ra.off_w + cg * ra.ph - ra.pt - ra.ph;  // + j: column pair j - pt - ph
   uint8_t* rp = tile + box * kBoxBytes + row * 128;
   const uint32_t sw = row & 7;
+  // two halves of 4 chunks (16 pairs): the half's (cos, sin) are loaded before its shared-memory
+  // reads and writes, so the table loads overlap instead of waiting one chunk at a time
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const int d0 = box * 64 + c * 8;
-    if (d0 >= D) break;
-    uint4* ptr = reinterpret_cast<uint4*>(rp + ((c ^ sw) << 4));
-    uint4 raw = *ptr;
-    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+  for (int half = 0; half < 2; ++half) {
+    const int c0 = half * 4;
+    if (box * 64 + c0 * 8 >= D) break;
+    float2 cs[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = (d0 >> 1) + i;  // pair index over the head dimension
+    for (int i = 0; i < 16; ++i) {
+      const int j = box * 32 + c0 * 4 + i;  // pair index over the head dimension
       const int e = j < ra.pt ? tb + j : (j < ra.pt + ra.ph ? rb + j : cb + j);
-      const float2 cs = __ldg(ra.tab + e);
-      const float2 v = __bfloat1622float2(p2[i]);
-      p2[i] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
+      cs[i] = 2 * j < D ? __ldg(ra.tab + e) : make_float2(1.f, 0.f);
     }
-    *ptr = raw;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c = c0 + cc;
+      if (box * 64 + c * 8 >= D) break;
+      uint4* ptr = reinterpret_cast<uint4*>(rp + ((c ^ sw) << 4));
+      uint4 raw = *ptr;
+      __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 w = cs[cc * 4 + i];
+        const float2 v = __bfloat1622float2(p2[i]);
+        p2[i] = __floats2bfloat162_rn(v.x * w.x - v.y * w.y, v.x * w.y + v.y * w.x);
+      }
+      *ptr = raw;
+    }
   }
 }
 

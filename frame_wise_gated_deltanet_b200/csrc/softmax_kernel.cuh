@@ -9,8 +9,8 @@
 // with chunk(r) = frame(r) / F: bidirectional inside a chunk of F frames, causal across chunks
 // (F >= T: fully bidirectional).
 //
-// One persistent CTA per SM takes work items (b, h, 128-query tile), heaviest tiles of a head
-// first, and walks the key tiles the tile's queries may see (128 keys each, up to the chunk limit
+// One persistent CTA per SM takes work items (b, h, 128-query tile) from a global counter in the
+// order of softmax_item, and walks the key tiles the tile's queries may see (128 keys each, up to the chunk limit
 // of its last query) with an online softmax:
 //   S_j = Q K_j^T                       tcgen05, Q and K_j K-major from 128B-swizzled TMA tiles,
 //                                       into one of two TMEM buffers (128 columns each)
@@ -22,10 +22,12 @@
 // warps, and otherwise left alone (P and l use the same stale maximum, so O / l is unchanged).
 // At the end of an item O / l is converted to bf16 in the Q tile's buffer and TMA-stored.
 //
-// Warp roles (6 warps): warp 0 TMA producer (Q once per item, K and V tiles through separate
+// Warp roles (10 warps): warp 0 TMA producer (Q once per item, K and V tiles through separate
 // 2-stage rings), warp 1 TMEM allocator + MMA issuer (S_{j+1} is issued before PV_j so the tensor
-// core computes the next scores while the softmax works on these), warps 2..5 softmax and
-// epilogue (one query row per thread: TMEM lane = row). Every wait is bounded (GDN_ERR_TIMEOUT).
+// core computes the next scores while the softmax works on these), warps 2..9 softmax and
+// epilogue (two threads per query row, each with half of the row's keys and of O's columns: TMEM
+// lane = row; the halves combine their maxima and sums through spare TMEM columns). Every wait
+// is bounded (GDN_ERR_TIMEOUT).
 #pragma once
 #include <cuda.h>
 
@@ -39,9 +41,12 @@ struct SoftmaxLayout {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // 128 rows x DP bf16
   static constexpr int kPBytes = 2 * kBoxBytes;          // 128 queries x 128 keys bf16
   static constexpr int kStages = 2;                      // K ring and V ring depth
-  static constexpr int kThreads = 6 * 32;
+  static constexpr int kSoftmaxWarps = 8;               // two per TMEM lane quarter
+  static constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+  static constexpr int kThreads = 64 + kSoftmaxThreads;
   static constexpr int kTmemCols = 512;                  // S buffers [0,256), O [256, 256+DP)
   static constexpr int kOCol = 256;
+  static constexpr int kXCol = 256 + DP;                 // 6 columns exchanging row partials
   static constexpr int kSmemBytes =
       kTileBytes + 2 * kStages * kTileBytes + 2 * kPBytes + 512 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -61,12 +66,22 @@ struct SoftmaxItem {
   int kmin;     // smallest key limit of its queries (tiles below it need no mask)
 };
 
-__device__ __forceinline__ SoftmaxItem softmax_item(long item, int B, int H, int T, int N,
-                                                    int F) {
+// Work items in the order CTAs take them from a global counter: (batch, head) pairs in groups of
+// G (whose K and V together fit in L2), and inside a group the query tiles from the last (the
+// most key tiles) to the first, the group's heads interleaved: the longest items start first,
+// so CTAs that take the short ones last finish together, and the K and V tiles every item of a
+// head re-reads stay in L2 while the group runs.
+__device__ __forceinline__ SoftmaxItem softmax_item(long item, int B, int H, int T, int N, int F,
+                                                    int G) {
   const int L = T * N;
   const int nqt = (L + kRowsPerTile - 1) / kRowsPerTile;
-  const int bh = static_cast<int>(item / nqt);
-  const int qt = nqt - 1 - static_cast<int>(item - static_cast<long>(bh) * nqt);  // heavy first
+  const int BH = B * H;
+  const long per_group = static_cast<long>(G) * nqt;
+  const int g = static_cast<int>(item / per_group);
+  const int r = static_cast<int>(item - g * per_group);
+  const int ng = min(G, BH - g * G);  // heads of this group (the last may have fewer)
+  const int bh = g * G + r % ng;
+  const int qt = nqt - 1 - r / ng;
   SoftmaxItem it;
   it.b = bh / H;
   it.h = bh - it.b * H;
@@ -78,14 +93,15 @@ __device__ __forceinline__ SoftmaxItem softmax_item(long item, int B, int H, int
 }
 
 // tm_q, tm_k, tm_v, tm_o: 4-D maps (D, H, T*N, B) of [B, T, N, H, D] bf16, boxes 64 x 1 x 128 x 1
-// (rows past T*N read as zero and are not stored). c = scale * log2(e).
+// (rows past T*N read as zero and are not stored). c = scale * log2(e). next_item: a zeroed
+// work counter; G: (batch, head) pairs per group of softmax_item.
 template <int DP>
 __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
     gdn_softmax_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_o, int B, int H, int T, int N,
-                       int F, float c) {
+                       int F, float c, int* next_item, int G) {
   using L = SoftmaxLayout<DP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
@@ -106,7 +122,9 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
   uint64_t* p_free = bars + 16;   // [2] PV_j complete (P buffer free, O updated)
   uint64_t* o_empty = bars + 18;  // the epilogue has read O (128 arrivals)
   uint64_t* mma_drain = bars + 19;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  // item ids from the producer to the other warps (it runs at most one item ahead: the Q buffer)
+  ItemRing ring{reinterpret_cast<int*>(bars + 28), bars + 20};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id();
@@ -124,12 +142,13 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_free[i], L::kSoftmaxWarps);  // one arrival per softmax warp
+      mbar_init(&p_full[i], L::kSoftmaxWarps);
       mbar_init(&p_free[i], 1);
     }
-    mbar_init(o_empty, 128);
+    mbar_init(o_empty, L::kSoftmaxWarps);
     mbar_init(mma_drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -157,9 +176,10 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
       StageFills<2> kf, vf;
       StageFills<1> qf;
       long g = 0;  // key tiles over all items of this CTA
-      int li = 0;
-      for (long item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x, ++li) {
-        const SoftmaxItem it = softmax_item(item, B, H, T, N, F);
+      for (int li = 0; !*abort_flag; ++li) {
+        const long item = ring.produce(li, next_item, n_items);
+        if (item < 0) break;
+        const SoftmaxItem it = softmax_item(item, B, H, T, N, F, G);
         if (li > 0 && !mbar_wait(q_empty, (li & 1) ^ 1)) {
           lost();
           break;
@@ -233,8 +253,11 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
       (void)j;
       return true;
     };
-    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
-      const SoftmaxItem it = softmax_item(item, B, H, T, N, F);
+    for (; ok; ++li) {
+      const long item = ring.consume(li);
+      if (item == -2) ok = false;
+      if (item < 0) break;
+      const SoftmaxItem it = softmax_item(item, B, H, T, N, F, G);
       if (!mbar_wait(q_full, li & 1)) {
         ok = false;
         break;
@@ -282,22 +305,38 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
     mbar_wait(mma_drain, 0);
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
+    // Warp w owns TMEM lane quarter w % 4 (query rows 32*(w%4)..) and half hf of the key columns
+    // of S and P (keys 64*hf..) and of the value columns of O; the two warps of a quarter combine
+    // their row maxima (and at the end their row sums) through spare TMEM columns.
     const uint32_t quarter = warp & 3;
+    const int hf = static_cast<int>(warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + ((quarter * 32) << 16);
+    const int pair_bar = 2 + static_cast<int>(quarter);  // named barrier of the quarter's 2 warps
     const bool leader = (threadIdx.x == 64);
     const uint64_t pol_out = policy_evict_first();
     if (leader) tma_prefetch_desc(&tm_o);
+    // this thread's partial of a row statistic -> the partner's, through TMEM column `col`
+    auto exchange = [&](uint32_t col_mine, uint32_t col_other, float x) -> float {
+      tmem_st1(lane_base + col_mine, x);
+      tc_fence_before();
+      named_bar(pair_bar, 64);
+      tc_fence_after();
+      return tmem_ld1(lane_base + col_other);
+    };
     long g = 0;
     int li = 0;
     bool ok = true;
     float v[32];
-    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
-      const SoftmaxItem it = softmax_item(item, B, H, T, N, F);
+    for (; ok; ++li) {
+      const long item = ring.consume(li);
+      if (item == -2) ok = false;
+      if (item < 0) break;
+      const SoftmaxItem it = softmax_item(item, B, H, T, N, F, G);
       const int r = min(it.q0 + row, Ltok - 1);  // rows past the clip take the last row's limit
       const int kmax = softmax_key_limit(r, N, T, F);
       float m_ref = -INFINITY;  // the maximum P is taken against (log2 units)
-      float l = 0.f;
+      float l = 0.f;            // this thread's half of the row sum
       for (int j = 0; j < it.n_kt; ++j) {
         const long gj = g + j;
         const int s = static_cast<int>(gj & 1);
@@ -307,22 +346,26 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t sacc = lane_base + s * 128;
-        const int k0 = j * kRowsPerTile;
-        const bool masked = k0 + kRowsPerTile > it.kmin;  // uniform over the CTA
-        // pass 1: the row's maximum over its visible keys
+        const int k0 = j * kRowsPerTile + hf * 64;  // first key of this thread's half
+        const bool masked = j * kRowsPerTile + kRowsPerTile > it.kmin;  // uniform over the CTA
+        // the half row's 64 scores in one TMEM read; invisible keys become -inf
+        float sv[64];
+        tmem_ld64(lane_base + s * 128 + hf * 64, sv);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[s]);  // S_j is read: its buffer may take S_{j+2}
         float mx = -INFINITY;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          tmem_ld32(sacc + cc * 32, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const bool vis = !masked || (k0 + cc * 32 + i < kmax);
-            mx = fmaxf(mx, vis ? v[i] : -INFINITY);
-          }
+        for (int i = 0; i < 64; ++i) {
+          if (masked && k0 + i >= kmax) sv[i] = -INFINITY;
+          mx = fmaxf(mx, sv[i]);
         }
+        // both halves' maxima (TMEM columns alternate with the tile's parity, so a partner that
+        // is a tile ahead never overwrites a value still to be read)
+        const uint32_t xc = L::kXCol + 2 * static_cast<uint32_t>(gj & 1);
+        mx = fmaxf(mx, exchange(xc + hf, xc + (hf ^ 1), mx));
         const float m_new = fmaxf(m_ref, mx * c);
-        const bool raise = m_new > m_ref + 8.f;
+        const bool raise = m_new > m_ref + 8.f;  // the same in both warps of the quarter
         if (__any_sync(0xffffffffu, raise)) {
           // the warp's rows take their new maxima; O (from PV_{j-1}) is rescaled in TMEM
           const float alpha = ex2_approx(m_ref - m_new);  // 0 while m_ref is -inf
@@ -336,11 +379,12 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
             }
             tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < DP / 32; ++cc) {
-              tmem_ld32(lane_base + L::kOCol + cc * 32, v);
+            for (int cc = 0; cc < DP / 64; ++cc) {
+              const uint32_t oc = L::kOCol + hf * (DP / 2) + cc * 32;
+              tmem_ld32(lane_base + oc, v);
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] *= alpha;
-              tmem_st32(lane_base + L::kOCol + cc * 32, v);
+              tmem_st32(lane_base + oc, v);
             }
           }
         }
@@ -349,34 +393,28 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
           ok = false;
           break;
         }
-        // pass 2: P = 2^(S c - m_ref) as bf16 into the K-major swizzled P tile, l += sum
-        uint8_t* prow = p_buf + s * L::kPBytes + row * 128;
+        // P = 2^(S c - m_ref) as bf16 into box hf of the K-major swizzled P tile, l += sum
+        uint8_t* prow = p_buf + s * L::kPBytes + hf * kBoxBytes + row * 128;
         const uint32_t sw = row & 7;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          tmem_ld32(sacc + cc * 32, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const bool vis = !masked || (k0 + cc * 32 + i < kmax);
-            v[i] = vis ? ex2_approx(v[i] * c - m_ref) : 0.f;
-            l += v[i];
-          }
-          // 32 keys = 4 chunks of 8 keys; chunk index over the 128 keys: cc * 4 + q
+        for (int kc = 0; kc < 8; ++kc) {  // 8 chunks of 8 keys
+          float pv[8];
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            const int kc = cc * 4 + qd;
-            uint4 pk;
-            pk.x = pack_bf16x2(v[qd * 8 + 0], v[qd * 8 + 1]);
-            pk.y = pack_bf16x2(v[qd * 8 + 2], v[qd * 8 + 3]);
-            pk.z = pack_bf16x2(v[qd * 8 + 4], v[qd * 8 + 5]);
-            pk.w = pack_bf16x2(v[qd * 8 + 6], v[qd * 8 + 7]);
-            *reinterpret_cast<uint4*>(prow + (kc >> 3) * kBoxBytes + (((kc & 7) ^ sw) << 4)) = pk;
+          for (int i = 0; i < 8; ++i) {
+            pv[i] = ex2_approx(fmaf(sv[kc * 8 + i], c, -m_ref));  // 2^-inf = 0: invisible keys
+            l += pv[i];
           }
+          uint4 pk;
+          pk.x = pack_bf16x2(pv[0], pv[1]);
+          pk.y = pack_bf16x2(pv[2], pv[3]);
+          pk.z = pack_bf16x2(pv[4], pv[5]);
+          pk.w = pack_bf16x2(pv[6], pv[7]);
+          *reinterpret_cast<uint4*>(prow + ((kc ^ sw) << 4)) = pk;
         }
         tc_fence_before();
-        mbar_arrive(&s_free[s]);  // both passes have read S_j
         fence_async_smem();
-        mbar_arrive(&p_full[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[s]);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 into the Q buffer (free: every S MMA of the item is done
@@ -387,10 +425,12 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
         break;
       }
       tc_fence_after();
+      l += exchange(L::kXCol + 4 + hf, L::kXCol + 4 + (hf ^ 1), l);
       const float inv_l = 1.f / l;
 #pragma unroll 1
-      for (int cc = 0; cc < DP / 32; ++cc) {
-        tmem_ld32(lane_base + L::kOCol + cc * 32, v);
+      for (int cc = 0; cc < DP / 64; ++cc) {
+        const int col = hf * (DP / 2) + cc * 32;
+        tmem_ld32(lane_base + L::kOCol + col, v);
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
           uint4 pk;
@@ -398,13 +438,14 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
           pk.y = pack_bf16x2(v[j + 2] * inv_l, v[j + 3] * inv_l);
           pk.z = pack_bf16x2(v[j + 4] * inv_l, v[j + 5] * inv_l);
           pk.w = pack_bf16x2(v[j + 6] * inv_l, v[j + 7] * inv_l);
-          *reinterpret_cast<uint4*>(q_buf + swz128_offset_bf16(row, cc * 32 + j, kBoxBytes)) = pk;
+          *reinterpret_cast<uint4*>(q_buf + swz128_offset_bf16(row, col + j, kBoxBytes)) = pk;
         }
       }
       tc_fence_before();
-      mbar_arrive(o_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
       fence_async_smem();
-      named_bar(1, 128);
+      named_bar(1, L::kSoftmaxThreads);
       if (leader) {
 #pragma unroll
         for (int kb = 0; kb < L::kBoxes; ++kb)

@@ -327,9 +327,10 @@ gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int 
  * q, k, v, out: [B, T, N, H, D] bf16 device pointers (the layout of the GDN entry points),
  * 16-byte aligned; out must not overlap q, k or v. scale: 0 selects 1/sqrt(D); otherwise finite
  * and > 0. D a multiple of 8 in [8, 128] (GDN_ERR_UNSUPPORTED otherwise); T*N < 2^31.
- * One launch, no workspace: a persistent tcgen05 kernel (S = Q K^T and O += P V on the tensor
- * cores with accumulators in TMEM, an online softmax with f32 row statistics, P rounded to bf16
- * for the second product, O / l rounded to bf16).
+ * One launch: a persistent tcgen05 kernel (S = Q K^T and O += P V on the tensor cores with
+ * accumulators in TMEM, an online softmax with f32 row statistics, P rounded to bf16 for the
+ * second product, O / l rounded to bf16) whose CTAs take (batch, head, query tile) items from a
+ * work counter, the only workspace it uses (256 bytes of the shared workspace).
  */
 gdn_status gdn_softmax_attention(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
                                  gdn_bf16* out, int B, int H, int T, int N, int D,
