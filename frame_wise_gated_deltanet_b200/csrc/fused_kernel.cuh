@@ -30,13 +30,21 @@ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 #endif
 constexpr int kFusedOutGroups = GDN_FUSED_OUT_GROUPS;
 
+// Threads per token row in the RoPE transform of the statistics and output roles (one 64-dim box
+// each at DP = 128). Three shares per row (12 transform warps, which the 19-warp CTA also fits)
+// measured slower at 720p: the rotation adds shared-memory traffic to roles whose tiles already
+// keep shared memory busy, so more threads do not shorten it.
+template <int DP>
+constexpr int kFusedRopeParts = 2;
+
 template <int DP>
 struct FusedLayout {
   static constexpr int kThreads = ChainLayout<DP>::kThreads;
   static_assert(kThreads >= StatsLayout<DP, false, DP == 128>::kThreads &&
                     kThreads >= OutputLayout<DP, false, kFusedOutGroups, DP == 128>::kThreads &&
-                    kThreads >= StatsLayout<DP, false, false, true>::kThreads &&
-                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, false, true>::kThreads,
+                    kThreads >= StatsLayout<DP, false, false, true, kFusedRopeParts<DP>>::kThreads &&
+                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, false, true,
+                                             kFusedRopeParts<DP>>::kThreads,
                 "the chain role's CTA size must cover the other roles' warps");
   static constexpr int kSmemBytes =
       cmax(ChainLayout<DP>::kSmemBytes,
@@ -64,11 +72,11 @@ __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
     chain_body<DP, true>(&tm_a_ring, B_ring, S_ring, gamma, beta, state_in, state_out, p,
                          h_chain, whole, smem);
   } else if (static_cast<int>(blockIdx.x) < h_out.base) {
-    stats_body<DP, false, true, true, kF8, kRope>(&tm_k, &tm_v, A_ring, B_ring, p, h_stats,
-                                                  smem);
+    stats_body<DP, false, true, true, kF8, kRope, kFusedRopeParts<DP>>(&tm_k, &tm_v, A_ring,
+                                                                       B_ring, p, h_stats, smem);
   } else {
-    output_body<DP, false, true, kFusedOutGroups, kF8, kRope>(&tm_q, &tm_q, S_ring, &tm_o, p, 1,
-                                                              h_out, smem);
+    output_body<DP, false, true, kFusedOutGroups, kF8, kRope, kFusedRopeParts<DP>>(
+        &tm_q, &tm_q, S_ring, &tm_o, p, 1, h_out, smem);
   }
 }
 

@@ -39,13 +39,16 @@
 
 namespace gdn {
 
-template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false>
+// kRopeParts: threads per Q row in the RoPE transform (each rotates an equal share of the row's
+// 16-byte chunks).
+template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false,
+          int kRopeParts = DP / 64>
 struct OutputLayout {
   static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
   static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
   static constexpr bool kTransform = kLA || kF8 || kRope;
-  // transform warps: 4 (one token row each), or for RoPE one 64-dim box of a row per thread
-  static constexpr int kXfWarps = kRope ? 4 * (DP / 64) : 4;
+  // transform warps: 4 (one token row each), or for RoPE kRopeParts per row
+  static constexpr int kXfWarps = kRope ? 4 * kRopeParts : 4;
   static constexpr int kEpiWarps = 4 * kG;
   static constexpr int kCols = DP / kG;                // columns per epilogue thread
   static constexpr int kChunk = kCols < 32 ? kCols : 32;
@@ -113,13 +116,14 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p, i
 // LA: tm_q and tm_o are 3-D maps over the flattened token rows, and out (the raw output) takes
 // the row stores of a block's last, partial tile (a 128-row TMA store would also overwrite the
 // first rows of the next block, which another CTA writes).
-template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false, bool kRope = false>
+template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false, bool kRope = false,
+          int kRopeParts = DP / 64>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
                                             const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
                                             uint8_t* smem, __nv_bfloat16* out = nullptr) {
-  using L = OutputLayout<DP, kLA, kG, kF8, kRope>;
+  using L = OutputLayout<DP, kLA, kG, kF8, kRope, kRopeParts>;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                          // 2 state buffers
   uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
@@ -410,8 +414,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     // (the fused kernel's output CTAs have more warps: the rest stay idle)
     if constexpr (kRope) {
       // ---------------------------------------------------------------- RoPE of the Q tiles
-      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // Q row tid % 128, box tid / 128
-      const int row = tid & 127, box = tid >> 7;
+      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // Q row tid % 128, share tid / 128
+      const int row = tid & 127, part = tid >> 7;
+      const int cb = rope_part_begin(part, kRopeParts, DP / 8);
+      const int ce = rope_part_begin(part + 1, kRopeParts, DP / 8);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -426,7 +432,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           }
           const int n = tile * kRowsPerTile + row;
           if (n < p.N)
-            rope_rotate_row(q_ring + stage * L::kQBytes, row, box, n, it.t, p.D, p.rope);
+            rope_rotate_row(q_ring + stage * L::kQBytes, row, cb, ce, n, it.t, p.D, p.rope);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(256)
 // grid row and column advance from token to token (incrementally, no division per vector).
 // Each thread reads and writes only its own vectors, so in place is safe.
 constexpr int kRopeTokens = 16;
+constexpr int kRopeBatch = 4;
 constexpr int kRopeMaxThreads = 512;
 
 __global__ void __launch_bounds__(kRopeMaxThreads)
@@ -92,60 +93,66 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
     }
     int row = n0 / r.grid_w;
     int col = n0 - row * r.grid_w;
-#pragma unroll 4
-    for (int n = n0; n < n1; ++n) {
-      const long vi = static_cast<long>(n) * per_tok + li;
-      uint4 raw = __ldcs(src + vi);
-      __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+    // groups of kRopeBatch tokens: the group's loads are issued before any of its stores (x and
+    // y may be the same memory, so the compiler could not move a load above a store itself)
+    for (int nb = n0; nb < n1; nb += kRopeBatch) {
+      uint4 raw[kRopeBatch];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float2 cs = axis[p] == 0 ? cs_t[p]
-                          : axis[p] == 1 ? __ldg(tab + r.off_h + row * ph + idx[p])
-                                         : __ldg(tab + r.off_w + col * ph + idx[p]);
-        const float2 v = __bfloat1622float2(p2[p]);
-        p2[p] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
-      }
-      __stcs(dst + vi, raw);
-      if (++col == r.grid_w) {
-        col = 0;
-        ++row;
+      for (int u = 0; u < kRopeBatch; ++u)
+        if (nb + u < n1) raw[u] = __ldcs(src + static_cast<long>(nb + u) * per_tok + li);
+#pragma unroll
+      for (int u = 0; u < kRopeBatch; ++u) {
+        if (nb + u < n1) {
+          __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw[u]);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 cs = axis[p] == 0 ? cs_t[p]
+                              : axis[p] == 1 ? __ldg(tab + r.off_h + row * ph + idx[p])
+                                             : __ldg(tab + r.off_w + col * ph + idx[p]);
+            const float2 v = __bfloat1622float2(p2[p]);
+            p2[p] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
+          }
+          __stcs(dst + static_cast<long>(nb + u) * per_tok + li, raw[u]);
+        }
+        if (++col == r.grid_w) {
+          col = 0;
+          ++row;
+        }
       }
     }
   }
 }
 
 // The same rotation applied in shared memory by the forward's statistics (K) and output (Q)
-// kernels to one token row of a bf16 operand tile just loaded by TMA: the 64 dims of box `box`
-// (each box is 128 rows of 128 B, 128B-swizzled, kBoxBytes apart) of row `row`, which holds
-// token n of frame t. Dims at or past D are left alone (TMA zero fill). The arithmetic and the
-// rounding are those of gdn_rope_kernel, so the operand equals the standalone pass's output.
-__device__ __forceinline__ void rope_rotate_row(uint8_t* tile, int row, int box, int n, int t,
-                                                int D, const RopeArgs& ra) {
+// kernels to one token row of a bf16 operand tile just loaded by TMA: chunks [c_begin, c_end) of
+// the row's 16-byte chunks of 8 dims (chunk c in box c / 8; each box is 128 rows of 128 B,
+// 128B-swizzled, kBoxBytes apart) of row `row`, which holds token n of frame t. Dims at or past D
+// are left alone (TMA zero fill). The arithmetic and the rounding are those of gdn_rope_kernel, so
+// the operand equals the standalone pass's output. The (cos, sin) of up to 4 chunks are loaded
+// before those chunks' shared-memory reads and writes, so the table loads overlap.
+__device__ __forceinline__ void rope_rotate_row(uint8_t* tile, int row, int c_begin, int c_end,
+                                                int n, int t, int D, const RopeArgs& ra) {
   const int rg = n / ra.grid_w;
   const int cg = n - rg * ra.grid_w;
   const int tb = t * ra.pt;                              // index of time pair 0
   const int rb = ra.off_h + rg * ra.ph - ra.pt;          // + j: row pair j - pt
   const int cb = ra.off_w + cg * ra.ph - ra.pt - ra.ph;  // + j: column pair j - pt - ph
-  uint8_t* rp = tile + box * kBoxBytes + row * 128;
   const uint32_t sw = row & 7;
-  // two halves of 4 chunks (16 pairs): the half's (cos, sin) are loaded before its shared-memory
-  // reads and writes, so the table loads overlap instead of waiting one chunk at a time
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int c0 = half * 4;
-    if (box * 64 + c0 * 8 >= D) break;
+  c_end = min(c_end, D / 8);
+  for (int c0 = c_begin; c0 < c_end; c0 += 4) {
     float2 cs[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int j = box * 32 + c0 * 4 + i;  // pair index over the head dimension
+      const int j = c0 * 4 + i;  // pair index over the head dimension
       const int e = j < ra.pt ? tb + j : (j < ra.pt + ra.ph ? rb + j : cb + j);
-      cs[i] = 2 * j < D ? __ldg(ra.tab + e) : make_float2(1.f, 0.f);
+      cs[i] = c0 + i / 4 < c_end ? __ldg(ra.tab + e) : make_float2(1.f, 0.f);
     }
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       const int c = c0 + cc;
-      if (box * 64 + c * 8 >= D) break;
-      uint4* ptr = reinterpret_cast<uint4*>(rp + ((c ^ sw) << 4));
+      if (c >= c_end) break;
+      uint4* ptr = reinterpret_cast<uint4*>(tile + (c >> 3) * kBoxBytes + row * 128 +
+                                            (((c & 7) ^ sw) << 4));
       uint4 raw = *ptr;
       __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
 #pragma unroll
@@ -157,6 +164,11 @@ __device__ __forceinline__ void rope_rotate_row(uint8_t* tile, int row, int box,
       *ptr = raw;
     }
   }
+}
+
+// Chunks [begin, end) of part `part` of `parts` equal shares of a row's DP / 8 chunks.
+__device__ __forceinline__ int rope_part_begin(int part, int parts, int chunks) {
+  return part * chunks / parts;
 }
 
 }  // namespace gdn

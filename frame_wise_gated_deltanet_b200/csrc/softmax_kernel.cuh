@@ -354,12 +354,14 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[s]);  // S_j is read: its buffer may take S_{j+2}
-        float mx = -INFINITY;
+        // four independent maxima (short dependency chains), then combined
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           if (masked && k0 + i >= kmax) sv[i] = -INFINITY;
-          mx = fmaxf(mx, sv[i]);
+          m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
         }
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         // both halves' maxima (TMEM columns alternate with the tile's parity, so a partner that
         // is a tile ahead never overwrites a value still to be read)
         const uint32_t xc = L::kXCol + 2 * static_cast<uint32_t>(gj & 1);
@@ -396,13 +398,14 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
         // P = 2^(S c - m_ref) as bf16 into box hf of the K-major swizzled P tile, l += sum
         uint8_t* prow = p_buf + s * L::kPBytes + hf * kBoxBytes + row * 128;
         const uint32_t sw = row & 7;
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {  // 8 chunks of 8 keys
           float pv[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             pv[i] = ex2_approx(fmaf(sv[kc * 8 + i], c, -m_ref));  // 2^-inf = 0: invisible keys
-            l += pv[i];
+            l8[i] += pv[i];
           }
           uint4 pk;
           pk.x = pack_bf16x2(pv[0], pv[1]);
@@ -411,6 +414,7 @@ __global__ void __launch_bounds__(SoftmaxLayout<DP>::kThreads, 1)
           pk.w = pack_bf16x2(pv[6], pv[7]);
           *reinterpret_cast<uint4*>(prow + ((kc ^ sw) << 4)) = pk;
         }
+        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         tc_fence_before();
         fence_async_smem();
         __syncwarp();

@@ -33,7 +33,9 @@
 
 namespace gdn {
 
-template <int DP, bool kLA, bool kF8 = false, bool kRope = false>
+// kRopeParts: threads per K row in the RoPE transform (each rotates an equal share of the row's
+// 16-byte chunks).
+template <int DP, bool kLA, bool kF8 = false, bool kRope = false, int kRopeParts = DP / 64>
 struct StatsLayout {
   static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
   static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
@@ -44,8 +46,8 @@ struct StatsLayout {
   static constexpr int kStages = (DP == 128) ? 3 : 6;
   static constexpr int kAccCols = kLA ? 128 : (DP == 128 ? 256 : 64);
   static constexpr int kTmemCols = 2 * kAccCols;
-  // fp8: one K or V row per thread; RoPE: one 64-dim box of one K row per thread
-  static constexpr int kTransformThreads = kF8 ? 256 : (kRope ? 128 * kBoxes : 128);
+  // fp8: one K or V row per thread; RoPE: a share of one K row per thread
+  static constexpr int kTransformThreads = kF8 ? 256 : (kRope ? 128 * kRopeParts : 128);
   static constexpr int kThreads = 192 + (kTransform ? kTransformThreads : 0);
   static constexpr int kLoadBytes = kF8 ? kStageBytes / 2 : kStageBytes;  // TMA bytes per stage
   static constexpr int kBarrierBytes = 512;
@@ -91,12 +93,13 @@ __device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, con
 
 // kB4: B_t stored in the four-key interleaved layout of b4_index (the chain's input) instead of
 // row-major (the public gdn_frame_stats layout and the block-causal path).
-template <int DP, bool kLA, bool kFused, bool kB4, bool kF8 = false, bool kRope = false>
+template <int DP, bool kLA, bool kFused, bool kB4, bool kF8 = false, bool kRope = false,
+          int kRopeParts = DP / 64>
 __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                            __nv_bfloat16* __restrict__ A_ws,
                                            float* __restrict__ B_ws, const Problem& p,
                                            const Handoff& hf, uint8_t* smem, int fpb = 1) {
-  using L = StatsLayout<DP, kLA, kF8, kRope>;
+  using L = StatsLayout<DP, kLA, kF8, kRope, kRopeParts>;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
   uint64_t* ready = full + L::kStages;   // LA / fp8: transformed stage
   uint64_t* empty = ready + L::kStages;
@@ -402,8 +405,10 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     // (the fused kernel's stats CTAs have more warps: the rest stay idle)
     if constexpr (kRope) {
       // ---------------------------------------------------------------- RoPE of the K tiles
-      const int tid = threadIdx.x - 192;  // K row tid % 128, 64-dim box tid / 128
-      const int row = tid & 127, box = tid >> 7;
+      const int tid = threadIdx.x - 192;  // K row tid % 128, share tid / 128 of its chunks
+      const int row = tid & 127, part = tid >> 7;
+      const int cb = rope_part_begin(part, kRopeParts, DP / 8);
+      const int ce = rope_part_begin(part + 1, kRopeParts, DP / 8);
       int stage = 0;
       uint32_t phase = 0;
       for (int li = 0;; ++li) {
@@ -417,7 +422,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
             break;
           }
           const int n = tile * kRowsPerTile + row;
-          if (n < p.N) rope_rotate_row(smem + stage * L::kStageBytes, row, box, n, t, p.D, p.rope);
+          if (n < p.N) rope_rotate_row(smem + stage * L::kStageBytes, row, cb, ce, n, t, p.D, p.rope);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {
