@@ -198,11 +198,13 @@ def per_launch_bytes(name, w, fp8, backward, steps, launches):
 # Sources each kernel is built from: an ncu traffic figure stays valid while these are unchanged.
 KERNEL_SOURCES = {
     "gdn_fused_kernel": ["fused_kernel.cuh", "chain_kernel.cuh", "stats_kernel.cuh",
-                         "output_kernel.cuh", "common.cuh", "ptx.cuh"],
+                         "output_kernel.cuh", "rope_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_step_kernel": ["step_kernel.cuh", "common.cuh", "ptx.cuh"],
-    "gdn_stats_kernel": ["stats_kernel.cuh", "common.cuh", "ptx.cuh"],
-    "gdn_stats_kernel_la": ["stats_kernel.cuh", "common.cuh", "ptx.cuh"],
-    "gdn_output_kernel": ["output_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_stats_kernel": ["stats_kernel.cuh", "rope_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_stats_kernel_la": ["stats_kernel.cuh", "rope_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_output_kernel": ["output_kernel.cuh", "rope_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_rope_kernel": ["rope_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_softmax_kernel": ["softmax_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_chain_kernel": ["chain_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_scan_kernel": ["scan_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_bwd_chain_kernel": ["bwd_chain_kernel.cuh", "common.cuh", "ptx.cuh"],
@@ -889,7 +891,33 @@ def measure_workloads(dev, stream, g720=None):
         step_bwd, stream, backward_bytes(w),
         lambda n, l, s, w=w: per_launch_bytes(n, w, False, True, s, l), w.tokens_heads,
         target_ms=150.0)
-    del d_out
+
+    # the training pair: a forward that keeps A_t, B_t, S_t, and the backward that reads them
+    _, _, saved = api.gdn_frame_forward_train(g["q"], g["k"], g["v"], g["gamma"], g["beta"],
+                                              key_scale=w.key_scale, stream=stream)
+
+    def step_bwd_saved():
+        api.gdn_frame_backward_saved(g["q"], g["k"], g["v"], g["gamma"], g["beta"], saved,
+                                     d_out, key_scale=w.key_scale, stream=stream)
+    recs["720p_backward_saved"] = workload_record(
+        "720p_backward_saved", w.name + " clip, gdn_frame_backward_saved (the backward reading "
+                                        "the states gdn_frame_forward_train kept)",
+        step_bwd_saved, stream, backward_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, False, s, l), w.tokens_heads,
+        target_ms=150.0)
+    out_t = torch.empty_like(g["q"])
+    st_t = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+
+    def step_fwd_train():
+        api.gdn_frame_forward_train(g["q"], g["k"], g["v"], g["gamma"], g["beta"], None, saved,
+                                    out_t, st_t, key_scale=w.key_scale, stream=stream)
+    recs["720p_forward_train"] = workload_record(
+        "720p_forward_train", w.name + " clip, gdn_frame_forward_train (three kernels, A_t, B_t, "
+                                       "S_t kept for the backward)",
+        step_fwd_train, stream, algorithmic_bytes(w),
+        lambda n, l, s, w=w: per_launch_bytes(n, w, False, False, s, l), w.tokens_heads,
+        target_ms=150.0)
+    del d_out, saved, out_t
     torch.cuda.empty_cache()
 
     gh, gw = (int(x) for x in w.grid.split("x"))

@@ -10,6 +10,9 @@ _API = (
     "gdn_frame_forward_rope",
     "gdn_frame_step",
     "gdn_frame_backward",
+    "gdn_frame_forward_train",
+    "gdn_frame_backward_saved",
+    "gdn_train_saved_bytes",
     "gdn_rope_3d",
     "gdn_softmax_attention",
     "gdn_frame_stats",

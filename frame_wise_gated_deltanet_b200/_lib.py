@@ -37,6 +37,9 @@ SIGNATURES = {
     "gdn_frame_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_backward": (_I, [_P] * 14 + [_I, _I, _I, _I, _I, _F, _P]),
     "gdn_backward_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "gdn_train_saved_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "gdn_frame_forward_train": (_I, [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P]),
+    "gdn_frame_backward_saved": (_I, [_P] * 15 + [_I, _I, _I, _I, _I, _F, _P]),
     "gdn_rope_3d": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gdn_softmax_attention": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gdn_frame_stats": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),

@@ -13,7 +13,8 @@ import torch
 from ._lib import LIB, GdnError, check
 
 __all__ = ["gdn_frame_forward", "gdn_frame_forward_fp8", "gdn_frame_forward_host",
-           "gdn_frame_forward_rope", "gdn_softmax_attention",
+           "gdn_frame_forward_rope", "gdn_softmax_attention", "gdn_frame_forward_train",
+           "gdn_frame_backward_saved", "gdn_train_saved_bytes",
            "gdn_frame_step", "gdn_frame_backward", "gdn_backward_workspace_bytes", "gdn_rope_3d", "gdn_frame_stats", "gdn_block_causal_la",
            "gdn_sync_status", "gdn_release_workspace", "gdn_workspace_bytes",
            "gdn_la_workspace_bytes", "GdnError"]
@@ -226,6 +227,68 @@ def gdn_frame_backward(q, k, v, gamma, beta, d_out, state_in=None, d_state_out=N
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(d_out),
             _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_gamma), _ptr(d_beta),
             _ptr(d_state_in), B, H, T, N, D, _scale(key_scale), _stream(stream, q.device)))
+    return dq, dk, dv, d_gamma, d_beta, d_state_in
+
+
+def gdn_train_saved_bytes(B, H, T, N, D) -> int:
+    return int(LIB.gdn_train_saved_bytes(B, H, T, N, D))
+
+
+def gdn_frame_forward_train(q, k, v, gamma, beta, state_in=None, saved=None, out=None,
+                            state_out=None, key_scale: Optional[float] = None, stream=None):
+    """gdn_frame_forward that also keeps, in `saved` (a uint8 CUDA tensor of
+    gdn_train_saved_bytes bytes; allocated if None), what gdn_frame_backward_saved needs.
+    64 < D <= 128. Returns (out, state_out, saved)."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    _req(gamma, "gamma", torch.float32, (B, T, H))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    nbytes = gdn_train_saved_bytes(B, H, T, N, D)
+    if saved is None:
+        saved = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _req(saved, "saved", torch.uint8, (nbytes,))
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, T, N, H, D))
+    if state_out is None:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    _req(state_out, "state_out", torch.float32, (B, H, D, D))
+    with torch.cuda.device(q.device):
+        check("gdn_frame_forward_train", LIB.gdn_frame_forward_train(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(out),
+            _ptr(state_out), _ptr(saved), B, H, T, N, D, _scale(key_scale),
+            _stream(stream, q.device)))
+    return out, state_out, saved
+
+
+def gdn_frame_backward_saved(q, k, v, gamma, beta, saved, d_out, state_in=None,
+                             d_state_out=None, key_scale: Optional[float] = None, stream=None,
+                             want_state_grad: bool = True):
+    """gdn_frame_backward using the states gdn_frame_forward_train saved. Returns (dq, dk, dv,
+    d_gamma, d_beta, d_state_in)."""
+    B, T, N, H, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("d_out", d_out)):
+        _req(t, name, torch.bfloat16, (B, T, N, H, D))
+    _req(gamma, "gamma", torch.float32, (B, T, H))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    _req(saved, "saved", torch.uint8, (gdn_train_saved_bytes(B, H, T, N, D),))
+    if state_in is not None:
+        _req(state_in, "state_in", torch.float32, (B, H, D, D))
+    if d_state_out is not None:
+        _req(d_state_out, "d_state_out", torch.float32, (B, H, D, D))
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    d_gamma, d_beta = torch.empty_like(gamma), torch.empty_like(beta)
+    d_state_in = (torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+                  if want_state_grad else None)
+    with torch.cuda.device(q.device):
+        check("gdn_frame_backward_saved", LIB.gdn_frame_backward_saved(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta), _ptr(state_in), _ptr(saved),
+            _ptr(d_out), _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_gamma),
+            _ptr(d_beta), _ptr(d_state_in), B, H, T, N, D, _scale(key_scale),
+            _stream(stream, q.device)))
     return dq, dk, dv, d_gamma, d_beta, d_state_in
 
 

@@ -46,6 +46,17 @@ struct FusedLayout {
                     kThreads >= OutputLayout<DP, false, kFusedOutGroups, false, true,
                                              kFusedRopeParts<DP>>::kThreads,
                 "the chain role's CTA size must cover the other roles' warps");
+  // the statistics role's publisher is the CTA's last warp (warp 18), past its transform warps
+  static_assert(kThreads / 32 - 1 == 18 &&
+                    6 + StatsLayout<DP, false, DP == 128>::kTransformThreads / 32 <= 18 &&
+                    6 + StatsLayout<DP, false, false, true, kFusedRopeParts<DP>>::kTransformThreads /
+                            32 <= 18,
+                "statistics publisher warp");
+  static_assert(2 + 4 * kFusedOutGroups + OutputLayout<DP, false, kFusedOutGroups, DP == 128>::kXfWarps <= 18 &&
+                    2 + 4 * kFusedOutGroups +
+                            OutputLayout<DP, false, kFusedOutGroups, false, true,
+                                         kFusedRopeParts<DP>>::kXfWarps <= 18,
+                "output publisher warp");
   static constexpr int kSmemBytes =
       cmax(ChainLayout<DP>::kSmemBytes,
            cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes));

@@ -446,18 +446,21 @@ struct FusedWs {
   size_t flag_bytes;
 };
 
-size_t fused_ws_bytes(long bh, long T, int D) {
-  const int kRing = fused_ring();
+// R, Rs: A_t/B_t and S_t ring slots per head (0: the tuned defaults). With R = Rs = T every
+// frame keeps its own slot, and the A, B, S blocks are laid out exactly like the three-kernel
+// workspace (row (b*H + h)*T + t): gdn_frame_forward_train keeps them for the backward.
+size_t fused_ws_bytes(long bh, long T, int D, int R = 0, int Rs = 0) {
+  const int kRing = R > 0 ? R : fused_ring();
   const size_t m = size_t(D) * D * bh * kRing;
-  const size_t dp = padded_dim(D), ms = dp * dp * bh * fused_sring();
+  const size_t dp = padded_dim(D), ms = dp * dp * bh * (Rs > 0 ? Rs : fused_sring());
   const size_t flags = sizeof(int) * (3 * bh * T + bh + 4);
   return align256(m * 2) + align256(m * 4) + align256(ms * 2) + align256(flags);
 }
 
-FusedWs carve_fused(void* base, long bh, long T, int D) {
-  const int kRing = fused_ring();
+FusedWs carve_fused(void* base, long bh, long T, int D, int R = 0, int Rs = 0) {
+  const int kRing = R > 0 ? R : fused_ring();
   const size_t m = size_t(D) * D * bh * kRing;
-  const size_t dp = padded_dim(D), ms = dp * dp * bh * fused_sring();
+  const size_t dp = padded_dim(D), ms = dp * dp * bh * (Rs > 0 ? Rs : fused_sring());
   uint8_t* p = static_cast<uint8_t*>(base);
   FusedWs w;
   w.A = p;
@@ -484,17 +487,21 @@ bool fused_applies(int dev, const Problem& p) {
   return bh * 3 <= sms && p.T >= 4;
 }
 
+// keep_all: every frame keeps its own A_t/B_t/S_t slot (R = Rs = T) in the caller's buffer
+// `kept` (fused_ws_bytes(bh, T, D, T, T) bytes) instead of the cached workspace's rings.
 template <int DP, bool kF8 = false, bool kRope = false>
 gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, const void* v,
                      const float* gamma, const float* beta, const float* s_in, void* out,
-                     float* s_out, cudaStream_t st) {
+                     float* s_out, cudaStream_t st, void* kept = nullptr) {
   using L = gdn::FusedLayout<DP>;
   const int sms = g_dev[dev].sms;
   const int bh = p.B * p.H;
-  const int kRing = fused_ring();
-  void* base = nullptr;
-  if (gdn_status s = get_workspace(dev, fused_ws_bytes(bh, p.T, p.D), st, &base)) return s;
-  FusedWs w = carve_fused(base, bh, p.T, p.D);
+  const int kRing = kept ? p.T : fused_ring();
+  const int kSRing = kept ? p.T : fused_sring();
+  void* base = kept;
+  if (!kept)
+    if (gdn_status s = get_workspace(dev, fused_ws_bytes(bh, p.T, p.D), st, &base)) return s;
+  FusedWs w = carve_fused(base, bh, p.T, p.D, kRing, kSRing);
   if (cudaMemsetAsync(w.flags, 0, w.flag_bytes, st) != cudaSuccess) return GDN_ERR_CUDA;
   CUtensorMap tk, tv, tq, to, ta;
   if (!tmap_in<kF8>(&tk, k, p) || !tmap_in<kF8>(&tv, v, p) || !tmap_in<kF8>(&tq, q, p) ||
@@ -516,8 +523,7 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   // but never published, so the chain's wait for them runs out and the call reports
   // GDN_ERR_TIMEOUT through gdn_sync_status
   static const int withhold = env_int("GDN_TEST_WITHHOLD_FRAME", -1, -1, 1 << 30);
-  gdn::Handoff hc{f, f + ft, f + 2 * ft, abort_word, nullptr, kRing, fused_sring(), withhold,
-                  0, bh};
+  gdn::Handoff hc{f, f + ft, f + 2 * ft, abort_word, nullptr, kRing, kSRing, withhold, 0, bh};
   hc.ready_tail = abort_word + 3;
   hc.ready_items = abort_word + 4;
   gdn::Handoff hs = hc;
@@ -818,6 +824,31 @@ size_t backward_ws_bytes(long count, int D, long bh) {
          align256(count * m * 4) + align256(bh * m * 4);
 }
 
+// With the forward's A_t, B_t, S_t saved by gdn_frame_forward_train, the workspace holds only
+// E_t, G_t, W'_t and the carried G.
+size_t backward_saved_ws_bytes(long count, int D, long bh) {
+  const size_t m = size_t(D) * D, dp2 = size_t(128) * 128;
+  return align256(count * m * 4) + 2 * align256(count * dp2 * 2) + align256(bh * m * 4);
+}
+
+BackwardWs carve_backward_saved(void* base, const void* saved, long count, int D) {
+  const size_t m = size_t(D) * D, dp2 = size_t(128) * 128;
+  const ForwardWs f = carve_forward(const_cast<void*>(saved), count, D);
+  uint8_t* p = static_cast<uint8_t*>(base);
+  BackwardWs w;
+  w.A = f.A;
+  w.B = f.B;
+  w.S = f.S;
+  w.E = reinterpret_cast<float*>(p);
+  p += align256(count * m * 4);
+  w.G = p;
+  p += align256(count * dp2 * 2);
+  w.W = p;
+  p += align256(count * dp2 * 2);
+  w.C = reinterpret_cast<float*>(p);
+  return w;
+}
+
 BackwardWs carve_backward(void* base, long count, int D) {
   const size_t m = size_t(D) * D, dp2 = size_t(128) * 128;
   uint8_t* p = static_cast<uint8_t*>(base);
@@ -928,16 +959,21 @@ gdn_status aux_stream(int dev, DeviceState** out) {
   return GDN_OK;
 }
 
+// saved: the forward's A_t, B_t, S_t as gdn_frame_forward_train stored them, or nullptr (the
+// statistics and the state chain of the forward are recomputed first).
 gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
                          const float* gamma, const float* beta, const float* s_in,
                          const void* d_out, const float* ds_out, void* dq, void* dk, void* dv,
                          float* d_gamma, float* d_beta, float* ds_in, const Problem& p,
-                         cudaStream_t st) {
+                         cudaStream_t st, const void* saved = nullptr) {
   const long count = long(p.B) * p.H * p.T;
   const long bh = long(p.B) * p.H;
   void* base = nullptr;
-  if (gdn_status s = get_workspace(dev, backward_ws_bytes(count, p.D, bh), st, &base)) return s;
-  const BackwardWs w = carve_backward(base, count, p.D);
+  const size_t ws_bytes =
+      saved ? backward_saved_ws_bytes(count, p.D, bh) : backward_ws_bytes(count, p.D, bh);
+  if (gdn_status s = get_workspace(dev, ws_bytes, st, &base)) return s;
+  const BackwardWs w =
+      saved ? carve_backward_saved(base, saved, count, p.D) : carve_backward(base, count, p.D);
   const gdn::ChainSeg whole{p.T, 1, 0, nullptr, nullptr};
   Problem pe = p;  // E_t = dO^T Q: the "B" statistic of (key = q, value = dO), key scale 1
   pe.key_scale = 1.0f;
@@ -958,12 +994,20 @@ gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
   const int n_seg = overlap ? std::max(1, (p.T + seg_target / 2) / seg_target) : 1;
   const int seg_len = (p.T + n_seg - 1) / n_seg;
 
-  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
-  if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the forward statistics
-  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole, st))
+  if (saved == nullptr) {
+    if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
+    if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the forward statistics
+    if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole,
+                                      st))
+      return s;
+  } else if (gdn_status s = link(st, sx, 0)) {  // [A]: aux after the caller's earlier work
     return s;
-  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, sx, side)) return s;
-  if (gdn_status s = link(st, sx, 1)) return s;  // [S]: dq after the forward chain
+  }
+  // E_t statistics beside the forward chain (or, with saved states, on all SMs)
+  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, sx, saved ? 0 : side))
+    return s;
+  if (saved == nullptr)
+    if (gdn_status s = link(st, sx, 1)) return s;  // [S]: dq after the forward chain
   if (gdn_status s = link(sx, st, 2)) return s;  // [E]: backward chain after E_t
   if (gdn_status s = run_bwd_token<1, true, false>(dev, p, d_out, nullptr, w.S, nullptr, nullptr,
                                                    dq, "gdn_bwd_token_kernel_dq", 22, sx, side))
@@ -1205,6 +1249,56 @@ gdn_status run_softmax(int dev, const void* q, const void* k, const void* v, voi
 }
 
 }  // namespace
+
+static gdn_status backward_entry(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                 const float* gamma, const float* beta, const float* state_in,
+                                 const gdn_bf16* d_out, const float* d_state_out, gdn_bf16* dq,
+                                 gdn_bf16* dk, gdn_bf16* dv, float* d_gamma, float* d_beta,
+                                 float* d_state_in, int B, int H, int T, int N, int D,
+                                 float key_scale, gdn_stream_t stream, const void* saved) {
+  if (!q || !k || !v || !gamma || !beta || !d_out || !dq || !dk || !dv || !d_gamma || !d_beta)
+    return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  if (D <= 64) return GDN_ERR_UNSUPPORTED;
+  if (!resolve_key_scale(key_scale, D, N, &key_scale)) return GDN_ERR_INVALID_ARG;
+  const void* dev_ptrs[] = {q, k, v, gamma, beta, d_out, dq, dk, dv, d_gamma, d_beta};
+  for (const void* ptr : dev_ptrs)
+    if (!aligned16(ptr)) return GDN_ERR_MISALIGNED;
+  if ((state_in && !aligned16(state_in)) || (d_state_out && !aligned16(d_state_out)) ||
+      (d_state_in && !aligned16(d_state_in)))
+    return GDN_ERR_MISALIGNED;
+  // outputs must not overlap the inputs or each other (d_state_in may alias d_state_out: each
+  // element is read once before it is written, by the same thread)
+  const size_t n = size_t(B) * T * N * H * D * 2, ng = size_t(B) * T * H * 4,
+               ns = size_t(B) * H * D * D * 4;
+  const void* ins[] = {q, k, v, d_out};
+  const void* outs[] = {dq, dk, dv};
+  for (const void* o : outs) {
+    for (const void* i : ins)
+      if (overlaps(o, n, i, n)) return GDN_ERR_INVALID_ARG;
+    for (const void* o2 : outs)
+      if (o != o2 && overlaps(o, n, o2, n)) return GDN_ERR_INVALID_ARG;
+  }
+  if (overlaps(d_gamma, ng, d_beta, ng) || overlaps(d_gamma, ng, gamma, ng) ||
+      overlaps(d_gamma, ng, beta, ng) || overlaps(d_beta, ng, gamma, ng) ||
+      overlaps(d_beta, ng, beta, ng))
+    return GDN_ERR_INVALID_ARG;
+  if (d_state_in && state_in && overlaps(d_state_in, ns, state_in, ns)) return GDN_ERR_INVALID_ARG;
+  int dev;
+  if (gdn_status s = current_device(&dev)) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const Problem p{B, H, T, N, D, key_scale};
+  if (saved) {  // the saved states must not overlap any output
+    const size_t sb = fused_ws_bytes(long(B) * H, T, D, T, T);
+    const void* outs2[] = {dq, dk, dv};
+    for (const void* o : outs2)
+      if (overlaps(saved, sb, o, n)) return GDN_ERR_INVALID_ARG;
+  }
+  return backward_path(dev, q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv,
+                       d_gamma, d_beta, d_state_in, p, reinterpret_cast<cudaStream_t>(stream),
+                       saved);
+}
+
 
 extern "C" {
 
@@ -1456,40 +1550,62 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
                               gdn_bf16* dk, gdn_bf16* dv, float* d_gamma, float* d_beta,
                               float* d_state_in, int B, int H, int T, int N, int D,
                               float key_scale, gdn_stream_t stream) {
-  if (!q || !k || !v || !gamma || !beta || !d_out || !dq || !dk || !dv || !d_gamma || !d_beta)
-    return GDN_ERR_INVALID_ARG;
-  if (gdn_status s = check_sizes(B, H, T, N, D, 128)) return s;
+  return backward_entry(q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv, d_gamma,
+                        d_beta, d_state_in, B, H, T, N, D, key_scale, stream, nullptr);
+}
+
+size_t gdn_train_saved_bytes(int B, int H, int T, int N, int D) {
+  (void)N;
+  if (B < 1 || H < 1 || T < 1 || D <= 64 || D > 128) return 0;
+  // the three-kernel workspace layout, followed by the fused kernel's hand-off flags
+  return fused_ws_bytes(long(B) * H, T, D, T, T);
+}
+
+gdn_status gdn_frame_forward_train(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                   const float* gamma, const float* beta, const float* state_in,
+                                   gdn_bf16* out, float* state_out, void* saved, int B, int H,
+                                   int T, int N, int D, float key_scale, gdn_stream_t stream) {
+  if (!saved) return GDN_ERR_INVALID_ARG;
+  if (gdn_status s = validate_common(q, k, v, out, gamma, beta, state_in, state_out, B, H, T, N,
+                                     D, key_scale))
+    return s;
   if (D <= 64) return GDN_ERR_UNSUPPORTED;
-  if (!resolve_key_scale(key_scale, D, N, &key_scale)) return GDN_ERR_INVALID_ARG;
-  const void* dev_ptrs[] = {q, k, v, gamma, beta, d_out, dq, dk, dv, d_gamma, d_beta};
-  for (const void* ptr : dev_ptrs)
-    if (!aligned16(ptr)) return GDN_ERR_MISALIGNED;
-  if ((state_in && !aligned16(state_in)) || (d_state_out && !aligned16(d_state_out)) ||
-      (d_state_in && !aligned16(d_state_in)))
-    return GDN_ERR_MISALIGNED;
-  // outputs must not overlap the inputs or each other (d_state_in may alias d_state_out: each
-  // element is read once before it is written, by the same thread)
-  const size_t n = size_t(B) * T * N * H * D * 2, ng = size_t(B) * T * H * 4,
-               ns = size_t(B) * H * D * D * 4;
-  const void* ins[] = {q, k, v, d_out};
-  const void* outs[] = {dq, dk, dv};
-  for (const void* o : outs) {
-    for (const void* i : ins)
-      if (overlaps(o, n, i, n)) return GDN_ERR_INVALID_ARG;
-    for (const void* o2 : outs)
-      if (o != o2 && overlaps(o, n, o2, n)) return GDN_ERR_INVALID_ARG;
-  }
-  if (overlaps(d_gamma, ng, d_beta, ng) || overlaps(d_gamma, ng, gamma, ng) ||
-      overlaps(d_gamma, ng, beta, ng) || overlaps(d_beta, ng, gamma, ng) ||
-      overlaps(d_beta, ng, beta, ng))
-    return GDN_ERR_INVALID_ARG;
-  if (d_state_in && state_in && overlaps(d_state_in, ns, state_in, ns)) return GDN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(saved) & 255) != 0) return GDN_ERR_MISALIGNED;
+  resolve_key_scale(key_scale, D, N, &key_scale);  // validated above
+  const long count = long(B) * H * T;
+  const size_t sb = fused_ws_bytes(long(B) * H, T, D, T, T), n = size_t(B) * T * N * H * D * 2;
+  const void* ins[] = {q, k, v, out};
+  for (const void* x : ins)
+    if (overlaps(saved, sb, x, n)) return GDN_ERR_INVALID_ARG;
   int dev;
   if (gdn_status s = current_device(&dev)) return s;
   std::lock_guard<std::mutex> lock(g_mu);
   const Problem p{B, H, T, N, D, key_scale};
-  return backward_path(dev, q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv,
-                       d_gamma, d_beta, d_state_in, p, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the fused kernel with one ring slot per frame writes A_t, B_t, S_t where the backward reads
+  // them (the three-kernel workspace layout); else the three kernels write them there
+  if (fused_applies(dev, p))
+    return run_fused<128>(dev, p, q, k, v, gamma, beta, state_in, out, state_out, st, saved);
+  const ForwardWs w = carve_forward(saved, count, D);
+  const gdn::ChainSeg whole{T, 1, 0, nullptr, nullptr};
+  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, state_in, w.S, state_out,
+                                    whole, st))
+    return s;
+  return run_output<128, false>(dev, p, q, w.S, D, out, 1, st);
+}
+
+gdn_status gdn_frame_backward_saved(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                    const float* gamma, const float* beta, const float* state_in,
+                                    const void* saved, const gdn_bf16* d_out,
+                                    const float* d_state_out, gdn_bf16* dq, gdn_bf16* dk,
+                                    gdn_bf16* dv, float* d_gamma, float* d_beta,
+                                    float* d_state_in, int B, int H, int T, int N, int D,
+                                    float key_scale, gdn_stream_t stream) {
+  if (!saved) return GDN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(saved) & 255) != 0) return GDN_ERR_MISALIGNED;
+  return backward_entry(q, k, v, gamma, beta, state_in, d_out, d_state_out, dq, dk, dv, d_gamma,
+                        d_beta, d_state_in, B, H, T, N, D, key_scale, stream, saved);
 }
 
 gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int H, int D,

@@ -60,7 +60,12 @@ struct OutputLayout {
   static constexpr int kQLoadBytes = kF8 ? kQBytes / 2 : kQBytes;  // TMA bytes per Q tile
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
   static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
-  static constexpr int kSmemBytes = 2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + 512 + 1024;
+  static constexpr int kBarrierBytes = 1024;
+  static constexpr int kSmemBytes =
+      2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + kBarrierBytes + 1024;
+  // barriers, item ring, TMEM slot and the fused publisher's ring within kBarrierBytes
+  static_assert(8 * (3 * kStages + 4 + 4 + 8 + 1) + 32 + 8 + 8 * 16 + 32 <= kBarrierBytes,
+                "barriers");
 };
 
 struct OutputItem {
@@ -139,6 +144,12 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   uint64_t* mma_drain = acc_empty + 2 + 8;  // all of this CTA's MMAs are complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // fused: the MMA warp hands each item's "S_t is in shared memory" to the publisher warp through
+  // an 8-slot ring, so the GPU-scope release of out_flag does not hold up the MMA issue
+  uint64_t* pub_full = reinterpret_cast<uint64_t*>(tmem_slot + 2);
+  uint64_t* pub_empty = pub_full + 8;
+  int* pub_ids = reinterpret_cast<int*>(pub_empty + 8);
+  constexpr uint32_t kPubWarp = 18;  // the fused CTA's last warp (idle in the output role)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -174,6 +185,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     }
     for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
     mbar_init(mma_drain, 1);
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(&pub_full[i], 1);
+      mbar_init(&pub_empty[i], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -270,10 +285,25 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     uint32_t phase = 0;
     int tc = 0;  // tiles processed (accumulator ring position)
     bool ok = true;
+    // fused: hand item li's out_flag (id >= 0) or the end (-2) to the publisher
+    auto hand_off = [&](int li, int id) -> bool {
+      const int ps = li & 7;
+      if (li >= 8 && !mbar_wait(&pub_empty[ps], ((li >> 3) & 1) ^ 1)) return false;
+      if (lane == 0) {
+        pub_ids[ps] = id;
+        mbar_arrive(&pub_full[ps]);
+      }
+      __syncwarp();
+      return true;
+    };
     for (int li = 0; ok; ++li) {
       const long item = consumer_item(li);
       if (item == -2) ok = false;
-      if (item < 0) break;
+      if (item < 0) {
+        if constexpr (kFused)
+          if (ok && !hand_off(li, -2)) ok = false;
+        break;
+      }
       const int sb = li & 1;
       if (!mbar_wait(&s_full[sb], (li >> 1) & 1)) {
         ok = false;
@@ -282,7 +312,10 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       const OutputItem it = output_item<kFused, kLA>(item, p, F);
       if constexpr (kFused) {
         // S_t is in shared memory: its ring slot may be overwritten by the chain
-        if (lane == 0) st_release(hf.out_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
+        if (!hand_off(li, static_cast<int>(static_cast<long>(it.bh) * p.T + it.t))) {
+          ok = false;
+          break;
+        }
       }
       const uint32_t s_base = smem_u32(s_buf + sb * L::kSBufBytes);
       for (int tile = 0; tile < it.n_tiles; ++tile, ++tc) {
@@ -410,6 +443,25 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     }
     if (leader) bulk_wait_all();
     if (!ok) give_up(hf, abort_flag);
+  } else if (kFused && warp == kPubWarp) {
+    // ---------------------------------------------------------------- publisher (fused)
+    // Releases out_flag of each item whose S_t the MMA warp has seen land in shared memory
+    // (the bulk copy completed on s_full before the hand-off), at GPU scope.
+    if (lane == 0) {
+      for (int li = 0;; ++li) {
+        const int ps = li & 7;
+        if (!mbar_wait(&pub_full[ps], (li >> 3) & 1)) {
+          if (*abort_flag) break;  // the MMA warp gave up: nothing more will arrive
+          give_up(hf, abort_flag);
+          break;
+        }
+        const int id = pub_ids[ps];
+        if (id == -2) break;
+        st_release(hf.out_flag + id, 1);
+        mbar_arrive(&pub_empty[ps]);
+      }
+    }
+    __syncwarp();
   } else if (L::kTransform && warp < 2 + L::kEpiWarps + L::kXfWarps) {
     // (the fused kernel's output CTAs have more warps: the rest stay idle)
     if constexpr (kRope) {

@@ -52,6 +52,8 @@ struct StatsLayout {
   static constexpr int kLoadBytes = kF8 ? kStageBytes / 2 : kStageBytes;  // TMA bytes per stage
   static constexpr int kBarrierBytes = 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+  // barriers, item ring, TMEM slot and the fused publisher's ring within kBarrierBytes
+  static_assert(8 * (3 * kStages + 4 + 8 + 1) + 32 + 8 + 8 * 16 + 32 <= kBarrierBytes, "barriers");
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
 };
 
@@ -109,6 +111,13 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
   uint64_t* mma_drain = acc_empty + 2 + 8;  // all of this CTA's MMAs are complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring.ids + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // fused: the epilogue hands each finished item to the publisher warp through an 8-slot ring
+  // (flag index in pub_ids, one arrival per epilogue warp on pub_full; the publisher frees the
+  // slot on pub_empty), so the GPU-scope release of the flag is off the epilogue's path
+  uint64_t* pub_full = reinterpret_cast<uint64_t*>(tmem_slot + 2);
+  uint64_t* pub_empty = pub_full + 8;
+  int* pub_ids = reinterpret_cast<int*>(pub_empty + 8);
+  constexpr uint32_t kPubWarp = 18;  // the fused CTA's last warp (idle in the statistics role)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -145,6 +154,10 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       mbar_init(&acc_empty[a], 128);
     }
     for (int i = 0; i < 8; ++i) mbar_init(&ring.bars[i], 1);
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(&pub_full[i], 4);
+      mbar_init(&pub_empty[i], 1);
+    }
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -303,7 +316,20 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
         give_up(hf, abort_flag);
         break;
       }
-      if (item < 0) break;
+      if (item < 0) {
+        if constexpr (kFused) {
+          // end of the items: the publisher stops at this slot
+          const int ps = li & 7;
+          if (li >= 8 && !mbar_wait(&pub_empty[ps], ((li >> 3) & 1) ^ 1)) {
+            give_up(hf, abort_flag);
+            break;
+          }
+          if (leader) pub_ids[ps] = -2;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pub_full[ps]);
+        }
+        break;
+      }
       const int acc = li & 1;
       const uint32_t aph = (li >> 1) & 1;
       const StatsItem it = stats_item<kFused>(item, p, hf, fpb);
@@ -393,14 +419,43 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       if constexpr (kFused) {
-        // publish: every epilogue thread's stores, then the flag (the chain reads by TMA)
+        // hand the item to the publisher: every epilogue thread's stores (the chain reads them
+        // by TMA and cp.async), then one arrival per warp on the slot's barrier
+        const int ps = li & 7;
+        if (li >= 8 && !mbar_wait(&pub_empty[ps], ((li >> 3) & 1) ^ 1)) {
+          give_up(hf, abort_flag);
+          break;
+        }
+        if (leader)
+          pub_ids[ps] = (it.bh == 0 && it.t == hf.withhold)
+                            ? -1  // test hook: never published
+                            : static_cast<int>(static_cast<long>(it.bh) * p.T + it.t);
         fence_async_global();
-        __threadfence();
-        named_bar(1, 128);
-        if (leader && !(it.bh == 0 && it.t == hf.withhold))
-          st_release(hf.stats_flag + static_cast<long>(it.bh) * p.T + it.t, 1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pub_full[ps]);
       }
     }
+
+  } else if (kFused && warp == kPubWarp) {
+    // ---------------------------------------------------------------- publisher (fused)
+    // Releases each finished item's stats_flag at GPU scope: the epilogue threads' stores
+    // happen-before their arrivals on the slot's barrier, which this thread acquires, and the
+    // release makes them visible to the chain (which fences the async proxy after its acquire).
+    if (lane == 0) {
+      for (int li = 0;; ++li) {
+        const int ps = li & 7;
+        if (!mbar_wait(&pub_full[ps], (li >> 3) & 1)) {
+          if (*abort_flag) break;  // the epilogue gave up: nothing more will arrive
+          give_up(hf, abort_flag);
+          break;
+        }
+        const int id = pub_ids[ps];
+        if (id == -2) break;
+        if (id >= 0) st_release(hf.stats_flag + id, 1);
+        mbar_arrive(&pub_empty[ps]);
+      }
+    }
+    __syncwarp();
   } else if (L::kTransform && warp < 6 + L::kTransformThreads / 32) {
     // (the fused kernel's stats CTAs have more warps: the rest stay idle)
     if constexpr (kRope) {

@@ -290,6 +290,34 @@ gdn_status gdn_frame_backward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf
 size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D);
 
 /*
+ * Training pair: a forward that keeps what the backward needs, and a backward that uses it
+ * instead of recomputing the forward's statistics and state chain (which read k and v again).
+ *
+ * gdn_frame_forward_train: gdn_frame_forward (same arguments and results; the three-kernel
+ * path) that also stores, in the caller's device buffer `saved` (gdn_train_saved_bytes(B, H, T,
+ * N, D) bytes, 256-byte aligned, not overlapping q, k, v or out), every frame's A_t (bf16), B_t
+ * (f32) and S_t (bf16) in the library's internal layout. 64 < D <= 128 (GDN_ERR_UNSUPPORTED
+ * otherwise); the buffer's contents are only meaningful to gdn_frame_backward_saved.
+ * gdn_frame_backward_saved: gdn_frame_backward (same arguments, results, alignment and overlap
+ * rules) for the same q, k, v, gamma, beta, state_in and key_scale that the forward saved, with
+ * `saved` read instead of recomputed: it skips one statistics pass over k and v and the forward
+ * state chain. Its workspace is smaller than gdn_frame_backward's (no A_t, B_t, S_t).
+ * gdn_train_saved_bytes returns 0 for unsupported sizes.
+ */
+size_t gdn_train_saved_bytes(int B, int H, int T, int N, int D);
+gdn_status gdn_frame_forward_train(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                   const float* gamma, const float* beta, const float* state_in,
+                                   gdn_bf16* out, float* state_out, void* saved, int B, int H,
+                                   int T, int N, int D, float key_scale, gdn_stream_t stream);
+gdn_status gdn_frame_backward_saved(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
+                                    const float* gamma, const float* beta, const float* state_in,
+                                    const void* saved, const gdn_bf16* d_out,
+                                    const float* d_state_out, gdn_bf16* dq, gdn_bf16* dk,
+                                    gdn_bf16* dv, float* d_gamma, float* d_beta,
+                                    float* d_state_in, int B, int H, int T, int N, int D,
+                                    float key_scale, gdn_stream_t stream);
+
+/*
  * gdn_rope_3d - 3D rotary position embedding of q or k before the attention layers.
  * (The transcript of the ICLR 2026 oral talk "SANA-Video: Efficient Video Generation with Block
  * Linear Diffusion Transformer" introduces a 3D RoPE for the linear attention. The pages give no

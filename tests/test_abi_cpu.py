@@ -249,3 +249,32 @@ def test_debug_library_builds_and_exports_the_same_symbols(lib):
         assert hasattr(dbg, s), f"libgdn_debug.so does not export {s}"
     assert dbg.gdn_debug_checks() == 1
     assert lib.gdn_debug_checks() == 0
+
+
+def test_training_pair_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gdn_frame_forward_train
+    S = P + 0x100000  # 256-byte aligned fake "saved" buffer
+
+    def fa(D=128, saved=S, q=P):
+        return (q, P + 0x10000, P + 0x20000, P + 0x30000, P + 0x31000, None, P + 0x40000, None,
+                saved, 1, 2, 3, 16, D, 0.0, None)
+    assert f(*fa(saved=None)) == 1
+    assert f(*fa(D=64)) == 2             # the pair needs 64 < D <= 128
+    assert f(*fa(saved=S + 16)) == 3     # saved must be 256-byte aligned
+    assert f(*fa(saved=P + 0x20000)) == 1  # saved overlaps v
+    assert lib.gdn_train_saved_bytes(1, 2, 3, 16, 64) == 0
+    assert lib.gdn_train_saved_bytes(1, 20, 961, 880, 128) == lib.gdn_workspace_bytes(1, 20, 961, 880, 128) or \
+        lib.gdn_train_saved_bytes(1, 20, 961, 880, 128) >= 19220 * 128 * 1024
+    b = lib.gdn_frame_backward_saved
+
+    def ba(saved=S, dq=P + 0x60000):
+        return (P, P + 0x10000, P + 0x20000, P + 0x30000, P + 0x31000, None, saved, P + 0x40000,
+                None, dq, P + 0x70000, P + 0x80000, P + 0x90000, P + 0x91000, None,
+                1, 2, 3, 16, 128, 0.0, None)
+    assert b(*ba(saved=None)) == 1
+    assert b(*ba(saved=S + 8)) == 3
+    assert b(*ba(dq=P + 0x10000)) == 1   # dq overlaps k
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*fa()) == 5
+        assert b(*ba()) == 5

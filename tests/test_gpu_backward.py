@@ -231,3 +231,58 @@ def test_backward_in_a_cuda_graph():
             os.environ["GDN_BWD_SEGMENT_FRAMES"] = old
     for r, o in zip(ref, got):
         assert torch.equal(r, o)
+
+
+# --------------------------------------------------------------------------- training pair
+
+
+@pytest.mark.parametrize("shape", SHAPES[:4], ids=lambda s: "B%dH%dT%dN%dD%d%s" % (s[:5] + ("s" if s[5] else "",)))
+def test_training_pair_matches_oracle(shape):
+    """gdn_frame_forward_train (the forward that keeps A_t, B_t, S_t) and
+    gdn_frame_backward_saved (the backward that reads them instead of recomputing) against the
+    oracle's forward and backward."""
+    B, H, T, N, D, with_state = shape
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, gamma_range=(0.9, 0.999), beta_range=(0.05, 0.95),
+                               seed=710 + T + D, state_std=0.3 if with_state else 0.0)
+    c = gdn_inputs.cotangents(B, H, T, N, D, seed=810 + T + D, state_std=1.0 if with_state else 0.0)
+    ks = 1.0 / math.sqrt(D * N)
+    g = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    gc = {k: (None if v is None else v.cuda()) for k, v in c.items()}
+    a = api()
+    out, st, saved = a.gdn_frame_forward_train(g["q"], g["k"], g["v"], g["gamma"], g["beta"],
+                                               g["state"], key_scale=ks)
+    got = a.gdn_frame_backward_saved(g["q"], g["k"], g["v"], g["gamma"], g["beta"], saved,
+                                     gc["d_out"], state_in=g["state"],
+                                     d_state_out=gc["d_state"], key_scale=ks)
+    assert a.gdn_sync_status() == 0
+    o_ref, s_ref = oracle.gdn_frame_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["gamma"]),
+                                            f64(x["beta"]), None if x["state"] is None else f64(x["state"]), ks)
+    assert relf(f64(out), o_ref) <= 1e-2 and relf(f64(st), s_ref) <= 5e-3
+    check_against_oracle(x, c, got, ks)
+
+
+def test_training_pair_equals_recomputing_backward_on_720p():
+    """On the 720p clip the saved states are those the recomputing backward builds (the same
+    statistics and chain kernels), so both backwards agree bit for bit; the forward that saves
+    them equals the three-kernel forward bit for bit."""
+    from frame_wise_gated_deltanet_b200 import _lib
+    w = gdn_inputs.WORKLOADS["720p"]
+    x = gdn_inputs.workload_inputs(w, device="cuda")
+    c = gdn_inputs.cotangents(w.B, w.H, w.T, w.N, w.D, seed=904, state_std=1.0, device="cuda")
+    a = api()
+    out, st, saved = a.gdn_frame_forward_train(x["q"], x["k"], x["v"], x["gamma"], x["beta"])
+    got = a.gdn_frame_backward_saved(x["q"], x["k"], x["v"], x["gamma"], x["beta"], saved,
+                                     c["d_out"], d_state_out=c["d_state"])
+    assert a.gdn_sync_status() == 0
+    del saved
+    ref = a.gdn_frame_backward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], c["d_out"],
+                               d_state_out=c["d_state"])
+    try:
+        assert _lib.LIB.gdn_set_forward_mode(1) == 0
+        o3, s3 = a.gdn_frame_forward(x["q"], x["k"], x["v"], x["gamma"], x["beta"])
+    finally:
+        _lib.LIB.gdn_set_forward_mode(0)
+    assert a.gdn_sync_status() == 0
+    assert torch.equal(out, o3) and torch.equal(st, s3)
+    for r, o in zip(ref, got):
+        assert torch.equal(r, o)
