@@ -219,7 +219,13 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
   } else if (warp == L::kWarpMma) {
     // ---------------------------------------------------------------- MMA: P = S_{t-1} A_t
     constexpr uint32_t idesc = idesc_bf16(128, DP, false, false);
-    const uint32_t s_base = smem_u32(s_tile);
+    // Operand descriptors built once (the step's issue is on the chain's path); a k-step adds its
+    // byte offset / 16 to the start-address field, which stays below 2^14 inside shared memory.
+    // S tile: key groups 2ks, 2ks+1 (2048 B apart), 8-row groups 128 B apart.
+    // A_t stages: 128B-swizzled, 64-key blocks of DP rows.
+    const uint64_t da0 = smem_desc_noswz(smem_u32(s_tile), 2048, 128);
+    const uint64_t db0 = smem_desc(smem_u32(smem), 16, 1024);
+    static_assert(L::kStages == 2, "stage descriptors");
     bool ok = true;
     for (int u = 0; u < n; ++u) {
       const int stage = u % L::kStages;
@@ -230,15 +236,11 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       }
       tc_fence_after();
       if (elect_one()) {
-        const uint32_t a_base = smem_u32(smem + stage * L::kABytes);
+        const uint64_t dbs = db0 + (stage ? (L::kABytes >> 4) : 0);
 #pragma unroll
-        for (int ks = 0; ks < DP / 16; ++ks) {
-          // S tile: key groups 2ks, 2ks+1 (2048 B apart), 8-row groups 128 B apart
-          const uint64_t da = smem_desc_noswz(s_base + ks * 2 * 2048, 2048, 128);
-          // A_t stage: 128B-swizzled, 64-key blocks of DP rows
-          const uint64_t db = smem_desc(a_base + (ks >> 2) * DP * 128 + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tmem_base, da, db, idesc, ks != 0);
-        }
+        for (int ks = 0; ks < DP / 16; ++ks)
+          mma_bf16(tmem_base, da0 + ((ks * 2 * 2048) >> 4),
+                   dbs + (((ks >> 2) * DP * 128 + (ks & 3) * 32) >> 4), idesc, ks != 0);
         mma_commit(mma_done);
         mma_commit(&empty[stage]);
       }
@@ -255,6 +257,9 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       if (elect_one()) {
         int published = 0;
         unsigned long long t0 = globaltimer_ns();
+        // queue position of the next frame, reserved a frame ahead so that publishing costs no
+        // atomic round trip (positions still follow the order in which frames are published)
+        int pos = atomicAdd(hf.ready_tail, 1);
         while (published < T) {
           const int done = static_cast<int>(ld_acquire_cta(s_written) / L::kEpiWarps);
           if (done > published) {
@@ -262,8 +267,12 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
             // has acquired; the GPU-scope release makes them visible to the outputs (which
             // fence the async proxy after their acquire)
             st_release(hf.chain_prog + bh, done);
-            for (int f = published; f < done; ++f)  // queue the frames for the outputs
-              st_release(hf.ready_items + atomicAdd(hf.ready_tail, 1), f * p.B * p.H + bh + 1);
+            // queue the frames for the outputs: a plain store suffices, since an output acquires
+            // chain_prog itself before it reads S_t
+            for (int f = published; f < done; ++f) {
+              st_relaxed(hf.ready_items + pos, f * p.B * p.H + bh + 1);
+              if (f + 1 < T) pos = atomicAdd(hf.ready_tail, 1);
+            }
             published = done;
             t0 = globaltimer_ns();
             continue;
@@ -371,27 +380,50 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       }
       const float g = __shfl_sync(0xffffffffu, g_cur, u & 31);
       const float be = __shfl_sync(0xffffffffu, b_cur, u & 31);
+      // S_t = gamma_t S_{t-1} + beta_t B_t - gamma_t beta_t S_{t-1} A_t. DP = 64: the part that
+      // does not need the product is formed while the MMA runs, so that one FMA per element
+      // follows the wait (the chain's step bounds short clips); DP = 128 keeps the B_t reads
+      // next to their use, which the fused kernel's register budget needs.
+      constexpr bool kEarlyB = DP == 64;
+      if constexpr (kEarlyB) {
+        cp_async_wait<1>();  // this thread's copy of B_t (B_{t+1} may still be in flight)
+#pragma unroll
+        for (int j = 0; j < L::kCols; j += 4) {
+          float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (use_b && row_ok && c0 + j < D)
+            bv = *reinterpret_cast<const float4*>(b_slot(u & 1, (c0 + j) >> 2));
+          S[j] = fmaf(g, S[j], be * bv.x);
+          S[j + 1] = fmaf(g, S[j + 1], be * bv.y);
+          S[j + 2] = fmaf(g, S[j + 2], be * bv.z);
+          S[j + 3] = fmaf(g, S[j + 3], be * bv.w);
+        }
+      }
       if (!mbar_wait(mma_done, u & 1)) {
         ok = false;
         break;
       }
-      cp_async_wait<1>();  // this thread's copy of B_t (B_{t+1} may still be in flight)
+      if constexpr (!kEarlyB) cp_async_wait<1>();
       tc_fence_after();
       const float gbe = g * be;
 #pragma unroll
       for (int c = 0; c < L::kCols; c += 16) {
         float P[16];
         tmem_ld16(taddr + c, P);
+        if constexpr (kEarlyB) {
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const int col = c0 + c + j;
-          float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (use_b && row_ok && col < D)
-            bv = *reinterpret_cast<const float4*>(b_slot(u & 1, col >> 2));
-          S[c + j] = fmaf(g, S[c + j], fmaf(be, bv.x, -gbe * P[j]));
-          S[c + j + 1] = fmaf(g, S[c + j + 1], fmaf(be, bv.y, -gbe * P[j + 1]));
-          S[c + j + 2] = fmaf(g, S[c + j + 2], fmaf(be, bv.z, -gbe * P[j + 2]));
-          S[c + j + 3] = fmaf(g, S[c + j + 3], fmaf(be, bv.w, -gbe * P[j + 3]));
+          for (int j = 0; j < 16; ++j) S[c + j] = fmaf(-gbe, P[j], S[c + j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            const int col = c0 + c + j;
+            float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (use_b && row_ok && col < D)
+              bv = *reinterpret_cast<const float4*>(b_slot(u & 1, col >> 2));
+            S[c + j] = fmaf(g, S[c + j], fmaf(be, bv.x, -gbe * P[j]));
+            S[c + j + 1] = fmaf(g, S[c + j + 1], fmaf(be, bv.y, -gbe * P[j + 1]));
+            S[c + j + 2] = fmaf(g, S[c + j + 2], fmaf(be, bv.z, -gbe * P[j + 2]));
+            S[c + j + 3] = fmaf(g, S[c + j + 3], fmaf(be, bv.w, -gbe * P[j + 3]));
+          }
         }
       }
       write_s_tile();

@@ -55,7 +55,9 @@ struct Handoff {
   int count;        // CTAs in this role
   // outputs in publish order: the chain appends item t*B*H + bh (+1) at ready_items[ready_tail++]
   // as soon as S_t is visible, and output CTAs take queue positions from next_item, so an output
-  // CTA only waits when no published state is left anywhere (not on one lagging head)
+  // CTA only waits when no published state is left anywhere (not on one lagging head). A fixed
+  // frame-major order, which would let an output CTA load its Q tiles before the chain reaches
+  // its frame, measured slower on the 480p and 720p clips.
   int* ready_items = nullptr;  // [B*H*T], 0 = not yet written
   int* ready_tail = nullptr;
 };

@@ -23,12 +23,17 @@ namespace gdn {
 
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-// Epilogue warp groups of the output role (see output_kernel.cuh). One group: with four the
-// 720p clip ran 16 % slower although the standalone output kernel gains from them.
+// Epilogue warp groups of the output role (see output_kernel.cuh). DP = 128: one group (with
+// four the 720p clip ran 16 % slower although the standalone output kernel gains from them).
+// DP = 64: two, so that the role's read-out keeps pace with the chain's short frame steps.
 #ifndef GDN_FUSED_OUT_GROUPS
 #define GDN_FUSED_OUT_GROUPS 1
 #endif
-constexpr int kFusedOutGroups = GDN_FUSED_OUT_GROUPS;
+#ifndef GDN_FUSED_OUT_GROUPS_64
+#define GDN_FUSED_OUT_GROUPS_64 2
+#endif
+template <int DP>
+constexpr int kFusedOutGroups = DP == 64 ? GDN_FUSED_OUT_GROUPS_64 : GDN_FUSED_OUT_GROUPS;
 
 // Threads per token row in the RoPE transform of the statistics and output roles (one 64-dim box
 // each at DP = 128). Three shares per row (12 transform warps, which the 19-warp CTA also fits)
@@ -41,9 +46,9 @@ template <int DP>
 struct FusedLayout {
   static constexpr int kThreads = ChainLayout<DP>::kThreads;
   static_assert(kThreads >= StatsLayout<DP, false, DP == 128>::kThreads &&
-                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, DP == 128>::kThreads &&
+                    kThreads >= OutputLayout<DP, false, kFusedOutGroups<DP>, DP == 128>::kThreads &&
                     kThreads >= StatsLayout<DP, false, false, true, kFusedRopeParts<DP>>::kThreads &&
-                    kThreads >= OutputLayout<DP, false, kFusedOutGroups, false, true,
+                    kThreads >= OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
                                              kFusedRopeParts<DP>>::kThreads,
                 "the chain role's CTA size must cover the other roles' warps");
   // the statistics role's publisher is the CTA's last warp (warp 18), past its transform warps
@@ -52,9 +57,9 @@ struct FusedLayout {
                     6 + StatsLayout<DP, false, false, true, kFusedRopeParts<DP>>::kTransformThreads /
                             32 <= 18,
                 "statistics publisher warp");
-  static_assert(2 + 4 * kFusedOutGroups + OutputLayout<DP, false, kFusedOutGroups, DP == 128>::kXfWarps <= 18 &&
-                    2 + 4 * kFusedOutGroups +
-                            OutputLayout<DP, false, kFusedOutGroups, false, true,
+  static_assert(2 + 4 * kFusedOutGroups<DP> + OutputLayout<DP, false, kFusedOutGroups<DP>, DP == 128>::kXfWarps <= 18 &&
+                    2 + 4 * kFusedOutGroups<DP> +
+                            OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
                                          kFusedRopeParts<DP>>::kXfWarps <= 18,
                 "output publisher warp");
   static constexpr int kSmemBytes =
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
     stats_body<DP, false, true, true, kF8, kRope, kFusedRopeParts<DP>>(&tm_k, &tm_v, A_ring,
                                                                        B_ring, p, h_stats, smem);
   } else {
-    output_body<DP, false, true, kFusedOutGroups, kF8, kRope, kFusedRopeParts<DP>>(
+    output_body<DP, false, true, kFusedOutGroups<DP>, kF8, kRope, kFusedRopeParts<DP>>(
         &tm_q, &tm_q, S_ring, &tm_o, p, 1, h_out, smem);
   }
 }

@@ -55,6 +55,9 @@ struct OutputLayout {
   static constexpr int kBoxes = DP / 64;
   static constexpr int kQBytes = kBoxes * kBoxBytes;   // 128 tokens x DP bf16
   static constexpr int kSBufBytes = DP * DP * 2;       // DP/64 blocks of DP rows x 128 B
+  // state buffers: items in flight past the state load (the fused role waits on the chain, so
+  // more of them hide its hand-off latency; DP = 128 has no shared memory left for more)
+  static constexpr int kSBufs = (DP == 128) ? 2 : 4;
   static constexpr int kStages = (DP == 128) ? 3 : 8;
   static constexpr int kThreads = (2 + kEpiWarps + (kTransform ? kXfWarps : 0)) * 32;
   static constexpr int kQLoadBytes = kF8 ? kQBytes / 2 : kQBytes;  // TMA bytes per Q tile
@@ -62,9 +65,9 @@ struct OutputLayout {
   static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes =
-      2 * kSBufBytes + kStages * kQBytes + 2 * kOBytes + kBarrierBytes + 1024;
+      kSBufs * kSBufBytes + kStages * kQBytes + 2 * kOBytes + kBarrierBytes + 1024;
   // barriers, item ring, TMEM slot and the fused publisher's ring within kBarrierBytes
-  static_assert(8 * (3 * kStages + 4 + 4 + 8 + 1) + 32 + 8 + 8 * 16 + 32 <= kBarrierBytes,
+  static_assert(8 * (3 * kStages + 2 * kSBufs + 4 + 8 + 1) + 32 + 8 + 8 * 16 + 32 <= kBarrierBytes,
                 "barriers");
 };
 
@@ -130,15 +133,15 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
                                             uint8_t* smem, __nv_bfloat16* out = nullptr) {
   using L = OutputLayout<DP, kLA, kG, kF8, kRope, kRopeParts>;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
-  uint8_t* s_buf = smem;                          // 2 state buffers
-  uint8_t* q_ring = smem + 2 * L::kSBufBytes;     // kStages Q tiles
+  uint8_t* s_buf = smem;                                  // kSBufs state buffers
+  uint8_t* q_ring = smem + L::kSBufs * L::kSBufBytes;     // kStages Q tiles
   uint8_t* o_stage = q_ring + L::kStages * L::kQBytes;  // 2 output staging tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(o_stage + 2 * L::kOBytes);
   uint64_t* ready = full + L::kStages;
   uint64_t* empty = ready + L::kStages;
   uint64_t* s_full = empty + L::kStages;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* acc_full = s_empty + 2;
+  uint64_t* s_empty = s_full + L::kSBufs;
+  uint64_t* acc_full = s_empty + L::kSBufs;
   uint64_t* acc_empty = acc_full + 2;
   ItemRing ring{reinterpret_cast<int*>(acc_empty + 2 + 9), acc_empty + 2};  // fused only
   uint64_t* mma_drain = acc_empty + 2 + 8;  // all of this CTA's MMAs are complete
@@ -177,9 +180,11 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       mbar_init(&ready[s], 32 * L::kXfWarps);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < L::kSBufs; ++a) {
       mbar_init(&s_full[a], 1);
       mbar_init(&s_empty[a], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], kEpiThreads);
     }
@@ -208,9 +213,36 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_state = policy_evict_last();
       StageFills<L::kStages> fills;
-      StageFills<2> s_fills;
+      StageFills<L::kSBufs> s_fills;
       int stage = 0;
       uint32_t phase = 0;
+      // Q tile `tile` of item `it` into the next stage; false if the wait for the stage ran out
+      auto load_q = [&](const OutputItem& it, int tile) -> bool {
+        if (!mbar_wait(&empty[stage], phase ^ 1)) return false;
+        mbar_arrive_expect_tx(&full[stage], L::kQLoadBytes);
+        if constexpr (kLA) {
+          // 128 flattened token rows (they may run into the next frame of the block)
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb)
+            tma_load_3d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
+                        kb * 64, it.h, it.row0 + tile * kRowsPerTile, pol_stream);
+        } else if constexpr (kF8) {
+          // one 128-byte-wide e4m3 box, into the stage's second bf16 box
+          tma_load_4d(q_ring + stage * L::kQBytes + kBoxBytes, tm_q, &full[stage], 0, it.h,
+                      tile * kRowsPerTile, it.bt, pol_stream);
+        } else {
+#pragma unroll
+          for (int kb = 0; kb < L::kBoxes; ++kb)
+            tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
+                        kb * 64, it.h, tile * kRowsPerTile, it.bt, pol_stream);
+        }
+        fills.filled(stage, phase);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        return true;
+      };
       for (int li = 0; !*abort_flag; ++li) {
         const long item = producer_item(li);
         if (item < 0) break;
@@ -223,8 +255,9 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           const int n_blocks = (p.T + F - 1) / F;
           srow = it.bh * n_blocks + it.t / F;
         }
-        const int sb = li & 1;
-        if (!mbar_wait(&s_empty[sb], ((li >> 1) & 1) ^ 1)) {
+        const int sb = li % L::kSBufs;
+        const uint32_t sph = (li / L::kSBufs) & 1;
+        if (!mbar_wait(&s_empty[sb], sph ^ 1)) {
           give_up(hf, abort_flag);
           break;
         }
@@ -245,34 +278,12 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           bulk_load(s_buf + sb * L::kSBufBytes, S_src + static_cast<long>(srow) * DP * DP,
                     L::kSBufBytes, &s_full[sb], pol_state);
         }
-        s_fills.filled(sb, (li >> 1) & 1);
-        for (int tile = 0; tile < it.n_tiles; ++tile) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            give_up(hf, abort_flag);
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], L::kQLoadBytes);
-          if constexpr (kLA) {
-            // 128 flattened token rows (they may run into the next frame of the block)
-#pragma unroll
-            for (int kb = 0; kb < L::kBoxes; ++kb)
-              tma_load_3d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
-                          kb * 64, it.h, it.row0 + tile * kRowsPerTile, pol_stream);
-          } else if constexpr (kF8) {
-            // one 128-byte-wide e4m3 box, into the stage's second bf16 box
-            tma_load_4d(q_ring + stage * L::kQBytes + kBoxBytes, tm_q, &full[stage], 0, it.h,
-                        tile * kRowsPerTile, it.bt, pol_stream);
-          } else {
-#pragma unroll
-            for (int kb = 0; kb < L::kBoxes; ++kb)
-              tma_load_4d(q_ring + stage * L::kQBytes + kb * kBoxBytes, tm_q, &full[stage],
-                          kb * 64, it.h, tile * kRowsPerTile, it.bt, pol_stream);
-          }
-          fills.filled(stage, phase);
-          if (++stage == L::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
+        s_fills.filled(sb, sph);
+        bool ok = true;
+        for (int tile = 0; ok && tile < it.n_tiles; ++tile) ok = load_q(it, tile);
+        if (!ok) {
+          give_up(hf, abort_flag);
+          break;
         }
       }
       // this thread's copies have landed, whatever the exit path
@@ -304,8 +315,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           if (ok && !hand_off(li, -2)) ok = false;
         break;
       }
-      const int sb = li & 1;
-      if (!mbar_wait(&s_full[sb], (li >> 1) & 1)) {
+      const int sb = li % L::kSBufs;
+      if (!mbar_wait(&s_full[sb], (li / L::kSBufs) & 1)) {
         ok = false;
         break;
       }
