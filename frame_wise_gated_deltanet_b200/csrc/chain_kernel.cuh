@@ -380,51 +380,35 @@ __device__ __forceinline__ void chain_body(const CUtensorMap* tm_a, const float*
       }
       const float g = __shfl_sync(0xffffffffu, g_cur, u & 31);
       const float be = __shfl_sync(0xffffffffu, b_cur, u & 31);
-      // S_t = gamma_t S_{t-1} + beta_t B_t - gamma_t beta_t S_{t-1} A_t. DP = 64: the part that
-      // does not need the product is formed while the MMA runs, so that one FMA per element
-      // follows the wait (the chain's step bounds short clips); DP = 128 keeps the B_t reads
-      // next to their use, which the fused kernel's register budget needs.
-      constexpr bool kEarlyB = DP == 64;
-      if constexpr (kEarlyB) {
-        cp_async_wait<1>();  // this thread's copy of B_t (B_{t+1} may still be in flight)
+      // S_t = gamma_t S_{t-1} + beta_t B_t - gamma_t beta_t S_{t-1} A_t: the part that does not
+      // need the product is formed while the MMA runs, so that one FMA per element follows the
+      // wait (the step is the chain's latency)
+      cp_async_wait<1>();  // this thread's copy of B_t (B_{t+1} may still be in flight)
 #pragma unroll
-        for (int j = 0; j < L::kCols; j += 4) {
-          float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (use_b && row_ok && c0 + j < D)
-            bv = *reinterpret_cast<const float4*>(b_slot(u & 1, (c0 + j) >> 2));
-          S[j] = fmaf(g, S[j], be * bv.x);
-          S[j + 1] = fmaf(g, S[j + 1], be * bv.y);
-          S[j + 2] = fmaf(g, S[j + 2], be * bv.z);
-          S[j + 3] = fmaf(g, S[j + 3], be * bv.w);
-        }
+      for (int j = 0; j < L::kCols; j += 4) {
+        float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (use_b && row_ok && c0 + j < D)
+          bv = *reinterpret_cast<const float4*>(b_slot(u & 1, (c0 + j) >> 2));
+        S[j] = fmaf(g, S[j], be * bv.x);
+        S[j + 1] = fmaf(g, S[j + 1], be * bv.y);
+        S[j + 2] = fmaf(g, S[j + 2], be * bv.z);
+        S[j + 3] = fmaf(g, S[j + 3], be * bv.w);
+        // at most 16 columns of B_t in registers at a time (the reads of the next 16 may not
+        // be hoisted above this point), which the fused kernel's register budget needs
+        if ((j & 15) == 12) asm volatile("" ::: "memory");
       }
       if (!mbar_wait(mma_done, u & 1)) {
         ok = false;
         break;
       }
-      if constexpr (!kEarlyB) cp_async_wait<1>();
       tc_fence_after();
-      const float gbe = g * be;
+      const float ngbe = -g * be;
 #pragma unroll
       for (int c = 0; c < L::kCols; c += 16) {
         float P[16];
         tmem_ld16(taddr + c, P);
-        if constexpr (kEarlyB) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) S[c + j] = fmaf(-gbe, P[j], S[c + j]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            const int col = c0 + c + j;
-            float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (use_b && row_ok && col < D)
-              bv = *reinterpret_cast<const float4*>(b_slot(u & 1, col >> 2));
-            S[c + j] = fmaf(g, S[c + j], fmaf(be, bv.x, -gbe * P[j]));
-            S[c + j + 1] = fmaf(g, S[c + j + 1], fmaf(be, bv.y, -gbe * P[j + 1]));
-            S[c + j + 2] = fmaf(g, S[c + j + 2], fmaf(be, bv.z, -gbe * P[j + 2]));
-            S[c + j + 3] = fmaf(g, S[c + j + 3], fmaf(be, bv.w, -gbe * P[j + 3]));
-          }
-        }
+        for (int j = 0; j < 16; ++j) S[c + j] = fmaf(ngbe, P[j], S[c + j]);
       }
       write_s_tile();
       fence_async_smem();

@@ -35,32 +35,35 @@ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 template <int DP>
 constexpr int kFusedOutGroups = DP == 64 ? GDN_FUSED_OUT_GROUPS_64 : GDN_FUSED_OUT_GROUPS;
 
-// Threads per token row in the RoPE transform of the statistics and output roles (one 64-dim box
-// each at DP = 128). Three shares per row (12 transform warps, which the 19-warp CTA also fits)
-// measured slower at 720p: the rotation adds shared-memory traffic to roles whose tiles already
-// keep shared memory busy, so more threads do not shorten it.
+// Groups of 128 threads in the RoPE transform of the statistics and output roles: three at
+// DP = 128 (12 warps; the 720p clip measured 4.90 ms against 5.25 with two), two at DP = 64
+// (whose output role has two epilogue groups, so 12 transform warps would not fit its 19).
+#ifndef GDN_FUSED_ROPE_GROUPS
+#define GDN_FUSED_ROPE_GROUPS 3
+#endif
 template <int DP>
-constexpr int kFusedRopeParts = 2;
+constexpr int kFusedRopeGroups = DP == 128 ? GDN_FUSED_ROPE_GROUPS : 2;
 
 template <int DP>
 struct FusedLayout {
   static constexpr int kThreads = ChainLayout<DP>::kThreads;
   static_assert(kThreads >= StatsLayout<DP, false, DP == 128>::kThreads &&
                     kThreads >= OutputLayout<DP, false, kFusedOutGroups<DP>, DP == 128>::kThreads &&
-                    kThreads >= StatsLayout<DP, false, false, true, kFusedRopeParts<DP>>::kThreads &&
+                    kThreads >= StatsLayout<DP, false, false, true, kFusedRopeGroups<DP>>::kThreads &&
                     kThreads >= OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
-                                             kFusedRopeParts<DP>>::kThreads,
+                                             kFusedRopeGroups<DP>>::kThreads,
                 "the chain role's CTA size must cover the other roles' warps");
   // the statistics role's publisher is the CTA's last warp (warp 18), past its transform warps
   static_assert(kThreads / 32 - 1 == 18 &&
                     6 + StatsLayout<DP, false, DP == 128>::kTransformThreads / 32 <= 18 &&
-                    6 + StatsLayout<DP, false, false, true, kFusedRopeParts<DP>>::kTransformThreads /
+                    6 + StatsLayout<DP, false, false, true, kFusedRopeGroups<DP>>::kTransformThreads /
                             32 <= 18,
                 "statistics publisher warp");
-  static_assert(2 + 4 * kFusedOutGroups<DP> + OutputLayout<DP, false, kFusedOutGroups<DP>, DP == 128>::kXfWarps <= 18 &&
+  static_assert(2 + 4 * kFusedOutGroups<DP> +
+                        OutputLayout<DP, false, kFusedOutGroups<DP>, DP == 128>::kXfWarps <= 18 &&
                     2 + 4 * kFusedOutGroups<DP> +
                             OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
-                                         kFusedRopeParts<DP>>::kXfWarps <= 18,
+                                         kFusedRopeGroups<DP>>::kXfWarps <= 18,
                 "output publisher warp");
   static constexpr int kSmemBytes =
       cmax(ChainLayout<DP>::kSmemBytes,
@@ -88,10 +91,10 @@ __global__ void __launch_bounds__(FusedLayout<DP>::kThreads, 1)
     chain_body<DP, true>(&tm_a_ring, B_ring, S_ring, gamma, beta, state_in, state_out, p,
                          h_chain, whole, smem);
   } else if (static_cast<int>(blockIdx.x) < h_out.base) {
-    stats_body<DP, false, true, true, kF8, kRope, kFusedRopeParts<DP>>(&tm_k, &tm_v, A_ring,
+    stats_body<DP, false, true, true, kF8, kRope, kFusedRopeGroups<DP>>(&tm_k, &tm_v, A_ring,
                                                                        B_ring, p, h_stats, smem);
   } else {
-    output_body<DP, false, true, kFusedOutGroups<DP>, kF8, kRope, kFusedRopeParts<DP>>(
+    output_body<DP, false, true, kFusedOutGroups<DP>, kF8, kRope, kFusedRopeGroups<DP>>(
         &tm_q, &tm_q, S_ring, &tm_o, p, 1, h_out, smem);
   }
 }

@@ -39,16 +39,16 @@
 
 namespace gdn {
 
-// kRopeParts: threads per Q row in the RoPE transform (each rotates an equal share of the row's
-// 16-byte chunks).
+// kRopeGroups: groups of 128 threads (4 warps) in the RoPE transform of the Q tiles.
 template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false,
-          int kRopeParts = DP / 64>
+          int kRopeGroups = DP / 64>
 struct OutputLayout {
   static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
   static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
   static constexpr bool kTransform = kLA || kF8 || kRope;
-  // transform warps: 4 (one token row each), or for RoPE kRopeParts per row
-  static constexpr int kXfWarps = kRope ? 4 * kRopeParts : 4;
+  // transform warps: 4 (one token row each; fp8: kF8Parts lanes per row), or for RoPE 4 per group
+  static constexpr int kF8Parts = 1;  // fp8: lanes per Q row in the e4m3 -> bf16 conversion
+  static constexpr int kXfWarps = kRope ? 4 * kRopeGroups : (kF8 ? 4 * kF8Parts : 4);
   static constexpr int kEpiWarps = 4 * kG;
   static constexpr int kCols = DP / kG;                // columns per epilogue thread
   static constexpr int kChunk = kCols < 32 ? kCols : 32;
@@ -125,13 +125,13 @@ __device__ __forceinline__ OutputItem output_item(long item, const Problem& p, i
 // the row stores of a block's last, partial tile (a 128-row TMA store would also overwrite the
 // first rows of the next block, which another CTA writes).
 template <int DP, bool kLA, bool kFused, int kG, bool kF8 = false, bool kRope = false,
-          int kRopeParts = DP / 64>
+          int kRopeGroups = DP / 64>
 __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUtensorMap* tm_s,
                                             const __nv_bfloat16* __restrict__ S_src,
                                             const CUtensorMap* tm_o, const Problem& p,
                                             int frames_per_block, const Handoff& hf,
                                             uint8_t* smem, __nv_bfloat16* out = nullptr) {
-  using L = OutputLayout<DP, kLA, kG, kF8, kRope, kRopeParts>;
+  using L = OutputLayout<DP, kLA, kG, kF8, kRope, kRopeGroups>;
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                                  // kSBufs state buffers
   uint8_t* q_ring = smem + L::kSBufs * L::kSBufBytes;     // kStages Q tiles
@@ -477,10 +477,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
     // (the fused kernel's output CTAs have more warps: the rest stay idle)
     if constexpr (kRope) {
       // ---------------------------------------------------------------- RoPE of the Q tiles
-      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // Q row tid % 128, share tid / 128
-      const int row = tid & 127, part = tid >> 7;
-      const int cb = rope_part_begin(part, kRopeParts, DP / 8);
-      const int ce = rope_part_begin(part + 1, kRopeParts, DP / 8);
+      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -493,9 +490,9 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
             ok = false;
             break;
           }
-          const int n = tile * kRowsPerTile + row;
-          if (n < p.N)
-            rope_rotate_row(q_ring + stage * L::kQBytes, row, cb, ce, n, it.t, p.D, p.rope);
+          const int n0 = tile * kRowsPerTile;
+          rope_rotate_tile<DP>(q_ring + stage * L::kQBytes, tid, 32 * L::kXfWarps,
+                               min(kRowsPerTile, p.N - n0), n0, it.t, p.D, p.rope);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {
@@ -507,7 +504,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
       if (!ok) give_up(hf, abort_flag);
     } else if constexpr (kF8) {
       // ---------------------------------------------------------------- e4m3 Q conversion
-      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // the token row it converts
+      const int tid = threadIdx.x - 32 * (2 + L::kEpiWarps);  // row tid / kF8Parts, its part
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -520,7 +517,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
             ok = false;
             break;
           }
-          e4m3_row_to_bf16_tile(q_ring + stage * L::kQBytes, tid);
+          e4m3_row_to_bf16_tile<L::kF8Parts>(q_ring + stage * L::kQBytes, tid / L::kF8Parts,
+                                             tid % L::kF8Parts);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {

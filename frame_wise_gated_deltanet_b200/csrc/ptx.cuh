@@ -403,6 +403,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A * B with e4m3 A and B (kind::f8f6f4), f32 accumulate; K = 32 per instruction.
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier when every previously issued tcgen05.mma of this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -481,21 +492,29 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4& in, uint4& lo, uint
 // An fp8 operand tile converted in place into the bf16 operand layout. The tile holds 128 token
 // rows; the bf16 form is two 128B-swizzled TMA boxes of 64 dims (box0 at `tile`, box1 at
 // tile + 16 KB, row r at r * 128 in each); the fp8 form was TMA-loaded 128B-swizzled into the
-// box1 region (row r: 128 e4m3 values at tile + 16 KB + r * 128). Thread `row` converts its own
-// row: it reads all of fp8 row r before writing box1 row r, which occupies the same bytes.
-__device__ __forceinline__ void e4m3_row_to_bf16_tile(uint8_t* tile, int row) {
+// box1 region (row r: 128 e4m3 values at tile + 16 KB + r * 128). kParts adjacent lanes of one
+// warp convert row `row` together, lane `part` taking fp8 chunks [part, part + 1) * 8 / kParts
+// (16 dims each): every lane of the warp reads its chunks before any lane writes, since box1 row
+// r occupies the bytes of fp8 row r. Every lane of the warp must call it.
+template <int kParts>
+__device__ __forceinline__ void e4m3_row_to_bf16_tile(uint8_t* tile, int row, int part) {
+  static_assert(kParts == 1 || kParts == 2 || kParts == 4, "parts of a row");
+  constexpr int kC = 8 / kParts;
   uint8_t* b0 = tile + row * 128;
   uint8_t* b1 = tile + 16384 + row * 128;
   const uint32_t sw = row & 7;
-  uint4 in[8];
+  uint4 in[kC];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) in[c] = *reinterpret_cast<const uint4*>(b1 + ((c ^ sw) << 4));
+  for (int i = 0; i < kC; ++i)
+    in[i] = *reinterpret_cast<const uint4*>(b1 + (((part * kC + i) ^ sw) << 4));
+  if (kParts > 1) __syncwarp();
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int i = 0; i < kC; ++i) {
     // fp8 chunk c = dims 16c..16c+15 -> bf16 chunks 2c, 2c+1 of the 16 chunks of 8 dims
+    const int c = part * kC + i;
     uint4 lo, hi;
-    e4m3x16_to_bf16(in[c], lo, hi);
-    const int k0 = 2 * c, k1 = 2 * c + 1;          // 8-dim chunk index over 128 dims
+    e4m3x16_to_bf16(in[i], lo, hi);
+    const int k0 = 2 * c, k1 = 2 * c + 1;  // 8-dim chunk index over 128 dims
     uint8_t* d0 = (k0 < 8 ? b0 : b1) + (((k0 & 7) ^ sw) << 4);
     uint8_t* d1 = (k1 < 8 ? b0 : b1) + (((k1 & 7) ^ sw) << 4);
     *reinterpret_cast<uint4*>(d0) = lo;
@@ -597,6 +616,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
   return (1u << 4)                                    // D format f32
          | (1u << 7)                                  // A bf16
          | (1u << 10)                                 // B bf16
+         | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::f8f6f4 with e4m3 A and B (format code 0 for both) and f32 D.
+// MN-major operands are valid for e4m3 (not for the 6- and 4-bit formats).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn_major,
+                                                  bool b_mn_major) {
+  return (1u << 4)                                    // D format f32
+         | (0u << 7)                                  // A e4m3
+         | (0u << 10)                                 // B e4m3
          | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }

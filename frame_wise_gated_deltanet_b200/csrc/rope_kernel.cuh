@@ -12,7 +12,7 @@
 // table, rotates in f32 and rounds to bf16. It is HBM-bound: every element is read and written
 // once. Each thread reads and writes the same 16 bytes, so x and y may be the same memory.
 //
-// Fused prologue (gdn_frame_forward_rope): the same table, and rope_rotate_row applied by
+// Fused prologue (gdn_frame_forward_rope): the same table, and rope_rotate_tile applied by
 // transform warps to the K tiles of the statistics kernel and the Q tiles of the output kernel in
 // shared memory, so q and k are rotated on their way to the tensor cores and never rewritten.
 #pragma once
@@ -124,51 +124,78 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
 }
 
 // The same rotation applied in shared memory by the forward's statistics (K) and output (Q)
-// kernels to one token row of a bf16 operand tile just loaded by TMA: chunks [c_begin, c_end) of
-// the row's 16-byte chunks of 8 dims (chunk c in box c / 8; each box is 128 rows of 128 B,
-// 128B-swizzled, kBoxBytes apart) of row `row`, which holds token n of frame t. Dims at or past D
-// are left alone (TMA zero fill). The arithmetic and the rounding are those of gdn_rope_kernel, so
-// the operand equals the standalone pass's output. The (cos, sin) of up to 4 chunks are loaded
-// before those chunks' shared-memory reads and writes, so the table loads overlap.
-__device__ __forceinline__ void rope_rotate_row(uint8_t* tile, int row, int c_begin, int c_end,
-                                                int n, int t, int D, const RopeArgs& ra) {
-  const int rg = n / ra.grid_w;
-  const int cg = n - rg * ra.grid_w;
-  const int tb = t * ra.pt;                              // index of time pair 0
-  const int rb = ra.off_h + rg * ra.ph - ra.pt;          // + j: row pair j - pt
-  const int cb = ra.off_w + cg * ra.ph - ra.pt - ra.ph;  // + j: column pair j - pt - ph
-  const uint32_t sw = row & 7;
-  c_end = min(c_end, D / 8);
-  for (int c0 = c_begin; c0 < c_end; c0 += 4) {
-    float2 cs[16];
+// kernels to a bf16 operand tile just loaded by TMA: `rows` token rows (token n0 + r in row r, all
+// of frame t), each DP/8 16-byte chunks of 8 dims (chunk c in box c / 8; a box is 128 rows of
+// 128 B, 128B-swizzled, kBoxBytes apart). Dims at or past D are left alone (TMA zero fill).
+// Thread tid of nthreads owns chunk c = tid % (DP/8) of rows tid / (DP/8), + nthreads / (DP/8),
+// ...: its 4 pairs, hence their axes and the time pairs' (cos, sin), are fixed for the tile; a
+// warp covers whole rows, so its shared-memory accesses take the minimum number of wavefronts
+// and its table reads for one token fall in a few adjacent sectors. The arithmetic and the
+// rounding are those of gdn_rope_kernel.
+template <int DP>
+__device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nthreads, int rows,
+                                                 int n0, int t, int D, const RopeArgs& ra) {
+  constexpr int kChunks = DP / 8;
+  const int c = tid % kChunks;
+  if (c * 8 >= D) return;
+  const int r_step = nthreads / kChunks;
+  int r = tid / kChunks;
+  if (r >= rows) return;
+  // pair p of the chunk: (cos, sin) if on the time axis, else its table offset without the
+  // token's row (rg * ph) or column (cg * ph) term
+  float2 ct[4];
+  int off[4], axis[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int j = c0 * 4 + i;  // pair index over the head dimension
-      const int e = j < ra.pt ? tb + j : (j < ra.pt + ra.ph ? rb + j : cb + j);
-      cs[i] = c0 + i / 4 < c_end ? __ldg(ra.tab + e) : make_float2(1.f, 0.f);
-    }
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int c = c0 + cc;
-      if (c >= c_end) break;
-      uint4* ptr = reinterpret_cast<uint4*>(tile + (c >> 3) * kBoxBytes + row * 128 +
-                                            (((c & 7) ^ sw) << 4));
-      uint4 raw = *ptr;
-      __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 w = cs[cc * 4 + i];
-        const float2 v = __bfloat1622float2(p2[i]);
-        p2[i] = __floats2bfloat162_rn(v.x * w.x - v.y * w.y, v.x * w.y + v.y * w.x);
-      }
-      *ptr = raw;
-    }
+  for (int p = 0; p < 4; ++p) {
+    const int j = 4 * c + p;
+    axis[p] = j < ra.pt ? 0 : (j < ra.pt + ra.ph ? 1 : 2);
+    off[p] = axis[p] == 1 ? ra.off_h + j - ra.pt : ra.off_w + j - ra.pt - ra.ph;
+    ct[p] = axis[p] == 0 ? __ldg(ra.tab + t * ra.pt + j) : make_float2(1.f, 0.f);
   }
-}
-
-// Chunks [begin, end) of part `part` of `parts` equal shares of a row's DP / 8 chunks.
-__device__ __forceinline__ int rope_part_begin(int part, int parts, int chunks) {
-  return part * chunks / parts;
+  uint8_t* const box = tile + (c >> 3) * kBoxBytes;
+  int n = n0 + r;
+  int rg = n / ra.grid_w;
+  int cg = n - rg * ra.grid_w;
+  const int drg = r_step / ra.grid_w, dcg = r_step - drg * ra.grid_w;
+  auto advance = [&](int& g_r, int& g_c) {
+    g_c += dcg;
+    g_r += drg;
+    if (g_c >= ra.grid_w) {
+      g_c -= ra.grid_w;
+      ++g_r;
+    }
+  };
+  auto rotate = [&](int row, const float2* cs) {
+    // 128B swizzle: the chunk's 16-byte slot in its 128-byte row is c % 8 XOR row % 8
+    uint4* ptr = reinterpret_cast<uint4*>(box + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+    uint4 raw = *ptr;
+    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 v = __bfloat1622float2(p2[p]);
+      p2[p] = __floats2bfloat162_rn(v.x * cs[p].x - v.y * cs[p].y, v.x * cs[p].y + v.y * cs[p].x);
+    }
+    *ptr = raw;
+  };
+  // two rows at a time: both rows' table reads are in flight together
+  for (; r < rows; r += 2 * r_step) {
+    const bool second = r + r_step < rows;
+    int rg2 = rg, cg2 = cg;
+    advance(rg2, cg2);
+    float2 cs[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      cs[p] = axis[p] == 0 ? ct[p] : __ldg(ra.tab + off[p] + (axis[p] == 1 ? rg : cg) * ra.ph);
+      cs[4 + p] = axis[p] == 0 || !second
+                      ? ct[p]
+                      : __ldg(ra.tab + off[p] + (axis[p] == 1 ? rg2 : cg2) * ra.ph);
+    }
+    rotate(r, cs);
+    if (second) rotate(r + r_step, cs + 4);
+    rg = rg2;
+    cg = cg2;
+    advance(rg, cg);
+  }
 }
 
 }  // namespace gdn

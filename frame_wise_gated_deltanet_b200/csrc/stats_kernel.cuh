@@ -33,23 +33,24 @@
 
 namespace gdn {
 
-// kRopeParts: threads per K row in the RoPE transform (each rotates an equal share of the row's
-// 16-byte chunks).
-template <int DP, bool kLA, bool kF8 = false, bool kRope = false, int kRopeParts = DP / 64>
+// kRopeGroups: groups of 128 threads (4 warps) in the RoPE transform of the K tiles.
+template <int DP, bool kLA, bool kF8 = false, bool kRope = false, int kRopeGroups = DP / 64>
 struct StatsLayout {
   static_assert(!kF8 || (DP == 128 && !kLA), "fp8 inputs: DP = 128, GDN only");
   static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
-  static constexpr bool kTransform = kLA || kF8 || kRope;
-  static constexpr int kBoxes = DP / 64;                // 64-dim boxes per operand tile
-  static constexpr int kOpBytes = kBoxes * kBoxBytes;   // 128 tokens x DP dims, bf16
-  static constexpr int kStageBytes = 2 * kOpBytes;      // K tile + V tile
-  static constexpr int kStages = (DP == 128) ? 3 : 6;
+  // fp8: the tensor core reads the e4m3 tiles as they land (kind::f8f6f4), no transform
+  static constexpr bool kTransform = kLA || kRope;
+  static constexpr int kBoxes = DP / 64;  // 64-dim boxes per bf16 operand tile
+  // 128 tokens x DP dims: bf16 in kBoxes boxes, e4m3 in one 128-byte-wide box
+  static constexpr int kOpBytes = kF8 ? kBoxBytes : kBoxes * kBoxBytes;
+  static constexpr int kStageBytes = 2 * kOpBytes;  // K tile + V tile
+  static constexpr int kStages = (DP == 128 && !kF8) ? 3 : 6;
   static constexpr int kAccCols = kLA ? 128 : (DP == 128 ? 256 : 64);
   static constexpr int kTmemCols = 2 * kAccCols;
-  // fp8: one K or V row per thread; RoPE: a share of one K row per thread
-  static constexpr int kTransformThreads = kF8 ? 256 : (kRope ? 128 * kRopeParts : 128);
+  // LA: one K row per thread; RoPE: kRopeGroups groups of 128 threads
+  static constexpr int kTransformThreads = kRope ? 128 * kRopeGroups : 128;
   static constexpr int kThreads = 192 + (kTransform ? kTransformThreads : 0);
-  static constexpr int kLoadBytes = kF8 ? kStageBytes / 2 : kStageBytes;  // TMA bytes per stage
+  static constexpr int kLoadBytes = kStageBytes;  // TMA bytes per stage
   static constexpr int kBarrierBytes = 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
   // barriers, item ring, TMEM slot and the fused publisher's ring within kBarrierBytes
@@ -96,12 +97,12 @@ __device__ __forceinline__ StatsItem stats_item(long item, const Problem& p, con
 // kB4: B_t stored in the four-key interleaved layout of b4_index (the chain's input) instead of
 // row-major (the public gdn_frame_stats layout and the block-causal path).
 template <int DP, bool kLA, bool kFused, bool kB4, bool kF8 = false, bool kRope = false,
-          int kRopeParts = DP / 64>
+          int kRopeGroups = DP / 64>
 __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                            __nv_bfloat16* __restrict__ A_ws,
                                            float* __restrict__ B_ws, const Problem& p,
                                            const Handoff& hf, uint8_t* smem, int fpb = 1) {
-  using L = StatsLayout<DP, kLA, kF8, kRope, kRopeParts>;
+  using L = StatsLayout<DP, kLA, kF8, kRope, kRopeGroups>;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
   uint64_t* ready = full + L::kStages;   // LA / fp8: transformed stage
   uint64_t* empty = ready + L::kStages;
@@ -204,11 +205,10 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
                           row, pol);
             }
           } else if constexpr (kF8) {
-            // one 128-byte-wide e4m3 box per operand, into its second bf16 box
-            tma_load_4d(st + kBoxBytes, tm_k, &full[stage], 0, it.h, tile * kRowsPerTile, bt,
+            // one 128-byte-wide e4m3 box per operand
+            tma_load_4d(st, tm_k, &full[stage], 0, it.h, tile * kRowsPerTile, bt, pol);
+            tma_load_4d(st + L::kOpBytes, tm_v, &full[stage], 0, it.h, tile * kRowsPerTile, bt,
                         pol);
-            tma_load_4d(st + L::kOpBytes + kBoxBytes, tm_v, &full[stage], 0, it.h,
-                        tile * kRowsPerTile, bt, pol);
           } else {
 #pragma unroll
             for (int j = 0; j < L::kBoxes; ++j) {
@@ -229,9 +229,10 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = kLA ? idesc_bf16(128, 128, true, true)
-                                   : (DP == 128 ? idesc_bf16(128, 128, true, true)
-                                                : idesc_bf16(128, 64, true, true));
+    constexpr uint32_t idesc = kF8 ? idesc_e4m3(128, 128, true, true)
+                               : kLA ? idesc_bf16(128, 128, true, true)
+                                     : (DP == 128 ? idesc_bf16(128, 128, true, true)
+                                                  : idesc_bf16(128, 64, true, true));
     int stage = 0;
     uint32_t phase = 0;
     for (int li = 0;; ++li) {
@@ -259,25 +260,38 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
         tc_fence_after();
         if (elect_one()) {
           const uint32_t base = smem_u32(smem + stage * L::kStageBytes);
+          if constexpr (kF8) {
+            // e4m3 K and V tiles, both MN-major (128 dims = one 128-byte swizzle atom per token
+            // row): 32 token rows (4 KB) per instruction, 8-row groups 1024 B apart
 #pragma unroll
-          for (int ks = 0; ks < kRowsPerTile / 16; ++ks) {
-            const uint32_t accum = (tile | ks) != 0;
-            const uint32_t koff = ks * 16 * 128;  // 16 token rows of 128 B
-            if constexpr (kLA) {
-              const uint64_t dv = smem_desc(base + L::kOpBytes + koff, kBoxBytes, 1024);
-              const uint64_t dk = smem_desc(base + koff, kBoxBytes, 1024);
-              mma_bf16(d, dv, dk, idesc, accum);
-            } else if constexpr (DP == 128) {
-              const uint64_t dk = smem_desc(base + koff, kBoxBytes, 1024);
-              const uint64_t dv = smem_desc(base + L::kOpBytes + koff, kBoxBytes, 1024);
-              mma_bf16(d, dk, dk, idesc, accum);        // A_t = K^T K
-              mma_bf16(d + 128, dv, dk, idesc, accum);  // B_t = V^T K
-            } else {
-              // [K | V] stacked along M (K box then V box, kOpBytes apart) times K:
-              // TMEM rows 0..63 = K^T K, rows 64..127 = V^T K.
-              const uint64_t da = smem_desc(base + koff, L::kOpBytes, 1024);
-              const uint64_t db = smem_desc(base + koff, kBoxBytes, 1024);
-              mma_bf16(d, da, db, idesc, accum);
+            for (int ks = 0; ks < kRowsPerTile / 32; ++ks) {
+              const uint32_t accum = (tile | ks) != 0;
+              const uint64_t dk = smem_desc(base + ks * 32 * 128, kBoxBytes, 1024);
+              const uint64_t dv = smem_desc(base + L::kOpBytes + ks * 32 * 128, kBoxBytes, 1024);
+              mma_e4m3(d, dk, dk, idesc, accum);        // A_t = K^T K
+              mma_e4m3(d + 128, dv, dk, idesc, accum);  // B_t = V^T K
+            }
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < kRowsPerTile / 16; ++ks) {
+              const uint32_t accum = (tile | ks) != 0;
+              const uint32_t koff = ks * 16 * 128;  // 16 token rows of 128 B
+              if constexpr (kLA) {
+                const uint64_t dv = smem_desc(base + L::kOpBytes + koff, kBoxBytes, 1024);
+                const uint64_t dk = smem_desc(base + koff, kBoxBytes, 1024);
+                mma_bf16(d, dv, dk, idesc, accum);
+              } else if constexpr (DP == 128) {
+                const uint64_t dk = smem_desc(base + koff, kBoxBytes, 1024);
+                const uint64_t dv = smem_desc(base + L::kOpBytes + koff, kBoxBytes, 1024);
+                mma_bf16(d, dk, dk, idesc, accum);        // A_t = K^T K
+                mma_bf16(d + 128, dv, dk, idesc, accum);  // B_t = V^T K
+              } else {
+                // [K | V] stacked along M (K box then V box, kOpBytes apart) times K:
+                // TMEM rows 0..63 = K^T K, rows 64..127 = V^T K.
+                const uint64_t da = smem_desc(base + koff, L::kOpBytes, 1024);
+                const uint64_t db = smem_desc(base + koff, kBoxBytes, 1024);
+                mma_bf16(d, da, db, idesc, accum);
+              }
             }
           }
           mma_commit(&empty[stage]);
@@ -460,10 +474,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     // (the fused kernel's stats CTAs have more warps: the rest stay idle)
     if constexpr (kRope) {
       // ---------------------------------------------------------------- RoPE of the K tiles
-      const int tid = threadIdx.x - 192;  // K row tid % 128, share tid / 128 of its chunks
-      const int row = tid & 127, part = tid >> 7;
-      const int cb = rope_part_begin(part, kRopeParts, DP / 8);
-      const int ce = rope_part_begin(part + 1, kRopeParts, DP / 8);
+      const int tid = threadIdx.x - 192;
       int stage = 0;
       uint32_t phase = 0;
       for (int li = 0;; ++li) {
@@ -476,36 +487,9 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
             ok = false;
             break;
           }
-          const int n = tile * kRowsPerTile + row;
-          if (n < p.N) rope_rotate_row(smem + stage * L::kStageBytes, row, cb, ce, n, t, p.D, p.rope);
-          fence_async_smem();
-          mbar_arrive(&ready[stage]);
-          if (++stage == L::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) {
-          give_up(hf, abort_flag);
-          break;
-        }
-      }
-    } else if constexpr (kF8) {
-      // ---------------------------------------------------------------- fp8 conversion warps
-      const int tid = threadIdx.x - 192;  // 0..255: K row tid, or V row tid - 128
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int li = 0;; ++li) {
-        const long item = consumer_item(li);
-        if (item < 0) break;
-        bool ok = true;
-        for (int tile = 0; tile < n_tiles; ++tile) {
-          if (!mbar_wait(&full[stage], phase)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + stage * L::kStageBytes;
-          e4m3_row_to_bf16_tile(st + (tid >> 7) * L::kOpBytes, tid & 127);
+          const int n0 = tile * kRowsPerTile;
+          rope_rotate_tile<DP>(smem + stage * L::kStageBytes, tid, L::kTransformThreads,
+                               min(kRowsPerTile, p.N - n0), n0, t, p.D, p.rope);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {
