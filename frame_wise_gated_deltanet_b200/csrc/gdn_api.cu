@@ -424,21 +424,28 @@ int env_int(const char* name, int dflt, int lo, int hi) {
   const int v = atoi(s);
   return v < lo ? lo : (v > hi ? hi : v);
 }
-int fused_ring() {
-  static const int r = env_int("GDN_FUSED_RING", 8, 4, 64);
-  return r;
+// A_t / B_t ring slots per head of the fused forward: how many frames the statistics may run
+// ahead of the chain. 16 when sixteen slots of every head (bf16 A_t and f32 B_t, 6 D^2 bytes a
+// slot) take at most 16 MB, so that they stay in L2 beside the streams; else 8. Measured: the
+// 480p clip (12.6 MB) 5-8 % faster with 16, the 720p clip (31 MB) 10 % slower.
+int fused_ring(long bh, int D) {
+  static const int r = env_int("GDN_FUSED_RING", 0, 0, 64);
+  if (r > 0) return r < 4 ? 4 : r;
+  return 16.0 * bh * D * D * 6 <= 16e6 ? 16 : 8;
 }
 int fused_sring() {
   static const int r = env_int("GDN_FUSED_SRING", 16, 8, 64);
   return r;
 }
 // Share of the worker SMs (those left after the chains) that run the statistics role, in %:
-// by default about the ratio of the two roles' per-frame times, 54 for bf16 inputs; 40 for e4m3
-// inputs, whose statistics read half the bytes of bf16 on the tensor core's f8f6f4 path while
-// the outputs still write bf16 (measured: 2.60 ms on the 720p clip against 3.03 at 54).
-int fused_stats_pct(bool f8) {
+// by default about the ratio of the two roles' per-frame times, 54 for bf16 inputs at DP = 128;
+// 40 for e4m3 inputs, whose statistics read half the bytes of bf16 on the tensor core's f8f6f4
+// path while the outputs still write bf16 (measured: 2.60 ms on the 720p clip against 3.03 at
+// 54); 40 at DP = 64, where the chain's short frame steps leave the outputs behind (the 480p
+// clip 6 % faster than at 54).
+int fused_stats_pct(bool f8, int DP) {
   static const int p = env_int("GDN_FUSED_STATS_PCT", 0, 0, 80);
-  return p > 0 ? p : (f8 ? 40 : 54);
+  return p > 0 ? p : ((f8 || DP == 64) ? 40 : 54);
 }
 
 struct FusedWs {
@@ -454,7 +461,7 @@ struct FusedWs {
 // frame keeps its own slot, and the A, B, S blocks are laid out exactly like the three-kernel
 // workspace (row (b*H + h)*T + t): gdn_frame_forward_train keeps them for the backward.
 size_t fused_ws_bytes(long bh, long T, int D, int R = 0, int Rs = 0) {
-  const int kRing = R > 0 ? R : fused_ring();
+  const int kRing = R > 0 ? R : fused_ring(bh, D);
   const size_t m = size_t(D) * D * bh * kRing;
   const size_t dp = padded_dim(D), ms = dp * dp * bh * (Rs > 0 ? Rs : fused_sring());
   const size_t flags = sizeof(int) * (3 * bh * T + bh + 4);
@@ -462,7 +469,7 @@ size_t fused_ws_bytes(long bh, long T, int D, int R = 0, int Rs = 0) {
 }
 
 FusedWs carve_fused(void* base, long bh, long T, int D, int R = 0, int Rs = 0) {
-  const int kRing = R > 0 ? R : fused_ring();
+  const int kRing = R > 0 ? R : fused_ring(bh, D);
   const size_t m = size_t(D) * D * bh * kRing;
   const size_t dp = padded_dim(D), ms = dp * dp * bh * (Rs > 0 ? Rs : fused_sring());
   uint8_t* p = static_cast<uint8_t*>(base);
@@ -500,7 +507,7 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   using L = gdn::FusedLayout<DP>;
   const int sms = g_dev[dev].sms;
   const int bh = p.B * p.H;
-  const int kRing = kept ? p.T : fused_ring();
+  const int kRing = kept ? p.T : fused_ring(bh, p.D);
   const int kSRing = kept ? p.T : fused_sring();
   void* base = kept;
   if (!kept)
@@ -516,7 +523,7 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   if (gdn_status s = ensure_smem_attr(dev, bit, kern, L::kSmemBytes)) return s;
   // split the SMs left after the chains between the stats and output roles (fused_stats_pct)
   const int workers = sms - bh;
-  int n_stats = (workers * fused_stats_pct(kF8) + 50) / 100;
+  int n_stats = (workers * fused_stats_pct(kF8, DP) + 50) / 100;
   if (n_stats < 1) n_stats = 1;
   if (n_stats > workers - 1) n_stats = workers - 1;
   int* f = w.flags;
