@@ -9,6 +9,10 @@
 //
 // kDualV: dK_t and dV_t from one pass (the K tile and G_t are shared): a second accumulator
 // takes K_t G_t^T, and the epilogue stores both tiles through one staging buffer.
+// kDualE: dQ_t and the output statistic E_t = dO_t^T Q_t from one pass over dO: each stage holds
+// a dO tile and a Q tile; dQ_t takes the dO tile K-major as above, and a per-frame accumulator sums
+// dO^T Q over the frame's tiles with both read MN-major (the statistics kernel's reduction, in the
+// same order); the epilogue writes E_t as f32 in the four-key interleaved layout of b4_index.
 //
 // with s the key scale, G_t = dL/dS_t from the backward chain and W'_t = -s gamma_t (S_{t-1}^T
 // G_t + G_t^T S_{t-1}) from the per-frame kernel (K_t here is the unscaled key tile, so both
@@ -25,25 +29,28 @@
 
 namespace gdn {
 
-template <int DP, int kTerms, bool kDualV = false>
+template <int DP, int kTerms, bool kDualV = false, bool kDualE = false>
 struct BwdTokenLayout {
   static_assert(DP == 128 && (kTerms == 1 || kTerms == 2), "DP = 128, one or two terms");
   static_assert(!kDualV || kTerms == 2, "the dK/dV pass has two terms");
+  static_assert(!kDualE || (kTerms == 2 && !kDualV), "the dQ/E pass has two token tiles");
   static constexpr int kAccs = kDualV ? 2 : 1;  // accumulators per tile
   static constexpr int kEpiWarps = 16;
   static constexpr int kCols = DP / 4;  // columns per epilogue thread
   static constexpr int kBoxes = DP / 64;
   static constexpr int kXBytes = kBoxes * kBoxBytes;  // one 128-token tile
   static constexpr int kYBytes = DP * DP * 2;
-  static constexpr int kYBufs = kTerms == 1 ? 2 : 1;
+  static constexpr int kYPer = kDualE ? 1 : kTerms;  // frame matrices per item
+  static constexpr int kYBufs = (kTerms == 1 || kDualE) ? 2 : 1;
   static constexpr int kStages = kTerms == 1 ? 3 : 2;
   static constexpr int kOBufs = kTerms == 1 ? 2 : 1;
   static constexpr int kStageBytes = kTerms * kXBytes;
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
-  static constexpr int kTmemCols = 2 * kAccs * DP;
+  // tile accumulators (two), then (kDualE) two per-frame E accumulators
+  static constexpr int kTmemCols = kDualE ? 4 * DP : 2 * kAccs * DP;
   static constexpr int kOBytes = kXBytes;
   static constexpr int kSmemBytes =
-      kYBufs * kTerms * kYBytes + kStages * kStageBytes + kOBufs * kOBytes + 512 + 1024;
+      kYBufs * kYPer * kYBytes + kStages * kStageBytes + kOBufs * kOBytes + 512 + 1024;
 };
 
 struct BwdTokenArgs {
@@ -51,23 +58,26 @@ struct BwdTokenArgs {
   const __nv_bfloat16* Y1;
   const float* beta;        // non-null: scale by key_scale * beta[b, t, h], else 1
   int t_lo, t_hi;           // the frames [t_lo, t_hi) of every head
+  float* E;                 // kDualE: E_t, f32 D x D per row (b*H+h)*T + t (b4_index layout)
 };
 
 // kMN0 / kMN1: the term's frame matrix is read MN-major (contraction over its rows).
 // kDualV: tm_o2 takes s beta_t * X1 Y0^T (Y0 read K-major) from a second accumulator.
-template <int DP, int kTerms, bool kMN0, bool kMN1, bool kDualV = false>
-__global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 1)
+// kDualE: X0 = dO, X1 = Q, one term (X0 Y0 with Y0 = S_t MN-major), and E_t = X0^T X1 into a.E.
+template <int DP, int kTerms, bool kMN0, bool kMN1, bool kDualV = false, bool kDualE = false>
+__global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV, kDualE>::kThreads, 1)
     gdn_bwd_token_kernel(const __grid_constant__ CUtensorMap tm_x0,
                          const __grid_constant__ CUtensorMap tm_x1,
                          const __grid_constant__ CUtensorMap tm_o,
                          const __grid_constant__ CUtensorMap tm_o2, BwdTokenArgs a, Problem p) {
-  using L = BwdTokenLayout<DP, kTerms, kDualV>;
+  using L = BwdTokenLayout<DP, kTerms, kDualV, kDualE>;
   constexpr int kAccs = L::kAccs;
+  constexpr int kMmaTerms = kDualE ? 1 : kTerms;  // products summed into a tile accumulator
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
-  uint8_t* y_buf = smem;                                     // [kYBufs][kTerms] frame matrices
-  uint8_t* x_ring = y_buf + L::kYBufs * kTerms * L::kYBytes;   // [kStages][kTerms] token tiles
+  uint8_t* y_buf = smem;                                     // [kYBufs][kYPer] frame matrices
+  uint8_t* x_ring = y_buf + L::kYBufs * L::kYPer * L::kYBytes;  // [kStages][kTerms] token tiles
   uint8_t* o_stage = x_ring + L::kStages * L::kStageBytes;    // [kOBufs] staging tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(o_stage + L::kOBufs * L::kOBytes);
   uint64_t* empty = full + L::kStages;
@@ -75,7 +85,9 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
   uint64_t* y_empty = y_full + 2;
   uint64_t* acc_full = y_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* mma_drain = acc_empty + 2;
+  uint64_t* e_full = acc_empty + 2;  // kDualE: E accumulator of item li % 2 complete / read
+  uint64_t* e_empty = e_full + 2;
+  uint64_t* mma_drain = e_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -105,6 +117,8 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
       mbar_init(&y_empty[i], 1);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&e_full[i], 1);
+      mbar_init(&e_empty[i], kEpiThreads);
     }
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
@@ -141,10 +155,10 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
           give_up(none, abort_flag);
           break;
         }
-        mbar_arrive_expect_tx(&y_full[yb], kTerms * L::kYBytes);
-        uint8_t* yd = y_buf + yb * kTerms * L::kYBytes;
+        mbar_arrive_expect_tx(&y_full[yb], L::kYPer * L::kYBytes);
+        uint8_t* yd = y_buf + yb * L::kYPer * L::kYBytes;
         bulk_load(yd, a.Y0 + yrow * DP * DP, L::kYBytes, &y_full[yb], pol_frame);
-        if (kTerms == 2)
+        if (L::kYPer == 2)
           bulk_load(yd + L::kYBytes, a.Y1 + yrow * DP * DP, L::kYBytes, &y_full[yb], pol_frame);
         y_fills.filled(yb, yph);
         for (int tile = 0; tile < n_tiles; ++tile) {
@@ -187,7 +201,13 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
         ok = false;
         break;
       }
-      const uint32_t y_base = smem_u32(y_buf + yb * kTerms * L::kYBytes);
+      const uint32_t y_base = smem_u32(y_buf + yb * L::kYPer * L::kYBytes);
+      // kDualE: this item's E accumulator is free once the epilogue has read item li - 2's
+      const uint32_t e_acc = tmem_base + 2 * DP + (li & 1) * DP;
+      if (kDualE && !mbar_wait(&e_empty[li & 1], ((li >> 1) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
       for (int tile = 0; tile < n_tiles; ++tile, ++tc) {
         const int acc = tc & 1;
         if (!mbar_wait(&acc_empty[acc], ((tc >> 1) & 1) ^ 1) || !mbar_wait(&full[stage], phase)) {
@@ -198,7 +218,7 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
         if (elect_one()) {
           const uint32_t x_base = smem_u32(x_ring + stage * L::kStageBytes);
 #pragma unroll
-          for (int term = 0; term < kTerms; ++term) {
+          for (int term = 0; term < kMmaTerms; ++term) {
             const bool mn = term == 0 ? kMN0 : kMN1;
             const uint32_t xb = x_base + term * L::kXBytes;
             const uint32_t yt = y_base + term * L::kYBytes;
@@ -225,6 +245,18 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
               mma_bf16(tmem_base + (acc * kAccs + 1) * DP, da, db, idesc_k, ks != 0);
             }
           }
+          if constexpr (kDualE) {
+            // E_t += dO^T Q over this tile's 128 tokens: both tiles MN-major (64-dim boxes
+            // kBoxBytes apart along M / N, 8-token groups 1024 bytes apart along K)
+            constexpr uint32_t idesc_e = idesc_bf16(128, DP, true, true);
+#pragma unroll
+            for (int ks = 0; ks < kRowsPerTile / 16; ++ks) {
+              const uint32_t koff = ks * 16 * 128;  // 16 token rows of 128 B
+              const uint64_t da = smem_desc(x_base + koff, kBoxBytes, 1024);
+              const uint64_t db = smem_desc(x_base + L::kXBytes + koff, kBoxBytes, 1024);
+              mma_bf16(e_acc, da, db, idesc_e, (tile | ks) != 0);
+            }
+          }
           mma_commit(&empty[stage]);
           mma_commit(&acc_full[acc]);
         }
@@ -235,7 +267,10 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
         }
       }
       if (!ok) break;
-      if (elect_one()) mma_commit(&y_empty[yb]);
+      if (elect_one()) {
+        if (kDualE) mma_commit(&e_full[li & 1]);
+        mma_commit(&y_empty[yb]);
+      }
       __syncwarp();
     }
     if (!ok) give_up(none, abort_flag);
@@ -257,7 +292,8 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
     int tc = 0;
     int nst = 0;  // staging tiles used (ring position)
     bool ok = true;
-    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    int li = 0;
+    for (long item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
       int bt, h;
       long yrow;
       decode(item, bt, h, yrow);
@@ -310,6 +346,29 @@ __global__ void __launch_bounds__(BwdTokenLayout<DP, kTerms, kDualV>::kThreads, 
         if (lost) {
           ok = false;
           break;
+        }
+      }
+      if constexpr (kDualE) {
+        // E_t of this item: thread = row v of E (TMEM lane), 32 key columns from c0
+        if (!ok) break;
+        const bool waited = mbar_wait(&e_full[li & 1], (li >> 1) & 1);
+        if (named_bar_any(1, kEpiThreads, !waited)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float v[32];
+        tmem_ld32(lane_base + 2 * DP + (li & 1) * DP + c0, v);
+        tc_fence_before();
+        mbar_arrive(&e_empty[li & 1]);
+        const int D = p.D;
+        if (row < D) {
+          float* em = a.E + yrow * D * D;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (c0 + j < D)
+              *reinterpret_cast<float4*>(em + b4_index(row, c0 + j, D)) =
+                  make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
       }
     }

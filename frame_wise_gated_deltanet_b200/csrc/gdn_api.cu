@@ -127,6 +127,8 @@ bool tmap_mats(CUtensorMap* m, const void* base, bool f32, int D, int rows, long
 }
 
 // ------------------------------------------------------------------ device info / workspace
+constexpr int kMaxSegEvents = 64;  // chain segments of the backward with saved states (events)
+
 struct DeviceState {
   int sms = 0;
   void* ws = nullptr;
@@ -137,7 +139,8 @@ struct DeviceState {
   int step_epoch = 0;
   // second stream of the backward (work that overlaps the state chains) and its fork/join events
   cudaStream_t aux = nullptr;
-  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  // (and one per chain segment of the backward with saved states)
+  cudaEvent_t ev[5 + kMaxSegEvents] = {};
   // (cos, sin) table of gdn_frame_forward_rope (kept apart from the forward's workspace)
   float2* rope_tab = nullptr;
   size_t rope_tab_bytes = 0;
@@ -919,25 +922,25 @@ gdn_status run_bwd_frame(int dev, const Problem& p, const BackwardWs& w, const f
 }
 
 // One of the token GEMMs of the backward: out = scale * sum over terms of X_i Y_i^(T)
-// (kDualV: also out2 = scale * X1 Y0^T).
-template <int kTerms, bool kMN0, bool kMN1, bool kDualV = false>
+// (kDualV: also out2 = scale * X1 Y0^T; kDualE: out = X0 Y0 and E = X0^T X1 per frame).
+template <int kTerms, bool kMN0, bool kMN1, bool kDualV = false, bool kDualE = false>
 gdn_status run_bwd_token(int dev, const Problem& p, const void* x0, const void* x1,
                          const void* Y0, const void* Y1, const float* beta, void* out,
                          const char* name, int attr_bit, cudaStream_t st, int max_ctas = 0,
-                         void* out2 = nullptr, int t_lo = 0, int t_hi = -1) {
+                         void* out2 = nullptr, int t_lo = 0, int t_hi = -1, float* E = nullptr) {
   if (t_hi < 0) t_hi = p.T;
-  using L = gdn::BwdTokenLayout<128, kTerms, kDualV>;
+  using L = gdn::BwdTokenLayout<128, kTerms, kDualV, kDualE>;
   CUtensorMap t0, t1, to, to2;
   if (!tmap_tokens(&t0, x0, p) || !tmap_tokens(&t1, kTerms == 2 ? x1 : x0, p) ||
       !tmap_tokens(&to, out, p) || !tmap_tokens(&to2, kDualV ? out2 : out, p))
     return GDN_ERR_CUDA;
-  auto kern = gdn::gdn_bwd_token_kernel<128, kTerms, kMN0, kMN1, kDualV>;
+  auto kern = gdn::gdn_bwd_token_kernel<128, kTerms, kMN0, kMN1, kDualV, kDualE>;
   if (gdn_status s = ensure_smem_attr(dev, attr_bit, kern, L::kSmemBytes)) return s;
   const long items = long(p.B) * (t_hi - t_lo) * p.H;
   const long cap = max_ctas > 0 ? max_ctas : g_dev[dev].sms;
   const int grid = static_cast<int>(items < cap ? items : cap);
   const gdn::BwdTokenArgs a{static_cast<const __nv_bfloat16*>(Y0),
-                            static_cast<const __nv_bfloat16*>(Y1), beta, t_lo, t_hi};
+                            static_cast<const __nv_bfloat16*>(Y1), beta, t_lo, t_hi, E};
   {
     ProfiledLaunch pl(name, st);
     kern<<<grid, L::kThreads, L::kSmemBytes, st>>>(t0, t1, to, to2, a, p);
@@ -1004,20 +1007,62 @@ gdn_status backward_path(int dev, const void* q, const void* k, const void* v,
   const int n_seg = overlap ? std::max(1, (p.T + seg_target / 2) / seg_target) : 1;
   const int seg_len = (p.T + n_seg - 1) / n_seg;
 
-  if (saved == nullptr) {
-    if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
-    if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the forward statistics
-    if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole,
-                                      st))
-      return s;
-  } else if (gdn_status s = link(st, sx, 0)) {  // [A]: aux after the caller's earlier work
-    return s;
+  if (saved != nullptr) {
+    // The forward's states are given: dQ_t and E_t come from one pass over dO (gdn_bwd_token_
+    // kernel_dqe), run segment by segment from the clip's end, so that each segment of the
+    // backward chain starts as soon as its E_t are stored:
+    //   aux: [A] dqe seg 1 -> dqe seg 2 -> ... -> [seg 1] frame, dk/dv -> [seg 2] frame, dk/dv
+    //   st:    [E1] chain seg 1 -> [E2] chain seg 2 -> ...                                 [end]
+    // (one event per chain segment, all recorded before the aux stream waits on the first)
+    const int n_s = std::min(n_seg, kMaxSegEvents);
+    const int len = (p.T + n_s - 1) / n_s;
+    if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the caller's earlier work
+    // A chain segment [lo, hi) ends with G_{lo-1}, which includes E_{lo-1}: the dQ/E pass
+    // before it covers frames [lo - 1, lo' - 1) (lo' the previous segment's start; T for the
+    // first), so every frame is covered once and each segment's E_t are stored before it runs.
+    int k_seg = 0;
+    int e_hi = p.T;
+    for (int hi = p.T, lo; hi > 0; hi = lo, ++k_seg) {
+      lo = std::max(0, hi - len);
+      const int e_lo = std::max(0, lo - 1);
+      // the first segment's pass runs alone: all SMs; later ones beside the chain
+      if (e_lo < e_hi)
+        if (gdn_status s = run_bwd_token<2, true, false, false, true>(
+                dev, p, d_out, q, w.S, nullptr, nullptr, dq, "gdn_bwd_token_kernel_dqe", 23, sx,
+                k_seg == 0 ? 0 : side, nullptr, e_lo, e_hi, w.E))
+          return s;
+      e_hi = e_lo;
+      if (gdn_status s = link(sx, st, 2)) return s;  // [E]: this segment's E_t are stored
+      if (gdn_status s = run_bwd_chain(dev, p, w.A, w.E, gamma, beta, ds_out, w.G, ds_in, w.C,
+                                       lo, hi, st))
+        return s;
+      if (overlap && cudaEventRecord(d->ev[5 + k_seg], st) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    k_seg = 0;
+    for (int hi = p.T, lo; hi > 0; hi = lo, ++k_seg) {
+      lo = std::max(0, hi - len);
+      // [segment]: its G_t are stored
+      if (overlap && cudaStreamWaitEvent(sx, d->ev[5 + k_seg], 0) != cudaSuccess)
+        return GDN_ERR_CUDA;
+      const int g = lo == 0 ? 0 : side;  // the last segment's passes run after the chain
+      if (gdn_status s = run_bwd_frame(dev, p, w, s_in, gamma, beta, d_gamma, d_beta, lo, hi, sx,
+                                       g))
+        return s;
+      if (gdn_status s = run_bwd_token<2, true, false, true>(
+              dev, p, v, k, w.G, w.W, beta, dk, "gdn_bwd_token_kernel_dkdv", 25, sx, g, dv, lo, hi))
+        return s;
+    }
+    return link(sx, st, 3);  // [end]: the call ends on `st` after everything
   }
-  // E_t statistics beside the forward chain (or, with saved states, on all SMs)
-  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, sx, saved ? 0 : side))
+
+  if (gdn_status s = run_stats<128, true>(dev, p, k, v, w.A, w.B, st)) return s;
+  if (gdn_status s = link(st, sx, 0)) return s;  // [A]: aux after the forward statistics
+  if (gdn_status s = run_chain<128>(dev, p, w.A, w.B, gamma, beta, s_in, w.S, nullptr, whole,
+                                    st))
     return s;
-  if (saved == nullptr)
-    if (gdn_status s = link(st, sx, 1)) return s;  // [S]: dq after the forward chain
+  // E_t statistics beside the forward chain
+  if (gdn_status s = run_stats<128, true>(dev, pe, q, d_out, w.W, w.E, sx, side)) return s;
+  if (gdn_status s = link(st, sx, 1)) return s;  // [S]: dq after the forward chain
   if (gdn_status s = link(sx, st, 2)) return s;  // [E]: backward chain after E_t
   if (gdn_status s = run_bwd_token<1, true, false>(dev, p, d_out, nullptr, w.S, nullptr, nullptr,
                                                    dq, "gdn_bwd_token_kernel_dq", 22, sx, side))

@@ -261,10 +261,42 @@ def test_training_pair_matches_oracle(shape):
     check_against_oracle(x, c, got, ks)
 
 
+@pytest.mark.parametrize("shape", SEGMENTED, ids=lambda s: "B%dH%dT%dN%dD%d%s_seg%d" % (s[:5] + ("s" if s[5] else "", s[6])))
+def test_training_pair_segmented_matches_oracle(shape):
+    """The backward with saved states in segments of frames: each segment's dQ/E pass runs
+    before its part of the reverse chain (from the clip's end), the per-frame and dk/dv passes
+    of every segment after it; against the oracle."""
+    B, H, T, N, D, with_state, seg = shape
+    old = os.environ.get("GDN_BWD_SEGMENT_FRAMES")
+    os.environ["GDN_BWD_SEGMENT_FRAMES"] = str(seg)
+    try:
+        x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=760 + T + seg,
+                                   state_std=0.3 if with_state else 0.0)
+        c = gdn_inputs.cotangents(B, H, T, N, D, seed=860 + T + seg,
+                                  state_std=1.0 if with_state else 0.0)
+        ks = 1.0 / math.sqrt(D * N)
+        g = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+        gc = {k: (None if v is None else v.cuda()) for k, v in c.items()}
+        a = api()
+        _, _, saved = a.gdn_frame_forward_train(g["q"], g["k"], g["v"], g["gamma"], g["beta"],
+                                                g["state"], key_scale=ks)
+        got = a.gdn_frame_backward_saved(g["q"], g["k"], g["v"], g["gamma"], g["beta"], saved,
+                                         gc["d_out"], state_in=g["state"],
+                                         d_state_out=gc["d_state"], key_scale=ks)
+        assert a.gdn_sync_status() == 0
+    finally:
+        if old is None:
+            os.environ.pop("GDN_BWD_SEGMENT_FRAMES", None)
+        else:
+            os.environ["GDN_BWD_SEGMENT_FRAMES"] = old
+    check_against_oracle(x, c, got, ks)
+
+
 def test_training_pair_equals_recomputing_backward_on_720p():
     """On the 720p clip the saved states are those the recomputing backward builds (the same
-    statistics and chain kernels), so both backwards agree bit for bit; the forward that saves
-    them equals the three-kernel forward bit for bit."""
+    statistics and chain kernels), and the saved path's dQ/E pass issues the same products in the
+    same order as the separate dq and E passes, so both backwards agree bit for bit; the forward
+    that saves them equals the three-kernel forward bit for bit."""
     from frame_wise_gated_deltanet_b200 import _lib
     w = gdn_inputs.WORKLOADS["720p"]
     x = gdn_inputs.workload_inputs(w, device="cuda")
