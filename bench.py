@@ -155,6 +155,8 @@ def kernel_bytes(name, w, fp8=False):
         return fh * 2 * nd2
     if name == "gdn_bwd_token_kernel_dkdv":  # read V, K, G_t, W'_t; write dK, dV
         return fh * (4 * nd2 + 2 * dd * 2)
+    if name == "gdn_bwd_token_kernel_dqe":  # read dO, Q, S_t; write dQ and E_t (f32)
+        return fh * (3 * nd2 + dd * 2 + dd * 4)
     if name.startswith("gdn_bwd_token_kernel_d"):  # read X tiles and frame matrices; write out
         terms = 2 if name.endswith("_dk") else 1
         return fh * ((terms + 1) * nd2 + terms * dd * 2)
@@ -213,6 +215,7 @@ KERNEL_SOURCES = {
     "gdn_bwd_token_kernel_dv": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_bwd_token_kernel_dk": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
     "gdn_bwd_token_kernel_dkdv": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
+    "gdn_bwd_token_kernel_dqe": ["bwd_token_kernel.cuh", "common.cuh", "ptx.cuh"],
 }
 
 
