@@ -47,7 +47,7 @@ struct OutputLayout {
   static_assert(!kRope || (!kF8 && !kLA), "RoPE prologue: bf16 GDN only");
   static constexpr bool kTransform = kLA || kF8 || kRope;
   // transform warps: 4 (one token row each; fp8: kF8Parts lanes per row), or for RoPE 4 per group
-  static constexpr int kF8Parts = 1;  // fp8: lanes per Q row in the e4m3 -> bf16 conversion
+  static constexpr int kF8Parts = 2;  // fp8: lanes per Q row in the e4m3 -> bf16 conversion
   static constexpr int kXfWarps = kRope ? 4 * kRopeGroups : (kF8 ? 4 * kF8Parts : 4);
   static constexpr int kEpiWarps = 4 * kG;
   static constexpr int kCols = DP / kG;                // columns per epilogue thread
