@@ -67,6 +67,9 @@ def args_parse():
                     help="E4M3 q, k, v with per-(frame, head) scales (gdn_frame_forward_fp8)")
     ap.add_argument("--backward", action="store_true",
                     help="time gdn_frame_backward (the training pass) instead of the forward")
+    ap.add_argument("--backward-saved", action="store_true",
+                    help="with --backward: time gdn_frame_backward_saved, reading the A_t, B_t, "
+                         "S_t that one gdn_frame_forward_train call kept (outside the timed region)")
     ap.add_argument("--rope", action="store_true",
                     help="time gdn_rope_3d on the clip's q and k (in place) instead of the forward")
     ap.add_argument("--rope-fused", action="store_true",
@@ -80,7 +83,9 @@ def args_parse():
                          "(strong scaling) instead of one clip per rank (weak scaling)")
     ap.add_argument("--forward-mode", type=int, default=0,
                     help="gdn_set_forward_mode: 0 auto, 1 three kernels, 2 fused, 3 chunked")
-    return ap.parse_args()
+    a = ap.parse_args()
+    a.backward = a.backward or a.backward_saved
+    return a
 
 
 def peaks():
@@ -527,9 +532,17 @@ def main():
                                       device=dev)["d_out"]
         out = st = None
 
-        def step():
-            api.gdn_frame_backward(q, k, v, gam, bet, d_out, key_scale=w.key_scale,
-                                   stream=stream)
+        if a.backward_saved:
+            _, _, saved = api.gdn_frame_forward_train(q, k, v, gam, bet, key_scale=w.key_scale,
+                                                      stream=stream)
+
+            def step():
+                api.gdn_frame_backward_saved(q, k, v, gam, bet, saved, d_out,
+                                             key_scale=w.key_scale, stream=stream)
+        else:
+            def step():
+                api.gdn_frame_backward(q, k, v, gam, bet, d_out, key_scale=w.key_scale,
+                                       stream=stream)
     else:
         g = gdn_inputs.workload_inputs(w, device=dev)
         if shard:
@@ -634,13 +647,18 @@ def main():
         "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
         "scaling": "strong" if shard else "weak", "vs_baseline": None,
         "dtype": "e4m3 q/k/v, bf16 out" if a.fp8 else "bf16", "data": "synthetic",
-        "config": workload_config(w_all, shard, world),
+        "config": dict(workload_config(w_all, shard, world),
+                       **({"backward": "saved states (gdn_frame_backward_saved)"
+                           if a.backward_saved else "recomputed forward (gdn_frame_backward)"}
+                          if a.backward else {})),
         "roofline": {
             "bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": (achieved / hbm) if achieved else None,
             "peak_source": f"{peak_kind} HBM copy bandwidth",
             "traffic": ncu_traffic(dom, w.name + ("+fp8" if a.fp8 else "")
-                                   + ("+bwd" if a.backward else "")),
+                                   + ("+bwd" if a.backward else "")
+                                   + ("+saved" if a.backward_saved else "")
+                                   + ("+rope" if a.rope_fused else "")),
             "algorithmic_bytes_per_launch": kb, "ms_per_launch": dom_ms,
             "path": {"algorithmic_bytes_per_step": path_bytes, "achieved_gbs": path_gbs,
                      "frac": path_gbs / hbm},
