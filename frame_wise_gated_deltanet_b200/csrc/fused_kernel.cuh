@@ -8,9 +8,10 @@
 // A_t (bf16), B_t (f32) and S_t (bf16) travel through per-head rings of R slots (a few tens of
 // MB, meant to stay in L2: A_t and S_t are loaded with evict_last while the q/k/v/out streams
 // use evict_first). Hand-off is by release/acquire flags in global memory with bounded waits;
-// every role processes its items in increasing frame order and every wait points at a
-// strictly earlier frame (or at the chain, which only waits on earlier frames), so with all
-// CTAs co-resident the grid cannot deadlock.
+// the statistics take items in frame-major order and the outputs in the order the chains
+// publish them (frame order within a head); every wait points at a strictly earlier frame, at
+// the chain (which only waits on earlier frames) or at a queue position the chains will fill, so
+// with all CTAs co-resident the grid cannot deadlock.
 #pragma once
 #include <cuda.h>
 

@@ -293,15 +293,18 @@ size_t gdn_backward_workspace_bytes(int B, int H, int T, int N, int D);
  * Training pair: a forward that keeps what the backward needs, and a backward that uses it
  * instead of recomputing the forward's statistics and state chain (which read k and v again).
  *
- * gdn_frame_forward_train: gdn_frame_forward (same arguments and results; the three-kernel
- * path) that also stores, in the caller's device buffer `saved` (gdn_train_saved_bytes(B, H, T,
- * N, D) bytes, 256-byte aligned, not overlapping q, k, v or out), every frame's A_t (bf16), B_t
- * (f32) and S_t (bf16) in the library's internal layout. 64 < D <= 128 (GDN_ERR_UNSUPPORTED
- * otherwise); the buffer's contents are only meaningful to gdn_frame_backward_saved.
+ * gdn_frame_forward_train: gdn_frame_forward (same arguments and results; the fused kernel with
+ * one ring slot per frame where the fused forward applies, else the three kernels) that also
+ * stores, in the caller's device buffer `saved` (gdn_train_saved_bytes(B, H, T, N, D) bytes,
+ * 256-byte aligned, not overlapping q, k, v or out), every frame's A_t (bf16), B_t (f32) and
+ * S_t (bf16) in the library's internal layout. 64 < D <= 128 (GDN_ERR_UNSUPPORTED otherwise);
+ * the buffer's contents are only meaningful to gdn_frame_backward_saved.
  * gdn_frame_backward_saved: gdn_frame_backward (same arguments, results, alignment and overlap
  * rules) for the same q, k, v, gamma, beta, state_in and key_scale that the forward saved, with
  * `saved` read instead of recomputed: it skips one statistics pass over k and v and the forward
- * state chain. Its workspace is smaller than gdn_frame_backward's (no A_t, B_t, S_t).
+ * state chain, and computes dq and the output statistic E_t = dO^T Q in one pass over dO, run
+ * ahead of the reverse state chain segment by segment. Results are bit-identical to
+ * gdn_frame_backward's. Its workspace is smaller than gdn_frame_backward's (no A_t, B_t, S_t).
  * gdn_train_saved_bytes returns 0 for unsupported sizes.
  */
 size_t gdn_train_saved_bytes(int B, int H, int T, int N, int D);
