@@ -222,6 +222,32 @@ def test_480p_workload_all_paths(forward_mode):
     assert relf(f64(st), s_ref) <= S_TOL
 
 
+@pytest.mark.parametrize("forward_mode", [1, 2, 3], indirect=True, ids=["split", "fused", "chunked"])
+def test_forward_in_a_cuda_graph(forward_mode):
+    """After one uncaptured call (which sizes the workspace), the forward can be captured in a
+    CUDA graph on every path (the fused path's cooperative launch and its flag memset become
+    graph nodes) and its replays give the uncaptured call's result bit for bit."""
+    B, H, T, N, D = 1, 3, 11, 150, 128
+    x = gdn_inputs.clip_inputs(B, H, T, N, D, seed=1910, state_std=0.3, device="cuda")
+    a = api()
+    ref_o, ref_s = a.gdn_frame_forward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["state"])
+    torch.cuda.synchronize()
+    out = torch.empty_like(ref_o)
+    st = torch.empty_like(ref_s)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            a.gdn_frame_forward(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["state"], out,
+                                st, stream=s)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert a.gdn_sync_status() == 0
+    assert torch.equal(out, ref_o) and torch.equal(st, ref_s)
+
+
 def test_fused_and_split_paths_agree_on_720p():
     """Both forward paths on the full 720p clip: same kernels' arithmetic, so they agree to the
     rounding of the bf16 copies of S (identical in practice)."""
