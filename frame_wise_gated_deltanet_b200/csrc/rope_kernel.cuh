@@ -81,18 +81,22 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
   const int pt = r.d_t / 2, ph = r.d_h / 2;
   for (int li = threadIdx.x; li < per_tok; li += blockDim.x) {
     const int dg = li % per_row;
-    // the 4 pairs of this vector: axis (0 time, 1 row, 2 column) and index within the axis
+    int row = n0 / r.grid_w;
+    int col = n0 - row * r.grid_w;
+    // the 4 pairs of this vector: axis (0 time, 1 row, 2 column) and index within the axis; the
+    // (cos, sin) of time pairs (fixed for the frame) and of row pairs (fixed along a grid row)
+    // are held in registers, only the column pairs' are read for every token
     int axis[4], idx[4];
-    float2 cs_t[4];
+    float2 cs_fix[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const int j = dg * 4 + p;  // pair index over the head dimension
       axis[p] = j < pt ? 0 : (j < pt + ph ? 1 : 2);
       idx[p] = axis[p] == 0 ? j : (axis[p] == 1 ? j - pt : j - pt - ph);
-      cs_t[p] = axis[p] == 0 ? __ldg(tab + t * pt + idx[p]) : make_float2(1.f, 0.f);
+      cs_fix[p] = axis[p] == 0   ? __ldg(tab + t * pt + idx[p])
+                  : axis[p] == 1 ? __ldg(tab + r.off_h + row * ph + idx[p])
+                                 : make_float2(1.f, 0.f);
     }
-    int row = n0 / r.grid_w;
-    int col = n0 - row * r.grid_w;
     // groups of kRopeBatch tokens: the group's loads are issued before any of its stores (x and
     // y may be the same memory, so the compiler could not move a load above a store itself)
     for (int nb = n0; nb < n1; nb += kRopeBatch) {
@@ -106,9 +110,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
           __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw[u]);
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
-            const float2 cs = axis[p] == 0 ? cs_t[p]
-                              : axis[p] == 1 ? __ldg(tab + r.off_h + row * ph + idx[p])
-                                             : __ldg(tab + r.off_w + col * ph + idx[p]);
+            const float2 cs = axis[p] == 2 ? __ldg(tab + r.off_w + col * ph + idx[p]) : cs_fix[p];
             const float2 v = __bfloat1622float2(p2[p]);
             p2[p] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
           }
@@ -117,6 +119,10 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
         if (++col == r.grid_w) {
           col = 0;
           ++row;
+          if (nb + u + 1 < n1)  // a next token exists: the new row's pairs
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+              if (axis[p] == 1) cs_fix[p] = __ldg(tab + r.off_h + row * ph + idx[p]);
         }
       }
     }
