@@ -16,15 +16,23 @@ __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_status, 0,
 
 constexpr int kErrTimeout = 6;  // == GDN_ERR_TIMEOUT
 
-// 3D rotary position embedding applied to q and k inside the forward's statistics and output
-// kernels (see rope_kernel.cuh for the reading). tab holds (cos, sin) per (axis, position,
-// pair): frame t's time pairs at t * pt, grid row r's pairs at off_h + r * ph, grid column c's
-// at off_w + c * ph (the row and column slices have the same width).
+// The (cos, sin) table of the 3D RoPE (see rope_kernel.cuh for the reading) and its layout. The
+// head dimension's D/2 pairs j split into the time slice [0, pt), the grid-row slice
+// [pt, pt + ph) and the grid-column slice [pt + ph, pt + 2 ph). For each axis and each position
+// on it (frame, grid row, grid column) the table holds one row of len entries indexed by the
+// absolute pair index: pair j at row offset j - j0, j0 = the axis's first pair rounded down to
+// even, len even, entries of the row outside the axis's slice (1, 0). Every row starts at an
+// even entry, so pairs (j, j + 1) with j even are one aligned 16-byte load from either pair's
+// axis. Rows: frame t at t * len_t, grid row r at off_h + r * len_h, grid column c at
+// off_w + c * len_w.
 struct RopeArgs {
   const float2* tab = nullptr;
   int grid_w = 1;
-  int pt = 0, ph = 0;        // pairs of the time slice and of the row (= column) slice
-  int off_h = 0, off_w = 0;  // first table entries of the row and column axes
+  int pt = 0, ph = 0;                   // pairs of the time slice and of the row (= column) slice
+  int len_t = 0, len_h = 0, len_w = 0;  // row lengths of the three axes (even)
+  int j0_h = 0, j0_w = 0;               // first pair of the row / column slice, rounded down to even
+  int off_h = 0, off_w = 0;             // first table entries of the row and column axes
+  int n_rc = 0;  // entries of the grid-row and grid-column rows (from off_h to the table's end)
 };
 
 // One problem: q/k/v/out are [B, T, N, H, D] bf16, gamma/beta [B, T, H] f32.

@@ -1238,16 +1238,28 @@ gdn_status rope_dims(int B, int T, int N, int H, int D, int grid_h, int grid_w, 
   r->N = N;
   r->H = H;
   r->D = D;
-  r->grid_w = grid_w;
   r->d_h = 2 * (D / 6);
   r->d_w = r->d_h;
   r->d_t = D - 2 * r->d_h;
-  if (double(T) * (r->d_t / 2) + double(grid_h) * (r->d_h / 2) + double(grid_w) * (r->d_w / 2) >
-      2147483647.0)
+  // the table layout of gdn::RopeArgs: per axis, rows of whole 16-byte entry pairs indexed by
+  // the absolute pair index from the axis's first pair rounded down to even
+  gdn::RopeArgs& a = r->ra;
+  a.tab = nullptr;
+  a.grid_w = grid_w;
+  a.pt = r->d_t / 2;
+  a.ph = r->d_h / 2;
+  auto even_up = [](int x) { return (x + 1) & ~1; };
+  a.len_t = even_up(a.pt);
+  a.j0_h = a.pt & ~1;
+  a.len_h = even_up(a.pt + a.ph - a.j0_h);
+  a.j0_w = (a.pt + a.ph) & ~1;
+  a.len_w = even_up(a.pt + 2 * a.ph - a.j0_w);
+  if (double(T) * a.len_t + double(grid_h) * a.len_h + double(grid_w) * a.len_w > 2147483647.0)
     return GDN_ERR_INVALID_ARG;
-  r->off_h = T * (r->d_t / 2);
-  r->off_w = r->off_h + grid_h * (r->d_h / 2);
-  *n_tab = long(r->off_w) + long(grid_w) * (r->d_w / 2);
+  a.off_h = T * a.len_t;
+  a.off_w = a.off_h + grid_h * a.len_h;
+  *n_tab = long(a.off_w) + long(grid_w) * a.len_w;
+  a.n_rc = static_cast<int>(*n_tab - a.off_h);
   return GDN_OK;
 }
 
@@ -1410,12 +1422,8 @@ gdn_status gdn_frame_forward_rope(const gdn_bf16* q, const gdn_bf16* k, const gd
     if (gdn_status s = launch_rope_table(tab, r, n_tab, t_offset, rope_base, st)) return s;
   }
   Problem p{B, H, T, N, D, key_scale};
+  p.rope = r.ra;
   p.rope.tab = tab;
-  p.rope.grid_w = grid_w;
-  p.rope.pt = r.d_t / 2;
-  p.rope.ph = r.d_h / 2;
-  p.rope.off_h = r.off_h;
-  p.rope.off_w = r.off_w;
   return forward_impl(q, k, v, gamma, beta, state_in, out, state_out, p, st);
 }
 
@@ -1682,6 +1690,7 @@ gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int 
     return s;
   float2* tab = static_cast<float2*>(base_ws);
   if (gdn_status s = launch_rope_table(tab, r, n_tab, t_offset, base, st)) return s;
+  r.ra.tab = tab;
   // one block row per frame of one batch element, one block per kRopeTokens of its tokens
   const long chunks = (long(N) + gdn::kRopeTokens - 1) / gdn::kRopeTokens;
   if (chunks > 65535) return GDN_ERR_INVALID_ARG;
@@ -1692,7 +1701,7 @@ gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int 
     const int threads = std::min(gdn::kRopeMaxThreads, (per_tok + 31) / 32 * 32);
     gdn::gdn_rope_kernel<<<dim3(static_cast<unsigned>(B * T), static_cast<unsigned>(chunks)),
                            threads, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x),
-                                    reinterpret_cast<__nv_bfloat16*>(y), tab, r);
+                                    reinterpret_cast<__nv_bfloat16*>(y), r);
   }
   return check_launch();
 }

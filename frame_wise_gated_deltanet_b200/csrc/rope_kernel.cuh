@@ -6,11 +6,12 @@
 // frame index (plus t_offset), the row n / grid_w or the column n % grid_w of the token.
 //
 // Standalone pass (gdn_rope_3d), two launches. A table kernel computes (cos, sin) of every
-// (axis, position, pair) once, in double precision: T * d_t/2 + grid_h * d_h/2 + grid_w * d_w/2
-// entries, about 180 KB for the 720p clip, which stay in L2. The rotation kernel then streams the
-// tensor in 16-byte vectors (8 dims of one token and head), reads each pair's (cos, sin) from the
-// table, rotates in f32 and rounds to bf16. It is HBM-bound: every element is read and written
-// once. Each thread reads and writes the same 16 bytes, so x and y may be the same memory.
+// (axis, position, pair) once, in double precision: one row per frame, grid row and grid column,
+// each row padded to whole 16-byte pairs of entries (the RopeArgs layout), about 180 KB for the
+// 720p clip, which stay in L2. The rotation kernel then streams the tensor in 16-byte vectors
+// (8 dims of one token and head), reads the (cos, sin) of the vector's pairs from the table,
+// rotates in f32 and rounds to bf16. It is HBM-bound: every element is read and written once.
+// Each thread reads and writes the same 16 bytes, so x and y may be the same memory.
 //
 // Fused prologue (gdn_frame_forward_rope): the same table, and rope_rotate_tile applied by
 // transform warps to the K tiles of the statistics kernel and the Q tiles of the output kernel in
@@ -22,37 +23,94 @@ namespace gdn {
 
 struct RopeDims {
   int B, T, N, H, D;
-  int grid_w;
   int d_t, d_h, d_w;
-  int off_h, off_w;  // first table entry of the row / column axis
+  RopeArgs ra;  // table layout (ra.tab set by the caller once the table has memory)
 };
 
+// The table: entry e of the RopeArgs layout. Entries of a row outside its axis's slice are
+// (1, 0); the others are (cos, sin) of pos * base^(-2i / d_axis) for the pair's index i within
+// its slice.
 __global__ void __launch_bounds__(256)
     gdn_rope_table_kernel(float2* __restrict__ tab, RopeDims r, int t_offset, double log2_base) {
-  const int nt = r.T * (r.d_t / 2);
-  const int n_all = r.off_w + r.grid_w * (r.d_w / 2);
+  const RopeArgs& a = r.ra;
+  const int n_all = a.off_w + a.grid_w * a.len_w;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= n_all) return;
-  int pos, i, da;
-  if (e < nt) {
-    pos = e / (r.d_t / 2) + t_offset;
-    i = e % (r.d_t / 2);
+  int pos, j, first, da;
+  if (e < a.off_h) {
+    pos = e / a.len_t + t_offset;
+    j = e % a.len_t;
+    first = 0;
     da = r.d_t;
-  } else if (e < r.off_w) {
-    const int f = e - r.off_h;
-    pos = f / (r.d_h / 2);
-    i = f % (r.d_h / 2);
+  } else if (e < a.off_w) {
+    const int f = e - a.off_h;
+    pos = f / a.len_h;
+    j = a.j0_h + f % a.len_h;
+    first = a.pt;
     da = r.d_h;
   } else {
-    const int f = e - r.off_w;
-    pos = f / (r.d_w / 2);
-    i = f % (r.d_w / 2);
+    const int f = e - a.off_w;
+    pos = f / a.len_w;
+    j = a.j0_w + f % a.len_w;
+    first = a.pt + a.ph;
     da = r.d_w;
+  }
+  const int i = j - first;
+  if (i < 0 || i >= da / 2) {
+    tab[e] = make_float2(1.f, 0.f);
+    return;
   }
   const double theta = exp2(-(2.0 * i / da) * log2_base);
   double s, c;
   sincos(static_cast<double>(pos) * theta, &s, &c);
   tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+// The 8 dims of chunk c (pairs 4c .. 4c + 3): each pair's axis (0 time, 1 grid row, 2 grid
+// column) and the offset, in its axis's table rows, of the 16-byte entry pair (j & ~1, j | 1).
+struct RopeChunk {
+  int ax[4];
+  int eo[4];
+};
+
+__device__ __forceinline__ RopeChunk rope_chunk(const RopeArgs& ra, int c) {
+  RopeChunk k;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int j = 4 * c + p;
+    const int a = j < ra.pt ? 0 : (j < ra.pt + ra.ph ? 1 : 2);
+    k.ax[p] = a;
+    k.eo[p] = (j & ~1) - (a == 0 ? 0 : (a == 1 ? ra.j0_h : ra.j0_w));
+  }
+  return k;
+}
+
+// (cos, sin) of the chunk's pairs on axis a at position pos (frame, grid row or grid column) into
+// cs; the chunk's other pairs are left alone. One 16-byte load per pair of pairs (2q, 2q + 1).
+__device__ __forceinline__ void rope_fetch(const RopeArgs& ra, const RopeChunk& k, int a, int pos,
+                                           float2* cs) {
+  const int row =
+      a == 0 ? pos * ra.len_t : (a == 1 ? ra.off_h + pos * ra.len_h : ra.off_w + pos * ra.len_w);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const bool lo = k.ax[2 * q] == a, hi = k.ax[2 * q + 1] == a;
+    // every lane loads (the row's first entries where neither pair is on the axis), so the load
+    // is not under a divergent branch
+    const int e = lo ? k.eo[2 * q] : (hi ? k.eo[2 * q + 1] : 0);
+    const float4 v = __ldg(reinterpret_cast<const float4*>(ra.tab + row) + (e >> 1));
+    if (lo) cs[2 * q] = make_float2(v.x, v.y);
+    if (hi) cs[2 * q + 1] = make_float2(v.z, v.w);
+  }
+}
+
+// Rotate the 4 pairs of a 16-byte chunk of bf16 (f32 arithmetic, bf16 rounding).
+__device__ __forceinline__ void rope_rotate_chunk(uint4& raw, const float2* cs) {
+  __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float2 v = __bfloat1622float2(p2[p]);
+    p2[p] = __floats2bfloat162_rn(v.x * cs[p].x - v.y * cs[p].y, v.x * cs[p].y + v.y * cs[p].x);
+  }
 }
 
 // x, y: [B, T, N, H, D] bf16 (may be the same memory). Grid (B*T, token chunks): blockIdx.x is
@@ -67,8 +125,8 @@ constexpr int kRopeBatch = 4;
 constexpr int kRopeMaxThreads = 512;
 
 __global__ void __launch_bounds__(kRopeMaxThreads)
-    gdn_rope_kernel(const __nv_bfloat16* x, __nv_bfloat16* y, const float2* __restrict__ tab,
-                    RopeDims r) {
+    gdn_rope_kernel(const __nv_bfloat16* x, __nv_bfloat16* y, RopeDims r) {
+  const RopeArgs& ra = r.ra;
   const int bt = blockIdx.x;
   const int t = bt % r.T;
   const int per_row = r.D / 8;  // 16-byte vectors per (token, head)
@@ -78,25 +136,17 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
   const long frame0 = static_cast<long>(bt) * r.N * per_tok;
   const uint4* src = reinterpret_cast<const uint4*>(x) + frame0;
   uint4* dst = reinterpret_cast<uint4*>(y) + frame0;
-  const int pt = r.d_t / 2, ph = r.d_h / 2;
   for (int li = threadIdx.x; li < per_tok; li += blockDim.x) {
-    const int dg = li % per_row;
-    int row = n0 / r.grid_w;
-    int col = n0 - row * r.grid_w;
-    // the 4 pairs of this vector: axis (0 time, 1 row, 2 column) and index within the axis; the
-    // (cos, sin) of time pairs (fixed for the frame) and of row pairs (fixed along a grid row)
-    // are held in registers, only the column pairs' are read for every token
-    int axis[4], idx[4];
+    const RopeChunk k = rope_chunk(ra, li % per_row);
+    int row = n0 / ra.grid_w;
+    int col = n0 - row * ra.grid_w;
+    // the (cos, sin) of the vector's time pairs (fixed for the frame) and grid-row pairs (fixed
+    // along a grid row) are held in registers; only the column pairs' are read for every token
     float2 cs_fix[4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const int j = dg * 4 + p;  // pair index over the head dimension
-      axis[p] = j < pt ? 0 : (j < pt + ph ? 1 : 2);
-      idx[p] = axis[p] == 0 ? j : (axis[p] == 1 ? j - pt : j - pt - ph);
-      cs_fix[p] = axis[p] == 0   ? __ldg(tab + t * pt + idx[p])
-                  : axis[p] == 1 ? __ldg(tab + r.off_h + row * ph + idx[p])
-                                 : make_float2(1.f, 0.f);
-    }
+    for (int p = 0; p < 4; ++p) cs_fix[p] = make_float2(1.f, 0.f);
+    rope_fetch(ra, k, 0, t, cs_fix);
+    rope_fetch(ra, k, 1, row, cs_fix);
     // groups of kRopeBatch tokens: the group's loads are issued before any of its stores (x and
     // y may be the same memory, so the compiler could not move a load above a store itself)
     for (int nb = n0; nb < n1; nb += kRopeBatch) {
@@ -107,26 +157,37 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
 #pragma unroll
       for (int u = 0; u < kRopeBatch; ++u) {
         if (nb + u < n1) {
-          __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw[u]);
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const float2 cs = axis[p] == 2 ? __ldg(tab + r.off_w + col * ph + idx[p]) : cs_fix[p];
-            const float2 v = __bfloat1622float2(p2[p]);
-            p2[p] = __floats2bfloat162_rn(v.x * cs.x - v.y * cs.y, v.x * cs.y + v.y * cs.x);
-          }
+          float2 cs[4] = {cs_fix[0], cs_fix[1], cs_fix[2], cs_fix[3]};
+          rope_fetch(ra, k, 2, col, cs);
+          rope_rotate_chunk(raw[u], cs);
           __stcs(dst + static_cast<long>(nb + u) * per_tok + li, raw[u]);
         }
-        if (++col == r.grid_w) {
+        if (++col == ra.grid_w) {
           col = 0;
           ++row;
-          if (nb + u + 1 < n1)  // a next token exists: the new row's pairs
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-              if (axis[p] == 1) cs_fix[p] = __ldg(tab + r.off_h + row * ph + idx[p]);
+          if (nb + u + 1 < n1) rope_fetch(ra, k, 1, row, cs_fix);  // a next token exists
         }
       }
     }
   }
+}
+
+// Shared memory the forward's statistics and output roles set aside for the table's grid-row and
+// grid-column rows (3072 entries: grid_h + grid_w up to 139 at D = 128). The CTA copies them
+// there once, before its first tile; a larger table is read from global memory instead.
+constexpr int kRopeSmemTabBytes = 24 * 1024;
+
+// Copy the grid-row and grid-column rows of the table into tab_s (kRopeSmemTabBytes, 16-byte
+// aligned) if they fit, by threads tid of nthreads; returns where rope_rotate_tile reads them.
+// The caller synchronises the CTA before the first read.
+__device__ __forceinline__ const float2* rope_stage_rc(float2* tab_s, const RopeArgs& ra, int tid,
+                                                       int nthreads) {
+  if (ra.n_rc * static_cast<int>(sizeof(float2)) > kRopeSmemTabBytes) return ra.tab + ra.off_h;
+  // off_h and n_rc are even (whole 16-byte entry pairs)
+  const float4* src = reinterpret_cast<const float4*>(ra.tab + ra.off_h);
+  float4* dst = reinterpret_cast<float4*>(tab_s);
+  for (int i = tid; i < ra.n_rc / 2; i += nthreads) dst[i] = __ldg(src + i);
+  return tab_s;
 }
 
 // The same rotation applied in shared memory by the forward's statistics (K) and output (Q)
@@ -135,28 +196,31 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
 // 128 B, 128B-swizzled, kBoxBytes apart). Dims at or past D are left alone (TMA zero fill).
 // Thread tid of nthreads owns chunk c = tid % (DP/8) of rows tid / (DP/8), + nthreads / (DP/8),
 // ...: its 4 pairs, hence their axes and the time pairs' (cos, sin), are fixed for the tile; a
-// warp covers whole rows, so its shared-memory accesses take the minimum number of wavefronts
-// and its table reads for one token fall in a few adjacent sectors. The arithmetic and the
-// rounding are those of gdn_rope_kernel.
+// warp covers whole rows, so its shared-memory accesses take the minimum number of wavefronts.
+// The grid-row and column pairs' entries are read per row from rc (rope_stage_rc: the CTA's
+// shared-memory copy of the table's grid-row and grid-column rows, else the table itself), one
+// 8-byte load per pair with no branch around it. The arithmetic and the rounding are those of
+// gdn_rope_kernel.
 template <int DP>
 __device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nthreads, int rows,
-                                                 int n0, int t, int D, const RopeArgs& ra) {
+                                                 int n0, int t, int D, const RopeArgs& ra,
+                                                 const float2* rc) {
   constexpr int kChunks = DP / 8;
   const int c = tid % kChunks;
   if (c * 8 >= D) return;
   const int r_step = nthreads / kChunks;
   int r = tid / kChunks;
   if (r >= rows) return;
-  // pair p of the chunk: (cos, sin) if on the time axis, else its table offset without the
-  // token's row (rg * ph) or column (cg * ph) term
+  // pair p of the chunk: (cos, sin) if on the time axis, else its entry's offset in rc (the row
+  // of the token's grid row or column adds rg * len_h or cg * len_w)
   float2 ct[4];
   int off[4], axis[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const int j = 4 * c + p;
     axis[p] = j < ra.pt ? 0 : (j < ra.pt + ra.ph ? 1 : 2);
-    off[p] = axis[p] == 1 ? ra.off_h + j - ra.pt : ra.off_w + j - ra.pt - ra.ph;
-    ct[p] = axis[p] == 0 ? __ldg(ra.tab + t * ra.pt + j) : make_float2(1.f, 0.f);
+    off[p] = axis[p] == 1 ? j - ra.j0_h : ra.off_w - ra.off_h + j - ra.j0_w;
+    ct[p] = axis[p] == 0 ? __ldg(ra.tab + t * ra.len_t + j) : make_float2(1.f, 0.f);
   }
   uint8_t* const box = tile + (c >> 3) * kBoxBytes;
   int n = n0 + r;
@@ -175,12 +239,7 @@ __device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nth
     // 128B swizzle: the chunk's 16-byte slot in its 128-byte row is c % 8 XOR row % 8
     uint4* ptr = reinterpret_cast<uint4*>(box + row * 128 + (((c & 7) ^ (row & 7)) << 4));
     uint4 raw = *ptr;
-    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float2 v = __bfloat1622float2(p2[p]);
-      p2[p] = __floats2bfloat162_rn(v.x * cs[p].x - v.y * cs[p].y, v.x * cs[p].y + v.y * cs[p].x);
-    }
+    rope_rotate_chunk(raw, cs);
     *ptr = raw;
   };
   // two rows at a time: both rows' table reads are in flight together
@@ -191,10 +250,10 @@ __device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nth
     float2 cs[8];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      cs[p] = axis[p] == 0 ? ct[p] : __ldg(ra.tab + off[p] + (axis[p] == 1 ? rg : cg) * ra.ph);
+      cs[p] = axis[p] == 0 ? ct[p] : rc[off[p] + (axis[p] == 1 ? rg * ra.len_h : cg * ra.len_w)];
       cs[4 + p] = axis[p] == 0 || !second
                       ? ct[p]
-                      : __ldg(ra.tab + off[p] + (axis[p] == 1 ? rg2 : cg2) * ra.ph);
+                      : rc[off[p] + (axis[p] == 1 ? rg2 * ra.len_h : cg2 * ra.len_w)];
     }
     rotate(r, cs);
     if (second) rotate(r + r_step, cs + 4);

@@ -52,7 +52,9 @@ struct StatsLayout {
   static constexpr int kThreads = 192 + (kTransform ? kTransformThreads : 0);
   static constexpr int kLoadBytes = kStageBytes;  // TMA bytes per stage
   static constexpr int kBarrierBytes = 512;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+  static constexpr int kTabBytes = kRope ? kRopeSmemTabBytes : 0;  // rope_stage_rc's table copy
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kTabBytes + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   // barriers, item ring, TMEM slot and the fused publisher's ring within kBarrierBytes
   static_assert(8 * (3 * kStages + 4 + 8 + 1) + 32 + 8 + 8 * 16 + 32 <= kBarrierBytes, "barriers");
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
@@ -167,6 +169,12 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
+  // RoPE: the table's grid-row and grid-column rows, copied past the barriers if they fit
+  const float2* rope_rc = nullptr;
+  if constexpr (kRope)
+    rope_rc = rope_stage_rc(
+        reinterpret_cast<float2*>(smem + L::kStages * L::kStageBytes + L::kBarrierBytes), p.rope,
+        threadIdx.x, blockDim.x);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -489,7 +497,7 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
           }
           const int n0 = tile * kRowsPerTile;
           rope_rotate_tile<DP>(smem + stage * L::kStageBytes, tid, L::kTransformThreads,
-                               min(kRowsPerTile, p.N - n0), n0, t, p.D, p.rope);
+                               min(kRowsPerTile, p.N - n0), n0, t, p.D, p.rope, rope_rc);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {

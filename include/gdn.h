@@ -112,7 +112,7 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
  * and t_offset (>= 0, the absolute index of the clip's first frame, so a resumed clip continues
  * its time positions). Host-side errors as gdn_frame_forward and gdn_rope_3d. Same path choice
  * (fused, three kernels, chunked) and workspace as gdn_frame_forward, plus a per-GPU cos/sin
- * table of 8 * (T * d_t / 2 + grid_h * d_h / 2 + grid_w * d_w / 2) bytes (grown like the
+ * table of 8 * (T * l_t + grid_h * l_h + grid_w * l_w) bytes (grown like the
  * workspace, freed by gdn_release_workspace), computed by one extra launch on `stream`.
  */
 gdn_status gdn_frame_forward_rope(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
@@ -340,7 +340,9 @@ gdn_status gdn_frame_backward_saved(const gdn_bf16* q, const gdn_bf16* k, const 
  * to bf16.
  * D must be a multiple of 8 (GDN_ERR_UNSUPPORTED otherwise). grid_h * grid_w == N, base > 1 and
  * t_offset >= 0 are required (GDN_ERR_INVALID_ARG). Two launches. Workspace: the cos/sin table,
- * 8 * (T * d_t / 2 + grid_h * d_h / 2 + grid_w * d_w / 2) bytes, from the shared workspace.
+ * 8 * (T * l_t + grid_h * l_h + grid_w * l_w) bytes, from the shared workspace, where l_t, l_h
+ * and l_w are the pair counts of the three slices (d_t / 2, d_h / 2, d_w / 2) padded to even row
+ * lengths that start on an even pair index (each at most 2 more than its slice's pair count).
  */
 gdn_status gdn_rope_3d(const gdn_bf16* x, gdn_bf16* y, int B, int T, int N, int H, int D,
                        int grid_h, int grid_w, float base, int t_offset, gdn_stream_t stream);
