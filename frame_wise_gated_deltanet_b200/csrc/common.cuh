@@ -27,7 +27,7 @@ constexpr int kErrTimeout = 6;  // == GDN_ERR_TIMEOUT
 // off_w + c * len_w.
 struct RopeArgs {
   const float2* tab = nullptr;
-  int grid_w = 1;
+  int grid_h = 1, grid_w = 1;
   int pt = 0, ph = 0;                   // pairs of the time slice and of the row (= column) slice
   int len_t = 0, len_h = 0, len_w = 0;  // row lengths of the three axes (even)
   int j0_h = 0, j0_w = 0;               // first pair of the row / column slice, rounded down to even

@@ -1245,6 +1245,7 @@ gdn_status rope_dims(int B, int T, int N, int H, int D, int grid_h, int grid_w, 
   // the absolute pair index from the axis's first pair rounded down to even
   gdn::RopeArgs& a = r->ra;
   a.tab = nullptr;
+  a.grid_h = grid_h;
   a.grid_w = grid_w;
   a.pt = r->d_t / 2;
   a.ph = r->d_h / 2;

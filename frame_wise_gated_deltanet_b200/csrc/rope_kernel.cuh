@@ -172,22 +172,50 @@ __global__ void __launch_bounds__(kRopeMaxThreads)
   }
 }
 
-// Shared memory the forward's statistics and output roles set aside for the table's grid-row and
-// grid-column rows (3072 entries: grid_h + grid_w up to 139 at D = 128). The CTA copies them
-// there once, before its first tile; a larger table is read from global memory instead.
-constexpr int kRopeSmemTabBytes = 24 * 1024;
+// Shared memory the forward's statistics and output roles set aside for a copy of the table's
+// grid-row and grid-column entries in the bank-conflict-free layout of rope_stage_rc (256 bytes
+// per grid row and per grid column: grid_h + grid_w up to 127). A larger grid is read from the
+// table in global memory instead.
+constexpr int kRopeSmemTabBytes = 32 * 1024;
 
-// Copy the grid-row and grid-column rows of the table into tab_s (kRopeSmemTabBytes, 16-byte
-// aligned) if they fit, by threads tid of nthreads; returns where rope_rotate_tile reads them.
-// The caller synchronises the CTA before the first read.
-__device__ __forceinline__ const float2* rope_stage_rc(float2* tab_s, const RopeArgs& ra, int tid,
-                                                       int nthreads) {
-  if (ra.n_rc * static_cast<int>(sizeof(float2)) > kRopeSmemTabBytes) return ra.tab + ra.off_h;
-  // off_h and n_rc are even (whole 16-byte entry pairs)
-  const float4* src = reinterpret_cast<const float4*>(ra.tab + ra.off_h);
-  float4* dst = reinterpret_cast<float4*>(tab_s);
-  for (int i = tid; i < ra.n_rc / 2; i += nthreads) dst[i] = __ldg(src + i);
-  return tab_s;
+// Where rope_rotate_tile reads the grid-row and grid-column pairs' (cos, sin).
+struct RopeRc {
+  const float2* p;  // the shared-memory copy, or the table from its first grid-row entry
+  int smem;         // 1: p is the copy
+};
+
+// The copy in shared memory: position (grid row rg, or grid column cg) holds 32 entries, 8 for
+// each pair index p of a chunk: entry p * 8 + s is pair 4 c + p of chunk c = c0 + s, c0 the first
+// chunk with a pair on the axis (at most 7 of them at D <= 128). Grid rows at rg * 32, grid
+// columns at grid_h * 32 + 8 + cg * 32. For a fixed p, the 16 lanes of one token (chunks c) read
+// words 8 bytes apart, grid-row lanes in the first 64 bytes of a 128-byte bank line and
+// grid-column lanes in the second: no two lanes of a token share a bank, and a warp's two tokens
+// take the two wavefronts an 8-byte load of 32 lanes needs anyway. (The table's own layout, pair
+// j of a row at j - j0, puts the lanes of a token 32 bytes apart, 2- to 4-way bank conflicts.)
+// Entries of chunks' pairs off the axis hold (1, 0) and are never read.
+__device__ __forceinline__ int rope_rc_entries(const RopeArgs& ra) {
+  return (ra.grid_h + ra.grid_w) * 32 + 8;
+}
+
+// Fill the copy (tab_s: kRopeSmemTabBytes, 128-byte aligned) by threads tid of nthreads if it
+// fits. The caller synchronises the CTA before the first read.
+__device__ __forceinline__ RopeRc rope_stage_rc(float2* tab_s, const RopeArgs& ra, int tid,
+                                                int nthreads) {
+  if (rope_rc_entries(ra) * static_cast<int>(sizeof(float2)) > kRopeSmemTabBytes)
+    return RopeRc{ra.tab + ra.off_h, 0};
+  const int n = (ra.grid_h + ra.grid_w) * 32;
+  for (int i = tid; i < n; i += nthreads) {
+    const int pos = i >> 5, p = (i >> 3) & 3, s = i & 7;
+    const bool row = pos < ra.grid_h;
+    const int first = row ? ra.pt : ra.pt + ra.ph;  // the axis's first pair
+    const int j = 4 * ((first >> 2) + s) + p;
+    float2 v = make_float2(1.f, 0.f);
+    if (j >= first && j < first + ra.ph)
+      v = row ? __ldg(ra.tab + ra.off_h + pos * ra.len_h + j - ra.j0_h)
+              : __ldg(ra.tab + ra.off_w + (pos - ra.grid_h) * ra.len_w + j - ra.j0_w);
+    tab_s[row ? i : i + 8] = v;
+  }
+  return RopeRc{tab_s, 1};
 }
 
 // The same rotation applied in shared memory by the forward's statistics (K) and output (Q)
@@ -197,29 +225,34 @@ __device__ __forceinline__ const float2* rope_stage_rc(float2* tab_s, const Rope
 // Thread tid of nthreads owns chunk c = tid % (DP/8) of rows tid / (DP/8), + nthreads / (DP/8),
 // ...: its 4 pairs, hence their axes and the time pairs' (cos, sin), are fixed for the tile; a
 // warp covers whole rows, so its shared-memory accesses take the minimum number of wavefronts.
-// The grid-row and column pairs' entries are read per row from rc (rope_stage_rc: the CTA's
-// shared-memory copy of the table's grid-row and grid-column rows, else the table itself), one
-// 8-byte load per pair with no branch around it. The arithmetic and the rounding are those of
+// The grid-row and column pairs' entries are read per row from rc (rope_stage_rc), one 8-byte
+// load per pair with no branch around it. The arithmetic and the rounding are those of
 // gdn_rope_kernel.
 template <int DP>
 __device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nthreads, int rows,
                                                  int n0, int t, int D, const RopeArgs& ra,
-                                                 const float2* rc) {
+                                                 const RopeRc& rc) {
   constexpr int kChunks = DP / 8;
   const int c = tid % kChunks;
   if (c * 8 >= D) return;
   const int r_step = nthreads / kChunks;
   int r = tid / kChunks;
   if (r >= rows) return;
-  // pair p of the chunk: (cos, sin) if on the time axis, else its entry's offset in rc (the row
-  // of the token's grid row or column adds rg * len_h or cg * len_w)
+  // entries of one grid row / grid column in rc.p
+  const int sh = rc.smem ? 32 : ra.len_h, sw = rc.smem ? 32 : ra.len_w;
+  // pair p of the chunk: (cos, sin) if on the time axis, else its entry's offset in rc.p (the
+  // token's grid row or column adds rg * sh or cg * sw)
   float2 ct[4];
   int off[4], axis[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const int j = 4 * c + p;
     axis[p] = j < ra.pt ? 0 : (j < ra.pt + ra.ph ? 1 : 2);
-    off[p] = axis[p] == 1 ? j - ra.j0_h : ra.off_w - ra.off_h + j - ra.j0_w;
+    if (rc.smem)
+      off[p] = axis[p] == 1 ? p * 8 + c - (ra.pt >> 2)
+                            : ra.grid_h * 32 + 8 + p * 8 + c - ((ra.pt + ra.ph) >> 2);
+    else
+      off[p] = axis[p] == 1 ? j - ra.j0_h : ra.off_w - ra.off_h + j - ra.j0_w;
     ct[p] = axis[p] == 0 ? __ldg(ra.tab + t * ra.len_t + j) : make_float2(1.f, 0.f);
   }
   uint8_t* const box = tile + (c >> 3) * kBoxBytes;
@@ -250,10 +283,9 @@ __device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nth
     float2 cs[8];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      cs[p] = axis[p] == 0 ? ct[p] : rc[off[p] + (axis[p] == 1 ? rg * ra.len_h : cg * ra.len_w)];
-      cs[4 + p] = axis[p] == 0 || !second
-                      ? ct[p]
-                      : rc[off[p] + (axis[p] == 1 ? rg2 * ra.len_h : cg2 * ra.len_w)];
+      cs[p] = axis[p] == 0 ? ct[p] : rc.p[off[p] + (axis[p] == 1 ? rg * sh : cg * sw)];
+      cs[4 + p] = axis[p] == 0 || !second ? ct[p]
+                                          : rc.p[off[p] + (axis[p] == 1 ? rg2 * sh : cg2 * sw)];
     }
     rotate(r, cs);
     if (second) rotate(r + r_step, cs + 4);

@@ -169,8 +169,8 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
-  // RoPE: the table's grid-row and grid-column rows, copied past the barriers if they fit
-  const float2* rope_rc = nullptr;
+  // RoPE: the table's grid-row and grid-column entries, copied past the barriers if they fit
+  RopeRc rope_rc{nullptr, 0};
   if constexpr (kRope)
     rope_rc = rope_stage_rc(
         reinterpret_cast<float2*>(smem + L::kStages * L::kStageBytes + L::kBarrierBytes), p.rope,

@@ -125,9 +125,8 @@ FWD_SHAPES = [
     (1, 1, 3, 1, 1, 128, 500.0, 5, True),        # one token per frame
     (1, 2, 20, 4, 8, 32, 10000.0, 0, False),     # many frames, small head dim
     (1, 2, 7, 11, 12, 96, 10000.0, 950, True),   # late frames of a resumed clip
-    # grid-row and grid-column rows of the table past the kernels' 24 KB shared-memory copy
-    # ((grid_h + grid_w) * 22 entries of 8 bytes at D = 128, * 10 at D = 64): read from the
-    # table in global memory instead
+    # grids past the kernels' 32 KB shared-memory copy of the table's grid-row and grid-column
+    # entries (256 bytes per grid row and per grid column): read from the table in global memory
     (1, 2, 3, 2, 150, 128, 10000.0, 0, True),
     (1, 2, 3, 1, 320, 64, 10000.0, 3, False),
 ]
