@@ -66,12 +66,14 @@ struct FusedLayout {
                             OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
                                          kFusedRopeGroups<DP>>::kXfWarps <= 18,
                 "output publisher warp");
-  static constexpr int kSmemBytes = cmax(
+  static constexpr int kSmemBytes =
       cmax(ChainLayout<DP>::kSmemBytes,
-           cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes)),
-      cmax(StatsLayout<DP, false, false, true, kFusedRopeGroups<DP>>::kSmemBytes,
-           OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
-                        kFusedRopeGroups<DP>>::kSmemBytes));
+           cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes));
+  // with RoPE the statistics and output roles also hold the table copy of rope_stage_rc
+  static constexpr int kSmemBytesRope =
+      cmax(kSmemBytes, cmax(StatsLayout<DP, false, false, true, kFusedRopeGroups<DP>>::kSmemBytes,
+                            OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
+                                         kFusedRopeGroups<DP>>::kSmemBytes));
 };
 
 // kF8: e4m3 q, k, v with per (b, t, h) scales in p (DP = 128 only). kRope: q and k rotated by

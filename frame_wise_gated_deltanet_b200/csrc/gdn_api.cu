@@ -508,6 +508,7 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
                      const float* gamma, const float* beta, const float* s_in, void* out,
                      float* s_out, cudaStream_t st, void* kept = nullptr) {
   using L = gdn::FusedLayout<DP>;
+  constexpr int kSmem = kRope ? L::kSmemBytesRope : L::kSmemBytes;
   const int sms = g_dev[dev].sms;
   const int bh = p.B * p.H;
   const int kRing = kept ? p.T : fused_ring(bh, p.D);
@@ -523,7 +524,7 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
     return GDN_ERR_CUDA;
   auto kern = gdn::gdn_fused_kernel<DP, kF8, kRope>;
   const int bit = kRope ? 44 + (DP == 128 ? 0 : 1) : (kF8 ? 17 : (DP == 128 ? 8 : 9));
-  if (gdn_status s = ensure_smem_attr(dev, bit, kern, L::kSmemBytes)) return s;
+  if (gdn_status s = ensure_smem_attr(dev, bit, kern, kSmem)) return s;
   // split the SMs left after the chains between the stats and output roles (fused_stats_pct)
   const int workers = sms - bh;
   int n_stats = (workers * fused_stats_pct(kF8, DP) + 50) / 100;
@@ -557,7 +558,7 @@ gdn_status run_fused(int dev, const Problem& p, const void* q, const void* k, co
   {
     ProfiledLaunch pl("gdn_fused_kernel", st);
     if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(sms),
-                                    dim3(L::kThreads), args, L::kSmemBytes, st) != cudaSuccess)
+                                    dim3(L::kThreads), args, kSmem, st) != cudaSuccess)
       return GDN_ERR_CUDA;
   }
   return check_launch();

@@ -48,6 +48,9 @@ namespace gdn {
 #ifndef GDN_ROPE_OUT_QSTAGES
 #define GDN_ROPE_OUT_QSTAGES 2
 #endif
+#ifndef GDN_ROPE_OUT_OBUFS
+#define GDN_ROPE_OUT_OBUFS 2
+#endif
 
 // kRopeGroups: groups of 128 threads (4 warps) in the RoPE transform of the Q tiles.
 template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false,
@@ -73,10 +76,11 @@ struct OutputLayout {
   static constexpr int kThreads = (2 + kEpiWarps + (kTransform ? kXfWarps : 0)) * 32;
   static constexpr int kQLoadBytes = kF8 ? kQBytes / 2 : kQBytes;  // TMA bytes per Q tile
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
-  static constexpr int kOBytes = kQBytes;  // one bf16 output tile (two staging buffers)
+  static constexpr int kOBytes = kQBytes;  // one bf16 output tile
+  static constexpr int kOBufs = (DP == 128 && kRope) ? GDN_ROPE_OUT_OBUFS : 2;  // staging tiles
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes =
-      kSBufs * kSBufBytes + kStages * kQBytes + 2 * kOBytes + kBarrierBytes + kTabBytes + 1024;
+      kSBufs * kSBufBytes + kStages * kQBytes + kOBufs * kOBytes + kBarrierBytes + kTabBytes + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   // barriers, item ring, TMEM slot and the fused publisher's ring within kBarrierBytes
   static_assert(8 * (3 * kStages + 2 * kSBufs + 4 + 8 + 1) + 32 + 8 + 8 * 16 + 32 <= kBarrierBytes,
@@ -147,8 +151,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   constexpr int kEpiThreads = 32 * L::kEpiWarps;
   uint8_t* s_buf = smem;                                  // kSBufs state buffers
   uint8_t* q_ring = smem + L::kSBufs * L::kSBufBytes;     // kStages Q tiles
-  uint8_t* o_stage = q_ring + L::kStages * L::kQBytes;  // 2 output staging tiles
-  uint64_t* full = reinterpret_cast<uint64_t*>(o_stage + 2 * L::kOBytes);
+  uint8_t* o_stage = q_ring + L::kStages * L::kQBytes;  // kOBufs output staging tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(o_stage + L::kOBufs * L::kOBytes);
   uint64_t* ready = full + L::kStages;
   uint64_t* empty = ready + L::kStages;
   uint64_t* s_full = empty + L::kStages;
@@ -216,7 +220,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
   // RoPE: the table's grid-row and grid-column entries, copied past the barriers if they fit
   RopeRc rope_rc{nullptr, 0};
   if constexpr (kRope)
-    rope_rc = rope_stage_rc(reinterpret_cast<float2*>(o_stage + 2 * L::kOBytes + L::kBarrierBytes),
+    rope_rc = rope_stage_rc(reinterpret_cast<float2*>(o_stage + L::kOBufs * L::kOBytes + L::kBarrierBytes),
                             p.rope, threadIdx.x, blockDim.x);
   tc_fence_before();
   __syncthreads();
@@ -411,8 +415,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         // row by row instead of through the TMA box
         const bool row_stores = kLA && valid < kRowsPerTile;
         const bool waited = mbar_wait(&acc_full[acc], (tc >> 1) & 1);
-        // staging buffer tc&1 is free once the store issued two tiles ago has read it
-        if (leader) bulk_wait_read<1>();
+        // staging buffer tc % kOBufs is free once the store issued kOBufs tiles ago has read it
+        if (leader) bulk_wait_read<L::kOBufs - 1>();
         if (named_bar_any(1, kEpiThreads, !waited)) {
           ok = false;
           break;
@@ -420,7 +424,7 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         tc_fence_after();
         // warps whose 32 rows are all past the item's last token skip the read-out: the TMA
         // store clips at N (GDN), and LA stores such tiles row by row
-        uint8_t* ob = o_stage + (tc & 1) * L::kOBytes;
+        uint8_t* ob = o_stage + (tc % L::kOBufs) * L::kOBytes;
         if (static_cast<int>(quarter) * 32 < valid) {
           const uint32_t tacc = lane_base + acc * DP;
           float scale = 1.f;
