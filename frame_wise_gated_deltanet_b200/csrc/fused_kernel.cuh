@@ -66,9 +66,11 @@ struct FusedLayout {
                             OutputLayout<DP, false, kFusedOutGroups<DP>, false, true,
                                          kFusedRopeGroups<DP>>::kXfWarps <= 18,
                 "output publisher warp");
-  static constexpr int kSmemBytes =
+  static constexpr int kSmemBytes = cmax(
       cmax(ChainLayout<DP>::kSmemBytes,
-           cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes));
+           cmax(StatsLayout<DP, false>::kSmemBytes, OutputLayout<DP, false>::kSmemBytes)),
+      cmax(StatsLayout<DP, false, DP == 128>::kSmemBytes,
+           OutputLayout<DP, false, kFusedOutGroups<DP>, DP == 128>::kSmemBytes));
   // with RoPE the statistics and output roles also hold the table copy of rope_stage_rc
   static constexpr int kSmemBytesRope =
       cmax(kSmemBytes, cmax(StatsLayout<DP, false, false, true, kFusedRopeGroups<DP>>::kSmemBytes,

@@ -51,6 +51,15 @@ namespace gdn {
 #ifndef GDN_ROPE_OUT_OBUFS
 #define GDN_ROPE_OUT_OBUFS 2
 #endif
+// fp8 inputs at DP = 128: Q stages and output staging tiles (the 720p clip: 2.31 ms with 3 and
+// 2, 2.63 with 4 and 1, 2.87 with 2 and 3; the role needs its stores in flight as much as its
+// loads)
+#ifndef GDN_F8_OUT_QSTAGES
+#define GDN_F8_OUT_QSTAGES 3
+#endif
+#ifndef GDN_F8_OUT_OBUFS
+#define GDN_F8_OUT_OBUFS 2
+#endif
 
 // kRopeGroups: groups of 128 threads (4 warps) in the RoPE transform of the Q tiles.
 template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false,
@@ -71,13 +80,15 @@ struct OutputLayout {
   // state buffers: items in flight past the state load (the fused role waits on the chain, so
   // more of them hide its hand-off latency; DP = 128 has no shared memory left for more)
   static constexpr int kSBufs = (DP == 128) ? (kRope ? GDN_ROPE_OUT_SBUFS : 2) : 4;
-  static constexpr int kStages = (DP == 128) ? (kRope ? GDN_ROPE_OUT_QSTAGES : 3) : 8;
+  static constexpr int kStages =
+      (DP == 128) ? (kRope ? GDN_ROPE_OUT_QSTAGES : (kF8 ? GDN_F8_OUT_QSTAGES : 3)) : 8;
   static constexpr int kTabBytes = kRope ? kRopeSmemTabBytes : 0;
   static constexpr int kThreads = (2 + kEpiWarps + (kTransform ? kXfWarps : 0)) * 32;
   static constexpr int kQLoadBytes = kF8 ? kQBytes / 2 : kQBytes;  // TMA bytes per Q tile
   static constexpr int kTmemCols = (2 * DP < 32) ? 32 : 2 * DP;
   static constexpr int kOBytes = kQBytes;  // one bf16 output tile
-  static constexpr int kOBufs = (DP == 128 && kRope) ? GDN_ROPE_OUT_OBUFS : 2;  // staging tiles
+  static constexpr int kOBufs =  // staging tiles
+      DP == 128 ? (kRope ? GDN_ROPE_OUT_OBUFS : (kF8 ? GDN_F8_OUT_OBUFS : 2)) : 2;
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes =
       kSBufs * kSBufBytes + kStages * kQBytes + kOBufs * kOBytes + kBarrierBytes + kTabBytes + 1024;
@@ -459,16 +470,22 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
         mbar_arrive(&acc_empty[acc]);
         fence_async_smem();
         named_bar(1, kEpiThreads);
-        if (leader && !row_stores) {
+        if (leader) {
+          if (!row_stores) {
 #pragma unroll
-          for (int kb = 0; kb < L::kBoxes; ++kb) {
-            if constexpr (kLA)
-              tma_store_3d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h,
-                           it.row0 + tile * kRowsPerTile, pol_out);
-            else
-              tma_store_4d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h, tile * kRowsPerTile, it.bt,
-                           pol_out);
+            for (int kb = 0; kb < L::kBoxes; ++kb) {
+              if constexpr (kLA)
+                tma_store_3d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h,
+                             it.row0 + tile * kRowsPerTile, pol_out);
+              else
+                tma_store_4d(tm_o, ob + kb * kBoxBytes, kb * 64, it.h, tile * kRowsPerTile,
+                             it.bt, pol_out);
+            }
           }
+          // one bulk group per tile, empty for a tile stored row by row, so that the wait for
+          // "the store issued kOBufs tiles ago has read its staging buffer" counts tiles: without
+          // it, after an LA block's row-stored last tile the next tile's epilogue could overwrite
+          // the staging buffer a still-pending store was reading
           bulk_commit();
         }
       }
@@ -568,15 +585,22 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
           // rows past the block's last token belong to other blocks: their outputs are not
           // stored, so they need no relu
           const int valid = min(kRowsPerTile, it.rows - tile * kRowsPerTile);
-  #pragma unroll 1
+#pragma unroll 1
           for (int kb = 0; kb < L::kBoxes; ++kb) {
+            // the thread's 8 chunks of the box (8 x 16 B per 128-byte box row, rows tid / 8 +
+            // 16 u): all loads issued before the first store
             uint4* qt = reinterpret_cast<uint4*>(q_ring + stage * L::kQBytes + kb * kBoxBytes);
-            for (int i = tid; i < valid * 8; i += 128) {  // 8 x 16 B per 128-byte box row
-              uint4 x = qt[i];
-              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
-  #pragma unroll
+            uint4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              if (((tid + 128 * u) >> 3) < valid) x[u] = qt[tid + 128 * u];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              if (((tid + 128 * u) >> 3) >= valid) continue;
+              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x[u]);
+#pragma unroll
               for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-              qt[i] = x;
+              qt[tid + 128 * u] = x[u];
             }
           }
           fence_async_smem();

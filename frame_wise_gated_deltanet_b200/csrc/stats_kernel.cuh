@@ -534,13 +534,19 @@ __device__ __forceinline__ void stats_body(const CUtensorMap* tm_k, const CUtens
           const int valid = min(kRowsPerTile, nf * p.N - tile * kRowsPerTile);
 #pragma unroll 1
           for (int kb = 0; kb < L::kOpBytes / kBoxBytes; ++kb) {
+            // the thread's 8 chunks of the box (8 x 16 B per 128-byte row, rows tid / 8 + 16 u):
+            // all loads issued before the first store
             uint4* kt = reinterpret_cast<uint4*>(st + kb * kBoxBytes);
-            for (int i = tid; i < kRowsPerTile * 8; i += 128) {  // 8 x 16 B per 128-byte row
-              uint4 x = kt[i];
-              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+            uint4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = kt[tid + 128 * u];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = tid + 128 * u;
+              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x[u]);
 #pragma unroll
               for (int j = 0; j < 4; ++j) h2[j] = __hmax2(h2[j], zero2);
-              kt[i] = (i >> 3) < valid ? x : make_uint4(0u, 0u, 0u, 0u);
+              kt[i] = (i >> 3) < valid ? x[u] : make_uint4(0u, 0u, 0u, 0u);
             }
           }
           // ones column at index D of every V row (token), for the normaliser
