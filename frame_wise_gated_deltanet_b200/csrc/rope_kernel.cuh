@@ -17,6 +17,8 @@
 // transform warps to the K tiles of the statistics kernel and the Q tiles of the output kernel in
 // shared memory, so q and k are rotated on their way to the tensor cores and never rewritten.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace gdn {
@@ -101,6 +103,28 @@ __device__ __forceinline__ void rope_fetch(const RopeArgs& ra, const RopeChunk& 
     if (lo) cs[2 * q] = make_float2(v.x, v.y);
     if (hi) cs[2 * q + 1] = make_float2(v.z, v.w);
   }
+}
+
+// Shared-space accesses (32-bit shared addresses) for the rotation of a tile in shared memory.
+__device__ __forceinline__ uint4 rope_lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void rope_sts128(uint32_t a, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ float2 rope_lds64(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
+  return v;
 }
 
 // Rotate the 4 pairs of a 16-byte chunk of bf16 (f32 arithmetic, bf16 rounding).
@@ -268,31 +292,48 @@ __device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, int tid, int nth
       ++g_r;
     }
   };
-  auto rotate = [&](int row, const float2* cs) {
+  // the tile (and the table copy, when rc.smem) through shared-space loads and stores, issued in
+  // program order: both rows' table entries and chunks are loaded before either is rotated
+  const uint32_t box_s = smem_u32(box);
+  auto slot = [&](int row) {
     // 128B swizzle: the chunk's 16-byte slot in its 128-byte row is c % 8 XOR row % 8
-    uint4* ptr = reinterpret_cast<uint4*>(box + row * 128 + (((c & 7) ^ (row & 7)) << 4));
-    uint4 raw = *ptr;
-    rope_rotate_chunk(raw, cs);
-    *ptr = raw;
+    return box_s + row * 128 + (((c & 7) ^ (row & 7)) << 4);
   };
-  // two rows at a time: both rows' table reads are in flight together
-  for (; r < rows; r += 2 * r_step) {
-    const bool second = r + r_step < rows;
-    int rg2 = rg, cg2 = cg;
-    advance(rg2, cg2);
-    float2 cs[8];
+  auto rows_loop = [&](auto smem_tab) {
+    constexpr bool kS = decltype(smem_tab)::value;
+    const uint32_t rc_s = kS ? smem_u32(rc.p) : 0u;
+    auto entry = [&](int i) { return kS ? rope_lds64(rc_s + 8u * i) : __ldg(rc.p + i); };
+    // two rows at a time: both rows' table reads are in flight together
+    for (; r < rows; r += 2 * r_step) {
+      const bool second = r + r_step < rows;
+      int rg2 = rg, cg2 = cg;
+      advance(rg2, cg2);
+      float2 cs[8];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      cs[p] = axis[p] == 0 ? ct[p] : rc.p[off[p] + (axis[p] == 1 ? rg * sh : cg * sw)];
-      cs[4 + p] = axis[p] == 0 || !second ? ct[p]
-                                          : rc.p[off[p] + (axis[p] == 1 ? rg2 * sh : cg2 * sw)];
+      for (int p = 0; p < 4; ++p) {
+        cs[p] = axis[p] == 0 ? ct[p] : entry(off[p] + (axis[p] == 1 ? rg * sh : cg * sw));
+        cs[4 + p] = axis[p] == 0 || !second
+                        ? ct[p]
+                        : entry(off[p] + (axis[p] == 1 ? rg2 * sh : cg2 * sw));
+      }
+      const uint32_t a0 = slot(r), a1 = slot(second ? r + r_step : r);
+      uint4 x0 = rope_lds128(a0);
+      uint4 x1 = second ? rope_lds128(a1) : x0;
+      rope_rotate_chunk(x0, cs);
+      rope_sts128(a0, x0);
+      if (second) {
+        rope_rotate_chunk(x1, cs + 4);
+        rope_sts128(a1, x1);
+      }
+      rg = rg2;
+      cg = cg2;
+      advance(rg, cg);
     }
-    rotate(r, cs);
-    if (second) rotate(r + r_step, cs + 4);
-    rg = rg2;
-    cg = cg2;
-    advance(rg, cg);
-  }
+  };
+  if (rc.smem)
+    rows_loop(std::true_type{});
+  else
+    rows_loop(std::false_type{});
 }
 
 }  // namespace gdn
