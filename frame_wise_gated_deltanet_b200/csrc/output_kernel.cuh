@@ -61,6 +61,32 @@ namespace gdn {
 #define GDN_F8_OUT_OBUFS 2
 #endif
 
+// e4m3_row_to_bf16_tile (the in-place conversion of an fp8 Q tile into the bf16 operand layout)
+// with explicit shared-space loads and stores on the tile's 32-bit shared address: every lane
+// of the warp reads its chunks before any lane writes, as there.
+template <int kParts>
+__device__ __forceinline__ void e4m3_row_to_bf16_tile_s(uint32_t tile, int row, int part) {
+  static_assert(kParts == 1 || kParts == 2 || kParts == 4, "parts of a row");
+  constexpr int kC = 8 / kParts;
+  const uint32_t b0 = tile + row * 128;
+  const uint32_t b1 = tile + 16384 + row * 128;
+  const uint32_t sw = row & 7;
+  uint4 in[kC];
+#pragma unroll
+  for (int i = 0; i < kC; ++i) in[i] = rope_lds128(b1 + (((part * kC + i) ^ sw) << 4));
+  if (kParts > 1) __syncwarp();
+#pragma unroll
+  for (int i = 0; i < kC; ++i) {
+    // fp8 chunk c = dims 16c..16c+15 -> bf16 chunks 2c, 2c+1 of the 16 chunks of 8 dims
+    const int c = part * kC + i;
+    uint4 lo, hi;
+    e4m3x16_to_bf16(in[i], lo, hi);
+    const int k0 = 2 * c, k1 = 2 * c + 1;  // 8-dim chunk index over 128 dims
+    rope_sts128((k0 < 8 ? b0 : b1) + (((k0 & 7) ^ sw) << 4), lo);
+    rope_sts128((k1 < 8 ? b0 : b1) + (((k1 & 7) ^ sw) << 4), hi);
+  }
+}
+
 // kRopeGroups: groups of 128 threads (4 warps) in the RoPE transform of the Q tiles.
 template <int DP, bool kLA, int kG = 4, bool kF8 = false, bool kRope = false,
           int kRopeGroups = DP / 64>
@@ -555,8 +581,8 @@ __device__ __forceinline__ void output_body(const CUtensorMap* tm_q, const CUten
             ok = false;
             break;
           }
-          e4m3_row_to_bf16_tile<L::kF8Parts>(q_ring + stage * L::kQBytes, tid / L::kF8Parts,
-                                             tid % L::kF8Parts);
+          e4m3_row_to_bf16_tile_s<L::kF8Parts>(smem_u32(q_ring + stage * L::kQBytes),
+                                               tid / L::kF8Parts, tid % L::kF8Parts);
           fence_async_smem();
           mbar_arrive(&ready[stage]);
           if (++stage == L::kStages) {
