@@ -112,8 +112,11 @@ gdn_status gdn_frame_forward(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf1
  * and t_offset (>= 0, the absolute index of the clip's first frame, so a resumed clip continues
  * its time positions). Host-side errors as gdn_frame_forward and gdn_rope_3d. Same path choice
  * (fused, three kernels, chunked) and workspace as gdn_frame_forward, plus a per-GPU cos/sin
- * table of 8 * (T * l_t + grid_h * l_h + grid_w * l_w) bytes (grown like the
- * workspace, freed by gdn_release_workspace), computed by one extra launch on `stream`.
+ * table of 8 * (T * l_t + grid_h * l_h + grid_w * l_w) bytes (l_t, l_h, l_w as under
+ * gdn_rope_3d; grown like the workspace, freed by gdn_release_workspace), computed by one extra
+ * launch on `stream`. The kernels copy the table's grid-row and grid-column entries into shared
+ * memory (256 bytes per grid row and per grid column) when grid_h + grid_w <= 127, and read them
+ * from the table in global memory otherwise; either way the result is the same.
  */
 gdn_status gdn_frame_forward_rope(const gdn_bf16* q, const gdn_bf16* k, const gdn_bf16* v,
                                   const float* gamma, const float* beta, const float* state_in,
